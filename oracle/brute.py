@@ -1,0 +1,57 @@
+"""Dense brute-force HSA in numpy, for tiny inputs only -- TEST INFRASTRUCTURE ONLY.
+
+A second, structurally different formulation of the same definition as ``hsa_oracle.c``, used to pin
+the C oracle on tiny shapes: it builds the full masked score matrix, ranks every row with numpy's
+stable argsort, attends every query to EVERY chunk (dense, whether selected or not) and fuses with a
+dense weight matrix that is zero off the selection. Source: explainer page of "Every Token Counts",
+"How It Works (Technically)", Steps 2-4, and "The algorithm, simplified".
+"""
+import itertools
+
+import numpy as np
+
+
+def forward(Q, K, V, L, chunk, topk, scale):
+    """Q, K, V [B, H, T, D], L [B, H, N, D] -> (out [B,H,T,D], sel_idx [B,H,T,topk], sel_w [B,H,T,topk])."""
+    Q, K, V, L = (np.asarray(x, np.float64) for x in (Q, K, V, L))
+    B, H, T, D = Q.shape
+    N = T // chunk
+    t = np.arange(T)
+    admissible = (np.arange(N)[None, :] + 1) * chunk - 1 <= t[:, None]           # [T, N]
+    S = scale * np.einsum("bhtd,bhnd->bhtn", Q, L)                                 # [B,H,T,N]
+    S_masked = np.where(admissible, S, -np.inf)
+    order = np.argsort(-S_masked, axis=-1, kind="stable")                         # ties -> lower index
+    n_t = admissible.sum(-1)                                                       # [T]
+    k_t = np.minimum(n_t, topk)
+    sel_idx = np.full((B, H, T, topk), -1, np.int32)
+    Wd = np.zeros((B, H, T, N))
+    for i in range(T):
+        k = int(k_t[i])
+        if k == 0:
+            continue
+        sel = order[:, :, i, :k]                                                   # [B,H,k]
+        sel_idx[:, :, i, :k] = sel
+        s_sel = np.take_along_axis(S[:, :, i, :], sel, axis=-1)
+        e = np.exp(s_sel - s_sel.max(-1, keepdims=True))
+        np.put_along_axis(Wd[:, :, i, :], sel, e / e.sum(-1, keepdims=True), axis=-1)
+    Kc = K[:, :, : N * chunk].reshape(B, H, N, chunk, D)
+    Vc = V[:, :, : N * chunk].reshape(B, H, N, chunk, D)
+    A = scale * np.einsum("bhtd,bhnud->bhtnu", Q, Kc)                               # every query x every chunk
+    P = np.exp(A - A.max(-1, keepdims=True))
+    P /= P.sum(-1, keepdims=True)
+    Obar = np.einsum("bhtnu,bhnud->bhtnd", P, Vc)
+    out = np.einsum("bhtn,bhtnd->bhtd", Wd, Obar)
+    sel_w = np.zeros((B, H, T, topk))
+    valid = sel_idx >= 0
+    sel_w[valid] = np.take_along_axis(Wd, np.where(valid, sel_idx, 0), axis=-1)[valid]
+    return out, sel_idx, sel_w
+
+
+def best_subset(scores, k):
+    """Top-k by exhaustive search: the k-subset with the largest score sum (distinct scores only)."""
+    best, best_sum = None, -np.inf
+    for comb in itertools.combinations(range(len(scores)), k):
+        s = sum(scores[i] for i in comb)
+        if s > best_sum:
+            best, best_sum = comb, s
+    return set(best)

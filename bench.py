@@ -1,0 +1,445 @@
+"""Benchmark of the HSA operator on B200.
+
+One step = one HSA prefill forward of the 32K workload (B2 T32768 H8 D128, chunk 64, topk 16,
+chunk-mean landmarks): retrieval scoring + top-K + fusion weights, chunk-major dispatch, per-chunk
+attention with the fused blend, bf16 output. The headline metric is prefill tokens/s (B*T tokens per
+step). The same run also times the 16M-token decode (B1, H8, D128, topk 32; microseconds per token)
+and the 64K forward+backward, each against its roofline, and times the CPU oracle on a bounded
+sample on the host cores as a reported baseline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--skip-decode] [--skip-backward]
+
+Multi-GPU (torchrun, one process per GPU): HSA's (batch, head) problems are independent, so every
+rank runs its own copy of the workload with no data-path collective (weak scaling); the only
+collectives are the timing barrier and a max-reduction of the elapsed time.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_FORWARD = 6     # score_topk, count, scan, scatter, chunk_attn, finalize
+KERNELS_PER_DECODE = 2      # decode_scan, decode_attend
+KERNELS_PER_BACKWARD = 5    # delta, count, scan, scatter, chunk_bwd
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons while the timed regions run."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"hsa_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        sm, mx, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                clk, mx = float(parts[1]), float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            sm.append(clk)
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        loaded = [c for c, p in zip(sm, power) if p > 300.0] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm), "samples_under_load": len(loaded)}
+
+
+def dist_setup(args):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    import torch
+
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    import torch
+
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def timed(fn, steps, warmup, world):
+    """Device time of `steps` calls of fn (CUDA events on the current stream), max over ranks, ms."""
+    import torch
+
+    for _ in range(warmup):
+        fn()
+    barrier(world)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        fn()
+    e1.record(s)
+    barrier(world)
+    return max_over_ranks(e0.elapsed_time(e1), world)
+
+
+def kernel_profile(fn, steps):
+    """Per-launch-site device time over `steps` calls, from the library's event hooks."""
+    import torch
+
+    from ultra_long_context_b200 import hsa
+
+    torch.cuda.synchronize()
+    hsa.hsa_profile_enable(True)
+    for _ in range(steps):
+        fn()
+    torch.cuda.synchronize()
+    prof = hsa.hsa_profile_summary()
+    hsa.hsa_profile_enable(False)
+    return prof
+
+
+# ------------------------------------------------------------------------------------------------
+# algorithmic work
+
+
+def forward_work(w, sel_idx):
+    """Causal scoring flops, chunk-attention flops (selected pairs only) and pair count."""
+    B, H, T, D, C = w.B, w.H, w.T, w.D, w.chunk
+    t = __import__("numpy").arange(T)
+    n_t = (t + 1) // C
+    score_flops = 2.0 * D * B * H * float(n_t.sum())
+    pairs = int((sel_idx >= 0).sum().item())
+    attn_flops = 4.0 * C * D * pairs
+    return score_flops, attn_flops, pairs
+
+
+def roofline_entry(name, prof, algo, unit, peak, bound, peak_kind, traffic=None):
+    cnt, ms = prof[name]
+    avg_s = ms / cnt / 1e3
+    achieved = algo / avg_s / (1e12 if unit == "TFLOP/s" else 1e9)
+    return {"kernel": name, "bound": bound, "achieved": round(achieved, 3), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4), "traffic": traffic, "avg_launch_us": round(avg_s * 1e6, 3),
+            "peak_source": peak_kind}
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle baseline
+
+
+def oracle_forward_sample(w, Qh, Kh, Vh, Lh, target_s=10.0, rng_seed=0):
+    """Time the oracle on a growing sample of token rows until ~target_s of wall time."""
+    import numpy as np
+
+    import oracle
+
+    rng = np.random.default_rng(rng_seed)
+    BH, T = w.B * w.H, w.T
+    n, spent, rows_done = 256, 0.0, 0
+    while spent < target_s and n <= (1 << 20):
+        rows = rng.integers(0, BH * T, n)
+        t0 = time.perf_counter()
+        oracle.forward(Qh, Kh, Vh, Lh, chunk=w.chunk, topk=w.topk, rows=rows)
+        dt = time.perf_counter() - t0
+        spent += dt
+        rows_done += n
+        n *= 2
+    # a token is H rows (one per head); sampled rows are uniform over (b, h, t)
+    tokens_per_s = rows_done / w.H / spent
+    return tokens_per_s, rows_done, spent
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+# ------------------------------------------------------------------------------------------------
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle, as it stands, on the host cores (rank 0 only)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+
+    from ultra_long_context_b200 import inputs
+
+    w = inputs.WORKLOADS["fwd_t32k_h8_d128_k16"]
+    Q, K, V, L = inputs.forward_inputs(w.B, w.H, w.T, w.D, w.seed, landmarks=w.landmarks, device="cpu")
+    Qh, Kh, Vh, Lh = (x.float().numpy() for x in (Q, K, V, L))
+    for _ in range(max(0, args.warmup)):
+        oracle_forward_sample(w, Qh, Kh, Vh, Lh, target_s=0.5)
+    vals = []
+    rows_total, spent_total = 0, 0.0
+    for i in range(args.steps):
+        v, rows, spent = oracle_forward_sample(w, Qh, Kh, Vh, Lh, target_s=max(1.0, 20.0 / max(1, args.steps)),
+                                               rng_seed=i)
+        vals.append(v)
+        rows_total += rows
+        spent_total += spent
+    value = rows_total / w.H / spent_total
+    sample = (f"{rows_total} token-head rows drawn uniformly from the 32K workload (B2 H8 T32768 D128 topk16), "
+              f"fp64 oracle, {spent_total:.1f} s")
+    line = {"impl": "reference", "metric": "HSA prefill tokens/s (B2 T32768 H8 D128 chunk64 topk16)",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * w.B * w.T / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "fwd_t32k_h8_d128_k16", "B": w.B, "T": w.T, "H": w.H, "D": w.D,
+                       "chunk": w.chunk, "topk": w.topk},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    del torch
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--skip-backward", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import numpy as np
+    import torch
+
+    from ultra_long_context_b200 import hsa, inputs
+
+    world, rank, local = dist_setup(args)
+    peaks, peak_kind = load_peaks()
+    clocks = ClockSampler(local)
+    dev = torch.device("cuda", local)
+
+    # ---------------- prefill forward (headline) ----------------
+    w = inputs.WORKLOADS["fwd_t32k_h8_d128_k16"]
+    Q, K, V, L = inputs.forward_inputs(w.B, w.H, w.T, w.D, w.seed + rank, landmarks=w.landmarks, device=dev)
+    out = torch.empty_like(Q)
+    sel_idx = torch.empty((w.B, w.H, w.T, w.topk), dtype=torch.int32, device=dev)
+    sel_w = torch.empty((w.B, w.H, w.T, w.topk), dtype=torch.float32, device=dev)
+    ws = torch.empty(hsa.hsa_forward_workspace_size(w.B, w.H, w.T, w.D, w.chunk, w.topk) + 256, dtype=torch.uint8,
+                     device=dev)
+
+    def fwd():
+        hsa.hsa_forward(Q, K, V, L, w.topk, out=out, sel_idx=sel_idx, sel_w=sel_w, workspace=ws)
+
+    clocks.start()
+    ms = timed(fwd, args.steps, args.warmup, world)
+    ms_per_step = ms / args.steps
+    tokens = w.B * w.T
+    value = world * tokens / (ms_per_step / 1e3)
+    prof_fwd = kernel_profile(fwd, args.steps)
+    score_flops, attn_flops, pairs = forward_work(w, sel_idx)
+    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    dominant = max((k for k in prof_fwd if k != "memset"), key=lambda k: prof_fwd[k][1])
+    algo = {"chunk_attn": attn_flops, "score_topk": score_flops}
+    roof = roofline_entry(dominant, prof_fwd, algo.get(dominant, attn_flops), "TFLOP/s", tensor_peak, "tensor",
+                          f"{peak_kind} bf16_tflops_sustained")
+    roof_score = roofline_entry("score_topk", prof_fwd, score_flops, "TFLOP/s", tensor_peak, "tensor",
+                                f"{peak_kind} bf16_tflops_sustained")
+    breakdown = {k: {"launches": c, "avg_us": round(t / c * 1e3, 2), "share": round(t / sum(x[1] for x in
+                                                                                           prof_fwd.values()), 4)}
+                 for k, (c, t) in prof_fwd.items()}
+
+    # ---------------- e2e: host buffers through the public API ----------------
+    hQ, hK, hV, hL = (x.cpu().pin_memory() for x in (Q, K, V, L))
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dQ_, dK_, dV_, dL_ = (torch.empty_like(x) for x in (Q, K, V, L))
+
+    def e2e_step():
+        dQ_.copy_(hQ, non_blocking=True)
+        dK_.copy_(hK, non_blocking=True)
+        dV_.copy_(hV, non_blocking=True)
+        dL_.copy_(hL, non_blocking=True)
+        hsa.hsa_forward(dQ_, dK_, dV_, dL_, w.topk, out=out, sel_idx=sel_idx, sel_w=sel_w, workspace=ws)
+        hout.copy_(out, non_blocking=True)
+
+    e2e_ms = timed(e2e_step, args.steps, args.warmup, world) / args.steps
+    h2d = sum(x.numel() * x.element_size() for x in (hQ, hK, hV, hL))
+    d2h = hout.numel() * hout.element_size()
+    e2e = {"value": world * tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)}
+    del hQ, hK, hV, hL, hout, dQ_, dK_, dV_, dL_
+
+    extra = {}
+    # ---------------- decode, 16M-token cache ----------------
+    if not args.skip_decode:
+        wd = inputs.WORKLOADS["decode_16m_b1_h8_d128_k32"]
+        q, Kc, Vc, Lc, lens, _ = inputs.workload_inputs(wd, device=dev)
+        dout_ = torch.empty_like(q)
+        didx = torch.empty((wd.B, wd.H, wd.topk), dtype=torch.int32, device=dev)
+        dw = torch.empty((wd.B, wd.H, wd.topk), dtype=torch.float32, device=dev)
+        dws = torch.empty(hsa.hsa_decode_workspace_size(wd.B, wd.H, wd.cache_len, wd.D, 64, wd.topk) + 256,
+                          dtype=torch.uint8, device=dev)
+
+        def dec():
+            hsa.hsa_decode(q, Kc, Vc, Lc, lens, wd.topk, out=dout_, sel_idx=didx, sel_w=dw, workspace=dws)
+
+        dsteps = max(args.steps, 50)
+        dms = timed(dec, dsteps, args.warmup, world) / dsteps
+        prof_dec = kernel_profile(dec, dsteps)
+        n = wd.cache_len // 64
+        scan_bytes = wd.B * wd.H * (n * wd.D * 2 + wd.D * 2)
+        gather_bytes = wd.B * wd.H * wd.topk * 2 * 64 * wd.D * 2
+        hbm_peak = peaks["hbm_gbs"]
+        extra["decode_16m"] = {
+            "workload": wd.name, "us_per_token": round(dms * 1e3 / wd.B, 3), "ms_per_step": round(dms, 5),
+            "steps": dsteps,
+            "roofline": roofline_entry("decode_scan", prof_dec, scan_bytes, "GB/s", hbm_peak, "hbm",
+                                       f"{peak_kind} hbm_gbs"),
+            "step_vs_hbm": {"algorithmic_bytes": scan_bytes + gather_bytes,
+                            "achieved_GBs": round((scan_bytes + gather_bytes) / (dms / 1e3) / 1e9, 1),
+                            "frac": round((scan_bytes + gather_bytes) / (dms / 1e3) / 1e9 / hbm_peak, 4)},
+            "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_dec.items()},
+        }
+        del q, Kc, Vc, Lc, dws
+        torch.cuda.empty_cache()
+
+    # ---------------- forward + backward, 64K ----------------
+    if not args.skip_backward:
+        wb = inputs.WORKLOADS["fwdbwd_t64k_h8_d128_k16"]
+        bQ, bK, bV, bL, bdO = inputs.workload_inputs(wb, device=dev)
+        bout = torch.empty_like(bQ)
+        bidx = torch.empty((wb.B, wb.H, wb.T, wb.topk), dtype=torch.int32, device=dev)
+        bw = torch.empty((wb.B, wb.H, wb.T, wb.topk), dtype=torch.float32, device=dev)
+        fws = torch.empty(hsa.hsa_forward_workspace_size(wb.B, wb.H, wb.T, wb.D, 64, wb.topk) + 256,
+                          dtype=torch.uint8, device=dev)
+        bws = torch.empty(hsa.hsa_backward_workspace_size(wb.B, wb.H, wb.T, wb.D, 64, wb.topk) + 256,
+                          dtype=torch.uint8, device=dev)
+        grads = (torch.empty(bQ.shape, dtype=torch.float32, device=dev),
+                 torch.empty(bQ.shape, dtype=torch.float32, device=dev),
+                 torch.empty(bQ.shape, dtype=torch.float32, device=dev),
+                 torch.empty(bL.shape, dtype=torch.float32, device=dev))
+
+        def fwdbwd():
+            hsa.hsa_forward(bQ, bK, bV, bL, wb.topk, out=bout, sel_idx=bidx, sel_w=bw, workspace=fws)
+            hsa.hsa_backward(bQ, bK, bV, bL, bout, bdO, bidx, bw, grads=grads, workspace=bws)
+
+        bsteps = max(3, args.steps // 2)
+        bms = timed(fwdbwd, bsteps, args.warmup, world) / bsteps
+        prof_b = kernel_profile(fwdbwd, bsteps)
+        sf, af, bpairs = forward_work(wb, bidx)
+        bwd_flops = 10.0 * 64 * wb.D * bpairs
+        extra["fwdbwd_64k"] = {
+            "workload": wb.name, "tokens_per_s": round(wb.B * wb.T / (bms / 1e3), 1), "ms_per_step": round(bms, 4),
+            "steps": bsteps,
+            "roofline": roofline_entry("chunk_bwd", prof_b, bwd_flops, "TFLOP/s", tensor_peak, "tensor",
+                                       f"{peak_kind} bf16_tflops_sustained"),
+            "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_b.items()},
+        }
+        del bQ, bK, bV, bL, bdO, fws, bws, grads
+        torch.cuda.empty_cache()
+    clk = clocks.stop()
+
+    # ---------------- CPU oracle baseline (rank 0, one GPU) ----------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        Qh, Kh, Vh, Lh = (x.float().cpu().numpy() for x in (Q, K, V, L))
+        v, rows_done, spent = oracle_forward_sample(w, Qh, Kh, Vh, Lh, target_s=10.0)
+        cpu = {"value": round(v, 2), "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
+               "sample": f"{rows_done} token-head rows drawn uniformly from the same 32K workload, fp64 oracle "
+                         f"with OpenMP, {spent:.1f} s wall"}
+
+    launches = args.steps * KERNELS_PER_FORWARD
+    if rank == 0:
+        line = {
+            "metric": "HSA prefill tokens/s (B2 T32768 H8 D128 chunk64 topk16)",
+            "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "D": w.D, "chunk": w.chunk,
+                       "topk": w.topk, "landmarks": "chunk mean + N(0, 0.1^2)", "pairs": pairs,
+                       "l2": "inputs larger than L2 (Q, K, V = 402 MB)", "parallelism": f"dp{world}"},
+            "roofline": roof,
+            "roofline_score_topk": roof_score,
+            "kernels": breakdown,
+            "gpu_launches": launches,
+            "e2e": e2e,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    del np
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,139 @@
+/*
+ * hsa.h -- C ABI of the B200 (sm_100a) Hierarchical Sparse Attention (HSA) library, libhsa_b200.so.
+ *
+ * The operation is the one described on the explainer page of "Every Token Counts: Generalizing 16M
+ * Ultra-Long Context in Large Language Models", section "How It Works (Technically)":
+ *   Step 1  the history is cut into chunks of 64 tokens; chunk c holds tokens 64c .. 64c+63 and
+ *           owns one landmark vector L[c];
+ *   Step 2  each query token t scores every chunk that has ended at or before t,
+ *           s[t,c] = scale * Q[t].L[c], and keeps the top-K chunks I_t;
+ *   Step 3  inside each selected chunk it runs ordinary softmax attention,
+ *           O[t,c] = softmax(scale * Q[t] K_c^T) V_c, separately per chunk;
+ *   Step 4  it blends the chunk outputs by the softmax of their retrieval scores,
+ *           w = softmax(s[t, I_t]),  out[t] = sum_{c in I_t} w_c O[t,c].
+ * and the per-token procedure of section "The algorithm, simplified" (stable sort of the scores in
+ * descending order, first top_k kept).
+ *
+ * Readings of points the page leaves open, used by every entry point below:
+ *   - causal rule: chunk c is admissible for token t iff 64c + 63 <= t, so a token sees
+ *     n_t = (t + 1) / 64 chunks (the token that completes a chunk may retrieve it);
+ *   - a token with n_t = 0 gets out = 0, sel_idx = -1, sel_w = 0 in every slot;
+ *   - n_t < topk: all n_t chunks are selected and the fusion softmax runs over those only;
+ *     the remaining slots hold sel_idx = -1, sel_w = 0;
+ *   - ties: equal scores keep ascending chunk order (lower chunk index wins);
+ *   - one query serves both as retrieval query and attention query; one scale serves both
+ *     (scale <= 0 selects 1/sqrt(D)); no query-key normalisation and no positional encoding
+ *     are applied (inputs are used as given);
+ *   - selection itself carries no gradient; the landmarks receive gradient through the selected
+ *     scores only (Step 4: w multiplies the output, so the loss reaches s).
+ *
+ * Conventions shared by all entry points:
+ *   - Tensor arguments are DEVICE pointers owned by the caller, contiguous, row-major in the
+ *     shapes given, 16-byte aligned. bf16 values are passed as raw 16-bit patterns (hsa_bf16).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy default
+ *     stream). Validation is done on the host before any launch; an invalid call launches
+ *     nothing and returns a negative status. No call synchronises the stream.
+ *   - Scratch memory is caller-provided: query its size with the matching *_workspace_size
+ *     function and pass at least that many bytes, 256-byte aligned. The library allocates no
+ *     device memory. Workspace contents on entry are irrelevant; they are clobbered.
+ *   - Supported now: D in {64, 128}, chunk == 64. Forward/backward: 1 <= topk <= 32;
+ *     decode: 1 <= topk <= 64. Anything else returns HSA_ERR_UNSUPPORTED.
+ *   - Every output element is written (including padding and all-zero rows).
+ *   - Inputs must be finite; NaN/Inf inputs give unspecified results.
+ *   - On any non-OK status, hsa_last_error() returns a message for the calling thread.
+ */
+#ifndef HSA_B200_H
+#define HSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t hsa_bf16; /* raw bfloat16 bit pattern */
+
+typedef enum {
+    HSA_OK = 0,
+    HSA_ERR_INVALID_ARG = -1, /* null pointer, bad size, misalignment */
+    HSA_ERR_UNSUPPORTED = -2, /* valid HSA call outside what the kernels implement (D, chunk, topk) */
+    HSA_ERR_WORKSPACE = -3,   /* workspace missing, misaligned or smaller than *_workspace_size */
+    HSA_ERR_CUDA = -4,        /* a CUDA runtime call failed; hsa_last_error() holds its text */
+    HSA_ERR_TIMEOUT = -5      /* reserved for bounded device-side waits */
+} hsa_status;
+
+/* Message describing the last non-OK status returned on the calling thread ("" if none). */
+const char *hsa_last_error(void);
+
+/* ---------------------------------------------------------------------------------------------
+ * Prefill forward (Steps 1-4 for every token of a sequence).
+ *
+ *   Q, K, V  [B, H, T, D] bf16      queries, keys, values
+ *   L        [B, H, T/64, D] bf16   one landmark per complete chunk (a trailing partial chunk has
+ *                                   no landmark and is never selected)
+ *   out      [B, H, T, D] bf16      required; rounded to nearest-even from fp32
+ *   sel_idx  [B, H, T, topk] int32  optional (NULL): selected chunk ids, by score descending then
+ *                                   chunk ascending; -1 padding
+ *   sel_w    [B, H, T, topk] fp32   optional (NULL): fusion weights in the same order; 0 padding
+ * Scores and softmaxes are computed in fp32 from bf16 inputs. Requires 1 <= T, B*H*T*topk < 2^31.
+ * ------------------------------------------------------------------------------------------- */
+size_t hsa_forward_workspace_size(int B, int H, int T, int D, int chunk, int topk);
+
+hsa_status hsa_forward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, const hsa_bf16 *L, int B, int H,
+                       int T, int D, int chunk, int topk, float scale, hsa_bf16 *out, int32_t *sel_idx,
+                       float *sel_w, void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Decode: one new query token per sequence against a cached history (Steps 2-4 with the query
+ * at the last cached position, so it sees n = cache_len[b] / 64 complete chunks).
+ *
+ *   q          [B, H, D] bf16
+ *   Kc, Vc     [B, H, Tmax, D] bf16     key / value cache
+ *   Lc         [B, H, Tmax/64, D] bf16  landmark cache
+ *   cache_len  [B] int64, DEVICE        tokens held by each sequence, 0 <= cache_len[b] <= Tmax
+ *   out        [B, H, D] bf16           required
+ *   sel_idx    [B, H, topk] int32       optional; sel_w [B, H, topk] fp32 optional
+ * The landmark scan is split over chunk ranges (split-over-chunks); each range keeps its exact
+ * top-K and the ranges are merged exactly, so the result equals a single global top-K.
+ * ------------------------------------------------------------------------------------------- */
+size_t hsa_decode_workspace_size(int B, int H, int64_t Tmax, int D, int chunk, int topk);
+
+hsa_status hsa_decode(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc, const hsa_bf16 *Lc,
+                      const int64_t *cache_len, int64_t Tmax, int B, int H, int D, int chunk, int topk,
+                      float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace,
+                      size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Backward of hsa_forward for the selection the forward made.
+ *
+ *   Q, K, V, L, out as in hsa_forward (out = the forward's output); dout [B, H, T, D] bf16
+ *   sel_idx [B, H, T, topk] int32, sel_w [B, H, T, topk] fp32: the forward's selection (required)
+ *   dQ, dK, dV [B, H, T, D] fp32, dL [B, H, T/64, D] fp32: overwritten (zeroed by the call)
+ * Chain rule through Step 3 (per-chunk softmax) and Step 4 (fusion softmax over the selected
+ * scores); the discrete selection is treated as constant.
+ * ------------------------------------------------------------------------------------------- */
+size_t hsa_backward_workspace_size(int B, int H, int T, int D, int chunk, int topk);
+
+hsa_status hsa_backward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, const hsa_bf16 *L,
+                        const hsa_bf16 *out, const hsa_bf16 *dout, const int32_t *sel_idx, const float *sel_w,
+                        int B, int H, int T, int D, int chunk, int topk, float scale, float *dQ, float *dK,
+                        float *dV, float *dL, void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Measurement hooks (no counterpart on the pages; used to time each kernel live).
+ *
+ * hsa_profile_enable(1) starts recording a pair of CUDA events around every kernel launch and
+ * memset the library issues, on the stream it is issued on (0 stops recording); either call
+ * discards earlier records. hsa_profile_summary() waits for the recorded events and writes one line
+ * per launch site, "name,launches,total_ms\n", into buf (truncated to cap - 1 bytes, NUL-terminated);
+ * it returns the full text length, or -1 if an event query failed. Host-side only; thread-safe.
+ * ------------------------------------------------------------------------------------------- */
+int hsa_profile_enable(int on);
+int hsa_profile_summary(char *buf, size_t cap);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSA_B200_H */

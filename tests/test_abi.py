@@ -1,0 +1,96 @@
+"""The C ABI without a GPU: the library loads, exports every function include/hsa.h declares, sizes
+its workspaces, and rejects invalid calls on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from ultra_long_context_b200 import hsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hsa.h")
+
+# a fake, 256-byte aligned address: only ever passed to calls that fail validation first
+FAKE = ctypes.c_void_p(1 << 20)
+ODD = ctypes.c_void_p((1 << 20) + 2)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_ ]*?\**\s*\**(hsa_[a-z0-9_]+)\s*\(",
+                                 text, flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_functions()
+    assert {"hsa_forward", "hsa_decode", "hsa_backward", "hsa_last_error"} <= set(names)
+    lib = ctypes.CDLL(hsa.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(hsa.SIGNATURES), "binding must declare every C entry point"
+
+
+def test_workspace_sizes_are_positive_and_monotone():
+    a = hsa.hsa_forward_workspace_size(1, 4, 4096, 64, 64, 8)
+    b = hsa.hsa_forward_workspace_size(2, 8, 32768, 128, 64, 16)
+    assert 0 < a < b
+    assert b >= 2 * 8 * 32768 * 128 * 4          # holds the fp32 output accumulator
+    assert hsa.hsa_decode_workspace_size(1, 8, 1 << 24, 128, 64, 32) > 0
+    assert hsa.hsa_backward_workspace_size(1, 8, 65536, 128, 64, 16) > 0
+    assert hsa.hsa_forward_workspace_size(0, 4, 4096, 64, 64, 8) == 0
+
+
+def _fwd(**kw):
+    args = dict(Q=FAKE, K=FAKE, V=FAKE, L=FAKE, B=1, H=1, T=256, D=64, chunk=64, topk=8, scale=0.0, out=FAKE,
+                sel_idx=None, sel_w=None, ws=FAKE, ws_bytes=1 << 40, stream=None)
+    args.update(kw)
+    return hsa.lib().hsa_forward(*args.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=96), -2), (dict(D=256), -2), (dict(chunk=32), -2), (dict(topk=33), -2),
+    (dict(topk=0), -1), (dict(B=0), -1), (dict(T=0), -1), (dict(Q=None), -1), (dict(out=None), -1),
+    (dict(L=None), -1), (dict(K=ODD), -1), (dict(sel_w=ODD), -1),
+    (dict(ws=None), -3), (dict(ws_bytes=100), -3), (dict(ws=ctypes.c_void_p((1 << 20) + 16)), -3),
+])
+def test_forward_rejects_invalid_calls_on_host(kw, status):
+    assert _fwd(**kw) == status
+    assert hsa.hsa_last_error() != ""
+
+
+def _dec(**kw):
+    args = dict(q=FAKE, Kc=FAKE, Vc=FAKE, Lc=FAKE, cache_len=FAKE, Tmax=1 << 20, B=2, H=2, D=128, chunk=64,
+                topk=16, scale=0.0, out=FAKE, sel_idx=None, sel_w=None, ws=FAKE, ws_bytes=1 << 40, stream=None)
+    args.update(kw)
+    return hsa.lib().hsa_decode(*args.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=80), -2), (dict(topk=65), -2), (dict(chunk=128), -2), (dict(Tmax=-1), -1), (dict(cache_len=None), -1),
+    (dict(Lc=ODD), -1), (dict(ws_bytes=8), -3),
+])
+def test_decode_rejects_invalid_calls_on_host(kw, status):
+    assert _dec(**kw) == status
+
+
+def _bwd(**kw):
+    args = dict(Q=FAKE, K=FAKE, V=FAKE, L=FAKE, out=FAKE, dout=FAKE, sel_idx=FAKE, sel_w=FAKE, B=1, H=1, T=256,
+                D=128, chunk=64, topk=16, scale=0.0, dQ=FAKE, dK=FAKE, dV=FAKE, dL=FAKE, ws=FAKE, ws_bytes=1 << 40,
+                stream=None)
+    args.update(kw)
+    return hsa.lib().hsa_backward(*args.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=32), -2), (dict(topk=40), -2), (dict(sel_idx=None), -1), (dict(dL=None), -1), (dict(dout=ODD), -1),
+    (dict(ws=None), -3),
+])
+def test_backward_rejects_invalid_calls_on_host(kw, status):
+    assert _bwd(**kw) == status
+
+
+def test_binding_raises_with_message():
+    with pytest.raises(hsa.HSAError, match="HSA_ERR_UNSUPPORTED"):
+        hsa._check("hsa_forward", _fwd(D=96))

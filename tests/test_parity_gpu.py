@@ -1,0 +1,226 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on seeded synthetic inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from tests.parity import compare_forward_rows, grad_close
+from ultra_long_context_b200 import hsa, inputs
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def host(x):
+    return x.float().cpu().numpy()
+
+
+def run_forward_case(oracle_mod, B, H, T, D, topk, seed, landmarks="iid", rows=None):
+    Q, K, V, L = inputs.forward_inputs(B, H, T, D, seed, landmarks=landmarks, device=DEV)
+    out, idx, w = hsa.hsa_forward(Q, K, V, L, topk)
+    torch.cuda.synchronize()
+    Qh, Kh, Vh, Lh = (host(x) for x in (Q, K, V, L))
+    scale = 1.0 / math.sqrt(D)
+    if rows is None:
+        rows = np.arange(B * H * T)
+    orc = oracle_mod.forward(Qh, Kh, Vh, Lh, chunk=64, topk=topk, scale=scale, rows=rows)
+    rr = torch.as_tensor(rows, device=DEV)
+    g_out = host(out.reshape(-1, D)[rr])
+    g_idx = idx.reshape(-1, topk)[rr].cpu().numpy()
+    g_w = w.reshape(-1, topk)[rr].cpu().numpy()
+    stats = compare_forward_rows(oracle_mod, g_out, g_idx, g_w, orc, Qh, Kh, Vh, Lh, rows, 64, scale)
+    # invariants that hold for every row: causal selection, weights sum to one, padding
+    t = rows % T
+    n_t = np.minimum((t + 1) // 64, T // 64)
+    assert np.all(g_idx < n_t[:, None])
+    k_t = np.minimum(n_t, topk)
+    assert np.all((g_idx >= 0).sum(1) == k_t)
+    wsum = g_w.sum(1)
+    assert np.allclose(wsum[k_t > 0], 1.0, atol=1e-5) and np.all(wsum[k_t == 0] == 0)
+    assert np.all(g_out[k_t == 0] == 0)
+    return stats, (Q, K, V, L, out, idx, w)
+
+
+@pytest.mark.parametrize("B,H,T,D,topk,landmarks", [
+    (1, 4, 4096, 64, 8, "iid"),            # the small benchmark workload, every row
+    (2, 2, 4096 + 37, 128, 16, "chunk_mean"),  # ragged tail, several 128-row tiles
+    (1, 2, 130, 64, 5, "iid"),             # topk above n_t; topk not a list length
+    (1, 1, 50, 128, 4, "iid"),             # no complete chunk at all
+    (1, 2, 1024, 128, 1, "iid"),
+    (1, 2, 2048 + 64, 64, 32, "iid"),
+    (1, 1, 64 * 40 + 63, 128, 3, "chunk_mean"),
+])
+def test_forward_matches_oracle(oracle_mod, B, H, T, D, topk, landmarks):
+    stats, _ = run_forward_case(oracle_mod, B, H, T, D, topk, seed=100 + T + topk, landmarks=landmarks)
+    assert stats["rows"] == B * H * T
+
+
+def test_forward_equal_scores_keep_lowest_chunks(oracle_mod):
+    B, H, T, D, topk = 1, 2, 640, 64, 4
+    Q, K, V, L = inputs.forward_inputs(B, H, T, D, 7, device=DEV)
+    L[:] = L[:, :, :1, :]
+    out, idx, w = hsa.hsa_forward(Q, K, V, L, topk)
+    idx = idx.cpu().numpy().reshape(-1, topk)
+    w = w.cpu().numpy().reshape(-1, topk)
+    for r in range(B * H * T):
+        n = min((r % T + 1) // 64, T // 64)
+        k = min(n, topk)
+        assert idx[r].tolist() == list(range(k)) + [-1] * (topk - k)
+        if k:
+            assert np.allclose(w[r, :k], 1.0 / k, atol=1e-6)
+
+
+def test_forward_full_size_32k_sampled_rows(oracle_mod):
+    """B2 T32768 H8 D128 topk16 with chunk-mean landmarks, checked on 1024 sampled rows plus edges."""
+    w = inputs.WORKLOADS["fwd_t32k_h8_d128_k16"]
+    rng = np.random.default_rng(5)
+    BH, T = w.B * w.H, w.T
+    edges = [bh * T + t for bh in (0, BH - 1) for t in (0, 62, 63, 64, 127, 128, 4095, T - 65, T - 1)]
+    rows = np.unique(np.concatenate([rng.integers(0, BH * T, 1024), edges]))
+    stats, _ = run_forward_case(oracle_mod, w.B, w.H, w.T, w.D, w.topk, w.seed, w.landmarks, rows=rows)
+    assert stats["rows"] == len(rows)
+
+
+def test_forward_is_deterministic_in_selection_and_close_in_output():
+    Q, K, V, L = inputs.forward_inputs(1, 2, 4096, 128, 3, device=DEV)
+    o1, i1, w1 = hsa.hsa_forward(Q, K, V, L, 16)
+    o2, i2, w2 = hsa.hsa_forward(Q, K, V, L, 16)
+    assert torch.equal(i1, i2) and torch.equal(w1, w2)
+    assert (o1.float() - o2.float()).abs().max().item() <= 2e-2
+
+
+# ---------------------------------------------------------------------------------------------
+# decode
+
+
+def oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, chunk=64):
+    """Oracle decode: selection from (q, Lc) on the host, then the selected chunks gathered."""
+    B, H, D = q.shape
+    sel = oracle_mod.decode_select(host(q), host(Lc), lens.cpu().numpy(), chunk=chunk, topk=topk,
+                                   scale=1 / math.sqrt(D))
+    idx = torch.as_tensor(sel["sel_idx"], device=Kc.device, dtype=torch.int64).clamp(min=0)   # [B,H,k]
+    tok = (idx[..., None] * chunk + torch.arange(chunk, device=Kc.device)).reshape(B, H, -1)
+    Kg = torch.gather(Kc, 2, tok[..., None].expand(-1, -1, -1, D)).reshape(B * H, topk, chunk, D)
+    Vg = torch.gather(Vc, 2, tok[..., None].expand(-1, -1, -1, D)).reshape(B * H, topk, chunk, D)
+    Lg = torch.gather(Lc, 2, idx[..., None].expand(-1, -1, -1, D)).reshape(B * H, topk, D)
+    nsel = (sel["sel_idx"] >= 0).sum(-1).reshape(-1)
+    out, w = oracle_mod.attend_gathered(host(q).reshape(B * H, D), host(Lg), host(Kg), host(Vg), nsel,
+                                        scale=1 / math.sqrt(D))
+    return dict(out=out, sel_idx=sel["sel_idx"].reshape(B * H, topk), sel_w=w, sel_s=sel["sel_s"].reshape(B * H, topk),
+                next_s=sel["next_s"].reshape(-1))
+
+
+def check_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk):
+    B, H, D = q.shape
+    out, idx, w = hsa.hsa_decode(q, Kc, Vc, Lc, lens, topk)
+    torch.cuda.synchronize()
+    orc = oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk)
+    g_idx = idx.reshape(B * H, topk).cpu().numpy()
+    g_w = w.reshape(B * H, topk).cpu().numpy()
+    g_out = host(out).reshape(B * H, D)
+    for i in range(B * H):
+        gs, os_ = set(g_idx[i][g_idx[i] >= 0].tolist()), set(orc["sel_idx"][i][orc["sel_idx"][i] >= 0].tolist())
+        if gs != os_:
+            k = len(os_)
+            assert orc["sel_s"][i, k - 1] - orc["next_s"][i] < 1e-3, f"(b,h)={i}: selection differs"
+            continue
+        d = np.abs(g_out[i] - orc["out"][i])
+        assert d.max() <= 2e-2
+        og = dict(zip(orc["sel_idx"][i].tolist(), orc["sel_w"][i].tolist()))
+        for c, ww in zip(g_idx[i].tolist(), g_w[i].tolist()):
+            if c >= 0:
+                assert abs(ww - og[c]) <= 1e-3
+    # ordering: by score descending (ties to the lower index) -> sel_w non-increasing
+    assert np.all(np.diff(g_w, axis=1) <= 1e-6)
+    return out, idx, w
+
+
+@pytest.mark.parametrize("B,H,D,Tmax,lens,topk", [
+    (3, 2, 128, 8192, [8192, 5000, 40], 16),
+    (2, 2, 64, 64 * 300, [64 * 300, 64 * 300 - 1], 64),
+    (1, 4, 128, 64 * 5000 + 17, [64 * 5000 + 17], 32),   # several scan ranges, ragged tail
+    (4, 1, 64, 256, [0, 63, 64, 200], 8),
+])
+def test_decode_matches_oracle(oracle_mod, B, H, D, Tmax, lens, topk):
+    q, Kc, Vc, Lc, lens_t, needle = inputs.decode_inputs(B, H, lens, D, seed=300 + Tmax, Tmax=Tmax, device=DEV)
+    out, idx, w = check_decode(oracle_mod, q, Kc, Vc, Lc, lens_t, topk)
+    for b in range(B):
+        n = lens[b] // 64
+        if n == 0:
+            assert torch.all(out[b] == 0) and torch.all(idx[b] == -1) and torch.all(w[b] == 0)
+        elif needle[b] >= 0:
+            assert torch.all(idx[b, :, 0] == int(needle[b]))
+
+
+def test_decode_equals_forward_last_row():
+    B, H, T, D, topk = 2, 2, 4096 + 64, 128, 16
+    Q, K, V, L = inputs.forward_inputs(B, H, T, D, 11, device=DEV)
+    out, idx, w = hsa.hsa_forward(Q, K, V, L, topk)
+    lens = torch.full((B,), T, dtype=torch.int64, device=DEV)
+    o2, i2, w2 = hsa.hsa_decode(Q[:, :, T - 1].contiguous(), K, V, L, lens, topk)
+    assert torch.equal(i2, idx[:, :, T - 1])
+    assert (w2 - w[:, :, T - 1]).abs().max().item() <= 1e-5
+    assert (o2.float() - out[:, :, T - 1].float()).abs().max().item() <= 2e-2
+
+
+@pytest.mark.parametrize("name", ["decode_1m_b16_h8_d128_k16", "decode_16m_b1_h8_d128_k32"])
+def test_decode_full_size(oracle_mod, name):
+    w = inputs.WORKLOADS[name]
+    q, Kc, Vc, Lc, lens, needle = inputs.workload_inputs(w, device=DEV)
+    out, idx, ww = check_decode(oracle_mod, q, Kc, Vc, Lc, lens, w.topk)
+    for b in range(w.B):
+        assert torch.all(idx[b, :, 0] == int(needle[b]))
+    del q, Kc, Vc, Lc
+    torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------------------------------------
+# backward
+
+
+@pytest.mark.parametrize("B,H,T,D,topk", [(1, 2, 1100, 64, 8), (1, 1, 2048 + 64, 128, 16), (2, 1, 700, 128, 5)])
+def test_backward_matches_oracle(oracle_mod, B, H, T, D, topk):
+    Q, K, V, L = inputs.forward_inputs(B, H, T, D, 500 + T, device=DEV)
+    dO = inputs.upstream_grad(B, H, T, D, 500 + T, device=DEV)
+    Qh, Kh, Vh, Lh, dOh = (host(x) for x in (Q, K, V, L, dO))
+    scale = 1 / math.sqrt(D)
+    orc = oracle_mod.forward(Qh, Kh, Vh, Lh, chunk=64, topk=topk, scale=scale)
+    sel_idx = torch.as_tensor(orc["sel_idx"].reshape(B, H, T, topk), device=DEV)
+    sel_w = torch.as_tensor(orc["sel_w"].reshape(B, H, T, topk), dtype=torch.float32, device=DEV)
+    out = torch.as_tensor(orc["out"].reshape(B, H, T, D), dtype=torch.float32, device=DEV).to(torch.bfloat16)
+    grads = hsa.hsa_backward(Q, K, V, L, out, dO, sel_idx, sel_w)
+    ref = oracle_mod.backward(Qh, Kh, Vh, Lh, dOh, orc["sel_idx"].reshape(B, H, T, topk), chunk=64, scale=scale)
+    for g, r, n in zip(grads, ref, ("dQ", "dK", "dV", "dL")):
+        grad_close(host(g), r, n)
+
+
+def test_backward_full_size_properties():
+    """B1 T65536 H8 D128 topk16, forward then backward on the GPU, checked by properties that hold at
+    any size: every gradient is finite; since each row of P sums to one, the sum of dV over a chunk's
+    64 keys equals the sum over the chunk's pairs of w * dO; chunks that no token selected get zero
+    dK, dV and dL."""
+    w = inputs.WORKLOADS["fwdbwd_t64k_h8_d128_k16"]
+    Q, K, V, L, dO = inputs.workload_inputs(w, device=DEV)
+    out, idx, sw = hsa.hsa_forward(Q, K, V, L, w.topk)
+    dQ, dK, dV, dL = hsa.hsa_backward(Q, K, V, L, out, dO, idx, sw)
+    torch.cuda.synchronize()
+    for g in (dQ, dK, dV, dL):
+        assert torch.isfinite(g).all()
+    B, H, T, D, N = w.B, w.H, w.T, w.D, w.T // 64
+    for b in range(B):
+        for h in range(H):
+            lhs = dV[b, h].reshape(N, 64, D).sum(1).double()
+            valid = idx[b, h] >= 0
+            rows = torch.arange(T, device=DEV)[:, None].expand(T, w.topk)[valid]
+            chunks = idx[b, h][valid].long()
+            contrib = sw[b, h][valid].double()[:, None] * dO[b, h][rows].double()
+            rhs = torch.zeros(N, D, dtype=torch.float64, device=DEV).index_add_(0, chunks, contrib)
+            err = (lhs - rhs).abs().max().item()
+            assert err <= 2e-2 * max(1.0, rhs.abs().max().item()), err
+            hit = torch.zeros(N, dtype=torch.bool, device=DEV)
+            hit[chunks] = True
+            assert torch.all(dL[b, h][~hit] == 0)
+            assert torch.all(dK[b, h].reshape(N, 64 * D)[~hit] == 0)
+            assert torch.all(dV[b, h].reshape(N, 64 * D)[~hit] == 0)

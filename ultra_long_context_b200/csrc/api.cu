@@ -1,0 +1,259 @@
+// api.cu -- the C ABI declared in include/hsa.h: host-side validation, workspace carving and
+// launches on the caller's stream. Nothing here synchronises, allocates device memory or computes
+// any part of the operator; every step of HSA runs in the kernels of decode.cu / prefill.cu /
+// backward.cu.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/hsa.h"
+#include "common.cuh"
+#include "launch.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+hsa_status fail(hsa_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+hsa_status cuda_status(cudaError_t e, const char *where) {
+    if (e == cudaSuccess) return HSA_OK;
+    return fail(HSA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Sequential carve-out of a caller-provided workspace.
+struct Carver {
+    char *base;
+    size_t used = 0;
+    template <typename T>
+    T *take(size_t count) {
+        T *p = base ? reinterpret_cast<T *>(base + used) : nullptr;
+        used += round_up(count * sizeof(T));
+        return p;
+    }
+};
+
+hsa_status check_common(int B, int H, int D, int chunk, int topk, int topk_max) {
+    if (B < 1 || H < 1) return fail(HSA_ERR_INVALID_ARG, "B and H must be >= 1 (got B=%d H=%d)", B, H);
+    if (topk < 1) return fail(HSA_ERR_INVALID_ARG, "topk must be >= 1 (got %d)", topk);
+    if (D < 1) return fail(HSA_ERR_INVALID_ARG, "D must be >= 1 (got %d)", D);
+    if (chunk < 1) return fail(HSA_ERR_INVALID_ARG, "chunk must be >= 1 (got %d)", chunk);
+    if (D != 64 && D != 128) return fail(HSA_ERR_UNSUPPORTED, "head dim D=%d not supported (64 or 128)", D);
+    if (chunk != hsa::kChunk) return fail(HSA_ERR_UNSUPPORTED, "chunk=%d not supported (64 only)", chunk);
+    if (topk > topk_max) return fail(HSA_ERR_UNSUPPORTED, "topk=%d not supported (max %d)", topk, topk_max);
+    return HSA_OK;
+}
+
+hsa_status check_ws(void *ws, size_t bytes, size_t need) {
+    if (need == 0) return HSA_OK;
+    if (!ws) return fail(HSA_ERR_WORKSPACE, "workspace is NULL but %zu bytes are needed", need);
+    if (reinterpret_cast<uintptr_t>(ws) % kAlign) return fail(HSA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+    if (bytes < need) return fail(HSA_ERR_WORKSPACE, "workspace too small: %zu < %zu bytes", bytes, need);
+    return HSA_OK;
+}
+
+// ---- forward / backward workspace layout ----
+struct FwdLayout {
+    float *o_acc;
+    int32_t *sel_idx;
+    float *sel_w;
+    int32_t *chunk_count, *chunk_off, *chunk_cursor, *pair_row;
+    float *pair_w;
+    hsa::PairTile *tiles;
+    int32_t *num_tiles;
+    float *delta;
+    int32_t *pair_slot;
+    size_t bytes;
+    int max_tiles;
+};
+
+FwdLayout fwd_layout(void *ws, int B, int H, int T, int D, int topk, bool backward) {
+    FwdLayout l{};
+    Carver c{static_cast<char *>(ws)};
+    const size_t rows = (size_t)B * H * T, chunks = (size_t)B * H * (T / 64), pairs = rows * topk;
+    l.max_tiles = (int)hsa::forward_max_tiles(B, H, T, topk);
+    l.o_acc = backward ? nullptr : c.take<float>(rows * D);
+    l.sel_idx = backward ? nullptr : c.take<int32_t>(pairs);
+    l.sel_w = backward ? nullptr : c.take<float>(pairs);
+    l.chunk_count = c.take<int32_t>(chunks);
+    l.chunk_off = c.take<int32_t>(chunks + 1);
+    l.chunk_cursor = c.take<int32_t>(chunks);
+    l.pair_row = c.take<int32_t>(pairs);
+    l.pair_w = c.take<float>(pairs);
+    l.tiles = c.take<hsa::PairTile>((size_t)l.max_tiles);
+    l.num_tiles = c.take<int32_t>(1);
+    l.delta = backward ? c.take<float>(rows) : nullptr;
+    l.pair_slot = backward ? c.take<int32_t>(pairs) : nullptr;
+    l.bytes = c.used;
+    return l;
+}
+
+struct DecLayout {
+    uint64_t *cand;
+    unsigned *counters;
+    int32_t *sel_idx;
+    float *sel_w, *partial;
+    size_t bytes;
+};
+
+DecLayout dec_layout(void *ws, int B, int H, int64_t Tmax, int D, int topk) {
+    DecLayout l{};
+    Carver c{static_cast<char *>(ws)};
+    const int64_t Nmax = Tmax / 64;
+    const int split = hsa::decode_split_size(Nmax, topk);
+    const int64_t nsplit = Nmax > 0 ? (Nmax + split - 1) / split : 1;
+    const size_t BH = (size_t)B * H;
+    l.cand = c.take<uint64_t>(BH * nsplit * topk);
+    l.counters = c.take<unsigned>(2 * BH);
+    l.sel_idx = c.take<int32_t>(BH * topk);
+    l.sel_w = c.take<float>(BH * topk);
+    l.partial = c.take<float>(BH * topk * D);
+    l.bytes = c.used;
+    return l;
+}
+
+float resolve_scale(float scale, int D) { return scale > 0.0f ? scale : 1.0f / sqrtf((float)D); }
+
+}  // namespace
+
+extern "C" {
+
+const char *hsa_last_error(void) { return g_last_error.c_str(); }
+
+size_t hsa_forward_workspace_size(int B, int H, int T, int D, int chunk, int topk) {
+    (void)chunk;
+    if (B < 1 || H < 1 || T < 1 || D < 1 || topk < 1) return 0;
+    return fwd_layout(nullptr, B, H, T, D, topk, false).bytes;
+}
+
+hsa_status hsa_forward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, const hsa_bf16 *L, int B, int H,
+                       int T, int D, int chunk, int topk, float scale, hsa_bf16 *out, int32_t *sel_idx,
+                       float *sel_w, void *workspace, size_t workspace_bytes, void *stream) {
+    g_last_error.clear();
+    hsa_status st = check_common(B, H, D, chunk, topk, 32);
+    if (st != HSA_OK) return st;
+    if (T < 1) return fail(HSA_ERR_INVALID_ARG, "T must be >= 1 (got %d)", T);
+    if ((double)B * H * T * topk >= 2147483647.0 || (double)B * H * T * D >= 9.0e15)
+        return fail(HSA_ERR_UNSUPPORTED, "B*H*T*topk must stay below 2^31");
+    if (!Q || !K || !V || !out) return fail(HSA_ERR_INVALID_ARG, "Q, K, V and out must not be NULL");
+    if (T >= 64 && !L) return fail(HSA_ERR_INVALID_ARG, "L must not be NULL when T >= 64");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || (L && !aligned16(L)))
+        return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if ((sel_idx && !aligned16(sel_idx)) || (sel_w && !aligned16(sel_w)))
+        return fail(HSA_ERR_INVALID_ARG, "sel_idx / sel_w must be 16-byte aligned");
+    FwdLayout need = fwd_layout(nullptr, B, H, T, D, topk, false);
+    if ((st = check_ws(workspace, workspace_bytes, need.bytes)) != HSA_OK) return st;
+    FwdLayout l = fwd_layout(workspace, B, H, T, D, topk, false);
+    hsa::ForwardArgs a{};
+    a.Q = Q; a.K = K; a.V = V; a.L = L;
+    a.B = B; a.H = H; a.T = T; a.D = D; a.N = T / 64; a.topk = topk;
+    a.scale = resolve_scale(scale, D);
+    a.out = out;
+    a.sel_idx = sel_idx ? sel_idx : l.sel_idx;
+    a.sel_w = sel_w ? sel_w : l.sel_w;
+    a.o_acc = l.o_acc;
+    a.chunk_count = l.chunk_count; a.chunk_off = l.chunk_off; a.chunk_cursor = l.chunk_cursor;
+    a.pair_row = l.pair_row; a.pair_w = l.pair_w; a.tiles = l.tiles; a.num_tiles = l.num_tiles;
+    a.max_tiles = l.max_tiles;
+    return cuda_status(hsa::launch_forward(a, static_cast<cudaStream_t>(stream)), "hsa_forward");
+}
+
+size_t hsa_decode_workspace_size(int B, int H, int64_t Tmax, int D, int chunk, int topk) {
+    (void)chunk;
+    if (B < 1 || H < 1 || Tmax < 0 || D < 1 || topk < 1) return 0;
+    return dec_layout(nullptr, B, H, Tmax, D, topk).bytes;
+}
+
+hsa_status hsa_decode(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc, const hsa_bf16 *Lc,
+                      const int64_t *cache_len, int64_t Tmax, int B, int H, int D, int chunk, int topk,
+                      float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace,
+                      size_t workspace_bytes, void *stream) {
+    g_last_error.clear();
+    hsa_status st = check_common(B, H, D, chunk, topk, 64);
+    if (st != HSA_OK) return st;
+    if (Tmax < 0) return fail(HSA_ERR_INVALID_ARG, "Tmax must be >= 0");
+    if (Tmax / 64 >= 2147483647LL) return fail(HSA_ERR_UNSUPPORTED, "Tmax / 64 must stay below 2^31");
+    if (!q || !Kc || !Vc || !Lc || !cache_len || !out)
+        return fail(HSA_ERR_INVALID_ARG, "q, Kc, Vc, Lc, cache_len and out must not be NULL");
+    if (!aligned16(q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(Lc) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(cache_len) & 7u))
+        return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned (cache_len 8-byte)");
+    if ((sel_idx && !aligned16(sel_idx)) || (sel_w && !aligned16(sel_w)))
+        return fail(HSA_ERR_INVALID_ARG, "sel_idx / sel_w must be 16-byte aligned");
+    {
+        const int64_t Nmax = Tmax / 64;
+        const int split = hsa::decode_split_size(Nmax, topk);
+        const int64_t nsplit = Nmax > 0 ? (Nmax + split - 1) / split : 1;
+        if (hsa::decode_scan_smem(split, (int)nsplit, topk) > 227 * 1024)
+            return fail(HSA_ERR_UNSUPPORTED, "Tmax=%lld too large for topk=%d (scan merge exceeds shared memory)",
+                        (long long)Tmax, topk);
+    }
+    DecLayout need = dec_layout(nullptr, B, H, Tmax, D, topk);
+    if ((st = check_ws(workspace, workspace_bytes, need.bytes)) != HSA_OK) return st;
+    DecLayout l = dec_layout(workspace, B, H, Tmax, D, topk);
+    hsa::DecodeArgs a{};
+    a.q = q; a.Kc = Kc; a.Vc = Vc; a.Lc = Lc; a.cache_len = cache_len;
+    a.Tmax = Tmax; a.Nmax = Tmax / 64;
+    a.B = B; a.H = H; a.D = D; a.K = topk;
+    a.scale = resolve_scale(scale, D);
+    a.out = out;
+    a.sel_idx = sel_idx ? sel_idx : l.sel_idx;
+    a.sel_w = sel_w ? sel_w : l.sel_w;
+    a.cand = l.cand; a.counters = l.counters; a.partial = l.partial;
+    return cuda_status(hsa::launch_decode(a, static_cast<cudaStream_t>(stream)), "hsa_decode");
+}
+
+size_t hsa_backward_workspace_size(int B, int H, int T, int D, int chunk, int topk) {
+    (void)chunk;
+    if (B < 1 || H < 1 || T < 1 || D < 1 || topk < 1) return 0;
+    return fwd_layout(nullptr, B, H, T, D, topk, true).bytes;
+}
+
+hsa_status hsa_backward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, const hsa_bf16 *L,
+                        const hsa_bf16 *out, const hsa_bf16 *dout, const int32_t *sel_idx, const float *sel_w,
+                        int B, int H, int T, int D, int chunk, int topk, float scale, float *dQ, float *dK,
+                        float *dV, float *dL, void *workspace, size_t workspace_bytes, void *stream) {
+    g_last_error.clear();
+    hsa_status st = check_common(B, H, D, chunk, topk, 32);
+    if (st != HSA_OK) return st;
+    if (T < 1) return fail(HSA_ERR_INVALID_ARG, "T must be >= 1 (got %d)", T);
+    if ((double)B * H * T * topk >= 2147483647.0)
+        return fail(HSA_ERR_UNSUPPORTED, "B*H*T*topk must stay below 2^31");
+    if (!Q || !K || !V || !out || !dout || !sel_idx || !sel_w || !dQ || !dK || !dV)
+        return fail(HSA_ERR_INVALID_ARG, "tensor pointers must not be NULL");
+    if (T >= 64 && (!L || !dL)) return fail(HSA_ERR_INVALID_ARG, "L and dL must not be NULL when T >= 64");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || !aligned16(dout) ||
+        !aligned16(sel_idx) || !aligned16(sel_w) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) ||
+        (L && !aligned16(L)) || (dL && !aligned16(dL)))
+        return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    FwdLayout need = fwd_layout(nullptr, B, H, T, D, topk, true);
+    if ((st = check_ws(workspace, workspace_bytes, need.bytes)) != HSA_OK) return st;
+    FwdLayout l = fwd_layout(workspace, B, H, T, D, topk, true);
+    hsa::BackwardArgs a{};
+    a.Q = Q; a.K = K; a.V = V; a.L = L; a.out = out; a.dout = dout;
+    a.sel_idx = sel_idx; a.sel_w = sel_w;
+    a.B = B; a.H = H; a.T = T; a.D = D; a.N = T / 64; a.topk = topk;
+    a.scale = resolve_scale(scale, D);
+    a.dQ = dQ; a.dK = dK; a.dV = dV; a.dL = dL;
+    a.delta = l.delta;
+    a.chunk_count = l.chunk_count; a.chunk_off = l.chunk_off; a.chunk_cursor = l.chunk_cursor;
+    a.pair_row = l.pair_row; a.pair_w = l.pair_w; a.pair_slot = l.pair_slot;
+    a.tiles = l.tiles; a.num_tiles = l.num_tiles; a.max_tiles = l.max_tiles;
+    return cuda_status(hsa::launch_backward(a, static_cast<cudaStream_t>(stream)), "hsa_backward");
+}
+
+}  // extern "C"

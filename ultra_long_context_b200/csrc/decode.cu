@@ -1,0 +1,251 @@
+// decode.cu -- HSA decode: one query token per sequence against a long KV/landmark cache.
+//
+// Explainer page of "Every Token Counts", "How It Works (Technically)": the token scores every
+// complete chunk's landmark (Step 2), keeps the top-K, attends inside each kept chunk (Step 3) and
+// blends by the softmax of the kept scores (Step 4). With a 1M-16M token cache the landmark scan is
+// the whole cost (hundreds of MiB streamed per step), so it is split over chunk ranges:
+//
+//   decode_scan_kernel     grid (splits, B*H). Streams its range of landmarks with 16-byte
+//                          coalesced loads (D/8 lanes per landmark), keeps the exact top-K of the
+//                          range (block radix select on unique 64-bit keys), writes K candidates.
+//                          The last CTA of each (b, h) to finish (atomic ticket, no waiting) merges
+//                          the candidates of all ranges exactly and writes sel_idx / sel_w.
+//   decode_attend_kernel   grid (K, B*H). One CTA per selected chunk: 64 logits, softmax, P.V_c;
+//                          the last CTA of each (b, h) blends the K chunk outputs and writes out.
+#include "common.cuh"
+#include "launch.h"
+#include "profile.h"
+
+namespace hsa {
+
+constexpr int kDecodeThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
+    const uint16_t *__restrict__ q, const uint16_t *__restrict__ Lc, const int64_t *__restrict__ cache_len, int H,
+    int64_t Nmax, int split, int nsplit, int K, float scale, uint64_t *__restrict__ cand, unsigned *counters,
+    int32_t *__restrict__ sel_idx, float *__restrict__ sel_w) {
+    constexpr int LPL = D / 8;              // lanes per landmark (one 16-byte vector each)
+    constexpr int LPW = 32 / LPL;           // landmarks per warp-wide load
+    constexpr int UNROLL = 8;               // independent loads in flight per lane
+    constexpr int WARP_SPAN = UNROLL * LPW; // consecutive landmarks per warp per batch
+    constexpr int NWARP = kDecodeThreads / 32;
+
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int cap = max(split, nsplit * K);
+    uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);
+    uint64_t *topk = keys + cap;            // 64
+    uint64_t *sorted = topk + 64;           // 64
+    uint32_t *hist = reinterpret_cast<uint32_t *>(sorted + 64);
+    int *misc = reinterpret_cast<int *>(hist + 256);  // 8 ints
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int sp = blockIdx.x, bh = blockIdx.y, b = bh / H;
+    int64_t nb = cache_len[b] / kChunk;
+    nb = nb < 0 ? 0 : (nb > Nmax ? Nmax : nb);
+    const int64_t c0 = (int64_t)sp * split;
+    const int64_t c1 = min(c0 + (int64_t)split, nb);
+    const int nloc = c1 > c0 ? (int)(c1 - c0) : 0;
+
+    const int g = lane / LPL, sub = lane % LPL;
+    float qr[8];
+    {
+        const uint4 v = *reinterpret_cast<const uint4 *>(q + (size_t)bh * D + sub * 8);
+        qr[0] = bf16_lo(v.x) * scale; qr[1] = bf16_hi(v.x) * scale;
+        qr[2] = bf16_lo(v.y) * scale; qr[3] = bf16_hi(v.y) * scale;
+        qr[4] = bf16_lo(v.z) * scale; qr[5] = bf16_hi(v.z) * scale;
+        qr[6] = bf16_lo(v.w) * scale; qr[7] = bf16_hi(v.w) * scale;
+    }
+    const uint16_t *Lbh = Lc + (size_t)bh * Nmax * D;
+    for (int64_t base = c0 + (int64_t)warp * WARP_SPAN; base < c1; base += (int64_t)NWARP * WARP_SPAN) {
+        uint4 v[UNROLL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            const int64_t c = base + u * LPW + g;
+            v[u] = c < c1 ? ld_stream16(Lbh + c * D + sub * 8) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+            float p = dot8(v[u], qr);
+#pragma unroll
+            for (int o = LPL / 2; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+            const int64_t c = base + u * LPW + g;
+            if (sub == 0 && c < c1) keys[c - c0] = make_key(p, (uint32_t)c);
+        }
+    }
+    __syncthreads();
+    const int cnt = block_topk_u64(keys, nloc, K, topk, hist, misc);
+    uint64_t *my_cand = cand + ((size_t)bh * nsplit + sp) * K;
+    for (int j = tid; j < K; j += kDecodeThreads) my_cand[j] = j < cnt ? topk[j] : 0ull;
+
+    // ---- last CTA of this (b, h) merges all ranges (ticket taken after a release fence) ----
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) misc[4] = (atomicAdd(&counters[bh], 1u) == (unsigned)(nsplit - 1));
+    __syncthreads();
+    if (!misc[4]) return;
+    __threadfence();
+    const int ncand = nsplit * K;
+    const uint64_t *all = cand + (size_t)bh * nsplit * K;
+    for (int i = tid; i < ncand; i += kDecodeThreads)
+        keys[i] = __ldcg(reinterpret_cast<const unsigned long long *>(all) + i);
+    __syncthreads();
+    const int m = block_topk_u64(keys, ncand, K, topk, hist, misc);
+    block_sort_desc_small(topk, m, sorted);  // empty (0) keys sort last
+    if (warp == 0) {
+        // fusion weights (Step 4): softmax over the kept scores, fp32, max-subtracted
+        const uint64_t k0 = lane < m ? sorted[lane] : 0ull;
+        const uint64_t k1 = lane + 32 < m ? sorted[lane + 32] : 0ull;
+        const float top = m > 0 && sorted[0] ? key_score(sorted[0]) : 0.0f;
+        const float e0 = k0 ? expf(key_score(k0) - top) : 0.0f;
+        const float e1 = k1 ? expf(key_score(k1) - top) : 0.0f;
+        const float z = warp_sum(e0 + e1);
+        for (int j = lane; j < K; j += 32) {
+            const uint64_t kk = j < 32 ? k0 : k1;
+            const float e = j < 32 ? e0 : e1;
+            sel_idx[(size_t)bh * K + j] = kk ? key_index(kk) : -1;
+            sel_w[(size_t)bh * K + j] = kk ? e / z : 0.0f;
+        }
+    }
+    if (tid == 0) counters[bh] = 0u;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
+    const uint16_t *__restrict__ q, const uint16_t *__restrict__ Kc, const uint16_t *__restrict__ Vc, int64_t Tmax,
+    int K, float scale, const int32_t *__restrict__ sel_idx, const float *__restrict__ sel_w,
+    float *__restrict__ partial, unsigned *counters, uint16_t *__restrict__ out) {
+    constexpr int LPL = D / 8, LPW = 32 / LPL, NWARP = kDecodeThreads / 32;
+    constexpr int GROUPS = kDecodeThreads / LPL;  // key groups for the P.V pass
+    constexpr int KEYS_PER_GROUP = kChunk / GROUPS;
+    __shared__ float s_p[kChunk];
+    __shared__ float s_red[GROUPS][D];
+    __shared__ int s_last;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int j = blockIdx.x, bh = blockIdx.y;
+    const int c = sel_idx[(size_t)bh * K + j];
+    float *my_part = partial + ((size_t)bh * K + j) * D;
+    if (c >= 0) {
+        const int g = lane / LPL, sub = lane % LPL;
+        float qr[8];
+        const uint4 qv = *reinterpret_cast<const uint4 *>(q + (size_t)bh * D + sub * 8);
+        qr[0] = bf16_lo(qv.x) * scale; qr[1] = bf16_hi(qv.x) * scale;
+        qr[2] = bf16_lo(qv.y) * scale; qr[3] = bf16_hi(qv.y) * scale;
+        qr[4] = bf16_lo(qv.z) * scale; qr[5] = bf16_hi(qv.z) * scale;
+        qr[6] = bf16_lo(qv.w) * scale; qr[7] = bf16_hi(qv.w) * scale;
+        const size_t row0 = ((size_t)bh * Tmax + (size_t)c * kChunk);
+        // Step 3 logits: a_u = scale * q . K_c[u]
+#pragma unroll
+        for (int r = 0; r < kChunk / (NWARP * LPW); ++r) {
+            const int u = (r * NWARP + warp) * LPW + g;
+            const uint4 kv = *reinterpret_cast<const uint4 *>(Kc + (row0 + u) * D + sub * 8);
+            float p = dot8(kv, qr);
+#pragma unroll
+            for (int o = LPL / 2; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+            if (sub == 0) s_p[u] = p;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            const float a0 = s_p[lane], a1 = s_p[lane + 32];
+            float mx = fmaxf(a0, a1);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const float e0 = expf(a0 - mx), e1 = expf(a1 - mx);
+            const float z = warp_sum(e0 + e1);
+            s_p[lane] = e0 / z;
+            s_p[lane + 32] = e1 / z;
+        }
+        __syncthreads();
+        // O_c = P . V_c
+        const int sl = tid % LPL, grp = tid / LPL;
+        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+        for (int i = 0; i < KEYS_PER_GROUP; ++i) {
+            const int u = grp * KEYS_PER_GROUP + i;
+            const uint4 vv = *reinterpret_cast<const uint4 *>(Vc + (row0 + u) * D + sl * 8);
+            const float p = s_p[u];
+            acc[0] = fmaf(p, bf16_lo(vv.x), acc[0]); acc[1] = fmaf(p, bf16_hi(vv.x), acc[1]);
+            acc[2] = fmaf(p, bf16_lo(vv.y), acc[2]); acc[3] = fmaf(p, bf16_hi(vv.y), acc[3]);
+            acc[4] = fmaf(p, bf16_lo(vv.z), acc[4]); acc[5] = fmaf(p, bf16_hi(vv.z), acc[5]);
+            acc[6] = fmaf(p, bf16_lo(vv.w), acc[6]); acc[7] = fmaf(p, bf16_hi(vv.w), acc[7]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s_red[grp][sl * 8 + e] = acc[e];
+        __syncthreads();
+        for (int d = tid; d < D; d += kDecodeThreads) {
+            float s = 0.0f;
+#pragma unroll 8
+            for (int gg = 0; gg < GROUPS; ++gg) s += s_red[gg][d];
+            my_part[d] = s;
+        }
+    }
+    // ---- last CTA of this (b, h) blends the K chunk outputs (Step 4) ----
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(&counters[bh], 1u) == (unsigned)(K - 1));
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int d = tid; d < D; d += kDecodeThreads) {
+        float o = 0.0f;
+        for (int jj = 0; jj < K; ++jj) {
+            if (sel_idx[(size_t)bh * K + jj] < 0) continue;
+            o = fmaf(sel_w[(size_t)bh * K + jj], __ldcg(partial + ((size_t)bh * K + jj) * D + d), o);
+        }
+        out[(size_t)bh * D + d] = (uint16_t)(pack_bf16x2(o, 0.0f) & 0xffffu);
+    }
+    if (tid == 0) counters[bh] = 0u;
+}
+
+int decode_split_size(int64_t Nmax, int K) {
+    int split = 2048;
+    while (split < 16384 && ((Nmax + split - 1) / split) * (int64_t)K > 8192) split *= 2;
+    return split;
+}
+
+size_t decode_scan_smem(int split, int nsplit, int K) {
+    const size_t cap = (size_t)(split > nsplit * K ? split : nsplit * K);
+    return (cap + 128) * sizeof(uint64_t) + 256 * sizeof(uint32_t) + 8 * sizeof(int);
+}
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
+    const int split = decode_split_size(a.Nmax, a.K);
+    const int nsplit = (int)((a.Nmax + split - 1) / split) > 0 ? (int)((a.Nmax + split - 1) / split) : 1;
+    const size_t smem = decode_scan_smem(split, nsplit, a.K);
+    const int BH = a.B * a.H;
+    cudaError_t e;
+    {
+        HSA_PROF("memset", s);
+        e = cudaMemsetAsync(a.counters, 0, 2 * (size_t)BH * sizeof(unsigned), s);
+    }
+    if (e != cudaSuccess) return e;
+    dim3 g1(nsplit, BH), g2(a.K, BH);
+    if (a.D == 128) {
+        e = cudaFuncSetAttribute(decode_scan_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        {
+            HSA_PROF("decode_scan", s);
+            decode_scan_kernel<128><<<g1, kDecodeThreads, smem, s>>>(a.q, a.Lc, a.cache_len, a.H, a.Nmax, split,
+                                                                     nsplit, a.K, a.scale, a.cand, a.counters,
+                                                                     a.sel_idx, a.sel_w);
+        }
+        HSA_PROF("decode_attend", s);
+        decode_attend_kernel<128><<<g2, kDecodeThreads, 0, s>>>(a.q, a.Kc, a.Vc, a.Tmax, a.K, a.scale, a.sel_idx,
+                                                                a.sel_w, a.partial, a.counters + BH, a.out);
+    } else {
+        e = cudaFuncSetAttribute(decode_scan_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        {
+            HSA_PROF("decode_scan", s);
+            decode_scan_kernel<64><<<g1, kDecodeThreads, smem, s>>>(a.q, a.Lc, a.cache_len, a.H, a.Nmax, split,
+                                                                    nsplit, a.K, a.scale, a.cand, a.counters,
+                                                                    a.sel_idx, a.sel_w);
+        }
+        HSA_PROF("decode_attend", s);
+        decode_attend_kernel<64><<<g2, kDecodeThreads, 0, s>>>(a.q, a.Kc, a.Vc, a.Tmax, a.K, a.scale, a.sel_idx,
+                                                               a.sel_w, a.partial, a.counters + BH, a.out);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace hsa

@@ -1,0 +1,81 @@
+// launch.h -- internal interface between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace hsa {
+
+struct DecodeArgs {
+    const uint16_t *q, *Kc, *Vc, *Lc;
+    const int64_t *cache_len;
+    int64_t Tmax, Nmax;
+    int B, H, D, K;
+    float scale;
+    uint16_t *out;
+    int32_t *sel_idx;  // [B*H, K] (caller's or workspace)
+    float *sel_w;      // [B*H, K]
+    uint64_t *cand;    // [B*H, nsplit, K]
+    unsigned *counters;  // [2, B*H]
+    float *partial;    // [B*H, K, D]
+};
+int decode_split_size(int64_t Nmax, int K);
+size_t decode_scan_smem(int split, int nsplit, int K);
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+
+// Chunk-major work list entry: one tile of up to kPairTile (token, slot) pairs of one chunk.
+struct PairTile {
+    int32_t chunk;  // flat (b*H + h) * N + c
+    int32_t start;  // first pair (offset into the pair arrays)
+    int32_t count;  // pairs in this tile (1 .. kPairTile)
+    int32_t pad;
+};
+constexpr int kPairTile = 64;
+
+struct ForwardArgs {
+    const uint16_t *Q, *K, *V, *L;
+    int B, H, T, D, N, topk;
+    float scale;
+    uint16_t *out;
+    int32_t *sel_idx;  // [B*H*T, topk] (caller's or workspace)
+    float *sel_w;
+    // workspace
+    float *o_acc;          // [B*H*T, D] fp32 accumulator
+    int32_t *chunk_count;  // [B*H*N]
+    int32_t *chunk_off;    // [B*H*N + 1]
+    int32_t *chunk_cursor; // [B*H*N]
+    int32_t *pair_row;     // [B*H*T*topk] flat token row (b*H + h)*T + t
+    float *pair_w;         // [B*H*T*topk]
+    PairTile *tiles;       // [max_tiles]
+    int32_t *num_tiles;    // [1]
+    int max_tiles;
+};
+size_t forward_max_tiles(int B, int H, int T, int topk);
+cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s);
+// Chunk-major dispatch shared by the forward and the backward: per-chunk pair counts, offsets, the
+// tile work list, and the (token row, weight[, slot]) pair arrays.
+cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, int H, int T, int N, int topk,
+                            int32_t *chunk_count, int32_t *chunk_off, int32_t *chunk_cursor, int32_t *pair_row,
+                            float *pair_w, int32_t *pair_slot, PairTile *tiles, int32_t *num_tiles, int max_tiles,
+                            cudaStream_t s);
+
+struct BackwardArgs {
+    const uint16_t *Q, *K, *V, *L, *out, *dout;
+    const int32_t *sel_idx;
+    const float *sel_w;
+    int B, H, T, D, N, topk;
+    float scale;
+    float *dQ, *dK, *dV, *dL;
+    // workspace (shares the dispatch layout of the forward)
+    float *delta;          // [B*H*T]  dO . O
+    int32_t *chunk_count, *chunk_off, *chunk_cursor, *pair_row;
+    float *pair_w;
+    int32_t *pair_slot;    // [B*H*T*topk] slot j of each pair (unused by the forward)
+    PairTile *tiles;
+    int32_t *num_tiles;
+    int max_tiles;
+};
+cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s);
+
+}  // namespace hsa

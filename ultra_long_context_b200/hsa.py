@@ -1,0 +1,224 @@
+"""Python binding of the C ABI in ``include/hsa.h`` (libhsa_b200.so).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and contiguity, outputs
+and the workspace are allocated with torch on the input's device, and the C entry point of the same
+name is called on the current torch stream. Every step of HSA runs in the CUDA library; there is
+no fallback. If the library is missing or cannot be loaded, the first call raises.
+"""
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhsa_b200.so")
+
+HSA_OK = 0
+STATUS_NAMES = {0: "HSA_OK", -1: "HSA_ERR_INVALID_ARG", -2: "HSA_ERR_UNSUPPORTED", -3: "HSA_ERR_WORKSPACE",
+                -4: "HSA_ERR_CUDA", -5: "HSA_ERR_TIMEOUT"}
+
+# C entry points and their argument types, as declared in include/hsa.h
+_P, _I, _I64, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "hsa_last_error": ([], ctypes.c_char_p),
+    "hsa_forward_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
+    "hsa_forward": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P], _I),
+    "hsa_decode_workspace_size": ([_I, _I, _I64, _I, _I, _I], _SZ),
+    "hsa_decode": ([_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P], _I),
+    "hsa_backward_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
+    "hsa_backward": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _P],
+                     _I),
+    "hsa_profile_enable": ([_I], _I),
+    "hsa_profile_summary": ([ctypes.c_char_p, _SZ], _I),
+}
+
+_lib = None
+
+
+class HSAError(RuntimeError):
+    def __init__(self, name, status, message):
+        super().__init__(f"{name} failed: {STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def lib():
+    """Load libhsa_b200.so (once) and declare its entry points. Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with ultra_long_context_b200/build.py "
+                               "(or __graft_entry__.build()); there is no fallback path")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = handle
+    return _lib
+
+
+def hsa_last_error():
+    return lib().hsa_last_error().decode()
+
+
+def _check(name, status):
+    if status != HSA_OK:
+        raise HSAError(name, status, hsa_last_error())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device, stream):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype, shape, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _workspace(nbytes, device, workspace):
+    if nbytes == 0:
+        return None
+    if workspace is not None:
+        return workspace
+    # +256 so a 256-byte aligned window always fits
+    return torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+
+
+def _aligned(ws):
+    if ws is None:
+        return None, 0
+    p = ws.data_ptr()
+    off = (-p) % 256
+    return ctypes.c_void_p(p + off), ws.numel() * ws.element_size() - off
+
+
+def hsa_forward_workspace_size(B, H, T, D, chunk=64, topk=16):
+    return int(lib().hsa_forward_workspace_size(B, H, T, D, chunk, topk))
+
+
+def hsa_forward(Q, K, V, L, topk, scale=0.0, chunk=64, out=None, sel_idx=None, sel_w=None, workspace=None,
+                stream=None, return_selection=True):
+    """HSA prefill forward. Q, K, V [B, H, T, D] bf16, L [B, H, T // 64, D] bf16 (CUDA).
+
+    Returns (out [B, H, T, D] bf16, sel_idx [B, H, T, topk] int32, sel_w [B, H, T, topk] fp32); the
+    selection is None when ``return_selection`` is False and none was passed in.
+    """
+    B, H, T, D = Q.shape
+    dev = Q.device
+    for n, t in (("Q", Q), ("K", K), ("V", V)):
+        _need(t, n, torch.bfloat16, (B, H, T, D), dev)
+    _need(L, "L", torch.bfloat16, (B, H, T // chunk, D), dev)
+    if out is None:
+        out = torch.empty_like(Q)
+    _need(out, "out", torch.bfloat16, (B, H, T, D), dev)
+    if return_selection and sel_idx is None:
+        sel_idx = torch.empty((B, H, T, topk), dtype=torch.int32, device=dev)
+    if return_selection and sel_w is None:
+        sel_w = torch.empty((B, H, T, topk), dtype=torch.float32, device=dev)
+    nbytes = hsa_forward_workspace_size(B, H, T, D, chunk, topk)
+    ws = _workspace(nbytes, dev, workspace)
+    wp, wn = _aligned(ws)
+    st = lib().hsa_forward(_ptr(Q), _ptr(K), _ptr(V), _ptr(L), B, H, T, D, chunk, topk, float(scale), _ptr(out),
+                           _ptr(sel_idx), _ptr(sel_w), wp, wn, _stream(dev, stream))
+    _check("hsa_forward", st)
+    return out, sel_idx, sel_w
+
+
+def hsa_decode_workspace_size(B, H, Tmax, D, chunk=64, topk=16):
+    return int(lib().hsa_decode_workspace_size(B, H, Tmax, D, chunk, topk))
+
+
+def hsa_decode(q, Kc, Vc, Lc, cache_len, topk, scale=0.0, chunk=64, out=None, sel_idx=None, sel_w=None,
+               workspace=None, stream=None):
+    """HSA decode. q [B, H, D], Kc / Vc [B, H, Tmax, D], Lc [B, H, Tmax // 64, D] bf16; cache_len [B] int64.
+
+    Returns (out [B, H, D] bf16, sel_idx [B, H, topk] int32, sel_w [B, H, topk] fp32).
+    """
+    B, H, D = q.shape
+    Tmax = Kc.shape[2]
+    dev = q.device
+    _need(q, "q", torch.bfloat16, (B, H, D), dev)
+    _need(Kc, "Kc", torch.bfloat16, (B, H, Tmax, D), dev)
+    _need(Vc, "Vc", torch.bfloat16, (B, H, Tmax, D), dev)
+    _need(Lc, "Lc", torch.bfloat16, (B, H, Tmax // chunk, D), dev)
+    _need(cache_len, "cache_len", torch.int64, (B,), dev)
+    if out is None:
+        out = torch.empty_like(q)
+    if sel_idx is None:
+        sel_idx = torch.empty((B, H, topk), dtype=torch.int32, device=dev)
+    if sel_w is None:
+        sel_w = torch.empty((B, H, topk), dtype=torch.float32, device=dev)
+    nbytes = hsa_decode_workspace_size(B, H, Tmax, D, chunk, topk)
+    ws = _workspace(nbytes, dev, workspace)
+    wp, wn = _aligned(ws)
+    st = lib().hsa_decode(_ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Lc), _ptr(cache_len), Tmax, B, H, D, chunk, topk,
+                          float(scale), _ptr(out), _ptr(sel_idx), _ptr(sel_w), wp, wn, _stream(dev, stream))
+    _check("hsa_decode", st)
+    return out, sel_idx, sel_w
+
+
+def hsa_backward_workspace_size(B, H, T, D, chunk=64, topk=16):
+    return int(lib().hsa_backward_workspace_size(B, H, T, D, chunk, topk))
+
+
+def hsa_backward(Q, K, V, L, out, dout, sel_idx, sel_w, scale=0.0, chunk=64, grads=None, workspace=None,
+                 stream=None):
+    """Backward of hsa_forward for its selection. Returns (dQ, dK, dV, dL), fp32."""
+    B, H, T, D = Q.shape
+    topk = sel_idx.shape[-1]
+    dev = Q.device
+    for n, t in (("Q", Q), ("K", K), ("V", V), ("out", out), ("dout", dout)):
+        _need(t, n, torch.bfloat16, (B, H, T, D), dev)
+    _need(L, "L", torch.bfloat16, (B, H, T // chunk, D), dev)
+    _need(sel_idx, "sel_idx", torch.int32, (B, H, T, topk), dev)
+    _need(sel_w, "sel_w", torch.float32, (B, H, T, topk), dev)
+    if grads is None:
+        grads = (torch.empty((B, H, T, D), dtype=torch.float32, device=dev),
+                 torch.empty((B, H, T, D), dtype=torch.float32, device=dev),
+                 torch.empty((B, H, T, D), dtype=torch.float32, device=dev),
+                 torch.empty((B, H, T // chunk, D), dtype=torch.float32, device=dev))
+    dQ, dK, dV, dL = grads
+    nbytes = hsa_backward_workspace_size(B, H, T, D, chunk, topk)
+    ws = _workspace(nbytes, dev, workspace)
+    wp, wn = _aligned(ws)
+    st = lib().hsa_backward(_ptr(Q), _ptr(K), _ptr(V), _ptr(L), _ptr(out), _ptr(dout), _ptr(sel_idx), _ptr(sel_w),
+                            B, H, T, D, chunk, topk, float(scale), _ptr(dQ), _ptr(dK), _ptr(dV),
+                            _ptr(dL) if dL.numel() else None, wp, wn, _stream(dev, stream))
+    _check("hsa_backward", st)
+    return dQ, dK, dV, dL
+
+
+def hsa_profile_enable(on=True):
+    lib().hsa_profile_enable(1 if on else 0)
+
+
+def hsa_profile_summary():
+    """{launch site: (launches, total device ms)} for the launches recorded since profiling was enabled."""
+    n = lib().hsa_profile_summary(None, 0)
+    if n < 0:
+        raise RuntimeError("hsa_profile_summary failed")
+    buf = ctypes.create_string_buffer(n + 1)
+    lib().hsa_profile_summary(buf, n + 1)
+    res = {}
+    for line in buf.value.decode().splitlines():
+        name, cnt, ms = line.split(",")
+        res[name] = (int(cnt), float(ms))
+    return res
+
+
+def default_scale(D):
+    return 1.0 / math.sqrt(D)

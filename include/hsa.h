@@ -105,6 +105,32 @@ hsa_status hsa_decode(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
                       size_t workspace_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * Decode without any allocation. The pages have no counterpart: this is an interface addition.
+ *
+ * Same operation, arguments and results as hsa_decode, minus the workspace. It is for callers that
+ * cannot allocate device memory when they run a decode step: an engine that has given all of HBM
+ * to its KV-cache pool and allows no allocation while serving, a plain C caller without a caching
+ * allocator for whom cudaMalloc / cudaFree per step would synchronise the device, or a thread that
+ * must not take the driver's allocation locks. The call allocates nothing (no cudaMalloc, no
+ * cudaFree, no allocating library routine). Its scratch lives in one fixed device array of
+ * HSA_DECODE_NOALLOC_SCRATCH_BYTES inside the library; every GPU that loads the library holds that
+ * array until the process exits.
+ *   - The first call on a device looks up the array's device address (with that device current)
+ *     and caches it; make that first call before any stream capture on that device.
+ *   - A call whose scratch would exceed the array (it grows with B*H*topk*(D + scan ranges)) is
+ *     rejected on the host with HSA_ERR_UNSUPPORTED and a message; use hsa_decode then.
+ *   - Every call shares the one array, which keeps the last call's contents; the parts that must
+ *     start at zero are cleared by each call on its stream. Calls that overlap on the GPU (issued on
+ *     streams not ordered with each other, or from several threads at once) race on the array and
+ *     give wrong results: order them, e.g. on a single stream.
+ * ------------------------------------------------------------------------------------------- */
+#define HSA_DECODE_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
+
+hsa_status hsa_decode_noalloc(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc, const hsa_bf16 *Lc,
+                              const int64_t *cache_len, int64_t Tmax, int B, int H, int D, int chunk, int topk,
+                              float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *stream);
+
+/* ---------------------------------------------------------------------------------------------
  * Backward of hsa_forward for the selection the forward made.
  *
  *   Q, K, V, L, out as in hsa_forward (out = the forward's output); dout [B, H, T, D] bf16

@@ -130,6 +130,11 @@ float resolve_scale(float scale, int D) { return scale > 0.0f ? scale : 1.0f / s
 
 }  // namespace
 
+namespace hsa {
+// Lets other translation units of the library report through hsa_last_error().
+void set_last_error(const char *msg) { g_last_error = msg ? msg : ""; }
+}  // namespace hsa
+
 extern "C" {
 
 const char *hsa_last_error(void) { return g_last_error.c_str(); }

@@ -78,4 +78,7 @@ struct BackwardArgs {
 };
 cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s);
 
+// Message returned by hsa_last_error() on the calling thread.
+void set_last_error(const char *msg);
+
 }  // namespace hsa

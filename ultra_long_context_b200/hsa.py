@@ -26,6 +26,7 @@ SIGNATURES = {
     "hsa_forward": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P], _I),
     "hsa_decode_workspace_size": ([_I, _I, _I64, _I, _I, _I], _SZ),
     "hsa_decode": ([_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P], _I),
+    "hsa_decode_noalloc": ([_P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P], _I),
     "hsa_backward_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
     "hsa_backward": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _P],
                      _I),
@@ -168,6 +169,32 @@ def hsa_decode(q, Kc, Vc, Lc, cache_len, topk, scale=0.0, chunk=64, out=None, se
     st = lib().hsa_decode(_ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Lc), _ptr(cache_len), Tmax, B, H, D, chunk, topk,
                           float(scale), _ptr(out), _ptr(sel_idx), _ptr(sel_w), wp, wn, _stream(dev, stream))
     _check("hsa_decode", st)
+    return out, sel_idx, sel_w
+
+
+def hsa_decode_noalloc(q, Kc, Vc, Lc, cache_len, topk, scale=0.0, chunk=64, out=None, sel_idx=None, sel_w=None,
+                       stream=None):
+    """HSA decode with no allocation inside the call: the library's fixed scratch array replaces the
+    workspace (for callers that cannot allocate device memory while they decode). Same arguments and
+    results as hsa_decode. Calls share that array, so calls overlapping on the GPU race; the first
+    call on a device sets up the array's address and should come before any stream capture."""
+    B, H, D = q.shape
+    Tmax = Kc.shape[2]
+    dev = q.device
+    _need(q, "q", torch.bfloat16, (B, H, D), dev)
+    _need(Kc, "Kc", torch.bfloat16, (B, H, Tmax, D), dev)
+    _need(Vc, "Vc", torch.bfloat16, (B, H, Tmax, D), dev)
+    _need(Lc, "Lc", torch.bfloat16, (B, H, Tmax // chunk, D), dev)
+    _need(cache_len, "cache_len", torch.int64, (B,), dev)
+    if out is None:
+        out = torch.empty_like(q)
+    if sel_idx is None:
+        sel_idx = torch.empty((B, H, topk), dtype=torch.int32, device=dev)
+    if sel_w is None:
+        sel_w = torch.empty((B, H, topk), dtype=torch.float32, device=dev)
+    st = lib().hsa_decode_noalloc(_ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Lc), _ptr(cache_len), Tmax, B, H, D, chunk, topk,
+                                  float(scale), _ptr(out), _ptr(sel_idx), _ptr(sel_w), _stream(dev, stream))
+    _check("hsa_decode_noalloc", st)
     return out, sel_idx, sel_w
 
 

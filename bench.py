@@ -8,6 +8,7 @@ and the 64K forward+backward, each against its roofline, and times the CPU oracl
 sample on the host cores as a reported baseline.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--skip-decode] [--skip-backward]
+                  [--skip-prefill] [--skip-cpu] [--decode-cache-len N]
 
 Multi-GPU (torchrun, one process per GPU): HSA's (batch, head) problems are independent, so every
 rank runs its own copy of the workload with no data-path collective (weak scaling); the only
@@ -26,9 +27,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_FORWARD = 6     # score_topk, count, scan, scatter, chunk_attn, finalize
+KERNELS_PER_FORWARD = 7     # score_topk, count, scan, tile list, scatter, chunk_attn, finalize
 KERNELS_PER_DECODE = 2      # decode_scan, decode_attend
-KERNELS_PER_BACKWARD = 5    # delta, count, scan, scatter, chunk_bwd
+KERNELS_PER_BACKWARD = 6    # delta, count, scan, tile list, scatter, chunk_bwd
 
 
 def load_peaks():
@@ -265,9 +266,12 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--skip-prefill", action="store_true", help="time only the decode / backward parts")
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-backward", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--decode-cache-len", type=int, default=None,
+                    help="override the decode cache length (small cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -285,60 +289,71 @@ def main():
     clocks = ClockSampler(local)
     dev = torch.device("cuda", local)
 
-    # ---------------- prefill forward (headline) ----------------
-    w = inputs.WORKLOADS["fwd_t32k_h8_d128_k16"]
-    Q, K, V, L = inputs.forward_inputs(w.B, w.H, w.T, w.D, w.seed + rank, landmarks=w.landmarks, device=dev)
-    out = torch.empty_like(Q)
-    sel_idx = torch.empty((w.B, w.H, w.T, w.topk), dtype=torch.int32, device=dev)
-    sel_w = torch.empty((w.B, w.H, w.T, w.topk), dtype=torch.float32, device=dev)
-    ws = torch.empty(hsa.hsa_forward_workspace_size(w.B, w.H, w.T, w.D, w.chunk, w.topk) + 256, dtype=torch.uint8,
-                     device=dev)
-
-    def fwd():
-        hsa.hsa_forward(Q, K, V, L, w.topk, out=out, sel_idx=sel_idx, sel_w=sel_w, workspace=ws)
-
     clocks.start()
-    ms = timed(fwd, args.steps, args.warmup, world)
-    ms_per_step = ms / args.steps
-    tokens = w.B * w.T
-    value = world * tokens / (ms_per_step / 1e3)
-    prof_fwd = kernel_profile(fwd, args.steps)
-    score_flops, attn_flops, pairs = forward_work(w, sel_idx)
+    # ---------------- prefill forward (headline) ----------------
+    value = ms_per_step = None
+    roof = roof_score = breakdown = e2e = None
+    pairs = 0
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-    dominant = max((k for k in prof_fwd if k != "memset"), key=lambda k: prof_fwd[k][1])
-    algo = {"chunk_attn": attn_flops, "score_topk": score_flops}
-    roof = roofline_entry(dominant, prof_fwd, algo.get(dominant, attn_flops), "TFLOP/s", tensor_peak, "tensor",
-                          f"{peak_kind} bf16_tflops_sustained")
-    roof_score = roofline_entry("score_topk", prof_fwd, score_flops, "TFLOP/s", tensor_peak, "tensor",
-                                f"{peak_kind} bf16_tflops_sustained")
-    breakdown = {k: {"launches": c, "avg_us": round(t / c * 1e3, 2), "share": round(t / sum(x[1] for x in
-                                                                                           prof_fwd.values()), 4)}
-                 for k, (c, t) in prof_fwd.items()}
+    w = inputs.WORKLOADS["fwd_t32k_h8_d128_k16"]
+    if not args.skip_prefill:
+        w = inputs.WORKLOADS["fwd_t32k_h8_d128_k16"]
+        Q, K, V, L = inputs.forward_inputs(w.B, w.H, w.T, w.D, w.seed + rank, landmarks=w.landmarks, device=dev)
+        out = torch.empty_like(Q)
+        sel_idx = torch.empty((w.B, w.H, w.T, w.topk), dtype=torch.int32, device=dev)
+        sel_w = torch.empty((w.B, w.H, w.T, w.topk), dtype=torch.float32, device=dev)
+        ws = torch.empty(hsa.hsa_forward_workspace_size(w.B, w.H, w.T, w.D, w.chunk, w.topk) + 256, dtype=torch.uint8,
+                         device=dev)
 
-    # ---------------- e2e: host buffers through the public API ----------------
-    hQ, hK, hV, hL = (x.cpu().pin_memory() for x in (Q, K, V, L))
-    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    dQ_, dK_, dV_, dL_ = (torch.empty_like(x) for x in (Q, K, V, L))
+        def fwd():
+            hsa.hsa_forward(Q, K, V, L, w.topk, out=out, sel_idx=sel_idx, sel_w=sel_w, workspace=ws)
 
-    def e2e_step():
-        dQ_.copy_(hQ, non_blocking=True)
-        dK_.copy_(hK, non_blocking=True)
-        dV_.copy_(hV, non_blocking=True)
-        dL_.copy_(hL, non_blocking=True)
-        hsa.hsa_forward(dQ_, dK_, dV_, dL_, w.topk, out=out, sel_idx=sel_idx, sel_w=sel_w, workspace=ws)
-        hout.copy_(out, non_blocking=True)
+        ms = timed(fwd, args.steps, args.warmup, world)
+        ms_per_step = ms / args.steps
+        tokens = w.B * w.T
+        value = world * tokens / (ms_per_step / 1e3)
+        prof_fwd = kernel_profile(fwd, args.steps)
+        score_flops, attn_flops, pairs = forward_work(w, sel_idx)
+        tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        dominant = max((k for k in prof_fwd if k != "memset"), key=lambda k: prof_fwd[k][1])
+        algo = {"chunk_attn": attn_flops, "score_topk": score_flops}
+        roof = roofline_entry(dominant, prof_fwd, algo.get(dominant, attn_flops), "TFLOP/s", tensor_peak, "tensor",
+                              f"{peak_kind} bf16_tflops_sustained")
+        roof_score = roofline_entry("score_topk", prof_fwd, score_flops, "TFLOP/s", tensor_peak, "tensor",
+                                    f"{peak_kind} bf16_tflops_sustained")
+        breakdown = {k: {"launches": c, "avg_us": round(t / c * 1e3, 2), "share": round(t / sum(x[1] for x in
+                                                                                               prof_fwd.values()), 4)}
+                     for k, (c, t) in prof_fwd.items()}
 
-    e2e_ms = timed(e2e_step, args.steps, args.warmup, world) / args.steps
-    h2d = sum(x.numel() * x.element_size() for x in (hQ, hK, hV, hL))
-    d2h = hout.numel() * hout.element_size()
-    e2e = {"value": world * tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)}
-    del hQ, hK, hV, hL, hout, dQ_, dK_, dV_, dL_
+        # ---------------- e2e: host buffers through the public API ----------------
+        hQ, hK, hV, hL = (x.cpu().pin_memory() for x in (Q, K, V, L))
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        dQ_, dK_, dV_, dL_ = (torch.empty_like(x) for x in (Q, K, V, L))
+
+        def e2e_step():
+            dQ_.copy_(hQ, non_blocking=True)
+            dK_.copy_(hK, non_blocking=True)
+            dV_.copy_(hV, non_blocking=True)
+            dL_.copy_(hL, non_blocking=True)
+            hsa.hsa_forward(dQ_, dK_, dV_, dL_, w.topk, out=out, sel_idx=sel_idx, sel_w=sel_w, workspace=ws)
+            hout.copy_(out, non_blocking=True)
+
+        e2e_ms = timed(e2e_step, args.steps, args.warmup, world) / args.steps
+        h2d = sum(x.numel() * x.element_size() for x in (hQ, hK, hV, hL))
+        d2h = hout.numel() * hout.element_size()
+        e2e = {"value": world * tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)}
+        del hQ, hK, hV, hL, hout, dQ_, dK_, dV_, dL_
 
     extra = {}
     # ---------------- decode, 16M-token cache ----------------
     if not args.skip_decode:
         wd = inputs.WORKLOADS["decode_16m_b1_h8_d128_k32"]
+        if args.decode_cache_len:
+            import dataclasses
+
+            wd = dataclasses.replace(wd, name=f"decode_{args.decode_cache_len}_b1_h8_d128_k32",
+                                     cache_len=args.decode_cache_len)
         q, Kc, Vc, Lc, lens, _ = inputs.workload_inputs(wd, device=dev)
         dout_ = torch.empty_like(q)
         didx = torch.empty((wd.B, wd.H, wd.topk), dtype=torch.int32, device=dev)
@@ -407,19 +422,20 @@ def main():
 
     # ---------------- CPU oracle baseline (rank 0, one GPU) ----------------
     cpu = None
-    if rank == 0 and world == 1 and not args.skip_cpu:
+    if rank == 0 and world == 1 and not args.skip_cpu and not args.skip_prefill:
         Qh, Kh, Vh, Lh = (x.float().cpu().numpy() for x in (Q, K, V, L))
         v, rows_done, spent = oracle_forward_sample(w, Qh, Kh, Vh, Lh, target_s=10.0)
         cpu = {"value": round(v, 2), "unit": "tokens/s", "cores": host_cores(), "kind": "oracle",
                "sample": f"{rows_done} token-head rows drawn uniformly from the same 32K workload, fp64 oracle "
                          f"with OpenMP, {spent:.1f} s wall"}
 
-    launches = args.steps * KERNELS_PER_FORWARD
+    launches = 0 if args.skip_prefill else args.steps * KERNELS_PER_FORWARD
     if rank == 0:
         line = {
             "metric": "HSA prefill tokens/s (B2 T32768 H8 D128 chunk64 topk16)",
-            "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "value": round(value, 1) if value else None, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4) if ms_per_step else None,
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "D": w.D, "chunk": w.chunk,
                        "topk": w.topk, "landmarks": "chunk mean + N(0, 0.1^2)", "pairs": pairs,

@@ -71,7 +71,7 @@ struct FwdLayout {
     float *o_acc;
     int32_t *sel_idx;
     float *sel_w;
-    int32_t *chunk_count, *chunk_off, *chunk_cursor, *pair_row;
+    int32_t *chunk_count, *chunk_off, *tile_off, *chunk_cursor, *pair_row;
     float *pair_w;
     hsa::PairTile *tiles;
     int32_t *num_tiles;
@@ -91,6 +91,7 @@ FwdLayout fwd_layout(void *ws, int B, int H, int T, int D, int topk, bool backwa
     l.sel_w = backward ? nullptr : c.take<float>(pairs);
     l.chunk_count = c.take<int32_t>(chunks);
     l.chunk_off = c.take<int32_t>(chunks + 1);
+    l.tile_off = c.take<int32_t>(chunks + 1);
     l.chunk_cursor = c.take<int32_t>(chunks);
     l.pair_row = c.take<int32_t>(pairs);
     l.pair_w = c.take<float>(pairs);
@@ -114,7 +115,7 @@ DecLayout dec_layout(void *ws, int B, int H, int64_t Tmax, int D, int topk) {
     DecLayout l{};
     Carver c{static_cast<char *>(ws)};
     const int64_t Nmax = Tmax / 64;
-    const int split = hsa::decode_split_size(Nmax, topk);
+    const int split = hsa::decode_split_size(Nmax, topk, B * H);
     const int64_t nsplit = Nmax > 0 ? (Nmax + split - 1) / split : 1;
     const size_t BH = (size_t)B * H;
     l.cand = c.take<uint64_t>(BH * nsplit * topk);
@@ -171,7 +172,8 @@ hsa_status hsa_forward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, 
     a.sel_idx = sel_idx ? sel_idx : l.sel_idx;
     a.sel_w = sel_w ? sel_w : l.sel_w;
     a.o_acc = l.o_acc;
-    a.chunk_count = l.chunk_count; a.chunk_off = l.chunk_off; a.chunk_cursor = l.chunk_cursor;
+    a.chunk_count = l.chunk_count; a.chunk_off = l.chunk_off; a.tile_off = l.tile_off;
+    a.chunk_cursor = l.chunk_cursor;
     a.pair_row = l.pair_row; a.pair_w = l.pair_w; a.tiles = l.tiles; a.num_tiles = l.num_tiles;
     a.max_tiles = l.max_tiles;
     return cuda_status(hsa::launch_forward(a, static_cast<cudaStream_t>(stream)), "hsa_forward");
@@ -201,7 +203,7 @@ hsa_status hsa_decode(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
         return fail(HSA_ERR_INVALID_ARG, "sel_idx / sel_w must be 16-byte aligned");
     {
         const int64_t Nmax = Tmax / 64;
-        const int split = hsa::decode_split_size(Nmax, topk);
+        const int split = hsa::decode_split_size(Nmax, topk, B * H);
         const int64_t nsplit = Nmax > 0 ? (Nmax + split - 1) / split : 1;
         if (hsa::decode_scan_smem(split, (int)nsplit, topk) > 227 * 1024)
             return fail(HSA_ERR_UNSUPPORTED, "Tmax=%lld too large for topk=%d (scan merge exceeds shared memory)",
@@ -255,7 +257,8 @@ hsa_status hsa_backward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
     a.scale = resolve_scale(scale, D);
     a.dQ = dQ; a.dK = dK; a.dV = dV; a.dL = dL;
     a.delta = l.delta;
-    a.chunk_count = l.chunk_count; a.chunk_off = l.chunk_off; a.chunk_cursor = l.chunk_cursor;
+    a.chunk_count = l.chunk_count; a.chunk_off = l.chunk_off; a.tile_off = l.tile_off;
+    a.chunk_cursor = l.chunk_cursor;
     a.pair_row = l.pair_row; a.pair_w = l.pair_w; a.pair_slot = l.pair_slot;
     a.tiles = l.tiles; a.num_tiles = l.num_tiles; a.max_tiles = l.max_tiles;
     return cuda_status(hsa::launch_backward(a, static_cast<cudaStream_t>(stream)), "hsa_backward");

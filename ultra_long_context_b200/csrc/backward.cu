@@ -305,7 +305,8 @@ cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
         if (a.D == 128) delta_kernel<128><<<dblocks, 256, 0, s>>>(a.out, a.dout, rows, a.delta);
         else delta_kernel<64><<<dblocks, 256, 0, s>>>(a.out, a.dout, rows, a.delta);
     }
-    e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.chunk_cursor,
+    e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.tile_off,
+                        a.chunk_cursor,
                         a.pair_row, a.pair_w, a.pair_slot, a.tiles, a.num_tiles, a.max_tiles, s);
     if (e != cudaSuccess) return e;
     if (a.D == 128) {

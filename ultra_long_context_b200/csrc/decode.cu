@@ -134,15 +134,23 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
         qr[4] = bf16_lo(qv.z) * scale; qr[5] = bf16_hi(qv.z) * scale;
         qr[6] = bf16_lo(qv.w) * scale; qr[7] = bf16_hi(qv.w) * scale;
         const size_t row0 = ((size_t)bh * Tmax + (size_t)c * kChunk);
+        constexpr int ROUNDS = kChunk / (NWARP * LPW);
+        const int sl = tid % LPL, grp = tid / LPL;
+        // issue every K and V load of this thread up front so both overlap the logit math
+        uint4 kv[ROUNDS], vv[KEYS_PER_GROUP];
+#pragma unroll
+        for (int r = 0; r < ROUNDS; ++r)
+            kv[r] = *reinterpret_cast<const uint4 *>(Kc + (row0 + (r * NWARP + warp) * LPW + g) * D + sub * 8);
+#pragma unroll
+        for (int i = 0; i < KEYS_PER_GROUP; ++i)
+            vv[i] = *reinterpret_cast<const uint4 *>(Vc + (row0 + grp * KEYS_PER_GROUP + i) * D + sl * 8);
         // Step 3 logits: a_u = scale * q . K_c[u]
 #pragma unroll
-        for (int r = 0; r < kChunk / (NWARP * LPW); ++r) {
-            const int u = (r * NWARP + warp) * LPW + g;
-            const uint4 kv = *reinterpret_cast<const uint4 *>(Kc + (row0 + u) * D + sub * 8);
-            float p = dot8(kv, qr);
+        for (int r = 0; r < ROUNDS; ++r) {
+            float p = dot8(kv[r], qr);
 #pragma unroll
             for (int o = LPL / 2; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-            if (sub == 0) s_p[u] = p;
+            if (sub == 0) s_p[(r * NWARP + warp) * LPW + g] = p;
         }
         __syncthreads();
         if (warp == 0) {
@@ -157,17 +165,14 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
         }
         __syncthreads();
         // O_c = P . V_c
-        const int sl = tid % LPL, grp = tid / LPL;
         float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
         for (int i = 0; i < KEYS_PER_GROUP; ++i) {
-            const int u = grp * KEYS_PER_GROUP + i;
-            const uint4 vv = *reinterpret_cast<const uint4 *>(Vc + (row0 + u) * D + sl * 8);
-            const float p = s_p[u];
-            acc[0] = fmaf(p, bf16_lo(vv.x), acc[0]); acc[1] = fmaf(p, bf16_hi(vv.x), acc[1]);
-            acc[2] = fmaf(p, bf16_lo(vv.y), acc[2]); acc[3] = fmaf(p, bf16_hi(vv.y), acc[3]);
-            acc[4] = fmaf(p, bf16_lo(vv.z), acc[4]); acc[5] = fmaf(p, bf16_hi(vv.z), acc[5]);
-            acc[6] = fmaf(p, bf16_lo(vv.w), acc[6]); acc[7] = fmaf(p, bf16_hi(vv.w), acc[7]);
+            const float p = s_p[grp * KEYS_PER_GROUP + i];
+            acc[0] = fmaf(p, bf16_lo(vv[i].x), acc[0]); acc[1] = fmaf(p, bf16_hi(vv[i].x), acc[1]);
+            acc[2] = fmaf(p, bf16_lo(vv[i].y), acc[2]); acc[3] = fmaf(p, bf16_hi(vv[i].y), acc[3]);
+            acc[4] = fmaf(p, bf16_lo(vv[i].z), acc[4]); acc[5] = fmaf(p, bf16_hi(vv[i].z), acc[5]);
+            acc[6] = fmaf(p, bf16_lo(vv[i].w), acc[6]); acc[7] = fmaf(p, bf16_hi(vv[i].w), acc[7]);
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) s_red[grp][sl * 8 + e] = acc[e];
@@ -197,10 +202,23 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
     if (tid == 0) counters[bh] = 0u;
 }
 
-int decode_split_size(int64_t Nmax, int K) {
-    int split = 2048;
-    while (split < 16384 && ((Nmax + split - 1) / split) * (int64_t)K > 8192) split *= 2;
-    return split;
+// Landmarks per scan range. The scan is HBM-bound and every range costs the same, so the ranges are
+// sized for a single wave of CTAs: B*H*ranges <= kDecodeWaveCtas (148 SMs x 4 resident CTAs of
+// 256 threads at the kernel's register count). A range keeps at least 256 landmarks and at most
+// 6144 (its keys live in shared memory), and ranges*K <= 8192 (the merge holds all candidates).
+constexpr int64_t kDecodeWaveCtas = 148 * 4;
+
+int decode_split_size(int64_t Nmax, int K, int BH) {
+    if (Nmax <= 0) return 1;
+    int64_t ns = BH > 0 ? kDecodeWaveCtas / BH : 1;
+    ns = ns < 1 ? 1 : ns;
+    const int64_t by_min = (Nmax + 255) / 256;
+    ns = ns < by_min ? ns : by_min;
+    if ((Nmax + ns - 1) / ns > 6144) ns = (Nmax + 6143) / 6144;
+    const int64_t merge_cap = 8192 / K > 0 ? 8192 / K : 1;
+    ns = ns < merge_cap ? ns : merge_cap;
+    ns = ns < 1 ? 1 : ns;
+    return (int)((Nmax + ns - 1) / ns);
 }
 
 size_t decode_scan_smem(int split, int nsplit, int K) {
@@ -209,7 +227,7 @@ size_t decode_scan_smem(int split, int nsplit, int K) {
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
-    const int split = decode_split_size(a.Nmax, a.K);
+    const int split = decode_split_size(a.Nmax, a.K, a.B * a.H);
     const int nsplit = (int)((a.Nmax + split - 1) / split) > 0 ? (int)((a.Nmax + split - 1) / split) : 1;
     const size_t smem = decode_scan_smem(split, nsplit, a.K);
     const int BH = a.B * a.H;

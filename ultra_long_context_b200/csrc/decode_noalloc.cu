@@ -45,7 +45,7 @@ struct NoAllocLayout {
 
 NoAllocLayout layout(int B, int H, int64_t Tmax, int D, int topk) {
     const int64_t Nmax = Tmax / hsa::kChunk;
-    const int split = hsa::decode_split_size(Nmax, topk);
+    const int split = hsa::decode_split_size(Nmax, topk, B * H);
     const int64_t nsplit = Nmax > 0 ? (Nmax + split - 1) / split : 1;
     const size_t BH = (size_t)B * H;
     NoAllocLayout l{};
@@ -100,7 +100,7 @@ hsa_status hsa_decode_noalloc(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_b
         return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned (cache_len 8-byte)");
     const int64_t Nmax = Tmax / hsa::kChunk;
     if (Nmax >= 2147483647LL) return fail(HSA_ERR_UNSUPPORTED, "Tmax / 64 must stay below 2^31");
-    const int split = hsa::decode_split_size(Nmax, topk);
+    const int split = hsa::decode_split_size(Nmax, topk, B * H);
     const int64_t nsplit = Nmax > 0 ? (Nmax + split - 1) / split : 1;
     if (hsa::decode_scan_smem(split, (int)nsplit, topk) > 227 * 1024)
         return fail(HSA_ERR_UNSUPPORTED, "Tmax too large for this topk (scan merge exceeds shared memory)");

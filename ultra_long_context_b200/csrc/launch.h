@@ -20,7 +20,7 @@ struct DecodeArgs {
     unsigned *counters;  // [2, B*H]
     float *partial;    // [B*H, K, D]
 };
-int decode_split_size(int64_t Nmax, int K);
+int decode_split_size(int64_t Nmax, int K, int BH);
 size_t decode_scan_smem(int split, int nsplit, int K);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 
@@ -44,6 +44,7 @@ struct ForwardArgs {
     float *o_acc;          // [B*H*T, D] fp32 accumulator
     int32_t *chunk_count;  // [B*H*N]
     int32_t *chunk_off;    // [B*H*N + 1]
+    int32_t *tile_off;     // [B*H*N + 1]
     int32_t *chunk_cursor; // [B*H*N]
     int32_t *pair_row;     // [B*H*T*topk] flat token row (b*H + h)*T + t
     float *pair_w;         // [B*H*T*topk]
@@ -56,7 +57,8 @@ cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s);
 // Chunk-major dispatch shared by the forward and the backward: per-chunk pair counts, offsets, the
 // tile work list, and the (token row, weight[, slot]) pair arrays.
 cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, int H, int T, int N, int topk,
-                            int32_t *chunk_count, int32_t *chunk_off, int32_t *chunk_cursor, int32_t *pair_row,
+                            int32_t *chunk_count, int32_t *chunk_off, int32_t *tile_off, int32_t *chunk_cursor,
+                            int32_t *pair_row,
                             float *pair_w, int32_t *pair_slot, PairTile *tiles, int32_t *num_tiles, int max_tiles,
                             cudaStream_t s);
 
@@ -69,7 +71,7 @@ struct BackwardArgs {
     float *dQ, *dK, *dV, *dL;
     // workspace (shares the dispatch layout of the forward)
     float *delta;          // [B*H*T]  dO . O
-    int32_t *chunk_count, *chunk_off, *chunk_cursor, *pair_row;
+    int32_t *chunk_count, *chunk_off, *tile_off, *chunk_cursor, *pair_row;
     float *pair_w;
     int32_t *pair_slot;    // [B*H*T*topk] slot j of each pair (unused by the forward)
     PairTile *tiles;

@@ -36,7 +36,9 @@ struct ScoreSmem {
     static constexpr size_t q_bytes = (size_t)kScoreRows * SD * 2;
     static constexpr size_t l_bytes = (size_t)kScoreCols * SD * 2;
     static constexpr size_t s_bytes = (size_t)kScoreRows * SS * 4;
-    static constexpr size_t total = q_bytes + 2 * l_bytes + s_bytes;
+    static constexpr int SJ = 68;  // bytes per row of candidate column ids (17 words: conflict-free)
+    static constexpr size_t j_bytes = (size_t)kScoreRows * SJ;
+    static constexpr size_t total = q_bytes + 2 * l_bytes + s_bytes + j_bytes;
 };
 
 // K is the compile-time length of the running list (8, 16 or 32); the first kout <= K entries
@@ -53,6 +55,7 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(const uint16_
     uint16_t *sQ = reinterpret_cast<uint16_t *>(smem_raw);
     uint16_t *sL = reinterpret_cast<uint16_t *>(smem_raw + SM::q_bytes);
     float *sS = reinterpret_cast<float *>(smem_raw + SM::q_bytes + 2 * SM::l_bytes);
+    uint8_t *sJ = smem_raw + SM::q_bytes + 2 * SM::l_bytes + SM::s_bytes;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int ntile = (T + kScoreRows - 1) / kScoreRows;
@@ -146,20 +149,35 @@ __global__ void __launch_bounds__(kScoreThreads) score_topk_kernel(const uint16_
                     sS[row * SS + col] = acc[mt][nt][r] * scale;
                 }
         __syncthreads();
+        // per-row top-K update in two phases, so that a warp does not serialise on every column in
+        // which any of its 32 rows inserts: (1) compact, in place, the columns that beat the row's
+        // current K-th score (branch-light); (2) insert only those candidates.
         const int cbase = blk * kScoreCols;
         const int ncol = min(kScoreCols, my_n - cbase);
+        float *row = sS + tid * SS;
+        uint8_t *rj = sJ + tid * SM::SJ;
+        const float tau = ls[K - 1];
+        int nc = 0;
         for (int j = 0; j < ncol; ++j) {
-            const float s = sS[tid * SS + j];
+            const float s = row[j];
+            if (s > tau) {  // nc <= j: the slot written was already read
+                row[nc] = s;
+                rj[nc] = (uint8_t)j;
+                ++nc;
+            }
+        }
+        for (int i = 0; i < nc; ++i) {
+            const float s = row[i];
             if (s > ls[K - 1]) {
-                const int c = cbase + j;
+                const int c = cbase + rj[i];
 #pragma unroll
-                for (int i = K - 1; i > 0; --i) {
-                    const bool prev_lt = ls[i - 1] < s;
-                    const bool cur_lt = ls[i] < s;
-                    const float ns = prev_lt ? ls[i - 1] : (cur_lt ? s : ls[i]);
-                    const int ni = prev_lt ? li[i - 1] : (cur_lt ? c : li[i]);
-                    ls[i] = ns;
-                    li[i] = ni;
+                for (int q = K - 1; q > 0; --q) {
+                    const bool prev_lt = ls[q - 1] < s;
+                    const bool cur_lt = ls[q] < s;
+                    const float ns = prev_lt ? ls[q - 1] : (cur_lt ? s : ls[q]);
+                    const int ni = prev_lt ? li[q - 1] : (cur_lt ? c : li[q]);
+                    ls[q] = ns;
+                    li[q] = ni;
                 }
                 if (ls[0] < s) { ls[0] = s; li[0] = c; }
             }
@@ -246,9 +264,9 @@ __device__ inline int block_exclusive_scan(int v, int *s_warp, int &total) {
     return res;
 }
 
-// One CTA: offsets of every chunk's pair list and the tile work list.
+// One CTA: exclusive offsets of every chunk's pair list and of its tiles (<= kPairTile pairs each).
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t *__restrict__ chunk_count, int M,
-                                                    int32_t *__restrict__ chunk_off, PairTile *__restrict__ tiles,
+                                                    int32_t *__restrict__ chunk_off, int32_t *__restrict__ tile_off,
                                                     int32_t *__restrict__ num_tiles, int max_tiles) {
     __shared__ int s_warp[33];
     const int per = (M + blockDim.x - 1) / blockDim.x;
@@ -265,22 +283,34 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t *__restrict__ 
     for (int i = lo; i < hi; ++i) {
         const int c = chunk_count[i];
         chunk_off[i] = off;
-        for (int k = 0; k * kPairTile < c; ++k) {
-            if (toff < max_tiles) {
-                PairTile pt;
-                pt.chunk = i;
-                pt.start = off + k * kPairTile;
-                pt.count = min(kPairTile, c - k * kPairTile);
-                pt.pad = 0;
-                tiles[toff] = pt;
-            }
-            ++toff;
-        }
+        tile_off[i] = toff;
         off += c;
+        toff += (c + kPairTile - 1) / kPairTile;
     }
     if (threadIdx.x == 0) {
         chunk_off[M] = total;
+        tile_off[M] = ttotal;
         num_tiles[0] = min(ttotal, max_tiles);
+    }
+}
+
+// One warp per chunk writes that chunk's tiles into the work list.
+__global__ void __launch_bounds__(256) tile_list_kernel(const int32_t *__restrict__ chunk_count,
+                                                        const int32_t *__restrict__ chunk_off,
+                                                        const int32_t *__restrict__ tile_off, int M,
+                                                        PairTile *__restrict__ tiles, int max_tiles) {
+    const int i = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (i >= M) return;
+    const int n = chunk_count[i], base = tile_off[i], off = chunk_off[i];
+    for (int k = lane; k * kPairTile < n; k += 32) {
+        if (base + k >= max_tiles) break;
+        PairTile pt;
+        pt.chunk = i;
+        pt.start = off + k * kPairTile;
+        pt.count = min(kPairTile, n - k * kPairTile);
+        pt.pad = 0;
+        tiles[base + k] = pt;
     }
 }
 
@@ -497,7 +527,8 @@ static cudaError_t launch_score_d(const ForwardArgs &a, cudaStream_t s) {
 }
 
 cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, int H, int T, int N, int topk,
-                            int32_t *chunk_count, int32_t *chunk_off, int32_t *chunk_cursor, int32_t *pair_row,
+                            int32_t *chunk_count, int32_t *chunk_off, int32_t *tile_off, int32_t *chunk_cursor,
+                            int32_t *pair_row,
                             float *pair_w, int32_t *pair_slot, PairTile *tiles, int32_t *num_tiles, int max_tiles,
                             cudaStream_t s) {
     const int BH = B * H;
@@ -513,7 +544,12 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
     }
     {
         HSA_PROF("dispatch_scan", s);
-        scan_kernel<<<1, 1024, 0, s>>>(chunk_count, BH * N, chunk_off, tiles, num_tiles, max_tiles);
+        scan_kernel<<<1, 1024, 0, s>>>(chunk_count, BH * N, chunk_off, tile_off, num_tiles, max_tiles);
+    }
+    {
+        HSA_PROF("dispatch_tiles", s);
+        tile_list_kernel<<<(BH * N + 7) / 8, 256, 0, s>>>(chunk_count, chunk_off, tile_off, BH * N, tiles,
+                                                          max_tiles);
     }
     const size_t ssmem = N <= kSmemHistMax / 2 ? 2 * (size_t)N * sizeof(int) : 0;
     if (ssmem > 48 * 1024) {
@@ -547,7 +583,7 @@ cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s) {
         finalize_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a.o_acc, a.out, n8);
         return cudaGetLastError();
     }
-    e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.T, a.N, a.topk, a.chunk_count, a.chunk_off,
+    e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.tile_off,
                         a.chunk_cursor, a.pair_row, a.pair_w, nullptr, a.tiles, a.num_tiles, a.max_tiles, s);
     if (e != cudaSuccess) return e;
     const size_t asmem = 3 * (size_t)kChunk * (a.D + 8) * 2;

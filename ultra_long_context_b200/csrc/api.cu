@@ -74,7 +74,7 @@ struct FwdLayout {
     int32_t *chunk_count, *chunk_off, *tile_off, *chunk_cursor, *pair_row;
     float *pair_w;
     hsa::PairTile *tiles;
-    int32_t *num_tiles;
+    int32_t *num_tiles, *err;
     float *delta;
     int32_t *pair_slot;
     size_t bytes;
@@ -97,6 +97,7 @@ FwdLayout fwd_layout(void *ws, int B, int H, int T, int D, int topk, bool backwa
     l.pair_w = c.take<float>(pairs);
     l.tiles = c.take<hsa::PairTile>((size_t)l.max_tiles);
     l.num_tiles = c.take<int32_t>(1);
+    l.err = c.take<int32_t>(1);
     l.delta = backward ? c.take<float>(rows) : nullptr;
     l.pair_slot = backward ? c.take<int32_t>(pairs) : nullptr;
     l.bytes = c.used;
@@ -175,6 +176,7 @@ hsa_status hsa_forward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, 
     a.chunk_count = l.chunk_count; a.chunk_off = l.chunk_off; a.tile_off = l.tile_off;
     a.chunk_cursor = l.chunk_cursor;
     a.pair_row = l.pair_row; a.pair_w = l.pair_w; a.tiles = l.tiles; a.num_tiles = l.num_tiles;
+    a.err = l.err;
     a.max_tiles = l.max_tiles;
     return cuda_status(hsa::launch_forward(a, static_cast<cudaStream_t>(stream)), "hsa_forward");
 }

@@ -307,7 +307,7 @@ cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
     }
     e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.tile_off,
                         a.chunk_cursor,
-                        a.pair_row, a.pair_w, a.pair_slot, a.tiles, a.num_tiles, a.max_tiles, s);
+                        a.pair_row, a.pair_w, a.pair_slot, a.tiles, a.num_tiles, a.max_tiles, kPairTile, s);
     if (e != cudaSuccess) return e;
     if (a.D == 128) {
         const size_t smem = BwdSmem<128>::total;

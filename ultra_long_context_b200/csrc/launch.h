@@ -31,7 +31,7 @@ struct PairTile {
     int32_t count;  // pairs in this tile (1 .. kPairTile)
     int32_t pad;
 };
-constexpr int kPairTile = 64;
+constexpr int kPairTile = 64;  // pairs per tile of the mma.sync kernels (backward)
 
 struct ForwardArgs {
     const uint16_t *Q, *K, *V, *L;
@@ -50,9 +50,12 @@ struct ForwardArgs {
     float *pair_w;         // [B*H*T*topk]
     PairTile *tiles;       // [max_tiles]
     int32_t *num_tiles;    // [1]
+    int32_t *err;          // [1] set when a bounded device wait ran out
     int max_tiles;
 };
 size_t forward_max_tiles(int B, int H, int T, int topk);
+// Step 3 + blend on the tcgen05 tensor cores (attn_tc.cu); tiles of up to 128 pairs.
+cudaError_t launch_attn_tc(const ForwardArgs &a, cudaStream_t s);
 cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s);
 // Chunk-major dispatch shared by the forward and the backward: per-chunk pair counts, offsets, the
 // tile work list, and the (token row, weight[, slot]) pair arrays.
@@ -60,7 +63,7 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
                             int32_t *chunk_count, int32_t *chunk_off, int32_t *tile_off, int32_t *chunk_cursor,
                             int32_t *pair_row,
                             float *pair_w, int32_t *pair_slot, PairTile *tiles, int32_t *num_tiles, int max_tiles,
-                            cudaStream_t s);
+                            int tile_pairs, cudaStream_t s);
 
 struct BackwardArgs {
     const uint16_t *Q, *K, *V, *L, *out, *dout;

@@ -267,7 +267,7 @@ __device__ inline int block_exclusive_scan(int v, int *s_warp, int &total) {
 // One CTA: exclusive offsets of every chunk's pair list and of its tiles (<= kPairTile pairs each).
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t *__restrict__ chunk_count, int M,
                                                     int32_t *__restrict__ chunk_off, int32_t *__restrict__ tile_off,
-                                                    int32_t *__restrict__ num_tiles, int max_tiles) {
+                                                    int32_t *__restrict__ num_tiles, int max_tiles, int tp) {
     __shared__ int s_warp[33];
     const int per = (M + blockDim.x - 1) / blockDim.x;
     const int lo = min(M, (int)threadIdx.x * per), hi = min(M, lo + per);
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t *__restrict__ 
     for (int i = lo; i < hi; ++i) {
         const int c = chunk_count[i];
         sum += c;
-        tsum += (c + kPairTile - 1) / kPairTile;
+        tsum += (c + tp - 1) / tp;
     }
     int total, ttotal;
     int off = block_exclusive_scan(sum, s_warp, total);
@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t *__restrict__ 
         chunk_off[i] = off;
         tile_off[i] = toff;
         off += c;
-        toff += (c + kPairTile - 1) / kPairTile;
+        toff += (c + tp - 1) / tp;
     }
     if (threadIdx.x == 0) {
         chunk_off[M] = total;
@@ -298,17 +298,17 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t *__restrict__ 
 __global__ void __launch_bounds__(256) tile_list_kernel(const int32_t *__restrict__ chunk_count,
                                                         const int32_t *__restrict__ chunk_off,
                                                         const int32_t *__restrict__ tile_off, int M,
-                                                        PairTile *__restrict__ tiles, int max_tiles) {
+                                                        PairTile *__restrict__ tiles, int max_tiles, int tp) {
     const int i = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (i >= M) return;
     const int n = chunk_count[i], base = tile_off[i], off = chunk_off[i];
-    for (int k = lane; k * kPairTile < n; k += 32) {
+    for (int k = lane; k * tp < n; k += 32) {
         if (base + k >= max_tiles) break;
         PairTile pt;
         pt.chunk = i;
-        pt.start = off + k * kPairTile;
-        pt.count = min(kPairTile, n - k * kPairTile);
+        pt.start = off + k * tp;
+        pt.count = min(tp, n - k * tp);
         pt.pad = 0;
         tiles[base + k] = pt;
     }
@@ -530,7 +530,7 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
                             int32_t *chunk_count, int32_t *chunk_off, int32_t *tile_off, int32_t *chunk_cursor,
                             int32_t *pair_row,
                             float *pair_w, int32_t *pair_slot, PairTile *tiles, int32_t *num_tiles, int max_tiles,
-                            cudaStream_t s) {
+                            int tile_pairs, cudaStream_t s) {
     const int BH = B * H;
     dim3 dgrid((T + kDispatchRows - 1) / kDispatchRows, BH);
     const size_t hsmem = N <= kSmemHistMax ? (size_t)N * sizeof(int) : 0;
@@ -544,12 +544,12 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
     }
     {
         HSA_PROF("dispatch_scan", s);
-        scan_kernel<<<1, 1024, 0, s>>>(chunk_count, BH * N, chunk_off, tile_off, num_tiles, max_tiles);
+        scan_kernel<<<1, 1024, 0, s>>>(chunk_count, BH * N, chunk_off, tile_off, num_tiles, max_tiles, tile_pairs);
     }
     {
         HSA_PROF("dispatch_tiles", s);
         tile_list_kernel<<<(BH * N + 7) / 8, 256, 0, s>>>(chunk_count, chunk_off, tile_off, BH * N, tiles,
-                                                          max_tiles);
+                                                          max_tiles, tile_pairs);
     }
     const size_t ssmem = N <= kSmemHistMax / 2 ? 2 * (size_t)N * sizeof(int) : 0;
     if (ssmem > 48 * 1024) {
@@ -573,6 +573,7 @@ cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s) {
         e = cudaMemsetAsync(a.o_acc, 0, rows * a.D * sizeof(float), s);
         if (e == cudaSuccess) e = cudaMemsetAsync(a.chunk_count, 0, (size_t)BH * a.N * sizeof(int32_t), s);
         if (e == cudaSuccess) e = cudaMemsetAsync(a.chunk_cursor, 0, (size_t)BH * a.N * sizeof(int32_t), s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(a.err, 0, sizeof(int32_t), s);
     }
     if (e != cudaSuccess) return e;
     e = a.D == 128 ? launch_score_d<128>(a, s) : launch_score_d<64>(a, s);
@@ -584,20 +585,10 @@ cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s) {
         return cudaGetLastError();
     }
     e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.tile_off,
-                        a.chunk_cursor, a.pair_row, a.pair_w, nullptr, a.tiles, a.num_tiles, a.max_tiles, s);
+                        a.chunk_cursor, a.pair_row, a.pair_w, nullptr, a.tiles, a.num_tiles, a.max_tiles, 128, s);
     if (e != cudaSuccess) return e;
-    const size_t asmem = 3 * (size_t)kChunk * (a.D + 8) * 2;
-    if (a.D == 128) {
-        e = cudaFuncSetAttribute(chunk_attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)asmem);
-        if (e != cudaSuccess) return e;
-        HSA_PROF("chunk_attn", s);
-        chunk_attn_kernel<128><<<a.max_tiles, kAttnThreads, asmem, s>>>(a.Q, a.K, a.V, a.T, a.N, a.scale, a.tiles,
-                                                                         a.num_tiles, a.pair_row, a.pair_w, a.o_acc);
-    } else {
-        HSA_PROF("chunk_attn", s);
-        chunk_attn_kernel<64><<<a.max_tiles, kAttnThreads, asmem, s>>>(a.Q, a.K, a.V, a.T, a.N, a.scale, a.tiles,
-                                                                        a.num_tiles, a.pair_row, a.pair_w, a.o_acc);
-    }
+    e = launch_attn_tc(a, s);
+    if (e != cudaSuccess) return e;
     const size_t n8 = rows * a.D / 8;
     {
         HSA_PROF("finalize", s);

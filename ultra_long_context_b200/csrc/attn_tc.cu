@@ -2,191 +2,319 @@
 //
 // Explainer page of "Every Token Counts", "How It Works (Technically)": every selected chunk is
 // attended separately (Step 3) and the chunk outputs are blended by the retrieval softmax (Step 4).
-// Work is chunk-major: one CTA takes a tile of up to 128 (token, weight) pairs that selected the
-// same chunk c of one (batch, head).
+// Work is chunk-major: a tile is up to 128 (token, weight) pairs that selected the same chunk c of
+// one (batch, head); for a tile
+//   S = Q_tile K_c^T   (128 x 64, fp32 in TMEM)      P = softmax over the 64 keys (bf16, in TMEM)
+//   O = P V_c          (128 x D, fp32 in TMEM)       o_acc[token] += (w / rowsum) * O[row]
 //
-//   smem      Q rows of the tile (gathered), K_c and V_c (64 x D), P (128 x 64) -- all bf16 in the
-//             canonical 128-byte-swizzled layouts the tensor core reads; filled with cp.async.
-//   TMEM      S = Q K_c^T (128 x 64 fp32) and O = P V_c (128 x D fp32), accumulated by tcgen05.mma
-//             issued from one thread, completion signalled through an mbarrier.
-//   softmax   one thread per pair row reads its S row from TMEM (tcgen05.ld), exact softmax over the
-//             chunk's 64 keys in fp32, P rounded to bf16 into shared memory.
-//   epilogue  O row * (w / rowsum) staged as fp32 in shared memory, then added into the token's
-//             fp32 accumulator row with one bulk asynchronous reduction (cp.reduce.async.bulk .add.f32,
-//             D*4 contiguous bytes) per pair.
+// Persistent, warp-specialised kernel, one CTA per SM, tiles assigned round-robin. Tile j of a CTA
+// uses operand stage j % 3 and TMEM buffer / softmax warpgroup j % 2:
+//   warps 8-11  loaders: the tile's Q rows gathered with coalesced 16-byte loads (a warp-wide load
+//               covers whole 256-byte rows) and stored into the 128-byte-swizzled layout tcgen05
+//               reads; K_c and V_c as 64-row TMA tiles. The next tile's token ids are prefetched
+//               while the current stage fills;
+//   warp 12     MMA issuer: allocates TMEM; one thread issues S(j) = Q K^T and O(j) = P V as soon as
+//               each is ready (neither order is forced, so the two softmax warpgroups never wait on
+//               each other); O takes P straight from TMEM (A operand in TMEM); completion via
+//               tcgen05.commit;
+//   warps 0-7   two softmax/epilogue warpgroups; warpgroup b owns the tiles with j % 2 == b, one
+//               thread per pair row: S row from TMEM, exact fp32 softmax, P (bf16) written back over
+//               its S columns; then the O row, scaled by w / rowsum, goes 16 columns at a time
+//               through the warp's smem tile so that each red.global.add.v4.f32 covers 8 rows x 64
+//               contiguous bytes of the tokens' fp32 accumulator rows.
+// Hand-offs (mbarriers, every wait bounded): op_full / op_empty (3 operand stages), s_full, p_full,
+// o_full, t_empty (TMEM buffer b free again).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "launch.h"
 #include "profile.h"
 #include "tc.cuh"
 
 namespace hsa {
 
-constexpr int kTcTile = 128;  // pairs per tile = MMA M
-constexpr int kTcThreads = 128;
+constexpr int kTcTile = 128;   // pairs per tile = MMA M
+constexpr int kTcGroups = 2;   // softmax/epilogue warpgroups (= TMEM buffers)
+constexpr int kTcStages = 3;   // operand stages
+constexpr int kTcLoaderWarps = 4;
+constexpr int kTcLoaderWarp0 = 4 * kTcGroups;
+constexpr int kTcMmaWarp = kTcLoaderWarp0 + kTcLoaderWarps;
+constexpr int kTcThreads = 32 * (kTcMmaWarp + 1);
 
 template <int D>
 struct TcAttnSmem {
-    static constexpr int KH = D / 64;                    // 64-element (128-byte) column blocks of D
-    static constexpr uint32_t Q = 0;                     // KH x [128 rows][128 B]
-    static constexpr uint32_t K = Q + KH * 16384;        // KH x [64 rows][128 B]
-    static constexpr uint32_t V = K + KH * 8192;         // KH x [64 rows][128 B]
-    static constexpr uint32_t P = V + KH * 8192;         // [128 rows][128 B]
-    static constexpr uint32_t OPS = P + 16384;
-    static constexpr uint32_t STAGE = D * 4 + 16;        // fp32 staging row stride (padded)
-    static_assert(kTcTile * STAGE <= OPS, "staging must fit over the operand buffers");
-    static constexpr uint32_t ROW = OPS;                 // int[128]
-    static constexpr uint32_t W = ROW + 512;             // float[128]
-    static constexpr uint32_t MBAR = W + 512;            // u64
-    static constexpr uint32_t TMEM = MBAR + 8;           // u32
-    static constexpr uint32_t BYTES = TMEM + 8;
-    static constexpr size_t DYN = BYTES + 1024;          // + slack for 1 KB alignment
-    static constexpr uint32_t TMEM_COLS = D == 128 ? 256 : 128;  // S: 64 columns, O: D columns
+    static constexpr int KH = D / 64;                          // 128-byte column blocks of D
+    static constexpr uint32_t QB = KH * 16384, KB = KH * 8192; // Q block [128][D], K or V block [64][D]
+    static constexpr uint32_t STAGE = QB + 2 * KB;             // Q, K, V of one tile
+    static constexpr uint32_t OPS = 0;
+    static constexpr uint32_t SLAB = 16;                       // epilogue columns per pass
+    static constexpr uint32_t OUT_ROW = SLAB * 4 + 16;         // fp32 staging row + pad
+    static constexpr uint32_t OUT = OPS + kTcStages * STAGE;   // per compute warp: [32 rows][OUT_ROW]
+    static constexpr uint32_t ROW = OUT + 8 * 32 * OUT_ROW;    // int[stages][128]
+    static constexpr uint32_t W = ROW + kTcStages * 512;       // float[stages][128]
+    static constexpr uint32_t BAR = W + kTcStages * 512;       // mbarriers
+    static constexpr int NBAR = 2 * kTcStages + 4 * kTcGroups;
+    static constexpr uint32_t TMEM = BAR + NBAR * 8;
+    static constexpr uint32_t BYTES = TMEM + 16;
+    static constexpr size_t DYN = BYTES + 1024;                // slack for the 1 KB alignment
+    static constexpr uint32_t S_COL = 0;                       // S / P buffers: columns [0, 128)
+    static constexpr uint32_t O_COL = 128;                     // O buffers: columns [128, 128 + 2D)
+    static constexpr uint32_t TMEM_COLS = D == 128 ? 512 : 256;
+    static_assert(DYN <= 227 * 1024, "shared memory budget");
 };
 
+// mbarrier slots
+enum { kOpFull = 0, kOpEmpty = kTcStages, kSFull = 2 * kTcStages, kPFull = kSFull + kTcGroups,
+       kOFull = kPFull + kTcGroups, kTEmpty = kOFull + kTcGroups };
+
 template <int D>
-__global__ void __launch_bounds__(kTcThreads) chunk_attn_tc_kernel(
-    const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K, const uint16_t *__restrict__ V, int T, int N,
-    float scale, const PairTile *__restrict__ tiles, const int32_t *__restrict__ num_tiles,
-    const int32_t *__restrict__ pair_row, const float *__restrict__ pair_w, float *__restrict__ o_acc,
-    int32_t *__restrict__ err) {
+__global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
+    const uint16_t *__restrict__ Q, int T, int N, float scale, const PairTile *__restrict__ tiles,
+    const int32_t *__restrict__ num_tiles, const int32_t *__restrict__ pair_row, const float *__restrict__ pair_w,
+    float *__restrict__ o_acc, int32_t *__restrict__ err, const __grid_constant__ CUtensorMap tmK,
+    const __grid_constant__ CUtensorMap tmV) {
     using SM = TcAttnSmem<D>;
-    constexpr int CPR = D / 8;  // 16-byte chunks per row
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
-    const uint32_t sb = (raw + 1023u) & ~1023u;  // 1 KB aligned base (swizzle atoms)
+    const uint32_t sb = (raw + 1023u) & ~1023u;  // 1 KB aligned (swizzle atoms)
     unsigned char *s = smem_raw + (sb - raw);
     int *s_row = reinterpret_cast<int *>(s + SM::ROW);
     float *s_w = reinterpret_cast<float *>(s + SM::W);
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(s + SM::TMEM);
-    const uint32_t mbar = sb + SM::MBAR;
+    auto bar = [&](int i) { return sb + SM::BAR + 8u * (uint32_t)i; };
 
-    if ((int)blockIdx.x >= num_tiles[0]) return;
-    const PairTile pt = tiles[blockIdx.x];
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int bh = pt.chunk / N, c = pt.chunk % N;
-    const uint16_t *Kc = K + ((size_t)bh * T + (size_t)c * kChunk) * D;
-    const uint16_t *Vc = V + ((size_t)bh * T + (size_t)c * kChunk) * D;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ntiles = num_tiles[0];
+    const int G = gridDim.x;
+    const int mine = (int)blockIdx.x < ntiles ? (ntiles - 1 - (int)blockIdx.x) / G + 1 : 0;
 
-    if (warp == 0) tc::tmem_alloc(sb + SM::TMEM, SM::TMEM_COLS);
+    if (warp == kTcMmaWarp) tc::tmem_alloc(sb + SM::TMEM, SM::TMEM_COLS);
     if (tid == 0) {
-        tc::mbar_init(mbar, 1);
+        for (int i = 0; i < kTcStages; ++i) {
+            tc::mbar_init(bar(kOpFull + i), 32 * kTcLoaderWarps);  // loader arrivals (+ K/V TMA bytes)
+            tc::mbar_init(bar(kOpEmpty + i), 1);
+        }
+        for (int i = 0; i < kTcGroups; ++i) {
+            tc::mbar_init(bar(kSFull + i), 1);
+            tc::mbar_init(bar(kPFull + i), kTcTile);
+            tc::mbar_init(bar(kOFull + i), 1);
+            tc::mbar_init(bar(kTEmpty + i), kTcTile);
+        }
         tc::fence_mbar_init();
-    }
-    {
-        const bool ok = tid < pt.count;
-        s_row[tid] = ok ? pair_row[pt.start + tid] : -1;
-        s_w[tid] = ok ? pair_w[pt.start + tid] : 0.0f;
-    }
-    __syncthreads();
-
-    // ---- operands into swizzled shared memory (16-byte cp.async; consecutive lanes cover a row) ----
-    for (int i = tid; i < kTcTile * CPR; i += kTcThreads) {
-        const int r = i / CPR, ch = i % CPR;
-        const int row = s_row[r];
-        cp_async16(s + SM::Q + (ch >> 3) * 16384 + tc::sw128(r, ch & 7),
-                   row >= 0 ? (const void *)(Q + (size_t)row * D + ch * 8) : (const void *)Q, row >= 0 ? 16 : 0);
-    }
-    for (int i = tid; i < kChunk * CPR; i += kTcThreads) {
-        const int r = i / CPR, ch = i % CPR;
-        cp_async16(s + SM::K + (ch >> 3) * 8192 + tc::sw128(r, ch & 7), Kc + (size_t)r * D + ch * 8, 16);
-        cp_async16(s + SM::V + (ch >> 3) * 8192 + tc::sw128(r, ch & 7), Vc + (size_t)r * D + ch * 8, 16);
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    tc::fence_proxy_async_smem();
-    __syncthreads();
-    tc::fence_after();
-
-    const uint32_t tmem = *s_tmem;
-    const uint32_t tS = tmem, tO = tmem + 64;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lanes
-    bool failed = false;
-    uint32_t pending_parity = 0;
-
-    // ---- S = Q K_c^T (M = 128 pairs, N = 64 keys, K = D) ----
-    if (tid == 0) {
-        constexpr uint32_t idesc = tc::idesc_bf16(kTcTile, kChunk, 0, 0);
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t koff = (uint32_t)((ks & 3) * 32);  // K step inside a 128-byte row
-            const uint64_t a = tc::desc_kmajor(sb + SM::Q + (ks >> 2) * 16384 + koff);
-            const uint64_t b = tc::desc_kmajor(sb + SM::K + (ks >> 2) * 8192 + koff);
-            tc::mma_bf16_ss(tS, a, b, idesc, ks > 0 ? 1u : 0u);
-        }
-        tc::commit(mbar);
-    }
-    failed = __syncthreads_or(!tc::mbar_wait(mbar, 0));
-    if (!failed) {
-        tc::fence_after();
-        const int row = s_row[tid];
-        // ---- exact softmax over the chunk's 64 keys (fp32), P -> bf16 in shared memory ----
-        float s0[32], s1[32];
-        tc::tmem_ld32(tS + lane_off, s0);
-        tc::tmem_ld32(tS + lane_off + 32, s1);
-        float mx = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(s0[i], s1[i]));
-        const float sl2 = scale * 1.4426950408889634f;
-        float l = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            s0[i] = exp2f((s0[i] - mx) * sl2);
-            s1[i] = exp2f((s1[i] - mx) * sl2);
-            l += s0[i] + s1[i];
-        }
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-            const float *p = cc < 4 ? s0 + cc * 8 : s1 + (cc - 4) * 8;
-            uint4 v;
-            v.x = pack_bf16x2(p[0], p[1]);
-            v.y = pack_bf16x2(p[2], p[3]);
-            v.z = pack_bf16x2(p[4], p[5]);
-            v.w = pack_bf16x2(p[6], p[7]);
-            *reinterpret_cast<uint4 *>(s + SM::P + tc::sw128(tid, cc)) = v;
-        }
-        tc::fence_proxy_async_smem();
-        tc::fence_before();
-        __syncthreads();
-        tc::fence_after();
-        // ---- O = P V_c (M = 128 pairs, N = D, K = 64 keys); V is the MN-major B operand ----
-        if (tid == 0) {
-            constexpr uint32_t idesc = tc::idesc_bf16(kTcTile, D, 0, 1);
-#pragma unroll
-            for (int ks = 0; ks < kChunk / 16; ++ks) {
-                const uint64_t a = tc::desc_kmajor(sb + SM::P + ks * 32);
-                const uint64_t b = tc::desc_mnmajor(sb + SM::V + ks * 2048, 8192);
-                tc::mma_bf16_ss(tO, a, b, idesc, ks > 0 ? 1u : 0u);
-            }
-            tc::commit(mbar);
-        }
-        pending_parity = 1;
-        failed = __syncthreads_or(!tc::mbar_wait(mbar, 1));
-        if (!failed) {
-            tc::fence_after();
-            // ---- epilogue: O row * (w / l) -> fp32 staging row -> bulk reduction into o_acc ----
-            const float f = row >= 0 ? s_w[tid] / l : 0.0f;
-            unsigned char *stage = s + tid * SM::STAGE;  // overlays the (consumed) operand buffers
-#pragma unroll
-            for (int cb = 0; cb < D / 32; ++cb) {
-                float o[32];
-                tc::tmem_ld32(tO + lane_off + cb * 32, o);
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    *reinterpret_cast<float4 *>(stage + (cb * 32 + q * 4) * 4) =
-                        make_float4(o[4 * q] * f, o[4 * q + 1] * f, o[4 * q + 2] * f, o[4 * q + 3] * f);
-            }
-            tc::fence_proxy_async_smem();
-            if (row >= 0) tc::bulk_reduce_add_f32(o_acc + (size_t)row * D, sb + tid * SM::STAGE, D * 4);
-            tc::bulk_commit();
-            tc::bulk_wait_all();
-        }
-    }
-    if (failed) {
-        if (tid == 0) atomicOr(err, 1);
-        tc::mbar_wait(mbar, pending_parity);  // bounded: let an MMA still in flight finish
     }
     tc::fence_before();
     __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, SM::TMEM_COLS);
+    tc::fence_after();
+    const uint32_t tmem = *reinterpret_cast<uint32_t *>(s + SM::TMEM);
+    bool ok = true;
+
+    if (warp >= kTcLoaderWarp0 && warp < kTcMmaWarp) {
+        // ================= loaders =================
+        constexpr int CPR = D / 8;        // 16-byte chunks per row
+        constexpr int RPW = 32 / CPR;     // rows per warp-wide load: 2 (D = 128) or 4 (D = 64)
+        constexpr int ITER = 32 / RPW;    // loads per thread per tile
+        const int lw = warp - kTcLoaderWarp0, lt = tid - 32 * kTcLoaderWarp0;
+        const int rsub = lane / CPR, ch = lane % CPR;
+        const int myr = 32 * lw + lane;  // the tile row whose token id this thread fetches
+        PairTile t = mine > 0 ? tiles[blockIdx.x] : PairTile{0, 0, 0, 0};
+        int myrow = (mine > 0 && myr < t.count) ? pair_row[t.start + myr] : -1;
+        float myw = (mine > 0 && myr < t.count) ? pair_w[t.start + myr] : 0.0f;
+        for (int j = 0; j < mine && ok; ++j) {
+            const int st = j % kTcStages;
+            ok = tc::mbar_wait(bar(kOpEmpty + st), ((uint32_t)(j / kTcStages) & 1u) ^ 1u);
+            if (!ok) break;
+            const uint32_t full = bar(kOpFull + st);
+            const uint32_t sqa = sb + SM::OPS + st * SM::STAGE;
+            if (lt == 0) {
+                const int bh = t.chunk / N, c = t.chunk % N;
+                tc::mbar_expect_tx(full, 2 * SM::KB);  // this thread arrives below, after its Q stores
+                const int y = bh * T + c * kChunk;
+#pragma unroll
+                for (int h = 0; h < SM::KH; ++h) {
+                    tc::tma_load_2d(sqa + SM::QB + h * 8192, &tmK, h * 64, y, full);
+                    tc::tma_load_2d(sqa + SM::QB + SM::KB + h * 8192, &tmV, h * 64, y, full);
+                }
+            }
+            s_row[st * kTcTile + myr] = myrow;
+            s_w[st * kTcTile + myr] = myw;
+            uint4 v[ITER];
+#pragma unroll
+            for (int k = 0; k < ITER; ++k) {
+                const int src = __shfl_sync(0xffffffffu, myrow, RPW * k + rsub);
+                v[k] = src >= 0 ? *reinterpret_cast<const uint4 *>(Q + (size_t)src * D + ch * 8)
+                                : make_uint4(0, 0, 0, 0);
+            }
+            // prefetch the next tile's descriptor and token ids while these loads are in flight
+            if (j + 1 < mine) {
+                t = tiles[blockIdx.x + (size_t)(j + 1) * G];
+                const bool valid = myr < t.count;
+                myrow = valid ? pair_row[t.start + myr] : -1;
+                myw = valid ? pair_w[t.start + myr] : 0.0f;
+            }
+            unsigned char *sq = s + SM::OPS + st * SM::STAGE;
+#pragma unroll
+            for (int k = 0; k < ITER; ++k) {
+                const int r = 32 * lw + RPW * k + rsub;
+                *reinterpret_cast<uint4 *>(sq + (ch >> 3) * 16384 + tc::sw128(r, ch & 7)) = v[k];
+            }
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(full);
+        }
+    } else if (warp == kTcMmaWarp) {
+        // ================= MMA issuer =================
+        if (lane == 0 && mine > 0) {
+            constexpr uint32_t idesc_s = tc::idesc_bf16(kTcTile, kChunk, 0, 0);
+            constexpr uint32_t idesc_o = tc::idesc_bf16(kTcTile, D, 0, 1);
+            auto issue_s = [&](int jj) {  // S(jj) = Q(jj) K_c(jj)^T into TMEM buffer jj % 2
+                const int st = jj % kTcStages, b = jj & 1;
+                const uint32_t sq = sb + SM::OPS + st * SM::STAGE;
+                const uint32_t sk = sq + SM::QB;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint32_t koff = (uint32_t)((ks & 3) * 32);  // K step inside a 128-byte row
+                    tc::mma_bf16_ss(tmem + SM::S_COL + b * kChunk, tc::desc_kmajor(sq + (ks >> 2) * 16384 + koff),
+                                    tc::desc_kmajor(sk + (ks >> 2) * 8192 + koff), idesc_s, ks > 0 ? 1u : 0u);
+                }
+                tc::commit(bar(kSFull + b));
+            };
+            auto issue_o = [&](int jj) {  // O(jj) = P(jj) V_c(jj), P read from TMEM
+                const int st = jj % kTcStages, b = jj & 1;
+                const uint32_t sv = sb + SM::OPS + st * SM::STAGE + SM::QB + SM::KB;
+#pragma unroll
+                for (int ks = 0; ks < kChunk / 16; ++ks)
+                    tc::mma_bf16_ts(tmem + SM::O_COL + b * D, tmem + SM::S_COL + b * kChunk + ks * 8,
+                                    tc::desc_mnmajor(sv + ks * 2048, 8192), idesc_o, ks > 0 ? 1u : 0u);
+                tc::commit(bar(kOFull + b));
+                tc::commit(bar(kOpEmpty + st));  // the operand stage is free once these MMAs finish
+            };
+            // Issue whichever is ready first: O(next_o) once its P is in TMEM, or S(next_s) once its
+            // operands have landed and its TMEM buffer has been released by the epilogue of tile
+            // next_s - 2. Neither order is forced, so one warpgroup's epilogue never waits on the
+            // other's. The probe loop is bounded: a long stretch without progress is an error.
+            int next_s = 0, next_o = 0;
+            uint32_t idle = 0;
+            while (next_o < mine) {
+                bool progress = false;
+                if (next_o < next_s && tc::mbar_test(bar(kPFull + (next_o & 1)), (uint32_t)(next_o >> 1) & 1u)) {
+                    tc::fence_after();
+                    issue_o(next_o++);
+                    progress = true;
+                }
+                if (next_s < mine && next_s < next_o + kTcGroups &&
+                    tc::mbar_test(bar(kOpFull + next_s % kTcStages), (uint32_t)(next_s / kTcStages) & 1u) &&
+                    tc::mbar_test(bar(kTEmpty + (next_s & 1)), ((uint32_t)(next_s >> 1) & 1u) ^ 1u)) {
+                    tc::fence_after();
+                    issue_s(next_s++);
+                    progress = true;
+                }
+                if (progress) {
+                    idle = 0;
+                } else if (++idle > (1u << 26)) {
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        __syncwarp();
+    } else {
+        // ================= softmax + epilogue: warpgroup g owns tiles j with j % 2 == g =================
+        const int g = warp >> 2;
+        const int r = tid & (kTcTile - 1);                    // pair row = TMEM lane
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const float sl2 = scale * 1.4426950408889634f;
+        unsigned char *wstage = s + SM::OUT + warp * 32 * SM::OUT_ROW;  // this warp's 32 staging rows
+        unsigned char *stage = wstage + lane * SM::OUT_ROW;
+        const uint32_t tS = tmem + lane_off + SM::S_COL + g * kChunk;
+        const uint32_t tO = tmem + lane_off + SM::O_COL + g * D;
+        for (int j = g; j < mine && ok; j += kTcGroups) {
+            const int st = j % kTcStages;
+            const uint32_t ph = (uint32_t)(j >> 1) & 1u;
+            ok = tc::mbar_wait(bar(kOpFull + st), (uint32_t)(j / kTcStages) & 1u) && tc::mbar_wait(bar(kSFull + g), ph);
+            if (!ok) break;
+            tc::fence_after();
+            const int row = s_row[st * kTcTile + r];
+            const float w = s_w[st * kTcTile + r];
+            float s0[32], s1[32];
+            tc::tmem_ld32(tS, s0);
+            tc::tmem_ld32(tS + 32, s1);
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(s0[i], s1[i]));
+            float l = 0.0f;
+            uint32_t pk[32];  // P row as bf16 pairs: the A operand of O = P V, written over S
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float a0 = exp2f((s0[2 * i] - mx) * sl2), a1 = exp2f((s0[2 * i + 1] - mx) * sl2);
+                const float b0 = exp2f((s1[2 * i] - mx) * sl2), b1 = exp2f((s1[2 * i + 1] - mx) * sl2);
+                l += (a0 + a1) + (b0 + b1);
+                pk[i] = pack_bf16x2(a0, a1);
+                pk[16 + i] = pack_bf16x2(b0, b1);
+            }
+            tc::tmem_st32(tS, pk);
+            tc::fence_before();
+            tc::mbar_arrive(bar(kPFull + g));
+
+            ok = tc::mbar_wait(bar(kOFull + g), ph);
+            if (!ok) break;
+            tc::fence_after();
+            const float f = row >= 0 ? w / l : 0.0f;
+            // 16 columns at a time: TMEM (thread = row) -> this warp's padded smem tile -> read back so
+            // that each warp-wide reduction covers 8 rows x 64 contiguous bytes
+#pragma unroll 1
+            for (int cb = 0; cb < D / (int)SM::SLAB; ++cb) {
+                float o[16];
+                tc::tmem_ld16(tO + cb * SM::SLAB, o);
+                __syncwarp();  // the previous slab has been read back
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<float4 *>(stage + q * 16) =
+                        make_float4(o[4 * q] * f, o[4 * q + 1] * f, o[4 * q + 2] * f, o[4 * q + 3] * f);
+                __syncwarp();
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int rr = 8 * q + (lane >> 2), c4 = (lane & 3) * 4;
+                    const int dst = __shfl_sync(0xffffffffu, row, rr);
+                    const float4 val = *reinterpret_cast<const float4 *>(wstage + rr * SM::OUT_ROW + c4 * 4);
+                    if (dst >= 0)
+                        red_add_v4(o_acc + (size_t)dst * D + cb * SM::SLAB + c4, val.x, val.y, val.z, val.w);
+                }
+            }
+            tc::fence_before();
+            tc::mbar_arrive(bar(kTEmpty + g));
+        }
+    }
+    if (!ok) atomicOr(err, 1);
+    tc::fence_before();
+    __syncthreads();
+    if (warp == kTcMmaWarp) {
+        tc::fence_after();
+        tc::tmem_dealloc(tmem, SM::TMEM_COLS);
+    }
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2D bf16 tensor [rows, D] (row stride D * 2 bytes), boxes of 64 columns x box_rows rows, 128-byte swizzle.
+static bool make_tmap(CUtensorMap *m, const void *base, uint64_t rows, int D, int box_rows) {
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int D>
@@ -195,10 +323,15 @@ static cudaError_t launch_attn_tc_d(const ForwardArgs &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(chunk_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
+    const uint64_t rows = (uint64_t)a.B * a.H * a.T;
+    CUtensorMap tk, tv;
+    if (!make_tmap(&tk, a.K, rows, D, kChunk) || !make_tmap(&tv, a.V, rows, D, kChunk)) return cudaErrorInvalidValue;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = sms < a.max_tiles ? sms : a.max_tiles;
     HSA_PROF("chunk_attn", s);
-    chunk_attn_tc_kernel<D><<<a.max_tiles, kTcThreads, smem, s>>>(a.Q, a.K, a.V, a.T, a.N, a.scale, a.tiles,
-                                                                   a.num_tiles, a.pair_row, a.pair_w, a.o_acc,
-                                                                   a.err);
+    chunk_attn_tc_kernel<D><<<grid, kTcThreads, smem, s>>>(a.Q, a.T, a.N, a.scale, a.tiles, a.num_tiles, a.pair_row,
+                                                            a.pair_w, a.o_acc, a.err, tk, tv);
     return cudaGetLastError();
 }
 

@@ -355,6 +355,69 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_kernel(const int32_t *_
     }
 }
 
+// Scatter as a block-level counting sort: the block's (token, slot) entries are ranked by chunk in
+// shared memory first, so each chunk's run of entries from this block is written to consecutive
+// pair-list positions (coalesced stores instead of one scattered store per entry). Used when the
+// chunk count per (b, h) fits the shared-memory tables (N <= kSortedScatterMaxN).
+constexpr int kSortedScatterMaxN = 2048;
+
+__global__ void __launch_bounds__(kDispatchRows) scatter_sorted_kernel(
+    const int32_t *__restrict__ sel_idx, const float *__restrict__ sel_w, int T, int N, int K,
+    const int32_t *__restrict__ chunk_off, int32_t *__restrict__ chunk_cursor, int32_t *__restrict__ pair_row,
+    float *__restrict__ pair_w, int32_t *__restrict__ pair_slot) {
+    extern __shared__ int s_mem[];
+    int *s_cnt = s_mem;                  // [N] entries per chunk in this block
+    int *s_scan = s_cnt + N;             // [N] exclusive scan of s_cnt
+    int *s_gbase = s_scan + N;           // [N] global position of this block's run for the chunk
+    int *s_cur = s_gbase + N;            // [N] ranks handed out so far
+    int *s_key = s_cur + N;              // [rows * K] (c << 14) | (t_local << 6) | slot, sorted by chunk
+    float *s_wt = reinterpret_cast<float *>(s_key + kDispatchRows * K);
+    __shared__ int s_warp[33];
+    const int bh = blockIdx.y, tid = threadIdx.x;
+    const int t0 = blockIdx.x * kDispatchRows;
+    const int t = t0 + tid;
+    for (int i = tid; i < N; i += blockDim.x) { s_cnt[i] = 0; s_cur[i] = 0; }
+    __syncthreads();
+    const int32_t *si = sel_idx + ((size_t)bh * T + (t < T ? t : 0)) * K;
+    if (t < T)
+        for (int j = 0; j < K; ++j) {
+            const int c = si[j];
+            if (c >= 0 && c < N) atomicAdd(&s_cnt[c], 1);
+        }
+    __syncthreads();
+    // block exclusive scan of the N counts (contiguous segment per thread)
+    const int per = (N + blockDim.x - 1) / blockDim.x;
+    const int lo = min(N, tid * per), hi = min(N, lo + per);
+    int sum = 0;
+    for (int i = lo; i < hi; ++i) sum += s_cnt[i];
+    int total;
+    int off = block_exclusive_scan(sum, s_warp, total);
+    for (int i = lo; i < hi; ++i) {
+        const int cnt = s_cnt[i];
+        s_scan[i] = off;
+        s_gbase[i] = cnt ? chunk_off[(size_t)bh * N + i] + atomicAdd(&chunk_cursor[(size_t)bh * N + i], cnt) : 0;
+        off += cnt;
+    }
+    __syncthreads();
+    if (t < T)
+        for (int j = 0; j < K; ++j) {
+            const int c = si[j];
+            if (c < 0 || c >= N) continue;
+            const int p = s_scan[c] + atomicAdd(&s_cur[c], 1);
+            s_key[p] = (c << 14) | (tid << 6) | j;
+            s_wt[p] = sel_w[((size_t)bh * T + t) * K + j];
+        }
+    __syncthreads();
+    for (int i = tid; i < total; i += blockDim.x) {
+        const int key = s_key[i];
+        const int c = key >> 14, tl = (key >> 6) & 0xff, j = key & 63;
+        const int pos = s_gbase[c] + (i - s_scan[c]);
+        pair_row[pos] = (int32_t)((size_t)bh * T + t0 + tl);
+        pair_w[pos] = s_wt[i];
+        if (pair_slot) pair_slot[pos] = j;
+    }
+}
+
 // ------------------------------------------------------------------------------------------------
 // Step 3 + Step 4 blend, chunk-major
 // ------------------------------------------------------------------------------------------------
@@ -551,12 +614,20 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
         tile_list_kernel<<<(BH * N + 7) / 8, 256, 0, s>>>(chunk_count, chunk_off, tile_off, BH * N, tiles,
                                                           max_tiles, tile_pairs);
     }
-    const size_t ssmem = N <= kSmemHistMax / 2 ? 2 * (size_t)N * sizeof(int) : 0;
-    if (ssmem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
+    if (N <= kSortedScatterMaxN) {
+        const size_t ssmem = 4 * (size_t)N * sizeof(int) + (size_t)kDispatchRows * topk * (sizeof(int) + sizeof(float));
+        cudaError_t e = cudaFuncSetAttribute(scatter_sorted_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)ssmem);
         if (e != cudaSuccess) return e;
-    }
-    {
+        HSA_PROF("dispatch_scatter", s);
+        scatter_sorted_kernel<<<dgrid, kDispatchRows, ssmem, s>>>(sel_idx, sel_w, T, N, topk, chunk_off, chunk_cursor,
+                                                                  pair_row, pair_w, pair_slot);
+    } else {
+        const size_t ssmem = N <= kSmemHistMax / 2 ? 2 * (size_t)N * sizeof(int) : 0;
+        if (ssmem > 48 * 1024) {
+            cudaError_t e = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
+            if (e != cudaSuccess) return e;
+        }
         HSA_PROF("dispatch_scatter", s);
         scatter_kernel<<<dgrid, kDispatchRows, ssmem, s>>>(sel_idx, sel_w, T, N, topk, chunk_off, chunk_cursor,
                                                            pair_row, pair_w, pair_slot);

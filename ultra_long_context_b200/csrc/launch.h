@@ -54,6 +54,8 @@ struct ForwardArgs {
     int max_tiles;
 };
 size_t forward_max_tiles(int B, int H, int T, int topk);
+// Step 2 scores + top-K + fusion weights on the tcgen05 tensor cores (score_tc.cu).
+cudaError_t launch_score_tc(const ForwardArgs &a, cudaStream_t s);
 // Step 3 + blend on the tcgen05 tensor cores (attn_tc.cu); tiles of up to 128 pairs.
 cudaError_t launch_attn_tc(const ForwardArgs &a, cudaStream_t s);
 cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s);

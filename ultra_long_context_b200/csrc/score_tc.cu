@@ -6,21 +6,27 @@
 // per-token procedure ("The algorithm, simplified") sorts the scores in descending order, stably,
 // so equal scores keep the lower chunk first. Step 4: w = softmax of the kept scores.
 //
-// One CTA per (128-token tile, batch*head), 4 warps, thread = token row = TMEM lane:
-//   * Q tile (128 x D) and landmark blocks (64 x D) arrive by TMA in the 128-byte-swizzled layout;
-//     one thread issues S_blk = Q L_blk^T (M = 128, N = 64, fp32) into one of two TMEM buffers while
-//     the warps read the other (tcgen05.ld), so the tensor core runs ahead of the selection.
-//   * Each 32-score slab read from TMEM is first compacted into a per-thread column of shared memory
-//     (only the scores that can matter), and only those are processed, so a warp's cost follows
-//     the candidates of its rows rather than every score.
-//   * Pass 1 keeps, per row, the K largest score VALUES in a sorted register list. A score that
-//     beats the current K-th value is inserted with new[i] = max(old[i], min(old[i-1], x)), which
-//     touches every slot independently (no dependent chain). The K-th value tau results.
-//   * Pass 2 recomputes the same blocks (bit-identical: same operands, same instruction sequence)
-//     and emits every chunk with s > tau, plus the lowest-index chunks with s == tau until K are
-//     kept -- exactly the stable-sort rule. A chunk's output slot is the number of kept values above
-//     it, ties taking the next free slot in chunk order (a bitmask of used slots).
-//   * Fusion weights w = softmax over the kept values (fp32, max-subtracted).
+// One CTA per (128-token tile, batch*head); thread = token row = TMEM lane. The design aims at many
+// resident warps (the selection is latency-bound per thread): a CTA holds 128 TMEM columns and about
+// 50 KB of shared memory, so four CTAs (16 selecting warps) share an SM.
+//   * The Q tile lives in TMEM: each selecting thread loads its own row and writes it to its lane
+//     (tcgen05.st, two bf16 per column), and the MMA reads it as the A operand.
+//   * Warp 4 (one lane) is the producer: 32-landmark blocks arrive by TMA in the 128-byte-swizzled
+//     layout (three stages), and it issues S_blk = Q L_blk^T (M = 128, N = 32, fp32) into one of the
+//     TMEM score buffers. Full/empty mbarriers link it to warps 0-3, which run decoupled.
+//   * Pass 1 keeps, per row, the K largest score VALUES in a sorted register list. The scores of a
+//     block that beat the current K-th value are first compacted into a per-thread column of shared
+//     memory (branch-free: every score is stored, the write index advances only on a candidate),
+//     then inserted one by one with new[i] = max(old[i], min(old[i-1], x)), which touches every slot
+//     independently (no dependent chain); a warp thus pays only for real candidates. The K-th value
+//     tau results.
+//   * Pass 2 recomputes the same blocks (bit-identical: same operands, same instruction sequence) and
+//     keeps every chunk with s > tau plus the lowest-index chunks with s == tau until K are kept --
+//     exactly the stable-sort rule -- stashing (score, chunk) in chunk order, branch-free as well.
+//   * At the end each row ranks its kept chunks (output slot = number of kept values above it, ties
+//     in chunk order), computes the fusion weights w = softmax over the kept values (fp32,
+//     max-subtracted), and the tile's rows, contiguous in [B, H, T, K], are written by coalesced
+//     stores through shared memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -30,153 +36,211 @@
 
 namespace hsa {
 
-constexpr int kStRows = 128;      // tokens per CTA (MMA M)
-constexpr int kStCols = 64;       // landmarks per block (MMA N)
-constexpr int kStThreads = 128;
+constexpr int kStRows = 128;                   // tokens per CTA (MMA M)
+constexpr int kStCols = 32;                    // landmarks per block (MMA N)
+constexpr int kStConsumers = 128;              // warps 0-3
+constexpr int kStThreads = kStConsumers + 32;  // + producer warp
+constexpr int kStLStages = 3;                  // landmark blocks in shared memory
+constexpr uint32_t kStTmemCols = 128;          // Q (D/2 columns) + score buffers
+constexpr int kStMaxCtasPerSm = 4;             // kStTmemCols x 4 = all 512 TMEM columns
 
-template <int D>
+template <int D, int K>
 struct StSmem {
     static constexpr int KH = D / 64;
-    static constexpr uint32_t QB = KH * 16384;      // [128 rows][D] bf16, swizzled halves
-    static constexpr uint32_t LB = KH * 8192;       // [64 rows][D] per landmark buffer
-    static constexpr uint32_t Qo = 0, L0 = QB, L1 = QB + LB;
-    static constexpr uint32_t CV = L1 + LB;         // candidate values [32][128 threads] fp32
-    static constexpr uint32_t CC = CV + 32 * 128 * 4;  // candidate chunk ids [32][128] (pass 2)
-    static constexpr uint32_t BAR = CC + 32 * 128 * 4;  // bar_q, bar_l[2], bar_s[2]
-    static constexpr uint32_t TMEM = BAR + 5 * 8;
+    static constexpr uint32_t QCOLS = D / 2;                          // TMEM columns of the Q tile
+    static constexpr int NB = (int)(kStTmemCols - QCOLS) / kStCols;   // TMEM score buffers
+    static constexpr uint32_t LH = kStCols * 128;                     // one 64-column half of a block
+    static constexpr uint32_t LB = KH * LH;                           // one landmark stage
+    static constexpr uint32_t STAGE = 128 * K * 8;                    // output staging: idx + w per row
+    // region U holds the landmark stages during the loop and the output staging at the end
+    static constexpr uint32_t U = kStLStages * LB > STAGE ? kStLStages * LB : STAGE;
+    // [33][128] fp32 candidates / kept scores; [K+1][128] int32 kept chunk ids. The spare row takes
+    // the unconditional store that follows the last real entry.
+    static constexpr uint32_t CV = U;
+    static constexpr uint32_t CC = CV + 33 * 128 * 4;
+    static constexpr uint32_t BAR = CC + (K + 1) * 128 * 4;  // q_ready, full_l[3], empty_l[3], full_s[NB], empty_s[NB]
+    static constexpr int NBAR = 1 + 2 * kStLStages + 2 * NB;
+    static constexpr uint32_t TMEM = BAR + NBAR * 8;
     static constexpr uint32_t BYTES = TMEM + 8;
-    static constexpr size_t DYN = BYTES + 1024;
+    // padded so that at most four CTAs share an SM and their TMEM allocations always fit
+    static constexpr size_t MIN_DYN = 228 * 1024 / (kStMaxCtasPerSm + 1) + 1024;
+    static constexpr size_t DYN = BYTES + 1024 > MIN_DYN ? BYTES + 1024 : MIN_DYN;
+    static_assert(NB >= 2, "need two score buffers");
 };
 
 template <int D, int K>
-__global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(int T, int N, float scale, int kout,
+__global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_t *__restrict__ Q, int T, int N,
+                                                                   float scale, int kout,
                                                                    int32_t *__restrict__ sel_idx,
                                                                    float *__restrict__ sel_w, int32_t *__restrict__ err,
-                                                                   const __grid_constant__ CUtensorMap tmQ,
                                                                    const __grid_constant__ CUtensorMap tmL) {
-    using SM = StSmem<D>;
+    using SM = StSmem<D, K>;
+    constexpr int NB = SM::NB;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sb = (raw + 1023u) & ~1023u;
     unsigned char *s = smem_raw + (sb - raw);
-    const uint32_t bar_q = sb + SM::BAR;
-    auto bar_l = [&](int i) { return sb + SM::BAR + 8u * (1 + i); };
-    auto bar_s = [&](int i) { return sb + SM::BAR + 8u * (3 + i); };
+    const uint32_t q_ready = sb + SM::BAR;
+    auto full_l = [&](int i) { return sb + SM::BAR + 8u * (1 + i); };
+    auto empty_l = [&](int i) { return sb + SM::BAR + 8u * (1 + kStLStages + i); };
+    auto full_s = [&](int i) { return sb + SM::BAR + 8u * (1 + 2 * kStLStages + i); };
+    auto empty_s = [&](int i) { return sb + SM::BAR + 8u * (1 + 2 * kStLStages + NB + i); };
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ntile = (T + kStRows - 1) / kStRows;
     const int tile = ntile - 1 - blockIdx.x;  // longest rows first
     const int bh = blockIdx.y;
     const int t0 = tile * kStRows;
-    const int t_last = min(T - 1, t0 + kStRows - 1);
+    const int nrows = min(kStRows, T - t0);
+    const int t_last = t0 + nrows - 1;
     const int n_max = min(N, (t_last + 1) / kChunk);
     const int nblk = (n_max + kStCols - 1) / kStCols;
-    const int my_t = t0 + tid;
-    const int my_n = my_t < T ? min(N, (my_t + 1) / kChunk) : 0;
-    const size_t row = (size_t)bh * T + my_t;
+    const size_t out0 = ((size_t)bh * T + t0) * kout;  // the tile's rows are contiguous
 
     if (nblk == 0) {  // no token of this tile has a complete chunk
-        if (my_t < T)
-            for (int i = 0; i < kout; ++i) {
-                sel_idx[row * kout + i] = -1;
-                sel_w[row * kout + i] = 0.0f;
-            }
+        for (int i = tid; i < nrows * kout; i += kStThreads) {
+            sel_idx[out0 + i] = -1;
+            sel_w[out0 + i] = 0.0f;
+        }
         return;
     }
 
-    if (warp == 0) tc::tmem_alloc(sb + SM::TMEM, 2 * kStCols);
-    if (tid == 0) {
-        for (int i = 0; i < 5; ++i) tc::mbar_init(sb + SM::BAR + 8u * i, 1);
+    if (warp == 0) tc::tmem_alloc(sb + SM::TMEM, kStTmemCols);
+    if (tid == kStConsumers) {
+        tc::mbar_init(q_ready, kStConsumers / 32);
+        for (int i = 0; i < kStLStages; ++i) {
+            tc::mbar_init(full_l(i), 1);
+            tc::mbar_init(empty_l(i), 1);
+        }
+        for (int i = 0; i < NB; ++i) {
+            tc::mbar_init(full_s(i), 1);
+            tc::mbar_init(empty_s(i), kStConsumers / 32);
+        }
         tc::fence_mbar_init();
     }
     tc::fence_before();
     __syncthreads();
     tc::fence_after();
     const uint32_t tmem = *reinterpret_cast<uint32_t *>(s + SM::TMEM);
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const int G = 2 * nblk;  // blocks visited: pass 1, then pass 2
     bool ok = true;
 
-    auto load_l = [&](int g) {  // landmark block (g % nblk) into buffer g % 2
-        const int b = g % nblk;
-        const uint32_t dst = sb + (g & 1 ? SM::L1 : SM::L0);
-        tc::mbar_arrive_expect_tx(bar_l(g & 1), SM::LB);
+    if (warp == kStConsumers / 32) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            auto load_l = [&](int h) {  // landmark block h % nblk into stage h % 3
+                const int st = h % kStLStages;
+                const uint32_t dst = sb + st * SM::LB;
+                tc::mbar_arrive_expect_tx(full_l(st), SM::LB);
 #pragma unroll
-        for (int h = 0; h < SM::KH; ++h) tc::tma_load_2d(dst + h * 8192, &tmL, h * 64, bh * N + b * kStCols, bar_l(g & 1));
-    };
-    auto issue_mma = [&](int g) -> bool {
-        if (!tc::mbar_wait(bar_l(g & 1), (uint32_t)(g >> 1) & 1u)) return false;
-        tc::fence_after();
-        constexpr uint32_t idesc = tc::idesc_bf16(kStRows, kStCols, 0, 0);
-        const uint32_t lb = sb + (g & 1 ? SM::L1 : SM::L0);
+                for (int k = 0; k < SM::KH; ++k)
+                    tc::tma_load_2d(dst + k * SM::LH, &tmL, k * 64, bh * N + (h % nblk) * kStCols, full_l(st));
+            };
+            int nload = 0, nmma = 0;
+            for (; nload < kStLStages && nload < G; ++nload) load_l(nload);
+            ok = tc::mbar_wait(q_ready, 0);
+            constexpr uint32_t idesc = tc::idesc_bf16(kStRows, kStCols, 0, 0);
+            for (int g = 0; ok && g < G; ++g) {
+                const int st = g % kStLStages, buf = g % NB;
+                if (!tc::mbar_wait(full_l(st), (uint32_t)(g / kStLStages) & 1u) ||
+                    (g >= NB && !tc::mbar_wait(empty_s(buf), (uint32_t)(g / NB - 1) & 1u))) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after();
+                const uint32_t lb = sb + st * SM::LB;
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t kin = (uint32_t)((ks & 3) * 32);  // K step inside a 128-byte row
-            tc::mma_bf16_ss(tmem + (g & 1) * kStCols, tc::desc_kmajor(sb + SM::Qo + (ks >> 2) * 16384 + kin),
-                            tc::desc_kmajor(lb + (ks >> 2) * 8192 + kin), idesc, ks > 0 ? 1u : 0u);
+                for (int ks = 0; ks < D / 16; ++ks)  // K step of 16: 8 TMEM columns of Q, 32 B of a swizzled row
+                    tc::mma_bf16_ts(tmem + SM::QCOLS + buf * kStCols, tmem + ks * 8,
+                                    tc::desc_kmajor(lb + (ks >> 2) * SM::LH + (ks & 3) * 32), idesc, ks > 0 ? 1u : 0u);
+                tc::commit(full_s(buf));
+                tc::commit(empty_l(st));
+                nmma = g + 1;
+                if (g + kStLStages < G) {  // refill this stage once MMA(g) has read it
+                    if (!tc::mbar_wait(empty_l(st), (uint32_t)(g / kStLStages) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    load_l(nload++);
+                }
+            }
+            if (!ok) {  // let every copy and MMA this CTA started finish before its memory goes away
+                atomicOr(err, 1);
+                for (int h = nmma; h < nload; ++h) tc::mbar_wait(full_l(h % kStLStages), (uint32_t)(h / kStLStages) & 1u);
+                if (nmma > 0) tc::mbar_wait(full_s((nmma - 1) % NB), (uint32_t)((nmma - 1) / NB) & 1u);
+            }
         }
-        tc::commit(bar_s(g & 1));
-        return true;
-    };
+        __syncwarp();
+    } else {
+        // ---------------- selecting warps: one token row per thread ----------------
+        const int my_t = t0 + tid;
+        const int my_n = my_t < T ? min(N, (my_t + 1) / kChunk) : 0;
+        const int k_keep = min(kout, my_n);
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
-    if (tid == 0) {
-        tc::mbar_arrive_expect_tx(bar_q, SM::QB);
+        {  // this row of Q into TMEM lane tid, columns [0, D/2)
+            const uint4 *src = reinterpret_cast<const uint4 *>(Q + ((size_t)bh * T + (my_t < T ? my_t : t0)) * D);
 #pragma unroll
-        for (int h = 0; h < SM::KH; ++h) tc::tma_load_2d(sb + SM::Qo + h * 16384, &tmQ, h * 64, bh * T + t0, bar_q);
-        load_l(0);
-        if (G > 1) load_l(1);
-        ok = tc::mbar_wait(bar_q, 0) && issue_mma(0);
-    }
-
-    float ls[K];  // pass 1: the K largest score values of this row, descending
+            for (int h = 0; h < D / 64; ++h) {
+                uint32_t r[32];
 #pragma unroll
-    for (int i = 0; i < K; ++i) ls[i] = -INFINITY;
-    float tau = -INFINITY, top = 0.0f, z = 0.0f;
-    int need_eq = 0;
-    uint64_t used = 0;  // pass 2: output slots taken
-    const int k_keep = min(kout, my_n);
-
-    for (int g = 0; g < G; ++g) {
-        if (tid == 0 && ok && g + 1 < G) ok = issue_mma(g + 1);
-        const bool fail = __syncthreads_or(!(ok && tc::mbar_wait(bar_s(g & 1), (uint32_t)(g >> 1) & 1u)));
-        if (fail) {
-            ok = false;
-            break;
+                for (int i = 0; i < 8; ++i) {
+                    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+                    if (my_t < T) u = __ldg(src + h * 8 + i);
+                    r[4 * i] = u.x;
+                    r[4 * i + 1] = u.y;
+                    r[4 * i + 2] = u.z;
+                    r[4 * i + 3] = u.w;
+                }
+                tc::tmem_st32(tmem + lane_off + h * 32, r);
+            }
+            tc::fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(q_ready);
         }
-        tc::fence_after();
-        if (tid == 0 && g + 2 < G) load_l(g + 2);  // MMA(g) is done with that landmark buffer
-        if (g == nblk) {
-            // end of pass 1: tau = the k_keep-th largest value; ties at tau are taken lowest chunk first
-            tau = k_keep > 0 ? -INFINITY : INFINITY;
-            int gt = 0;
-#pragma unroll
-            for (int i = 0; i < K; ++i)
-                if (i < k_keep) tau = ls[i];
-#pragma unroll
-            for (int i = 0; i < K; ++i) gt += (i < k_keep && ls[i] > tau) ? 1 : 0;
-            need_eq = k_keep - gt;
-            top = ls[0];
-#pragma unroll
-            for (int i = 0; i < K; ++i) z += i < k_keep ? expf(ls[i] - top) : 0.0f;
-        }
-        const int b = g % nblk;
-        const int ncol = min(kStCols, my_n - b * kStCols);
-        const uint32_t tS = tmem + lane_off + (g & 1) * kStCols;
+
         float *cv = reinterpret_cast<float *>(s + SM::CV) + tid;  // this thread's column of slots
         int *cc = reinterpret_cast<int *>(s + SM::CC) + tid;
-#pragma unroll 1
-        for (int q = 0; q < kStCols / 32; ++q) {
+        float ls[K];  // pass 1: the K largest score values of this row, descending
+#pragma unroll
+        for (int i = 0; i < K; ++i) ls[i] = -INFINITY;
+        float tau = -INFINITY;
+        int need_eq = 0, kept = 0;
+
+        for (int g = 0; g < G; ++g) {
+            const int buf = g % NB;
+            if (!__all_sync(~0u, tc::mbar_wait(full_s(buf), (uint32_t)(g / NB) & 1u))) {
+                ok = false;
+                break;
+            }
+            tc::fence_after();
             float v[32];
-            tc::tmem_ld32(tS + q * 32, v);
-            // compact this slab's candidates (cheap predicated stores), then handle only those, so a
-            // warp never pays an insertion for lanes that have nothing to insert
-            int n = 0;
+            tc::tmem_ld32(tmem + lane_off + SM::QCOLS + buf * kStCols, v);
+            tc::fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(empty_s(buf));  // the scores are in registers now
+
+            if (g == nblk) {
+                // end of pass 1: tau = the k_keep-th largest value; ties at tau go lowest chunk first
+                tau = k_keep > 0 ? -INFINITY : INFINITY;
+                int gt = 0;
+#pragma unroll
+                for (int i = 0; i < K; ++i)
+                    if (i < k_keep) tau = ls[i];
+#pragma unroll
+                for (int i = 0; i < K; ++i) gt += (i < k_keep && ls[i] > tau) ? 1 : 0;
+                need_eq = k_keep - gt;
+            }
+            const int b = g % nblk;
+            const int ncol = min(kStCols, my_n - b * kStCols);
             if (g < nblk) {
+                int n = 0;
                 const float thr = ls[K - 1];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < 32; ++i) {  // branch-free: store always, advance on a candidate
                     const float x = v[i] * scale;
-                    if (q * 32 + i < ncol && x > thr) cv[128 * n++] = x;
+                    cv[128 * n] = x;
+                    n += (i < ncol && x > thr) ? 1 : 0;
                 }
                 for (int k = 0; k < n; ++k) {
                     const float x = cv[128 * k];
@@ -188,48 +252,60 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(int T, int N,
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < 32; ++i) {  // branch-free, as in pass 1
                     const float x = v[i] * scale;
-                    if (q * 32 + i < ncol && x >= tau) {
-                        cv[128 * n] = x;
-                        cc[128 * n] = b * kStCols + q * 32 + i;
-                        ++n;
-                    }
-                }
-                for (int k = 0; k < n; ++k) {
-                    const float x = cv[128 * k];
-                    bool take = x > tau;
-                    if (!take && need_eq > 0) {  // x == tau: lowest chunks first (they arrive in order)
-                        take = true;
-                        --need_eq;
-                    }
-                    if (take) {
-                        int lo = 0;
-#pragma unroll
-                        for (int j = 0; j < K; ++j) lo += (j < k_keep && ls[j] > x) ? 1 : 0;
-                        const uint64_t freeb = ~used & (~0ull << lo);
-                        const int slot = __ffsll((long long)freeb) - 1;
-                        used |= 1ull << slot;
-                        sel_idx[row * kout + slot] = cc[128 * k];
-                        sel_w[row * kout + slot] = expf(x - top) / z;
-                    }
+                    const bool eq = x == tau && need_eq > 0;
+                    const bool take = i < ncol && (x > tau || eq) && kept < k_keep;
+                    cv[128 * kept] = x;
+                    cc[128 * kept] = b * kStCols + i;
+                    kept += take ? 1 : 0;
+                    need_eq -= (take && eq) ? 1 : 0;
                 }
             }
         }
-        tc::fence_before();
-        __syncthreads();  // TMEM buffer g % 2 is rewritten by MMA(g + 2)
-    }
-    if (ok && my_t < T)
-        for (int i = k_keep; i < kout; ++i) {
-            sel_idx[row * kout + i] = -1;
-            sel_w[row * kout + i] = 0.0f;
+
+        // rank the kept chunks, weights, and stage the tile's rows in shared memory (the landmark
+        // stages are free: every MMA has completed)
+        asm volatile("bar.sync 1, %0;" ::"n"(kStConsumers) : "memory");
+        int32_t *st_idx = reinterpret_cast<int32_t *>(s);
+        float *st_w = reinterpret_cast<float *>(s) + kStRows * kout;
+        if (tid < nrows) {
+            const float top = ls[0];
+            float z = 0.0f;
+#pragma unroll
+            for (int i = 0; i < K; ++i) z += i < k_keep ? expf(ls[i] - top) : 0.0f;
+            const float rz = 1.0f / z;
+            uint64_t used = 0;
+            for (int k = 0; k < kept; ++k) {
+                const float x = cv[128 * k];
+                int lo = 0;
+#pragma unroll
+                for (int j = 0; j < K; ++j) lo += (j < k_keep && ls[j] > x) ? 1 : 0;
+                const uint64_t freeb = ~used & (~0ull << lo);
+                const int slot = __ffsll((long long)freeb) - 1;
+                if (slot < 0 || slot >= kout) continue;  // only if pass 2 disagreed with pass 1
+                used |= 1ull << slot;
+                st_idx[tid * kout + slot] = cc[128 * k];
+                st_w[tid * kout + slot] = expf(x - top) * rz;
+            }
+            for (int i = 0; i < kout; ++i)
+                if (!((used >> i) & 1ull)) {
+                    st_idx[tid * kout + i] = -1;
+                    st_w[tid * kout + i] = 0.0f;
+                }
         }
-    if (!ok && tid == 0) atomicOr(err, 1);
+        asm volatile("bar.sync 1, %0;" ::"n"(kStConsumers) : "memory");
+        for (int i = tid; i < nrows * kout; i += kStConsumers) {
+            sel_idx[out0 + i] = st_idx[i];
+            sel_w[out0 + i] = st_w[i];
+        }
+        if (!ok && lane == 0) atomicOr(err, 1);
+    }
     tc::fence_before();
     __syncthreads();
     if (warp == 0) {
         tc::fence_after();
-        tc::tmem_dealloc(tmem, 2 * kStCols);
+        tc::tmem_dealloc(tmem, kStTmemCols);
     }
 }
 
@@ -259,29 +335,28 @@ static bool st_tmap(CUtensorMap *m, const void *base, uint64_t rows, int D, int 
 }
 
 template <int D, int K>
-static cudaError_t launch_st(const ForwardArgs &a, const CUtensorMap &tq, const CUtensorMap &tl, cudaStream_t s) {
-    const size_t smem = StSmem<D>::DYN;
+static cudaError_t launch_st(const ForwardArgs &a, const CUtensorMap &tl, cudaStream_t s) {
+    const size_t smem = StSmem<D, K>::DYN;
     cudaError_t e = cudaFuncSetAttribute(score_topk_tc_kernel<D, K>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid((a.T + kStRows - 1) / kStRows, a.B * a.H);
     HSA_PROF("score_topk", s);
-    score_topk_tc_kernel<D, K><<<grid, kStThreads, smem, s>>>(a.T, a.N, a.scale, a.topk, a.sel_idx, a.sel_w, a.err,
-                                                              tq, tl);
+    score_topk_tc_kernel<D, K><<<grid, kStThreads, smem, s>>>(a.Q, a.T, a.N, a.scale, a.topk, a.sel_idx, a.sel_w,
+                                                              a.err, tl);
     return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t launch_st_d(const ForwardArgs &a, cudaStream_t s) {
-    CUtensorMap tq, tl;
-    if (!st_tmap(&tq, a.Q, (uint64_t)a.B * a.H * a.T, D, kStRows)) return cudaErrorInvalidValue;
+    CUtensorMap tl;
     // with no complete chunk the landmark tensor may be empty: point the map at Q (never read)
     if (!st_tmap(&tl, a.N > 0 ? (const void *)a.L : (const void *)a.Q,
                  a.N > 0 ? (uint64_t)a.B * a.H * a.N : (uint64_t)a.B * a.H * a.T, D, kStCols))
         return cudaErrorInvalidValue;
-    if (a.topk <= 8) return launch_st<D, 8>(a, tq, tl, s);
-    if (a.topk <= 16) return launch_st<D, 16>(a, tq, tl, s);
-    return launch_st<D, 32>(a, tq, tl, s);
+    if (a.topk <= 8) return launch_st<D, 8>(a, tl, s);
+    if (a.topk <= 16) return launch_st<D, 16>(a, tl, s);
+    return launch_st<D, 32>(a, tl, s);
 }
 
 cudaError_t launch_score_tc(const ForwardArgs &a, cudaStream_t s) {

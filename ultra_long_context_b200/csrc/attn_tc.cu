@@ -8,22 +8,26 @@
 //   O = P V_c          (128 x D, fp32 in TMEM)       o_acc[token] += (w / rowsum) * O[row]
 //
 // Persistent, warp-specialised kernel, one CTA per SM, tiles assigned round-robin. Tile j of a CTA
-// uses operand stage j % 3 and TMEM buffer / softmax warpgroup j % 2:
-//   warps 8-11  loaders: the tile's Q rows gathered with coalesced 16-byte loads (a warp-wide load
+// uses operand stage j % 2 and TMEM buffers / warpgroups b = j % 2:
+//   warps 16-19 loaders: the tile's Q rows gathered with coalesced 16-byte loads (a warp-wide load
 //               covers whole 256-byte rows) and stored into the 128-byte-swizzled layout tcgen05
 //               reads; K_c and V_c as 64-row TMA tiles. The next tile's token ids are prefetched
 //               while the current stage fills;
-//   warp 12     MMA issuer: allocates TMEM; one thread issues S(j) = Q K^T and O(j) = P V as soon as
-//               each is ready (neither order is forced, so the two softmax warpgroups never wait on
-//               each other); O takes P straight from TMEM (A operand in TMEM); completion via
-//               tcgen05.commit;
-//   warps 0-7   two softmax/epilogue warpgroups; warpgroup b owns the tiles with j % 2 == b, one
-//               thread per pair row: S row from TMEM, exact fp32 softmax, P (bf16) written back over
-//               its S columns; then the O row, scaled by w / rowsum, goes 16 columns at a time
-//               through the warp's smem tile so that each red.global.add.v4.f32 covers 8 rows x 64
-//               contiguous bytes of the tokens' fp32 accumulator rows.
-// Hand-offs (mbarriers, every wait bounded): op_full / op_empty (3 operand stages), s_full, p_full,
-// o_full, t_empty (TMEM buffer b free again).
+//   warp 20     MMA issuer: allocates TMEM; one thread issues S(j) = Q K^T and O(j) = P V as soon as
+//               each is ready (neither order is forced); O takes P straight from TMEM (A operand in
+//               TMEM); completion via tcgen05.commit. S buffer b is free again as soon as O(j) has
+//               read P, so the next softmax of a warpgroup overlaps the epilogue of the previous tile;
+//   warps 0-7   two softmax warpgroups (b = 0, 1), one thread per pair row: S row from TMEM, exact
+//               fp32 softmax, P (bf16) written back over its S columns; then the epilogue of the
+//               first half of the O columns;
+//   warps 8-15  two epilogue warpgroups (b = 0, 1): the second half of the O columns.
+// The combine into the tokens' fp32 accumulator rows is bound by the rate of global reductions,
+// which needs many warps issuing them: here 16 warps do, each red.global.add.v4.f32 covering
+// 4 rows x 128 contiguous bytes (the O row, scaled by w / rowsum, goes 32 columns at a time through
+// the warp's padded smem tile).
+// Hand-offs (mbarriers, every wait bounded): op_full / op_empty (2 operand stages), s_full, p_full,
+// o_full, s_empty (P consumed), o_empty (O buffer read by both epilogue halves), e_ready (token rows
+// and scale factors of a tile handed from the softmax to the epilogue warpgroup).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -34,11 +38,12 @@
 namespace hsa {
 
 constexpr int kTcTile = 128;   // pairs per tile = MMA M
-constexpr int kTcGroups = 2;   // softmax/epilogue warpgroups (= TMEM buffers)
-constexpr int kTcStages = 3;   // operand stages
+constexpr int kTcGroups = 2;   // TMEM buffers = softmax warpgroups = epilogue warpgroups
+constexpr int kTcStages = 2;   // operand stages
+constexpr int kTcEpiWarp0 = 4 * kTcGroups;                 // warps 8-15
 constexpr int kTcLoaderWarps = 4;
-constexpr int kTcLoaderWarp0 = 4 * kTcGroups;
-constexpr int kTcMmaWarp = kTcLoaderWarp0 + kTcLoaderWarps;
+constexpr int kTcLoaderWarp0 = kTcEpiWarp0 + 4 * kTcGroups;  // warps 16-19
+constexpr int kTcMmaWarp = kTcLoaderWarp0 + kTcLoaderWarps;  // warp 20
 constexpr int kTcThreads = 32 * (kTcMmaWarp + 1);
 
 template <int D>
@@ -47,13 +52,15 @@ struct TcAttnSmem {
     static constexpr uint32_t QB = KH * 16384, KB = KH * 8192; // Q block [128][D], K or V block [64][D]
     static constexpr uint32_t STAGE = QB + 2 * KB;             // Q, K, V of one tile
     static constexpr uint32_t OPS = 0;
-    static constexpr uint32_t SLAB = 16;                       // epilogue columns per pass
-    static constexpr uint32_t OUT_ROW = SLAB * 4 + 16;         // fp32 staging row + pad
-    static constexpr uint32_t OUT = OPS + kTcStages * STAGE;   // per compute warp: [32 rows][OUT_ROW]
-    static constexpr uint32_t ROW = OUT + 8 * 32 * OUT_ROW;    // int[stages][128]
-    static constexpr uint32_t W = ROW + kTcStages * 512;       // float[stages][128]
-    static constexpr uint32_t BAR = W + kTcStages * 512;       // mbarriers
-    static constexpr int NBAR = 2 * kTcStages + 4 * kTcGroups;
+    static constexpr uint32_t SLAB = 32;                       // epilogue columns per pass
+    static constexpr uint32_t OUT_ROW = SLAB * 4 + 16;         // fp32 staging row + pad (conflict-free)
+    static constexpr uint32_t OUT = OPS + kTcStages * STAGE;   // per epilogue warp: [32 rows][OUT_ROW]
+    static constexpr uint32_t ROW = OUT + 16 * 32 * OUT_ROW;   // int[stages][128]: token rows
+    static constexpr uint32_t W = ROW + kTcStages * 512;       // float[stages][128]: fusion weights
+    static constexpr uint32_t EROW = W + kTcStages * 512;      // int[groups][2][128]: rows for the epilogue
+    static constexpr uint32_t EF = EROW + kTcGroups * 2 * 512; // float[groups][2][128]: w / rowsum
+    static constexpr uint32_t BAR = EF + kTcGroups * 2 * 512;  // mbarriers
+    static constexpr int NBAR = 2 * kTcStages + 7 * kTcGroups;
     static constexpr uint32_t TMEM = BAR + NBAR * 8;
     static constexpr uint32_t BYTES = TMEM + 16;
     static constexpr size_t DYN = BYTES + 1024;                // slack for the 1 KB alignment
@@ -65,7 +72,36 @@ struct TcAttnSmem {
 
 // mbarrier slots
 enum { kOpFull = 0, kOpEmpty = kTcStages, kSFull = 2 * kTcStages, kPFull = kSFull + kTcGroups,
-       kOFull = kPFull + kTcGroups, kTEmpty = kOFull + kTcGroups };
+       kOFull = kPFull + kTcGroups, kSEmpty = kOFull + kTcGroups, kOEmpty = kSEmpty + kTcGroups,
+       kEReady = kOEmpty + kTcGroups /* [group][2 slots] */ };
+
+// Half of the O columns of one tile, [c0, c0 + D/2), scaled by f and added into the tokens' fp32
+// rows: 32 columns at a time, TMEM (thread = row) -> this warp's padded smem tile -> read back so
+// that each warp-wide reduction covers 4 rows x 128 contiguous bytes.
+template <int D>
+__device__ __forceinline__ void epilogue_half(uint32_t tO, int c0, int row, float f, unsigned char *wstage, int lane,
+                                              float *__restrict__ o_acc) {
+    using SM = TcAttnSmem<D>;
+    unsigned char *stage = wstage + lane * SM::OUT_ROW;
+#pragma unroll 1
+    for (int cb = 0; cb < D / 2 / (int)SM::SLAB; ++cb) {
+        float o[32];
+        tc::tmem_ld32(tO + c0 + cb * SM::SLAB, o);
+        __syncwarp();  // the previous slab has been read back
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4 *>(stage + q * 16) =
+                make_float4(o[4 * q] * f, o[4 * q + 1] * f, o[4 * q + 2] * f, o[4 * q + 3] * f);
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int rr = 4 * q + (lane >> 3), c4 = (lane & 7) * 4;
+            const int dst = __shfl_sync(0xffffffffu, row, rr);
+            const float4 val = *reinterpret_cast<const float4 *>(wstage + rr * SM::OUT_ROW + c4 * 4);
+            if (dst >= 0) red_add_v4(o_acc + (size_t)dst * D + c0 + cb * SM::SLAB + c4, val.x, val.y, val.z, val.w);
+        }
+    }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
@@ -80,6 +116,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
     unsigned char *s = smem_raw + (sb - raw);
     int *s_row = reinterpret_cast<int *>(s + SM::ROW);
     float *s_w = reinterpret_cast<float *>(s + SM::W);
+    int *e_row = reinterpret_cast<int *>(s + SM::EROW);
+    float *e_f = reinterpret_cast<float *>(s + SM::EF);
     auto bar = [&](int i) { return sb + SM::BAR + 8u * (uint32_t)i; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -97,7 +135,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
             tc::mbar_init(bar(kSFull + i), 1);
             tc::mbar_init(bar(kPFull + i), kTcTile);
             tc::mbar_init(bar(kOFull + i), 1);
-            tc::mbar_init(bar(kTEmpty + i), kTcTile);
+            tc::mbar_init(bar(kSEmpty + i), 1);
+            tc::mbar_init(bar(kOEmpty + i), 2 * kTcTile);
+            tc::mbar_init(bar(kEReady + 2 * i), kTcTile);
+            tc::mbar_init(bar(kEReady + 2 * i + 1), kTcTile);
         }
         tc::fence_mbar_init();
     }
@@ -136,25 +177,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
             }
             s_row[st * kTcTile + myr] = myrow;
             s_w[st * kTcTile + myr] = myw;
-            uint4 v[ITER];
-#pragma unroll
-            for (int k = 0; k < ITER; ++k) {
-                const int src = __shfl_sync(0xffffffffu, myrow, RPW * k + rsub);
-                v[k] = src >= 0 ? *reinterpret_cast<const uint4 *>(Q + (size_t)src * D + ch * 8)
-                                : make_uint4(0, 0, 0, 0);
-            }
-            // prefetch the next tile's descriptor and token ids while these loads are in flight
-            if (j + 1 < mine) {
-                t = tiles[blockIdx.x + (size_t)(j + 1) * G];
-                const bool valid = myr < t.count;
-                myrow = valid ? pair_row[t.start + myr] : -1;
-                myw = valid ? pair_w[t.start + myr] : 0.0f;
-            }
+            // the next tile's descriptor and token ids are fetched while the first batch is in flight
             unsigned char *sq = s + SM::OPS + st * SM::STAGE;
+            const int myrow_now = myrow;
+            constexpr int BATCH = ITER < 8 ? ITER : 8;  // 16-byte loads in flight per thread
 #pragma unroll
-            for (int k = 0; k < ITER; ++k) {
-                const int r = 32 * lw + RPW * k + rsub;
-                *reinterpret_cast<uint4 *>(sq + (ch >> 3) * 16384 + tc::sw128(r, ch & 7)) = v[k];
+            for (int k0 = 0; k0 < ITER; k0 += BATCH) {
+                uint4 v[BATCH];
+#pragma unroll
+                for (int k = 0; k < BATCH; ++k) {
+                    const int src = __shfl_sync(0xffffffffu, myrow_now, RPW * (k0 + k) + rsub);
+                    v[k] = src >= 0 ? *reinterpret_cast<const uint4 *>(Q + (size_t)src * D + ch * 8)
+                                    : make_uint4(0, 0, 0, 0);
+                }
+                if (k0 == 0 && j + 1 < mine) {
+                    t = tiles[blockIdx.x + (size_t)(j + 1) * G];
+                    const bool valid = myr < t.count;
+                    myrow = valid ? pair_row[t.start + myr] : -1;
+                    myw = valid ? pair_w[t.start + myr] : 0.0f;
+                }
+#pragma unroll
+                for (int k = 0; k < BATCH; ++k) {
+                    const int r = 32 * lw + RPW * (k0 + k) + rsub;
+                    *reinterpret_cast<uint4 *>(sq + (ch >> 3) * 16384 + tc::sw128(r, ch & 7)) = v[k];
+                }
             }
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(full);
@@ -184,24 +230,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
                     tc::mma_bf16_ts(tmem + SM::O_COL + b * D, tmem + SM::S_COL + b * kChunk + ks * 8,
                                     tc::desc_mnmajor(sv + ks * 2048, 8192), idesc_o, ks > 0 ? 1u : 0u);
                 tc::commit(bar(kOFull + b));
+                tc::commit(bar(kSEmpty + b));    // P has been read: S buffer b is free
                 tc::commit(bar(kOpEmpty + st));  // the operand stage is free once these MMAs finish
             };
-            // Issue whichever is ready first: O(next_o) once its P is in TMEM, or S(next_s) once its
-            // operands have landed and its TMEM buffer has been released by the epilogue of tile
-            // next_s - 2. Neither order is forced, so one warpgroup's epilogue never waits on the
-            // other's. The probe loop is bounded: a long stretch without progress is an error.
+            // Issue whichever is ready first: O(next_o) once its P is in TMEM and the epilogue of tile
+            // next_o - 2 has read O buffer b, or S(next_s) once its operands have landed and O(next_s - 2)
+            // has consumed P. The probe loop is bounded: a long stretch without progress is an error.
             int next_s = 0, next_o = 0;
             uint32_t idle = 0;
             while (next_o < mine) {
                 bool progress = false;
-                if (next_o < next_s && tc::mbar_test(bar(kPFull + (next_o & 1)), (uint32_t)(next_o >> 1) & 1u)) {
+                if (next_o < next_s && tc::mbar_test(bar(kPFull + (next_o & 1)), (uint32_t)(next_o >> 1) & 1u) &&
+                    tc::mbar_test(bar(kOEmpty + (next_o & 1)), ((uint32_t)(next_o >> 1) & 1u) ^ 1u)) {
                     tc::fence_after();
                     issue_o(next_o++);
                     progress = true;
                 }
                 if (next_s < mine && next_s < next_o + kTcGroups &&
                     tc::mbar_test(bar(kOpFull + next_s % kTcStages), (uint32_t)(next_s / kTcStages) & 1u) &&
-                    tc::mbar_test(bar(kTEmpty + (next_s & 1)), ((uint32_t)(next_s >> 1) & 1u) ^ 1u)) {
+                    tc::mbar_test(bar(kSEmpty + (next_s & 1)), ((uint32_t)(next_s >> 1) & 1u) ^ 1u)) {
                     tc::fence_after();
                     issue_s(next_s++);
                     progress = true;
@@ -216,70 +263,66 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
         }
         __syncwarp();
     } else {
-        // ================= softmax + epilogue: warpgroup g owns tiles j with j % 2 == g =================
-        const int g = warp >> 2;
-        const int r = tid & (kTcTile - 1);                    // pair row = TMEM lane
+        // ================= softmax (warps 0-7) and epilogue (warps 0-15) =================
+        const bool softmax = warp < kTcEpiWarp0;
+        const int g = (warp >> 2) & 1;                        // TMEM buffer / tile parity
+        const int r = (warp & 3) * 32 + lane;                 // pair row = TMEM lane
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const float sl2 = scale * 1.4426950408889634f;
         unsigned char *wstage = s + SM::OUT + warp * 32 * SM::OUT_ROW;  // this warp's 32 staging rows
-        unsigned char *stage = wstage + lane * SM::OUT_ROW;
         const uint32_t tS = tmem + lane_off + SM::S_COL + g * kChunk;
         const uint32_t tO = tmem + lane_off + SM::O_COL + g * D;
         for (int j = g; j < mine && ok; j += kTcGroups) {
             const int st = j % kTcStages;
             const uint32_t ph = (uint32_t)(j >> 1) & 1u;
-            ok = tc::mbar_wait(bar(kOpFull + st), (uint32_t)(j / kTcStages) & 1u) && tc::mbar_wait(bar(kSFull + g), ph);
-            if (!ok) break;
-            tc::fence_after();
-            const int row = s_row[st * kTcTile + r];
-            const float w = s_w[st * kTcTile + r];
-            float s0[32], s1[32];
-            tc::tmem_ld32(tS, s0);
-            tc::tmem_ld32(tS + 32, s1);
-            float mx = -INFINITY;
+            const int slot = (j >> 1) & 1;  // e_row / e_f double buffer of this group
+            int row;
+            float f;
+            if (softmax) {
+                ok = tc::mbar_wait(bar(kOpFull + st), (uint32_t)(j / kTcStages) & 1u) &&
+                     tc::mbar_wait(bar(kSFull + g), ph);
+                if (!ok) break;
+                tc::fence_after();
+                row = s_row[st * kTcTile + r];
+                const float w = s_w[st * kTcTile + r];
+                float s0[32], s1[32];
+                tc::tmem_ld32(tS, s0);
+                tc::tmem_ld32(tS + 32, s1);
+                float mx = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(s0[i], s1[i]));
-            float l = 0.0f;
-            uint32_t pk[32];  // P row as bf16 pairs: the A operand of O = P V, written over S
+                for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(s0[i], s1[i]));
+                float l = 0.0f;
+                uint32_t pk[32];  // P row as bf16 pairs: the A operand of O = P V, written over S
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float a0 = exp2f((s0[2 * i] - mx) * sl2), a1 = exp2f((s0[2 * i + 1] - mx) * sl2);
-                const float b0 = exp2f((s1[2 * i] - mx) * sl2), b1 = exp2f((s1[2 * i + 1] - mx) * sl2);
-                l += (a0 + a1) + (b0 + b1);
-                pk[i] = pack_bf16x2(a0, a1);
-                pk[16 + i] = pack_bf16x2(b0, b1);
-            }
-            tc::tmem_st32(tS, pk);
-            tc::fence_before();
-            tc::mbar_arrive(bar(kPFull + g));
-
-            ok = tc::mbar_wait(bar(kOFull + g), ph);
-            if (!ok) break;
-            tc::fence_after();
-            const float f = row >= 0 ? w / l : 0.0f;
-            // 16 columns at a time: TMEM (thread = row) -> this warp's padded smem tile -> read back so
-            // that each warp-wide reduction covers 8 rows x 64 contiguous bytes
-#pragma unroll 1
-            for (int cb = 0; cb < D / (int)SM::SLAB; ++cb) {
-                float o[16];
-                tc::tmem_ld16(tO + cb * SM::SLAB, o);
-                __syncwarp();  // the previous slab has been read back
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<float4 *>(stage + q * 16) =
-                        make_float4(o[4 * q] * f, o[4 * q + 1] * f, o[4 * q + 2] * f, o[4 * q + 3] * f);
-                __syncwarp();
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int rr = 8 * q + (lane >> 2), c4 = (lane & 3) * 4;
-                    const int dst = __shfl_sync(0xffffffffu, row, rr);
-                    const float4 val = *reinterpret_cast<const float4 *>(wstage + rr * SM::OUT_ROW + c4 * 4);
-                    if (dst >= 0)
-                        red_add_v4(o_acc + (size_t)dst * D + cb * SM::SLAB + c4, val.x, val.y, val.z, val.w);
+                for (int i = 0; i < 16; ++i) {
+                    const float a0 = exp2f((s0[2 * i] - mx) * sl2), a1 = exp2f((s0[2 * i + 1] - mx) * sl2);
+                    const float b0 = exp2f((s1[2 * i] - mx) * sl2), b1 = exp2f((s1[2 * i + 1] - mx) * sl2);
+                    l += (a0 + a1) + (b0 + b1);
+                    pk[i] = pack_bf16x2(a0, a1);
+                    pk[16 + i] = pack_bf16x2(b0, b1);
                 }
+                tc::tmem_st32(tS, pk);
+                f = row >= 0 ? w / l : 0.0f;
+                tc::fence_before();
+                tc::mbar_arrive(bar(kPFull + g));
+                e_row[(g * 2 + slot) * kTcTile + r] = row;  // for the other half of the epilogue
+                e_f[(g * 2 + slot) * kTcTile + r] = f;
+                tc::mbar_arrive(bar(kEReady + g * 2 + slot));
+                ok = tc::mbar_wait(bar(kOFull + g), ph);
+            } else {
+                // e_ready (one per group and slot, a phase per 4 tiles) orders the softmax threads'
+                // e_row / e_f stores before these loads; it cannot run a phase ahead of this wait, as
+                // tile j + 4 needs this warpgroup's o_empty arrival for tile j first
+                ok = tc::mbar_wait(bar(kEReady + g * 2 + slot), (uint32_t)(j >> 2) & 1u) &&
+                     tc::mbar_wait(bar(kOFull + g), ph);
+                row = e_row[(g * 2 + slot) * kTcTile + r];
+                f = e_f[(g * 2 + slot) * kTcTile + r];
             }
+            if (!ok) break;
+            tc::fence_after();
+            epilogue_half<D>(tO, softmax ? 0 : D / 2, row, f, wstage, lane, o_acc);
             tc::fence_before();
-            tc::mbar_arrive(bar(kTEmpty + g));
+            tc::mbar_arrive(bar(kOEmpty + g));
         }
     }
     if (!ok) atomicOr(err, 1);

@@ -8,11 +8,12 @@
 //   O = P V_c          (128 x D, fp32 in TMEM)       o_acc[token] += (w / rowsum) * O[row]
 //
 // Persistent, warp-specialised kernel, one CTA per SM, tiles assigned round-robin. Tile j of a CTA
-// uses operand stage j % 2 and TMEM buffers / warpgroups b = j % 2:
-//   warps 16-19 loaders: the tile's Q rows gathered with coalesced 16-byte loads (a warp-wide load
-//               covers whole 256-byte rows) and stored into the 128-byte-swizzled layout tcgen05
-//               reads; K_c and V_c as 64-row TMA tiles. The next tile's token ids are prefetched
-//               while the current stage fills;
+// uses Q/K slot j % 2 (free again once S(j) is computed), V slot j % 3 (free once O(j) is computed)
+// and TMEM buffers / warpgroups b = j % 2:
+//   warps 16-19 loaders: the tile's Q rows gathered with cp.async (a warp-wide copy covers whole
+//               256-byte rows) into the 128-byte-swizzled layout tcgen05 reads, two tiles of copies in
+//               flight per thread; K_c and V_c as 64-row TMA tiles. The next tile's token ids are
+//               prefetched while the copies run;
 //   warp 20     MMA issuer: allocates TMEM; one thread issues S(j) = Q K^T and O(j) = P V as soon as
 //               each is ready (neither order is forced); O takes P straight from TMEM (A operand in
 //               TMEM); completion via tcgen05.commit. S buffer b is free again as soon as O(j) has
@@ -25,7 +26,7 @@
 // which needs many warps issuing them: here 16 warps do, each red.global.add.v4.f32 covering
 // 4 rows x 128 contiguous bytes (the O row, scaled by w / rowsum, goes 32 columns at a time through
 // the warp's padded smem tile).
-// Hand-offs (mbarriers, every wait bounded): op_full / op_empty (2 operand stages), s_full, p_full,
+// Hand-offs (mbarriers, every wait bounded): qk_full / qk_empty, v_full / v_empty, s_full, p_full,
 // o_full, s_empty (P consumed), o_empty (O buffer read by both epilogue halves), e_ready (token rows
 // and scale factors of a tile handed from the softmax to the epilogue warpgroup).
 #include <cuda.h>
@@ -39,7 +40,8 @@ namespace hsa {
 
 constexpr int kTcTile = 128;   // pairs per tile = MMA M
 constexpr int kTcGroups = 2;   // TMEM buffers = softmax warpgroups = epilogue warpgroups
-constexpr int kTcStages = 2;   // operand stages
+constexpr int kTcQkSlots = 2;  // Q + K operand slots
+constexpr int kTcVSlots = 3;   // V operand slots (also index the per-tile token rows and weights)
 constexpr int kTcEpiWarp0 = 4 * kTcGroups;                 // warps 8-15
 constexpr int kTcLoaderWarps = 4;
 constexpr int kTcLoaderWarp0 = kTcEpiWarp0 + 4 * kTcGroups;  // warps 16-19
@@ -50,17 +52,22 @@ template <int D>
 struct TcAttnSmem {
     static constexpr int KH = D / 64;                          // 128-byte column blocks of D
     static constexpr uint32_t QB = KH * 16384, KB = KH * 8192; // Q block [128][D], K or V block [64][D]
-    static constexpr uint32_t STAGE = QB + 2 * KB;             // Q, K, V of one tile
-    static constexpr uint32_t OPS = 0;
+    static constexpr uint32_t QK = QB + KB;                    // one Q + K slot
+    static constexpr uint32_t OPS = 0;                         // Q+K slots, then V slots
+    static constexpr uint32_t VS = OPS + kTcQkSlots * QK;
     static constexpr uint32_t SLAB = 32;                       // epilogue columns per pass
+    static constexpr int NSLAB = D / SLAB;
+    // slabs [0, SPLIT) go to the softmax warpgroup, the rest to the epilogue warpgroup: the softmax
+    // warpgroup's chain (softmax, wait for O, its slabs) is the longer one, so it takes fewer
+    static constexpr int SPLIT = NSLAB >= 4 ? NSLAB / 4 : 1;
     static constexpr uint32_t OUT_ROW = SLAB * 4 + 16;         // fp32 staging row + pad (conflict-free)
-    static constexpr uint32_t OUT = OPS + kTcStages * STAGE;   // per epilogue warp: [32 rows][OUT_ROW]
-    static constexpr uint32_t ROW = OUT + 16 * 32 * OUT_ROW;   // int[stages][128]: token rows
-    static constexpr uint32_t W = ROW + kTcStages * 512;       // float[stages][128]: fusion weights
-    static constexpr uint32_t EROW = W + kTcStages * 512;      // int[groups][2][128]: rows for the epilogue
+    static constexpr uint32_t OUT = VS + kTcVSlots * KB;       // per epilogue warp: [32 rows][OUT_ROW]
+    static constexpr uint32_t ROW = OUT + 16 * 32 * OUT_ROW;   // int[V slots][128]: token rows
+    static constexpr uint32_t W = ROW + kTcVSlots * 512;       // float[V slots][128]: fusion weights
+    static constexpr uint32_t EROW = W + kTcVSlots * 512;      // int[groups][2][128]: rows for the epilogue
     static constexpr uint32_t EF = EROW + kTcGroups * 2 * 512; // float[groups][2][128]: w / rowsum
     static constexpr uint32_t BAR = EF + kTcGroups * 2 * 512;  // mbarriers
-    static constexpr int NBAR = 2 * kTcStages + 7 * kTcGroups;
+    static constexpr int NBAR = 2 * kTcQkSlots + 2 * kTcVSlots + 7 * kTcGroups;
     static constexpr uint32_t TMEM = BAR + NBAR * 8;
     static constexpr uint32_t BYTES = TMEM + 16;
     static constexpr size_t DYN = BYTES + 1024;                // slack for the 1 KB alignment
@@ -71,22 +78,23 @@ struct TcAttnSmem {
 };
 
 // mbarrier slots
-enum { kOpFull = 0, kOpEmpty = kTcStages, kSFull = 2 * kTcStages, kPFull = kSFull + kTcGroups,
+enum { kQkFull = 0, kQkEmpty = kTcQkSlots, kVFull = 2 * kTcQkSlots, kVEmpty = kVFull + kTcVSlots,
+       kSFull = kVEmpty + kTcVSlots, kPFull = kSFull + kTcGroups,
        kOFull = kPFull + kTcGroups, kSEmpty = kOFull + kTcGroups, kOEmpty = kSEmpty + kTcGroups,
        kEReady = kOEmpty + kTcGroups /* [group][2 slots] */ };
 
-// Half of the O columns of one tile, [c0, c0 + D/2), scaled by f and added into the tokens' fp32
-// rows: 32 columns at a time, TMEM (thread = row) -> this warp's padded smem tile -> read back so
-// that each warp-wide reduction covers 4 rows x 128 contiguous bytes.
+// Slabs [cb0, cb1) of 32 O columns of one tile, scaled by f and added into the tokens' fp32 rows:
+// TMEM (thread = row) -> this warp's padded smem tile -> read back so that each warp-wide reduction
+// covers 4 rows x 128 contiguous bytes.
 template <int D>
-__device__ __forceinline__ void epilogue_half(uint32_t tO, int c0, int row, float f, unsigned char *wstage, int lane,
-                                              float *__restrict__ o_acc) {
+__device__ __forceinline__ void epilogue_slabs(uint32_t tO, int cb0, int cb1, int row, float f, unsigned char *wstage,
+                                               int lane, float *__restrict__ o_acc) {
     using SM = TcAttnSmem<D>;
     unsigned char *stage = wstage + lane * SM::OUT_ROW;
 #pragma unroll 1
-    for (int cb = 0; cb < D / 2 / (int)SM::SLAB; ++cb) {
+    for (int cb = cb0; cb < cb1; ++cb) {
         float o[32];
-        tc::tmem_ld32(tO + c0 + cb * SM::SLAB, o);
+        tc::tmem_ld32(tO + cb * SM::SLAB, o);
         __syncwarp();  // the previous slab has been read back
 #pragma unroll
         for (int q = 0; q < 8; ++q)
@@ -98,7 +106,7 @@ __device__ __forceinline__ void epilogue_half(uint32_t tO, int c0, int row, floa
             const int rr = 4 * q + (lane >> 3), c4 = (lane & 7) * 4;
             const int dst = __shfl_sync(0xffffffffu, row, rr);
             const float4 val = *reinterpret_cast<const float4 *>(wstage + rr * SM::OUT_ROW + c4 * 4);
-            if (dst >= 0) red_add_v4(o_acc + (size_t)dst * D + c0 + cb * SM::SLAB + c4, val.x, val.y, val.z, val.w);
+            if (dst >= 0) red_add_v4(o_acc + (size_t)dst * D + cb * SM::SLAB + c4, val.x, val.y, val.z, val.w);
         }
     }
 }
@@ -127,9 +135,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
 
     if (warp == kTcMmaWarp) tc::tmem_alloc(sb + SM::TMEM, SM::TMEM_COLS);
     if (tid == 0) {
-        for (int i = 0; i < kTcStages; ++i) {
-            tc::mbar_init(bar(kOpFull + i), 32 * kTcLoaderWarps);  // loader arrivals (+ K/V TMA bytes)
-            tc::mbar_init(bar(kOpEmpty + i), 1);
+        for (int i = 0; i < kTcQkSlots; ++i) {
+            tc::mbar_init(bar(kQkFull + i), 32 * kTcLoaderWarps);  // loader arrivals after their Q copies (+ K bytes)
+            tc::mbar_init(bar(kQkEmpty + i), 1);
+        }
+        for (int i = 0; i < kTcVSlots; ++i) {
+            tc::mbar_init(bar(kVFull + i), 32 * kTcLoaderWarps);   // loader arrivals after the rows / weights (+ V bytes)
+            tc::mbar_init(bar(kVEmpty + i), 1);
         }
         for (int i = 0; i < kTcGroups; ++i) {
             tc::mbar_init(bar(kSFull + i), 1);
@@ -159,51 +171,54 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
         PairTile t = mine > 0 ? tiles[blockIdx.x] : PairTile{0, 0, 0, 0};
         int myrow = (mine > 0 && myr < t.count) ? pair_row[t.start + myr] : -1;
         float myw = (mine > 0 && myr < t.count) ? pair_w[t.start + myr] : 0.0f;
+        int pending = -1;  // tile whose Q copies are in flight and not yet published
         for (int j = 0; j < mine && ok; ++j) {
-            const int st = j % kTcStages;
-            ok = tc::mbar_wait(bar(kOpEmpty + st), ((uint32_t)(j / kTcStages) & 1u) ^ 1u);
+            const int sq = j % kTcQkSlots, sv = j % kTcVSlots;
+            ok = tc::mbar_wait(bar(kQkEmpty + sq), ((uint32_t)(j / kTcQkSlots) & 1u) ^ 1u) &&
+                 tc::mbar_wait(bar(kVEmpty + sv), ((uint32_t)(j / kTcVSlots) & 1u) ^ 1u);
             if (!ok) break;
-            const uint32_t full = bar(kOpFull + st);
-            const uint32_t sqa = sb + SM::OPS + st * SM::STAGE;
+            const uint32_t sqa = sb + SM::OPS + sq * SM::QK;
             if (lt == 0) {
                 const int bh = t.chunk / N, c = t.chunk % N;
-                tc::mbar_expect_tx(full, 2 * SM::KB);  // this thread arrives below, after its Q stores
+                tc::mbar_expect_tx(bar(kQkFull + sq), SM::KB);  // this thread arrives below, after its copies
+                tc::mbar_expect_tx(bar(kVFull + sv), SM::KB);
                 const int y = bh * T + c * kChunk;
 #pragma unroll
                 for (int h = 0; h < SM::KH; ++h) {
-                    tc::tma_load_2d(sqa + SM::QB + h * 8192, &tmK, h * 64, y, full);
-                    tc::tma_load_2d(sqa + SM::QB + SM::KB + h * 8192, &tmV, h * 64, y, full);
+                    tc::tma_load_2d(sqa + SM::QB + h * 8192, &tmK, h * 64, y, bar(kQkFull + sq));
+                    tc::tma_load_2d(sb + SM::VS + sv * SM::KB + h * 8192, &tmV, h * 64, y, bar(kVFull + sv));
                 }
             }
-            s_row[st * kTcTile + myr] = myrow;
-            s_w[st * kTcTile + myr] = myw;
-            // the next tile's descriptor and token ids are fetched while the first batch is in flight
-            unsigned char *sq = s + SM::OPS + st * SM::STAGE;
-            const int myrow_now = myrow;
-            constexpr int BATCH = ITER < 8 ? ITER : 8;  // 16-byte loads in flight per thread
+            s_row[sv * kTcTile + myr] = myrow;
+            s_w[sv * kTcTile + myr] = myw;
+            tc::mbar_arrive(bar(kVFull + sv));
 #pragma unroll
-            for (int k0 = 0; k0 < ITER; k0 += BATCH) {
-                uint4 v[BATCH];
-#pragma unroll
-                for (int k = 0; k < BATCH; ++k) {
-                    const int src = __shfl_sync(0xffffffffu, myrow_now, RPW * (k0 + k) + rsub);
-                    v[k] = src >= 0 ? *reinterpret_cast<const uint4 *>(Q + (size_t)src * D + ch * 8)
-                                    : make_uint4(0, 0, 0, 0);
-                }
-                if (k0 == 0 && j + 1 < mine) {
-                    t = tiles[blockIdx.x + (size_t)(j + 1) * G];
-                    const bool valid = myr < t.count;
-                    myrow = valid ? pair_row[t.start + myr] : -1;
-                    myw = valid ? pair_w[t.start + myr] : 0.0f;
-                }
-#pragma unroll
-                for (int k = 0; k < BATCH; ++k) {
-                    const int r = 32 * lw + RPW * (k0 + k) + rsub;
-                    *reinterpret_cast<uint4 *>(sq + (ch >> 3) * 16384 + tc::sw128(r, ch & 7)) = v[k];
-                }
+            for (int k = 0; k < ITER; ++k) {  // padding rows (token -1) are zero-filled
+                const int r = 32 * lw + RPW * k + rsub;
+                const int src = __shfl_sync(0xffffffffu, myrow, RPW * k + rsub);
+                cp_async16_u32(sqa + (ch >> 3) * 16384 + tc::sw128(r, ch & 7),
+                               src >= 0 ? (const void *)(Q + (size_t)src * D + ch * 8) : (const void *)Q,
+                               src >= 0 ? 16 : 0);
             }
+            cp_async_commit();
+            // the next tile's descriptor and token ids, fetched while the copies run
+            if (j + 1 < mine) {
+                t = tiles[blockIdx.x + (size_t)(j + 1) * G];
+                const bool valid = myr < t.count;
+                myrow = valid ? pair_row[t.start + myr] : -1;
+                myw = valid ? pair_w[t.start + myr] : 0.0f;
+            }
+            if (pending >= 0) {  // publish the previous tile once its copies have landed
+                cp_async_wait<1>();
+                tc::fence_proxy_async_smem();
+                tc::mbar_arrive(bar(kQkFull + pending % kTcQkSlots));
+            }
+            pending = j;
+        }
+        cp_async_wait<0>();
+        if (ok && pending >= 0) {
             tc::fence_proxy_async_smem();
-            tc::mbar_arrive(full);
+            tc::mbar_arrive(bar(kQkFull + pending % kTcQkSlots));
         }
     } else if (warp == kTcMmaWarp) {
         // ================= MMA issuer =================
@@ -211,8 +226,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
             constexpr uint32_t idesc_s = tc::idesc_bf16(kTcTile, kChunk, 0, 0);
             constexpr uint32_t idesc_o = tc::idesc_bf16(kTcTile, D, 0, 1);
             auto issue_s = [&](int jj) {  // S(jj) = Q(jj) K_c(jj)^T into TMEM buffer jj % 2
-                const int st = jj % kTcStages, b = jj & 1;
-                const uint32_t sq = sb + SM::OPS + st * SM::STAGE;
+                const int b = jj & 1;
+                const uint32_t sq = sb + SM::OPS + (jj % kTcQkSlots) * SM::QK;
                 const uint32_t sk = sq + SM::QB;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
@@ -221,17 +236,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
                                     tc::desc_kmajor(sk + (ks >> 2) * 8192 + koff), idesc_s, ks > 0 ? 1u : 0u);
                 }
                 tc::commit(bar(kSFull + b));
+                tc::commit(bar(kQkEmpty + jj % kTcQkSlots));  // Q and K are free once S is computed
             };
             auto issue_o = [&](int jj) {  // O(jj) = P(jj) V_c(jj), P read from TMEM
-                const int st = jj % kTcStages, b = jj & 1;
-                const uint32_t sv = sb + SM::OPS + st * SM::STAGE + SM::QB + SM::KB;
+                const int b = jj & 1;
+                const uint32_t sv = sb + SM::VS + (jj % kTcVSlots) * SM::KB;
 #pragma unroll
                 for (int ks = 0; ks < kChunk / 16; ++ks)
                     tc::mma_bf16_ts(tmem + SM::O_COL + b * D, tmem + SM::S_COL + b * kChunk + ks * 8,
                                     tc::desc_mnmajor(sv + ks * 2048, 8192), idesc_o, ks > 0 ? 1u : 0u);
                 tc::commit(bar(kOFull + b));
-                tc::commit(bar(kSEmpty + b));    // P has been read: S buffer b is free
-                tc::commit(bar(kOpEmpty + st));  // the operand stage is free once these MMAs finish
+                tc::commit(bar(kSEmpty + b));                // P has been read: S buffer b is free
+                tc::commit(bar(kVEmpty + jj % kTcVSlots));   // and V slot jj % 3
             };
             // Issue whichever is ready first: O(next_o) once its P is in TMEM and the epilogue of tile
             // next_o - 2 has read O buffer b, or S(next_s) once its operands have landed and O(next_s - 2)
@@ -241,13 +257,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
             while (next_o < mine) {
                 bool progress = false;
                 if (next_o < next_s && tc::mbar_test(bar(kPFull + (next_o & 1)), (uint32_t)(next_o >> 1) & 1u) &&
-                    tc::mbar_test(bar(kOEmpty + (next_o & 1)), ((uint32_t)(next_o >> 1) & 1u) ^ 1u)) {
+                    tc::mbar_test(bar(kOEmpty + (next_o & 1)), ((uint32_t)(next_o >> 1) & 1u) ^ 1u) &&
+                    tc::mbar_test(bar(kVFull + next_o % kTcVSlots), (uint32_t)(next_o / kTcVSlots) & 1u)) {
                     tc::fence_after();
                     issue_o(next_o++);
                     progress = true;
                 }
                 if (next_s < mine && next_s < next_o + kTcGroups &&
-                    tc::mbar_test(bar(kOpFull + next_s % kTcStages), (uint32_t)(next_s / kTcStages) & 1u) &&
+                    tc::mbar_test(bar(kQkFull + next_s % kTcQkSlots), (uint32_t)(next_s / kTcQkSlots) & 1u) &&
                     tc::mbar_test(bar(kSEmpty + (next_s & 1)), ((uint32_t)(next_s >> 1) & 1u) ^ 1u)) {
                     tc::fence_after();
                     issue_s(next_s++);
@@ -273,34 +290,44 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
         const uint32_t tS = tmem + lane_off + SM::S_COL + g * kChunk;
         const uint32_t tO = tmem + lane_off + SM::O_COL + g * D;
         for (int j = g; j < mine && ok; j += kTcGroups) {
-            const int st = j % kTcStages;
+            const int sv = j % kTcVSlots;
             const uint32_t ph = (uint32_t)(j >> 1) & 1u;
             const int slot = (j >> 1) & 1;  // e_row / e_f double buffer of this group
             int row;
             float f;
             if (softmax) {
-                ok = tc::mbar_wait(bar(kOpFull + st), (uint32_t)(j / kTcStages) & 1u) &&
+                // v_full also publishes the loaders' token rows and weights of this tile; it cannot run a
+                // phase ahead of this wait (tile j + 3 needs V slot j % 3, freed only by O(j))
+                ok = tc::mbar_wait(bar(kVFull + sv), (uint32_t)(j / kTcVSlots) & 1u) &&
                      tc::mbar_wait(bar(kSFull + g), ph);
                 if (!ok) break;
                 tc::fence_after();
-                row = s_row[st * kTcTile + r];
-                const float w = s_w[st * kTcTile + r];
+                row = s_row[sv * kTcTile + r];
+                const float w = s_w[sv * kTcTile + r];
                 float s0[32], s1[32];
                 tc::tmem_ld32(tS, s0);
                 tc::tmem_ld32(tS + 32, s1);
-                float mx = -INFINITY;
+                float m8[8];  // row max as a tree (no 64-deep dependent chain)
 #pragma unroll
-                for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fmaxf(s0[i], s1[i]));
-                float l = 0.0f;
+                for (int k = 0; k < 8; ++k) {
+                    m8[k] = fmaxf(fmaxf(s0[k], s0[k + 8]), fmaxf(s0[k + 16], s0[k + 24]));
+                    m8[k] = fmaxf(m8[k], fmaxf(fmaxf(s1[k], s1[k + 8]), fmaxf(s1[k + 16], s1[k + 24])));
+                }
+                const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                const float mxs = mx * sl2;
+                float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                 uint32_t pk[32];  // P row as bf16 pairs: the A operand of O = P V, written over S
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float a0 = exp2f((s0[2 * i] - mx) * sl2), a1 = exp2f((s0[2 * i + 1] - mx) * sl2);
-                    const float b0 = exp2f((s1[2 * i] - mx) * sl2), b1 = exp2f((s1[2 * i + 1] - mx) * sl2);
-                    l += (a0 + a1) + (b0 + b1);
+                    // exponent <= 0: exp2 of (s - max) * scale * log2(e) by the MUFU instruction
+                    const float a0 = ex2_approx(fmaf(s0[2 * i], sl2, -mxs)), a1 = ex2_approx(fmaf(s0[2 * i + 1], sl2, -mxs));
+                    const float b0 = ex2_approx(fmaf(s1[2 * i], sl2, -mxs)), b1 = ex2_approx(fmaf(s1[2 * i + 1], sl2, -mxs));
+                    l4[i & 3] += (a0 + a1) + (b0 + b1);
                     pk[i] = pack_bf16x2(a0, a1);
                     pk[16 + i] = pack_bf16x2(b0, b1);
                 }
+                const float l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
                 tc::tmem_st32(tS, pk);
                 f = row >= 0 ? w / l : 0.0f;
                 tc::fence_before();
@@ -320,7 +347,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
             }
             if (!ok) break;
             tc::fence_after();
-            epilogue_half<D>(tO, softmax ? 0 : D / 2, row, f, wstage, lane, o_acc);
+            epilogue_slabs<D>(tO, softmax ? 0 : SM::SPLIT, softmax ? SM::SPLIT : SM::NSLAB, row, f, wstage, lane,
+                              o_acc);
             tc::fence_before();
             tc::mbar_arrive(bar(kOEmpty + g));
         }

@@ -162,6 +162,21 @@ def kernel_profile(fn, steps):
 
 
 # ------------------------------------------------------------------------------------------------
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of the
+# current kernels on these workloads; set back to None whenever the kernel changes.
+TRAFFIC_BYTES = {
+    ("fwd_t32k_h8_d128_k16", "chunk_attn"): 737_362_176 + 241_751_808,
+    ("fwd_t32k_h8_d128_k16", "score_topk"): 136_370_176 + 36_087_296,
+    # captured on a 4M-token cache (134.3 MB of landmarks read per scan); the scan's traffic grows in
+    # proportion to the landmarks, so the 16M-token figure is four times that capture
+    ("decode_16m_b1_h8_d128_k32", "decode_scan"): 4 * (134_288_640 + 718_080),
+}
+# fp32 reductions into L2-resident rows, 4 rows x 128 B per red.global.add.v4.f32, 16-24 warps per SM:
+# the ceiling measured on this GPU type for the combine of the chunk attention (GB/s)
+COMBINE_PEAK_GBS = 6252.1
+
+
+# ------------------------------------------------------------------------------------------------
 # algorithmic work
 
 
@@ -292,7 +307,7 @@ def main():
     clocks.start()
     # ---------------- prefill forward (headline) ----------------
     value = ms_per_step = None
-    roof = roof_score = breakdown = e2e = None
+    roof = roof_score = roof_combine = breakdown = e2e = None
     pairs = 0
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     w = inputs.WORKLOADS["fwd_t32k_h8_d128_k16"]
@@ -318,9 +333,13 @@ def main():
         dominant = max((k for k in prof_fwd if k != "memset"), key=lambda k: prof_fwd[k][1])
         algo = {"chunk_attn": attn_flops, "score_topk": score_flops}
         roof = roofline_entry(dominant, prof_fwd, algo.get(dominant, attn_flops), "TFLOP/s", tensor_peak, "tensor",
-                              f"{peak_kind} bf16_tflops_sustained")
+                              f"{peak_kind} bf16_tflops_sustained", TRAFFIC_BYTES.get((w.name, dominant)))
         roof_score = roofline_entry("score_topk", prof_fwd, score_flops, "TFLOP/s", tensor_peak, "tensor",
-                                    f"{peak_kind} bf16_tflops_sustained")
+                                    f"{peak_kind} bf16_tflops_sustained", TRAFFIC_BYTES.get((w.name, "score_topk")))
+        roof_score["limiter"] = "ALU pipe (per-row top-K selection); the tensor pipe idles between blocks"
+        # the combine of the chunk attention: pairs x D fp32 reductions into the tokens' accumulator rows
+        roof_combine = roofline_entry("chunk_attn", prof_fwd, pairs * w.D * 4, "GB/s", COMBINE_PEAK_GBS, "l2-red",
+                                      "measured red.global.add.v4.f32 ceiling, L2-resident rows")
         breakdown = {k: {"launches": c, "avg_us": round(t / c * 1e3, 2), "share": round(t / sum(x[1] for x in
                                                                                                prof_fwd.values()), 4)}
                      for k, (c, t) in prof_fwd.items()}
@@ -375,7 +394,7 @@ def main():
             "workload": wd.name, "us_per_token": round(dms * 1e3 / wd.B, 3), "ms_per_step": round(dms, 5),
             "steps": dsteps,
             "roofline": roofline_entry("decode_scan", prof_dec, scan_bytes, "GB/s", hbm_peak, "hbm",
-                                       f"{peak_kind} hbm_gbs"),
+                                       f"{peak_kind} hbm_gbs", TRAFFIC_BYTES.get((wd.name, "decode_scan"))),
             "step_vs_hbm": {"algorithmic_bytes": scan_bytes + gather_bytes,
                             "achieved_GBs": round((scan_bytes + gather_bytes) / (dms / 1e3) / 1e9, 1),
                             "frac": round((scan_bytes + gather_bytes) / (dms / 1e3) / 1e9 / hbm_peak, 4)},
@@ -442,6 +461,7 @@ def main():
                        "l2": "inputs larger than L2 (Q, K, V = 402 MB)", "parallelism": f"dp{world}"},
             "roofline": roof,
             "roofline_score_topk": roof_score,
+            "roofline_combine": roof_combine,
             "kernels": breakdown,
             "gpu_launches": launches,
             "e2e": e2e,

@@ -262,7 +262,7 @@ hsa_status hsa_backward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
     a.chunk_count = l.chunk_count; a.chunk_off = l.chunk_off; a.tile_off = l.tile_off;
     a.chunk_cursor = l.chunk_cursor;
     a.pair_row = l.pair_row; a.pair_w = l.pair_w; a.pair_slot = l.pair_slot;
-    a.tiles = l.tiles; a.num_tiles = l.num_tiles; a.max_tiles = l.max_tiles;
+    a.tiles = l.tiles; a.num_tiles = l.num_tiles; a.max_tiles = l.max_tiles; a.err = l.err;
     return cuda_status(hsa::launch_backward(a, static_cast<cudaStream_t>(stream)), "hsa_backward");
 }
 

@@ -376,7 +376,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2D bf16 tensor [rows, D] (row stride D * 2 bytes), boxes of 64 columns x box_rows rows, 128-byte swizzle.
-static bool make_tmap(CUtensorMap *m, const void *base, uint64_t rows, int D, int box_rows) {
+bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t rows, int D, int box_rows) {
     PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
@@ -396,7 +396,7 @@ static cudaError_t launch_attn_tc_d(const ForwardArgs &a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const uint64_t rows = (uint64_t)a.B * a.H * a.T;
     CUtensorMap tk, tv;
-    if (!make_tmap(&tk, a.K, rows, D, kChunk) || !make_tmap(&tv, a.V, rows, D, kChunk)) return cudaErrorInvalidValue;
+    if (!make_tmap_bf16(&tk, a.K, rows, D, kChunk) || !make_tmap_bf16(&tv, a.V, rows, D, kChunk)) return cudaErrorInvalidValue;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = sms < a.max_tiles ? sms : a.max_tiles;

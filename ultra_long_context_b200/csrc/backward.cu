@@ -297,6 +297,7 @@ cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
             e = cudaMemsetAsync(a.chunk_count, 0, (size_t)BH * a.N * sizeof(int32_t), s);
         if (e == cudaSuccess && a.N > 0)
             e = cudaMemsetAsync(a.chunk_cursor, 0, (size_t)BH * a.N * sizeof(int32_t), s);
+        if (e == cudaSuccess && a.err) e = cudaMemsetAsync(a.err, 0, sizeof(int32_t), s);
     }
     if (e != cudaSuccess || a.N == 0) return e;
     const unsigned dblocks = (unsigned)((rows + 7) / 8);
@@ -305,10 +306,14 @@ cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
         if (a.D == 128) delta_kernel<128><<<dblocks, 256, 0, s>>>(a.out, a.dout, rows, a.delta);
         else delta_kernel<64><<<dblocks, 256, 0, s>>>(a.out, a.dout, rows, a.delta);
     }
+    // head dim 128: tcgen05 kernel over work units of up to kBwdUnitPairs pairs of one chunk;
+    // head dim 64: the mma.sync kernel over tiles of kPairTile pairs
+    const bool tc = a.D == 128;
     e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.tile_off,
-                        a.chunk_cursor,
-                        a.pair_row, a.pair_w, a.pair_slot, a.tiles, a.num_tiles, a.max_tiles, kPairTile, s);
+                        a.chunk_cursor, a.pair_row, a.pair_w, a.pair_slot, a.tiles, a.num_tiles, a.max_tiles,
+                        tc ? kBwdUnitPairs : kPairTile, s);
     if (e != cudaSuccess) return e;
+    if (tc) return launch_backward_tc(a, s);
     if (a.D == 128) {
         const size_t smem = BwdSmem<128>::total;
         e = cudaFuncSetAttribute(chunk_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

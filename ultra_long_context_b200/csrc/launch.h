@@ -1,6 +1,8 @@
 // launch.h -- internal interface between the C ABI (api.cu) and the kernel files.
 #pragma once
 
+#include <cuda.h>
+
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -81,9 +83,17 @@ struct BackwardArgs {
     int32_t *pair_slot;    // [B*H*T*topk] slot j of each pair (unused by the forward)
     PairTile *tiles;
     int32_t *num_tiles;
+    int32_t *err;          // [1] set when a bounded device wait ran out
     int max_tiles;
 };
 cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s);
+// Gradients on the tcgen05 tensor cores (bwd_tc.cu), head dim 128; work units of up to 1024 pairs.
+constexpr int kBwdUnitPairs = 1024;
+cudaError_t launch_backward_tc(const BackwardArgs &a, cudaStream_t s);
+
+// 2-D bf16 tensor map over a [rows, D] row-major tensor: boxes of 64 columns x box_rows rows,
+// 128-byte swizzle (attn_tc.cu). False if the driver entry point is missing or the encoding fails.
+bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t rows, int D, int box_rows);
 
 // Message returned by hsa_last_error() on the calling thread.
 void set_last_error(const char *msg);

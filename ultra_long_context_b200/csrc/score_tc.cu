@@ -309,31 +309,6 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
     }
 }
 
-// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
-static PFN_cuTensorMapEncodeTiled_v12000 st_encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
-static bool st_tmap(CUtensorMap *m, const void *base, uint64_t rows, int D, int box_rows) {
-    PFN_cuTensorMapEncodeTiled_v12000 fn = st_encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
-    const cuuint32_t estr[2] = {1u, 1u};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, int K>
 static cudaError_t launch_st(const ForwardArgs &a, const CUtensorMap &tl, cudaStream_t s) {
     const size_t smem = StSmem<D, K>::DYN;
@@ -351,7 +326,7 @@ template <int D>
 static cudaError_t launch_st_d(const ForwardArgs &a, cudaStream_t s) {
     CUtensorMap tl;
     // with no complete chunk the landmark tensor may be empty: point the map at Q (never read)
-    if (!st_tmap(&tl, a.N > 0 ? (const void *)a.L : (const void *)a.Q,
+    if (!make_tmap_bf16(&tl, a.N > 0 ? (const void *)a.L : (const void *)a.Q,
                  a.N > 0 ? (uint64_t)a.B * a.H * a.N : (uint64_t)a.B * a.H * a.T, D, kStCols))
         return cudaErrorInvalidValue;
     if (a.topk <= 8) return launch_st<D, 8>(a, tl, s);

@@ -58,7 +58,8 @@ struct BtSmem {  // head dim 128
     static constexpr uint32_t EROW = LROW + 1024;      // int[2][128]: token rows for the dQ epilogue
     static constexpr uint32_t EDS = EROW + 1024;       // float[2][128]: ds for the dQ epilogue
     static constexpr uint32_t SDS = EDS + 1024;        // float[2][128]: ds for dL
-    static constexpr uint32_t BAR = SDS + 1024;
+    static constexpr uint32_t SDL = SDS + 1024;        // float[4][128]: the unit's dL per compute warp
+    static constexpr uint32_t BAR = SDL + 2048;
     static constexpr int NBAR = 20;
     static constexpr uint32_t TMEM = BAR + NBAR * 8;
     static constexpr uint32_t BYTES = TMEM + 16;
@@ -134,9 +135,11 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
     int *e_row = reinterpret_cast<int *>(s + SM::EROW);
     float *e_ds = reinterpret_cast<float *>(s + SM::EDS);
     float *s_ds = reinterpret_cast<float *>(s + SM::SDS);
+    float *s_dl = reinterpret_cast<float *>(s + SM::SDL);
     auto bar = [&](int i) { return sb + SM::BAR + 8u * (uint32_t)i; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid < 4 * D) s_dl[tid] = 0.0f;  // ordered before use by the __syncthreads below
     const int nunits = num_units[0];
     const int G = gridDim.x;
     const int mine = (int)blockIdx.x < nunits ? (nunits - 1 - (int)blockIdx.x) / G + 1 : 0;
@@ -174,19 +177,20 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
         const int lw = warp - kBtLoaderWarp0, lt = tid - 32 * kBtLoaderWarp0;
         const int rsub = lane / CPR, ch = lane % CPR;
         const int myr = 32 * lw + lane;
-        int pending = -1;
+        // this thread's pair of the current tile: token row, weight, delta (fetched one tile ahead)
+        auto fetch = [&](const BtCursor &t, int &row, float &wt, float &dl) {
+            const int p = t.i * kBtTile + myr;
+            row = (!t.done() && p < t.u.count) ? pair_row[t.u.start + p] : -1;
+            wt = row >= 0 ? pair_w[t.u.start + p] : 0.0f;
+            dl = row >= 0 ? delta[row] : 0.0f;
+        };
+        int myrow;
+        float myw, mydel;
+        fetch(cur, myrow, myw, mydel);
         for (; !cur.done() && ok; cur.next()) {
             const int j = cur.j, st = j & 1;
             const int bh = cur.u.chunk / N, c = cur.u.chunk % N;
             if (cur.first_tile()) {
-                // publish the previous tile first: the previous unit can only finish (and free K, V and
-                // its landmark row) once that tile has been computed
-                if (pending >= 0) {
-                    cp_async_wait<0>();
-                    tc::fence_proxy_async_smem();
-                    tc::mbar_arrive(bar(kBQdFull + (pending & 1)));
-                    pending = -1;
-                }
                 // every loader thread waits: the landmark row written below is read by the dQ epilogue
                 // of the unit two back, which kv_empty of the previous unit orders before this point
                 ok = tc::mbar_wait(bar(kBKvEmpty), ((uint32_t)cur.k & 1u) ^ 1u);
@@ -202,11 +206,9 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             }
             ok = ok && tc::mbar_wait(bar(kBQdEmpty + st), ((uint32_t)(j >> 1) & 1u) ^ 1u);
             if (!ok) break;
-            const int p = cur.i * kBtTile + myr;
-            const int myrow = p < cur.u.count ? pair_row[cur.u.start + p] : -1;
             s_row[st * 128 + myr] = myrow;
-            s_w[st * 128 + myr] = myrow >= 0 ? pair_w[cur.u.start + p] : 0.0f;
-            s_del[st * 128 + myr] = myrow >= 0 ? delta[myrow] : 0.0f;
+            s_w[st * 128 + myr] = myw;
+            s_del[st * 128 + myr] = mydel;
             if (cur.first_tile())  // the unit's landmark row, fp32, for the ds L_c term of dQ
                 s_L[(cur.k & 1) * 128 + myr] = __uint_as_float((uint32_t)L[((size_t)bh * N + c) * D + myr] << 16);
             const uint32_t sq = sb + SM::STG + st * SM::QD;
@@ -222,18 +224,18 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                                src >= 0 ? 16 : 0);
             }
             cp_async_commit();
-            if (pending >= 0) {  // publish the previous tile once its copies have landed
-                cp_async_wait<1>();
-                tc::fence_proxy_async_smem();
-                tc::mbar_arrive(bar(kBQdFull + (pending & 1)));
+            {  // the next tile's metadata while the copies run
+                BtCursor nx = cur;
+                nx.next();
+                fetch(nx, myrow, myw, mydel);
             }
-            pending = j;
+            // publish this tile as soon as its copies have landed: the next stage frees only after the
+            // previous tile's gradient MMAs, so waiting for it first would serialise the tiles
+            cp_async_wait<0>();
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(bar(kBQdFull + st));
         }
         cp_async_wait<0>();
-        if (ok && pending >= 0) {
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(bar(kBQdFull + (pending & 1)));
-        }
     } else if (warp == kBtMmaWarp) {
         // ================= MMA issuer =================
         if (lane == 0 && mine > 0) {
@@ -307,7 +309,6 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
         const int r = tid;
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const float sl2 = scale * 1.4426950408889634f;
-        float dl = 0.0f;  // dL_c[d = r] over the unit's pairs (without the scale)
         for (; !cur.done() && ok; cur.next()) {
             const int j = cur.j, b = j & 1;
             const uint32_t ph = (uint32_t)(j >> 1) & 1u;
@@ -388,16 +389,28 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             e_ds[b * 128 + r] = ds;
             tc::fence_proxy_async_smem();  // w P / dS stores -> tensor core reads
             asm volatile("bar.sync 1, 128;" ::: "memory");  // every ds of the tile is in s_ds
-            {  // dL: thread r takes column d = r of this tile's Q rows
-                const unsigned char *q = s + SM::STG + b * SM::QD + (r >> 6) * SM::HALF;
-                const int cc = (r & 63) >> 3, e = r & 7;
-                float a4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 8
-                for (int p = 0; p < kBtTile; ++p) {
-                    const uint16_t qv = *reinterpret_cast<const uint16_t *>(q + tc::sw128(p, cc) + e * 2);
-                    a4[p & 3] = fmaf(s_ds[b * 128 + p], __uint_as_float((uint32_t)qv << 16), a4[p & 3]);
+            {  // dL: thread r takes the 16-byte column chunk cc (columns 8 cc .. 8 cc + 7) of pairs 16 gq .. + 15
+                const int cc = r & 15, gq = r >> 4;
+                const unsigned char *qt = s + SM::STG + b * SM::QD + (cc >> 3) * SM::HALF;
+                float a8[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 4
+                for (int i = 0; i < 16; ++i) {
+                    const int p = 16 * gq + i;
+                    const uint4 qv = *reinterpret_cast<const uint4 *>(qt + tc::sw128(p, cc & 7));
+                    const float dsp = s_ds[b * 128 + p];
+                    a8[0] = fmaf(dsp, bf16_lo(qv.x), a8[0]); a8[1] = fmaf(dsp, bf16_hi(qv.x), a8[1]);
+                    a8[2] = fmaf(dsp, bf16_lo(qv.y), a8[2]); a8[3] = fmaf(dsp, bf16_hi(qv.y), a8[3]);
+                    a8[4] = fmaf(dsp, bf16_lo(qv.z), a8[4]); a8[5] = fmaf(dsp, bf16_hi(qv.z), a8[5]);
+                    a8[6] = fmaf(dsp, bf16_lo(qv.w), a8[6]); a8[7] = fmaf(dsp, bf16_hi(qv.w), a8[7]);
                 }
-                dl += (a4[0] + a4[1]) + (a4[2] + a4[3]);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) a8[k] += __shfl_xor_sync(0xffffffffu, a8[k], 16);  // same cc
+                if (lane < 16) {  // this warp's own partial row: no other thread touches these 8 entries
+                    float4 *dst = reinterpret_cast<float4 *>(s_dl + warp * D + 8 * cc);
+                    const float4 x0 = dst[0], x1 = dst[1];
+                    dst[0] = make_float4(x0.x + a8[0], x0.y + a8[1], x0.z + a8[2], x0.w + a8[3]);
+                    dst[1] = make_float4(x1.x + a8[4], x1.y + a8[5], x1.z + a8[6], x1.w + a8[7]);
+                }
             }
             tc::mbar_arrive(bar(kBDsFull));
             tc::mbar_arrive(bar(kBEReady + b));
@@ -419,8 +432,11 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                 }
                 tc::fence_before();
                 tc::mbar_arrive(bar(kBAccEmpty));
-                atomicAdd(dL + ((size_t)bh * N + c) * D + r, scale * dl);
-                dl = 0.0f;
+                asm volatile("bar.sync 1, 128;" ::: "memory");  // every warp's dL partials are in s_dl
+                atomicAdd(dL + ((size_t)bh * N + c) * D + r,
+                          scale * ((s_dl[r] + s_dl[D + r]) + (s_dl[2 * D + r] + s_dl[3 * D + r])));
+                asm volatile("bar.sync 1, 128;" ::: "memory");  // all reads done before the reset
+                s_dl[r] = s_dl[D + r] = s_dl[2 * D + r] = s_dl[3 * D + r] = 0.0f;
             }
         }
     } else {

@@ -19,8 +19,8 @@
 // and K / V are 128-byte-swizzled rows that serve as K-major operands (for S, dP') and as MN-major
 // operands (Q^T and dO^T for dK^T, dV^T; K for dQ); w P and dS are [pair][key] swizzled rows that
 // serve as the K-major A operand of dQ and the MN-major B operand of dK^T / dV^T.
-// Warps: 0-3 compute (one thread per pair row: softmax, g, ds, dS, w P; dL; the unit's dK / dV
-// output), 4-11 dQ epilogue (two warpgroups, one per half of the columns), 12-15 loaders (cp.async
+// Warps: 0-3 compute (one thread per pair row: softmax, g, ds, dS, w P; dL), 4-11 epilogue (two
+// warpgroups: one half of the dQ columns each, and the unit's dV or dK), 12-15 loaders (cp.async
 // gathers of Q and dO rows, TMA tiles of K and V), 16 MMA issuer.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -55,40 +55,39 @@ struct BtSmem {  // head dim 128
     static constexpr uint32_t W = ROW + 1024;          // float[2][128]: fusion weights
     static constexpr uint32_t DEL = W + 1024;          // float[2][128]: delta of the pair's token
     static constexpr uint32_t LROW = DEL + 1024;       // float[2][128]: the unit's landmark row (fp32)
-    static constexpr uint32_t EROW = LROW + 1024;      // int[2][128]: token rows for the dQ epilogue
-    static constexpr uint32_t EDS = EROW + 1024;       // float[2][128]: ds for the dQ epilogue
-    static constexpr uint32_t SDS = EDS + 1024;        // float[2][128]: ds for dL
-    static constexpr uint32_t SDL = SDS + 1024;        // float[4][128]: the unit's dL per compute warp
+    static constexpr uint32_t EROW = LROW + 1024;      // int[4][128]: token rows for the dQ epilogue
+    static constexpr uint32_t EDS = EROW + 2048;       // float[4][128]: ds (dQ epilogue and dL)
+    static constexpr uint32_t SDL = EDS + 2048;        // float[4][128]: the unit's dL per compute warp
     static constexpr uint32_t BAR = SDL + 2048;
-    static constexpr int NBAR = 20;
+    static constexpr int NBAR = 22;
     static constexpr uint32_t TMEM = BAR + NBAR * 8;
     static constexpr uint32_t BYTES = TMEM + 16;
     static constexpr size_t DYN = BYTES + 1024;
     static_assert(DYN <= 227 * 1024, "shared memory budget");
     // TMEM columns
-    static constexpr uint32_t S_COL = 0;     // S buffers [2] x 64 (P, fp32, is written back over S)
-    static constexpr uint32_t DP_COL = 128;  // dP' buffers [2] x 64
-    static constexpr uint32_t DQ_COL = 256;  // dQ: 128
+    static constexpr uint32_t S_COL = 0;     // S: 64 (P, fp32, is written back over S)
+    static constexpr uint32_t DP_COL = 64;   // dP': 64
+    static constexpr uint32_t DQ_COL = 128;  // dQ buffers [2] x 128
     static constexpr uint32_t DV_COL = 384;  // dV^T: 64 (lane = d)
     static constexpr uint32_t DK_COL = 448;  // dK^T: 64 (lane = d)
 };
 
-// mbarrier slots. Phases: qd_* and s_* and e_ready per tile pair (j / 2), ds_* and dq_* per tile (j),
-// kv_* and acc_* per unit (k).
+// mbarrier slots. Phases: qd_* and dq_* per tile pair (j / 2), e_ready per 4 tiles (j / 4), s_* and
+// ds_* per tile (j), kv_* and acc_* per unit (k).
 enum {
     kBQdFull = 0,          // [2] loaders (128 arrivals, after their Q / dO copies have landed)
     kBQdEmpty = 2,         // [2] commit after the last MMA that reads the stage
     kBKvFull = 4,          // loader thread 0 (arrive + K, V bytes)
     kBKvEmpty = 5,         // commit after the unit's last MMA
-    kBSFull = 6,           // [2] commit after S and dP'
-    kBSEmpty = 8,          // [2] compute warps (128) once P / dP' are consumed
-    kBDsFull = 10,         // compute warps (128) once w P and dS are in shared memory
-    kBDsEmpty = 11,        // commit after dQ, dK^T, dV^T
-    kBDqFull = 12,         // commit after dQ
-    kBDqEmpty = 13,        // epilogue warps (256) once dQ is read
+    kBSFull = 6,           // commit after S and dP'
+    kBSEmpty = 7,          // compute warps (128) once P / dP' are consumed
+    kBDsFull = 8,          // compute warps (128) once w P and dS are in shared memory
+    kBDsEmpty = 9,         // commit after dQ, dK^T, dV^T
+    kBDqFull = 10,         // [2] commit after dQ into TMEM buffer j % 2
+    kBDqEmpty = 12,        // [2] epilogue warps (256) once that buffer is read
     kBAccFull = 14,        // commit after the unit's last dK^T / dV^T
-    kBAccEmpty = 15,       // compute warps (128) once dK^T / dV^T are read
-    kBEReady = 16,         // [2] compute warps (128): rows and ds of a tile for the dQ epilogue
+    kBAccEmpty = 15,       // epilogue warps (256) once dK^T / dV^T are read
+    kBEReady = 16,         // [4] compute warps (128): rows and ds of tile j for the dQ epilogue (slot j % 4)
 };
 
 // Walks this CTA's units and their 128-pair tiles in order.
@@ -134,7 +133,6 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
     float *s_L = reinterpret_cast<float *>(s + SM::LROW);
     int *e_row = reinterpret_cast<int *>(s + SM::EROW);
     float *e_ds = reinterpret_cast<float *>(s + SM::EDS);
-    float *s_ds = reinterpret_cast<float *>(s + SM::SDS);
     float *s_dl = reinterpret_cast<float *>(s + SM::SDL);
     auto bar = [&](int i) { return sb + SM::BAR + 8u * (uint32_t)i; };
 
@@ -149,18 +147,18 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(bar(kBQdFull + i), 128);
             tc::mbar_init(bar(kBQdEmpty + i), 1);
-            tc::mbar_init(bar(kBSFull + i), 1);
-            tc::mbar_init(bar(kBSEmpty + i), 128);
-            tc::mbar_init(bar(kBEReady + i), 128);
+            tc::mbar_init(bar(kBDqFull + i), 1);
+            tc::mbar_init(bar(kBDqEmpty + i), 256);
         }
+        for (int i = 0; i < 4; ++i) tc::mbar_init(bar(kBEReady + i), 128);
         tc::mbar_init(bar(kBKvFull), 1);
         tc::mbar_init(bar(kBKvEmpty), 1);
+        tc::mbar_init(bar(kBSFull), 1);
+        tc::mbar_init(bar(kBSEmpty), 128);
         tc::mbar_init(bar(kBDsFull), 128);
         tc::mbar_init(bar(kBDsEmpty), 1);
-        tc::mbar_init(bar(kBDqFull), 1);
-        tc::mbar_init(bar(kBDqEmpty), 256);
         tc::mbar_init(bar(kBAccFull), 1);
-        tc::mbar_init(bar(kBAccEmpty), 128);
+        tc::mbar_init(bar(kBAccEmpty), 256);
         tc::fence_mbar_init();
     }
     tc::fence_before();
@@ -247,14 +245,14 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             while (!cg.done()) {
                 bool progress = false;
                 if (cg.j < cs.j && tc::mbar_test(bar(kBDsFull), (uint32_t)cg.j & 1u) &&
-                    tc::mbar_test(bar(kBDqEmpty), ((uint32_t)cg.j & 1u) ^ 1u) &&
+                    tc::mbar_test(bar(kBDqEmpty + (cg.j & 1)), ((uint32_t)(cg.j >> 1) & 1u) ^ 1u) &&
                     (!cg.first_tile() || tc::mbar_test(bar(kBAccEmpty), ((uint32_t)cg.k & 1u) ^ 1u))) {
                     tc::fence_after();
                     const int st = cg.j & 1;
                     const uint32_t sq = sb + SM::STG + st * SM::QD, sdo = sq + 2 * SM::HALF;
 #pragma unroll 1
                     for (int ks = 0; ks < kChunk / 16; ++ks)  // dQ = dS K: K = 64 keys
-                        tc::mma_bf16_ss(tmem + SM::DQ_COL, tc::desc_kmajor(sb + SM::DS + ks * 32),
+                        tc::mma_bf16_ss(tmem + SM::DQ_COL + st * 128, tc::desc_kmajor(sb + SM::DS + ks * 32),
                                         tc::desc_mnmajor(sb + SM::KO + ks * 2048, SM::KH), id_q, ks > 0 ? 1u : 0u);
                     const uint32_t acc0 = cg.first_tile() ? 0u : 1u;
 #pragma unroll 1
@@ -264,7 +262,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                         tc::mma_bf16_ss(tmem + SM::DK_COL, tc::desc_mnmajor(sq + ks * 2048, SM::HALF),
                                         tc::desc_mnmajor(sb + SM::DS + ks * 2048, 8192), id_t, ks > 0 ? 1u : acc0);
                     }
-                    tc::commit(bar(kBDqFull));
+                    tc::commit(bar(kBDqFull + st));
                     tc::commit(bar(kBDsEmpty));
                     tc::commit(bar(kBQdEmpty + st));
                     if (cg.last_tile()) {
@@ -276,7 +274,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                 }
                 if (!cs.done() && cs.j < cg.j + 2 &&
                     tc::mbar_test(bar(kBQdFull + (cs.j & 1)), (uint32_t)(cs.j >> 1) & 1u) &&
-                    tc::mbar_test(bar(kBSEmpty + (cs.j & 1)), ((uint32_t)(cs.j >> 1) & 1u) ^ 1u) &&
+                    tc::mbar_test(bar(kBSEmpty), ((uint32_t)cs.j & 1u) ^ 1u) &&
                     (!cs.first_tile() || tc::mbar_test(bar(kBKvFull), (uint32_t)cs.k & 1u))) {
                     tc::fence_after();
                     const int b = cs.j & 1;
@@ -285,12 +283,12 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                     for (int ks = 0; ks < D / 16; ++ks) {
                         const uint32_t koff = (uint32_t)((ks >> 2) * SM::HALF + (ks & 3) * 32);
                         const uint32_t kk = (uint32_t)((ks >> 2) * SM::KH + (ks & 3) * 32);
-                        tc::mma_bf16_ss(tmem + SM::S_COL + b * 64, tc::desc_kmajor(sq + koff),
+                        tc::mma_bf16_ss(tmem + SM::S_COL, tc::desc_kmajor(sq + koff),
                                         tc::desc_kmajor(sb + SM::KO + kk), id_s, ks > 0 ? 1u : 0u);
-                        tc::mma_bf16_ss(tmem + SM::DP_COL + b * 64, tc::desc_kmajor(sdo + koff),
+                        tc::mma_bf16_ss(tmem + SM::DP_COL, tc::desc_kmajor(sdo + koff),
                                         tc::desc_kmajor(sb + SM::VO + kk), id_s, ks > 0 ? 1u : 0u);
                     }
-                    tc::commit(bar(kBSFull + b));
+                    tc::commit(bar(kBSFull));
                     cs.next();
                     progress = true;
                 }
@@ -315,17 +313,16 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             // qd_full publishes the loaders' rows / weights / deltas of this stage; it cannot run a phase
             // ahead of this wait (stage b is reloaded only after this tile's gradient MMAs, which need
             // this warpgroup's ds_full)
-            ok = tc::mbar_wait(bar(kBQdFull + b), ph) && tc::mbar_wait(bar(kBSFull + b), ph);
+            ok = tc::mbar_wait(bar(kBQdFull + b), ph) && tc::mbar_wait(bar(kBSFull), (uint32_t)j & 1u);
             if (!ok) break;
             tc::fence_after();
             const int row = s_row[b * 128 + r];
             const float w = s_w[b * 128 + r], del = s_del[b * 128 + r];
-            const uint32_t tS = tmem + lane_off + SM::S_COL + b * 64;
-            const uint32_t tDP = tmem + lane_off + SM::DP_COL + b * 64;
+            const uint32_t tS = tmem + lane_off + SM::S_COL;
+            const uint32_t tDP = tmem + lane_off + SM::DP_COL;
             {  // P = softmax over the chunk's 64 keys (fp32), written back over S
                 float v0[32], v1[32];
-                tc::tmem_ld32(tS, v0);
-                tc::tmem_ld32(tS + 32, v1);
+                tc::tmem_ld32x2(tS, v0, tS + 32, v1);
                 float m8[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
@@ -353,8 +350,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
 #pragma unroll 1
             for (int h = 0; h < 4; ++h) {
                 float pv[16], dv[16];
-                tc::tmem_ld16(tS + 16 * h, pv);
-                tc::tmem_ld16(tDP + 16 * h, dv);
+                tc::tmem_ld16x2(tS + 16 * h, pv, tDP + 16 * h, dv);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) g4[i & 3] = fmaf(pv[i], dv[i], g4[i & 3]);
             }
@@ -366,8 +362,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
 #pragma unroll 1
             for (int h = 0; h < 4; ++h) {
                 float pv[16], dv[16];
-                tc::tmem_ld16(tS + 16 * h, pv);
-                tc::tmem_ld16(tDP + 16 * h, dv);
+                tc::tmem_ld16x2(tS + 16 * h, pv, tDP + 16 * h, dv);
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {  // 16-byte chunk 2h + q = keys 16h + 8q .. + 7
                     uint32_t a[4], d4[4];
@@ -383,12 +378,12 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                 }
             }
             tc::fence_before();
-            tc::mbar_arrive(bar(kBSEmpty + b));  // P / dP' of buffer b are consumed
-            s_ds[b * 128 + r] = ds;
-            e_row[b * 128 + r] = row;
-            e_ds[b * 128 + r] = ds;
+            tc::mbar_arrive(bar(kBSEmpty));  // P / dP' are consumed: S(j + 1) may overwrite them
+            const int slot = j & 3;
+            e_row[slot * 128 + r] = row;
+            e_ds[slot * 128 + r] = ds;
             tc::fence_proxy_async_smem();  // w P / dS stores -> tensor core reads
-            asm volatile("bar.sync 1, 128;" ::: "memory");  // every ds of the tile is in s_ds
+            asm volatile("bar.sync 1, 128;" ::: "memory");  // every ds of the tile is in e_ds
             {  // dL: thread r takes the 16-byte column chunk cc (columns 8 cc .. 8 cc + 7) of pairs 16 gq .. + 15
                 const int cc = r & 15, gq = r >> 4;
                 const unsigned char *qt = s + SM::STG + b * SM::QD + (cc >> 3) * SM::HALF;
@@ -397,7 +392,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                 for (int i = 0; i < 16; ++i) {
                     const int p = 16 * gq + i;
                     const uint4 qv = *reinterpret_cast<const uint4 *>(qt + tc::sw128(p, cc & 7));
-                    const float dsp = s_ds[b * 128 + p];
+                    const float dsp = e_ds[slot * 128 + p];
                     a8[0] = fmaf(dsp, bf16_lo(qv.x), a8[0]); a8[1] = fmaf(dsp, bf16_hi(qv.x), a8[1]);
                     a8[2] = fmaf(dsp, bf16_lo(qv.y), a8[2]); a8[3] = fmaf(dsp, bf16_hi(qv.y), a8[3]);
                     a8[4] = fmaf(dsp, bf16_lo(qv.z), a8[4]); a8[5] = fmaf(dsp, bf16_hi(qv.z), a8[5]);
@@ -413,25 +408,9 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                 }
             }
             tc::mbar_arrive(bar(kBDsFull));
-            tc::mbar_arrive(bar(kBEReady + b));
-            if (cur.last_tile()) {  // the unit's dK, dV, dL: thread r = column d (TMEM lane of dK^T, dV^T)
-                ok = tc::mbar_wait(bar(kBAccFull), (uint32_t)cur.k & 1u);
-                if (!ok) break;
-                tc::fence_after();
+            tc::mbar_arrive(bar(kBEReady + slot));
+            if (cur.last_tile()) {  // the unit's dL (the epilogue warps add its dK and dV)
                 const int bh = cur.u.chunk / N, c = cur.u.chunk % N;
-                const size_t krow0 = (size_t)bh * T + (size_t)c * kChunk;
-#pragma unroll 1
-                for (int h = 0; h < 2; ++h) {
-                    float v[32];
-                    tc::tmem_ld32(tmem + lane_off + SM::DV_COL + 32 * h, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) atomicAdd(dV + (krow0 + 32 * h + i) * D + r, v[i]);
-                    tc::tmem_ld32(tmem + lane_off + SM::DK_COL + 32 * h, v);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) atomicAdd(dK + (krow0 + 32 * h + i) * D + r, scale * v[i]);
-                }
-                tc::fence_before();
-                tc::mbar_arrive(bar(kBAccEmpty));
                 asm volatile("bar.sync 1, 128;" ::: "memory");  // every warp's dL partials are in s_dl
                 atomicAdd(dL + ((size_t)bh * N + c) * D + r,
                           scale * ((s_dl[r] + s_dl[D + r]) + (s_dl[2 * D + r] + s_dl[3 * D + r])));
@@ -448,20 +427,21 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
         unsigned char *stage = wstage + lane * SM::OUT_ROW;
         for (; !cur.done() && ok; cur.next()) {
             const int j = cur.j, b = j & 1;
-            // e_ready cannot run a phase ahead: the compute warps write tile j + 2's rows only after
-            // dQ(j + 1) was issued, which needs this warpgroup's dq_empty for tile j
-            ok = tc::mbar_wait(bar(kBEReady + b), (uint32_t)(j >> 1) & 1u) &&
-                 tc::mbar_wait(bar(kBDqFull), (uint32_t)j & 1u);
+            // e_ready (slot j % 4) cannot run a phase ahead: the compute warps write tile j + 4's rows
+            // only after dQ(j + 3) was issued, which needs this warpgroup's dq_empty for tile j + 1
+            const int slot = j & 3;
+            ok = tc::mbar_wait(bar(kBEReady + slot), (uint32_t)(j >> 2) & 1u) &&
+                 tc::mbar_wait(bar(kBDqFull + b), (uint32_t)(j >> 1) & 1u);
             if (!ok) break;
             tc::fence_after();
-            const int row = e_row[b * 128 + r];
-            const float ds = e_ds[b * 128 + r];
+            const int row = e_row[slot * 128 + r];
+            const float ds = e_ds[slot * 128 + r];
             const float *Lr = s_L + (cur.k & 1) * 128;
 #pragma unroll 1
             for (int cb = 0; cb < 64 / (int)SM::SLAB; ++cb) {
                 const int col0 = 64 * e + cb * (int)SM::SLAB;
                 float o[16];
-                tc::tmem_ld16(tmem + lane_off + SM::DQ_COL + col0, o);
+                tc::tmem_ld16(tmem + lane_off + SM::DQ_COL + b * 128 + col0, o);
                 __syncwarp();  // the previous slab has been read back
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
@@ -480,7 +460,28 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                 }
             }
             tc::fence_before();
-            tc::mbar_arrive(bar(kBDqEmpty));
+            tc::mbar_arrive(bar(kBDqEmpty + b));
+            if (cur.last_tile()) {
+                // the unit's dV (warpgroup 0) or dK (warpgroup 1): thread = column d = TMEM lane of
+                // dV^T / dK^T; each warp-wide reduction covers one key row's 32 consecutive columns
+                ok = tc::mbar_wait(bar(kBAccFull), (uint32_t)cur.k & 1u);
+                if (!ok) break;
+                tc::fence_after();
+                const int bh = cur.u.chunk / N, c = cur.u.chunk % N;
+                const size_t krow0 = (size_t)bh * T + (size_t)c * kChunk;
+                float *dst = e == 0 ? dV : dK;
+                const float f = e == 0 ? 1.0f : scale;
+                const uint32_t tacc = tmem + lane_off + (e == 0 ? SM::DV_COL : SM::DK_COL);
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    float v[32];
+                    tc::tmem_ld32(tacc + 32 * h, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) atomicAdd(dst + (krow0 + 32 * h + i) * D + r, f * v[i]);
+                }
+                tc::fence_before();
+                tc::mbar_arrive(bar(kBAccEmpty));
+            }
         }
     }
     if (!ok) atomicOr(err, 1);

@@ -19,9 +19,10 @@
 // and K / V are 128-byte-swizzled rows that serve as K-major operands (for S, dP') and as MN-major
 // operands (Q^T and dO^T for dK^T, dV^T; K for dQ); w P and dS are [pair][key] swizzled rows that
 // serve as the K-major A operand of dQ and the MN-major B operand of dK^T / dV^T.
-// Warps: 0-3 compute (one thread per pair row: softmax, g, ds, dS, w P; dL), 4-11 epilogue (two
+// Warps: 0-3 compute (one thread per pair row: softmax, g, ds, dS, w P), 4-11 epilogue (two
 // warpgroups: one half of the dQ columns each, and the unit's dV or dK), 12-15 loaders (cp.async
-// gathers of Q and dO rows, TMA tiles of K and V), 16 MMA issuer.
+// gathers of Q and dO rows, TMA tiles of K and V; dL from a tile's Q rows before its stage is
+// reloaded), 16 MMA issuer.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -185,6 +186,48 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
         int myrow;
         float myw, mydel;
         fetch(cur, myrow, myw, mydel);
+        // dL_c += sum over a tile's pairs of ds q, computed here from the tile's Q rows just before the
+        // stage is reloaded (the tile two back). Thread lt takes the 16-byte column chunk cc of pairs
+        // 16 gq .. + 15; each loader warp keeps its own partial row in s_dl.
+        BtCursor lag = cur;
+        auto do_dl = [&]() {
+            const int jl = lag.j, slot = jl & 3, stl = jl & 1;
+            // qd_full (all loaders' copies of that tile) and e_ready (its ds) have completed long ago
+            // and cannot run a phase ahead: the stage's next fill and that slot's next tile come after
+            ok = ok && tc::mbar_wait(bar(kBQdFull + stl), (uint32_t)(jl >> 1) & 1u) &&
+                 tc::mbar_wait(bar(kBEReady + slot), (uint32_t)(jl >> 2) & 1u);
+            if (!ok) return;
+            const int cc = lt & 15, gq = lt >> 4;
+            const unsigned char *qt = s + SM::STG + stl * SM::QD + (cc >> 3) * SM::HALF;
+            float a8[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 4
+            for (int i = 0; i < 16; ++i) {
+                const int p = 16 * gq + i;
+                const uint4 qv = *reinterpret_cast<const uint4 *>(qt + tc::sw128(p, cc & 7));
+                const float dsp = e_ds[slot * 128 + p];
+                a8[0] = fmaf(dsp, bf16_lo(qv.x), a8[0]); a8[1] = fmaf(dsp, bf16_hi(qv.x), a8[1]);
+                a8[2] = fmaf(dsp, bf16_lo(qv.y), a8[2]); a8[3] = fmaf(dsp, bf16_hi(qv.y), a8[3]);
+                a8[4] = fmaf(dsp, bf16_lo(qv.z), a8[4]); a8[5] = fmaf(dsp, bf16_hi(qv.z), a8[5]);
+                a8[6] = fmaf(dsp, bf16_lo(qv.w), a8[6]); a8[7] = fmaf(dsp, bf16_hi(qv.w), a8[7]);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) a8[k] += __shfl_xor_sync(0xffffffffu, a8[k], 16);  // same cc
+            float4 *own = reinterpret_cast<float4 *>(s_dl + lw * D + 8 * cc);  // only this lane writes these
+            if (lane < 16) {
+                const float4 x0 = own[0], x1 = own[1];
+                own[0] = make_float4(x0.x + a8[0], x0.y + a8[1], x0.z + a8[2], x0.w + a8[3]);
+                own[1] = make_float4(x1.x + a8[4], x1.y + a8[5], x1.z + a8[6], x1.w + a8[7]);
+            }
+            if (lag.last_tile()) {  // the unit's dL: thread lt = column d
+                const int bhl = lag.u.chunk / N, cl = lag.u.chunk % N;
+                asm volatile("bar.sync 2, 128;" ::: "memory");  // every loader warp's partials are in s_dl
+                atomicAdd(dL + ((size_t)bhl * N + cl) * D + lt,
+                          scale * ((s_dl[lt] + s_dl[D + lt]) + (s_dl[2 * D + lt] + s_dl[3 * D + lt])));
+                asm volatile("bar.sync 2, 128;" ::: "memory");  // all reads done before the owners reset
+                if (lane < 16) own[0] = own[1] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            }
+            lag.next();
+        };
         for (; !cur.done() && ok; cur.next()) {
             const int j = cur.j, st = j & 1;
             const int bh = cur.u.chunk / N, c = cur.u.chunk % N;
@@ -202,6 +245,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                     }
                 }
             }
+            if (j >= 2) do_dl();  // the stage about to be reloaded holds tile j - 2
             ok = ok && tc::mbar_wait(bar(kBQdEmpty + st), ((uint32_t)(j >> 1) & 1u) ^ 1u);
             if (!ok) break;
             s_row[st * 128 + myr] = myrow;
@@ -233,6 +277,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             tc::fence_proxy_async_smem();
             tc::mbar_arrive(bar(kBQdFull + st));
         }
+        while (ok && !lag.done()) do_dl();  // the last tiles
         cp_async_wait<0>();
     } else if (warp == kBtMmaWarp) {
         // ================= MMA issuer =================
@@ -383,40 +428,8 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             e_row[slot * 128 + r] = row;
             e_ds[slot * 128 + r] = ds;
             tc::fence_proxy_async_smem();  // w P / dS stores -> tensor core reads
-            asm volatile("bar.sync 1, 128;" ::: "memory");  // every ds of the tile is in e_ds
-            {  // dL: thread r takes the 16-byte column chunk cc (columns 8 cc .. 8 cc + 7) of pairs 16 gq .. + 15
-                const int cc = r & 15, gq = r >> 4;
-                const unsigned char *qt = s + SM::STG + b * SM::QD + (cc >> 3) * SM::HALF;
-                float a8[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 4
-                for (int i = 0; i < 16; ++i) {
-                    const int p = 16 * gq + i;
-                    const uint4 qv = *reinterpret_cast<const uint4 *>(qt + tc::sw128(p, cc & 7));
-                    const float dsp = e_ds[slot * 128 + p];
-                    a8[0] = fmaf(dsp, bf16_lo(qv.x), a8[0]); a8[1] = fmaf(dsp, bf16_hi(qv.x), a8[1]);
-                    a8[2] = fmaf(dsp, bf16_lo(qv.y), a8[2]); a8[3] = fmaf(dsp, bf16_hi(qv.y), a8[3]);
-                    a8[4] = fmaf(dsp, bf16_lo(qv.z), a8[4]); a8[5] = fmaf(dsp, bf16_hi(qv.z), a8[5]);
-                    a8[6] = fmaf(dsp, bf16_lo(qv.w), a8[6]); a8[7] = fmaf(dsp, bf16_hi(qv.w), a8[7]);
-                }
-#pragma unroll
-                for (int k = 0; k < 8; ++k) a8[k] += __shfl_xor_sync(0xffffffffu, a8[k], 16);  // same cc
-                if (lane < 16) {  // this warp's own partial row: no other thread touches these 8 entries
-                    float4 *dst = reinterpret_cast<float4 *>(s_dl + warp * D + 8 * cc);
-                    const float4 x0 = dst[0], x1 = dst[1];
-                    dst[0] = make_float4(x0.x + a8[0], x0.y + a8[1], x0.z + a8[2], x0.w + a8[3]);
-                    dst[1] = make_float4(x1.x + a8[4], x1.y + a8[5], x1.z + a8[6], x1.w + a8[7]);
-                }
-            }
             tc::mbar_arrive(bar(kBDsFull));
             tc::mbar_arrive(bar(kBEReady + slot));
-            if (cur.last_tile()) {  // the unit's dL (the epilogue warps add its dK and dV)
-                const int bh = cur.u.chunk / N, c = cur.u.chunk % N;
-                asm volatile("bar.sync 1, 128;" ::: "memory");  // every warp's dL partials are in s_dl
-                atomicAdd(dL + ((size_t)bh * N + c) * D + r,
-                          scale * ((s_dl[r] + s_dl[D + r]) + (s_dl[2 * D + r] + s_dl[3 * D + r])));
-                asm volatile("bar.sync 1, 128;" ::: "memory");  // all reads done before the reset
-                s_dl[r] = s_dl[D + r] = s_dl[2 * D + r] = s_dl[3 * D + r] = 0.0f;
-            }
         }
     } else {
         // ================= dQ epilogue: warpgroup e takes columns [64 e, 64 e + 64) =================

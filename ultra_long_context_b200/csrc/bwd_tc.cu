@@ -55,8 +55,8 @@ struct BtSmem {  // head dim 128
     static constexpr uint32_t ROW = OUT + 8 * 32 * OUT_ROW;  // int[2][128]: token rows of a stage
     static constexpr uint32_t W = ROW + 1024;          // float[2][128]: fusion weights
     static constexpr uint32_t DEL = W + 1024;          // float[2][128]: delta of the pair's token
-    static constexpr uint32_t LROW = DEL + 1024;       // float[2][128]: the unit's landmark row (fp32)
-    static constexpr uint32_t EROW = LROW + 1024;      // int[4][128]: token rows for the dQ epilogue
+    static constexpr uint32_t LROW = DEL + 1024;       // float[4][128]: a unit's landmark row (fp32), slot k % 4
+    static constexpr uint32_t EROW = LROW + 2048;      // int[4][128]: token rows for the dQ epilogue
     static constexpr uint32_t EDS = EROW + 2048;       // float[4][128]: ds (dQ epilogue and dL)
     static constexpr uint32_t SDL = EDS + 2048;        // float[4][128]: the unit's dL per compute warp
     static constexpr uint32_t BAR = SDL + 2048;
@@ -231,28 +231,12 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
         for (; !cur.done() && ok; cur.next()) {
             const int j = cur.j, st = j & 1;
             const int bh = cur.u.chunk / N, c = cur.u.chunk % N;
-            if (cur.first_tile()) {
-                // every loader thread waits: the landmark row written below is read by the dQ epilogue
-                // of the unit two back, which kv_empty of the previous unit orders before this point
-                ok = tc::mbar_wait(bar(kBKvEmpty), ((uint32_t)cur.k & 1u) ^ 1u);
-                if (ok && lt == 0) {  // the unit's K and V
-                    tc::mbar_arrive_expect_tx(bar(kBKvFull), 4 * SM::KH);
-                    const int y = bh * T + c * kChunk;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        tc::tma_load_2d(sb + SM::KO + h * SM::KH, &tmK, h * 64, y, bar(kBKvFull));
-                        tc::tma_load_2d(sb + SM::VO + h * SM::KH, &tmV, h * 64, y, bar(kBKvFull));
-                    }
-                }
-            }
             if (j >= 2) do_dl();  // the stage about to be reloaded holds tile j - 2
             ok = ok && tc::mbar_wait(bar(kBQdEmpty + st), ((uint32_t)(j >> 1) & 1u) ^ 1u);
             if (!ok) break;
             s_row[st * 128 + myr] = myrow;
             s_w[st * 128 + myr] = myw;
             s_del[st * 128 + myr] = mydel;
-            if (cur.first_tile())  // the unit's landmark row, fp32, for the ds L_c term of dQ
-                s_L[(cur.k & 1) * 128 + myr] = __uint_as_float((uint32_t)L[((size_t)bh * N + c) * D + myr] << 16);
             const uint32_t sq = sb + SM::STG + st * SM::QD;
 #pragma unroll
             for (int k = 0; k < ITER; ++k) {  // padding rows (token -1) are zero-filled
@@ -266,6 +250,29 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                                src >= 0 ? 16 : 0);
             }
             cp_async_commit();
+            if (cur.first_tile() && lt == 0) {
+                // the unit's K and V, once the previous unit's last MMA is done with them (the Q / dO
+                // copies of this tile are already in flight); the next unit's tiles are prefetched to L2
+                ok = tc::mbar_wait(bar(kBKvEmpty), ((uint32_t)cur.k & 1u) ^ 1u);
+                if (ok) {
+                    tc::mbar_arrive_expect_tx(bar(kBKvFull), 4 * SM::KH);
+                    const int y = bh * T + c * kChunk;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        tc::tma_load_2d(sb + SM::KO + h * SM::KH, &tmK, h * 64, y, bar(kBKvFull));
+                        tc::tma_load_2d(sb + SM::VO + h * SM::KH, &tmV, h * 64, y, bar(kBKvFull));
+                    }
+                    if (cur.k + 1 < mine) {
+                        const PairTile nu = units[blockIdx.x + (size_t)(cur.k + 1) * G];
+                        const int yn = (nu.chunk / N) * T + (nu.chunk % N) * kChunk;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            tc::tma_prefetch_2d(&tmK, h * 64, yn);
+                            tc::tma_prefetch_2d(&tmV, h * 64, yn);
+                        }
+                    }
+                }
+            }
             {  // the next tile's metadata while the copies run
                 BtCursor nx = cur;
                 nx.next();
@@ -363,6 +370,13 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             tc::fence_after();
             const int row = s_row[b * 128 + r];
             const float w = s_w[b * 128 + r], del = s_del[b * 128 + r];
+            if (cur.first_tile()) {
+                // the unit's landmark row (fp32) for the ds L_c term of dQ, slot k % 4: the dQ epilogue
+                // of unit k - 4 is done with that slot, since this tile's S needed unit k - 1's last
+                // MMA, which needed the epilogue of a tile after unit k - 4's last
+                const int bhu = cur.u.chunk / N, cu = cur.u.chunk % N;
+                s_L[(cur.k & 3) * 128 + r] = __uint_as_float((uint32_t)L[((size_t)bhu * N + cu) * D + r] << 16);
+            }
             const uint32_t tS = tmem + lane_off + SM::S_COL;
             const uint32_t tDP = tmem + lane_off + SM::DP_COL;
             {  // P = softmax over the chunk's 64 keys (fp32), written back over S
@@ -449,7 +463,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             tc::fence_after();
             const int row = e_row[slot * 128 + r];
             const float ds = e_ds[slot * 128 + r];
-            const float *Lr = s_L + (cur.k & 1) * 128;
+            const float *Lr = s_L + (cur.k & 3) * 128;  // published with e_ready
 #pragma unroll 1
             for (int cb = 0; cb < 64 / (int)SM::SLAB; ++cb) {
                 const int col0 = 64 * e + cb * (int)SM::SLAB;

@@ -249,6 +249,11 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int 
         "l"(tmap), "r"(x), "r"(y), "r"(mbar)
         : "memory");
 }
+// Prefetch a 2D tile of a tensor map into L2 (no shared memory, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_2d(const void *tmap, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(tmap), "r"(x), "r"(y)
+                 : "memory");
+}
 // Four rows y0..y3 (tensor map with a one-row box) at column x, written as four consecutive box rows.
 __device__ __forceinline__ void tma_gather4(uint32_t dst, const void *tmap, int x, int y0, int y1, int y2, int y3,
                                             uint32_t mbar) {

@@ -170,6 +170,7 @@ TRAFFIC_BYTES = {
     # captured on a 4M-token cache (134.3 MB of landmarks read per scan); the scan's traffic grows in
     # proportion to the landmarks, so the 16M-token figure is four times that capture
     ("decode_16m_b1_h8_d128_k32", "decode_scan"): 4 * (134_288_640 + 718_080),
+    ("fwdbwd_t64k_h8_d128_k16", "chunk_bwd"): 2_291_017_000 + 1_258_746_000,
 }
 # fp32 reductions into L2-resident rows, 4 rows x 128 B per red.global.add.v4.f32, 16-24 warps per SM:
 # the ceiling measured on this GPU type for the combine of the chunk attention (GB/s)
@@ -432,7 +433,7 @@ def main():
             "workload": wb.name, "tokens_per_s": round(wb.B * wb.T / (bms / 1e3), 1), "ms_per_step": round(bms, 4),
             "steps": bsteps,
             "roofline": roofline_entry("chunk_bwd", prof_b, bwd_flops, "TFLOP/s", tensor_peak, "tensor",
-                                       f"{peak_kind} bf16_tflops_sustained"),
+                                       f"{peak_kind} bf16_tflops_sustained", TRAFFIC_BYTES.get((wb.name, "chunk_bwd"))),
             "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_b.items()},
         }
         del bQ, bK, bV, bL, bdO, fws, bws, grads

@@ -36,6 +36,10 @@
  *   - Scratch memory is caller-provided: query its size with the matching *_workspace_size
  *     function and pass at least that many bytes, 256-byte aligned. The library allocates no
  *     device memory. Workspace contents on entry are irrelevant; they are clobbered.
+ *   - Every device-side wait of the kernels is bounded. A wait that runs out (a stalled pipeline:
+ *     never expected, but possible on a faulty device) sets a status flag that lives in the first
+ *     bytes of the call's workspace and lets the kernel unwind; the call itself has already
+ *     returned (calls are asynchronous). hsa_workspace_status() reads that flag.
  *   - Supported now: D in {64, 128}, chunk == 64. Forward/backward: 1 <= topk <= 32;
  *     decode: 1 <= topk <= 64. Anything else returns HSA_ERR_UNSUPPORTED.
  *   - Every output element is written (including padding and all-zero rows).
@@ -60,11 +64,18 @@ typedef enum {
     HSA_ERR_UNSUPPORTED = -2, /* valid HSA call outside what the kernels implement (D, chunk, topk) */
     HSA_ERR_WORKSPACE = -3,   /* workspace missing, misaligned or smaller than *_workspace_size */
     HSA_ERR_CUDA = -4,        /* a CUDA runtime call failed; hsa_last_error() holds its text */
-    HSA_ERR_TIMEOUT = -5      /* reserved for bounded device-side waits */
+    HSA_ERR_TIMEOUT = -5      /* a bounded device-side wait ran out (see hsa_workspace_status) */
 } hsa_status;
 
 /* Message describing the last non-OK status returned on the calling thread ("" if none). */
 const char *hsa_last_error(void);
+
+/* Device-side status of the last hsa_forward / hsa_backward / hsa_decode call that used `workspace`
+ * (the pointer passed to that call). Synchronizes `stream` (cudaStream_t, NULL = legacy default
+ * stream), then reads the flag stored in the first 4 bytes of the workspace.
+ * Returns HSA_OK, HSA_ERR_TIMEOUT if a bounded device wait of that call ran out (its outputs are
+ * then unspecified), HSA_ERR_INVALID_ARG for a NULL workspace, or HSA_ERR_CUDA. */
+hsa_status hsa_workspace_status(const void *workspace, void *stream);
 
 /* ---------------------------------------------------------------------------------------------
  * Prefill forward (Steps 1-4 for every token of a sequence).

@@ -94,3 +94,9 @@ def test_backward_rejects_invalid_calls_on_host(kw, status):
 def test_binding_raises_with_message():
     with pytest.raises(hsa.HSAError, match="HSA_ERR_UNSUPPORTED"):
         hsa._check("hsa_forward", _fwd(D=96))
+
+
+def test_workspace_status_rejects_null_on_host():
+    """hsa_workspace_status validates its argument before touching the device."""
+    assert hsa.lib().hsa_workspace_status(None, None) == -1
+    assert "workspace" in hsa.hsa_last_error()

@@ -224,3 +224,21 @@ def test_backward_full_size_properties():
             assert torch.all(dL[b, h][~hit] == 0)
             assert torch.all(dK[b, h].reshape(N, 64 * D)[~hit] == 0)
             assert torch.all(dV[b, h].reshape(N, 64 * D)[~hit] == 0)
+
+
+def test_workspace_status_clear_after_calls():
+    """A completed forward, backward and decode leave the device status flag of their workspace clear
+    (every bounded wait was satisfied)."""
+    B, H, T, D, topk = 1, 2, 1100, 128, 8
+    Q, K, V, L = inputs.forward_inputs(B, H, T, D, 21, device=DEV)
+    ws = torch.empty(hsa.hsa_forward_workspace_size(B, H, T, D, 64, topk), dtype=torch.uint8, device=DEV)
+    out, idx, sw = hsa.hsa_forward(Q, K, V, L, topk, workspace=ws)
+    hsa.hsa_workspace_status(ws)
+    dO = inputs.upstream_grad(B, H, T, D, 21, device=DEV)
+    wsb = torch.empty(hsa.hsa_backward_workspace_size(B, H, T, D, 64, topk), dtype=torch.uint8, device=DEV)
+    hsa.hsa_backward(Q, K, V, L, out, dO, idx, sw, workspace=wsb)
+    hsa.hsa_workspace_status(wsb)
+    q, Kc, Vc, Lc, lens_t, _ = inputs.decode_inputs(2, 2, [5000, 777], D, seed=22, Tmax=5056, device=DEV)
+    wsd = torch.empty(hsa.hsa_decode_workspace_size(2, 2, 5056, D, 64, topk), dtype=torch.uint8, device=DEV)
+    hsa.hsa_decode(q, Kc, Vc, Lc, lens_t, topk, workspace=wsd)
+    hsa.hsa_workspace_status(wsd)

@@ -84,6 +84,7 @@ struct FwdLayout {
 FwdLayout fwd_layout(void *ws, int B, int H, int T, int D, int topk, bool backward) {
     FwdLayout l{};
     Carver c{static_cast<char *>(ws)};
+    l.err = c.take<int32_t>(1);  // first: hsa_workspace_status reads it at offset 0
     const size_t rows = (size_t)B * H * T, chunks = (size_t)B * H * (T / 64), pairs = rows * topk;
     l.max_tiles = (int)hsa::forward_max_tiles(B, H, T, topk);
     l.o_acc = backward ? nullptr : c.take<float>(rows * D);
@@ -97,7 +98,6 @@ FwdLayout fwd_layout(void *ws, int B, int H, int T, int D, int topk, bool backwa
     l.pair_w = c.take<float>(pairs);
     l.tiles = c.take<hsa::PairTile>((size_t)l.max_tiles);
     l.num_tiles = c.take<int32_t>(1);
-    l.err = c.take<int32_t>(1);
     l.delta = backward ? c.take<float>(rows) : nullptr;
     l.pair_slot = backward ? c.take<int32_t>(pairs) : nullptr;
     l.bytes = c.used;
@@ -105,6 +105,7 @@ FwdLayout fwd_layout(void *ws, int B, int H, int T, int D, int topk, bool backwa
 }
 
 struct DecLayout {
+    int32_t *err;
     uint64_t *cand;
     unsigned *counters;
     int32_t *sel_idx;
@@ -119,6 +120,7 @@ DecLayout dec_layout(void *ws, int B, int H, int64_t Tmax, int D, int topk) {
     const int split = hsa::decode_split_size(Nmax, topk, B * H);
     const int64_t nsplit = Nmax > 0 ? (Nmax + split - 1) / split : 1;
     const size_t BH = (size_t)B * H;
+    l.err = c.take<int32_t>(1);  // first: hsa_workspace_status reads it at offset 0
     l.cand = c.take<uint64_t>(BH * nsplit * topk);
     l.counters = c.take<unsigned>(2 * BH);
     l.sel_idx = c.take<int32_t>(BH * topk);
@@ -140,6 +142,20 @@ void set_last_error(const char *msg) { g_last_error = msg ? msg : ""; }
 extern "C" {
 
 const char *hsa_last_error(void) { return g_last_error.c_str(); }
+
+hsa_status hsa_workspace_status(const void *workspace, void *stream) {
+    g_last_error.clear();
+    if (!workspace) return fail(HSA_ERR_INVALID_ARG, "workspace must not be NULL");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(s);
+    int32_t flag = 0;
+    if (e == cudaSuccess) e = cudaMemcpy(&flag, workspace, sizeof(flag), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e, "hsa_workspace_status");
+    if (flag != 0)
+        return fail(HSA_ERR_TIMEOUT, "a bounded device-side wait ran out in the last call on this workspace (flag %d)",
+                    (int)flag);
+    return HSA_OK;
+}
 
 size_t hsa_forward_workspace_size(int B, int H, int T, int D, int chunk, int topk) {
     (void)chunk;
@@ -223,6 +239,10 @@ hsa_status hsa_decode(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
     a.sel_idx = sel_idx ? sel_idx : l.sel_idx;
     a.sel_w = sel_w ? sel_w : l.sel_w;
     a.cand = l.cand; a.counters = l.counters; a.partial = l.partial;
+    // the decode kernels never wait on one another; the flag is cleared so that a status query
+    // after this call reports this call
+    cudaError_t ce = cudaMemsetAsync(l.err, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
+    if (ce != cudaSuccess) return cuda_status(ce, "hsa_decode");
     return cuda_status(hsa::launch_decode(a, static_cast<cudaStream_t>(stream)), "hsa_decode");
 }
 

@@ -22,6 +22,7 @@ STATUS_NAMES = {0: "HSA_OK", -1: "HSA_ERR_INVALID_ARG", -2: "HSA_ERR_UNSUPPORTED
 _P, _I, _I64, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "hsa_last_error": ([], ctypes.c_char_p),
+    "hsa_workspace_status": ([_P, _P], _I),
     "hsa_forward_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
     "hsa_forward": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P], _I),
     "hsa_decode_workspace_size": ([_I, _I, _I64, _I, _I, _I], _SZ),
@@ -66,6 +67,14 @@ def hsa_last_error():
 def _check(name, status):
     if status != HSA_OK:
         raise HSAError(name, status, hsa_last_error())
+
+
+def hsa_workspace_status(workspace, stream=None):
+    """Device-side status of the last call that used ``workspace`` (a uint8 CUDA tensor): synchronizes
+    the stream and raises HSAError (HSA_ERR_TIMEOUT) if a bounded device wait of that call ran out."""
+    if not (isinstance(workspace, torch.Tensor) and workspace.is_cuda):
+        raise ValueError("workspace must be a CUDA tensor")
+    _check("hsa_workspace_status", lib().hsa_workspace_status(_ptr(workspace), _stream(workspace.device, stream)))
 
 
 def _ptr(t):

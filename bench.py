@@ -106,26 +106,37 @@ def dist_setup(args):
     return world, rank, local
 
 
-def barrier(world):
+def barrier(world, cuda=True):
+    """All ranks meet (when there are several), then this rank's device work is drained."""
     import torch
 
     if world > 1:
         import torch.distributed as dist
 
         dist.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(x, world):
+    """The largest x over all ranks (the slowest rank's time); the reduction runs where the process
+    group's backend keeps its tensors (the GPU for NCCL, the CPU for gloo)."""
     import torch
 
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms_per_step):
+    """Throughput of the whole job: every rank processes units_per_rank per step, and a step lasts as
+    long as the slowest rank's (ms_per_step, already the max over ranks)."""
+    return world * units_per_rank / (ms_per_step / 1e3)
 
 
 def timed(fn, steps, warmup, world):
@@ -327,7 +338,7 @@ def main():
         ms = timed(fwd, args.steps, args.warmup, world)
         ms_per_step = ms / args.steps
         tokens = w.B * w.T
-        value = world * tokens / (ms_per_step / 1e3)
+        value = whole_job_rate(tokens, world, ms_per_step)
         prof_fwd = kernel_profile(fwd, args.steps)
         score_flops, attn_flops, pairs = forward_work(w, sel_idx)
         tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
@@ -361,7 +372,7 @@ def main():
         e2e_ms = timed(e2e_step, args.steps, args.warmup, world) / args.steps
         h2d = sum(x.numel() * x.element_size() for x in (hQ, hK, hV, hL))
         d2h = hout.numel() * hout.element_size()
-        e2e = {"value": world * tokens / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": whole_job_rate(tokens, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)}
         del hQ, hK, hV, hL, hout, dQ_, dK_, dV_, dL_
 

@@ -74,7 +74,51 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
         }
     }
     __syncthreads();
-    const int cnt = block_topk_u64(keys, nloc, K, topk, hist, misc);
+    // Exact pre-filter before the selection: the first S0 = K * G keys form K groups of G; the smallest
+    // of the K group maxima, tau, has at least K keys of the range at or above it, so no key below tau
+    // can be in the range's top K. The keys >= tau are compacted in place (in rounds that are read
+    // whole before any of their slots is written), and the radix selection runs over those only.
+    constexpr int G = 32;
+    const int S0 = K * G;
+    int nkeys = nloc;
+    if (nloc >= 2 * S0) {
+        unsigned long long *tau_s = reinterpret_cast<unsigned long long *>(topk);  // scratch until selection
+        if (tid == 0) {
+            *tau_s = ~0ull;
+            misc[5] = 0;
+        }
+        __syncthreads();
+        if (tid < K) {
+            uint64_t m = 0;
+            for (int i = 0; i < G; ++i) m = max(m, keys[tid * G + i]);
+            atomicMin(tau_s, (unsigned long long)m);
+        }
+        __syncthreads();
+        const uint64_t tau = *tau_s;
+        constexpr int PER = 4, ROUND = PER * kDecodeThreads;
+        for (int r0 = 0; r0 < nloc; r0 += ROUND) {
+            uint64_t mine[PER];
+#pragma unroll
+            for (int r = 0; r < PER; ++r) {
+                const int i = r0 + r * kDecodeThreads + tid;
+                mine[r] = i < nloc ? keys[i] : 0ull;
+            }
+            __syncthreads();  // the round is read whole; kept slots never pass its end
+#pragma unroll
+            for (int r = 0; r < PER; ++r) {
+                const bool keep = mine[r] != 0ull && mine[r] >= tau;
+                const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                int pos0 = 0;
+                if (lane == 0 && bal) pos0 = atomicAdd(&misc[5], __popc(bal));
+                pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+                if (keep) keys[pos0 + __popc(bal & ((1u << lane) - 1u))] = mine[r];
+            }
+            __syncthreads();
+        }
+        nkeys = misc[5];
+        __syncthreads();
+    }
+    const int cnt = block_topk_u64(keys, nkeys, K, topk, hist, misc);
     uint64_t *my_cand = cand + ((size_t)bh * nsplit + sp) * K;
     for (int j = tid; j < K; j += kDecodeThreads) my_cand[j] = j < cnt ? topk[j] : 0ull;
 

@@ -20,6 +20,39 @@ namespace hsa {
 
 constexpr int kDecodeThreads = 256;
 
+// Compacts, in place and in order-free fashion, the keys[0..n) that are >= tau to the front; returns
+// their number. Rounds of 4 x blockDim keys are read whole before any slot is written, and the kept
+// count never passes the end of what has been read, so no unread key is overwritten. Uses misc[5].
+__device__ inline int compact_at_least(uint64_t *keys, int n, uint64_t tau, int *misc) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    if (tid == 0) misc[5] = 0;
+    __syncthreads();
+    constexpr int PER = 4;
+    const int round = PER * (int)blockDim.x;
+    for (int r0 = 0; r0 < n; r0 += round) {
+        uint64_t mine[PER];
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const int i = r0 + r * (int)blockDim.x + tid;
+            mine[r] = i < n ? keys[i] : 0ull;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < PER; ++r) {
+            const bool keep = mine[r] != 0ull && mine[r] >= tau;
+            const unsigned bal = __ballot_sync(0xffffffffu, keep);
+            int pos0 = 0;
+            if (lane == 0 && bal) pos0 = atomicAdd(&misc[5], __popc(bal));
+            pos0 = __shfl_sync(0xffffffffu, pos0, 0);
+            if (keep) keys[pos0 + __popc(bal & ((1u << lane) - 1u))] = mine[r];
+        }
+        __syncthreads();
+    }
+    const int kept = misc[5];
+    __syncthreads();
+    return kept;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ Lc, const int64_t *__restrict__ cache_len, int H,
@@ -39,6 +72,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
     uint32_t *hist = reinterpret_cast<uint32_t *>(sorted + 64);
     int *misc = reinterpret_cast<int *>(hist + 256);  // 8 ints
 
+    // the attend kernel may be scheduled now: it waits (griddepcontrol.wait) for this grid to complete
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int sp = blockIdx.x, bh = blockIdx.y, b = bh / H;
     int64_t nb = cache_len[b] / kChunk;
@@ -83,10 +118,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
     int nkeys = nloc;
     if (nloc >= 2 * S0) {
         unsigned long long *tau_s = reinterpret_cast<unsigned long long *>(topk);  // scratch until selection
-        if (tid == 0) {
-            *tau_s = ~0ull;
-            misc[5] = 0;
-        }
+        if (tid == 0) *tau_s = ~0ull;
         __syncthreads();
         if (tid < K) {
             uint64_t m = 0;
@@ -95,28 +127,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
         }
         __syncthreads();
         const uint64_t tau = *tau_s;
-        constexpr int PER = 4, ROUND = PER * kDecodeThreads;
-        for (int r0 = 0; r0 < nloc; r0 += ROUND) {
-            uint64_t mine[PER];
-#pragma unroll
-            for (int r = 0; r < PER; ++r) {
-                const int i = r0 + r * kDecodeThreads + tid;
-                mine[r] = i < nloc ? keys[i] : 0ull;
-            }
-            __syncthreads();  // the round is read whole; kept slots never pass its end
-#pragma unroll
-            for (int r = 0; r < PER; ++r) {
-                const bool keep = mine[r] != 0ull && mine[r] >= tau;
-                const unsigned bal = __ballot_sync(0xffffffffu, keep);
-                int pos0 = 0;
-                if (lane == 0 && bal) pos0 = atomicAdd(&misc[5], __popc(bal));
-                pos0 = __shfl_sync(0xffffffffu, pos0, 0);
-                if (keep) keys[pos0 + __popc(bal & ((1u << lane) - 1u))] = mine[r];
-            }
-            __syncthreads();
-        }
-        nkeys = misc[5];
-        __syncthreads();
+        nkeys = compact_at_least(keys, nloc, tau, misc);
     }
     const int cnt = block_topk_u64(keys, nkeys, K, topk, hist, misc);
     uint64_t *my_cand = cand + ((size_t)bh * nsplit + sp) * K;
@@ -134,7 +145,22 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
     for (int i = tid; i < ncand; i += kDecodeThreads)
         keys[i] = __ldcg(reinterpret_cast<const unsigned long long *>(all) + i);
     __syncthreads();
-    const int m = block_topk_u64(keys, ncand, K, topk, hist, misc);
+    // Each range contributed its top K; the largest of the ranges' K-th keys has at least K
+    // candidates at or above it (that range's), so candidates below it cannot be in the top K.
+    int nmerge = ncand;
+    if (nsplit > 2) {
+        unsigned long long *tau_s = reinterpret_cast<unsigned long long *>(topk);  // scratch until selection
+        if (tid == 0) *tau_s = 0ull;
+        __syncthreads();
+        for (int r = tid; r < nsplit; r += kDecodeThreads) {
+            uint64_t mn = ~0ull;
+            for (int i = 0; i < K; ++i) mn = min(mn, keys[r * K + i]);  // 0 (empty) if the range had < K
+            atomicMax(tau_s, (unsigned long long)mn);
+        }
+        __syncthreads();
+        nmerge = compact_at_least(keys, ncand, *tau_s, misc);
+    }
+    const int m = block_topk_u64(keys, nmerge, K, topk, hist, misc);
     block_sort_desc_small(topk, m, sorted);  // empty (0) keys sort last
     if (warp == 0) {
         // fusion weights (Step 4): softmax over the kept scores, fp32, max-subtracted
@@ -167,6 +193,9 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
     __shared__ int s_last;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int j = blockIdx.x, bh = blockIdx.y;
+    // launched early (programmatic dependent launch): wait until the scan grid has completed and its
+    // selection is visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int c = sel_idx[(size_t)bh * K + j];
     float *my_part = partial + ((size_t)bh * K + j) * D;
     if (c >= 0) {
@@ -270,6 +299,25 @@ size_t decode_scan_smem(int split, int nsplit, int K) {
     return (cap + 128) * sizeof(uint64_t) + 256 * sizeof(uint32_t) + 8 * sizeof(int);
 }
 
+// The attend kernel is launched as a programmatic dependent of the scan, so that its launch overlaps
+// the scan's tail; it waits for the scan grid's completion before reading the selection.
+template <int D>
+static cudaError_t launch_attend(const DecodeArgs &a, dim3 grid, cudaStream_t s) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kDecodeThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_attend_kernel<D>, a.q, a.Kc, a.Vc, a.Tmax, a.K, a.scale,
+                              (const int32_t *)a.sel_idx, (const float *)a.sel_w, a.partial, a.counters + a.B * a.H,
+                              a.out);
+}
+
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
     const int split = decode_split_size(a.Nmax, a.K, a.B * a.H);
     const int nsplit = (int)((a.Nmax + split - 1) / split) > 0 ? (int)((a.Nmax + split - 1) / split) : 1;
@@ -292,8 +340,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
                                                                      a.sel_idx, a.sel_w);
         }
         HSA_PROF("decode_attend", s);
-        decode_attend_kernel<128><<<g2, kDecodeThreads, 0, s>>>(a.q, a.Kc, a.Vc, a.Tmax, a.K, a.scale, a.sel_idx,
-                                                                a.sel_w, a.partial, a.counters + BH, a.out);
+        e = launch_attend<128>(a, g2, s);
     } else {
         e = cudaFuncSetAttribute(decode_scan_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
@@ -304,9 +351,9 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
                                                                     a.sel_idx, a.sel_w);
         }
         HSA_PROF("decode_attend", s);
-        decode_attend_kernel<64><<<g2, kDecodeThreads, 0, s>>>(a.q, a.Kc, a.Vc, a.Tmax, a.K, a.scale, a.sel_idx,
-                                                               a.sel_w, a.partial, a.counters + BH, a.out);
+        e = launch_attend<64>(a, g2, s);
     }
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -51,6 +51,8 @@ def run_forward_case(oracle_mod, B, H, T, D, topk, seed, landmarks="iid", rows=N
     (1, 2, 1024, 128, 1, "iid"),
     (1, 2, 2048 + 64, 64, 32, "iid"),
     (1, 1, 64 * 40 + 63, 128, 3, "chunk_mean"),
+    (1, 2, 2048 + 64, 128, 32, "chunk_mean"),  # the 32-wide selection list at head dim 128
+    (1, 1, 3000, 128, 24, "iid"),              # kout below the list length, ragged tail
 ])
 def test_forward_matches_oracle(oracle_mod, B, H, T, D, topk, landmarks):
     stats, _ = run_forward_case(oracle_mod, B, H, T, D, topk, seed=100 + T + topk, landmarks=landmarks)
@@ -180,7 +182,9 @@ def test_decode_full_size(oracle_mod, name):
 # backward
 
 
-@pytest.mark.parametrize("B,H,T,D,topk", [(1, 2, 1100, 64, 8), (1, 1, 2048 + 64, 128, 16), (2, 1, 700, 128, 5)])
+@pytest.mark.parametrize("B,H,T,D,topk", [(1, 2, 1100, 64, 8), (1, 1, 2048 + 64, 128, 16), (2, 1, 700, 128, 5),
+                                           # chunks with thousands of pairs: several work units each
+                                           (1, 2, 8192 + 81, 128, 16)])
 def test_backward_matches_oracle(oracle_mod, B, H, T, D, topk):
     Q, K, V, L = inputs.forward_inputs(B, H, T, D, 500 + T, device=DEV)
     dO = inputs.upstream_grad(B, H, T, D, 500 + T, device=DEV)

@@ -27,7 +27,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_FORWARD = 7     # score_topk, count, scan, tile list, scatter, chunk_attn, finalize
+KERNELS_PER_FORWARD = 6     # score_topk (with the chunk counts), scan, tile list, scatter, chunk_attn, finalize
 KERNELS_PER_DECODE = 2      # decode_scan, decode_attend
 KERNELS_PER_BACKWARD = 6    # delta, count, scan, tile list, scatter, chunk_bwd
 

@@ -311,7 +311,7 @@ cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
     const bool tc = a.D == 128;
     e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.tile_off,
                         a.chunk_cursor, a.pair_row, a.pair_w, a.pair_slot, a.tiles, a.num_tiles, a.max_tiles,
-                        tc ? kBwdUnitPairs : kPairTile, s);
+                        tc ? kBwdUnitPairs : kPairTile, false, s);
     if (e != cudaSuccess) return e;
     if (tc) return launch_backward_tc(a, s);
     if (a.D == 128) {

@@ -67,7 +67,7 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
                             int32_t *chunk_count, int32_t *chunk_off, int32_t *tile_off, int32_t *chunk_cursor,
                             int32_t *pair_row,
                             float *pair_w, int32_t *pair_slot, PairTile *tiles, int32_t *num_tiles, int max_tiles,
-                            int tile_pairs, cudaStream_t s);
+                            int tile_pairs, bool counts_ready, cudaStream_t s);
 
 struct BackwardArgs {
     const uint16_t *Q, *K, *V, *L, *out, *dout;

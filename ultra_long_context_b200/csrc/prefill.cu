@@ -259,7 +259,7 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
                             int32_t *chunk_count, int32_t *chunk_off, int32_t *tile_off, int32_t *chunk_cursor,
                             int32_t *pair_row,
                             float *pair_w, int32_t *pair_slot, PairTile *tiles, int32_t *num_tiles, int max_tiles,
-                            int tile_pairs, cudaStream_t s) {
+                            int tile_pairs, bool counts_ready, cudaStream_t s) {
     const int BH = B * H;
     dim3 dgrid((T + kDispatchRows - 1) / kDispatchRows, BH);
     const size_t hsmem = N <= kSmemHistMax ? (size_t)N * sizeof(int) : 0;
@@ -267,7 +267,7 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
         cudaError_t e = cudaFuncSetAttribute(count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hsmem);
         if (e != cudaSuccess) return e;
     }
-    {
+    if (!counts_ready) {  // the forward's score kernel has counted them already
         HSA_PROF("dispatch_count", s);
         count_kernel<<<dgrid, kDispatchRows, hsmem, s>>>(sel_idx, T, N, topk, chunk_count);
     }
@@ -307,8 +307,8 @@ cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s) {
     cudaError_t e;
     {
         HSA_PROF("memset", s);
-        e = cudaMemsetAsync(a.o_acc, 0, rows * a.D * sizeof(float), s);
-        if (e == cudaSuccess) e = cudaMemsetAsync(a.chunk_count, 0, (size_t)BH * a.N * sizeof(int32_t), s);
+        // o_acc is zeroed by the score kernel, tile by tile
+        e = cudaMemsetAsync(a.chunk_count, 0, (size_t)BH * a.N * sizeof(int32_t), s);
         if (e == cudaSuccess) e = cudaMemsetAsync(a.chunk_cursor, 0, (size_t)BH * a.N * sizeof(int32_t), s);
         if (e == cudaSuccess) e = cudaMemsetAsync(a.err, 0, sizeof(int32_t), s);
     }
@@ -322,7 +322,7 @@ cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s) {
         return cudaGetLastError();
     }
     e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.tile_off,
-                        a.chunk_cursor, a.pair_row, a.pair_w, nullptr, a.tiles, a.num_tiles, a.max_tiles, 128, s);
+                        a.chunk_cursor, a.pair_row, a.pair_w, nullptr, a.tiles, a.num_tiles, a.max_tiles, 128, true, s);
     if (e != cudaSuccess) return e;
     e = launch_attn_tc(a, s);
     if (e != cudaSuccess) return e;

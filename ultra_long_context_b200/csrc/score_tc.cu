@@ -27,6 +27,9 @@
 //     in chunk order), computes the fusion weights w = softmax over the kept values (fp32,
 //     max-subtracted), and the tile's rows, contiguous in [B, H, T, K], are written by coalesced
 //     stores through shared memory.
+//   * Two pieces of the dispatch ride along, on memory bandwidth this ALU-bound kernel leaves idle:
+//     the tile's rows of the fp32 output accumulator are zeroed, and the number of selected pairs per
+//     chunk is counted in a shared-memory histogram and added into the dispatch's chunk counts.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -43,6 +46,7 @@ constexpr int kStThreads = kStConsumers + 32;  // + producer warp
 constexpr int kStLStages = 3;                  // landmark blocks in shared memory
 constexpr uint32_t kStTmemCols = 128;          // Q (D/2 columns) + score buffers
 constexpr int kStMaxCtasPerSm = 4;             // kStTmemCols x 4 = all 512 TMEM columns
+constexpr int kStHistMax = 1024;               // chunks per (b, h) counted in shared memory
 
 template <int D, int K>
 struct StSmem {
@@ -58,7 +62,8 @@ struct StSmem {
     // the unconditional store that follows the last real entry.
     static constexpr uint32_t CV = U;
     static constexpr uint32_t CC = CV + 33 * 128 * 4;
-    static constexpr uint32_t BAR = CC + (K + 1) * 128 * 4;  // q_ready, full_l[3], empty_l[3], full_s[NB], empty_s[NB]
+    static constexpr uint32_t HIST = CC + (K + 1) * 128 * 4;  // int[kStHistMax]: selected pairs per chunk
+    static constexpr uint32_t BAR = HIST + kStHistMax * 4;  // q_ready, full_l[3], empty_l[3], full_s[NB], empty_s[NB]
     static constexpr int NBAR = 1 + 2 * kStLStages + 2 * NB;
     static constexpr uint32_t TMEM = BAR + NBAR * 8;
     static constexpr uint32_t BYTES = TMEM + 8;
@@ -72,7 +77,9 @@ template <int D, int K>
 __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_t *__restrict__ Q, int T, int N,
                                                                    float scale, int kout,
                                                                    int32_t *__restrict__ sel_idx,
-                                                                   float *__restrict__ sel_w, int32_t *__restrict__ err,
+                                                                   float *__restrict__ sel_w, float *__restrict__ o_acc,
+                                                                   int32_t *__restrict__ chunk_count,
+                                                                   int32_t *__restrict__ err,
                                                                    const __grid_constant__ CUtensorMap tmL) {
     using SM = StSmem<D, K>;
     constexpr int NB = SM::NB;
@@ -97,6 +104,10 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
     const int nblk = (n_max + kStCols - 1) / kStCols;
     const size_t out0 = ((size_t)bh * T + t0) * kout;  // the tile's rows are contiguous
 
+    {  // this tile's rows of the fp32 output accumulator start at zero (the chunk attention adds into them)
+        float4 *acc = reinterpret_cast<float4 *>(o_acc + ((size_t)bh * T + t0) * D);
+        for (int i = tid; i < nrows * (D / 4); i += kStThreads) acc[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
     if (nblk == 0) {  // no token of this tile has a complete chunk
         for (int i = tid; i < nrows * kout; i += kStThreads) {
             sel_idx[out0 + i] = -1;
@@ -104,6 +115,10 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
         }
         return;
     }
+    int *s_hist = reinterpret_cast<int *>(s + SM::HIST);  // pairs per chunk of this tile (n_max <= N)
+    const bool hist_smem = n_max <= kStHistMax;
+    if (hist_smem)
+        for (int i = tid; i < n_max; i += kStThreads) s_hist[i] = 0;  // ordered by the __syncthreads below
 
     if (warp == 0) tc::tmem_alloc(sb + SM::TMEM, kStTmemCols);
     if (tid == kStConsumers) {
@@ -287,6 +302,8 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
                 used |= 1ull << slot;
                 st_idx[tid * kout + slot] = cc[128 * k];
                 st_w[tid * kout + slot] = expf(x - top) * rz;
+                if (hist_smem) atomicAdd(&s_hist[cc[128 * k]], 1);
+                else atomicAdd(&chunk_count[(size_t)bh * N + cc[128 * k]], 1);
             }
             for (int i = 0; i < kout; ++i)
                 if (!((used >> i) & 1ull)) {
@@ -299,6 +316,9 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
             sel_idx[out0 + i] = st_idx[i];
             sel_w[out0 + i] = st_w[i];
         }
+        if (hist_smem)  // the tile's per-chunk counts into the dispatch's histogram
+            for (int i = tid; i < n_max; i += kStConsumers)
+                if (s_hist[i]) atomicAdd(&chunk_count[(size_t)bh * N + i], s_hist[i]);
         if (!ok && lane == 0) atomicOr(err, 1);
     }
     tc::fence_before();
@@ -318,7 +338,7 @@ static cudaError_t launch_st(const ForwardArgs &a, const CUtensorMap &tl, cudaSt
     dim3 grid((a.T + kStRows - 1) / kStRows, a.B * a.H);
     HSA_PROF("score_topk", s);
     score_topk_tc_kernel<D, K><<<grid, kStThreads, smem, s>>>(a.Q, a.T, a.N, a.scale, a.topk, a.sel_idx, a.sel_w,
-                                                              a.err, tl);
+                                                              a.o_acc, a.chunk_count, a.err, tl);
     return cudaGetLastError();
 }
 

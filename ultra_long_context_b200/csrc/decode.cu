@@ -20,6 +20,32 @@ namespace hsa {
 
 constexpr int kDecodeThreads = 256;
 
+// The rank select below does O(n) dependent shared-memory compares per key: faster than the radix
+// select for a few dozen keys (the filtered merge), slower for hundreds (measured on B200).
+constexpr int kRankSelectMax = 128;
+
+// Top K of n <= 2 * blockDim keys (nonzero keys unique; 0 = empty), written to out[0..K) in descending
+// order with 0 in the slots nothing fills; returns K (the caller treats 0 as empty). A nonzero key's
+// rank is the number of keys above it, which for unique keys is its position in the descending order:
+// selection and sort in one pass, O(n) compares per key.
+__device__ inline int block_topk_rank(const uint64_t *keys, int n, int K, uint64_t *out) {
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    for (int i = tid; i < K; i += nthr) out[i] = 0ull;
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int i = tid + h * nthr;
+        if (i < n) {
+            const uint64_t k = keys[i];
+            int rank = 0;
+            for (int j = 0; j < n; ++j) rank += keys[j] > k ? 1 : 0;
+            if (k != 0ull && rank < K) out[rank] = k;
+        }
+    }
+    __syncthreads();
+    return K;
+}
+
 // Compacts, in place and in order-free fashion, the keys[0..n) that are >= tau to the front; returns
 // their number. Rounds of 4 x blockDim keys are read whole before any slot is written, and the kept
 // count never passes the end of what has been read, so no unread key is overwritten. Uses misc[5].
@@ -129,9 +155,16 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
         const uint64_t tau = *tau_s;
         nkeys = compact_at_least(keys, nloc, tau, misc);
     }
-    const int cnt = block_topk_u64(keys, nkeys, K, topk, hist, misc);
+    // the range's top K, in descending order (the merge reads each range's maximum at its head)
+    int cnt;
+    if (nkeys <= kRankSelectMax) {
+        cnt = block_topk_rank(keys, nkeys, K, sorted);
+    } else {
+        cnt = block_topk_u64(keys, nkeys, K, topk, hist, misc);
+        block_sort_desc_small(topk, cnt, sorted);
+    }
     uint64_t *my_cand = cand + ((size_t)bh * nsplit + sp) * K;
-    for (int j = tid; j < K; j += kDecodeThreads) my_cand[j] = j < cnt ? topk[j] : 0ull;
+    for (int j = tid; j < K; j += kDecodeThreads) my_cand[j] = j < cnt ? sorted[j] : 0ull;
 
     // ---- last CTA of this (b, h) merges all ranges (ticket taken after a release fence) ----
     __threadfence();
@@ -145,23 +178,34 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
     for (int i = tid; i < ncand; i += kDecodeThreads)
         keys[i] = __ldcg(reinterpret_cast<const unsigned long long *>(all) + i);
     __syncthreads();
-    // Each range contributed its top K; the largest of the ranges' K-th keys has at least K
-    // candidates at or above it (that range's), so candidates below it cannot be in the top K.
+    // Each range contributed its top K in descending order. The K-th largest of the range maxima, tau,
+    // has K ranges with a key at or above it, so no candidate below tau can be in the top K.
     int nmerge = ncand;
-    if (nsplit > 2) {
+    if (nsplit > K && nsplit <= 2 * kDecodeThreads) {
         unsigned long long *tau_s = reinterpret_cast<unsigned long long *>(topk);  // scratch until selection
-        if (tid == 0) *tau_s = 0ull;
+        if (tid == 0) *tau_s = 0ull;  // stays 0 (keep every nonzero key) if fewer than K maxima are nonzero
         __syncthreads();
-        for (int r = tid; r < nsplit; r += kDecodeThreads) {
-            uint64_t mn = ~0ull;
-            for (int i = 0; i < K; ++i) mn = min(mn, keys[r * K + i]);  // 0 (empty) if the range had < K
-            atomicMax(tau_s, (unsigned long long)mn);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int r = tid + h * kDecodeThreads;
+            if (r < nsplit) {
+                const uint64_t mr = keys[r * K];
+                int rank = 0;
+                for (int q = 0; q < nsplit; ++q) rank += keys[q * K] > mr ? 1 : 0;
+                if (rank == K - 1 && mr != 0ull) *tau_s = mr;  // unique nonzero keys: at most one range
+            }
         }
         __syncthreads();
-        nmerge = compact_at_least(keys, ncand, *tau_s, misc);
+        const uint64_t tau = *tau_s;
+        nmerge = compact_at_least(keys, ncand, tau == 0ull ? 1ull : tau, misc);
     }
-    const int m = block_topk_u64(keys, nmerge, K, topk, hist, misc);
-    block_sort_desc_small(topk, m, sorted);  // empty (0) keys sort last
+    int m;
+    if (nmerge <= kRankSelectMax) {
+        m = block_topk_rank(keys, nmerge, K, sorted);
+    } else {
+        m = block_topk_u64(keys, nmerge, K, topk, hist, misc);
+        block_sort_desc_small(topk, m, sorted);  // empty (0) keys sort last
+    }
     if (warp == 0) {
         // fusion weights (Step 4): softmax over the kept scores, fp32, max-subtracted
         const uint64_t k0 = lane < m ? sorted[lane] : 0ull;

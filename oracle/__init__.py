@@ -30,16 +30,16 @@ def _load():
     global _lib
     if _lib is None:
         lib = ctypes.CDLL(_build.build())
-        lib.hsa_oracle_forward_rows.argtypes = [_f32p, _f32p, _f32p, _f32p, _i64, _i64, _i64, _i64, _i64, _i64,
+        lib.hsa_oracle_forward_rows.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _i64, _i64, _i64, _i64, _i64, _i64,
                                                 ctypes.c_double, _i64, _i64p, _f64p, _i32p, _f64p, _f64p, _f64p]
         lib.hsa_oracle_scores_rows.argtypes = [_f32p, _f32p, _i64, _i64, _i64, _i64, _i64, ctypes.c_double, _i64,
                                                _i64p, _f64p]
         lib.hsa_oracle_decode_select.argtypes = [_f32p, _f32p, _i64p, _i64, _i64, _i64, _i64, _i64, _i64,
                                                  ctypes.c_double, _i32p, _f64p, _f64p, _f64p]
-        lib.hsa_oracle_attend_gathered.argtypes = [_f32p, _f32p, _f32p, _f32p, _i32p, _i64, _i64, _i64, _i64,
+        lib.hsa_oracle_attend_gathered.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _i32p, _i64, _i64, _i64, _i64,
                                                    ctypes.c_double, _f64p, _f64p]
-        lib.hsa_oracle_backward.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _i32p, _i64, _i64, _i64, _i64, _i64,
-                                            _i64, ctypes.c_double, _f64p, _f64p, _f64p, _f64p]
+        lib.hsa_oracle_backward.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _i32p, _i64, _i64, _i64, _i64,
+                                            _i64, _i64, ctypes.c_double, _f64p, _f64p, _f64p, _f64p, _f64p]
         for f in (lib.hsa_oracle_forward_rows, lib.hsa_oracle_scores_rows, lib.hsa_oracle_decode_select,
                   lib.hsa_oracle_attend_gathered, lib.hsa_oracle_backward):
             f.restype = ctypes.c_int
@@ -65,8 +65,19 @@ def default_scale(D):
     return 1.0 / math.sqrt(D)
 
 
-def forward(Q, K, V, L, chunk=64, topk=8, scale=None, rows=None):
+def _opt_f32(a, like):
+    if a is None:
+        return None, None
+    a, p = _f32(a)
+    assert a.shape == like.shape, "the retrieval query must have the shape of the attention query"
+    return a, p
+
+
+def forward(Q, K, V, L, chunk=64, topk=8, scale=None, rows=None, Qs=None):
     """HSA forward of rows of [B, H, T, D] inputs (float arrays holding bf16-exact values).
+
+    Qs: separate retrieval queries shaped like Q (Step 2 scores Qs . L; Step 3 attends with Q), or
+    None when Q does both.
 
     Returns a dict with out [R, D] (float64), sel_idx [R, topk] (int32, -1 padding), sel_w and sel_s
     [R, topk] (float64, 0 padding) and next_s [R] (score of the best unselected chunk, -inf if none),
@@ -76,6 +87,7 @@ def forward(Q, K, V, L, chunk=64, topk=8, scale=None, rows=None):
     K, kp = _f32(K)
     V, vp = _f32(V)
     L, lp = _f32(L)
+    Qs, qsp = _opt_f32(Qs, Q)
     B, H, T, D = Q.shape
     if scale is None:
         scale = default_scale(D)
@@ -89,7 +101,7 @@ def forward(Q, K, V, L, chunk=64, topk=8, scale=None, rows=None):
     sel_w = np.zeros((R, topk), np.float64)
     sel_s = np.zeros((R, topk), np.float64)
     next_s = np.zeros((R,), np.float64)
-    rc = _load().hsa_oracle_forward_rows(qp, kp, vp, lp, B, H, T, D, chunk, topk, scale, R, _ptr(rows, _i64p),
+    rc = _load().hsa_oracle_forward_rows(qp, qsp, kp, vp, lp, B, H, T, D, chunk, topk, scale, R, _ptr(rows, _i64p),
                                          _ptr(out, _f64p), _ptr(sel_idx, _i32p), _ptr(sel_w, _f64p),
                                          _ptr(sel_s, _f64p), _ptr(next_s, _f64p))
     _check(rc, "hsa_oracle_forward_rows")
@@ -132,12 +144,14 @@ def decode_select(q, Lc, cache_len, chunk=64, topk=16, scale=None):
     return dict(sel_idx=sel_idx, sel_s=sel_s, sel_w=sel_w, next_s=next_s)
 
 
-def attend_gathered(q, Lg, Kg, Vg, nsel, scale=None):
+def attend_gathered(q, Lg, Kg, Vg, nsel, scale=None, qs=None):
     """Steps 3-4 for R rows given their selected chunks gathered.
 
     q [R, D], Lg [R, topk, D], Kg / Vg [R, topk, chunk, D], nsel [R] -> (out [R, D], sel_w [R, topk]).
+    qs [R, D]: separate retrieval queries (the fusion weights come from qs . Lg), or None.
     """
     q, qp = _f32(q)
+    qs, qsp = _opt_f32(qs, q)
     Lg, lp = _f32(Lg)
     Kg, kp = _f32(Kg)
     Vg, vp = _f32(Vg)
@@ -148,22 +162,24 @@ def attend_gathered(q, Lg, Kg, Vg, nsel, scale=None):
     ns = np.ascontiguousarray(nsel, dtype=np.int32)
     out = np.zeros((R, D), np.float64)
     sel_w = np.zeros((R, topk), np.float64)
-    rc = _load().hsa_oracle_attend_gathered(qp, lp, kp, vp, _ptr(ns, _i32p), R, D, chunk, topk, scale,
+    rc = _load().hsa_oracle_attend_gathered(qp, qsp, lp, kp, vp, _ptr(ns, _i32p), R, D, chunk, topk, scale,
                                             _ptr(out, _f64p), _ptr(sel_w, _f64p))
     _check(rc, "hsa_oracle_attend_gathered")
     return out, sel_w
 
 
-def backward(Q, K, V, L, dO, sel_idx, chunk=64, scale=None):
+def backward(Q, K, V, L, dO, sel_idx, chunk=64, scale=None, Qs=None):
     """Gradients of the HSA forward for a fixed selection sel_idx [B, H, T, topk] (-1 = empty).
 
-    Returns (dQ, dK, dV, dL) as float64 arrays shaped like Q, K, V, L.
+    Returns (dQ, dK, dV, dL) as float64 arrays shaped like Q, K, V, L; with separate retrieval queries
+    Qs, (dQ, dK, dV, dL, dQs) where dQ is the attention query's gradient and dQs the retrieval query's.
     """
     Q, qp = _f32(Q)
     K, kp = _f32(K)
     V, vp = _f32(V)
     L, lp = _f32(L)
     dO, gp = _f32(dO)
+    Qs, qsp = _opt_f32(Qs, Q)
     B, H, T, D = Q.shape
     if scale is None:
         scale = default_scale(D)
@@ -173,7 +189,9 @@ def backward(Q, K, V, L, dO, sel_idx, chunk=64, scale=None):
     dK = np.zeros(K.shape, np.float64)
     dV = np.zeros(V.shape, np.float64)
     dL = np.zeros(L.shape, np.float64)
-    rc = _load().hsa_oracle_backward(qp, kp, vp, lp, gp, _ptr(si, _i32p), B, H, T, D, chunk, topk, scale,
-                                     _ptr(dQ, _f64p), _ptr(dK, _f64p), _ptr(dV, _f64p), _ptr(dL, _f64p))
+    dQs = np.zeros(Q.shape, np.float64) if Qs is not None else None
+    rc = _load().hsa_oracle_backward(qp, qsp, kp, vp, lp, gp, _ptr(si, _i32p), B, H, T, D, chunk, topk, scale,
+                                     _ptr(dQ, _f64p), _ptr(dK, _f64p), _ptr(dV, _f64p), _ptr(dL, _f64p),
+                                     _ptr(dQs, _f64p))
     _check(rc, "hsa_oracle_backward")
-    return dQ, dK, dV, dL
+    return (dQ, dK, dV, dL) if Qs is None else (dQ, dK, dV, dL, dQs)

@@ -11,14 +11,17 @@ import itertools
 import numpy as np
 
 
-def forward(Q, K, V, L, chunk, topk, scale):
-    """Q, K, V [B, H, T, D], L [B, H, N, D] -> (out [B,H,T,D], sel_idx [B,H,T,topk], sel_w [B,H,T,topk])."""
+def forward(Q, K, V, L, chunk, topk, scale, Qs=None):
+    """Q, K, V [B, H, T, D], L [B, H, N, D] -> (out [B,H,T,D], sel_idx [B,H,T,topk], sel_w [B,H,T,topk]).
+
+    Qs: separate retrieval queries (scores Qs . L), or None when Q also retrieves."""
     Q, K, V, L = (np.asarray(x, np.float64) for x in (Q, K, V, L))
+    Qs = Q if Qs is None else np.asarray(Qs, np.float64)
     B, H, T, D = Q.shape
     N = T // chunk
     t = np.arange(T)
     admissible = (np.arange(N)[None, :] + 1) * chunk - 1 <= t[:, None]           # [T, N]
-    S = scale * np.einsum("bhtd,bhnd->bhtn", Q, L)                                 # [B,H,T,N]
+    S = scale * np.einsum("bhtd,bhnd->bhtn", Qs, L)                                # [B,H,T,N]
     S_masked = np.where(admissible, S, -np.inf)
     order = np.argsort(-S_masked, axis=-1, kind="stable")                         # ties -> lower index
     n_t = admissible.sum(-1)                                                       # [T]

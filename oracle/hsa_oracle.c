@@ -158,7 +158,7 @@ static int attend_and_fuse(const float *q, const float *const *chunk_k, const fl
  *   next_s[i] = score of the best unselected admissible chunk, -INFINITY if none.
  * Any output pointer except out may be NULL.
  */
-int hsa_oracle_forward_rows(const float *Q, const float *K, const float *V, const float *L, int64_t B,
+int hsa_oracle_forward_rows(const float *Q, const float *Qs, const float *K, const float *V, const float *L, int64_t B,
                             int64_t H, int64_t T, int64_t D, int64_t chunk, int64_t topk, double scale,
                             int64_t nrows, const int64_t *rows, double *out, int32_t *sel_idx, double *sel_w,
                             double *sel_s, double *next_s) {
@@ -173,6 +173,7 @@ int hsa_oracle_forward_rows(const float *Q, const float *K, const float *V, cons
         if (r < 0 || r >= B * H * T) { status = ORACLE_EINVAL; continue; }
         int64_t bh = r / T, t = r % T;
         const float *q = Q + r * D;
+        const float *qs = (Qs ? Qs : Q) + r * D;  /* retrieval query (Step 2); q attends (Step 3) */
         int64_t n = admissible_chunks(t, chunk);
         if (n > N) n = N;
         double *score = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
@@ -184,7 +185,7 @@ int hsa_oracle_forward_rows(const float *Q, const float *K, const float *V, cons
         if (!score || !sel || !ss || !w || !ck || !cv) {
             status = ORACLE_ENOMEM;
         } else {
-            for (int64_t c = 0; c < n; ++c) score[c] = retrieval_score(q, L + (bh * N + c) * D, D, scale);
+            for (int64_t c = 0; c < n; ++c) score[c] = retrieval_score(qs, L + (bh * N + c) * D, D, scale);
             double nxt;
             int64_t k = select_topk(score, n, topk, sel, ss, &nxt);
             if (k < 0) {
@@ -285,7 +286,7 @@ int hsa_oracle_decode_select(const float *q, const float *Lc, const int64_t *cac
  * Used for decode (with chunks gathered from a cache too large for host memory) and to evaluate
  * the HSA output of a given selection.
  */
-int hsa_oracle_attend_gathered(const float *q, const float *Lg, const float *Kg, const float *Vg,
+int hsa_oracle_attend_gathered(const float *q, const float *qs, const float *Lg, const float *Kg, const float *Vg,
                                const int32_t *nsel, int64_t R, int64_t D, int64_t chunk, int64_t topk,
                                double scale, double *out, double *sel_w) {
     if (!q || !Lg || !Kg || !Vg || !nsel || !out || D < 1 || chunk < 1 || topk < 1) return ORACLE_EINVAL;
@@ -302,7 +303,7 @@ int hsa_oracle_attend_gathered(const float *q, const float *Lg, const float *Kg,
             status = ORACLE_ENOMEM;
         } else {
             for (int64_t j = 0; j < k; ++j) {
-                ss[j] = retrieval_score(q + i * D, Lg + (i * topk + j) * D, D, scale);
+                ss[j] = retrieval_score((qs ? qs : q) + i * D, Lg + (i * topk + j) * D, D, scale);
                 ck[j] = Kg + (i * topk + j) * chunk * D;
                 cv[j] = Vg + (i * topk + j) * chunk * D;
             }
@@ -322,7 +323,9 @@ int hsa_oracle_attend_gathered(const float *q, const float *Lg, const float *Kg,
  * explainer's Step 4 says retrieval is learned: w multiplies the output, so dLoss/ds flows).
  *
  *   Q, K, V, dO : [B, H, T, D]   L : [B, H, N, D]   sel_idx : [B, H, T, topk] (-1 = empty slot)
- * Outputs (overwritten): dQ, dK, dV [B, H, T, D], dL [B, H, N, D], all double.
+ *   Qs : [B, H, T, D] retrieval queries, or NULL when Q also retrieves (then dQs must be NULL too)
+ * Outputs (overwritten): dQ, dK, dV [B, H, T, D], dL [B, H, N, D], all double; with a separate Qs,
+ * dQ holds the attention part only and dQs [B, H, T, D] the retrieval part (the ds L terms).
  *
  * Chain rule, per row t with selected chunks j (scores s_j, weights w = softmax(s)):
  *   O_j  = P_j V_j,  P_j = softmax(a_j),  a_j[u] = scale * q.K_j[u]      (Step 3)
@@ -335,13 +338,16 @@ int hsa_oracle_attend_gathered(const float *q, const float *Lg, const float *Kg,
  * Rows are processed in order inside one (b, h), and (b, h) slices in parallel, so the
  * accumulation order is fixed.
  */
-int hsa_oracle_backward(const float *Q, const float *K, const float *V, const float *L, const float *dO,
-                        const int32_t *sel_idx, int64_t B, int64_t H, int64_t T, int64_t D, int64_t chunk,
-                        int64_t topk, double scale, double *dQ, double *dK, double *dV, double *dL) {
+int hsa_oracle_backward(const float *Q, const float *Qs, const float *K, const float *V, const float *L,
+                        const float *dO, const int32_t *sel_idx, int64_t B, int64_t H, int64_t T, int64_t D,
+                        int64_t chunk, int64_t topk, double scale, double *dQ, double *dK, double *dV, double *dL,
+                        double *dQs) {
     if (!Q || !K || !V || !L || !dO || !sel_idx || !dQ || !dK || !dV || !dL || D < 1 || chunk < 1 || topk < 1)
         return ORACLE_EINVAL;
+    if ((Qs == NULL) != (dQs == NULL)) return ORACLE_EINVAL;
     const int64_t N = T / chunk;
     memset(dQ, 0, (size_t)(B * H * T * D) * sizeof(double));
+    if (dQs) memset(dQs, 0, (size_t)(B * H * T * D) * sizeof(double));
     memset(dK, 0, (size_t)(B * H * T * D) * sizeof(double));
     memset(dV, 0, (size_t)(B * H * T * D) * sizeof(double));
     memset(dL, 0, (size_t)(B * H * N * D) * sizeof(double));
@@ -361,6 +367,8 @@ int hsa_oracle_backward(const float *Q, const float *K, const float *V, const fl
             for (int64_t t = 0; t < T; ++t) {
                 const int64_t r = bh * T + t;
                 const float *q = Q + r * D;
+                const float *qs = (Qs ? Qs : Q) + r * D;  /* retrieval query */
+                double *dq_ret = (dQs ? dQs : dQ) + r * D;  /* its gradient */
                 const float *go = dO + r * D;
                 int64_t k = 0;
                 for (int64_t j = 0; j < topk; ++j) {
@@ -370,7 +378,7 @@ int hsa_oracle_backward(const float *Q, const float *K, const float *V, const fl
                     cj[k++] = c;
                 }
                 if (k == 0) continue;
-                for (int64_t j = 0; j < k; ++j) s[j] = retrieval_score(q, L + (bh * N + cj[j]) * D, D, scale);
+                for (int64_t j = 0; j < k; ++j) s[j] = retrieval_score(qs, L + (bh * N + cj[j]) * D, D, scale);
                 fusion_weights(s, k, w);
                 double wdw = 0.0;
                 for (int64_t j = 0; j < k; ++j) {
@@ -408,8 +416,8 @@ int hsa_oracle_backward(const float *Q, const float *K, const float *V, const fl
                         }
                     }
                     for (int64_t d = 0; d < D; ++d) {
-                        dQ[r * D + d] += scale * ds * (double)Lc[d];
-                        dLc[d] += scale * ds * (double)q[d];
+                        dq_ret[d] += scale * ds * (double)Lc[d];
+                        dLc[d] += scale * ds * (double)qs[d];
                     }
                 }
             }

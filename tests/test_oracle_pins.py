@@ -356,11 +356,12 @@ def test_backward_matches_central_differences(oracle_mod):
         assert np.abs(g).max() > 0
 
 
-def dense_masked_hsa_torch(Q, K, V, L, sel_idx, chunk, scale):
-    """HSA with a fixed selection as dense masked torch ops (every query x every chunk)."""
+def dense_masked_hsa_torch(Q, K, V, L, sel_idx, chunk, scale, Qs=None):
+    """HSA with a fixed selection as dense masked torch ops (every query x every chunk). Qs: separate
+    retrieval queries (the fusion weights come from Qs . L), or None when Q also retrieves."""
     B, H, T, D = Q.shape
     N = L.shape[2]
-    S = scale * torch.einsum("bhtd,bhnd->bhtn", Q, L)
+    S = scale * torch.einsum("bhtd,bhnd->bhtn", Q if Qs is None else Qs, L)
     si = torch.as_tensor(sel_idx, dtype=torch.int64)
     hits = torch.zeros(B, H, T, N + 1, dtype=torch.int64)
     hits.scatter_add_(-1, torch.where(si >= 0, si, N), torch.ones_like(si))   # empty slots -> column N
@@ -387,3 +388,57 @@ def test_backward_matches_torch_autograd(oracle_mod, T, chunk, topk):
     grads = oracle_mod.backward(Q, K, V, L, G, sel, chunk=chunk, scale=scale)
     for t_, g in zip(ts, grads):
         np.testing.assert_allclose(g, t_.grad.numpy(), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# Separate retrieval query (the pages' hsa_step takes a retrieval query q_slc and an attention query
+# q_attn): Step 2 scores q_slc . L, Step 3 attends with q_attn, Step 4 weights by the retrieval scores
+
+
+@pytest.mark.parametrize("B,H,T,D,chunk,topk", [(1, 2, 48, 8, 4, 3), (2, 1, 70, 16, 8, 2), (1, 2, 40, 4, 4, 20)])
+def test_separate_retrieval_query_matches_dense_brute_force(oracle_mod, B, H, T, D, chunk, topk):
+    Q, K, V, L = bf16_arrays(B, H, T, D, chunk, seed=11 + T + D)
+    Qs = bf16_arrays(B, H, T, D, chunk, seed=99 + T + D)[0]
+    scale = 1.0 / math.sqrt(D)
+    r = oracle_mod.forward(Q, K, V, L, chunk=chunk, topk=topk, scale=scale, Qs=Qs)
+    out_b, idx_b, w_b = brute.forward(Q, K, V, L, chunk, topk, scale, Qs=Qs)
+    np.testing.assert_array_equal(r["sel_idx"].reshape(idx_b.shape), idx_b)
+    np.testing.assert_allclose(r["out"].reshape(out_b.shape), out_b, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r["sel_w"].reshape(w_b.shape), w_b, rtol=0, atol=1e-13)
+    # and the retrieval query really decides: the selection differs from the one Q would make
+    r_same = oracle_mod.forward(Q, K, V, L, chunk=chunk, topk=topk, scale=scale)
+    if topk < T // chunk:
+        assert not np.array_equal(r["sel_idx"], r_same["sel_idx"])
+
+
+def test_retrieval_query_equal_to_q_is_the_shared_path(oracle_mod):
+    B, H, T, D, chunk, topk = 1, 2, 96, 8, 8, 3
+    Q, K, V, L = bf16_arrays(B, H, T, D, chunk, seed=5)
+    G = np.random.default_rng(9).standard_normal((B, H, T, D)).astype(np.float32)
+    a = oracle_mod.forward(Q, K, V, L, chunk=chunk, topk=topk)
+    b = oracle_mod.forward(Q, K, V, L, chunk=chunk, topk=topk, Qs=Q.copy())
+    np.testing.assert_array_equal(a["sel_idx"], b["sel_idx"])
+    np.testing.assert_array_equal(a["out"], b["out"])
+    sel = a["sel_idx"].reshape(B, H, T, topk)
+    dQ, dK, dV, dL = oracle_mod.backward(Q, K, V, L, G, sel, chunk=chunk)
+    dQa, dK2, dV2, dL2, dQs = oracle_mod.backward(Q, K, V, L, G, sel, chunk=chunk, Qs=Q.copy())
+    np.testing.assert_allclose(dQa + dQs, dQ, rtol=0, atol=1e-12)  # the two parts of one query's gradient
+    for x, y in ((dK, dK2), (dV, dV2), (dL, dL2)):
+        np.testing.assert_array_equal(x, y)
+
+
+@pytest.mark.parametrize("T,chunk,topk", [(96, 8, 3), (70, 8, 20)])
+def test_separate_retrieval_query_backward_matches_torch_autograd(oracle_mod, T, chunk, topk):
+    B, H, D = 2, 2, 8
+    Q, K, V, L = bf16_arrays(B, H, T, D, chunk, seed=53)
+    Qs = bf16_arrays(B, H, T, D, chunk, seed=59)[0]
+    G = np.random.default_rng(6).standard_normal((B, H, T, D)).astype(np.float32)
+    scale = 1.0 / math.sqrt(D)
+    sel = oracle_mod.forward(Q, K, V, L, chunk=chunk, topk=topk, Qs=Qs)["sel_idx"].reshape(B, H, T, topk)
+    ts = [torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (Q, K, V, L, Qs)]
+    out = dense_masked_hsa_torch(*ts[:4], sel, chunk, scale, Qs=ts[4])
+    (out * torch.tensor(G, dtype=torch.float64)).sum().backward()
+    grads = oracle_mod.backward(Q, K, V, L, G, sel, chunk=chunk, scale=scale, Qs=Qs)
+    for t_, g in zip(ts, grads):  # dQ (attention), dK, dV, dL, dQs (retrieval)
+        np.testing.assert_allclose(g, t_.grad.numpy(), rtol=0, atol=1e-12)
+        assert np.abs(g).max() > 0

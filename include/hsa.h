@@ -158,6 +158,36 @@ hsa_status hsa_backward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
                         float *dV, float *dL, void *workspace, size_t workspace_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * Separate retrieval query. Explainer of "Every Token Counts", "How It Works (Technically)" Steps 2-3,
+ * and the per-token procedure in "The algorithm, simplified": the query that scores the landmarks
+ * (q_slc) and the query that attends inside the selected chunks (q_attn) are separate projections.
+ * These entry points take both: Qs / qs [same shape as Q / q] retrieve (Step 2 scores and the Step 4
+ * fusion weights come from Qs . L), Q / q attend (Step 3). Everything else -- shapes, layouts,
+ * ownership, workspace rules, error behaviour, outputs -- is as for the single-query calls above;
+ * with Qs == Q they compute the same result.
+ * hsa_backward_qslc writes dQ (the attention query's gradient: the dS K_c terms only) and dQs (the
+ * retrieval query's: the ds L_c terms), both fp32 [B, H, T, D], zero-initialised by the call; its
+ * workspace (hsa_backward_qslc_workspace_size) also holds ds for every (token, slot).
+ * -------------------------------------------------------------------------------------------*/
+hsa_status hsa_forward_qslc(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
+                            const hsa_bf16 *L, int B, int H, int T, int D, int chunk, int topk, float scale,
+                            hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace, size_t workspace_bytes,
+                            void *stream);
+
+hsa_status hsa_decode_qslc(const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
+                           const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B, int H, int D,
+                           int chunk, int topk, float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+size_t hsa_backward_qslc_workspace_size(int B, int H, int T, int D, int chunk, int topk);
+
+hsa_status hsa_backward_qslc(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
+                             const hsa_bf16 *L, const hsa_bf16 *out, const hsa_bf16 *dout, const int32_t *sel_idx,
+                             const float *sel_w, int B, int H, int T, int D, int chunk, int topk, float scale,
+                             float *dQ, float *dK, float *dV, float *dL, float *dQs, void *workspace,
+                             size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------------------------
  * Measurement hooks (no counterpart on the pages; used to time each kernel live).
  *
  * hsa_profile_enable(1) starts recording a pair of CUDA events around every kernel launch and

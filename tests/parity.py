@@ -15,10 +15,11 @@ OUT_MEAN_ABS = 2e-3
 W_MAX_ABS = 1e-3
 
 
-def compare_forward_rows(oracle_mod, gpu_out, gpu_idx, gpu_w, orc, Q, K, V, L, rows, chunk, scale):
+def compare_forward_rows(oracle_mod, gpu_out, gpu_idx, gpu_w, orc, Q, K, V, L, rows, chunk, scale, Qs=None):
     """gpu_* and orc[...] are per-row arrays aligned with ``rows`` (flat (b*H+h)*T+t ids).
 
-    Q, K, V, L: float32 host arrays [B, H, T, D] / [B, H, N, D] (needed for tie rows only).
+    Q, K, V, L: float32 host arrays [B, H, T, D] / [B, H, N, D] (needed for tie rows only); Qs: the
+    separate retrieval queries when there are any (they decide the ties).
     Returns a dict of statistics; raises AssertionError on a violation.
     """
     gpu_out = np.asarray(gpu_out, np.float64)
@@ -58,7 +59,7 @@ def compare_forward_rows(oracle_mod, gpu_out, gpu_idx, gpu_w, orc, Q, K, V, L, r
     if tie_rows:
         B, H, T, D = Q.shape
         rr = np.asarray([rows[i] for i in tie_rows])
-        S = oracle_mod.scores(Q, L, rr, chunk=chunk, scale=scale)
+        S = oracle_mod.scores(Q if Qs is None else Qs, L, rr, chunk=chunk, scale=scale)
         topk = gpu_idx.shape[1]
         Lg = np.zeros((len(rr), topk, D), np.float32)
         Kg = np.zeros((len(rr), topk, chunk, D), np.float32)
@@ -76,7 +77,8 @@ def compare_forward_rows(oracle_mod, gpu_out, gpu_idx, gpu_w, orc, Q, K, V, L, r
                 Kg[n, j] = K[bh // H, bh % H, c * chunk:(c + 1) * chunk]
                 Vg[n, j] = V[bh // H, bh % H, c * chunk:(c + 1) * chunk]
             nsel[n] = len(kept)
-        o, _ = oracle_mod.attend_gathered(Qr, Lg, Kg, Vg, nsel, scale=scale)
+        Qsr = None if Qs is None else Qs.reshape(-1, D)[rr]
+        o, _ = oracle_mod.attend_gathered(Qr, Lg, Kg, Vg, nsel, scale=scale, qs=Qsr)
         dt = np.abs(gpu_out[tie_rows] - o)
         assert dt.max() <= OUT_MAX_ABS, f"tie rows max-abs {dt.max():.4g}"
     return stats

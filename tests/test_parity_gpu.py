@@ -97,10 +97,10 @@ def test_forward_is_deterministic_in_selection_and_close_in_output():
 # decode
 
 
-def oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, chunk=64):
-    """Oracle decode: selection from (q, Lc) on the host, then the selected chunks gathered."""
+def oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, chunk=64, qs=None):
+    """Oracle decode: selection from (q or qs, Lc) on the host, then the selected chunks gathered."""
     B, H, D = q.shape
-    sel = oracle_mod.decode_select(host(q), host(Lc), lens.cpu().numpy(), chunk=chunk, topk=topk,
+    sel = oracle_mod.decode_select(host(q if qs is None else qs), host(Lc), lens.cpu().numpy(), chunk=chunk, topk=topk,
                                    scale=1 / math.sqrt(D))
     idx = torch.as_tensor(sel["sel_idx"], device=Kc.device, dtype=torch.int64).clamp(min=0)   # [B,H,k]
     tok = (idx[..., None] * chunk + torch.arange(chunk, device=Kc.device)).reshape(B, H, -1)
@@ -109,16 +109,17 @@ def oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, chunk=64):
     Lg = torch.gather(Lc, 2, idx[..., None].expand(-1, -1, -1, D)).reshape(B * H, topk, D)
     nsel = (sel["sel_idx"] >= 0).sum(-1).reshape(-1)
     out, w = oracle_mod.attend_gathered(host(q).reshape(B * H, D), host(Lg), host(Kg), host(Vg), nsel,
-                                        scale=1 / math.sqrt(D))
+                                        scale=1 / math.sqrt(D),
+                                        qs=None if qs is None else host(qs).reshape(B * H, D))
     return dict(out=out, sel_idx=sel["sel_idx"].reshape(B * H, topk), sel_w=w, sel_s=sel["sel_s"].reshape(B * H, topk),
                 next_s=sel["next_s"].reshape(-1))
 
 
-def check_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk):
+def check_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, qs=None):
     B, H, D = q.shape
-    out, idx, w = hsa.hsa_decode(q, Kc, Vc, Lc, lens, topk)
+    out, idx, w = hsa.hsa_decode(q, Kc, Vc, Lc, lens, topk, qs=qs)
     torch.cuda.synchronize()
-    orc = oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk)
+    orc = oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, qs=qs)
     g_idx = idx.reshape(B * H, topk).cpu().numpy()
     g_w = w.reshape(B * H, topk).cpu().numpy()
     g_out = host(out).reshape(B * H, D)
@@ -246,3 +247,51 @@ def test_workspace_status_clear_after_calls():
     wsd = torch.empty(hsa.hsa_decode_workspace_size(2, 2, 5056, D, 64, topk), dtype=torch.uint8, device=DEV)
     hsa.hsa_decode(q, Kc, Vc, Lc, lens_t, topk, workspace=wsd)
     hsa.hsa_workspace_status(wsd)
+
+
+# ---------------------------------------------------------------------------------------------
+# separate retrieval query (q_slc scores the landmarks, q_attn attends)
+
+
+@pytest.mark.parametrize("B,H,T,D,topk", [(1, 2, 2048 + 37, 128, 16), (1, 2, 1100, 64, 8)])
+def test_forward_separate_retrieval_query_matches_oracle(oracle_mod, B, H, T, D, topk):
+    Q, K, V, L = inputs.forward_inputs(B, H, T, D, 600 + T, device=DEV)
+    Qs = inputs.forward_inputs(B, H, T, D, 700 + T, device=DEV)[0]
+    out, idx, w = hsa.hsa_forward(Q, K, V, L, topk, Qs=Qs)
+    Qh, Kh, Vh, Lh, Qsh = (host(x) for x in (Q, K, V, L, Qs))
+    scale = 1 / math.sqrt(D)
+    orc = oracle_mod.forward(Qh, Kh, Vh, Lh, chunk=64, topk=topk, scale=scale, Qs=Qsh)
+    rows = np.arange(B * H * T)
+    compare_forward_rows(oracle_mod, host(out).reshape(-1, D), host(idx).reshape(-1, topk),
+                         host(w).reshape(-1, topk), orc, Qh, Kh, Vh, Lh, rows, 64, scale, Qs=Qsh)
+    # the retrieval query decides: the single-query call selects differently
+    _, idx_q, _ = hsa.hsa_forward(Q, K, V, L, topk)
+    assert not torch.equal(idx, idx_q)
+
+
+@pytest.mark.parametrize("D,lens,topk", [(128, [9000, 4100], 8), (64, [64 * 300 - 1, 640], 32)])
+def test_decode_separate_retrieval_query_matches_oracle(oracle_mod, D, lens, topk):
+    B, H = len(lens), 2
+    q, Kc, Vc, Lc, lens_t, _ = inputs.decode_inputs(B, H, lens, D, seed=31 + D, Tmax=max(lens) + 64, device=DEV)
+    qs = inputs.decode_inputs(B, H, lens, D, seed=32 + D, Tmax=max(lens) + 64, device=DEV)[0]
+    _, idx, _ = check_decode(oracle_mod, q, Kc, Vc, Lc, lens_t, topk, qs=qs)
+    _, idx_q, _ = hsa.hsa_decode(q, Kc, Vc, Lc, lens_t, topk)
+    assert not torch.equal(idx, idx_q)
+
+
+@pytest.mark.parametrize("B,H,T,D,topk", [(1, 2, 2048 + 64, 128, 16), (1, 2, 1100, 64, 8)])
+def test_backward_separate_retrieval_query_matches_oracle(oracle_mod, B, H, T, D, topk):
+    Q, K, V, L = inputs.forward_inputs(B, H, T, D, 800 + T, device=DEV)
+    Qs = inputs.forward_inputs(B, H, T, D, 900 + T, device=DEV)[0]
+    dO = inputs.upstream_grad(B, H, T, D, 800 + T, device=DEV)
+    Qh, Kh, Vh, Lh, Qsh, dOh = (host(x) for x in (Q, K, V, L, Qs, dO))
+    scale = 1 / math.sqrt(D)
+    orc = oracle_mod.forward(Qh, Kh, Vh, Lh, chunk=64, topk=topk, scale=scale, Qs=Qsh)
+    sel_idx = torch.as_tensor(orc["sel_idx"].reshape(B, H, T, topk), device=DEV)
+    sel_w = torch.as_tensor(orc["sel_w"].reshape(B, H, T, topk), dtype=torch.float32, device=DEV)
+    out = torch.as_tensor(orc["out"].reshape(B, H, T, D), dtype=torch.float32, device=DEV).to(torch.bfloat16)
+    grads = hsa.hsa_backward(Q, K, V, L, out, dO, sel_idx, sel_w, Qs=Qs)
+    ref = oracle_mod.backward(Qh, Kh, Vh, Lh, dOh, orc["sel_idx"].reshape(B, H, T, topk), chunk=64, scale=scale,
+                              Qs=Qsh)
+    for g, r, n in zip(grads, ref, ("dQ", "dK", "dV", "dL", "dQs")):
+        grad_close(host(g), r, n)

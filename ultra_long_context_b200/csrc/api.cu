@@ -77,11 +77,12 @@ struct FwdLayout {
     int32_t *num_tiles, *err;
     float *delta;
     int32_t *pair_slot;
+    float *ds_pair;  // [B*H*T, topk] ds per (token, slot): separate retrieval query only
     size_t bytes;
     int max_tiles;
 };
 
-FwdLayout fwd_layout(void *ws, int B, int H, int T, int D, int topk, bool backward) {
+FwdLayout fwd_layout(void *ws, int B, int H, int T, int D, int topk, bool backward, bool qslc = false) {
     FwdLayout l{};
     Carver c{static_cast<char *>(ws)};
     l.err = c.take<int32_t>(1);  // first: hsa_workspace_status reads it at offset 0
@@ -100,6 +101,7 @@ FwdLayout fwd_layout(void *ws, int B, int H, int T, int D, int topk, bool backwa
     l.num_tiles = c.take<int32_t>(1);
     l.delta = backward ? c.take<float>(rows) : nullptr;
     l.pair_slot = backward ? c.take<int32_t>(pairs) : nullptr;
+    l.ds_pair = backward && qslc ? c.take<float>(pairs) : nullptr;
     l.bytes = c.used;
     return l;
 }
@@ -163,18 +165,20 @@ size_t hsa_forward_workspace_size(int B, int H, int T, int D, int chunk, int top
     return fwd_layout(nullptr, B, H, T, D, topk, false).bytes;
 }
 
-hsa_status hsa_forward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, const hsa_bf16 *L, int B, int H,
-                       int T, int D, int chunk, int topk, float scale, hsa_bf16 *out, int32_t *sel_idx,
-                       float *sel_w, void *workspace, size_t workspace_bytes, void *stream) {
+// Qs retrieves (Step 2 scores, Step 4 weights), Q attends (Step 3); the single-query call passes Q twice.
+static hsa_status forward_impl(const char *name, const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K,
+                               const hsa_bf16 *V, const hsa_bf16 *L, int B, int H, int T, int D, int chunk, int topk,
+                               float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace,
+                               size_t workspace_bytes, void *stream) {
     g_last_error.clear();
     hsa_status st = check_common(B, H, D, chunk, topk, 32);
     if (st != HSA_OK) return st;
     if (T < 1) return fail(HSA_ERR_INVALID_ARG, "T must be >= 1 (got %d)", T);
     if ((double)B * H * T * topk >= 2147483647.0 || (double)B * H * T * D >= 9.0e15)
         return fail(HSA_ERR_UNSUPPORTED, "B*H*T*topk must stay below 2^31");
-    if (!Q || !K || !V || !out) return fail(HSA_ERR_INVALID_ARG, "Q, K, V and out must not be NULL");
+    if (!Qs || !Q || !K || !V || !out) return fail(HSA_ERR_INVALID_ARG, "Q, Qs, K, V and out must not be NULL");
     if (T >= 64 && !L) return fail(HSA_ERR_INVALID_ARG, "L must not be NULL when T >= 64");
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || (L && !aligned16(L)))
+    if (!aligned16(Qs) || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || (L && !aligned16(L)))
         return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
     if ((sel_idx && !aligned16(sel_idx)) || (sel_w && !aligned16(sel_w)))
         return fail(HSA_ERR_INVALID_ARG, "sel_idx / sel_w must be 16-byte aligned");
@@ -182,7 +186,7 @@ hsa_status hsa_forward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, 
     if ((st = check_ws(workspace, workspace_bytes, need.bytes)) != HSA_OK) return st;
     FwdLayout l = fwd_layout(workspace, B, H, T, D, topk, false);
     hsa::ForwardArgs a{};
-    a.Q = Q; a.K = K; a.V = V; a.L = L;
+    a.Qs = Qs; a.Q = Q; a.K = K; a.V = V; a.L = L;
     a.B = B; a.H = H; a.T = T; a.D = D; a.N = T / 64; a.topk = topk;
     a.scale = resolve_scale(scale, D);
     a.out = out;
@@ -194,7 +198,22 @@ hsa_status hsa_forward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, 
     a.pair_row = l.pair_row; a.pair_w = l.pair_w; a.tiles = l.tiles; a.num_tiles = l.num_tiles;
     a.err = l.err;
     a.max_tiles = l.max_tiles;
-    return cuda_status(hsa::launch_forward(a, static_cast<cudaStream_t>(stream)), "hsa_forward");
+    return cuda_status(hsa::launch_forward(a, static_cast<cudaStream_t>(stream)), name);
+}
+
+hsa_status hsa_forward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, const hsa_bf16 *L, int B, int H,
+                       int T, int D, int chunk, int topk, float scale, hsa_bf16 *out, int32_t *sel_idx,
+                       float *sel_w, void *workspace, size_t workspace_bytes, void *stream) {
+    return forward_impl("hsa_forward", Q, Q, K, V, L, B, H, T, D, chunk, topk, scale, out, sel_idx, sel_w, workspace,
+                        workspace_bytes, stream);
+}
+
+hsa_status hsa_forward_qslc(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
+                            const hsa_bf16 *L, int B, int H, int T, int D, int chunk, int topk, float scale,
+                            hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace, size_t workspace_bytes,
+                            void *stream) {
+    return forward_impl("hsa_forward_qslc", Qs, Q, K, V, L, B, H, T, D, chunk, topk, scale, out, sel_idx, sel_w,
+                        workspace, workspace_bytes, stream);
 }
 
 size_t hsa_decode_workspace_size(int B, int H, int64_t Tmax, int D, int chunk, int topk) {
@@ -203,18 +222,18 @@ size_t hsa_decode_workspace_size(int B, int H, int64_t Tmax, int D, int chunk, i
     return dec_layout(nullptr, B, H, Tmax, D, topk).bytes;
 }
 
-hsa_status hsa_decode(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc, const hsa_bf16 *Lc,
-                      const int64_t *cache_len, int64_t Tmax, int B, int H, int D, int chunk, int topk,
-                      float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace,
-                      size_t workspace_bytes, void *stream) {
+static hsa_status decode_impl(const char *name, const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *Kc,
+                              const hsa_bf16 *Vc, const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B,
+                              int H, int D, int chunk, int topk, float scale, hsa_bf16 *out, int32_t *sel_idx,
+                              float *sel_w, void *workspace, size_t workspace_bytes, void *stream) {
     g_last_error.clear();
     hsa_status st = check_common(B, H, D, chunk, topk, 64);
     if (st != HSA_OK) return st;
     if (Tmax < 0) return fail(HSA_ERR_INVALID_ARG, "Tmax must be >= 0");
     if (Tmax / 64 >= 2147483647LL) return fail(HSA_ERR_UNSUPPORTED, "Tmax / 64 must stay below 2^31");
-    if (!q || !Kc || !Vc || !Lc || !cache_len || !out)
-        return fail(HSA_ERR_INVALID_ARG, "q, Kc, Vc, Lc, cache_len and out must not be NULL");
-    if (!aligned16(q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(Lc) || !aligned16(out) ||
+    if (!qs || !q || !Kc || !Vc || !Lc || !cache_len || !out)
+        return fail(HSA_ERR_INVALID_ARG, "q, qs, Kc, Vc, Lc, cache_len and out must not be NULL");
+    if (!aligned16(qs) || !aligned16(q) || !aligned16(Kc) || !aligned16(Vc) || !aligned16(Lc) || !aligned16(out) ||
         (reinterpret_cast<uintptr_t>(cache_len) & 7u))
         return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned (cache_len 8-byte)");
     if ((sel_idx && !aligned16(sel_idx)) || (sel_w && !aligned16(sel_w)))
@@ -231,7 +250,7 @@ hsa_status hsa_decode(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
     if ((st = check_ws(workspace, workspace_bytes, need.bytes)) != HSA_OK) return st;
     DecLayout l = dec_layout(workspace, B, H, Tmax, D, topk);
     hsa::DecodeArgs a{};
-    a.q = q; a.Kc = Kc; a.Vc = Vc; a.Lc = Lc; a.cache_len = cache_len;
+    a.qs = qs; a.q = q; a.Kc = Kc; a.Vc = Vc; a.Lc = Lc; a.cache_len = cache_len;
     a.Tmax = Tmax; a.Nmax = Tmax / 64;
     a.B = B; a.H = H; a.D = D; a.K = topk;
     a.scale = resolve_scale(scale, D);
@@ -242,8 +261,24 @@ hsa_status hsa_decode(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
     // the decode kernels never wait on one another; the flag is cleared so that a status query
     // after this call reports this call
     cudaError_t ce = cudaMemsetAsync(l.err, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
-    if (ce != cudaSuccess) return cuda_status(ce, "hsa_decode");
-    return cuda_status(hsa::launch_decode(a, static_cast<cudaStream_t>(stream)), "hsa_decode");
+    if (ce != cudaSuccess) return cuda_status(ce, name);
+    return cuda_status(hsa::launch_decode(a, static_cast<cudaStream_t>(stream)), name);
+}
+
+hsa_status hsa_decode(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc, const hsa_bf16 *Lc,
+                      const int64_t *cache_len, int64_t Tmax, int B, int H, int D, int chunk, int topk,
+                      float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace,
+                      size_t workspace_bytes, void *stream) {
+    return decode_impl("hsa_decode", q, q, Kc, Vc, Lc, cache_len, Tmax, B, H, D, chunk, topk, scale, out, sel_idx,
+                       sel_w, workspace, workspace_bytes, stream);
+}
+
+hsa_status hsa_decode_qslc(const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
+                           const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B, int H, int D,
+                           int chunk, int topk, float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+    return decode_impl("hsa_decode_qslc", qs, q, Kc, Vc, Lc, cache_len, Tmax, B, H, D, chunk, topk, scale, out,
+                       sel_idx, sel_w, workspace, workspace_bytes, stream);
 }
 
 size_t hsa_backward_workspace_size(int B, int H, int T, int D, int chunk, int topk) {
@@ -252,10 +287,18 @@ size_t hsa_backward_workspace_size(int B, int H, int T, int D, int chunk, int to
     return fwd_layout(nullptr, B, H, T, D, topk, true).bytes;
 }
 
-hsa_status hsa_backward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, const hsa_bf16 *L,
-                        const hsa_bf16 *out, const hsa_bf16 *dout, const int32_t *sel_idx, const float *sel_w,
-                        int B, int H, int T, int D, int chunk, int topk, float scale, float *dQ, float *dK,
-                        float *dV, float *dL, void *workspace, size_t workspace_bytes, void *stream) {
+size_t hsa_backward_qslc_workspace_size(int B, int H, int T, int D, int chunk, int topk) {
+    (void)chunk;
+    if (B < 1 || H < 1 || T < 1 || D < 1 || topk < 1) return 0;
+    return fwd_layout(nullptr, B, H, T, D, topk, true, true).bytes;
+}
+
+// Qs / dQs are NULL for the single-query call (Q retrieves too and dQ takes both parts).
+static hsa_status backward_impl(const char *name, const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K,
+                                const hsa_bf16 *V, const hsa_bf16 *L, const hsa_bf16 *out, const hsa_bf16 *dout,
+                                const int32_t *sel_idx, const float *sel_w, int B, int H, int T, int D, int chunk,
+                                int topk, float scale, float *dQ, float *dK, float *dV, float *dL, float *dQs,
+                                bool qslc, void *workspace, size_t workspace_bytes, void *stream) {
     g_last_error.clear();
     hsa_status st = check_common(B, H, D, chunk, topk, 32);
     if (st != HSA_OK) return st;
@@ -265,14 +308,18 @@ hsa_status hsa_backward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
     if (!Q || !K || !V || !out || !dout || !sel_idx || !sel_w || !dQ || !dK || !dV)
         return fail(HSA_ERR_INVALID_ARG, "tensor pointers must not be NULL");
     if (T >= 64 && (!L || !dL)) return fail(HSA_ERR_INVALID_ARG, "L and dL must not be NULL when T >= 64");
+    if (qslc && (!Qs || !dQs)) return fail(HSA_ERR_INVALID_ARG, "Qs and dQs must not be NULL");
+    if (qslc && (!aligned16(Qs) || !aligned16(dQs)))
+        return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || !aligned16(dout) ||
         !aligned16(sel_idx) || !aligned16(sel_w) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) ||
         (L && !aligned16(L)) || (dL && !aligned16(dL)))
         return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-    FwdLayout need = fwd_layout(nullptr, B, H, T, D, topk, true);
+    FwdLayout need = fwd_layout(nullptr, B, H, T, D, topk, true, qslc);
     if ((st = check_ws(workspace, workspace_bytes, need.bytes)) != HSA_OK) return st;
-    FwdLayout l = fwd_layout(workspace, B, H, T, D, topk, true);
+    FwdLayout l = fwd_layout(workspace, B, H, T, D, topk, true, qslc);
     hsa::BackwardArgs a{};
+    a.Qs = qslc ? Qs : nullptr; a.dQs = qslc ? dQs : nullptr; a.ds_pair = l.ds_pair;
     a.Q = Q; a.K = K; a.V = V; a.L = L; a.out = out; a.dout = dout;
     a.sel_idx = sel_idx; a.sel_w = sel_w;
     a.B = B; a.H = H; a.T = T; a.D = D; a.N = T / 64; a.topk = topk;
@@ -283,7 +330,24 @@ hsa_status hsa_backward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
     a.chunk_cursor = l.chunk_cursor;
     a.pair_row = l.pair_row; a.pair_w = l.pair_w; a.pair_slot = l.pair_slot;
     a.tiles = l.tiles; a.num_tiles = l.num_tiles; a.max_tiles = l.max_tiles; a.err = l.err;
-    return cuda_status(hsa::launch_backward(a, static_cast<cudaStream_t>(stream)), "hsa_backward");
+    return cuda_status(hsa::launch_backward(a, static_cast<cudaStream_t>(stream)), name);
+}
+
+hsa_status hsa_backward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, const hsa_bf16 *L,
+                        const hsa_bf16 *out, const hsa_bf16 *dout, const int32_t *sel_idx, const float *sel_w,
+                        int B, int H, int T, int D, int chunk, int topk, float scale, float *dQ, float *dK,
+                        float *dV, float *dL, void *workspace, size_t workspace_bytes, void *stream) {
+    return backward_impl("hsa_backward", nullptr, Q, K, V, L, out, dout, sel_idx, sel_w, B, H, T, D, chunk, topk,
+                         scale, dQ, dK, dV, dL, nullptr, false, workspace, workspace_bytes, stream);
+}
+
+hsa_status hsa_backward_qslc(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
+                             const hsa_bf16 *L, const hsa_bf16 *out, const hsa_bf16 *dout, const int32_t *sel_idx,
+                             const float *sel_w, int B, int H, int T, int D, int chunk, int topk, float scale,
+                             float *dQ, float *dK, float *dV, float *dL, float *dQs, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+    return backward_impl("hsa_backward_qslc", Qs, Q, K, V, L, out, dout, sel_idx, sel_w, B, H, T, D, chunk, topk,
+                         scale, dQ, dK, dV, dL, dQs, true, workspace, workspace_bytes, stream);
 }
 
 }  // extern "C"

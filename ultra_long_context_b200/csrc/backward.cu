@@ -108,7 +108,10 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
     const uint16_t *__restrict__ L, const uint16_t *__restrict__ dout, const float *__restrict__ delta, int T, int N,
     float scale, const PairTile *__restrict__ tiles, const int32_t *__restrict__ num_tiles,
     const int32_t *__restrict__ pair_row, const float *__restrict__ pair_w, float *__restrict__ dQ,
-    float *__restrict__ dK, float *__restrict__ dV, float *__restrict__ dL) {
+    float *__restrict__ dK, float *__restrict__ dV, float *__restrict__ dL, const uint16_t *__restrict__ Qs,
+    const int32_t *__restrict__ pair_slot, float *__restrict__ ds_pair, int Kslots) {
+    // Qs != NULL: separate retrieval queries. dL takes ds times the retrieval query, dQ leaves out the
+    // ds L_c term, and ds goes to ds_pair[token row, slot] for the retrieval query's gradient.
     using SM = BwdSmem<D>;
     constexpr int SD = SM::SD, SP = SM::SP, VPR = D / 8;
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -118,7 +121,7 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
     uint16_t *sG = sQ + kChunk * SD;        // gathered dO rows
     uint16_t *sP = sG + kChunk * SD;        // w P     [pair][key]
     uint16_t *sdS = sP + kPairTile * SP;    // dS      [pair][key]
-    __shared__ int s_row[kPairTile];
+    __shared__ int s_row[kPairTile], s_slot[kPairTile];
     __shared__ float s_w[kPairTile], s_ds[kPairTile], s_L[D];
 
     if ((int)blockIdx.x >= num_tiles[0]) return;
@@ -130,6 +133,7 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
         const bool ok = tid < pt.count;
         s_row[tid] = ok ? pair_row[pt.start + tid] : -1;
         s_w[tid] = ok ? pair_w[pt.start + tid] : 0.0f;
+        s_slot[tid] = ok && Qs ? pair_slot[pt.start + tid] : 0;
     }
     for (int d = tid; d < D; d += kBwdThreads) s_L[d] = __uint_as_float((uint32_t)L[((size_t)bh * N + c) * D + d] << 16);
     __syncthreads();
@@ -207,7 +211,12 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
     if ((lane & 3) == 0) {
         s_ds[p0] = ds0;
         s_ds[p1] = ds1;
+        if (Qs) {
+            if (row0 >= 0) ds_pair[(size_t)row0 * Kslots + s_slot[p0]] = ds0;
+            if (row1 >= 0) ds_pair[(size_t)row1 * Kslots + s_slot[p1]] = ds1;
+        }
     }
+    const float lsel = Qs ? 0.0f : 1.0f;  // the ds L_c term belongs to dQ only when Q retrieves
     // dS = w P (dP' - g) and w P, both to shared memory as bf16 [pair][key]
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
@@ -248,11 +257,11 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
         for (int nt = 0; nt < D / 8; ++nt) {
             const int col = nt * 8 + (lane & 3) * 2;
             if (row0 >= 0)
-                red_add_v2(dQ + (size_t)row0 * D + col, scale * (acc[nt][0] + ds0 * s_L[col]),
-                           scale * (acc[nt][1] + ds0 * s_L[col + 1]));
+                red_add_v2(dQ + (size_t)row0 * D + col, scale * (acc[nt][0] + lsel * ds0 * s_L[col]),
+                           scale * (acc[nt][1] + lsel * ds0 * s_L[col + 1]));
             if (row1 >= 0)
-                red_add_v2(dQ + (size_t)row1 * D + col, scale * (acc[nt][2] + ds1 * s_L[col]),
-                           scale * (acc[nt][3] + ds1 * s_L[col + 1]));
+                red_add_v2(dQ + (size_t)row1 * D + col, scale * (acc[nt][2] + lsel * ds1 * s_L[col]),
+                           scale * (acc[nt][3] + lsel * ds1 * s_L[col + 1]));
         }
     }
     __syncthreads();  // sP, sdS, s_ds complete
@@ -275,12 +284,51 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
             red_add_v2(dK + (krow0 + key1) * D + col, scale * acc[nt][2], scale * acc[nt][3]);
         }
     }
-    // dL_c += scale * sum_pairs ds q
+    // dL_c += scale * sum_pairs ds q (q: the retrieval query)
     for (int d = tid; d < D; d += kBwdThreads) {
         float acc = 0.0f;
-        for (int p = 0; p < pt.count; ++p) acc = fmaf(s_ds[p], __uint_as_float((uint32_t)sQ[p * SD + d] << 16), acc);
+        for (int p = 0; p < pt.count; ++p) {
+            const uint16_t qv = Qs ? Qs[(size_t)s_row[p] * D + d] : sQ[p * SD + d];
+            acc = fmaf(s_ds[p], __uint_as_float((uint32_t)qv << 16), acc);
+        }
         atomicAdd(dL + ((size_t)bh * N + c) * D + d, scale * acc);
     }
+}
+
+// dQs[t] = scale * sum_j ds[t, j] L[c_j] for a separate retrieval query: one warp per token row, D / 32
+// columns per lane; the selected landmark rows are few and stay in L2.
+template <int D>
+__global__ void __launch_bounds__(256) dqs_kernel(const int32_t *__restrict__ sel_idx, const float *__restrict__ ds_pair,
+                                                  const uint16_t *__restrict__ L, int T, int N, int K, float scale,
+                                                  size_t rows, float *__restrict__ dQs) {
+    constexpr int PER = D / 32;
+    const size_t row = (size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    const size_t bh = row / T;
+    float acc[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
+    for (int j = 0; j < K; ++j) {
+        const int c = sel_idx[row * K + j];
+        if (c < 0 || c >= N) continue;  // empty slot (the dispatch skips the same ids)
+        const float ds = ds_pair[row * K + j];
+        const uint16_t *lr = L + (bh * N + c) * D + lane * PER;
+        if constexpr (PER == 4) {
+            const uint2 v = *reinterpret_cast<const uint2 *>(lr);
+            acc[0] = fmaf(ds, bf16_lo(v.x), acc[0]);
+            acc[1] = fmaf(ds, bf16_hi(v.x), acc[1]);
+            acc[2] = fmaf(ds, bf16_lo(v.y), acc[2]);
+            acc[3] = fmaf(ds, bf16_hi(v.y), acc[3]);
+        } else {
+            const uint32_t v = *reinterpret_cast<const uint32_t *>(lr);
+            acc[0] = fmaf(ds, bf16_lo(v), acc[0]);
+            acc[1] = fmaf(ds, bf16_hi(v), acc[1]);
+        }
+    }
+    float *dst = dQs + row * D + lane * PER;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) dst[i] = scale * acc[i];
 }
 
 cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
@@ -298,6 +346,8 @@ cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
         if (e == cudaSuccess && a.N > 0)
             e = cudaMemsetAsync(a.chunk_cursor, 0, (size_t)BH * a.N * sizeof(int32_t), s);
         if (e == cudaSuccess && a.err) e = cudaMemsetAsync(a.err, 0, sizeof(int32_t), s);
+        // with chunks, dqs_kernel writes every row of dQs
+        if (e == cudaSuccess && a.Qs && a.N == 0) e = cudaMemsetAsync(a.dQs, 0, rows * a.D * sizeof(float), s);
     }
     if (e != cudaSuccess || a.N == 0) return e;
     const unsigned dblocks = (unsigned)((rows + 7) / 8);
@@ -313,15 +363,8 @@ cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
                         a.chunk_cursor, a.pair_row, a.pair_w, a.pair_slot, a.tiles, a.num_tiles, a.max_tiles,
                         tc ? kBwdUnitPairs : kPairTile, false, s);
     if (e != cudaSuccess) return e;
-    if (tc) return launch_backward_tc(a, s);
-    if (a.D == 128) {
-        const size_t smem = BwdSmem<128>::total;
-        e = cudaFuncSetAttribute(chunk_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        HSA_PROF("chunk_bwd", s);
-        chunk_bwd_kernel<128><<<a.max_tiles, kBwdThreads, smem, s>>>(a.Q, a.K, a.V, a.L, a.dout, a.delta, a.T, a.N,
-                                                                      a.scale, a.tiles, a.num_tiles, a.pair_row,
-                                                                      a.pair_w, a.dQ, a.dK, a.dV, a.dL);
+    if (tc) {
+        e = launch_backward_tc(a, s);
     } else {
         const size_t smem = BwdSmem<64>::total;
         e = cudaFuncSetAttribute(chunk_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -329,7 +372,18 @@ cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
         HSA_PROF("chunk_bwd", s);
         chunk_bwd_kernel<64><<<a.max_tiles, kBwdThreads, smem, s>>>(a.Q, a.K, a.V, a.L, a.dout, a.delta, a.T, a.N,
                                                                      a.scale, a.tiles, a.num_tiles, a.pair_row,
-                                                                     a.pair_w, a.dQ, a.dK, a.dV, a.dL);
+                                                                     a.pair_w, a.dQ, a.dK, a.dV, a.dL, a.Qs,
+                                                                     a.pair_slot, a.ds_pair, a.topk);
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess || !a.Qs) return e;
+    {  // the retrieval query's gradient, token-major from the stored ds
+        HSA_PROF("bwd_dqs", s);
+        const unsigned blocks = (unsigned)((rows + 7) / 8);
+        if (a.D == 128) dqs_kernel<128><<<blocks, 256, 0, s>>>(a.sel_idx, a.ds_pair, a.L, a.T, a.N, a.topk, a.scale,
+                                                                rows, a.dQs);
+        else dqs_kernel<64><<<blocks, 256, 0, s>>>(a.sel_idx, a.ds_pair, a.L, a.T, a.N, a.topk, a.scale, rows,
+                                                    a.dQs);
     }
     return cudaGetLastError();
 }

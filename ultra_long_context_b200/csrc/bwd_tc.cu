@@ -59,7 +59,8 @@ struct BtSmem {  // head dim 128
     static constexpr uint32_t EROW = LROW + 2048;      // int[4][128]: token rows for the dQ epilogue
     static constexpr uint32_t EDS = EROW + 2048;       // float[4][128]: ds (dQ epilogue and dL)
     static constexpr uint32_t SDL = EDS + 2048;        // float[4][128]: the unit's dL per compute warp
-    static constexpr uint32_t BAR = SDL + 2048;
+    static constexpr uint32_t SSLOT = SDL + 2048;      // int[2][128]: slot of each pair (separate Qs only)
+    static constexpr uint32_t BAR = SSLOT + 1024;
     static constexpr int NBAR = 22;
     static constexpr uint32_t TMEM = BAR + NBAR * 8;
     static constexpr uint32_t BYTES = TMEM + 16;
@@ -116,12 +117,17 @@ struct BtCursor {
     }
 };
 
+template <bool QSLC>
 __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
     const uint16_t *__restrict__ Q, const uint16_t *__restrict__ L, const uint16_t *__restrict__ dout,
     const float *__restrict__ delta, int T, int N, float scale, const PairTile *__restrict__ units,
     const int32_t *__restrict__ num_units, const int32_t *__restrict__ pair_row, const float *__restrict__ pair_w,
     float *__restrict__ dQ, float *__restrict__ dK, float *__restrict__ dV, float *__restrict__ dL,
-    int32_t *__restrict__ err, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
+    int32_t *__restrict__ err, const uint16_t *__restrict__ Qs, const int32_t *__restrict__ pair_slot,
+    float *__restrict__ ds_pair, int Kslots, const __grid_constant__ CUtensorMap tmK,
+    const __grid_constant__ CUtensorMap tmV) {
+    // QSLC: separate retrieval queries Qs. dL takes ds times the retrieval query (read from global
+    // memory), dQ leaves out the ds L_c term, and ds goes to ds_pair[token row, slot].
     using SM = BtSmem;
     constexpr int D = SM::D;
     extern __shared__ unsigned char smem_raw[];
@@ -135,6 +141,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
     int *e_row = reinterpret_cast<int *>(s + SM::EROW);
     float *e_ds = reinterpret_cast<float *>(s + SM::EDS);
     float *s_dl = reinterpret_cast<float *>(s + SM::SDL);
+    int *s_slot = reinterpret_cast<int *>(s + SM::SSLOT);
     auto bar = [&](int i) { return sb + SM::BAR + 8u * (uint32_t)i; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -177,15 +184,16 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
         const int rsub = lane / CPR, ch = lane % CPR;
         const int myr = 32 * lw + lane;
         // this thread's pair of the current tile: token row, weight, delta (fetched one tile ahead)
-        auto fetch = [&](const BtCursor &t, int &row, float &wt, float &dl) {
+        auto fetch = [&](const BtCursor &t, int &row, float &wt, float &dl, int &sl) {
             const int p = t.i * kBtTile + myr;
             row = (!t.done() && p < t.u.count) ? pair_row[t.u.start + p] : -1;
             wt = row >= 0 ? pair_w[t.u.start + p] : 0.0f;
             dl = row >= 0 ? delta[row] : 0.0f;
+            sl = (QSLC && row >= 0) ? pair_slot[t.u.start + p] : 0;
         };
-        int myrow;
+        int myrow, myslot;
         float myw, mydel;
-        fetch(cur, myrow, myw, mydel);
+        fetch(cur, myrow, myw, mydel, myslot);
         // dL_c += sum over a tile's pairs of ds q, computed here from the tile's Q rows just before the
         // stage is reloaded (the tile two back). Thread lt takes the 16-byte column chunk cc of pairs
         // 16 gq .. + 15; each loader warp keeps its own partial row in s_dl.
@@ -203,7 +211,14 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
 #pragma unroll 4
             for (int i = 0; i < 16; ++i) {
                 const int p = 16 * gq + i;
-                const uint4 qv = *reinterpret_cast<const uint4 *>(qt + tc::sw128(p, cc & 7));
+                uint4 qv;
+                if constexpr (QSLC) {  // the retrieval query's row (the stage's metadata is still this tile's)
+                    const int rp = s_row[stl * 128 + p];
+                    qv = rp >= 0 ? __ldg(reinterpret_cast<const uint4 *>(Qs + (size_t)rp * D + 8 * cc))
+                                 : make_uint4(0u, 0u, 0u, 0u);
+                } else {
+                    qv = *reinterpret_cast<const uint4 *>(qt + tc::sw128(p, cc & 7));
+                }
                 const float dsp = e_ds[slot * 128 + p];
                 a8[0] = fmaf(dsp, bf16_lo(qv.x), a8[0]); a8[1] = fmaf(dsp, bf16_hi(qv.x), a8[1]);
                 a8[2] = fmaf(dsp, bf16_lo(qv.y), a8[2]); a8[3] = fmaf(dsp, bf16_hi(qv.y), a8[3]);
@@ -237,6 +252,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             s_row[st * 128 + myr] = myrow;
             s_w[st * 128 + myr] = myw;
             s_del[st * 128 + myr] = mydel;
+            if constexpr (QSLC) s_slot[st * 128 + myr] = myslot;
             const uint32_t sq = sb + SM::STG + st * SM::QD;
 #pragma unroll
             for (int k = 0; k < ITER; ++k) {  // padding rows (token -1) are zero-filled
@@ -276,7 +292,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             {  // the next tile's metadata while the copies run
                 BtCursor nx = cur;
                 nx.next();
-                fetch(nx, myrow, myw, mydel);
+                fetch(nx, myrow, myw, mydel, myslot);
             }
             // publish this tile as soon as its copies have landed: the next stage frees only after the
             // previous tile's gradient MMAs, so waiting for it first would serialise the tiles
@@ -415,6 +431,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             }
             const float g = (g4[0] + g4[1]) + (g4[2] + g4[3]);
             const float ds = row >= 0 ? w * (g - del) : 0.0f;
+            if (QSLC && row >= 0) ds_pair[(size_t)row * Kslots + s_slot[b * 128 + r]] = ds;
             // w P and dS into shared memory once the previous tile's dQ / dK / dV MMAs have read them
             ok = tc::mbar_wait(bar(kBDsEmpty), ((uint32_t)j & 1u) ^ 1u);
             if (!ok) break;
@@ -462,7 +479,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             if (!ok) break;
             tc::fence_after();
             const int row = e_row[slot * 128 + r];
-            const float ds = e_ds[slot * 128 + r];
+            const float ds = QSLC ? 0.0f : e_ds[slot * 128 + r];  // the ds L_c term belongs to dQ only without Qs
             const float *Lr = s_L + (cur.k & 3) * 128;  // published with e_ready
 #pragma unroll 1
             for (int cb = 0; cb < 64 / (int)SM::SLAB; ++cb) {
@@ -523,7 +540,8 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
 cudaError_t launch_backward_tc(const BackwardArgs &a, cudaStream_t s) {
     if (a.D != BtSmem::D) return cudaErrorInvalidValue;
     const size_t smem = BtSmem::DYN;
-    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = a.Qs ? chunk_bwd_tc_kernel<true> : chunk_bwd_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const uint64_t rows = (uint64_t)a.B * a.H * a.T;
     CUtensorMap tk, tv;
@@ -533,9 +551,9 @@ cudaError_t launch_backward_tc(const BackwardArgs &a, cudaStream_t s) {
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = sms < a.max_tiles ? sms : a.max_tiles;
     HSA_PROF("chunk_bwd", s);
-    chunk_bwd_tc_kernel<<<grid, kBtThreads, smem, s>>>(a.Q, a.L, a.dout, a.delta, a.T, a.N, a.scale, a.tiles,
-                                                       a.num_tiles, a.pair_row, a.pair_w, a.dQ, a.dK, a.dV, a.dL,
-                                                       a.err, tk, tv);
+    kern<<<grid, kBtThreads, smem, s>>>(a.Q, a.L, a.dout, a.delta, a.T, a.N, a.scale, a.tiles, a.num_tiles,
+                                        a.pair_row, a.pair_w, a.dQ, a.dK, a.dV, a.dL, a.err, a.Qs, a.pair_slot,
+                                        a.ds_pair, a.topk, tk, tv);
     return cudaGetLastError();
 }
 

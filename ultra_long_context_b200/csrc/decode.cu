@@ -379,7 +379,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         {
             HSA_PROF("decode_scan", s);
-            decode_scan_kernel<128><<<g1, kDecodeThreads, smem, s>>>(a.q, a.Lc, a.cache_len, a.H, a.Nmax, split,
+            decode_scan_kernel<128><<<g1, kDecodeThreads, smem, s>>>(a.qs, a.Lc, a.cache_len, a.H, a.Nmax, split,
                                                                      nsplit, a.K, a.scale, a.cand, a.counters,
                                                                      a.sel_idx, a.sel_w);
         }
@@ -390,7 +390,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         {
             HSA_PROF("decode_scan", s);
-            decode_scan_kernel<64><<<g1, kDecodeThreads, smem, s>>>(a.q, a.Lc, a.cache_len, a.H, a.Nmax, split,
+            decode_scan_kernel<64><<<g1, kDecodeThreads, smem, s>>>(a.qs, a.Lc, a.cache_len, a.H, a.Nmax, split,
                                                                     nsplit, a.K, a.scale, a.cand, a.counters,
                                                                     a.sel_idx, a.sel_w);
         }

@@ -118,7 +118,7 @@ hsa_status hsa_decode_noalloc(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_b
     if (st != HSA_OK) return st;
     char *b = static_cast<char *>(base);
     hsa::DecodeArgs a{};
-    a.q = q; a.Kc = Kc; a.Vc = Vc; a.Lc = Lc; a.cache_len = cache_len;
+    a.qs = q; a.q = q; a.Kc = Kc; a.Vc = Vc; a.Lc = Lc; a.cache_len = cache_len;
     a.Tmax = Tmax; a.Nmax = Nmax;
     a.B = B; a.H = H; a.D = D; a.K = topk;
     a.scale = scale > 0.0f ? scale : 1.0f / sqrtf((float)D);

@@ -10,6 +10,7 @@
 namespace hsa {
 
 struct DecodeArgs {
+    const uint16_t *qs;  // retrieval query (scan); q attends
     const uint16_t *q, *Kc, *Vc, *Lc;
     const int64_t *cache_len;
     int64_t Tmax, Nmax;
@@ -36,6 +37,7 @@ struct PairTile {
 constexpr int kPairTile = 64;  // pairs per tile of the mma.sync kernels (backward)
 
 struct ForwardArgs {
+    const uint16_t *Qs;  // retrieval queries (scores, fusion weights); Q attends
     const uint16_t *Q, *K, *V, *L;
     int B, H, T, D, N, topk;
     float scale;
@@ -70,6 +72,9 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
                             int tile_pairs, bool counts_ready, cudaStream_t s);
 
 struct BackwardArgs {
+    const uint16_t *Qs;  // separate retrieval queries, or NULL when Q retrieves too
+    float *dQs;          // their gradient (the ds L_c terms), with Qs
+    float *ds_pair;      // [B*H*T, topk] workspace: ds per (token, slot), with Qs
     const uint16_t *Q, *K, *V, *L, *out, *dout;
     const int32_t *sel_idx;
     const float *sel_w;

@@ -337,7 +337,7 @@ static cudaError_t launch_st(const ForwardArgs &a, const CUtensorMap &tl, cudaSt
     if (e != cudaSuccess) return e;
     dim3 grid((a.T + kStRows - 1) / kStRows, a.B * a.H);
     HSA_PROF("score_topk", s);
-    score_topk_tc_kernel<D, K><<<grid, kStThreads, smem, s>>>(a.Q, a.T, a.N, a.scale, a.topk, a.sel_idx, a.sel_w,
+    score_topk_tc_kernel<D, K><<<grid, kStThreads, smem, s>>>(a.Qs, a.T, a.N, a.scale, a.topk, a.sel_idx, a.sel_w,
                                                               a.o_acc, a.chunk_count, a.err, tl);
     return cudaGetLastError();
 }

@@ -31,6 +31,11 @@ SIGNATURES = {
     "hsa_backward_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
     "hsa_backward": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _P],
                      _I),
+    "hsa_forward_qslc": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P], _I),
+    "hsa_decode_qslc": ([_P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P], _I),
+    "hsa_backward_qslc_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
+    "hsa_backward_qslc": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _P,
+                           _SZ, _P], _I),
     "hsa_profile_enable": ([_I], _I),
     "hsa_profile_summary": ([ctypes.c_char_p, _SZ], _I),
 }
@@ -121,14 +126,18 @@ def hsa_forward_workspace_size(B, H, T, D, chunk=64, topk=16):
 
 
 def hsa_forward(Q, K, V, L, topk, scale=0.0, chunk=64, out=None, sel_idx=None, sel_w=None, workspace=None,
-                stream=None, return_selection=True):
+                stream=None, return_selection=True, Qs=None):
     """HSA prefill forward. Q, K, V [B, H, T, D] bf16, L [B, H, T // 64, D] bf16 (CUDA).
 
+    Qs: separate retrieval queries [B, H, T, D] bf16 (hsa_forward_qslc: Qs scores the landmarks, Q
+    attends), or None when Q does both.
     Returns (out [B, H, T, D] bf16, sel_idx [B, H, T, topk] int32, sel_w [B, H, T, topk] fp32); the
     selection is None when ``return_selection`` is False and none was passed in.
     """
     B, H, T, D = Q.shape
     dev = Q.device
+    if Qs is not None:
+        _need(Qs, "Qs", torch.bfloat16, (B, H, T, D), dev)
     for n, t in (("Q", Q), ("K", K), ("V", V)):
         _need(t, n, torch.bfloat16, (B, H, T, D), dev)
     _need(L, "L", torch.bfloat16, (B, H, T // chunk, D), dev)
@@ -142,9 +151,14 @@ def hsa_forward(Q, K, V, L, topk, scale=0.0, chunk=64, out=None, sel_idx=None, s
     nbytes = hsa_forward_workspace_size(B, H, T, D, chunk, topk)
     ws = _workspace(nbytes, dev, workspace)
     wp, wn = _aligned(ws)
-    st = lib().hsa_forward(_ptr(Q), _ptr(K), _ptr(V), _ptr(L), B, H, T, D, chunk, topk, float(scale), _ptr(out),
-                           _ptr(sel_idx), _ptr(sel_w), wp, wn, _stream(dev, stream))
-    _check("hsa_forward", st)
+    if Qs is None:
+        st = lib().hsa_forward(_ptr(Q), _ptr(K), _ptr(V), _ptr(L), B, H, T, D, chunk, topk, float(scale), _ptr(out),
+                               _ptr(sel_idx), _ptr(sel_w), wp, wn, _stream(dev, stream))
+        _check("hsa_forward", st)
+    else:
+        st = lib().hsa_forward_qslc(_ptr(Qs), _ptr(Q), _ptr(K), _ptr(V), _ptr(L), B, H, T, D, chunk, topk,
+                                    float(scale), _ptr(out), _ptr(sel_idx), _ptr(sel_w), wp, wn, _stream(dev, stream))
+        _check("hsa_forward_qslc", st)
     return out, sel_idx, sel_w
 
 
@@ -153,15 +167,18 @@ def hsa_decode_workspace_size(B, H, Tmax, D, chunk=64, topk=16):
 
 
 def hsa_decode(q, Kc, Vc, Lc, cache_len, topk, scale=0.0, chunk=64, out=None, sel_idx=None, sel_w=None,
-               workspace=None, stream=None):
+               workspace=None, stream=None, qs=None):
     """HSA decode. q [B, H, D], Kc / Vc [B, H, Tmax, D], Lc [B, H, Tmax // 64, D] bf16; cache_len [B] int64.
 
+    qs: a separate retrieval query [B, H, D] bf16 (hsa_decode_qslc), or None when q does both.
     Returns (out [B, H, D] bf16, sel_idx [B, H, topk] int32, sel_w [B, H, topk] fp32).
     """
     B, H, D = q.shape
     Tmax = Kc.shape[2]
     dev = q.device
     _need(q, "q", torch.bfloat16, (B, H, D), dev)
+    if qs is not None:
+        _need(qs, "qs", torch.bfloat16, (B, H, D), dev)
     _need(Kc, "Kc", torch.bfloat16, (B, H, Tmax, D), dev)
     _need(Vc, "Vc", torch.bfloat16, (B, H, Tmax, D), dev)
     _need(Lc, "Lc", torch.bfloat16, (B, H, Tmax // chunk, D), dev)
@@ -175,9 +192,15 @@ def hsa_decode(q, Kc, Vc, Lc, cache_len, topk, scale=0.0, chunk=64, out=None, se
     nbytes = hsa_decode_workspace_size(B, H, Tmax, D, chunk, topk)
     ws = _workspace(nbytes, dev, workspace)
     wp, wn = _aligned(ws)
-    st = lib().hsa_decode(_ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Lc), _ptr(cache_len), Tmax, B, H, D, chunk, topk,
-                          float(scale), _ptr(out), _ptr(sel_idx), _ptr(sel_w), wp, wn, _stream(dev, stream))
-    _check("hsa_decode", st)
+    if qs is None:
+        st = lib().hsa_decode(_ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Lc), _ptr(cache_len), Tmax, B, H, D, chunk, topk,
+                              float(scale), _ptr(out), _ptr(sel_idx), _ptr(sel_w), wp, wn, _stream(dev, stream))
+        _check("hsa_decode", st)
+    else:
+        st = lib().hsa_decode_qslc(_ptr(qs), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Lc), _ptr(cache_len), Tmax, B, H, D,
+                                   chunk, topk, float(scale), _ptr(out), _ptr(sel_idx), _ptr(sel_w), wp, wn,
+                                   _stream(dev, stream))
+        _check("hsa_decode_qslc", st)
     return out, sel_idx, sel_w
 
 
@@ -211,12 +234,19 @@ def hsa_backward_workspace_size(B, H, T, D, chunk=64, topk=16):
     return int(lib().hsa_backward_workspace_size(B, H, T, D, chunk, topk))
 
 
+def hsa_backward_qslc_workspace_size(B, H, T, D, chunk=64, topk=16):
+    return int(lib().hsa_backward_qslc_workspace_size(B, H, T, D, chunk, topk))
+
+
 def hsa_backward(Q, K, V, L, out, dout, sel_idx, sel_w, scale=0.0, chunk=64, grads=None, workspace=None,
-                 stream=None):
-    """Backward of hsa_forward for its selection. Returns (dQ, dK, dV, dL), fp32."""
+                 stream=None, Qs=None):
+    """Backward of hsa_forward for its selection. Returns (dQ, dK, dV, dL), fp32; with separate retrieval
+    queries Qs (hsa_backward_qslc), (dQ, dK, dV, dL, dQs) where dQ is the attention query's gradient."""
     B, H, T, D = Q.shape
     topk = sel_idx.shape[-1]
     dev = Q.device
+    if Qs is not None:
+        _need(Qs, "Qs", torch.bfloat16, (B, H, T, D), dev)
     for n, t in (("Q", Q), ("K", K), ("V", V), ("out", out), ("dout", dout)):
         _need(t, n, torch.bfloat16, (B, H, T, D), dev)
     _need(L, "L", torch.bfloat16, (B, H, T // chunk, D), dev)
@@ -227,15 +257,25 @@ def hsa_backward(Q, K, V, L, out, dout, sel_idx, sel_w, scale=0.0, chunk=64, gra
                  torch.empty((B, H, T, D), dtype=torch.float32, device=dev),
                  torch.empty((B, H, T, D), dtype=torch.float32, device=dev),
                  torch.empty((B, H, T // chunk, D), dtype=torch.float32, device=dev))
-    dQ, dK, dV, dL = grads
-    nbytes = hsa_backward_workspace_size(B, H, T, D, chunk, topk)
+    dQ, dK, dV, dL = grads[:4]
+    if Qs is None:
+        nbytes = hsa_backward_workspace_size(B, H, T, D, chunk, topk)
+        ws = _workspace(nbytes, dev, workspace)
+        wp, wn = _aligned(ws)
+        st = lib().hsa_backward(_ptr(Q), _ptr(K), _ptr(V), _ptr(L), _ptr(out), _ptr(dout), _ptr(sel_idx),
+                                _ptr(sel_w), B, H, T, D, chunk, topk, float(scale), _ptr(dQ), _ptr(dK), _ptr(dV),
+                                _ptr(dL) if dL.numel() else None, wp, wn, _stream(dev, stream))
+        _check("hsa_backward", st)
+        return dQ, dK, dV, dL
+    dQs = grads[4] if len(grads) > 4 else torch.empty((B, H, T, D), dtype=torch.float32, device=dev)
+    nbytes = hsa_backward_qslc_workspace_size(B, H, T, D, chunk, topk)
     ws = _workspace(nbytes, dev, workspace)
     wp, wn = _aligned(ws)
-    st = lib().hsa_backward(_ptr(Q), _ptr(K), _ptr(V), _ptr(L), _ptr(out), _ptr(dout), _ptr(sel_idx), _ptr(sel_w),
-                            B, H, T, D, chunk, topk, float(scale), _ptr(dQ), _ptr(dK), _ptr(dV),
-                            _ptr(dL) if dL.numel() else None, wp, wn, _stream(dev, stream))
-    _check("hsa_backward", st)
-    return dQ, dK, dV, dL
+    st = lib().hsa_backward_qslc(_ptr(Qs), _ptr(Q), _ptr(K), _ptr(V), _ptr(L), _ptr(out), _ptr(dout), _ptr(sel_idx),
+                                 _ptr(sel_w), B, H, T, D, chunk, topk, float(scale), _ptr(dQ), _ptr(dK), _ptr(dV),
+                                 _ptr(dL) if dL.numel() else None, _ptr(dQs), wp, wn, _stream(dev, stream))
+    _check("hsa_backward_qslc", st)
+    return dQ, dK, dV, dL, dQs
 
 
 def hsa_profile_enable(on=True):

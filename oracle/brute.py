@@ -11,13 +11,22 @@ import itertools
 import numpy as np
 
 
-def forward(Q, K, V, L, chunk, topk, scale, Qs=None):
-    """Q, K, V [B, H, T, D], L [B, H, N, D] -> (out [B,H,T,D], sel_idx [B,H,T,topk], sel_w [B,H,T,topk]).
+def forward(Q, K, V, L, chunk, topk, scale, Qs=None, qk_norm=False, eps=1e-6):
+    """Q [B, H, T, D], K, V [B, Hkv, T, D], L [B, Hkv, N, D] -> (out [B,H,T,D], sel_idx [B,H,T,topk],
+    sel_w [B,H,T,topk]).
 
-    Qs: separate retrieval queries (scores Qs . L), or None when Q also retrieves."""
+    Qs: separate retrieval queries (scores Qs . L), or None when Q also retrieves. Fewer key heads than
+    query heads: each key head is repeated for its H // Hkv consecutive query heads. qk_norm: Step 3
+    uses x / max(||x||, eps) for the query and the keys."""
     Q, K, V, L = (np.asarray(x, np.float64) for x in (Q, K, V, L))
     Qs = Q if Qs is None else np.asarray(Qs, np.float64)
     B, H, T, D = Q.shape
+    G = H // K.shape[1]
+    K, V, L = (np.repeat(x, G, axis=1) for x in (K, V, L))
+    Qa = Q
+    if qk_norm:
+        Qa = Q / np.maximum(np.linalg.norm(Q, axis=-1, keepdims=True), eps)
+        K = K / np.maximum(np.linalg.norm(K, axis=-1, keepdims=True), eps)
     N = T // chunk
     t = np.arange(T)
     admissible = (np.arange(N)[None, :] + 1) * chunk - 1 <= t[:, None]           # [T, N]
@@ -39,7 +48,7 @@ def forward(Q, K, V, L, chunk, topk, scale, Qs=None):
         np.put_along_axis(Wd[:, :, i, :], sel, e / e.sum(-1, keepdims=True), axis=-1)
     Kc = K[:, :, : N * chunk].reshape(B, H, N, chunk, D)
     Vc = V[:, :, : N * chunk].reshape(B, H, N, chunk, D)
-    A = scale * np.einsum("bhtd,bhnud->bhtnu", Q, Kc)                               # every query x every chunk
+    A = scale * np.einsum("bhtd,bhnud->bhtnu", Qa, Kc)                              # every query x every chunk
     P = np.exp(A - A.max(-1, keepdims=True))
     P /= P.sum(-1, keepdims=True)
     Obar = np.einsum("bhtnu,bhnud->bhtnd", P, Vc)

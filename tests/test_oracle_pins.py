@@ -356,10 +356,17 @@ def test_backward_matches_central_differences(oracle_mod):
         assert np.abs(g).max() > 0
 
 
-def dense_masked_hsa_torch(Q, K, V, L, sel_idx, chunk, scale, Qs=None):
+def dense_masked_hsa_torch(Q, K, V, L, sel_idx, chunk, scale, Qs=None, qk_norm=False):
     """HSA with a fixed selection as dense masked torch ops (every query x every chunk). Qs: separate
-    retrieval queries (the fusion weights come from Qs . L), or None when Q also retrieves."""
+    retrieval queries (the fusion weights come from Qs . L), or None when Q also retrieves. K, V, L with
+    fewer heads than Q are repeated over consecutive query heads (torch.repeat_interleave); qk_norm
+    attends with torch.nn.functional.normalize(., eps=1e-6) of the query and the keys."""
     B, H, T, D = Q.shape
+    G = H // K.shape[1]
+    K, V, L = (x.repeat_interleave(G, dim=1) for x in (K, V, L))
+    Qa = torch.nn.functional.normalize(Q, dim=-1, eps=1e-6) if qk_norm else Q
+    if qk_norm:
+        K = torch.nn.functional.normalize(K, dim=-1, eps=1e-6)
     N = L.shape[2]
     S = scale * torch.einsum("bhtd,bhnd->bhtn", Q if Qs is None else Qs, L)
     si = torch.as_tensor(sel_idx, dtype=torch.int64)
@@ -370,7 +377,7 @@ def dense_masked_hsa_torch(Q, K, V, L, sel_idx, chunk, scale, Qs=None):
     W = torch.where(M.any(-1, keepdim=True), W, torch.zeros_like(W))
     Kc = K[:, :, : N * chunk].reshape(B, H, N, chunk, D)
     Vc = V[:, :, : N * chunk].reshape(B, H, N, chunk, D)
-    P = torch.softmax(scale * torch.einsum("bhtd,bhnud->bhtnu", Q, Kc), dim=-1)
+    P = torch.softmax(scale * torch.einsum("bhtd,bhnud->bhtnu", Qa, Kc), dim=-1)
     Obar = torch.einsum("bhtnu,bhnud->bhtnd", P, Vc)
     return torch.einsum("bhtn,bhtnd->bhtd", W, Obar)
 
@@ -442,3 +449,130 @@ def test_separate_retrieval_query_backward_matches_torch_autograd(oracle_mod, T,
     for t_, g in zip(ts, grads):  # dQ (attention), dK, dV, dL, dQs (retrieval)
         np.testing.assert_allclose(g, t_.grad.numpy(), rtol=0, atol=1e-12)
         assert np.abs(g).max() > 0
+
+
+# ---------------------------------------------------------------------------------------------
+# Query-key normalisation (explainer, Step 3: the attention logits are norm(q_attn) . norm(K) / sqrt(d),
+# norm = L2 normalisation, as in the per-token procedure's l2norm(q_attn), l2norm(K)). Reading: the
+# retrieval scores of Step 2 stay unnormalised; norm(x) = x / max(||x||, 1e-6).
+
+
+def normalized(x):
+    return torch.nn.functional.normalize(torch.tensor(x, dtype=torch.float64), dim=-1, eps=1e-6).numpy()
+
+
+@pytest.mark.parametrize("B,H,T,D,chunk,topk", [(1, 2, 48, 8, 4, 3), (2, 1, 70, 16, 8, 2), (1, 2, 40, 4, 4, 20)])
+def test_qk_norm_matches_dense_brute_force(oracle_mod, B, H, T, D, chunk, topk):
+    Q, K, V, L = bf16_arrays(B, H, T, D, chunk, seed=13 + T + D)
+    scale = 1.0 / math.sqrt(D)
+    for Qs in (None, bf16_arrays(B, H, T, D, chunk, seed=17 + T)[0]):
+        r = oracle_mod.forward(Q, K, V, L, chunk=chunk, topk=topk, scale=scale, Qs=Qs, qk_norm=True)
+        out_b, idx_b, w_b = brute.forward(Q, K, V, L, chunk, topk, scale, Qs=Qs, qk_norm=True)
+        np.testing.assert_array_equal(r["sel_idx"].reshape(idx_b.shape), idx_b)
+        np.testing.assert_allclose(r["out"].reshape(out_b.shape), out_b, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(r["sel_w"].reshape(w_b.shape), w_b, rtol=0, atol=1e-13)
+
+
+def test_qk_norm_is_attention_on_normalised_inputs(oracle_mod):
+    """Normalising inside equals normalising the inputs first (torch's normalize) while the raw query
+    still retrieves; the selection is the raw query's."""
+    B, H, T, D, chunk, topk = 1, 2, 256, 16, 16, 4
+    Q, K, V, L = bf16_arrays(B, H, T, D, chunk, seed=23)
+    a = oracle_mod.forward(Q, K, V, L, chunk=chunk, topk=topk, qk_norm=True)
+    b = oracle_mod.forward(normalized(Q), normalized(K), V, L, chunk=chunk, topk=topk, Qs=Q)
+    np.testing.assert_array_equal(a["sel_idx"], b["sel_idx"])
+    np.testing.assert_allclose(a["out"], b["out"], rtol=0, atol=2e-6)  # the normalised inputs pass as float32
+    c = oracle_mod.forward(Q, K, V, L, chunk=chunk, topk=topk)
+    np.testing.assert_array_equal(a["sel_idx"], c["sel_idx"])
+    assert np.abs(a["out"] - c["out"]).max() > 1e-2
+
+
+def test_qk_norm_ignores_query_and_key_lengths(oracle_mod):
+    """Rescaling attention queries and keys by positive powers of two (exact in float) changes nothing
+    once they are normalised; the retrieval query is held fixed."""
+    B, H, T, D, chunk, topk = 1, 2, 128, 8, 8, 3
+    Q, K, V, L = bf16_arrays(B, H, T, D, chunk, seed=29)
+    rng = np.random.default_rng(3)
+    Q2 = Q * np.exp2(rng.integers(-3, 4, (B, H, T, 1))).astype(np.float32)
+    K2 = K * np.exp2(rng.integers(-3, 4, (B, H, T, 1))).astype(np.float32)
+    a = oracle_mod.forward(Q, K, V, L, chunk=chunk, topk=topk, Qs=Q, qk_norm=True)
+    b = oracle_mod.forward(Q2, K2, V, L, chunk=chunk, topk=topk, Qs=Q, qk_norm=True)
+    np.testing.assert_array_equal(a["sel_idx"], b["sel_idx"])
+    np.testing.assert_allclose(a["out"], b["out"], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("separate", [False, True])
+def test_qk_norm_backward_matches_torch_autograd(oracle_mod, separate):
+    B, H, T, D, chunk, topk = 2, 2, 96, 8, 8, 3
+    Q, K, V, L = bf16_arrays(B, H, T, D, chunk, seed=61)
+    K[0, 1, 20] *= np.float32(2.0 ** -40)  # a key shorter than eps: the other branch of the norm's gradient
+    Qs = bf16_arrays(B, H, T, D, chunk, seed=67)[0] if separate else None
+    G = np.random.default_rng(8).standard_normal((B, H, T, D)).astype(np.float32)
+    scale = 1.0 / math.sqrt(D)
+    sel = oracle_mod.forward(Q, K, V, L, chunk=chunk, topk=topk, Qs=Qs, qk_norm=True)["sel_idx"]
+    sel = sel.reshape(B, H, T, topk)
+    assert (sel == 2).any()  # chunk 2 holds the short key of head (0, 1)
+    ts = [torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (Q, K, V, L)]
+    qs_t = torch.tensor(Qs, dtype=torch.float64, requires_grad=True) if separate else None
+    out = dense_masked_hsa_torch(*ts, sel, chunk, scale, Qs=qs_t, qk_norm=True)
+    (out * torch.tensor(G, dtype=torch.float64)).sum().backward()
+    grads = oracle_mod.backward(Q, K, V, L, G, sel, chunk=chunk, scale=scale, Qs=Qs, qk_norm=True)
+    refs = ts + ([qs_t] if separate else [])
+    for t_, g in zip(refs, grads):
+        np.testing.assert_allclose(g, t_.grad.numpy(), rtol=1e-10, atol=1e-10)
+        assert np.abs(g).max() > 0
+
+
+# ---------------------------------------------------------------------------------------------
+# Grouped heads ("How to Improve It" #2: several query heads per key/value head). Reading: consecutive
+# query heads h share key head h // (H // Hkv), and each query head selects on its own.
+
+
+def repeat_heads(x, G):
+    return np.repeat(x, G, axis=1)
+
+
+@pytest.mark.parametrize("H,Hkv", [(4, 2), (4, 1), (6, 3)])
+def test_grouped_heads_equal_repeated_heads(oracle_mod, H, Hkv):
+    B, T, D, chunk, topk = 2, 100, 8, 8, 3
+    Q = bf16_arrays(B, H, T, D, chunk, seed=71)[0]
+    _, K, V, L = bf16_arrays(B, Hkv, T, D, chunk, seed=73)
+    G = H // Hkv
+    Kr, Vr, Lr = repeat_heads(K, G), repeat_heads(V, G), repeat_heads(L, G)
+    for qk_norm in (False, True):
+        a = oracle_mod.forward(Q, K, V, L, chunk=chunk, topk=topk, qk_norm=qk_norm)
+        b = oracle_mod.forward(Q, Kr, Vr, Lr, chunk=chunk, topk=topk, qk_norm=qk_norm)
+        for key in ("out", "sel_idx", "sel_w"):
+            np.testing.assert_array_equal(a[key], b[key])
+        dO = np.random.default_rng(4).standard_normal(Q.shape).astype(np.float32)
+        sel = a["sel_idx"].reshape(B, H, T, topk)
+        ga = oracle_mod.backward(Q, K, V, L, dO, sel, chunk=chunk, qk_norm=qk_norm)
+        gb = oracle_mod.backward(Q, Kr, Vr, Lr, dO, sel, chunk=chunk, qk_norm=qk_norm)
+        np.testing.assert_allclose(ga[0], gb[0], rtol=0, atol=1e-12)
+        for x, y in zip(ga[1:], gb[1:]):  # a key head's gradient is the sum over its query heads
+            np.testing.assert_allclose(x, y.reshape(B, Hkv, G, *y.shape[2:]).sum(2), rtol=0, atol=1e-12)
+    q = Q[:, :, -1]
+    lens = np.array([T, 37])
+    s1 = oracle_mod.decode_select(q, L, lens, chunk=chunk, topk=topk)
+    s2 = oracle_mod.decode_select(q, Lr, lens, chunk=chunk, topk=topk)
+    for key in s1:
+        np.testing.assert_array_equal(s1[key], s2[key])
+
+
+@pytest.mark.parametrize("T,chunk,topk", [(96, 8, 3), (70, 8, 20)])
+def test_grouped_heads_match_brute_force_and_autograd(oracle_mod, T, chunk, topk):
+    B, H, Hkv, D = 1, 4, 2, 8
+    Q = bf16_arrays(B, H, T, D, chunk, seed=79)[0]
+    _, K, V, L = bf16_arrays(B, Hkv, T, D, chunk, seed=83)
+    scale = 1.0 / math.sqrt(D)
+    r = oracle_mod.forward(Q, K, V, L, chunk=chunk, topk=topk, scale=scale)
+    out_b, idx_b, w_b = brute.forward(Q, K, V, L, chunk, topk, scale)
+    np.testing.assert_array_equal(r["sel_idx"].reshape(idx_b.shape), idx_b)
+    np.testing.assert_allclose(r["out"].reshape(out_b.shape), out_b, rtol=0, atol=1e-12)
+    G = np.random.default_rng(10).standard_normal(Q.shape).astype(np.float32)
+    sel = r["sel_idx"].reshape(B, H, T, topk)
+    ts = [torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (Q, K, V, L)]
+    out = dense_masked_hsa_torch(*ts, sel, chunk, scale)
+    (out * torch.tensor(G, dtype=torch.float64)).sum().backward()
+    for t_, g in zip(ts, oracle_mod.backward(Q, K, V, L, G, sel, chunk=chunk, scale=scale)):
+        np.testing.assert_allclose(g, t_.grad.numpy(), rtol=0, atol=1e-12)

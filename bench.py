@@ -297,6 +297,8 @@ def main():
     ap.add_argument("--skip-decode", action="store_true")
     ap.add_argument("--skip-backward", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--skip-options", action="store_true",
+                    help="skip the timings of the optional paths (query-key norm, separate retrieval query)")
     ap.add_argument("--decode-cache-len", type=int, default=None,
                     help="override the decode cache length (small cases for profiling)")
     args = ap.parse_args()
@@ -377,6 +379,38 @@ def main():
         del hQ, hK, hV, hL, hout, dQ_, dK_, dV_, dL_
 
     extra = {}
+    # ---------------- optional paths on the same 32K workload ----------------
+    if not args.skip_prefill and not args.skip_options:
+        osteps = max(3, args.steps // 2)
+        opts = {}
+        ws_n = torch.empty(hsa.hsa_forward_ex_workspace_size(w.B, w.H, w.H, w.T, w.D, w.chunk, w.topk,
+                                                             hsa.HSA_QK_NORM) + 256, dtype=torch.uint8, device=dev)
+
+        def fwd_norm():
+            hsa.hsa_forward(Q, K, V, L, w.topk, out=out, sel_idx=sel_idx, sel_w=sel_w, workspace=ws_n, qk_norm=True)
+
+        n_ms = timed(fwd_norm, osteps, args.warmup, world) / osteps
+        prof_n = kernel_profile(fwd_norm, osteps)
+        norm_bytes = 2 * (2 * w.B * w.H * w.T * w.D * 2)  # read Q and K, write their normalised copies
+        opts["qk_norm"] = {
+            "ms_per_step": round(n_ms, 4), "tokens_per_s": round(whole_job_rate(w.B * w.T, world, n_ms), 1),
+            "vs_plain": round(n_ms / ms_per_step, 4),
+            "roofline": roofline_entry("qk_norm", prof_n, norm_bytes, "GB/s", peaks["hbm_gbs"], "hbm",
+                                       f"{peak_kind} hbm_gbs"),
+        }
+        Qs_ = inputs.forward_inputs(w.B, w.H, w.T, w.D, w.seed + 7 + rank, landmarks=w.landmarks, device=dev)[0]
+
+        def fwd_qs():
+            hsa.hsa_forward(Q, K, V, L, w.topk, out=out, sel_idx=sel_idx, sel_w=sel_w, workspace=ws, Qs=Qs_)
+
+        s_ms = timed(fwd_qs, osteps, args.warmup, world) / osteps
+        opts["separate_retrieval_query"] = {
+            "ms_per_step": round(s_ms, 4), "tokens_per_s": round(whole_job_rate(w.B * w.T, world, s_ms), 1),
+            "vs_plain": round(s_ms / ms_per_step, 4)}
+        extra["fwd_options"] = dict(workload=w.name, steps=osteps, **opts)
+        del ws_n, Qs_
+        torch.cuda.empty_cache()
+
     # ---------------- decode, 16M-token cache ----------------
     if not args.skip_decode:
         wd = inputs.WORKLOADS["decode_16m_b1_h8_d128_k32"]
@@ -447,6 +481,25 @@ def main():
                                        f"{peak_kind} bf16_tflops_sustained", TRAFFIC_BYTES.get((wb.name, "chunk_bwd"))),
             "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_b.items()},
         }
+        if not args.skip_options:  # the same step with query-key normalisation
+            fws_n = torch.empty(hsa.hsa_forward_ex_workspace_size(wb.B, wb.H, wb.H, wb.T, wb.D, 64, wb.topk,
+                                                                  hsa.HSA_QK_NORM) + 256, dtype=torch.uint8,
+                                device=dev)
+            bws_n = torch.empty(hsa.hsa_backward_ex_workspace_size(wb.B, wb.H, wb.H, wb.T, wb.D, 64, wb.topk,
+                                                                   hsa.HSA_QK_NORM) + 256, dtype=torch.uint8,
+                                device=dev)
+
+            def fwdbwd_norm():
+                hsa.hsa_forward(bQ, bK, bV, bL, wb.topk, out=bout, sel_idx=bidx, sel_w=bw, workspace=fws_n,
+                                qk_norm=True)
+                hsa.hsa_backward(bQ, bK, bV, bL, bout, bdO, bidx, bw, grads=grads, workspace=bws_n, qk_norm=True)
+
+            nms = timed(fwdbwd_norm, bsteps, args.warmup, world) / bsteps
+            prof_bn = kernel_profile(fwdbwd_norm, bsteps)
+            extra["fwdbwd_64k"]["qk_norm"] = {
+                "ms_per_step": round(nms, 4), "vs_plain": round(nms / bms, 4),
+                "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_bn.items()}}
+            del fws_n, bws_n
         del bQ, bK, bV, bL, bdO, fws, bws, grads
         torch.cuda.empty_cache()
     clk = clocks.stop()

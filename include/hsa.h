@@ -23,7 +23,8 @@
  *   - ties: equal scores keep ascending chunk order (lower chunk index wins);
  *   - one query serves both as retrieval query and attention query; one scale serves both
  *     (scale <= 0 selects 1/sqrt(D)); no query-key normalisation and no positional encoding
- *     are applied (inputs are used as given);
+ *     are applied (inputs are used as given). The *_ex entry points at the end add a separate
+ *     retrieval query, query-key normalisation and grouped key/value heads;
  *   - selection itself carries no gradient; the landmarks receive gradient through the selected
  *     scores only (Step 4: w multiplies the output, so the loss reaches s).
  *
@@ -158,34 +159,56 @@ hsa_status hsa_backward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
                         float *dV, float *dL, void *workspace, size_t workspace_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------------------------
- * Separate retrieval query. Explainer of "Every Token Counts", "How It Works (Technically)" Steps 2-3,
- * and the per-token procedure in "The algorithm, simplified": the query that scores the landmarks
- * (q_slc) and the query that attends inside the selected chunks (q_attn) are separate projections.
- * These entry points take both: Qs / qs [same shape as Q / q] retrieve (Step 2 scores and the Step 4
- * fusion weights come from Qs . L), Q / q attend (Step 3). Everything else -- shapes, layouts,
- * ownership, workspace rules, error behaviour, outputs -- is as for the single-query calls above;
- * with Qs == Q they compute the same result.
- * hsa_backward_qslc writes dQ (the attention query's gradient: the dS K_c terms only) and dQs (the
- * retrieval query's: the ds L_c terms), both fp32 [B, H, T, D], zero-initialised by the call; its
- * workspace (hsa_backward_qslc_workspace_size) also holds ds for every (token, slot).
+ * Extended entry points: a separate retrieval query, query-key normalisation, grouped key heads.
+ *
+ * Same operation, shapes, layouts, ownership, workspace rules, error behaviour and outputs as the
+ * calls above, with three additions. Each is off when its argument takes the value shown in brackets,
+ * and then the result is that of the plain call.
+ *
+ *   Qs / qs [NULL]   separate retrieval query, shaped like Q / q. Explainer of "Every Token Counts",
+ *                    "How It Works (Technically)" Steps 2-3 and the per-token procedure in "The
+ *                    algorithm, simplified": the query that scores the landmarks (q_slc) and the query
+ *                    that attends inside the selected chunks (q_attn) are separate projections. Qs gives
+ *                    the Step 2 scores, the top-K and the Step 4 fusion weights; Q attends in Step 3.
+ *   flags & HSA_QK_NORM [0]   query-key normalisation (Step 3: the in-chunk logits are
+ *                    norm(q_attn) . norm(K_c)^T * scale, norm = L2 normalisation, as in the
+ *                    procedure's l2norm calls). Reading: norm(x) = x / max(||x||_2, 1e-6) per row; the
+ *                    retrieval scores (Step 2) are not normalised. The prefill forward and backward
+ *                    normalise Q and K into bf16 copies in the workspace; the decode normalises in fp32
+ *                    on the fly.
+ *   Hkv [H]          grouped heads ("How to Improve It" #2: several query heads per key/value head):
+ *                    K, V, L (Kc, Vc, Lc) have Hkv heads, H a multiple of Hkv, and query head h uses
+ *                    head h / (H / Hkv). Each query head still selects its own chunks.
+ *                    Shapes: K, V [B, Hkv, T, D], L [B, Hkv, T/64, D]; dK, dV, dL likewise.
+ *
+ * Unknown flag bits give HSA_ERR_INVALID_ARG. hsa_backward_ex writes dQ (the attention query's
+ * gradient, taken back through the normalisation when it is on) and, when Qs is given, dQs (the
+ * retrieval query's gradient) -- both fp32 [B, H, T, D] and overwritten; without Qs, dQ holds both
+ * parts and dQs must be NULL. The *_ex_workspace_size functions take the same Hkv and flags.
  * -------------------------------------------------------------------------------------------*/
-hsa_status hsa_forward_qslc(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
-                            const hsa_bf16 *L, int B, int H, int T, int D, int chunk, int topk, float scale,
-                            hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace, size_t workspace_bytes,
-                            void *stream);
+#define HSA_QK_NORM 1u
 
-hsa_status hsa_decode_qslc(const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
-                           const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B, int H, int D,
-                           int chunk, int topk, float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w,
-                           void *workspace, size_t workspace_bytes, void *stream);
+size_t hsa_forward_ex_workspace_size(int B, int H, int Hkv, int T, int D, int chunk, int topk, unsigned flags);
 
-size_t hsa_backward_qslc_workspace_size(int B, int H, int T, int D, int chunk, int topk);
+hsa_status hsa_forward_ex(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
+                          const hsa_bf16 *L, int B, int H, int Hkv, int T, int D, int chunk, int topk, float scale,
+                          unsigned flags, hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace,
+                          size_t workspace_bytes, void *stream);
 
-hsa_status hsa_backward_qslc(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
-                             const hsa_bf16 *L, const hsa_bf16 *out, const hsa_bf16 *dout, const int32_t *sel_idx,
-                             const float *sel_w, int B, int H, int T, int D, int chunk, int topk, float scale,
-                             float *dQ, float *dK, float *dV, float *dL, float *dQs, void *workspace,
-                             size_t workspace_bytes, void *stream);
+size_t hsa_decode_ex_workspace_size(int B, int H, int Hkv, int64_t Tmax, int D, int chunk, int topk, unsigned flags);
+
+hsa_status hsa_decode_ex(const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
+                         const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B, int H, int Hkv, int D,
+                         int chunk, int topk, float scale, unsigned flags, hsa_bf16 *out, int32_t *sel_idx,
+                         float *sel_w, void *workspace, size_t workspace_bytes, void *stream);
+
+size_t hsa_backward_ex_workspace_size(int B, int H, int Hkv, int T, int D, int chunk, int topk, unsigned flags);
+
+hsa_status hsa_backward_ex(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
+                           const hsa_bf16 *L, const hsa_bf16 *out, const hsa_bf16 *dout, const int32_t *sel_idx,
+                           const float *sel_w, int B, int H, int Hkv, int T, int D, int chunk, int topk, float scale,
+                           unsigned flags, float *dQ, float *dK, float *dV, float *dL, float *dQs, void *workspace,
+                           size_t workspace_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------------------------
  * Measurement hooks (no counterpart on the pages; used to time each kernel live).

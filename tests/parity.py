@@ -15,11 +15,12 @@ OUT_MEAN_ABS = 2e-3
 W_MAX_ABS = 1e-3
 
 
-def compare_forward_rows(oracle_mod, gpu_out, gpu_idx, gpu_w, orc, Q, K, V, L, rows, chunk, scale, Qs=None):
+def compare_forward_rows(oracle_mod, gpu_out, gpu_idx, gpu_w, orc, Q, K, V, L, rows, chunk, scale, Qs=None,
+                         qk_norm=False):
     """gpu_* and orc[...] are per-row arrays aligned with ``rows`` (flat (b*H+h)*T+t ids).
 
     Q, K, V, L: float32 host arrays [B, H, T, D] / [B, H, N, D] (needed for tie rows only); Qs: the
-    separate retrieval queries when there are any (they decide the ties).
+    separate retrieval queries when there are any (they decide the ties); qk_norm as in the oracle.
     Returns a dict of statistics; raises AssertionError on a violation.
     """
     gpu_out = np.asarray(gpu_out, np.float64)
@@ -58,6 +59,7 @@ def compare_forward_rows(oracle_mod, gpu_out, gpu_idx, gpu_w, orc, Q, K, V, L, r
     # tie rows: validity of the GPU set, then its output against the oracle on that set
     if tie_rows:
         B, H, T, D = Q.shape
+        G = H // K.shape[1]  # query heads per key head
         rr = np.asarray([rows[i] for i in tie_rows])
         S = oracle_mod.scores(Q if Qs is None else Qs, L, rr, chunk=chunk, scale=scale)
         topk = gpu_idx.shape[1]
@@ -68,17 +70,18 @@ def compare_forward_rows(oracle_mod, gpu_out, gpu_idx, gpu_w, orc, Q, K, V, L, r
         Qr = Q.reshape(-1, D)[rr]
         for n, i in enumerate(tie_rows):
             bh = rows[i] // T
+            b, hk = bh // H, (bh % H) // G
             k = len([c for c in orc["sel_idx"][i] if c >= 0])
             s_k = orc["sel_s"][i, k - 1]
             kept = [int(c) for c in gpu_idx[i] if c >= 0]
             for j, c in enumerate(kept):
                 assert S[n, c] >= s_k - TIE, f"row {rows[i]}: chunk {c} is not a near-tie choice"
-                Lg[n, j] = L[bh // H, bh % H, c]
-                Kg[n, j] = K[bh // H, bh % H, c * chunk:(c + 1) * chunk]
-                Vg[n, j] = V[bh // H, bh % H, c * chunk:(c + 1) * chunk]
+                Lg[n, j] = L[b, hk, c]
+                Kg[n, j] = K[b, hk, c * chunk:(c + 1) * chunk]
+                Vg[n, j] = V[b, hk, c * chunk:(c + 1) * chunk]
             nsel[n] = len(kept)
         Qsr = None if Qs is None else Qs.reshape(-1, D)[rr]
-        o, _ = oracle_mod.attend_gathered(Qr, Lg, Kg, Vg, nsel, scale=scale, qs=Qsr)
+        o, _ = oracle_mod.attend_gathered(Qr, Lg, Kg, Vg, nsel, scale=scale, qs=Qsr, qk_norm=qk_norm)
         dt = np.abs(gpu_out[tie_rows] - o)
         assert dt.max() <= OUT_MAX_ABS, f"tie rows max-abs {dt.max():.4g}"
     return stats

@@ -100,3 +100,54 @@ def test_workspace_status_rejects_null_on_host():
     """hsa_workspace_status validates its argument before touching the device."""
     assert hsa.lib().hsa_workspace_status(None, None) == -1
     assert "workspace" in hsa.hsa_last_error()
+
+
+def _fwd_ex(**kw):
+    args = dict(Qs=None, Q=FAKE, K=FAKE, V=FAKE, L=FAKE, B=1, H=4, Hkv=4, T=256, D=64, chunk=64, topk=8, scale=0.0,
+                flags=0, out=FAKE, sel_idx=None, sel_w=None, ws=FAKE, ws_bytes=1 << 40, stream=None)
+    args.update(kw)
+    return hsa.lib().hsa_forward_ex(*args.values())
+
+
+def _bwd_ex(**kw):
+    args = dict(Qs=None, Q=FAKE, K=FAKE, V=FAKE, L=FAKE, out=FAKE, dout=FAKE, sel_idx=FAKE, sel_w=FAKE, B=1, H=4,
+                Hkv=4, T=256, D=128, chunk=64, topk=16, scale=0.0, flags=0, dQ=FAKE, dK=FAKE, dV=FAKE, dL=FAKE,
+                dQs=None, ws=FAKE, ws_bytes=1 << 40, stream=None)
+    args.update(kw)
+    return hsa.lib().hsa_backward_ex(*args.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(flags=2), -1), (dict(flags=0x80000000), -1), (dict(Hkv=3), -1), (dict(Hkv=0), -1), (dict(Hkv=8), -1),
+    (dict(Qs=ODD), -1), (dict(D=96), -2), (dict(ws_bytes=100, flags=1), -3),
+])
+def test_forward_ex_rejects_invalid_calls_on_host(kw, status):
+    assert _fwd_ex(**kw) == status
+    assert hsa.hsa_last_error() != ""
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Qs=FAKE), -1), (dict(dQs=FAKE), -1), (dict(flags=4), -1), (dict(Hkv=5), -1), (dict(ws=None, flags=1), -3),
+])
+def test_backward_ex_rejects_invalid_calls_on_host(kw, status):
+    assert _bwd_ex(**kw) == status
+
+
+def test_decode_ex_rejects_invalid_calls_on_host():
+    args = dict(qs=None, q=FAKE, Kc=FAKE, Vc=FAKE, Lc=FAKE, cache_len=FAKE, Tmax=1 << 20, B=2, H=2, Hkv=2, D=128,
+                chunk=64, topk=16, scale=0.0, flags=8, out=FAKE, sel_idx=None, sel_w=None, ws=FAKE, ws_bytes=1 << 40,
+                stream=None)
+    assert hsa.lib().hsa_decode_ex(*args.values()) == -1
+    args.update(flags=1, Hkv=3)
+    assert hsa.lib().hsa_decode_ex(*args.values()) == -1
+
+
+def test_ex_workspace_sizes_cover_the_options():
+    base = hsa.hsa_forward_workspace_size(1, 4, 4096, 128, 64, 16)
+    assert hsa.hsa_forward_ex_workspace_size(1, 4, 4, 4096, 128, 64, 16, 0) == base
+    # query-key normalisation keeps bf16 copies of Q and K
+    assert hsa.hsa_forward_ex_workspace_size(1, 4, 4, 4096, 128, 64, 16, 1) >= base + 2 * 4 * 4096 * 128 * 2
+    assert hsa.hsa_backward_ex_workspace_size(1, 4, 4, 4096, 128, 64, 16, 0) >= \
+        hsa.hsa_backward_workspace_size(1, 4, 4096, 128, 64, 16) + 4 * 4096 * 16 * 4  # ds per pair
+    assert hsa.hsa_decode_ex_workspace_size(1, 8, 8, 1 << 20, 128, 64, 32, 1) == \
+        hsa.hsa_decode_workspace_size(1, 8, 1 << 20, 128, 64, 32)

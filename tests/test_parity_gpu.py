@@ -97,11 +97,12 @@ def test_forward_is_deterministic_in_selection_and_close_in_output():
 # decode
 
 
-def oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, chunk=64, qs=None):
+def oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, chunk=64, qs=None, qk_norm=False, scale=None):
     """Oracle decode: selection from (q or qs, Lc) on the host, then the selected chunks gathered."""
     B, H, D = q.shape
+    scale = scale or 1 / math.sqrt(D)
     sel = oracle_mod.decode_select(host(q if qs is None else qs), host(Lc), lens.cpu().numpy(), chunk=chunk, topk=topk,
-                                   scale=1 / math.sqrt(D))
+                                   scale=scale)
     idx = torch.as_tensor(sel["sel_idx"], device=Kc.device, dtype=torch.int64).clamp(min=0)   # [B,H,k]
     tok = (idx[..., None] * chunk + torch.arange(chunk, device=Kc.device)).reshape(B, H, -1)
     Kg = torch.gather(Kc, 2, tok[..., None].expand(-1, -1, -1, D)).reshape(B * H, topk, chunk, D)
@@ -109,17 +110,17 @@ def oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, chunk=64, qs=None):
     Lg = torch.gather(Lc, 2, idx[..., None].expand(-1, -1, -1, D)).reshape(B * H, topk, D)
     nsel = (sel["sel_idx"] >= 0).sum(-1).reshape(-1)
     out, w = oracle_mod.attend_gathered(host(q).reshape(B * H, D), host(Lg), host(Kg), host(Vg), nsel,
-                                        scale=1 / math.sqrt(D),
+                                        scale=scale, qk_norm=qk_norm,
                                         qs=None if qs is None else host(qs).reshape(B * H, D))
     return dict(out=out, sel_idx=sel["sel_idx"].reshape(B * H, topk), sel_w=w, sel_s=sel["sel_s"].reshape(B * H, topk),
                 next_s=sel["next_s"].reshape(-1))
 
 
-def check_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, qs=None):
+def check_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, qs=None, qk_norm=False, scale=None):
     B, H, D = q.shape
-    out, idx, w = hsa.hsa_decode(q, Kc, Vc, Lc, lens, topk, qs=qs)
+    out, idx, w = hsa.hsa_decode(q, Kc, Vc, Lc, lens, topk, qs=qs, qk_norm=qk_norm, scale=scale or 0.0)
     torch.cuda.synchronize()
-    orc = oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, qs=qs)
+    orc = oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, qs=qs, qk_norm=qk_norm, scale=scale)
     g_idx = idx.reshape(B * H, topk).cpu().numpy()
     g_w = w.reshape(B * H, topk).cpu().numpy()
     g_out = host(out).reshape(B * H, D)
@@ -295,3 +296,67 @@ def test_backward_separate_retrieval_query_matches_oracle(oracle_mod, B, H, T, D
                               Qs=Qsh)
     for g, r, n in zip(grads, ref, ("dQ", "dK", "dV", "dL", "dQs")):
         grad_close(host(g), r, n)
+
+
+# ---------------------------------------------------------------------------------------------
+# query-key normalisation (Step 3 attends with norm(q) . norm(K_c)); scale 4 as well as 1/sqrt(D), since
+# unit vectors at 1/sqrt(D) give nearly uniform in-chunk weights
+
+
+@pytest.mark.parametrize("B,H,T,D,topk,scale,separate", [
+    (1, 2, 2048 + 37, 128, 16, 4.0, False), (1, 2, 2048 + 37, 128, 16, None, True),
+    (1, 2, 1100, 64, 8, 4.0, True), (2, 1, 700, 64, 5, None, False),
+])
+def test_forward_qk_norm_matches_oracle(oracle_mod, B, H, T, D, topk, scale, separate):
+    Q, K, V, L = inputs.forward_inputs(B, H, T, D, 1000 + T, device=DEV)
+    Qs = inputs.forward_inputs(B, H, T, D, 1100 + T, device=DEV)[0] if separate else None
+    sc = scale if scale else 1 / math.sqrt(D)
+    out, idx, w = hsa.hsa_forward(Q, K, V, L, topk, scale=sc, Qs=Qs, qk_norm=True)
+    Qh, Kh, Vh, Lh = (host(x) for x in (Q, K, V, L))
+    Qsh = host(Qs) if separate else None
+    orc = oracle_mod.forward(Qh, Kh, Vh, Lh, chunk=64, topk=topk, scale=sc, Qs=Qsh, qk_norm=True)
+    rows = np.arange(B * H * T)
+    compare_forward_rows(oracle_mod, host(out).reshape(-1, D), host(idx).reshape(-1, topk),
+                         host(w).reshape(-1, topk), orc, Qh, Kh, Vh, Lh, rows, 64, sc, Qs=Qsh, qk_norm=True)
+    plain = oracle_mod.forward(Qh, Kh, Vh, Lh, chunk=64, topk=topk, scale=sc, Qs=Qsh)
+    if scale:  # the normalisation changes the result well beyond the tolerance
+        assert np.abs(plain["out"] - orc["out"]).max() > 0.1
+
+
+@pytest.mark.parametrize("D,lens,topk,separate", [(128, [9000, 4100], 8, False), (64, [64 * 300 - 1, 640], 32, True)])
+def test_decode_qk_norm_matches_oracle(oracle_mod, D, lens, topk, separate):
+    B, H = len(lens), 2
+    q, Kc, Vc, Lc, lens_t, _ = inputs.decode_inputs(B, H, lens, D, seed=41 + D, Tmax=max(lens) + 64, device=DEV)
+    qs = inputs.decode_inputs(B, H, lens, D, seed=42 + D, Tmax=max(lens) + 64, device=DEV)[0] if separate else None
+    out, _, _ = check_decode(oracle_mod, q, Kc, Vc, Lc, lens_t, topk, qs=qs, qk_norm=True, scale=4.0)
+    plain, _, _ = hsa.hsa_decode(q, Kc, Vc, Lc, lens_t, topk, qs=qs, scale=4.0)
+    assert (out.float() - plain.float()).abs().max() > 0.1
+
+
+@pytest.mark.parametrize("B,H,T,D,topk,separate", [
+    (1, 2, 2048 + 64, 128, 16, False), (1, 2, 2048 + 64, 128, 16, True), (1, 2, 1100, 64, 8, False),
+    (1, 1, 1100, 64, 8, True),
+])
+def test_backward_qk_norm_matches_oracle(oracle_mod, B, H, T, D, topk, separate):
+    Q, K, V, L = inputs.forward_inputs(B, H, T, D, 1200 + T, device=DEV)
+    Qs = inputs.forward_inputs(B, H, T, D, 1300 + T, device=DEV)[0] if separate else None
+    dO = inputs.upstream_grad(B, H, T, D, 1200 + T, device=DEV)
+    Qh, Kh, Vh, Lh, dOh = (host(x) for x in (Q, K, V, L, dO))
+    Qsh = host(Qs) if separate else None
+    # the pages' scale: at much larger scales the fusion softmax saturates and ds = w (dO.O_c - dO.out)
+    # cancels down to the bf16 rounding of the stored output (the retrieval gradients lose relative
+    # accuracy with or without the normalisation)
+    sc = 1 / math.sqrt(D)
+    orc = oracle_mod.forward(Qh, Kh, Vh, Lh, chunk=64, topk=topk, scale=sc, Qs=Qsh, qk_norm=True)
+    sel_idx = torch.as_tensor(orc["sel_idx"].reshape(B, H, T, topk), device=DEV)
+    sel_w = torch.as_tensor(orc["sel_w"].reshape(B, H, T, topk), dtype=torch.float32, device=DEV)
+    out = torch.as_tensor(orc["out"].reshape(B, H, T, D), dtype=torch.float32, device=DEV).to(torch.bfloat16)
+    grads = hsa.hsa_backward(Q, K, V, L, out, dO, sel_idx, sel_w, scale=sc, Qs=Qs, qk_norm=True)
+    ref = oracle_mod.backward(Qh, Kh, Vh, Lh, dOh, orc["sel_idx"].reshape(B, H, T, topk), chunk=64, scale=sc,
+                              Qs=Qsh, qk_norm=True)
+    for g, r, n in zip(grads, ref, ("dQ", "dK", "dV", "dL", "dQs")):
+        grad_close(host(g), r, n)
+    plain = oracle_mod.backward(Qh, Kh, Vh, Lh, dOh, orc["sel_idx"].reshape(B, H, T, topk), chunk=64, scale=sc,
+                                Qs=Qsh)
+    for x, y in zip(ref[:2], plain[:2]):  # dQ and dK: the normalisation's Jacobian matters
+        assert np.abs(x - y).sum() > 0.5 * np.abs(x).sum()

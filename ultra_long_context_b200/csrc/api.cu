@@ -77,12 +77,16 @@ struct FwdLayout {
     int32_t *num_tiles, *err;
     float *delta;
     int32_t *pair_slot;
-    float *ds_pair;  // [B*H*T, topk] ds per (token, slot): separate retrieval query only
+    float *ds_pair;  // [B*H*T, topk] ds per (token, slot): separate retrieval query or query-key norm
+    uint16_t *Qn, *Kn;  // [B*H*T, D] bf16 normalised copies: query-key norm only
     size_t bytes;
     int max_tiles;
 };
 
-FwdLayout fwd_layout(void *ws, int B, int H, int T, int D, int topk, bool backward, bool qslc = false) {
+// qslc: the backward keeps ds per pair (a separate retrieval query, or the raw query retrieving while
+// the normalised one attends); qk_norm: room for the normalised copies of Q and K.
+FwdLayout fwd_layout(void *ws, int B, int H, int T, int D, int topk, bool backward, bool qslc = false,
+                     bool qk_norm = false) {
     FwdLayout l{};
     Carver c{static_cast<char *>(ws)};
     l.err = c.take<int32_t>(1);  // first: hsa_workspace_status reads it at offset 0
@@ -101,7 +105,9 @@ FwdLayout fwd_layout(void *ws, int B, int H, int T, int D, int topk, bool backwa
     l.num_tiles = c.take<int32_t>(1);
     l.delta = backward ? c.take<float>(rows) : nullptr;
     l.pair_slot = backward ? c.take<int32_t>(pairs) : nullptr;
-    l.ds_pair = backward && qslc ? c.take<float>(pairs) : nullptr;
+    l.ds_pair = backward && (qslc || qk_norm) ? c.take<float>(pairs) : nullptr;
+    l.Qn = qk_norm ? c.take<uint16_t>(rows * D) : nullptr;
+    l.Kn = qk_norm ? c.take<uint16_t>(rows * D) : nullptr;
     l.bytes = c.used;
     return l;
 }
@@ -134,6 +140,15 @@ DecLayout dec_layout(void *ws, int B, int H, int64_t Tmax, int D, int topk) {
 
 float resolve_scale(float scale, int D) { return scale > 0.0f ? scale : 1.0f / sqrtf((float)D); }
 
+// Checks of the *_ex arguments shared by the three calls.
+hsa_status check_ex(int H, int Hkv, unsigned flags) {
+    if (flags & ~HSA_QK_NORM) return fail(HSA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags & ~HSA_QK_NORM);
+    if (Hkv < 1 || H % Hkv != 0)
+        return fail(HSA_ERR_INVALID_ARG, "H (%d) must be a positive multiple of Hkv (%d)", H, Hkv);
+    if (Hkv != H) return fail(HSA_ERR_UNSUPPORTED, "grouped key/value heads (Hkv < H) are not implemented yet");
+    return HSA_OK;
+}
+
 }  // namespace
 
 namespace hsa {
@@ -165,11 +180,17 @@ size_t hsa_forward_workspace_size(int B, int H, int T, int D, int chunk, int top
     return fwd_layout(nullptr, B, H, T, D, topk, false).bytes;
 }
 
+size_t hsa_forward_ex_workspace_size(int B, int H, int Hkv, int T, int D, int chunk, int topk, unsigned flags) {
+    (void)chunk;
+    if (B < 1 || H < 1 || Hkv < 1 || T < 1 || D < 1 || topk < 1) return 0;
+    return fwd_layout(nullptr, B, H, T, D, topk, false, false, (flags & HSA_QK_NORM) != 0).bytes;
+}
+
 // Qs retrieves (Step 2 scores, Step 4 weights), Q attends (Step 3); the single-query call passes Q twice.
 static hsa_status forward_impl(const char *name, const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K,
                                const hsa_bf16 *V, const hsa_bf16 *L, int B, int H, int T, int D, int chunk, int topk,
-                               float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace,
-                               size_t workspace_bytes, void *stream) {
+                               float scale, bool qk_norm, hsa_bf16 *out, int32_t *sel_idx, float *sel_w,
+                               void *workspace, size_t workspace_bytes, void *stream) {
     g_last_error.clear();
     hsa_status st = check_common(B, H, D, chunk, topk, 32);
     if (st != HSA_OK) return st;
@@ -182,10 +203,11 @@ static hsa_status forward_impl(const char *name, const hsa_bf16 *Qs, const hsa_b
         return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
     if ((sel_idx && !aligned16(sel_idx)) || (sel_w && !aligned16(sel_w)))
         return fail(HSA_ERR_INVALID_ARG, "sel_idx / sel_w must be 16-byte aligned");
-    FwdLayout need = fwd_layout(nullptr, B, H, T, D, topk, false);
+    FwdLayout need = fwd_layout(nullptr, B, H, T, D, topk, false, false, qk_norm);
     if ((st = check_ws(workspace, workspace_bytes, need.bytes)) != HSA_OK) return st;
-    FwdLayout l = fwd_layout(workspace, B, H, T, D, topk, false);
+    FwdLayout l = fwd_layout(workspace, B, H, T, D, topk, false, false, qk_norm);
     hsa::ForwardArgs a{};
+    a.qk_norm = qk_norm; a.Qn = l.Qn; a.Kn = l.Kn;
     a.Qs = Qs; a.Q = Q; a.K = K; a.V = V; a.L = L;
     a.B = B; a.H = H; a.T = T; a.D = D; a.N = T / 64; a.topk = topk;
     a.scale = resolve_scale(scale, D);
@@ -204,16 +226,19 @@ static hsa_status forward_impl(const char *name, const hsa_bf16 *Qs, const hsa_b
 hsa_status hsa_forward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, const hsa_bf16 *L, int B, int H,
                        int T, int D, int chunk, int topk, float scale, hsa_bf16 *out, int32_t *sel_idx,
                        float *sel_w, void *workspace, size_t workspace_bytes, void *stream) {
-    return forward_impl("hsa_forward", Q, Q, K, V, L, B, H, T, D, chunk, topk, scale, out, sel_idx, sel_w, workspace,
-                        workspace_bytes, stream);
+    return forward_impl("hsa_forward", Q, Q, K, V, L, B, H, T, D, chunk, topk, scale, false, out, sel_idx, sel_w,
+                        workspace, workspace_bytes, stream);
 }
 
-hsa_status hsa_forward_qslc(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
-                            const hsa_bf16 *L, int B, int H, int T, int D, int chunk, int topk, float scale,
-                            hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace, size_t workspace_bytes,
-                            void *stream) {
-    return forward_impl("hsa_forward_qslc", Qs, Q, K, V, L, B, H, T, D, chunk, topk, scale, out, sel_idx, sel_w,
-                        workspace, workspace_bytes, stream);
+hsa_status hsa_forward_ex(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
+                          const hsa_bf16 *L, int B, int H, int Hkv, int T, int D, int chunk, int topk, float scale,
+                          unsigned flags, hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace,
+                          size_t workspace_bytes, void *stream) {
+    g_last_error.clear();
+    hsa_status st = check_ex(H, Hkv, flags);
+    if (st != HSA_OK) return st;
+    return forward_impl("hsa_forward_ex", Qs ? Qs : Q, Q, K, V, L, B, H, T, D, chunk, topk, scale,
+                        (flags & HSA_QK_NORM) != 0, out, sel_idx, sel_w, workspace, workspace_bytes, stream);
 }
 
 size_t hsa_decode_workspace_size(int B, int H, int64_t Tmax, int D, int chunk, int topk) {
@@ -222,10 +247,18 @@ size_t hsa_decode_workspace_size(int B, int H, int64_t Tmax, int D, int chunk, i
     return dec_layout(nullptr, B, H, Tmax, D, topk).bytes;
 }
 
+size_t hsa_decode_ex_workspace_size(int B, int H, int Hkv, int64_t Tmax, int D, int chunk, int topk, unsigned flags) {
+    (void)chunk;
+    (void)flags;
+    if (B < 1 || H < 1 || Hkv < 1 || Tmax < 0 || D < 1 || topk < 1) return 0;
+    return dec_layout(nullptr, B, H, Tmax, D, topk).bytes;
+}
+
 static hsa_status decode_impl(const char *name, const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *Kc,
                               const hsa_bf16 *Vc, const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B,
-                              int H, int D, int chunk, int topk, float scale, hsa_bf16 *out, int32_t *sel_idx,
-                              float *sel_w, void *workspace, size_t workspace_bytes, void *stream) {
+                              int H, int D, int chunk, int topk, float scale, bool qk_norm, hsa_bf16 *out,
+                              int32_t *sel_idx, float *sel_w, void *workspace, size_t workspace_bytes,
+                              void *stream) {
     g_last_error.clear();
     hsa_status st = check_common(B, H, D, chunk, topk, 64);
     if (st != HSA_OK) return st;
@@ -258,6 +291,7 @@ static hsa_status decode_impl(const char *name, const hsa_bf16 *qs, const hsa_bf
     a.sel_idx = sel_idx ? sel_idx : l.sel_idx;
     a.sel_w = sel_w ? sel_w : l.sel_w;
     a.cand = l.cand; a.counters = l.counters; a.partial = l.partial;
+    a.qk_norm = qk_norm;
     // the decode kernels never wait on one another; the flag is cleared so that a status query
     // after this call reports this call
     cudaError_t ce = cudaMemsetAsync(l.err, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
@@ -269,16 +303,19 @@ hsa_status hsa_decode(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
                       const int64_t *cache_len, int64_t Tmax, int B, int H, int D, int chunk, int topk,
                       float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace,
                       size_t workspace_bytes, void *stream) {
-    return decode_impl("hsa_decode", q, q, Kc, Vc, Lc, cache_len, Tmax, B, H, D, chunk, topk, scale, out, sel_idx,
-                       sel_w, workspace, workspace_bytes, stream);
+    return decode_impl("hsa_decode", q, q, Kc, Vc, Lc, cache_len, Tmax, B, H, D, chunk, topk, scale, false, out,
+                       sel_idx, sel_w, workspace, workspace_bytes, stream);
 }
 
-hsa_status hsa_decode_qslc(const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
-                           const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B, int H, int D,
-                           int chunk, int topk, float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w,
-                           void *workspace, size_t workspace_bytes, void *stream) {
-    return decode_impl("hsa_decode_qslc", qs, q, Kc, Vc, Lc, cache_len, Tmax, B, H, D, chunk, topk, scale, out,
-                       sel_idx, sel_w, workspace, workspace_bytes, stream);
+hsa_status hsa_decode_ex(const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
+                         const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B, int H, int Hkv, int D,
+                         int chunk, int topk, float scale, unsigned flags, hsa_bf16 *out, int32_t *sel_idx,
+                         float *sel_w, void *workspace, size_t workspace_bytes, void *stream) {
+    g_last_error.clear();
+    hsa_status st = check_ex(H, Hkv, flags);
+    if (st != HSA_OK) return st;
+    return decode_impl("hsa_decode_ex", qs ? qs : q, q, Kc, Vc, Lc, cache_len, Tmax, B, H, D, chunk, topk, scale,
+                       (flags & HSA_QK_NORM) != 0, out, sel_idx, sel_w, workspace, workspace_bytes, stream);
 }
 
 size_t hsa_backward_workspace_size(int B, int H, int T, int D, int chunk, int topk) {
@@ -287,10 +324,10 @@ size_t hsa_backward_workspace_size(int B, int H, int T, int D, int chunk, int to
     return fwd_layout(nullptr, B, H, T, D, topk, true).bytes;
 }
 
-size_t hsa_backward_qslc_workspace_size(int B, int H, int T, int D, int chunk, int topk) {
+size_t hsa_backward_ex_workspace_size(int B, int H, int Hkv, int T, int D, int chunk, int topk, unsigned flags) {
     (void)chunk;
-    if (B < 1 || H < 1 || T < 1 || D < 1 || topk < 1) return 0;
-    return fwd_layout(nullptr, B, H, T, D, topk, true, true).bytes;
+    if (B < 1 || H < 1 || Hkv < 1 || T < 1 || D < 1 || topk < 1) return 0;
+    return fwd_layout(nullptr, B, H, T, D, topk, true, true, (flags & HSA_QK_NORM) != 0).bytes;
 }
 
 // Qs / dQs are NULL for the single-query call (Q retrieves too and dQ takes both parts).
@@ -298,7 +335,7 @@ static hsa_status backward_impl(const char *name, const hsa_bf16 *Qs, const hsa_
                                 const hsa_bf16 *V, const hsa_bf16 *L, const hsa_bf16 *out, const hsa_bf16 *dout,
                                 const int32_t *sel_idx, const float *sel_w, int B, int H, int T, int D, int chunk,
                                 int topk, float scale, float *dQ, float *dK, float *dV, float *dL, float *dQs,
-                                bool qslc, void *workspace, size_t workspace_bytes, void *stream) {
+                                bool qslc, bool qk_norm, void *workspace, size_t workspace_bytes, void *stream) {
     g_last_error.clear();
     hsa_status st = check_common(B, H, D, chunk, topk, 32);
     if (st != HSA_OK) return st;
@@ -315,10 +352,11 @@ static hsa_status backward_impl(const char *name, const hsa_bf16 *Qs, const hsa_
         !aligned16(sel_idx) || !aligned16(sel_w) || !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) ||
         (L && !aligned16(L)) || (dL && !aligned16(dL)))
         return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-    FwdLayout need = fwd_layout(nullptr, B, H, T, D, topk, true, qslc);
+    FwdLayout need = fwd_layout(nullptr, B, H, T, D, topk, true, qslc, qk_norm);
     if ((st = check_ws(workspace, workspace_bytes, need.bytes)) != HSA_OK) return st;
-    FwdLayout l = fwd_layout(workspace, B, H, T, D, topk, true, qslc);
+    FwdLayout l = fwd_layout(workspace, B, H, T, D, topk, true, qslc, qk_norm);
     hsa::BackwardArgs a{};
+    a.qk_norm = qk_norm; a.Qn = l.Qn; a.Kn = l.Kn;
     a.Qs = qslc ? Qs : nullptr; a.dQs = qslc ? dQs : nullptr; a.ds_pair = l.ds_pair;
     a.Q = Q; a.K = K; a.V = V; a.L = L; a.out = out; a.dout = dout;
     a.sel_idx = sel_idx; a.sel_w = sel_w;
@@ -338,16 +376,23 @@ hsa_status hsa_backward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
                         int B, int H, int T, int D, int chunk, int topk, float scale, float *dQ, float *dK,
                         float *dV, float *dL, void *workspace, size_t workspace_bytes, void *stream) {
     return backward_impl("hsa_backward", nullptr, Q, K, V, L, out, dout, sel_idx, sel_w, B, H, T, D, chunk, topk,
-                         scale, dQ, dK, dV, dL, nullptr, false, workspace, workspace_bytes, stream);
+                         scale, dQ, dK, dV, dL, nullptr, false, false, workspace, workspace_bytes, stream);
 }
 
-hsa_status hsa_backward_qslc(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
-                             const hsa_bf16 *L, const hsa_bf16 *out, const hsa_bf16 *dout, const int32_t *sel_idx,
-                             const float *sel_w, int B, int H, int T, int D, int chunk, int topk, float scale,
-                             float *dQ, float *dK, float *dV, float *dL, float *dQs, void *workspace,
-                             size_t workspace_bytes, void *stream) {
-    return backward_impl("hsa_backward_qslc", Qs, Q, K, V, L, out, dout, sel_idx, sel_w, B, H, T, D, chunk, topk,
-                         scale, dQ, dK, dV, dL, dQs, true, workspace, workspace_bytes, stream);
+hsa_status hsa_backward_ex(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
+                           const hsa_bf16 *L, const hsa_bf16 *out, const hsa_bf16 *dout, const int32_t *sel_idx,
+                           const float *sel_w, int B, int H, int Hkv, int T, int D, int chunk, int topk, float scale,
+                           unsigned flags, float *dQ, float *dK, float *dV, float *dL, float *dQs, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+    g_last_error.clear();
+    hsa_status st = check_ex(H, Hkv, flags);
+    if (st != HSA_OK) return st;
+    if ((Qs == nullptr) != (dQs == nullptr))
+        return fail(HSA_ERR_INVALID_ARG, "dQs must be given exactly when Qs is (got Qs %s, dQs %s)",
+                    Qs ? "set" : "NULL", dQs ? "set" : "NULL");
+    return backward_impl("hsa_backward_ex", Qs, Q, K, V, L, out, dout, sel_idx, sel_w, B, H, T, D, chunk, topk, scale,
+                         dQ, dK, dV, dL, dQs, Qs != nullptr, (flags & HSA_QK_NORM) != 0, workspace, workspace_bytes,
+                         stream);
 }
 
 }  // extern "C"

@@ -295,12 +295,18 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
     }
 }
 
-// dQs[t] = scale * sum_j ds[t, j] L[c_j] for a separate retrieval query: one warp per token row, D / 32
-// columns per lane; the selected landmark rows are few and stay in L2.
-template <int D>
-__global__ void __launch_bounds__(256) dqs_kernel(const int32_t *__restrict__ sel_idx, const float *__restrict__ ds_pair,
-                                                  const uint16_t *__restrict__ L, int T, int N, int K, float scale,
-                                                  size_t rows, float *__restrict__ dQs) {
+// The query gradients once the chunk kernel ran with a retrieval query of its own (a separate Qs, or
+// the raw Q under query-key normalisation), when dQ holds only the attention part. One warp per token
+// row, D / 32 columns per lane; the selected landmark rows are few and stay in L2.
+//   ret[t] = scale * sum_j ds[t, j] L[c_j]           (the retrieval query's gradient)
+//   QKN: dQ[t] <- dQ[t] taken back through q / max(|q|, eps) at the raw query Qraw[t]
+//   dQs != NULL: dQs[t] = ret[t];  else dQ[t] += ret[t] (one query did both)
+template <int D, bool QKN>
+__global__ void __launch_bounds__(256) dq_finish_kernel(const int32_t *__restrict__ sel_idx,
+                                                        const float *__restrict__ ds_pair,
+                                                        const uint16_t *__restrict__ L, int T, int N, int K,
+                                                        float scale, size_t rows, const uint16_t *__restrict__ Qraw,
+                                                        float *__restrict__ dQ, float *__restrict__ dQs) {
     constexpr int PER = D / 32;
     const size_t row = (size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -309,10 +315,15 @@ __global__ void __launch_bounds__(256) dqs_kernel(const int32_t *__restrict__ se
     float acc[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
+    // lane j holds slot j's chunk and ds (K <= 32); the landmark loads of the slots are independent, so
+    // several are in flight at once
+    const int c_l = lane < K ? sel_idx[row * K + lane] : -1;
+    const float ds_l = lane < K ? ds_pair[row * K + lane] : 0.0f;
+#pragma unroll 8
     for (int j = 0; j < K; ++j) {
-        const int c = sel_idx[row * K + j];
-        if (c < 0 || c >= N) continue;  // empty slot (the dispatch skips the same ids)
-        const float ds = ds_pair[row * K + j];
+        const int c = __shfl_sync(0xffffffffu, c_l, j);
+        const float ds = __shfl_sync(0xffffffffu, ds_l, j);
+        if (c < 0 || c >= N) continue;  // empty slot (the dispatch skips the same ids); warp-uniform
         const uint16_t *lr = L + (bh * N + c) * D + lane * PER;
         if constexpr (PER == 4) {
             const uint2 v = *reinterpret_cast<const uint2 *>(lr);
@@ -326,12 +337,65 @@ __global__ void __launch_bounds__(256) dqs_kernel(const int32_t *__restrict__ se
             acc[1] = fmaf(ds, bf16_hi(v), acc[1]);
         }
     }
-    float *dst = dQs + row * D + lane * PER;
+    float *dq = dQ + row * D + lane * PER;
+    float g[PER];
+    if constexpr (QKN) {
+        float x[PER];
+        const uint16_t *xr = Qraw + row * D + lane * PER;
+        if constexpr (PER == 4) {
+            const uint2 xv = *reinterpret_cast<const uint2 *>(xr);
+            const float4 gv = *reinterpret_cast<const float4 *>(dq);
+            x[0] = bf16_lo(xv.x); x[1] = bf16_hi(xv.x); x[2] = bf16_lo(xv.y); x[3] = bf16_hi(xv.y);
+            g[0] = gv.x; g[1] = gv.y; g[2] = gv.z; g[3] = gv.w;
+        } else {
+            const uint32_t xv = *reinterpret_cast<const uint32_t *>(xr);
+            const float2 gv = *reinterpret_cast<const float2 *>(dq);
+            x[0] = bf16_lo(xv); x[1] = bf16_hi(xv);
+            g[0] = gv.x; g[1] = gv.y;
+        }
+        float n2 = 0.0f, xg = 0.0f;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) dst[i] = scale * acc[i];
+        for (int i = 0; i < PER; ++i) {
+            n2 = fmaf(x[i], x[i], n2);
+            xg = fmaf(x[i], g[i], xg);
+        }
+        n2 = warp_sum(n2);
+        xg = warp_sum(xg);
+        if (n2 > kQkNormEps * kQkNormEps) {  // (g - y (y . g)) / |x|, y = x / |x|
+            const float rn = rsqrtf(n2), c = xg * rn * rn;
+#pragma unroll
+            for (int i = 0; i < PER; ++i) g[i] = (g[i] - x[i] * c) * rn;
+        } else {
+#pragma unroll
+            for (int i = 0; i < PER; ++i) g[i] *= 1.0f / kQkNormEps;
+        }
+        if (!dQs) {
+#pragma unroll
+            for (int i = 0; i < PER; ++i) g[i] = fmaf(scale, acc[i], g[i]);
+        }
+#pragma unroll
+        for (int i = 0; i < PER; ++i) dq[i] = g[i];
+    }
+    if (dQs) {
+        float *dst = dQs + row * D + lane * PER;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) dst[i] = scale * acc[i];
+    } else if constexpr (!QKN) {
+#pragma unroll
+        for (int i = 0; i < PER; ++i) dq[i] += scale * acc[i];
+    }
 }
 
-cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
+cudaError_t launch_backward(const BackwardArgs &a0, cudaStream_t s) {
+    BackwardArgs a = a0;
+    if (a0.qk_norm) {  // the kernels run on the normalised Q and K; the raw Q retrieves unless Qs does
+        cudaError_t e = launch_l2norm_rows(a0.Q, a0.Qn, (size_t)a0.B * a0.H * a0.T, a0.K, a0.Kn,
+                                           (size_t)a0.B * a0.H * a0.T, a0.D, s);
+        if (e != cudaSuccess) return e;
+        a.Q = a0.Qn;
+        a.K = a0.Kn;
+        if (!a.Qs) a.Qs = a0.Q;
+    }
     const int BH = a.B * a.H;
     const size_t rows = (size_t)BH * a.T;
     cudaError_t e;
@@ -346,8 +410,8 @@ cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
         if (e == cudaSuccess && a.N > 0)
             e = cudaMemsetAsync(a.chunk_cursor, 0, (size_t)BH * a.N * sizeof(int32_t), s);
         if (e == cudaSuccess && a.err) e = cudaMemsetAsync(a.err, 0, sizeof(int32_t), s);
-        // with chunks, dqs_kernel writes every row of dQs
-        if (e == cudaSuccess && a.Qs && a.N == 0) e = cudaMemsetAsync(a.dQs, 0, rows * a.D * sizeof(float), s);
+        // with chunks, dq_finish_kernel writes every row of dQs
+        if (e == cudaSuccess && a.dQs && a.N == 0) e = cudaMemsetAsync(a.dQs, 0, rows * a.D * sizeof(float), s);
     }
     if (e != cudaSuccess || a.N == 0) return e;
     const unsigned dblocks = (unsigned)((rows + 7) / 8);
@@ -377,15 +441,16 @@ cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s) {
         e = cudaGetLastError();
     }
     if (e != cudaSuccess || !a.Qs) return e;
-    {  // the retrieval query's gradient, token-major from the stored ds
-        HSA_PROF("bwd_dqs", s);
+    {  // the retrieval query's gradient (and the attention part back through the normalisation)
+        HSA_PROF("bwd_dq_finish", s);
         const unsigned blocks = (unsigned)((rows + 7) / 8);
-        if (a.D == 128) dqs_kernel<128><<<blocks, 256, 0, s>>>(a.sel_idx, a.ds_pair, a.L, a.T, a.N, a.topk, a.scale,
-                                                                rows, a.dQs);
-        else dqs_kernel<64><<<blocks, 256, 0, s>>>(a.sel_idx, a.ds_pair, a.L, a.T, a.N, a.topk, a.scale, rows,
-                                                    a.dQs);
+        auto kern = a.D == 128 ? (a0.qk_norm ? dq_finish_kernel<128, true> : dq_finish_kernel<128, false>)
+                               : (a0.qk_norm ? dq_finish_kernel<64, true> : dq_finish_kernel<64, false>);
+        kern<<<blocks, 256, 0, s>>>(a.sel_idx, a.ds_pair, a.L, a.T, a.N, a.topk, a.scale, rows, a0.Q, a.dQ, a.dQs);
+        e = cudaGetLastError();
     }
-    return cudaGetLastError();
+    if (e != cudaSuccess || !a0.qk_norm) return e;
+    return launch_l2norm_grad_rows(a0.K, a.dK, rows, a.D, s);
 }
 
 }  // namespace hsa

@@ -190,6 +190,11 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             wt = row >= 0 ? pair_w[t.u.start + p] : 0.0f;
             dl = row >= 0 ? delta[row] : 0.0f;
             sl = (QSLC && row >= 0) ? pair_slot[t.u.start + p] : 0;
+            if (QSLC && row >= 0) {  // the retrieval query's row is read by do_dl two tiles later: into L2 now
+                const uint16_t *qr = Qs + (size_t)row * D;
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(qr));
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(qr + 64));
+            }
         };
         int myrow, myslot;
         float myw, mydel;

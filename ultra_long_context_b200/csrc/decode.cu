@@ -224,7 +224,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
     if (tid == 0) counters[bh] = 0u;
 }
 
-template <int D>
+// QKN: query-key normalisation, the logits use q / max(|q|, eps) and k / max(|k|, eps) (fp32, on the fly).
+template <int D, bool QKN>
 __global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ Kc, const uint16_t *__restrict__ Vc, int64_t Tmax,
     int K, float scale, const int32_t *__restrict__ sel_idx, const float *__restrict__ sel_w,
@@ -250,6 +251,16 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
         qr[2] = bf16_lo(qv.y) * scale; qr[3] = bf16_hi(qv.y) * scale;
         qr[4] = bf16_lo(qv.z) * scale; qr[5] = bf16_hi(qv.z) * scale;
         qr[6] = bf16_lo(qv.w) * scale; qr[7] = bf16_hi(qv.w) * scale;
+        if constexpr (QKN) {  // |scale q|^2 over the row's LPL lanes -> q / max(|q|, eps), times scale
+            float n2 = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) n2 = fmaf(qr[e], qr[e], n2);
+#pragma unroll
+            for (int o = LPL / 2; o > 0; o >>= 1) n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+            const float rq = rsqrtf(fmaxf(n2, kQkNormEps * kQkNormEps * scale * scale)) * scale;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qr[e] *= rq;
+        }
         const size_t row0 = ((size_t)bh * Tmax + (size_t)c * kChunk);
         constexpr int ROUNDS = kChunk / (NWARP * LPW);
         const int sl = tid % LPL, grp = tid / LPL;
@@ -261,12 +272,24 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
 #pragma unroll
         for (int i = 0; i < KEYS_PER_GROUP; ++i)
             vv[i] = *reinterpret_cast<const uint4 *>(Vc + (row0 + grp * KEYS_PER_GROUP + i) * D + sl * 8);
-        // Step 3 logits: a_u = scale * q . K_c[u]
+        // Step 3 logits: a_u = scale * q . K_c[u] (with QKN: scale * norm(q) . norm(K_c[u]))
 #pragma unroll
         for (int r = 0; r < ROUNDS; ++r) {
             float p = dot8(kv[r], qr);
 #pragma unroll
             for (int o = LPL / 2; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+            if constexpr (QKN) {
+                const uint32_t w[4] = {kv[r].x, kv[r].y, kv[r].z, kv[r].w};
+                float k2 = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    k2 = fmaf(bf16_lo(w[e]), bf16_lo(w[e]), k2);
+                    k2 = fmaf(bf16_hi(w[e]), bf16_hi(w[e]), k2);
+                }
+#pragma unroll
+                for (int o = LPL / 2; o > 0; o >>= 1) k2 += __shfl_xor_sync(0xffffffffu, k2, o);
+                p *= rsqrtf(fmaxf(k2, kQkNormEps * kQkNormEps));
+            }
             if (sub == 0) s_p[(r * NWARP + warp) * LPW + g] = p;
         }
         __syncthreads();
@@ -357,9 +380,9 @@ static cudaError_t launch_attend(const DecodeArgs &a, dim3 grid, cudaStream_t s)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_attend_kernel<D>, a.q, a.Kc, a.Vc, a.Tmax, a.K, a.scale,
-                              (const int32_t *)a.sel_idx, (const float *)a.sel_w, a.partial, a.counters + a.B * a.H,
-                              a.out);
+    auto kern = a.qk_norm ? decode_attend_kernel<D, true> : decode_attend_kernel<D, false>;
+    return cudaLaunchKernelEx(&cfg, kern, a.q, a.Kc, a.Vc, a.Tmax, a.K, a.scale, (const int32_t *)a.sel_idx,
+                              (const float *)a.sel_w, a.partial, a.counters + a.B * a.H, a.out);
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {

@@ -22,6 +22,7 @@ struct DecodeArgs {
     uint64_t *cand;    // [B*H, nsplit, K]
     unsigned *counters;  // [2, B*H]
     float *partial;    // [B*H, K, D]
+    bool qk_norm;      // Step 3 attends with q / max(|q|, eps) and k / max(|k|, eps)
 };
 int decode_split_size(int64_t Nmax, int K, int BH);
 size_t decode_scan_smem(int split, int nsplit, int K);
@@ -56,6 +57,9 @@ struct ForwardArgs {
     int32_t *num_tiles;    // [1]
     int32_t *err;          // [1] set when a bounded device wait ran out
     int max_tiles;
+    // query-key normalisation: Q and K are normalised into these bf16 workspace copies first
+    bool qk_norm;
+    uint16_t *Qn, *Kn;     // [B*H*T, D] each
 };
 size_t forward_max_tiles(int B, int H, int T, int topk);
 // Step 2 scores + top-K + fusion weights on the tcgen05 tensor cores (score_tc.cu).
@@ -90,6 +94,11 @@ struct BackwardArgs {
     int32_t *num_tiles;
     int32_t *err;          // [1] set when a bounded device wait ran out
     int max_tiles;
+    // query-key normalisation: Q and K are normalised into these bf16 workspace copies, the kernels
+    // run on them (with the raw Q as retrieval query when there is no Qs), and dQ / dK go back
+    // through the normalisation at the end
+    bool qk_norm;
+    uint16_t *Qn, *Kn;     // [B*H*T, D] each
 };
 cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s);
 // Gradients on the tcgen05 tensor cores (bwd_tc.cu), head dim 128; work units of up to 1024 pairs.
@@ -99,6 +108,14 @@ cudaError_t launch_backward_tc(const BackwardArgs &a, cudaStream_t s);
 // 2-D bf16 tensor map over a [rows, D] row-major tensor: boxes of 64 columns x box_rows rows,
 // 128-byte swizzle (attn_tc.cu). False if the driver entry point is missing or the encoding fails.
 bool make_tmap_bf16(CUtensorMap *m, const void *base, uint64_t rows, int D, int box_rows);
+
+// Query-key normalisation (qknorm.cu), y = x / max(|x|_2, 1e-6) per row of D elements.
+// Rows X0 -> Y0 and X1 -> Y1 in one launch (bf16 in, bf16 out, round to nearest even).
+cudaError_t launch_l2norm_rows(const uint16_t *X0, uint16_t *Y0, size_t R0, const uint16_t *X1, uint16_t *Y1,
+                               size_t R1, int D, cudaStream_t s);
+// In place, per row: dX <- dX taken back through that normalisation of X (fp32 gradients).
+cudaError_t launch_l2norm_grad_rows(const uint16_t *X, float *dX, size_t rows, int D, cudaStream_t s);
+constexpr float kQkNormEps = 1e-6f;
 
 // Message returned by hsa_last_error() on the calling thread.
 void set_last_error(const char *msg);

@@ -301,7 +301,16 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
     return cudaGetLastError();
 }
 
-cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s) {
+cudaError_t launch_forward(const ForwardArgs &a0, cudaStream_t s) {
+    ForwardArgs a = a0;
+    if (a0.qk_norm) {  // Step 3 attends with the normalised query and keys; Qs (the raw Q unless
+                       // separate) still scores the landmarks
+        cudaError_t e = launch_l2norm_rows(a0.Q, a0.Qn, (size_t)a0.B * a0.H * a0.T, a0.K, a0.Kn,
+                                           (size_t)a0.B * a0.H * a0.T, a0.D, s);
+        if (e != cudaSuccess) return e;
+        a.Q = a0.Qn;
+        a.K = a0.Kn;
+    }
     const int BH = a.B * a.H;
     const size_t rows = (size_t)BH * a.T;
     cudaError_t e;

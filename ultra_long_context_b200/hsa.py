@@ -20,6 +20,8 @@ STATUS_NAMES = {0: "HSA_OK", -1: "HSA_ERR_INVALID_ARG", -2: "HSA_ERR_UNSUPPORTED
 
 # C entry points and their argument types, as declared in include/hsa.h
 _P, _I, _I64, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+_U = ctypes.c_uint
+HSA_QK_NORM = 1
 SIGNATURES = {
     "hsa_last_error": ([], ctypes.c_char_p),
     "hsa_workspace_status": ([_P, _P], _I),
@@ -31,11 +33,13 @@ SIGNATURES = {
     "hsa_backward_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
     "hsa_backward": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _SZ, _P],
                      _I),
-    "hsa_forward_qslc": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P], _I),
-    "hsa_decode_qslc": ([_P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _SZ, _P], _I),
-    "hsa_backward_qslc_workspace_size": ([_I, _I, _I, _I, _I, _I], _SZ),
-    "hsa_backward_qslc": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _P, _P, _P, _P, _P,
-                           _SZ, _P], _I),
+    "hsa_forward_ex_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _U], _SZ),
+    "hsa_forward_ex": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _U, _P, _P, _P, _P, _SZ, _P], _I),
+    "hsa_decode_ex_workspace_size": ([_I, _I, _I, _I64, _I, _I, _I, _U], _SZ),
+    "hsa_decode_ex": ([_P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _F, _U, _P, _P, _P, _P, _SZ, _P], _I),
+    "hsa_backward_ex_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _U], _SZ),
+    "hsa_backward_ex": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _U, _P, _P, _P, _P, _P,
+                         _P, _SZ, _P], _I),
     "hsa_profile_enable": ([_I], _I),
     "hsa_profile_summary": ([ctypes.c_char_p, _SZ], _I),
 }
@@ -125,22 +129,34 @@ def hsa_forward_workspace_size(B, H, T, D, chunk=64, topk=16):
     return int(lib().hsa_forward_workspace_size(B, H, T, D, chunk, topk))
 
 
-def hsa_forward(Q, K, V, L, topk, scale=0.0, chunk=64, out=None, sel_idx=None, sel_w=None, workspace=None,
-                stream=None, return_selection=True, Qs=None):
-    """HSA prefill forward. Q, K, V [B, H, T, D] bf16, L [B, H, T // 64, D] bf16 (CUDA).
+def hsa_forward_ex_workspace_size(B, H, Hkv, T, D, chunk=64, topk=16, flags=0):
+    return int(lib().hsa_forward_ex_workspace_size(B, H, Hkv, T, D, chunk, topk, flags))
 
-    Qs: separate retrieval queries [B, H, T, D] bf16 (hsa_forward_qslc: Qs scores the landmarks, Q
-    attends), or None when Q does both.
+
+def _flags(qk_norm):
+    return HSA_QK_NORM if qk_norm else 0
+
+
+def hsa_forward(Q, K, V, L, topk, scale=0.0, chunk=64, out=None, sel_idx=None, sel_w=None, workspace=None,
+                stream=None, return_selection=True, Qs=None, qk_norm=False):
+    """HSA prefill forward. Q [B, H, T, D], K, V [B, Hkv, T, D], L [B, Hkv, T // 64, D] bf16 (CUDA); Hkv = H
+    unless key/value heads are grouped (query head h uses head h // (H // Hkv)).
+
+    Qs: separate retrieval queries [B, H, T, D] bf16 (Qs scores the landmarks, Q attends), or None when Q
+    does both. qk_norm: Step 3 attends with the L2-normalised query and keys. Any of the three calls
+    hsa_forward_ex, else hsa_forward.
     Returns (out [B, H, T, D] bf16, sel_idx [B, H, T, topk] int32, sel_w [B, H, T, topk] fp32); the
     selection is None when ``return_selection`` is False and none was passed in.
     """
     B, H, T, D = Q.shape
+    Hkv = K.shape[1]
     dev = Q.device
+    _need(Q, "Q", torch.bfloat16, (B, H, T, D), dev)
     if Qs is not None:
         _need(Qs, "Qs", torch.bfloat16, (B, H, T, D), dev)
-    for n, t in (("Q", Q), ("K", K), ("V", V)):
-        _need(t, n, torch.bfloat16, (B, H, T, D), dev)
-    _need(L, "L", torch.bfloat16, (B, H, T // chunk, D), dev)
+    for n, t in (("K", K), ("V", V)):
+        _need(t, n, torch.bfloat16, (B, Hkv, T, D), dev)
+    _need(L, "L", torch.bfloat16, (B, Hkv, T // chunk, D), dev)
     if out is None:
         out = torch.empty_like(Q)
     _need(out, "out", torch.bfloat16, (B, H, T, D), dev)
@@ -148,17 +164,21 @@ def hsa_forward(Q, K, V, L, topk, scale=0.0, chunk=64, out=None, sel_idx=None, s
         sel_idx = torch.empty((B, H, T, topk), dtype=torch.int32, device=dev)
     if return_selection and sel_w is None:
         sel_w = torch.empty((B, H, T, topk), dtype=torch.float32, device=dev)
-    nbytes = hsa_forward_workspace_size(B, H, T, D, chunk, topk)
-    ws = _workspace(nbytes, dev, workspace)
-    wp, wn = _aligned(ws)
-    if Qs is None:
+    if Qs is None and not qk_norm and Hkv == H:
+        nbytes = hsa_forward_workspace_size(B, H, T, D, chunk, topk)
+        ws = _workspace(nbytes, dev, workspace)
+        wp, wn = _aligned(ws)
         st = lib().hsa_forward(_ptr(Q), _ptr(K), _ptr(V), _ptr(L), B, H, T, D, chunk, topk, float(scale), _ptr(out),
                                _ptr(sel_idx), _ptr(sel_w), wp, wn, _stream(dev, stream))
         _check("hsa_forward", st)
     else:
-        st = lib().hsa_forward_qslc(_ptr(Qs), _ptr(Q), _ptr(K), _ptr(V), _ptr(L), B, H, T, D, chunk, topk,
-                                    float(scale), _ptr(out), _ptr(sel_idx), _ptr(sel_w), wp, wn, _stream(dev, stream))
-        _check("hsa_forward_qslc", st)
+        fl = _flags(qk_norm)
+        ws = _workspace(hsa_forward_ex_workspace_size(B, H, Hkv, T, D, chunk, topk, fl), dev, workspace)
+        wp, wn = _aligned(ws)
+        st = lib().hsa_forward_ex(_ptr(Qs), _ptr(Q), _ptr(K), _ptr(V), _ptr(L), B, H, Hkv, T, D, chunk, topk,
+                                  float(scale), fl, _ptr(out), _ptr(sel_idx), _ptr(sel_w), wp, wn,
+                                  _stream(dev, stream))
+        _check("hsa_forward_ex", st)
     return out, sel_idx, sel_w
 
 
@@ -166,22 +186,28 @@ def hsa_decode_workspace_size(B, H, Tmax, D, chunk=64, topk=16):
     return int(lib().hsa_decode_workspace_size(B, H, Tmax, D, chunk, topk))
 
 
-def hsa_decode(q, Kc, Vc, Lc, cache_len, topk, scale=0.0, chunk=64, out=None, sel_idx=None, sel_w=None,
-               workspace=None, stream=None, qs=None):
-    """HSA decode. q [B, H, D], Kc / Vc [B, H, Tmax, D], Lc [B, H, Tmax // 64, D] bf16; cache_len [B] int64.
+def hsa_decode_ex_workspace_size(B, H, Hkv, Tmax, D, chunk=64, topk=16, flags=0):
+    return int(lib().hsa_decode_ex_workspace_size(B, H, Hkv, Tmax, D, chunk, topk, flags))
 
-    qs: a separate retrieval query [B, H, D] bf16 (hsa_decode_qslc), or None when q does both.
+
+def hsa_decode(q, Kc, Vc, Lc, cache_len, topk, scale=0.0, chunk=64, out=None, sel_idx=None, sel_w=None,
+               workspace=None, stream=None, qs=None, qk_norm=False):
+    """HSA decode. q [B, H, D], Kc / Vc [B, Hkv, Tmax, D], Lc [B, Hkv, Tmax // 64, D] bf16; cache_len [B]
+    int64 (Hkv = H unless key/value heads are grouped).
+
+    qs: a separate retrieval query [B, H, D] bf16, or None when q does both. qk_norm: Step 3 attends with
+    the L2-normalised query and keys. Any of the three calls hsa_decode_ex, else hsa_decode.
     Returns (out [B, H, D] bf16, sel_idx [B, H, topk] int32, sel_w [B, H, topk] fp32).
     """
     B, H, D = q.shape
-    Tmax = Kc.shape[2]
+    Hkv, Tmax = Kc.shape[1], Kc.shape[2]
     dev = q.device
     _need(q, "q", torch.bfloat16, (B, H, D), dev)
     if qs is not None:
         _need(qs, "qs", torch.bfloat16, (B, H, D), dev)
-    _need(Kc, "Kc", torch.bfloat16, (B, H, Tmax, D), dev)
-    _need(Vc, "Vc", torch.bfloat16, (B, H, Tmax, D), dev)
-    _need(Lc, "Lc", torch.bfloat16, (B, H, Tmax // chunk, D), dev)
+    _need(Kc, "Kc", torch.bfloat16, (B, Hkv, Tmax, D), dev)
+    _need(Vc, "Vc", torch.bfloat16, (B, Hkv, Tmax, D), dev)
+    _need(Lc, "Lc", torch.bfloat16, (B, Hkv, Tmax // chunk, D), dev)
     _need(cache_len, "cache_len", torch.int64, (B,), dev)
     if out is None:
         out = torch.empty_like(q)
@@ -189,18 +215,21 @@ def hsa_decode(q, Kc, Vc, Lc, cache_len, topk, scale=0.0, chunk=64, out=None, se
         sel_idx = torch.empty((B, H, topk), dtype=torch.int32, device=dev)
     if sel_w is None:
         sel_w = torch.empty((B, H, topk), dtype=torch.float32, device=dev)
-    nbytes = hsa_decode_workspace_size(B, H, Tmax, D, chunk, topk)
-    ws = _workspace(nbytes, dev, workspace)
-    wp, wn = _aligned(ws)
-    if qs is None:
+    if qs is None and not qk_norm and Hkv == H:
+        nbytes = hsa_decode_workspace_size(B, H, Tmax, D, chunk, topk)
+        ws = _workspace(nbytes, dev, workspace)
+        wp, wn = _aligned(ws)
         st = lib().hsa_decode(_ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Lc), _ptr(cache_len), Tmax, B, H, D, chunk, topk,
                               float(scale), _ptr(out), _ptr(sel_idx), _ptr(sel_w), wp, wn, _stream(dev, stream))
         _check("hsa_decode", st)
     else:
-        st = lib().hsa_decode_qslc(_ptr(qs), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Lc), _ptr(cache_len), Tmax, B, H, D,
-                                   chunk, topk, float(scale), _ptr(out), _ptr(sel_idx), _ptr(sel_w), wp, wn,
-                                   _stream(dev, stream))
-        _check("hsa_decode_qslc", st)
+        fl = _flags(qk_norm)
+        ws = _workspace(hsa_decode_ex_workspace_size(B, H, Hkv, Tmax, D, chunk, topk, fl), dev, workspace)
+        wp, wn = _aligned(ws)
+        st = lib().hsa_decode_ex(_ptr(qs), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Lc), _ptr(cache_len), Tmax, B, H, Hkv,
+                                 D, chunk, topk, float(scale), fl, _ptr(out), _ptr(sel_idx), _ptr(sel_w), wp, wn,
+                                 _stream(dev, stream))
+        _check("hsa_decode_ex", st)
     return out, sel_idx, sel_w
 
 
@@ -234,31 +263,35 @@ def hsa_backward_workspace_size(B, H, T, D, chunk=64, topk=16):
     return int(lib().hsa_backward_workspace_size(B, H, T, D, chunk, topk))
 
 
-def hsa_backward_qslc_workspace_size(B, H, T, D, chunk=64, topk=16):
-    return int(lib().hsa_backward_qslc_workspace_size(B, H, T, D, chunk, topk))
+def hsa_backward_ex_workspace_size(B, H, Hkv, T, D, chunk=64, topk=16, flags=0):
+    return int(lib().hsa_backward_ex_workspace_size(B, H, Hkv, T, D, chunk, topk, flags))
 
 
 def hsa_backward(Q, K, V, L, out, dout, sel_idx, sel_w, scale=0.0, chunk=64, grads=None, workspace=None,
-                 stream=None, Qs=None):
-    """Backward of hsa_forward for its selection. Returns (dQ, dK, dV, dL), fp32; with separate retrieval
-    queries Qs (hsa_backward_qslc), (dQ, dK, dV, dL, dQs) where dQ is the attention query's gradient."""
+                 stream=None, Qs=None, qk_norm=False):
+    """Backward of hsa_forward for its selection (same options). Returns (dQ, dK, dV, dL), fp32, shaped like
+    Q, K, V, L; with separate retrieval queries Qs, (dQ, dK, dV, dL, dQs) where dQ is the attention
+    query's gradient. Any option (Qs, qk_norm, grouped heads) calls hsa_backward_ex."""
     B, H, T, D = Q.shape
+    Hkv = K.shape[1]
     topk = sel_idx.shape[-1]
     dev = Q.device
     if Qs is not None:
         _need(Qs, "Qs", torch.bfloat16, (B, H, T, D), dev)
-    for n, t in (("Q", Q), ("K", K), ("V", V), ("out", out), ("dout", dout)):
+    for n, t in (("Q", Q), ("out", out), ("dout", dout)):
         _need(t, n, torch.bfloat16, (B, H, T, D), dev)
-    _need(L, "L", torch.bfloat16, (B, H, T // chunk, D), dev)
+    for n, t in (("K", K), ("V", V)):
+        _need(t, n, torch.bfloat16, (B, Hkv, T, D), dev)
+    _need(L, "L", torch.bfloat16, (B, Hkv, T // chunk, D), dev)
     _need(sel_idx, "sel_idx", torch.int32, (B, H, T, topk), dev)
     _need(sel_w, "sel_w", torch.float32, (B, H, T, topk), dev)
     if grads is None:
         grads = (torch.empty((B, H, T, D), dtype=torch.float32, device=dev),
-                 torch.empty((B, H, T, D), dtype=torch.float32, device=dev),
-                 torch.empty((B, H, T, D), dtype=torch.float32, device=dev),
-                 torch.empty((B, H, T // chunk, D), dtype=torch.float32, device=dev))
+                 torch.empty((B, Hkv, T, D), dtype=torch.float32, device=dev),
+                 torch.empty((B, Hkv, T, D), dtype=torch.float32, device=dev),
+                 torch.empty((B, Hkv, T // chunk, D), dtype=torch.float32, device=dev))
     dQ, dK, dV, dL = grads[:4]
-    if Qs is None:
+    if Qs is None and not qk_norm and Hkv == H:
         nbytes = hsa_backward_workspace_size(B, H, T, D, chunk, topk)
         ws = _workspace(nbytes, dev, workspace)
         wp, wn = _aligned(ws)
@@ -267,15 +300,17 @@ def hsa_backward(Q, K, V, L, out, dout, sel_idx, sel_w, scale=0.0, chunk=64, gra
                                 _ptr(dL) if dL.numel() else None, wp, wn, _stream(dev, stream))
         _check("hsa_backward", st)
         return dQ, dK, dV, dL
-    dQs = grads[4] if len(grads) > 4 else torch.empty((B, H, T, D), dtype=torch.float32, device=dev)
-    nbytes = hsa_backward_qslc_workspace_size(B, H, T, D, chunk, topk)
-    ws = _workspace(nbytes, dev, workspace)
+    dQs = None
+    if Qs is not None:
+        dQs = grads[4] if len(grads) > 4 else torch.empty((B, H, T, D), dtype=torch.float32, device=dev)
+    fl = _flags(qk_norm)
+    ws = _workspace(hsa_backward_ex_workspace_size(B, H, Hkv, T, D, chunk, topk, fl), dev, workspace)
     wp, wn = _aligned(ws)
-    st = lib().hsa_backward_qslc(_ptr(Qs), _ptr(Q), _ptr(K), _ptr(V), _ptr(L), _ptr(out), _ptr(dout), _ptr(sel_idx),
-                                 _ptr(sel_w), B, H, T, D, chunk, topk, float(scale), _ptr(dQ), _ptr(dK), _ptr(dV),
-                                 _ptr(dL) if dL.numel() else None, _ptr(dQs), wp, wn, _stream(dev, stream))
-    _check("hsa_backward_qslc", st)
-    return dQ, dK, dV, dL, dQs
+    st = lib().hsa_backward_ex(_ptr(Qs), _ptr(Q), _ptr(K), _ptr(V), _ptr(L), _ptr(out), _ptr(dout), _ptr(sel_idx),
+                               _ptr(sel_w), B, H, Hkv, T, D, chunk, topk, float(scale), fl, _ptr(dQ), _ptr(dK),
+                               _ptr(dV), _ptr(dL) if dL.numel() else None, _ptr(dQs), wp, wn, _stream(dev, stream))
+    _check("hsa_backward_ex", st)
+    return (dQ, dK, dV, dL) if Qs is None else (dQ, dK, dV, dL, dQs)
 
 
 def hsa_profile_enable(on=True):

@@ -103,6 +103,8 @@ def oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, chunk=64, qs=None, qk_n
     scale = scale or 1 / math.sqrt(D)
     sel = oracle_mod.decode_select(host(q if qs is None else qs), host(Lc), lens.cpu().numpy(), chunk=chunk, topk=topk,
                                    scale=scale)
+    if Kc.shape[1] != H:  # grouped key heads: each query head gathers from its key head's cache
+        Kc, Vc, Lc = (x.repeat_interleave(H // Kc.shape[1], dim=1) for x in (Kc, Vc, Lc))
     idx = torch.as_tensor(sel["sel_idx"], device=Kc.device, dtype=torch.int64).clamp(min=0)   # [B,H,k]
     tok = (idx[..., None] * chunk + torch.arange(chunk, device=Kc.device)).reshape(B, H, -1)
     Kg = torch.gather(Kc, 2, tok[..., None].expand(-1, -1, -1, D)).reshape(B * H, topk, chunk, D)
@@ -360,3 +362,62 @@ def test_backward_qk_norm_matches_oracle(oracle_mod, B, H, T, D, topk, separate)
                                 Qs=Qsh)
     for x, y in zip(ref[:2], plain[:2]):  # dQ and dK: the normalisation's Jacobian matters
         assert np.abs(x - y).sum() > 0.5 * np.abs(x).sum()
+
+
+# ---------------------------------------------------------------------------------------------
+# grouped key/value heads: query head h reads key head h // (H // Hkv); each query head selects its own
+
+
+def gqa_inputs(B, H, Hkv, T, D, seed):
+    Q = inputs.forward_inputs(B, H, T, D, seed, device=DEV)[0]
+    _, K, V, L = inputs.forward_inputs(B, Hkv, T, D, seed + 1, device=DEV)
+    return Q, K, V, L
+
+
+@pytest.mark.parametrize("B,H,Hkv,T,D,topk,opts", [
+    (1, 4, 2, 2048 + 37, 128, 16, {}), (2, 4, 1, 1100, 64, 8, {}), (1, 8, 2, 1500, 128, 8, {"qk_norm": True}),
+    (1, 4, 2, 777, 64, 5, {"separate": True}),
+])
+def test_forward_grouped_heads_match_oracle(oracle_mod, B, H, Hkv, T, D, topk, opts):
+    Q, K, V, L = gqa_inputs(B, H, Hkv, T, D, 1400 + T)
+    Qs = inputs.forward_inputs(B, H, T, D, 1500 + T, device=DEV)[0] if opts.get("separate") else None
+    qk = opts.get("qk_norm", False)
+    sc = 1 / math.sqrt(D)
+    out, idx, w = hsa.hsa_forward(Q, K, V, L, topk, Qs=Qs, qk_norm=qk)
+    Qh, Kh, Vh, Lh = (host(x) for x in (Q, K, V, L))
+    Qsh = None if Qs is None else host(Qs)
+    orc = oracle_mod.forward(Qh, Kh, Vh, Lh, chunk=64, topk=topk, scale=sc, Qs=Qsh, qk_norm=qk)
+    compare_forward_rows(oracle_mod, host(out).reshape(-1, D), host(idx).reshape(-1, topk), host(w).reshape(-1, topk),
+                         orc, Qh, Kh, Vh, Lh, np.arange(B * H * T), 64, sc, Qs=Qsh, qk_norm=qk)
+
+
+@pytest.mark.parametrize("B,H,Hkv,D,lens,topk", [(2, 4, 2, 128, [9000, 4100], 16), (1, 8, 1, 64, [64 * 700 + 5], 32)])
+def test_decode_grouped_heads_match_oracle(oracle_mod, B, H, Hkv, D, lens, topk):
+    Tmax = max(lens) + 64
+    q = inputs.decode_inputs(B, H, lens, D, seed=51 + D, Tmax=Tmax, device=DEV)[0]
+    _, Kc, Vc, Lc, lens_t, _ = inputs.decode_inputs(B, Hkv, lens, D, seed=52 + D, Tmax=Tmax, device=DEV)
+    check_decode(oracle_mod, q, Kc, Vc, Lc, lens_t, topk)
+
+
+@pytest.mark.parametrize("B,H,Hkv,T,D,topk,opts", [
+    (1, 4, 2, 2048 + 64, 128, 16, {}), (1, 4, 1, 1100, 64, 8, {}), (1, 4, 2, 1500, 128, 8, {"qk_norm": True}),
+    (1, 4, 2, 1100, 64, 8, {"separate": True, "qk_norm": True}),
+])
+def test_backward_grouped_heads_match_oracle(oracle_mod, B, H, Hkv, T, D, topk, opts):
+    Q, K, V, L = gqa_inputs(B, H, Hkv, T, D, 1600 + T)
+    Qs = inputs.forward_inputs(B, H, T, D, 1700 + T, device=DEV)[0] if opts.get("separate") else None
+    qk = opts.get("qk_norm", False)
+    dO = inputs.upstream_grad(B, H, T, D, 1600 + T, device=DEV)
+    Qh, Kh, Vh, Lh, dOh = (host(x) for x in (Q, K, V, L, dO))
+    Qsh = None if Qs is None else host(Qs)
+    sc = 1 / math.sqrt(D)
+    orc = oracle_mod.forward(Qh, Kh, Vh, Lh, chunk=64, topk=topk, scale=sc, Qs=Qsh, qk_norm=qk)
+    sel_idx = torch.as_tensor(orc["sel_idx"].reshape(B, H, T, topk), device=DEV)
+    sel_w = torch.as_tensor(orc["sel_w"].reshape(B, H, T, topk), dtype=torch.float32, device=DEV)
+    out = torch.as_tensor(orc["out"].reshape(B, H, T, D), dtype=torch.float32, device=DEV).to(torch.bfloat16)
+    grads = hsa.hsa_backward(Q, K, V, L, out, dO, sel_idx, sel_w, Qs=Qs, qk_norm=qk)
+    ref = oracle_mod.backward(Qh, Kh, Vh, Lh, dOh, orc["sel_idx"].reshape(B, H, T, topk), chunk=64, scale=sc, Qs=Qsh,
+                              qk_norm=qk)
+    assert grads[1].shape == (B, Hkv, T, D) and grads[3].shape == (B, Hkv, T // 64, D)
+    for g, r, n in zip(grads, ref, ("dQ", "dK", "dV", "dL", "dQs")):
+        grad_close(host(g), r, n)

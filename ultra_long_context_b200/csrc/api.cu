@@ -145,7 +145,6 @@ hsa_status check_ex(int H, int Hkv, unsigned flags) {
     if (flags & ~HSA_QK_NORM) return fail(HSA_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags & ~HSA_QK_NORM);
     if (Hkv < 1 || H % Hkv != 0)
         return fail(HSA_ERR_INVALID_ARG, "H (%d) must be a positive multiple of Hkv (%d)", H, Hkv);
-    if (Hkv != H) return fail(HSA_ERR_UNSUPPORTED, "grouped key/value heads (Hkv < H) are not implemented yet");
     return HSA_OK;
 }
 
@@ -188,7 +187,8 @@ size_t hsa_forward_ex_workspace_size(int B, int H, int Hkv, int T, int D, int ch
 
 // Qs retrieves (Step 2 scores, Step 4 weights), Q attends (Step 3); the single-query call passes Q twice.
 static hsa_status forward_impl(const char *name, const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K,
-                               const hsa_bf16 *V, const hsa_bf16 *L, int B, int H, int T, int D, int chunk, int topk,
+                               const hsa_bf16 *V, const hsa_bf16 *L, int B, int H, int Hkv, int T, int D, int chunk,
+                               int topk,
                                float scale, bool qk_norm, hsa_bf16 *out, int32_t *sel_idx, float *sel_w,
                                void *workspace, size_t workspace_bytes, void *stream) {
     g_last_error.clear();
@@ -209,7 +209,7 @@ static hsa_status forward_impl(const char *name, const hsa_bf16 *Qs, const hsa_b
     hsa::ForwardArgs a{};
     a.qk_norm = qk_norm; a.Qn = l.Qn; a.Kn = l.Kn;
     a.Qs = Qs; a.Q = Q; a.K = K; a.V = V; a.L = L;
-    a.B = B; a.H = H; a.T = T; a.D = D; a.N = T / 64; a.topk = topk;
+    a.B = B; a.H = H; a.Hkv = Hkv; a.T = T; a.D = D; a.N = T / 64; a.topk = topk;
     a.scale = resolve_scale(scale, D);
     a.out = out;
     a.sel_idx = sel_idx ? sel_idx : l.sel_idx;
@@ -226,7 +226,7 @@ static hsa_status forward_impl(const char *name, const hsa_bf16 *Qs, const hsa_b
 hsa_status hsa_forward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V, const hsa_bf16 *L, int B, int H,
                        int T, int D, int chunk, int topk, float scale, hsa_bf16 *out, int32_t *sel_idx,
                        float *sel_w, void *workspace, size_t workspace_bytes, void *stream) {
-    return forward_impl("hsa_forward", Q, Q, K, V, L, B, H, T, D, chunk, topk, scale, false, out, sel_idx, sel_w,
+    return forward_impl("hsa_forward", Q, Q, K, V, L, B, H, H, T, D, chunk, topk, scale, false, out, sel_idx, sel_w,
                         workspace, workspace_bytes, stream);
 }
 
@@ -237,7 +237,7 @@ hsa_status hsa_forward_ex(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 
     g_last_error.clear();
     hsa_status st = check_ex(H, Hkv, flags);
     if (st != HSA_OK) return st;
-    return forward_impl("hsa_forward_ex", Qs ? Qs : Q, Q, K, V, L, B, H, T, D, chunk, topk, scale,
+    return forward_impl("hsa_forward_ex", Qs ? Qs : Q, Q, K, V, L, B, H, Hkv, T, D, chunk, topk, scale,
                         (flags & HSA_QK_NORM) != 0, out, sel_idx, sel_w, workspace, workspace_bytes, stream);
 }
 
@@ -256,7 +256,7 @@ size_t hsa_decode_ex_workspace_size(int B, int H, int Hkv, int64_t Tmax, int D, 
 
 static hsa_status decode_impl(const char *name, const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *Kc,
                               const hsa_bf16 *Vc, const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B,
-                              int H, int D, int chunk, int topk, float scale, bool qk_norm, hsa_bf16 *out,
+                              int H, int Hkv, int D, int chunk, int topk, float scale, bool qk_norm, hsa_bf16 *out,
                               int32_t *sel_idx, float *sel_w, void *workspace, size_t workspace_bytes,
                               void *stream) {
     g_last_error.clear();
@@ -285,7 +285,7 @@ static hsa_status decode_impl(const char *name, const hsa_bf16 *qs, const hsa_bf
     hsa::DecodeArgs a{};
     a.qs = qs; a.q = q; a.Kc = Kc; a.Vc = Vc; a.Lc = Lc; a.cache_len = cache_len;
     a.Tmax = Tmax; a.Nmax = Tmax / 64;
-    a.B = B; a.H = H; a.D = D; a.K = topk;
+    a.B = B; a.H = H; a.Hkv = Hkv; a.D = D; a.K = topk;
     a.scale = resolve_scale(scale, D);
     a.out = out;
     a.sel_idx = sel_idx ? sel_idx : l.sel_idx;
@@ -303,7 +303,7 @@ hsa_status hsa_decode(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
                       const int64_t *cache_len, int64_t Tmax, int B, int H, int D, int chunk, int topk,
                       float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace,
                       size_t workspace_bytes, void *stream) {
-    return decode_impl("hsa_decode", q, q, Kc, Vc, Lc, cache_len, Tmax, B, H, D, chunk, topk, scale, false, out,
+    return decode_impl("hsa_decode", q, q, Kc, Vc, Lc, cache_len, Tmax, B, H, H, D, chunk, topk, scale, false, out,
                        sel_idx, sel_w, workspace, workspace_bytes, stream);
 }
 
@@ -314,7 +314,7 @@ hsa_status hsa_decode_ex(const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *
     g_last_error.clear();
     hsa_status st = check_ex(H, Hkv, flags);
     if (st != HSA_OK) return st;
-    return decode_impl("hsa_decode_ex", qs ? qs : q, q, Kc, Vc, Lc, cache_len, Tmax, B, H, D, chunk, topk, scale,
+    return decode_impl("hsa_decode_ex", qs ? qs : q, q, Kc, Vc, Lc, cache_len, Tmax, B, H, Hkv, D, chunk, topk, scale,
                        (flags & HSA_QK_NORM) != 0, out, sel_idx, sel_w, workspace, workspace_bytes, stream);
 }
 
@@ -333,8 +333,8 @@ size_t hsa_backward_ex_workspace_size(int B, int H, int Hkv, int T, int D, int c
 // Qs / dQs are NULL for the single-query call (Q retrieves too and dQ takes both parts).
 static hsa_status backward_impl(const char *name, const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K,
                                 const hsa_bf16 *V, const hsa_bf16 *L, const hsa_bf16 *out, const hsa_bf16 *dout,
-                                const int32_t *sel_idx, const float *sel_w, int B, int H, int T, int D, int chunk,
-                                int topk, float scale, float *dQ, float *dK, float *dV, float *dL, float *dQs,
+                                const int32_t *sel_idx, const float *sel_w, int B, int H, int Hkv, int T, int D,
+                                int chunk, int topk, float scale, float *dQ, float *dK, float *dV, float *dL, float *dQs,
                                 bool qslc, bool qk_norm, void *workspace, size_t workspace_bytes, void *stream) {
     g_last_error.clear();
     hsa_status st = check_common(B, H, D, chunk, topk, 32);
@@ -360,7 +360,7 @@ static hsa_status backward_impl(const char *name, const hsa_bf16 *Qs, const hsa_
     a.Qs = qslc ? Qs : nullptr; a.dQs = qslc ? dQs : nullptr; a.ds_pair = l.ds_pair;
     a.Q = Q; a.K = K; a.V = V; a.L = L; a.out = out; a.dout = dout;
     a.sel_idx = sel_idx; a.sel_w = sel_w;
-    a.B = B; a.H = H; a.T = T; a.D = D; a.N = T / 64; a.topk = topk;
+    a.B = B; a.H = H; a.Hkv = Hkv; a.T = T; a.D = D; a.N = T / 64; a.topk = topk;
     a.scale = resolve_scale(scale, D);
     a.dQ = dQ; a.dK = dK; a.dV = dV; a.dL = dL;
     a.delta = l.delta;
@@ -375,7 +375,7 @@ hsa_status hsa_backward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
                         const hsa_bf16 *out, const hsa_bf16 *dout, const int32_t *sel_idx, const float *sel_w,
                         int B, int H, int T, int D, int chunk, int topk, float scale, float *dQ, float *dK,
                         float *dV, float *dL, void *workspace, size_t workspace_bytes, void *stream) {
-    return backward_impl("hsa_backward", nullptr, Q, K, V, L, out, dout, sel_idx, sel_w, B, H, T, D, chunk, topk,
+    return backward_impl("hsa_backward", nullptr, Q, K, V, L, out, dout, sel_idx, sel_w, B, H, H, T, D, chunk, topk,
                          scale, dQ, dK, dV, dL, nullptr, false, false, workspace, workspace_bytes, stream);
 }
 
@@ -390,9 +390,9 @@ hsa_status hsa_backward_ex(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16
     if ((Qs == nullptr) != (dQs == nullptr))
         return fail(HSA_ERR_INVALID_ARG, "dQs must be given exactly when Qs is (got Qs %s, dQs %s)",
                     Qs ? "set" : "NULL", dQs ? "set" : "NULL");
-    return backward_impl("hsa_backward_ex", Qs, Q, K, V, L, out, dout, sel_idx, sel_w, B, H, T, D, chunk, topk, scale,
-                         dQ, dK, dV, dL, dQs, Qs != nullptr, (flags & HSA_QK_NORM) != 0, workspace, workspace_bytes,
-                         stream);
+    return backward_impl("hsa_backward_ex", Qs, Q, K, V, L, out, dout, sel_idx, sel_w, B, H, Hkv, T, D, chunk, topk,
+                         scale, dQ, dK, dV, dL, dQs, Qs != nullptr, (flags & HSA_QK_NORM) != 0, workspace,
+                         workspace_bytes, stream);
 }
 
 }  // extern "C"

@@ -394,7 +394,7 @@ static cudaError_t launch_attn_tc_d(const ForwardArgs &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(chunk_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const uint64_t rows = (uint64_t)a.B * a.H * a.T;
+    const uint64_t rows = (uint64_t)a.B * a.Hkv * a.T;  // tiles address K, V by key head (chunk id / N)
     CUtensorMap tk, tv;
     if (!make_tmap_bf16(&tk, a.K, rows, D, kChunk) || !make_tmap_bf16(&tv, a.V, rows, D, kChunk)) return cudaErrorInvalidValue;
     int dev = 0, sms = 148;

@@ -304,14 +304,14 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
 template <int D, bool QKN>
 __global__ void __launch_bounds__(256) dq_finish_kernel(const int32_t *__restrict__ sel_idx,
                                                         const float *__restrict__ ds_pair,
-                                                        const uint16_t *__restrict__ L, int T, int N, int K,
+                                                        const uint16_t *__restrict__ L, int T, int N, int K, int G,
                                                         float scale, size_t rows, const uint16_t *__restrict__ Qraw,
                                                         float *__restrict__ dQ, float *__restrict__ dQs) {
     constexpr int PER = D / 32;
     const size_t row = (size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
-    const size_t bh = row / T;
+    const size_t kvh = row / T / G;  // the landmark head of this token's query head
     float acc[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
@@ -324,7 +324,7 @@ __global__ void __launch_bounds__(256) dq_finish_kernel(const int32_t *__restric
         const int c = __shfl_sync(0xffffffffu, c_l, j);
         const float ds = __shfl_sync(0xffffffffu, ds_l, j);
         if (c < 0 || c >= N) continue;  // empty slot (the dispatch skips the same ids); warp-uniform
-        const uint16_t *lr = L + (bh * N + c) * D + lane * PER;
+        const uint16_t *lr = L + (kvh * N + c) * D + lane * PER;
         if constexpr (PER == 4) {
             const uint2 v = *reinterpret_cast<const uint2 *>(lr);
             acc[0] = fmaf(ds, bf16_lo(v.x), acc[0]);
@@ -388,9 +388,12 @@ __global__ void __launch_bounds__(256) dq_finish_kernel(const int32_t *__restric
 
 cudaError_t launch_backward(const BackwardArgs &a0, cudaStream_t s) {
     BackwardArgs a = a0;
+    if (a.Hkv <= 0) a.Hkv = a.H;
+    if (a.H % a.Hkv != 0) return cudaErrorInvalidValue;
+    const int G = a.H / a.Hkv;  // query heads per key head
+    const size_t kv_rows = (size_t)a.B * a.Hkv * a.T, chunks = (size_t)a.B * a.Hkv * a.N;
     if (a0.qk_norm) {  // the kernels run on the normalised Q and K; the raw Q retrieves unless Qs does
-        cudaError_t e = launch_l2norm_rows(a0.Q, a0.Qn, (size_t)a0.B * a0.H * a0.T, a0.K, a0.Kn,
-                                           (size_t)a0.B * a0.H * a0.T, a0.D, s);
+        cudaError_t e = launch_l2norm_rows(a0.Q, a0.Qn, (size_t)a.B * a.H * a.T, a0.K, a0.Kn, kv_rows, a.D, s);
         if (e != cudaSuccess) return e;
         a.Q = a0.Qn;
         a.K = a0.Kn;
@@ -402,13 +405,11 @@ cudaError_t launch_backward(const BackwardArgs &a0, cudaStream_t s) {
     {
         HSA_PROF("memset", s);
         e = cudaMemsetAsync(a.dQ, 0, rows * a.D * sizeof(float), s);
-        if (e == cudaSuccess) e = cudaMemsetAsync(a.dK, 0, rows * a.D * sizeof(float), s);
-        if (e == cudaSuccess) e = cudaMemsetAsync(a.dV, 0, rows * a.D * sizeof(float), s);
-        if (e == cudaSuccess && a.N > 0) e = cudaMemsetAsync(a.dL, 0, (size_t)BH * a.N * a.D * sizeof(float), s);
-        if (e == cudaSuccess && a.N > 0)
-            e = cudaMemsetAsync(a.chunk_count, 0, (size_t)BH * a.N * sizeof(int32_t), s);
-        if (e == cudaSuccess && a.N > 0)
-            e = cudaMemsetAsync(a.chunk_cursor, 0, (size_t)BH * a.N * sizeof(int32_t), s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(a.dK, 0, kv_rows * a.D * sizeof(float), s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(a.dV, 0, kv_rows * a.D * sizeof(float), s);
+        if (e == cudaSuccess && a.N > 0) e = cudaMemsetAsync(a.dL, 0, chunks * a.D * sizeof(float), s);
+        if (e == cudaSuccess && a.N > 0) e = cudaMemsetAsync(a.chunk_count, 0, chunks * sizeof(int32_t), s);
+        if (e == cudaSuccess && a.N > 0) e = cudaMemsetAsync(a.chunk_cursor, 0, chunks * sizeof(int32_t), s);
         if (e == cudaSuccess && a.err) e = cudaMemsetAsync(a.err, 0, sizeof(int32_t), s);
         // with chunks, dq_finish_kernel writes every row of dQs
         if (e == cudaSuccess && a.dQs && a.N == 0) e = cudaMemsetAsync(a.dQs, 0, rows * a.D * sizeof(float), s);
@@ -423,7 +424,7 @@ cudaError_t launch_backward(const BackwardArgs &a0, cudaStream_t s) {
     // head dim 128: tcgen05 kernel over work units of up to kBwdUnitPairs pairs of one chunk;
     // head dim 64: the mma.sync kernel over tiles of kPairTile pairs
     const bool tc = a.D == 128;
-    e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.tile_off,
+    e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, G, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.tile_off,
                         a.chunk_cursor, a.pair_row, a.pair_w, a.pair_slot, a.tiles, a.num_tiles, a.max_tiles,
                         tc ? kBwdUnitPairs : kPairTile, false, s);
     if (e != cudaSuccess) return e;
@@ -446,11 +447,11 @@ cudaError_t launch_backward(const BackwardArgs &a0, cudaStream_t s) {
         const unsigned blocks = (unsigned)((rows + 7) / 8);
         auto kern = a.D == 128 ? (a0.qk_norm ? dq_finish_kernel<128, true> : dq_finish_kernel<128, false>)
                                : (a0.qk_norm ? dq_finish_kernel<64, true> : dq_finish_kernel<64, false>);
-        kern<<<blocks, 256, 0, s>>>(a.sel_idx, a.ds_pair, a.L, a.T, a.N, a.topk, a.scale, rows, a0.Q, a.dQ, a.dQs);
+        kern<<<blocks, 256, 0, s>>>(a.sel_idx, a.ds_pair, a.L, a.T, a.N, a.topk, G, a.scale, rows, a0.Q, a.dQ, a.dQs);
         e = cudaGetLastError();
     }
     if (e != cudaSuccess || !a0.qk_norm) return e;
-    return launch_l2norm_grad_rows(a0.K, a.dK, rows, a.D, s);
+    return launch_l2norm_grad_rows(a0.K, a.dK, kv_rows, a.D, s);
 }
 
 }  // namespace hsa

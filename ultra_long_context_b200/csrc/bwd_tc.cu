@@ -548,7 +548,7 @@ cudaError_t launch_backward_tc(const BackwardArgs &a, cudaStream_t s) {
     auto kern = a.Qs ? chunk_bwd_tc_kernel<true> : chunk_bwd_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const uint64_t rows = (uint64_t)a.B * a.H * a.T;
+    const uint64_t rows = (uint64_t)a.B * a.Hkv * a.T;  // units address K, V by key head (chunk id / N)
     CUtensorMap tk, tv;
     if (!make_tmap_bf16(&tk, a.K, rows, a.D, kChunk) || !make_tmap_bf16(&tv, a.V, rows, a.D, kChunk))
         return cudaErrorInvalidValue;

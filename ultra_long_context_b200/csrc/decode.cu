@@ -82,7 +82,7 @@ __device__ inline int compact_at_least(uint64_t *keys, int n, uint64_t tau, int 
 template <int D>
 __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ Lc, const int64_t *__restrict__ cache_len, int H,
-    int64_t Nmax, int split, int nsplit, int K, float scale, uint64_t *__restrict__ cand, unsigned *counters,
+    int Gh, int64_t Nmax, int split, int nsplit, int K, float scale, uint64_t *__restrict__ cand, unsigned *counters,
     int32_t *__restrict__ sel_idx, float *__restrict__ sel_w) {
     constexpr int LPL = D / 8;              // lanes per landmark (one 16-byte vector each)
     constexpr int LPW = 32 / LPL;           // landmarks per warp-wide load
@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
     // the attend kernel may be scheduled now: it waits (griddepcontrol.wait) for this grid to complete
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int sp = blockIdx.x, bh = blockIdx.y, b = bh / H;
+    const int sp = blockIdx.x, bh = blockIdx.y, b = bh / H, kvh = bh / Gh;  // Gh query heads per landmark head
     int64_t nb = cache_len[b] / kChunk;
     nb = nb < 0 ? 0 : (nb > Nmax ? Nmax : nb);
     const int64_t c0 = (int64_t)sp * split;
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
         qr[4] = bf16_lo(v.z) * scale; qr[5] = bf16_hi(v.z) * scale;
         qr[6] = bf16_lo(v.w) * scale; qr[7] = bf16_hi(v.w) * scale;
     }
-    const uint16_t *Lbh = Lc + (size_t)bh * Nmax * D;
+    const uint16_t *Lbh = Lc + (size_t)kvh * Nmax * D;
     for (int64_t base = c0 + (int64_t)warp * WARP_SPAN; base < c1; base += (int64_t)NWARP * WARP_SPAN) {
         uint4 v[UNROLL];
 #pragma unroll
@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
 template <int D, bool QKN>
 __global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ Kc, const uint16_t *__restrict__ Vc, int64_t Tmax,
-    int K, float scale, const int32_t *__restrict__ sel_idx, const float *__restrict__ sel_w,
+    int Gh, int K, float scale, const int32_t *__restrict__ sel_idx, const float *__restrict__ sel_w,
     float *__restrict__ partial, unsigned *counters, uint16_t *__restrict__ out) {
     constexpr int LPL = D / 8, LPW = 32 / LPL, NWARP = kDecodeThreads / 32;
     constexpr int GROUPS = kDecodeThreads / LPL;  // key groups for the P.V pass
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
 #pragma unroll
             for (int e = 0; e < 8; ++e) qr[e] *= rq;
         }
-        const size_t row0 = ((size_t)bh * Tmax + (size_t)c * kChunk);
+        const size_t row0 = ((size_t)(bh / Gh) * Tmax + (size_t)c * kChunk);  // the key head's cache
         constexpr int ROUNDS = kChunk / (NWARP * LPW);
         const int sl = tid % LPL, grp = tid / LPL;
         // issue every K and V load of this thread up front so both overlap the logit math
@@ -381,11 +381,14 @@ static cudaError_t launch_attend(const DecodeArgs &a, dim3 grid, cudaStream_t s)
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     auto kern = a.qk_norm ? decode_attend_kernel<D, true> : decode_attend_kernel<D, false>;
-    return cudaLaunchKernelEx(&cfg, kern, a.q, a.Kc, a.Vc, a.Tmax, a.K, a.scale, (const int32_t *)a.sel_idx,
+    return cudaLaunchKernelEx(&cfg, kern, a.q, a.Kc, a.Vc, a.Tmax, a.H / a.Hkv, a.K, a.scale, (const int32_t *)a.sel_idx,
                               (const float *)a.sel_w, a.partial, a.counters + a.B * a.H, a.out);
 }
 
-cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
+cudaError_t launch_decode(const DecodeArgs &a0, cudaStream_t s) {
+    DecodeArgs a = a0;
+    if (a.Hkv <= 0) a.Hkv = a.H;
+    if (a.H % a.Hkv != 0) return cudaErrorInvalidValue;
     const int split = decode_split_size(a.Nmax, a.K, a.B * a.H);
     const int nsplit = (int)((a.Nmax + split - 1) / split) > 0 ? (int)((a.Nmax + split - 1) / split) : 1;
     const size_t smem = decode_scan_smem(split, nsplit, a.K);
@@ -402,7 +405,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         {
             HSA_PROF("decode_scan", s);
-            decode_scan_kernel<128><<<g1, kDecodeThreads, smem, s>>>(a.qs, a.Lc, a.cache_len, a.H, a.Nmax, split,
+            decode_scan_kernel<128><<<g1, kDecodeThreads, smem, s>>>(a.qs, a.Lc, a.cache_len, a.H, a.H / a.Hkv, a.Nmax, split,
                                                                      nsplit, a.K, a.scale, a.cand, a.counters,
                                                                      a.sel_idx, a.sel_w);
         }
@@ -413,7 +416,7 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
         if (e != cudaSuccess) return e;
         {
             HSA_PROF("decode_scan", s);
-            decode_scan_kernel<64><<<g1, kDecodeThreads, smem, s>>>(a.qs, a.Lc, a.cache_len, a.H, a.Nmax, split,
+            decode_scan_kernel<64><<<g1, kDecodeThreads, smem, s>>>(a.qs, a.Lc, a.cache_len, a.H, a.H / a.Hkv, a.Nmax, split,
                                                                     nsplit, a.K, a.scale, a.cand, a.counters,
                                                                     a.sel_idx, a.sel_w);
         }

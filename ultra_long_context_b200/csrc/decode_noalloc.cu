@@ -120,7 +120,7 @@ hsa_status hsa_decode_noalloc(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_b
     hsa::DecodeArgs a{};
     a.qs = q; a.q = q; a.Kc = Kc; a.Vc = Vc; a.Lc = Lc; a.cache_len = cache_len;
     a.Tmax = Tmax; a.Nmax = Nmax;
-    a.B = B; a.H = H; a.D = D; a.K = topk;
+    a.B = B; a.H = H; a.Hkv = H; a.D = D; a.K = topk;
     a.scale = scale > 0.0f ? scale : 1.0f / sqrtf((float)D);
     a.out = out;
     a.sel_idx = sel_idx ? sel_idx : reinterpret_cast<int32_t *>(b + l.sel_idx);

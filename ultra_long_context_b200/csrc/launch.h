@@ -15,6 +15,7 @@ struct DecodeArgs {
     const int64_t *cache_len;
     int64_t Tmax, Nmax;
     int B, H, D, K;
+    int Hkv;           // key/value/landmark heads (H a multiple; query head h reads h / (H / Hkv))
     float scale;
     uint16_t *out;
     int32_t *sel_idx;  // [B*H, K] (caller's or workspace)
@@ -41,16 +42,18 @@ struct ForwardArgs {
     const uint16_t *Qs;  // retrieval queries (scores, fusion weights); Q attends
     const uint16_t *Q, *K, *V, *L;
     int B, H, T, D, N, topk;
+    int Hkv;  // key/value/landmark heads: K, V [B, Hkv, T, D], L [B, Hkv, N, D]
     float scale;
     uint16_t *out;
     int32_t *sel_idx;  // [B*H*T, topk] (caller's or workspace)
     float *sel_w;
     // workspace
     float *o_acc;          // [B*H*T, D] fp32 accumulator
-    int32_t *chunk_count;  // [B*H*N]
-    int32_t *chunk_off;    // [B*H*N + 1]
-    int32_t *tile_off;     // [B*H*N + 1]
-    int32_t *chunk_cursor; // [B*H*N]
+    // chunk ids are flat over the key heads: (b*Hkv + h / (H / Hkv)) * N + c
+    int32_t *chunk_count;  // [B*Hkv*N]
+    int32_t *chunk_off;    // [B*Hkv*N + 1]
+    int32_t *tile_off;     // [B*Hkv*N + 1]
+    int32_t *chunk_cursor; // [B*Hkv*N]
     int32_t *pair_row;     // [B*H*T*topk] flat token row (b*H + h)*T + t
     float *pair_w;         // [B*H*T*topk]
     PairTile *tiles;       // [max_tiles]
@@ -59,7 +62,7 @@ struct ForwardArgs {
     int max_tiles;
     // query-key normalisation: Q and K are normalised into these bf16 workspace copies first
     bool qk_norm;
-    uint16_t *Qn, *Kn;     // [B*H*T, D] each
+    uint16_t *Qn, *Kn;     // [B*H*T, D] and [B*Hkv*T, D]
 };
 size_t forward_max_tiles(int B, int H, int T, int topk);
 // Step 2 scores + top-K + fusion weights on the tcgen05 tensor cores (score_tc.cu).
@@ -68,8 +71,9 @@ cudaError_t launch_score_tc(const ForwardArgs &a, cudaStream_t s);
 cudaError_t launch_attn_tc(const ForwardArgs &a, cudaStream_t s);
 cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s);
 // Chunk-major dispatch shared by the forward and the backward: per-chunk pair counts, offsets, the
-// tile work list, and the (token row, weight[, slot]) pair arrays.
-cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, int H, int T, int N, int topk,
+// tile work list, and the (token row, weight[, slot]) pair arrays. G query heads share a key head;
+// the chunk lists are per key head, so a chunk's list holds the pairs of every query head of its group.
+cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, int H, int G, int T, int N, int topk,
                             int32_t *chunk_count, int32_t *chunk_off, int32_t *tile_off, int32_t *chunk_cursor,
                             int32_t *pair_row,
                             float *pair_w, int32_t *pair_slot, PairTile *tiles, int32_t *num_tiles, int max_tiles,
@@ -83,6 +87,7 @@ struct BackwardArgs {
     const int32_t *sel_idx;
     const float *sel_w;
     int B, H, T, D, N, topk;
+    int Hkv;  // key/value/landmark heads: K, V, dK, dV [B, Hkv, T, D], L, dL [B, Hkv, N, D]
     float scale;
     float *dQ, *dK, *dV, *dL;
     // workspace (shares the dispatch layout of the forward)
@@ -98,7 +103,7 @@ struct BackwardArgs {
     // run on them (with the raw Q as retrieval query when there is no Qs), and dQ / dK go back
     // through the normalisation at the end
     bool qk_norm;
-    uint16_t *Qn, *Kn;     // [B*H*T, D] each
+    uint16_t *Qn, *Kn;     // [B*H*T, D] and [B*Hkv*T, D]
 };
 cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s);
 // Gradients on the tcgen05 tensor cores (bwd_tc.cu), head dim 128; work units of up to 1024 pairs.

@@ -75,7 +75,7 @@ struct StSmem {
 
 template <int D, int K>
 __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_t *__restrict__ Q, int T, int N,
-                                                                   float scale, int kout,
+                                                                   int Gh, float scale, int kout,
                                                                    int32_t *__restrict__ sel_idx,
                                                                    float *__restrict__ sel_w, float *__restrict__ o_acc,
                                                                    int32_t *__restrict__ chunk_count,
@@ -96,7 +96,7 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ntile = (T + kStRows - 1) / kStRows;
     const int tile = ntile - 1 - blockIdx.x;  // longest rows first
-    const int bh = blockIdx.y;
+    const int bh = blockIdx.y, kvh = bh / Gh;  // Gh query heads share a landmark head
     const int t0 = tile * kStRows;
     const int nrows = min(kStRows, T - t0);
     const int t_last = t0 + nrows - 1;
@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
                 tc::mbar_arrive_expect_tx(full_l(st), SM::LB);
 #pragma unroll
                 for (int k = 0; k < SM::KH; ++k)
-                    tc::tma_load_2d(dst + k * SM::LH, &tmL, k * 64, bh * N + (h % nblk) * kStCols, full_l(st));
+                    tc::tma_load_2d(dst + k * SM::LH, &tmL, k * 64, kvh * N + (h % nblk) * kStCols, full_l(st));
             };
             int nload = 0, nmma = 0;
             for (; nload < kStLStages && nload < G; ++nload) load_l(nload);
@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
                 st_idx[tid * kout + slot] = cc[128 * k];
                 st_w[tid * kout + slot] = expf(x - top) * rz;
                 if (hist_smem) atomicAdd(&s_hist[cc[128 * k]], 1);
-                else atomicAdd(&chunk_count[(size_t)bh * N + cc[128 * k]], 1);
+                else atomicAdd(&chunk_count[(size_t)kvh * N + cc[128 * k]], 1);
             }
             for (int i = 0; i < kout; ++i)
                 if (!((used >> i) & 1ull)) {
@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
         }
         if (hist_smem)  // the tile's per-chunk counts into the dispatch's histogram
             for (int i = tid; i < n_max; i += kStConsumers)
-                if (s_hist[i]) atomicAdd(&chunk_count[(size_t)bh * N + i], s_hist[i]);
+                if (s_hist[i]) atomicAdd(&chunk_count[(size_t)kvh * N + i], s_hist[i]);
         if (!ok && lane == 0) atomicOr(err, 1);
     }
     tc::fence_before();
@@ -337,8 +337,8 @@ static cudaError_t launch_st(const ForwardArgs &a, const CUtensorMap &tl, cudaSt
     if (e != cudaSuccess) return e;
     dim3 grid((a.T + kStRows - 1) / kStRows, a.B * a.H);
     HSA_PROF("score_topk", s);
-    score_topk_tc_kernel<D, K><<<grid, kStThreads, smem, s>>>(a.Qs, a.T, a.N, a.scale, a.topk, a.sel_idx, a.sel_w,
-                                                              a.o_acc, a.chunk_count, a.err, tl);
+    score_topk_tc_kernel<D, K><<<grid, kStThreads, smem, s>>>(a.Qs, a.T, a.N, a.H / a.Hkv, a.scale, a.topk,
+                                                              a.sel_idx, a.sel_w, a.o_acc, a.chunk_count, a.err, tl);
     return cudaGetLastError();
 }
 
@@ -347,7 +347,7 @@ static cudaError_t launch_st_d(const ForwardArgs &a, cudaStream_t s) {
     CUtensorMap tl;
     // with no complete chunk the landmark tensor may be empty: point the map at Q (never read)
     if (!make_tmap_bf16(&tl, a.N > 0 ? (const void *)a.L : (const void *)a.Q,
-                 a.N > 0 ? (uint64_t)a.B * a.H * a.N : (uint64_t)a.B * a.H * a.T, D, kStCols))
+                 a.N > 0 ? (uint64_t)a.B * a.Hkv * a.N : (uint64_t)a.B * a.H * a.T, D, kStCols))
         return cudaErrorInvalidValue;
     if (a.topk <= 8) return launch_st<D, 8>(a, tl, s);
     if (a.topk <= 16) return launch_st<D, 16>(a, tl, s);

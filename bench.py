@@ -407,8 +407,31 @@ def main():
         opts["separate_retrieval_query"] = {
             "ms_per_step": round(s_ms, 4), "tokens_per_s": round(whole_job_rate(w.B * w.T, world, s_ms), 1),
             "vs_plain": round(s_ms / ms_per_step, 4)}
-        extra["fwd_options"] = dict(workload=w.name, steps=osteps, **opts)
         del ws_n, Qs_
+        # 16 query heads per key/value head (the pages' ratio): B1 H16 Hkv1, the same query rows and pairs
+        # as the headline workload, one K/V/L head
+        Hg, Hkv_g, Bg = 16, 1, 1
+        gQ = inputs.forward_inputs(Bg, Hg, w.T, w.D, w.seed + 11 + rank, landmarks=w.landmarks, device=dev)[0]
+        _, gK, gV, gL = inputs.forward_inputs(Bg, Hkv_g, w.T, w.D, w.seed + 12 + rank, landmarks=w.landmarks,
+                                              device=dev)
+        gout = torch.empty_like(gQ)
+        gidx = torch.empty((Bg, Hg, w.T, w.topk), dtype=torch.int32, device=dev)
+        gw = torch.empty((Bg, Hg, w.T, w.topk), dtype=torch.float32, device=dev)
+        gws = torch.empty(hsa.hsa_forward_ex_workspace_size(Bg, Hg, Hkv_g, w.T, w.D, w.chunk, w.topk, 0) + 256,
+                          dtype=torch.uint8, device=dev)
+
+        def fwd_gqa():
+            hsa.hsa_forward(gQ, gK, gV, gL, w.topk, out=gout, sel_idx=gidx, sel_w=gw, workspace=gws)
+
+        g_ms = timed(fwd_gqa, osteps, args.warmup, world) / osteps
+        prof_g = kernel_profile(fwd_gqa, osteps)
+        opts["grouped_heads_16to1"] = {
+            "shape": f"B{Bg} H{Hg} Hkv{Hkv_g} T{w.T} D{w.D} topk{w.topk}", "ms_per_step": round(g_ms, 4),
+            "tokens_per_s": round(whole_job_rate(Bg * w.T, world, g_ms), 1),
+            "token_heads_per_s": round(whole_job_rate(Bg * w.T * Hg, world, g_ms), 1),
+            "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_g.items()}}
+        extra["fwd_options"] = dict(workload=w.name, steps=osteps, **opts)
+        del gQ, gK, gV, gL, gout, gidx, gw, gws
         torch.cuda.empty_cache()
 
     # ---------------- decode, 16M-token cache ----------------
@@ -448,6 +471,30 @@ def main():
         }
         del q, Kc, Vc, Lc, dws
         torch.cuda.empty_cache()
+        if not args.skip_options:  # 16 query heads on one key/value head, same cache length
+            Hg = 16
+            gq = inputs.decode_inputs(wd.B, Hg, 0, wd.D, seed=wd.seed + 3, Tmax=64, device=dev)[0]
+            _, gKc, gVc, gLc, glens, _ = inputs.decode_inputs(wd.B, 1, wd.cache_len, wd.D, seed=wd.seed + 4,
+                                                              device=dev)
+            gout_ = torch.empty_like(gq)
+            gidx_ = torch.empty((wd.B, Hg, wd.topk), dtype=torch.int32, device=dev)
+            gw_ = torch.empty((wd.B, Hg, wd.topk), dtype=torch.float32, device=dev)
+            gdws = torch.empty(hsa.hsa_decode_ex_workspace_size(wd.B, Hg, 1, wd.cache_len, wd.D, 64, wd.topk, 0) + 256,
+                               dtype=torch.uint8, device=dev)
+
+            def dec_gqa():
+                hsa.hsa_decode(gq, gKc, gVc, gLc, glens, wd.topk, out=gout_, sel_idx=gidx_, sel_w=gw_, workspace=gdws)
+
+            gms = timed(dec_gqa, dsteps, args.warmup, world) / dsteps
+            prof_gd = kernel_profile(dec_gqa, dsteps)
+            lm_bytes = wd.B * (n * wd.D * 2)  # one landmark head, read once from HBM at best
+            extra["decode_16m"]["grouped_heads_16to1"] = {
+                "shape": f"B{wd.B} H{Hg} Hkv1 cache {wd.cache_len} D{wd.D} topk{wd.topk}",
+                "us_per_token": round(gms * 1e3 / wd.B, 3),
+                "landmark_bytes": lm_bytes,
+                "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_gd.items()}}
+            del gq, gKc, gVc, gLc, gdws
+            torch.cuda.empty_cache()
 
     # ---------------- forward + backward, 64K ----------------
     if not args.skip_backward:

@@ -113,7 +113,7 @@ __device__ __forceinline__ void epilogue_slabs(uint32_t tO, int cb0, int cb1, in
 
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
-    const uint16_t *__restrict__ Q, int T, int N, float scale, const PairTile *__restrict__ tiles,
+    const uint16_t *__restrict__ Q, int T, int N, int Gh, float scale, const PairTile *__restrict__ tiles,
     const int32_t *__restrict__ num_tiles, const int32_t *__restrict__ pair_row, const float *__restrict__ pair_w,
     float *__restrict__ o_acc, int32_t *__restrict__ err, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV) {
@@ -179,10 +179,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
             if (!ok) break;
             const uint32_t sqa = sb + SM::OPS + sq * SM::QK;
             if (lt == 0) {
-                const int bh = t.chunk / N, c = t.chunk % N;
+                const int kvh = t.chunk / N / Gh, c = t.chunk % N;  // Gh query heads per key head
                 tc::mbar_expect_tx(bar(kQkFull + sq), SM::KB);  // this thread arrives below, after its copies
                 tc::mbar_expect_tx(bar(kVFull + sv), SM::KB);
-                const int y = bh * T + c * kChunk;
+                const int y = kvh * T + c * kChunk;
 #pragma unroll
                 for (int h = 0; h < SM::KH; ++h) {
                     tc::tma_load_2d(sqa + SM::QB + h * 8192, &tmK, h * 64, y, bar(kQkFull + sq));
@@ -394,15 +394,15 @@ static cudaError_t launch_attn_tc_d(const ForwardArgs &a, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(chunk_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const uint64_t rows = (uint64_t)a.B * a.Hkv * a.T;  // tiles address K, V by key head (chunk id / N)
+    const uint64_t rows = (uint64_t)a.B * a.Hkv * a.T;  // tiles address K, V by key head
     CUtensorMap tk, tv;
     if (!make_tmap_bf16(&tk, a.K, rows, D, kChunk) || !make_tmap_bf16(&tv, a.V, rows, D, kChunk)) return cudaErrorInvalidValue;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = sms < a.max_tiles ? sms : a.max_tiles;
     HSA_PROF("chunk_attn", s);
-    chunk_attn_tc_kernel<D><<<grid, kTcThreads, smem, s>>>(a.Q, a.T, a.N, a.scale, a.tiles, a.num_tiles, a.pair_row,
-                                                            a.pair_w, a.o_acc, a.err, tk, tv);
+    chunk_attn_tc_kernel<D><<<grid, kTcThreads, smem, s>>>(a.Q, a.T, a.N, a.H / a.Hkv, a.scale, a.tiles,
+                                                            a.num_tiles, a.pair_row, a.pair_w, a.o_acc, a.err, tk, tv);
     return cudaGetLastError();
 }
 

@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
     float scale, const PairTile *__restrict__ tiles, const int32_t *__restrict__ num_tiles,
     const int32_t *__restrict__ pair_row, const float *__restrict__ pair_w, float *__restrict__ dQ,
     float *__restrict__ dK, float *__restrict__ dV, float *__restrict__ dL, const uint16_t *__restrict__ Qs,
-    const int32_t *__restrict__ pair_slot, float *__restrict__ ds_pair, int Kslots) {
+    const int32_t *__restrict__ pair_slot, float *__restrict__ ds_pair, int Kslots, int Gh) {
     // Qs != NULL: separate retrieval queries. dL takes ds times the retrieval query, dQ leaves out the
     // ds L_c term, and ds goes to ds_pair[token row, slot] for the retrieval query's gradient.
     using SM = BwdSmem<D>;
@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(kBwdThreads) chunk_bwd_kernel(
     if ((int)blockIdx.x >= num_tiles[0]) return;
     const PairTile pt = tiles[blockIdx.x];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int bh = pt.chunk / N, c = pt.chunk % N;
+    const int bh = pt.chunk / N / Gh, c = pt.chunk % N;  // key head (Gh query heads per key head)
     const size_t krow0 = (size_t)bh * T + (size_t)c * kChunk;
     if (tid < kPairTile) {
         const bool ok = tid < pt.count;
@@ -391,7 +391,7 @@ cudaError_t launch_backward(const BackwardArgs &a0, cudaStream_t s) {
     if (a.Hkv <= 0) a.Hkv = a.H;
     if (a.H % a.Hkv != 0) return cudaErrorInvalidValue;
     const int G = a.H / a.Hkv;  // query heads per key head
-    const size_t kv_rows = (size_t)a.B * a.Hkv * a.T, chunks = (size_t)a.B * a.Hkv * a.N;
+    const size_t kv_rows = (size_t)a.B * a.Hkv * a.T, chunks = (size_t)a.B * a.H * a.N;
     if (a0.qk_norm) {  // the kernels run on the normalised Q and K; the raw Q retrieves unless Qs does
         cudaError_t e = launch_l2norm_rows(a0.Q, a0.Qn, (size_t)a.B * a.H * a.T, a0.K, a0.Kn, kv_rows, a.D, s);
         if (e != cudaSuccess) return e;
@@ -407,7 +407,8 @@ cudaError_t launch_backward(const BackwardArgs &a0, cudaStream_t s) {
         e = cudaMemsetAsync(a.dQ, 0, rows * a.D * sizeof(float), s);
         if (e == cudaSuccess) e = cudaMemsetAsync(a.dK, 0, kv_rows * a.D * sizeof(float), s);
         if (e == cudaSuccess) e = cudaMemsetAsync(a.dV, 0, kv_rows * a.D * sizeof(float), s);
-        if (e == cudaSuccess && a.N > 0) e = cudaMemsetAsync(a.dL, 0, chunks * a.D * sizeof(float), s);
+        if (e == cudaSuccess && a.N > 0)
+            e = cudaMemsetAsync(a.dL, 0, (size_t)a.B * a.Hkv * a.N * a.D * sizeof(float), s);
         if (e == cudaSuccess && a.N > 0) e = cudaMemsetAsync(a.chunk_count, 0, chunks * sizeof(int32_t), s);
         if (e == cudaSuccess && a.N > 0) e = cudaMemsetAsync(a.chunk_cursor, 0, chunks * sizeof(int32_t), s);
         if (e == cudaSuccess && a.err) e = cudaMemsetAsync(a.err, 0, sizeof(int32_t), s);
@@ -424,7 +425,7 @@ cudaError_t launch_backward(const BackwardArgs &a0, cudaStream_t s) {
     // head dim 128: tcgen05 kernel over work units of up to kBwdUnitPairs pairs of one chunk;
     // head dim 64: the mma.sync kernel over tiles of kPairTile pairs
     const bool tc = a.D == 128;
-    e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, G, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.tile_off,
+    e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.tile_off,
                         a.chunk_cursor, a.pair_row, a.pair_w, a.pair_slot, a.tiles, a.num_tiles, a.max_tiles,
                         tc ? kBwdUnitPairs : kPairTile, false, s);
     if (e != cudaSuccess) return e;
@@ -438,7 +439,7 @@ cudaError_t launch_backward(const BackwardArgs &a0, cudaStream_t s) {
         chunk_bwd_kernel<64><<<a.max_tiles, kBwdThreads, smem, s>>>(a.Q, a.K, a.V, a.L, a.dout, a.delta, a.T, a.N,
                                                                      a.scale, a.tiles, a.num_tiles, a.pair_row,
                                                                      a.pair_w, a.dQ, a.dK, a.dV, a.dL, a.Qs,
-                                                                     a.pair_slot, a.ds_pair, a.topk);
+                                                                     a.pair_slot, a.ds_pair, a.topk, G);
         e = cudaGetLastError();
     }
     if (e != cudaSuccess || !a.Qs) return e;

@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
     const int32_t *__restrict__ num_units, const int32_t *__restrict__ pair_row, const float *__restrict__ pair_w,
     float *__restrict__ dQ, float *__restrict__ dK, float *__restrict__ dV, float *__restrict__ dL,
     int32_t *__restrict__ err, const uint16_t *__restrict__ Qs, const int32_t *__restrict__ pair_slot,
-    float *__restrict__ ds_pair, int Kslots, const __grid_constant__ CUtensorMap tmK,
+    float *__restrict__ ds_pair, int Kslots, int Gh, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV) {
     // QSLC: separate retrieval queries Qs. dL takes ds times the retrieval query (read from global
     // memory), dQ leaves out the ds L_c term, and ds goes to ds_pair[token row, slot].
@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                 own[1] = make_float4(x1.x + a8[4], x1.y + a8[5], x1.z + a8[6], x1.w + a8[7]);
             }
             if (lag.last_tile()) {  // the unit's dL: thread lt = column d
-                const int bhl = lag.u.chunk / N, cl = lag.u.chunk % N;
+                const int bhl = lag.u.chunk / N / Gh, cl = lag.u.chunk % N;  // key head
                 asm volatile("bar.sync 2, 128;" ::: "memory");  // every loader warp's partials are in s_dl
                 atomicAdd(dL + ((size_t)bhl * N + cl) * D + lt,
                           scale * ((s_dl[lt] + s_dl[D + lt]) + (s_dl[2 * D + lt] + s_dl[3 * D + lt])));
@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
         };
         for (; !cur.done() && ok; cur.next()) {
             const int j = cur.j, st = j & 1;
-            const int bh = cur.u.chunk / N, c = cur.u.chunk % N;
+            const int bh = cur.u.chunk / N / Gh, c = cur.u.chunk % N;  // key head
             if (j >= 2) do_dl();  // the stage about to be reloaded holds tile j - 2
             ok = ok && tc::mbar_wait(bar(kBQdEmpty + st), ((uint32_t)(j >> 1) & 1u) ^ 1u);
             if (!ok) break;
@@ -285,7 +285,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                     }
                     if (cur.k + 1 < mine) {
                         const PairTile nu = units[blockIdx.x + (size_t)(cur.k + 1) * G];
-                        const int yn = (nu.chunk / N) * T + (nu.chunk % N) * kChunk;
+                        const int yn = (nu.chunk / N / Gh) * T + (nu.chunk % N) * kChunk;
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             tc::tma_prefetch_2d(&tmK, h * 64, yn);
@@ -395,7 +395,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                 // the unit's landmark row (fp32) for the ds L_c term of dQ, slot k % 4: the dQ epilogue
                 // of unit k - 4 is done with that slot, since this tile's S needed unit k - 1's last
                 // MMA, which needed the epilogue of a tile after unit k - 4's last
-                const int bhu = cur.u.chunk / N, cu = cur.u.chunk % N;
+                const int bhu = cur.u.chunk / N / Gh, cu = cur.u.chunk % N;  // key head
                 s_L[(cur.k & 3) * 128 + r] = __uint_as_float((uint32_t)L[((size_t)bhu * N + cu) * D + r] << 16);
             }
             const uint32_t tS = tmem + lane_off + SM::S_COL;
@@ -516,7 +516,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                 ok = tc::mbar_wait(bar(kBAccFull), (uint32_t)cur.k & 1u);
                 if (!ok) break;
                 tc::fence_after();
-                const int bh = cur.u.chunk / N, c = cur.u.chunk % N;
+                const int bh = cur.u.chunk / N / Gh, c = cur.u.chunk % N;  // key head
                 const size_t krow0 = (size_t)bh * T + (size_t)c * kChunk;
                 float *dst = e == 0 ? dV : dK;
                 const float f = e == 0 ? 1.0f : scale;
@@ -548,7 +548,7 @@ cudaError_t launch_backward_tc(const BackwardArgs &a, cudaStream_t s) {
     auto kern = a.Qs ? chunk_bwd_tc_kernel<true> : chunk_bwd_tc_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const uint64_t rows = (uint64_t)a.B * a.Hkv * a.T;  // units address K, V by key head (chunk id / N)
+    const uint64_t rows = (uint64_t)a.B * a.Hkv * a.T;  // units address K, V by key head
     CUtensorMap tk, tv;
     if (!make_tmap_bf16(&tk, a.K, rows, a.D, kChunk) || !make_tmap_bf16(&tv, a.V, rows, a.D, kChunk))
         return cudaErrorInvalidValue;
@@ -558,7 +558,7 @@ cudaError_t launch_backward_tc(const BackwardArgs &a, cudaStream_t s) {
     HSA_PROF("chunk_bwd", s);
     kern<<<grid, kBtThreads, smem, s>>>(a.Q, a.L, a.dout, a.delta, a.T, a.N, a.scale, a.tiles, a.num_tiles,
                                         a.pair_row, a.pair_w, a.dQ, a.dK, a.dV, a.dL, a.err, a.Qs, a.pair_slot,
-                                        a.ds_pair, a.topk, tk, tv);
+                                        a.ds_pair, a.topk, a.H / a.Hkv, tk, tv);
     return cudaGetLastError();
 }
 

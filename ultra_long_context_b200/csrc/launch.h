@@ -49,11 +49,12 @@ struct ForwardArgs {
     float *sel_w;
     // workspace
     float *o_acc;          // [B*H*T, D] fp32 accumulator
-    // chunk ids are flat over the key heads: (b*Hkv + h / (H / Hkv)) * N + c
-    int32_t *chunk_count;  // [B*Hkv*N]
-    int32_t *chunk_off;    // [B*Hkv*N + 1]
-    int32_t *tile_off;     // [B*Hkv*N + 1]
-    int32_t *chunk_cursor; // [B*Hkv*N]
+    // chunk ids are flat over the QUERY heads, (b*H + h) * N + c; a kernel that reads K, V or L for a
+    // chunk id uses key head (chunk id / N) / (H / Hkv)
+    int32_t *chunk_count;  // [B*H*N]
+    int32_t *chunk_off;    // [B*H*N + 1]
+    int32_t *tile_off;     // [B*H*N + 1]
+    int32_t *chunk_cursor; // [B*H*N]
     int32_t *pair_row;     // [B*H*T*topk] flat token row (b*H + h)*T + t
     float *pair_w;         // [B*H*T*topk]
     PairTile *tiles;       // [max_tiles]
@@ -71,9 +72,10 @@ cudaError_t launch_score_tc(const ForwardArgs &a, cudaStream_t s);
 cudaError_t launch_attn_tc(const ForwardArgs &a, cudaStream_t s);
 cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s);
 // Chunk-major dispatch shared by the forward and the backward: per-chunk pair counts, offsets, the
-// tile work list, and the (token row, weight[, slot]) pair arrays. G query heads share a key head;
-// the chunk lists are per key head, so a chunk's list holds the pairs of every query head of its group.
-cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, int H, int G, int T, int N, int topk,
+// tile work list, and the (token row, weight[, slot]) pair arrays. The lists are per query head even
+// when query heads share key heads: a tile's pairs then all write accumulator rows of one query head,
+// which keeps the rows that the concurrent tiles reduce into within L2.
+cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, int H, int T, int N, int topk,
                             int32_t *chunk_count, int32_t *chunk_off, int32_t *tile_off, int32_t *chunk_cursor,
                             int32_t *pair_row,
                             float *pair_w, int32_t *pair_slot, PairTile *tiles, int32_t *num_tiles, int max_tiles,

@@ -27,9 +27,9 @@ constexpr int kDispatchRows = 256;
 constexpr int kSmemHistMax = 8192;  // chunks per (b, h) histogrammed in shared memory
 
 __global__ void __launch_bounds__(kDispatchRows) count_kernel(const int32_t *__restrict__ sel_idx, int T, int N,
-                                                              int K, int G, int32_t *__restrict__ chunk_count) {
+                                                              int K, int32_t *__restrict__ chunk_count) {
     extern __shared__ int s_hist[];
-    const int bh = blockIdx.y, kvh = bh / G;
+    const int bh = blockIdx.y;
     const bool use_smem = N <= kSmemHistMax;
     if (use_smem) {
         for (int i = threadIdx.x; i < N; i += blockDim.x) s_hist[i] = 0;
@@ -42,13 +42,13 @@ __global__ void __launch_bounds__(kDispatchRows) count_kernel(const int32_t *__r
             const int c = si[j];
             if (c < 0 || c >= N) continue;  // -1 = empty slot; ids past N are ignored
             if (use_smem) atomicAdd(&s_hist[c], 1);
-            else atomicAdd(&chunk_count[(size_t)kvh * N + c], 1);
+            else atomicAdd(&chunk_count[(size_t)bh * N + c], 1);
         }
     }
     if (use_smem) {
         __syncthreads();
         for (int i = threadIdx.x; i < N; i += blockDim.x)
-            if (s_hist[i]) atomicAdd(&chunk_count[(size_t)kvh * N + i], s_hist[i]);
+            if (s_hist[i]) atomicAdd(&chunk_count[(size_t)bh * N + i], s_hist[i]);
     }
 }
 
@@ -133,13 +133,13 @@ __global__ void __launch_bounds__(256) tile_list_kernel(const int32_t *__restric
 
 __global__ void __launch_bounds__(kDispatchRows) scatter_kernel(const int32_t *__restrict__ sel_idx,
                                                                 const float *__restrict__ sel_w, int T, int N, int K,
-                                                                int G, const int32_t *__restrict__ chunk_off,
+                                                                const int32_t *__restrict__ chunk_off,
                                                                 int32_t *__restrict__ chunk_cursor,
                                                                 int32_t *__restrict__ pair_row,
                                                                 float *__restrict__ pair_w,
                                                                 int32_t *__restrict__ pair_slot) {
     extern __shared__ int s_mem[];
-    const int bh = blockIdx.y, kvh = bh / G;
+    const int bh = blockIdx.y;
     const bool use_smem = N <= kSmemHistMax / 2;
     int *s_cnt = s_mem, *s_base = s_mem + (use_smem ? N : 0);
     const int t = blockIdx.x * kDispatchRows + threadIdx.x;
@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_kernel(const int32_t *_
         __syncthreads();
         for (int i = threadIdx.x; i < N; i += blockDim.x) {
             const int c = s_cnt[i];
-            s_base[i] = c ? atomicAdd(&chunk_cursor[(size_t)kvh * N + i], c) : 0;
+            s_base[i] = c ? atomicAdd(&chunk_cursor[(size_t)bh * N + i], c) : 0;
             s_cnt[i] = 0;
         }
         __syncthreads();
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_kernel(const int32_t *_
     for (int j = 0; j < K; ++j) {
         const int c = si[j];
         if (c < 0 || c >= N) continue;
-        const size_t ch = (size_t)kvh * N + c;
+        const size_t ch = (size_t)bh * N + c;
         const int local = use_smem ? s_base[c] + atomicAdd(&s_cnt[c], 1) : atomicAdd(&chunk_cursor[ch], 1);
         const int pos = chunk_off[ch] + local;
         pair_row[pos] = (int32_t)row;
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_kernel(const int32_t *_
 constexpr int kSortedScatterMaxN = 2048;
 
 __global__ void __launch_bounds__(kDispatchRows) scatter_sorted_kernel(
-    const int32_t *__restrict__ sel_idx, const float *__restrict__ sel_w, int T, int N, int K, int G,
+    const int32_t *__restrict__ sel_idx, const float *__restrict__ sel_w, int T, int N, int K,
     const int32_t *__restrict__ chunk_off, int32_t *__restrict__ chunk_cursor, int32_t *__restrict__ pair_row,
     float *__restrict__ pair_w, int32_t *__restrict__ pair_slot) {
     extern __shared__ int s_mem[];
@@ -190,7 +190,7 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_sorted_kernel(
     int *s_key = s_cur + N;              // [rows * K] (c << 14) | (t_local << 6) | slot, sorted by chunk
     float *s_wt = reinterpret_cast<float *>(s_key + kDispatchRows * K);
     __shared__ int s_warp[33];
-    const int bh = blockIdx.y, kvh = bh / G, tid = threadIdx.x;
+    const int bh = blockIdx.y, tid = threadIdx.x;
     const int t0 = blockIdx.x * kDispatchRows;
     const int t = t0 + tid;
     for (int i = tid; i < N; i += blockDim.x) { s_cnt[i] = 0; s_cur[i] = 0; }
@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_sorted_kernel(
     for (int i = lo; i < hi; ++i) {
         const int cnt = s_cnt[i];
         s_scan[i] = off;
-        s_gbase[i] = cnt ? chunk_off[(size_t)kvh * N + i] + atomicAdd(&chunk_cursor[(size_t)kvh * N + i], cnt) : 0;
+        s_gbase[i] = cnt ? chunk_off[(size_t)bh * N + i] + atomicAdd(&chunk_cursor[(size_t)bh * N + i], cnt) : 0;
         off += cnt;
     }
     __syncthreads();
@@ -255,12 +255,12 @@ size_t forward_max_tiles(int B, int H, int T, int topk) {
     return pairs / kPairTile + chunks + 1;
 }
 
-cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, int H, int G, int T, int N, int topk,
+cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, int H, int T, int N, int topk,
                             int32_t *chunk_count, int32_t *chunk_off, int32_t *tile_off, int32_t *chunk_cursor,
                             int32_t *pair_row,
                             float *pair_w, int32_t *pair_slot, PairTile *tiles, int32_t *num_tiles, int max_tiles,
                             int tile_pairs, bool counts_ready, cudaStream_t s) {
-    const int BH = B * H, M = B * (H / G) * N;  // query heads; chunks over the key heads
+    const int BH = B * H, M = BH * N;
     dim3 dgrid((T + kDispatchRows - 1) / kDispatchRows, BH);
     const size_t hsmem = N <= kSmemHistMax ? (size_t)N * sizeof(int) : 0;
     if (hsmem > 48 * 1024) {
@@ -269,7 +269,7 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
     }
     if (!counts_ready) {  // the forward's score kernel has counted them already
         HSA_PROF("dispatch_count", s);
-        count_kernel<<<dgrid, kDispatchRows, hsmem, s>>>(sel_idx, T, N, topk, G, chunk_count);
+        count_kernel<<<dgrid, kDispatchRows, hsmem, s>>>(sel_idx, T, N, topk, chunk_count);
     }
     {
         HSA_PROF("dispatch_scan", s);
@@ -286,7 +286,7 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
                                              (int)ssmem);
         if (e != cudaSuccess) return e;
         HSA_PROF("dispatch_scatter", s);
-        scatter_sorted_kernel<<<dgrid, kDispatchRows, ssmem, s>>>(sel_idx, sel_w, T, N, topk, G, chunk_off,
+        scatter_sorted_kernel<<<dgrid, kDispatchRows, ssmem, s>>>(sel_idx, sel_w, T, N, topk, chunk_off,
                                                                   chunk_cursor, pair_row, pair_w, pair_slot);
     } else {
         const size_t ssmem = N <= kSmemHistMax / 2 ? 2 * (size_t)N * sizeof(int) : 0;
@@ -295,7 +295,7 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
             if (e != cudaSuccess) return e;
         }
         HSA_PROF("dispatch_scatter", s);
-        scatter_kernel<<<dgrid, kDispatchRows, ssmem, s>>>(sel_idx, sel_w, T, N, topk, G, chunk_off, chunk_cursor,
+        scatter_kernel<<<dgrid, kDispatchRows, ssmem, s>>>(sel_idx, sel_w, T, N, topk, chunk_off, chunk_cursor,
                                                            pair_row, pair_w, pair_slot);
     }
     return cudaGetLastError();
@@ -314,7 +314,7 @@ cudaError_t launch_forward(const ForwardArgs &a0, cudaStream_t s) {
         a.K = a0.Kn;
     }
     const int BH = a.B * a.H;
-    const size_t rows = (size_t)BH * a.T, chunks = (size_t)a.B * a.Hkv * a.N;
+    const size_t rows = (size_t)BH * a.T, chunks = (size_t)BH * a.N;
     cudaError_t e;
     {
         HSA_PROF("memset", s);
@@ -332,9 +332,8 @@ cudaError_t launch_forward(const ForwardArgs &a0, cudaStream_t s) {
         finalize_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a.o_acc, a.out, n8);
         return cudaGetLastError();
     }
-    e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.H / a.Hkv, a.T, a.N, a.topk, a.chunk_count, a.chunk_off,
-                        a.tile_off, a.chunk_cursor, a.pair_row, a.pair_w, nullptr, a.tiles, a.num_tiles, a.max_tiles,
-                        128, true, s);
+    e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.tile_off,
+                        a.chunk_cursor, a.pair_row, a.pair_w, nullptr, a.tiles, a.num_tiles, a.max_tiles, 128, true, s);
     if (e != cudaSuccess) return e;
     e = launch_attn_tc(a, s);
     if (e != cudaSuccess) return e;

@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
                 st_idx[tid * kout + slot] = cc[128 * k];
                 st_w[tid * kout + slot] = expf(x - top) * rz;
                 if (hist_smem) atomicAdd(&s_hist[cc[128 * k]], 1);
-                else atomicAdd(&chunk_count[(size_t)kvh * N + cc[128 * k]], 1);
+                else atomicAdd(&chunk_count[(size_t)bh * N + cc[128 * k]], 1);
             }
             for (int i = 0; i < kout; ++i)
                 if (!((used >> i) & 1ull)) {
@@ -318,7 +318,7 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
         }
         if (hist_smem)  // the tile's per-chunk counts into the dispatch's histogram
             for (int i = tid; i < n_max; i += kStConsumers)
-                if (s_hist[i]) atomicAdd(&chunk_count[(size_t)kvh * N + i], s_hist[i]);
+                if (s_hist[i]) atomicAdd(&chunk_count[(size_t)bh * N + i], s_hist[i]);
         if (!ok && lane == 0) atomicOr(err, 1);
     }
     tc::fence_before();

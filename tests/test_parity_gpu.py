@@ -391,12 +391,31 @@ def test_forward_grouped_heads_match_oracle(oracle_mod, B, H, Hkv, T, D, topk, o
                          orc, Qh, Kh, Vh, Lh, np.arange(B * H * T), 64, sc, Qs=Qsh, qk_norm=qk)
 
 
-@pytest.mark.parametrize("B,H,Hkv,D,lens,topk", [(2, 4, 2, 128, [9000, 4100], 16), (1, 8, 1, 64, [64 * 700 + 5], 32)])
+@pytest.mark.parametrize("B,H,Hkv,D,lens,topk", [
+    (2, 4, 2, 128, [9000, 4100], 16), (1, 8, 1, 64, [64 * 700 + 5], 32),
+    (1, 16, 1, 128, [64 * 5000 + 17], 32),          # 16 heads per key head, several ranges, ragged tail
+    (4, 6, 2, 64, [0, 63, 64 * 20 + 3, 64 * 40], 8),  # empty caches and ranges shorter than 32 landmarks
+    (1, 4, 1, 128, [64 * 3000], 40),                # topk above 32: the per-head scan serves it
+])
 def test_decode_grouped_heads_match_oracle(oracle_mod, B, H, Hkv, D, lens, topk):
     Tmax = max(lens) + 64
     q = inputs.decode_inputs(B, H, lens, D, seed=51 + D, Tmax=Tmax, device=DEV)[0]
     _, Kc, Vc, Lc, lens_t, _ = inputs.decode_inputs(B, Hkv, lens, D, seed=52 + D, Tmax=Tmax, device=DEV)
-    check_decode(oracle_mod, q, Kc, Vc, Lc, lens_t, topk)
+    out, idx, w = check_decode(oracle_mod, q, Kc, Vc, Lc, lens_t, topk)
+    for b in range(B):
+        if lens[b] < 64:
+            assert torch.all(out[b] == 0) and torch.all(idx[b] == -1) and torch.all(w[b] == 0)
+
+
+def test_decode_grouped_heads_equal_landmarks_keep_lowest_chunks():
+    B, H, Hkv, D, topk = 1, 8, 2, 128, 16
+    lens = [64 * 3000]
+    q = inputs.decode_inputs(B, H, lens, D, seed=61, device=DEV)[0]
+    _, Kc, Vc, Lc, lens_t, _ = inputs.decode_inputs(B, Hkv, lens, D, seed=62, device=DEV)
+    Lc[:] = Lc[:, :, :1]
+    _, idx, w = hsa.hsa_decode(q, Kc, Vc, Lc, lens_t, topk)
+    assert torch.equal(idx.cpu(), torch.arange(topk, dtype=torch.int32).expand(B, H, topk))
+    assert torch.allclose(w, torch.full_like(w, 1.0 / topk))
 
 
 @pytest.mark.parametrize("B,H,Hkv,T,D,topk,opts", [

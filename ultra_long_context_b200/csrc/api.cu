@@ -121,12 +121,11 @@ struct DecLayout {
     size_t bytes;
 };
 
-DecLayout dec_layout(void *ws, int B, int H, int64_t Tmax, int D, int topk) {
+DecLayout dec_layout(void *ws, int B, int H, int Hkv, int64_t Tmax, int D, int topk) {
     DecLayout l{};
     Carver c{static_cast<char *>(ws)};
-    const int64_t Nmax = Tmax / 64;
-    const int split = hsa::decode_split_size(Nmax, topk, B * H);
-    const int64_t nsplit = Nmax > 0 ? (Nmax + split - 1) / split : 1;
+    const hsa::DecodePlan pl = hsa::decode_plan(Tmax / 64, topk, B, H, Hkv);
+    const int64_t nsplit = pl.nsplit;
     const size_t BH = (size_t)B * H;
     l.err = c.take<int32_t>(1);  // first: hsa_workspace_status reads it at offset 0
     l.cand = c.take<uint64_t>(BH * nsplit * topk);
@@ -244,14 +243,14 @@ hsa_status hsa_forward_ex(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 
 size_t hsa_decode_workspace_size(int B, int H, int64_t Tmax, int D, int chunk, int topk) {
     (void)chunk;
     if (B < 1 || H < 1 || Tmax < 0 || D < 1 || topk < 1) return 0;
-    return dec_layout(nullptr, B, H, Tmax, D, topk).bytes;
+    return dec_layout(nullptr, B, H, H, Tmax, D, topk).bytes;
 }
 
 size_t hsa_decode_ex_workspace_size(int B, int H, int Hkv, int64_t Tmax, int D, int chunk, int topk, unsigned flags) {
     (void)chunk;
     (void)flags;
-    if (B < 1 || H < 1 || Hkv < 1 || Tmax < 0 || D < 1 || topk < 1) return 0;
-    return dec_layout(nullptr, B, H, Tmax, D, topk).bytes;
+    if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || Tmax < 0 || D < 1 || topk < 1) return 0;
+    return dec_layout(nullptr, B, H, Hkv, Tmax, D, topk).bytes;
 }
 
 static hsa_status decode_impl(const char *name, const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *Kc,
@@ -271,17 +270,12 @@ static hsa_status decode_impl(const char *name, const hsa_bf16 *qs, const hsa_bf
         return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned (cache_len 8-byte)");
     if ((sel_idx && !aligned16(sel_idx)) || (sel_w && !aligned16(sel_w)))
         return fail(HSA_ERR_INVALID_ARG, "sel_idx / sel_w must be 16-byte aligned");
-    {
-        const int64_t Nmax = Tmax / 64;
-        const int split = hsa::decode_split_size(Nmax, topk, B * H);
-        const int64_t nsplit = Nmax > 0 ? (Nmax + split - 1) / split : 1;
-        if (hsa::decode_scan_smem(split, (int)nsplit, topk) > 227 * 1024)
-            return fail(HSA_ERR_UNSUPPORTED, "Tmax=%lld too large for topk=%d (scan merge exceeds shared memory)",
-                        (long long)Tmax, topk);
-    }
-    DecLayout need = dec_layout(nullptr, B, H, Tmax, D, topk);
+    if (hsa::decode_plan_smem(hsa::decode_plan(Tmax / 64, topk, B, H, Hkv), topk) > 227 * 1024)
+        return fail(HSA_ERR_UNSUPPORTED, "Tmax=%lld too large for topk=%d (scan merge exceeds shared memory)",
+                    (long long)Tmax, topk);
+    DecLayout need = dec_layout(nullptr, B, H, Hkv, Tmax, D, topk);
     if ((st = check_ws(workspace, workspace_bytes, need.bytes)) != HSA_OK) return st;
-    DecLayout l = dec_layout(workspace, B, H, Tmax, D, topk);
+    DecLayout l = dec_layout(workspace, B, H, Hkv, Tmax, D, topk);
     hsa::DecodeArgs a{};
     a.qs = qs; a.q = q; a.Kc = Kc; a.Vc = Vc; a.Lc = Lc; a.cache_len = cache_len;
     a.Tmax = Tmax; a.Nmax = Tmax / 64;

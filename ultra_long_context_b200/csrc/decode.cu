@@ -79,6 +79,63 @@ __device__ inline int compact_at_least(uint64_t *keys, int n, uint64_t tau, int 
     return kept;
 }
 
+// Exact merge of the per-range candidates of one (b, h): all[r * K + j] holds range r's top K in
+// descending order (0 = empty). Writes the head's selection (sel_idx_h[0..K), descending score, -1
+// padding) and its fusion weights (Step 4, softmax of the kept scores; 0 padding). Block-wide; keys
+// holds at least nsplit * K entries, topk and sorted 64 each, hist 256, misc 8.
+__device__ void merge_ranges(const uint64_t *all, int nsplit, int K, uint64_t *keys, uint64_t *topk,
+                             uint64_t *sorted, uint32_t *hist, int *misc, int32_t *sel_idx_h, float *sel_w_h) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int ncand = nsplit * K;
+#pragma unroll 8
+    for (int i = tid; i < ncand; i += kDecodeThreads)
+        keys[i] = __ldcg(reinterpret_cast<const unsigned long long *>(all) + i);
+    __syncthreads();
+    // Each range contributed its top K in descending order. The K-th largest of the range maxima, tau,
+    // has K ranges with a key at or above it, so no candidate below tau can be in the top K.
+    int nmerge = ncand;
+    if (nsplit > K && nsplit <= 2 * kDecodeThreads) {
+        unsigned long long *tau_s = reinterpret_cast<unsigned long long *>(topk);  // scratch until selection
+        if (tid == 0) *tau_s = 0ull;  // stays 0 (keep every nonzero key) if fewer than K maxima are nonzero
+        __syncthreads();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int r = tid + h * kDecodeThreads;
+            if (r < nsplit) {
+                const uint64_t mr = keys[r * K];
+                int rank = 0;
+                for (int q = 0; q < nsplit; ++q) rank += keys[q * K] > mr ? 1 : 0;
+                if (rank == K - 1 && mr != 0ull) *tau_s = mr;  // unique nonzero keys: at most one range
+            }
+        }
+        __syncthreads();
+        const uint64_t tau = *tau_s;
+        nmerge = compact_at_least(keys, ncand, tau == 0ull ? 1ull : tau, misc);
+    }
+    int m;
+    if (nmerge <= kRankSelectMax) {
+        m = block_topk_rank(keys, nmerge, K, sorted);
+    } else {
+        m = block_topk_u64(keys, nmerge, K, topk, hist, misc);
+        block_sort_desc_small(topk, m, sorted);  // empty (0) keys sort last
+    }
+    if (warp == 0) {
+        // fusion weights (Step 4): softmax over the kept scores, fp32, max-subtracted
+        const uint64_t k0 = lane < m ? sorted[lane] : 0ull;
+        const uint64_t k1 = lane + 32 < m ? sorted[lane + 32] : 0ull;
+        const float top = m > 0 && sorted[0] ? key_score(sorted[0]) : 0.0f;
+        const float e0 = k0 ? expf(key_score(k0) - top) : 0.0f;
+        const float e1 = k1 ? expf(key_score(k1) - top) : 0.0f;
+        const float z = warp_sum(e0 + e1);
+        for (int j = lane; j < K; j += 32) {
+            const uint64_t kk = j < 32 ? k0 : k1;
+            const float e = j < 32 ? e0 : e1;
+            sel_idx_h[j] = kk ? key_index(kk) : -1;
+            sel_w_h[j] = kk ? e / z : 0.0f;
+        }
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ Lc, const int64_t *__restrict__ cache_len, int H,
@@ -173,55 +230,199 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
     __syncthreads();
     if (!misc[4]) return;
     __threadfence();
-    const int ncand = nsplit * K;
-    const uint64_t *all = cand + (size_t)bh * nsplit * K;
-    for (int i = tid; i < ncand; i += kDecodeThreads)
-        keys[i] = __ldcg(reinterpret_cast<const unsigned long long *>(all) + i);
-    __syncthreads();
-    // Each range contributed its top K in descending order. The K-th largest of the range maxima, tau,
-    // has K ranges with a key at or above it, so no candidate below tau can be in the top K.
-    int nmerge = ncand;
-    if (nsplit > K && nsplit <= 2 * kDecodeThreads) {
-        unsigned long long *tau_s = reinterpret_cast<unsigned long long *>(topk);  // scratch until selection
-        if (tid == 0) *tau_s = 0ull;  // stays 0 (keep every nonzero key) if fewer than K maxima are nonzero
-        __syncthreads();
+    merge_ranges(cand + (size_t)bh * nsplit * K, nsplit, K, keys, topk, sorted, hist, misc,
+                 sel_idx + (size_t)bh * K, sel_w + (size_t)bh * K);
+    if (tid == 0) counters[bh] = 0u;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Grouped heads (G query heads per landmark head): one CTA scores a landmark range for all G heads of
+// the group, so the range leaves HBM (and L2) once instead of G times.
+// ------------------------------------------------------------------------------------------------
+
+// Sorts the warp's 32 keys (one per lane) into descending order across the lanes (bitonic network:
+// 15 compare-exchange stages between lanes l and l ^ j).
+__device__ inline uint64_t warp_sort_desc(uint64_t x) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int r = tid + h * kDecodeThreads;
-            if (r < nsplit) {
-                const uint64_t mr = keys[r * K];
-                int rank = 0;
-                for (int q = 0; q < nsplit; ++q) rank += keys[q * K] > mr ? 1 : 0;
-                if (rank == K - 1 && mr != 0ull) *tau_s = mr;  // unique nonzero keys: at most one range
+    for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const uint64_t y = __shfl_xor_sync(0xffffffffu, x, j);
+            const bool desc = (lane & k) == 0;  // k = 32: every lane, the whole warp descending
+            const bool lower = (lane & j) == 0;
+            x = (lower == desc) ? (x > y ? x : y) : (x < y ? x : y);
+        }
+    return x;
+}
+
+// The 32 largest of two descending 32-key lists (one key per lane), descending. The elementwise maximum
+// of one list and the other reversed holds exactly those 32 keys as a bitonic sequence, which five
+// half-cleaner stages sort.
+__device__ inline uint64_t warp_merge_desc(uint64_t a, uint64_t b) {
+    const int lane = threadIdx.x & 31;
+    const uint64_t r = __shfl_sync(0xffffffffu, b, 31 - lane);
+    uint64_t m = a > r ? a : r;
+#pragma unroll
+    for (int j = 16; j > 0; j >>= 1) {
+        const uint64_t y = __shfl_xor_sync(0xffffffffu, m, j);
+        m = (lane & j) == 0 ? (m > y ? m : y) : (m < y ? m : y);
+    }
+    return m;
+}
+
+// The exact top K (K <= 32) of one head's n scores sc[0..n) (chunks c0 + i), by one warp; lane l < K
+// returns the l-th largest key (0 = empty). Filter: the elements are cut into 64 disjoint groups (lane
+// l, even or odd rounds); if K group maxima are at or above a value, so are K different scores, so the
+// K-th largest group maximum tau is a lower bound of the K-th largest score and nothing below it can be
+// selected. The survivors (and, once K keys are kept, only keys above the K-th kept) are staged in
+// groups of 32, sorted, and merged into the running top 32.
+__device__ inline uint64_t warp_topk_scores(const float *sc, int n, int64_t c0, int K, uint64_t *stage) {
+    const int lane = threadIdx.x & 31;
+    float m0 = -INFINITY, m1 = -INFINITY;
+    for (int r = 0; 32 * r < n; ++r) {
+        const int i = 32 * r + lane;
+        if (i < n) {
+            if (r & 1) m1 = fmaxf(m1, sc[i]);
+            else m0 = fmaxf(m0, sc[i]);
+        }
+    }
+    // tau = the largest group maximum v with at least K group maxima >= v (-inf if none: keep all)
+    int ge0 = 0, ge1 = 0;
+#pragma unroll 8
+    for (int j = 0; j < 32; ++j) {
+        const float x0 = __shfl_sync(0xffffffffu, m0, j), x1 = __shfl_sync(0xffffffffu, m1, j);
+        ge0 += (x0 >= m0 ? 1 : 0) + (x1 >= m0 ? 1 : 0);
+        ge1 += (x0 >= m1 ? 1 : 0) + (x1 >= m1 ? 1 : 0);
+    }
+    float tau = fmaxf(ge0 >= K ? m0 : -INFINITY, ge1 >= K ? m1 : -INFINITY);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tau = fmaxf(tau, __shfl_xor_sync(0xffffffffu, tau, o));
+    // thr: tau, raised to the K-th kept score once K keys are kept; a score equal to it can still win on
+    // the lower chunk index, so the float test keeps ties and the merge decides on the full key
+    uint64_t best = 0ull;
+    float thr = tau;
+    int ns = 0;  // staged keys (warp-uniform)
+    for (int r = 0; r < n; r += 32) {
+        const int i = r + lane;
+        const bool cand = i < n && sc[i] >= thr;
+        const unsigned bal = __ballot_sync(0xffffffffu, cand);
+        if (bal == 0u) continue;
+        if (cand) stage[ns + __popc(bal & ((1u << lane) - 1u))] = make_key(sc[i], (uint32_t)(c0 + i));
+        ns += __popc(bal);
+        __syncwarp();
+        if (ns >= 32) {
+            best = warp_merge_desc(best, warp_sort_desc(stage[lane]));
+            const uint64_t rest = lane + 32 < ns ? stage[lane + 32] : 0ull;
+            __syncwarp();
+            if (lane + 32 < ns) stage[lane] = rest;
+            __syncwarp();
+            ns -= 32;
+            const uint64_t kth = __shfl_sync(0xffffffffu, best, K - 1);  // 0 until K keys are kept
+            if (kth != 0ull) thr = fmaxf(thr, key_score(kth));
+        }
+    }
+    if (ns > 0) best = warp_merge_desc(best, warp_sort_desc(lane < ns ? stage[lane] : 0ull));
+    return lane < K ? best : 0ull;
+}
+
+// grid (nsplit, B*Hkv): the landmark range sp of key head kvh, for its Gh <= 16 query heads. The
+// scores of a tile of 8 landmarks for all heads are one m16n8k16 tensor-core product per 16 columns of
+// D (rows: the heads; M = 16 is below the tcgen05 tile, so the warp-level MMA). The reduction index is
+// permuted the same way in both operands, so that each lane loads whole 16-byte chunks: lane (g, t4)
+// holds columns 32 s + 8 t4 .. + 7 of head rows g, g + 8 and of landmark g of the tile, and k-steps
+// 2 s, 2 s + 1 take the first and the second half of that chunk.
+constexpr int kDecodeGroupThreads = 512;  // one CTA per SM: 16 warps stream, then one head per warp selects
+
+template <int D>
+__global__ void __launch_bounds__(kDecodeGroupThreads, 1) decode_scan_group_kernel(
+    const uint16_t *__restrict__ q, const uint16_t *__restrict__ Lc, const int64_t *__restrict__ cache_len, int Hkv,
+    int Gh, int64_t Nmax, int split, int nsplit, int K, float scale, uint64_t *__restrict__ cand) {
+    constexpr int S = D / 32;      // 16-byte chunks per lane per row
+    constexpr int NWARP = kDecodeGroupThreads / 32;
+    constexpr int U = 4;           // landmark tiles in flight per warp
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int ld = split + 8;      // score row stride (fewer bank conflicts on the fragment stores)
+    float *sc = reinterpret_cast<float *>(smem_raw);                             // [16][ld]
+    uint64_t *stage = reinterpret_cast<uint64_t *>(smem_raw + (size_t)16 * ld * sizeof(float));  // [NWARP][64]
+
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t4 = lane & 3;
+    const int sp = blockIdx.x, kvh = blockIdx.y, b = kvh / Hkv;
+    int64_t nb = cache_len[b] / kChunk;
+    nb = nb < 0 ? 0 : (nb > Nmax ? Nmax : nb);
+    const int64_t c0 = (int64_t)sp * split;
+    const int64_t c1 = min(c0 + (int64_t)split, nb);
+    const int nloc = c1 > c0 ? (int)(c1 - c0) : 0;
+    const size_t bh0 = (size_t)kvh * Gh;  // first query head of the group
+
+    uint32_t a[S][2][4];
+#pragma unroll
+    for (int s = 0; s < S; ++s) {
+        const uint4 qa = g < Gh ? *reinterpret_cast<const uint4 *>(q + (bh0 + g) * D + 32 * s + 8 * t4)
+                                : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 qb = g + 8 < Gh ? *reinterpret_cast<const uint4 *>(q + (bh0 + g + 8) * D + 32 * s + 8 * t4)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+        a[s][0][0] = qa.x; a[s][0][1] = qb.x; a[s][0][2] = qa.y; a[s][0][3] = qb.y;
+        a[s][1][0] = qa.z; a[s][1][1] = qb.z; a[s][1][2] = qa.w; a[s][1][3] = qb.w;
+    }
+    const uint16_t *Lh = Lc + (size_t)kvh * Nmax * D;
+    const int ntile = (nloc + 7) / 8;
+    for (int t0 = warp; t0 < ntile; t0 += NWARP * U) {
+        uint4 v[U][S];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int tile = t0 + u * NWARP;
+            const int i = tile * 8 + g;
+#pragma unroll
+            for (int s = 0; s < S; ++s)
+                v[u][s] = (tile < ntile && i < nloc) ? ld_stream16(Lh + (c0 + i) * D + 32 * s + 8 * t4)
+                                                     : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int tile = t0 + u * NWARP;  // warp-uniform
+            if (tile >= ntile) break;
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+                mma_bf16_16816(acc, a[s][0], v[u][s].x, v[u][s].y);
+                mma_bf16_16816(acc, a[s][1], v[u][s].z, v[u][s].w);
+            }
+            const int i0 = tile * 8 + 2 * t4;  // acc: heads g (0, 1) and g + 8 (2, 3), landmarks i0, i0 + 1
+            if (g < Gh) {
+                if (i0 < nloc) sc[g * ld + i0] = acc[0] * scale;
+                if (i0 + 1 < nloc) sc[g * ld + i0 + 1] = acc[1] * scale;
+            }
+            if (g + 8 < Gh) {
+                if (i0 < nloc) sc[(g + 8) * ld + i0] = acc[2] * scale;
+                if (i0 + 1 < nloc) sc[(g + 8) * ld + i0 + 1] = acc[3] * scale;
             }
         }
-        __syncthreads();
-        const uint64_t tau = *tau_s;
-        nmerge = compact_at_least(keys, ncand, tau == 0ull ? 1ull : tau, misc);
     }
-    int m;
-    if (nmerge <= kRankSelectMax) {
-        m = block_topk_rank(keys, nmerge, K, sorted);
-    } else {
-        m = block_topk_u64(keys, nmerge, K, topk, hist, misc);
-        block_sort_desc_small(topk, m, sorted);  // empty (0) keys sort last
+    __syncthreads();
+    for (int h = warp; h < Gh; h += NWARP) {
+        const uint64_t best = warp_topk_scores(sc + h * ld, nloc, c0, K, stage + warp * 64);
+        if (lane < K) cand[((bh0 + h) * nsplit + sp) * K + lane] = best;
     }
-    if (warp == 0) {
-        // fusion weights (Step 4): softmax over the kept scores, fp32, max-subtracted
-        const uint64_t k0 = lane < m ? sorted[lane] : 0ull;
-        const uint64_t k1 = lane + 32 < m ? sorted[lane + 32] : 0ull;
-        const float top = m > 0 && sorted[0] ? key_score(sorted[0]) : 0.0f;
-        const float e0 = k0 ? expf(key_score(k0) - top) : 0.0f;
-        const float e1 = k1 ? expf(key_score(k1) - top) : 0.0f;
-        const float z = warp_sum(e0 + e1);
-        for (int j = lane; j < K; j += 32) {
-            const uint64_t kk = j < 32 ? k0 : k1;
-            const float e = j < 32 ? e0 : e1;
-            sel_idx[(size_t)bh * K + j] = kk ? key_index(kk) : -1;
-            sel_w[(size_t)bh * K + j] = kk ? e / z : 0.0f;
-        }
-    }
-    if (tid == 0) counters[bh] = 0u;
+}
+
+// grid (B*H): the exact merge of one query head's range candidates. Launched as a programmatic
+// dependent of the grouped scan; waits for that grid before reading its candidates.
+__global__ void __launch_bounds__(kDecodeThreads) decode_merge_kernel(const uint64_t *__restrict__ cand, int nsplit,
+                                                                      int K, int32_t *__restrict__ sel_idx,
+                                                                      float *__restrict__ sel_w) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int cap = nsplit * K;
+    uint64_t *keys = reinterpret_cast<uint64_t *>(smem_raw);
+    uint64_t *topk = keys + cap;
+    uint64_t *sorted = topk + 64;
+    uint32_t *hist = reinterpret_cast<uint32_t *>(sorted + 64);
+    int *misc = reinterpret_cast<int *>(hist + 256);
+    const size_t bh = blockIdx.x;
+    merge_ranges(cand + bh * nsplit * K, nsplit, K, keys, topk, sorted, hist, misc, sel_idx + bh * K, sel_w + bh * K);
 }
 
 // QKN: query-key normalisation, the logits use q / max(|q|, eps) and k / max(|k|, eps) (fp32, on the fly).
@@ -346,7 +547,8 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
 // sized for a single wave of CTAs: B*H*ranges <= kDecodeWaveCtas (148 SMs x 4 resident CTAs of
 // 256 threads at the kernel's register count). A range keeps at least 256 landmarks and at most
 // 6144 (its keys live in shared memory), and ranges*K <= 8192 (the merge holds all candidates).
-constexpr int64_t kDecodeWaveCtas = 148 * 4;
+constexpr int64_t kDecodeSms = 148;
+constexpr int64_t kDecodeWaveCtas = kDecodeSms * 4;
 
 int decode_split_size(int64_t Nmax, int K, int BH) {
     if (Nmax <= 0) return 1;
@@ -364,6 +566,47 @@ int decode_split_size(int64_t Nmax, int K, int BH) {
 size_t decode_scan_smem(int split, int nsplit, int K) {
     const size_t cap = (size_t)(split > nsplit * K ? split : nsplit * K);
     return (cap + 128) * sizeof(uint64_t) + 256 * sizeof(uint32_t) + 8 * sizeof(int);
+}
+
+// Grouped scan: scores of 16 head rows per landmark (fp32, row stride split + 8) plus the warps'
+// staging and merge buffers.
+static size_t decode_group_smem(int split) {
+    return (size_t)16 * (split + 8) * sizeof(float) + (size_t)(kDecodeGroupThreads / 32) * 64 * sizeof(uint64_t);
+}
+constexpr int kDecodeGroupMaxSplit = 3072;
+
+DecodePlan decode_plan(int64_t Nmax, int K, int B, int H, int Hkv) {
+    DecodePlan p{};
+    const int Gh = Hkv > 0 ? H / Hkv : 1;
+    if (Gh >= 2 && Gh <= 16 && K <= 32 && Nmax > 0) {
+        // one CTA per SM in a single wave, >= 256 landmarks per range; the merge keeps every candidate in
+        // shared memory (ranges * K <= 8192, ranges <= 512)
+        int64_t ns = (int64_t)kDecodeSms / ((int64_t)B * Hkv);
+        ns = ns < 1 ? 1 : ns;
+        const int64_t by_min = (Nmax + 255) / 256;
+        ns = ns < by_min ? ns : by_min;
+        const int64_t cap = (8192 / K < 512) ? 8192 / K : 512;
+        ns = ns < cap ? ns : cap;
+        int64_t split = (Nmax + ns - 1) / ns;
+        split = (split + 63) / 64 * 64;
+        if (split <= kDecodeGroupMaxSplit) {
+            p.grouped = true;
+            p.split = (int)split;
+            p.nsplit = (int)((Nmax + split - 1) / split);
+            return p;
+        }
+    }
+    p.split = decode_split_size(Nmax, K, B * H);
+    const int64_t ns = (Nmax + p.split - 1) / p.split;
+    p.nsplit = ns > 0 ? (int)ns : 1;
+    return p;
+}
+
+size_t decode_plan_smem(const DecodePlan &p, int K) {
+    if (!p.grouped) return decode_scan_smem(p.split, p.nsplit, K);
+    const size_t merge = ((size_t)p.nsplit * K + 128) * sizeof(uint64_t) + 256 * sizeof(uint32_t) + 8 * sizeof(int);
+    const size_t scan = decode_group_smem(p.split);
+    return merge > scan ? merge : scan;
 }
 
 // The attend kernel is launched as a programmatic dependent of the scan, so that its launch overlaps
@@ -385,10 +628,57 @@ static cudaError_t launch_attend(const DecodeArgs &a, dim3 grid, cudaStream_t s)
                               (const float *)a.sel_w, a.partial, a.counters + a.B * a.H, a.out);
 }
 
+template <int D>
+static cudaError_t launch_decode_grouped(const DecodeArgs &a, const DecodePlan &pl, cudaStream_t s) {
+    const int Gh = a.H / a.Hkv;
+    const size_t gsmem = decode_group_smem(pl.split);
+    cudaError_t e = cudaFuncSetAttribute(decode_scan_group_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)gsmem);
+    if (e != cudaSuccess) return e;
+    {
+        HSA_PROF("decode_scan", s);
+        decode_scan_group_kernel<D><<<dim3(pl.nsplit, a.B * a.Hkv), kDecodeGroupThreads, gsmem, s>>>(
+            a.qs, a.Lc, a.cache_len, a.Hkv, Gh, a.Nmax, pl.split, pl.nsplit, a.K, a.scale, a.cand);
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) return e;
+    const size_t msmem = ((size_t)pl.nsplit * a.K + 128) * sizeof(uint64_t) + 256 * sizeof(uint32_t) + 8 * sizeof(int);
+    e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(a.B * a.H);
+    cfg.blockDim = dim3(kDecodeThreads);
+    cfg.dynamicSmemBytes = msmem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    {
+        HSA_PROF("decode_merge", s);
+        e = cudaLaunchKernelEx(&cfg, decode_merge_kernel, (const uint64_t *)a.cand, pl.nsplit, a.K, a.sel_idx, a.sel_w);
+    }
+    if (e != cudaSuccess) return e;
+    HSA_PROF("decode_attend", s);
+    return launch_attend<D>(a, dim3(a.K, a.B * a.H), s);
+}
+
 cudaError_t launch_decode(const DecodeArgs &a0, cudaStream_t s) {
     DecodeArgs a = a0;
     if (a.Hkv <= 0) a.Hkv = a.H;
     if (a.H % a.Hkv != 0) return cudaErrorInvalidValue;
+    const DecodePlan pl = decode_plan(a.Nmax, a.K, a.B, a.H, a.Hkv);
+    if (pl.grouped) {
+        cudaError_t e;
+        {
+            HSA_PROF("memset", s);
+            e = cudaMemsetAsync(a.counters, 0, 2 * (size_t)a.B * a.H * sizeof(unsigned), s);
+        }
+        if (e != cudaSuccess) return e;
+        e = a.D == 128 ? launch_decode_grouped<128>(a, pl, s) : launch_decode_grouped<64>(a, pl, s);
+        return e != cudaSuccess ? e : cudaGetLastError();
+    }
     const int split = decode_split_size(a.Nmax, a.K, a.B * a.H);
     const int nsplit = (int)((a.Nmax + split - 1) / split) > 0 ? (int)((a.Nmax + split - 1) / split) : 1;
     const size_t smem = decode_scan_smem(split, nsplit, a.K);

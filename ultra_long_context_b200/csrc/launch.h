@@ -27,6 +27,14 @@ struct DecodeArgs {
 };
 int decode_split_size(int64_t Nmax, int K, int BH);
 size_t decode_scan_smem(int split, int nsplit, int K);
+// How a decode call splits the landmark scan: ranges of `split` landmarks, `nsplit` of them; grouped:
+// one CTA per (range, key head) scores all query heads of the group and a merge kernel follows.
+struct DecodePlan {
+    int split, nsplit;
+    bool grouped;
+};
+DecodePlan decode_plan(int64_t Nmax, int K, int B, int H, int Hkv);
+size_t decode_plan_smem(const DecodePlan &p, int K);  // the largest dynamic shared memory of its kernels
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 
 // Chunk-major work list entry: one tile of up to kPairTile (token, slot) pairs of one chunk.

@@ -14,17 +14,21 @@
 //   * Warp 4 (one lane) is the producer: 32-landmark blocks arrive by TMA in the 128-byte-swizzled
 //     layout (three stages), and it issues S_blk = Q L_blk^T (M = 128, N = 32, fp32) into one of the
 //     TMEM score buffers. Full/empty mbarriers link it to warps 0-3, which run decoupled.
-//   * Pass 1 keeps, per row, the K largest score VALUES in a sorted register list. The scores of a
-//     block that beat the current K-th value are first compacted into a per-thread column of shared
-//     memory (branch-free: every score is stored, the write index advances only on a candidate),
-//     then inserted one by one with new[i] = max(old[i], min(old[i-1], x)), which touches every slot
-//     independently (no dependent chain); a warp thus pays only for real candidates. The K-th value
-//     tau results.
-//   * Pass 2 recomputes the same blocks (bit-identical: same operands, same instruction sequence) and
-//     keeps every chunk with s > tau plus the lowest-index chunks with s == tau until K are kept --
-//     exactly the stable-sort rule -- stashing (score, chunk) in chunk order, branch-free as well.
-//   * At the end each row ranks its kept chunks (output slot = number of kept values above it, ties
-//     in chunk order), computes the fusion weights w = softmax over the kept values (fp32,
+//   * Scores are compared unscaled (the scale is positive, so the order is the same); it enters the
+//     fusion weights only. For each 32-landmark block a thread stores its row's 32 scores to a
+//     per-thread column of shared memory at fixed offsets and sets one bit per candidate, so the
+//     per-score cost is a store, a compare and an OR; only the set bits are visited afterwards.
+//   * Pass 1 keeps, per row, the K largest score VALUES in a sorted register list: the candidates
+//     are the scores above the current K-th value, each inserted with
+//     new[i] = max(old[i], min(old[i-1], x)), which touches every slot independently (no dependent
+//     chain). The K-th value tau results.
+//   * Pass 2 recomputes the same blocks (bit-identical: same operands, same instruction sequence);
+//     the candidates are the scores >= tau, visited in chunk order, and it keeps every one above tau
+//     plus the lowest-index ones equal to tau until K are kept -- exactly the stable-sort rule. A
+//     kept chunk's output slot is known when it is taken (the number of kept values above it, ties
+//     in chunk order), so only its chunk id is stored; its value is the slot's entry of the sorted
+//     list.
+//   * At the end each row computes the fusion weights w = softmax over the kept values (fp32,
 //     max-subtracted), and the tile's rows, contiguous in [B, H, T, K], are written by coalesced
 //     stores through shared memory.
 //   * Two pieces of the dispatch ride along, on memory bandwidth this ALU-bound kernel leaves idle:
@@ -58,8 +62,8 @@ struct StSmem {
     static constexpr uint32_t STAGE = 128 * K * 8;                    // output staging: idx + w per row
     // region U holds the landmark stages during the loop and the output staging at the end
     static constexpr uint32_t U = kStLStages * LB > STAGE ? kStLStages * LB : STAGE;
-    // [33][128] fp32 candidates / kept scores; [K+1][128] int32 kept chunk ids. The spare row takes
-    // the unconditional store that follows the last real entry.
+    // [33][128] fp32: a block's scores, one column per thread; [K+1][128] int32: the chunk of each
+    // output slot.
     static constexpr uint32_t CV = U;
     static constexpr uint32_t CC = CV + 33 * 128 * 4;
     static constexpr uint32_t HIST = CC + (K + 1) * 128 * 4;  // int[kStHistMax]: selected pairs per chunk
@@ -214,13 +218,15 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
             if (lane == 0) tc::mbar_arrive(q_ready);
         }
 
-        float *cv = reinterpret_cast<float *>(s + SM::CV) + tid;  // this thread's column of slots
-        int *cc = reinterpret_cast<int *>(s + SM::CC) + tid;
+        // Scores are compared unscaled (scale > 0 keeps their order); the scale enters the weights only.
+        float *cv = reinterpret_cast<float *>(s + SM::CV) + tid;  // this thread's column: a block's scores
+        int *cc = reinterpret_cast<int *>(s + SM::CC) + tid;      // chunk of each output slot
         float ls[K];  // pass 1: the K largest score values of this row, descending
 #pragma unroll
         for (int i = 0; i < K; ++i) ls[i] = -INFINITY;
         float tau = -INFINITY;
-        int need_eq = 0, kept = 0;
+        int need_eq = 0;
+        uint64_t used = 0;  // pass 2: output slots filled
 
         for (int g = 0; g < G; ++g) {
             const int buf = g % NB;
@@ -248,38 +254,57 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
             }
             const int b = g % nblk;
             const int ncol = min(kStCols, my_n - b * kStCols);
-            if (g < nblk) {
-                int n = 0;
+            const uint32_t valid = ncol >= 32 ? 0xffffffffu : (ncol > 0 ? (1u << ncol) - 1u : 0u);
+            // every score of the block to this thread's column; one bit per candidate
+            uint32_t m = 0;
+            if (g < nblk) {  // warp-uniform
                 const float thr = ls[K - 1];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {  // branch-free: store always, advance on a candidate
-                    const float x = v[i] * scale;
-                    cv[128 * n] = x;
-                    n += (i < ncol && x > thr) ? 1 : 0;
+                for (int i = 0; i < 32; ++i) {
+                    cv[128 * i] = v[i];
+                    m |= v[i] > thr ? 1u << i : 0u;
                 }
-                for (int k = 0; k < n; ++k) {
-                    const float x = cv[128 * k];
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    cv[128 * i] = v[i];
+                    m |= v[i] >= tau ? 1u << i : 0u;
+                }
+            }
+            m &= valid;
+            if (g < nblk) {  // pass 1: insert the candidates that still beat the K-th value
+                while (m) {
+                    const int i = __ffs(m) - 1;
+                    m &= m - 1;
+                    const float x = cv[128 * i];
                     if (x > ls[K - 1]) {
 #pragma unroll
                         for (int j = K - 1; j > 0; --j) ls[j] = fmaxf(ls[j], fminf(ls[j - 1], x));
                         ls[0] = fmaxf(ls[0], x);
                     }
                 }
-            } else {
+            } else {  // pass 2: take every score > tau and the lowest chunks at tau, in chunk order
+                while (m) {
+                    const int i = __ffs(m) - 1;
+                    m &= m - 1;
+                    const float x = cv[128 * i];
+                    const bool eq = !(x > tau);
+                    if (eq && need_eq <= 0) continue;
+                    need_eq -= eq ? 1 : 0;
+                    // output slot: after the kept values above x, ties in chunk order
+                    int lo = 0;
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {  // branch-free, as in pass 1
-                    const float x = v[i] * scale;
-                    const bool eq = x == tau && need_eq > 0;
-                    const bool take = i < ncol && (x > tau || eq) && kept < k_keep;
-                    cv[128 * kept] = x;
-                    cc[128 * kept] = b * kStCols + i;
-                    kept += take ? 1 : 0;
-                    need_eq -= (take && eq) ? 1 : 0;
+                    for (int jj = 0; jj < K; ++jj) lo += (jj < k_keep && ls[jj] > x) ? 1 : 0;
+                    const uint64_t freeb = ~used & (~0ull << lo);
+                    const int slot = __ffsll((long long)freeb) - 1;
+                    if (slot < 0 || slot >= k_keep) continue;  // only if pass 2 disagreed with pass 1
+                    used |= 1ull << slot;
+                    cc[128 * slot] = b * kStCols + i;
                 }
             }
         }
 
-        // rank the kept chunks, weights, and stage the tile's rows in shared memory (the landmark
+        // weights from the sorted values, and the tile's rows staged in shared memory (the landmark
         // stages are free: every MMA has completed)
         asm volatile("bar.sync 1, %0;" ::"n"(kStConsumers) : "memory");
         int32_t *st_idx = reinterpret_cast<int32_t *>(s);
@@ -288,28 +313,20 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
             const float top = ls[0];
             float z = 0.0f;
 #pragma unroll
-            for (int i = 0; i < K; ++i) z += i < k_keep ? expf(ls[i] - top) : 0.0f;
+            for (int i = 0; i < K; ++i) z += i < k_keep ? expf((ls[i] - top) * scale) : 0.0f;
             const float rz = 1.0f / z;
-            uint64_t used = 0;
-            for (int k = 0; k < kept; ++k) {
-                const float x = cv[128 * k];
-                int lo = 0;
 #pragma unroll
-                for (int j = 0; j < K; ++j) lo += (j < k_keep && ls[j] > x) ? 1 : 0;
-                const uint64_t freeb = ~used & (~0ull << lo);
-                const int slot = __ffsll((long long)freeb) - 1;
-                if (slot < 0 || slot >= kout) continue;  // only if pass 2 disagreed with pass 1
-                used |= 1ull << slot;
-                st_idx[tid * kout + slot] = cc[128 * k];
-                st_w[tid * kout + slot] = expf(x - top) * rz;
-                if (hist_smem) atomicAdd(&s_hist[cc[128 * k]], 1);
-                else atomicAdd(&chunk_count[(size_t)bh * N + cc[128 * k]], 1);
-            }
-            for (int i = 0; i < kout; ++i)
-                if (!((used >> i) & 1ull)) {
-                    st_idx[tid * kout + i] = -1;
-                    st_w[tid * kout + i] = 0.0f;
+            for (int i = 0; i < K; ++i) {
+                if (i >= kout) break;
+                const bool u = (used >> i) & 1ull;
+                const int c = u ? cc[128 * i] : -1;
+                st_idx[tid * kout + i] = c;
+                st_w[tid * kout + i] = u ? expf((ls[i] - top) * scale) * rz : 0.0f;
+                if (u) {
+                    if (hist_smem) atomicAdd(&s_hist[c], 1);
+                    else atomicAdd(&chunk_count[(size_t)bh * N + c], 1);
                 }
+            }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kStConsumers) : "memory");
         for (int i = tid; i < nrows * kout; i += kStConsumers) {

@@ -469,6 +469,25 @@ def main():
                             "frac": round((scan_bytes + gather_bytes) / (dms / 1e3) / 1e9 / hbm_peak, 4)},
             "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_dec.items()},
         }
+        if not args.skip_options:  # 4 query tokens per sequence in one step (e.g. verifying 4 drafted tokens)
+            Tq = 4
+            mq = inputs.forward_inputs(wd.B, wd.H, Tq, wd.D, wd.seed + 5, device=dev)[0]
+            mout = torch.empty_like(mq)
+            midx = torch.empty((wd.B, wd.H, Tq, wd.topk), dtype=torch.int32, device=dev)
+            mw = torch.empty((wd.B, wd.H, Tq, wd.topk), dtype=torch.float32, device=dev)
+            mws = torch.empty(hsa.hsa_decode_ex_workspace_size(wd.B, wd.H, wd.H, wd.cache_len, wd.D, 64, wd.topk, 0, Tq)
+                              + 256, dtype=torch.uint8, device=dev)
+
+            def dec_multi():
+                hsa.hsa_decode(mq, Kc, Vc, Lc, lens, wd.topk, out=mout, sel_idx=midx, sel_w=mw, workspace=mws)
+
+            mms = timed(dec_multi, dsteps, args.warmup, world) / dsteps
+            prof_m = kernel_profile(dec_multi, dsteps)
+            extra["decode_16m"]["multi_token_4"] = {
+                "shape": f"B{wd.B} H{wd.H} Tq{Tq} cache {wd.cache_len} D{wd.D} topk{wd.topk}",
+                "us_per_step": round(mms * 1e3, 3), "us_per_token": round(mms * 1e3 / (wd.B * Tq), 3),
+                "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_m.items()}}
+            del mq, mout, mws
         del q, Kc, Vc, Lc, dws
         torch.cuda.empty_cache()
         if not args.skip_options:  # 16 query heads on one key/value head, same cache length

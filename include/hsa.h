@@ -180,6 +180,14 @@ hsa_status hsa_backward(const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
  *                    K, V, L (Kc, Vc, Lc) have Hkv heads, H a multiple of Hkv, and query head h uses
  *                    head h / (H / Hkv). Each query head still selects its own chunks.
  *                    Shapes: K, V [B, Hkv, T, D], L [B, Hkv, T/64, D]; dK, dV, dL likewise.
+ *   Tq [1] (decode)  several query tokens per sequence and head in one decode step (verifying drafted
+ *                    tokens, or decoding a few tokens at once): q, qs, out [B, H, Tq, D], sel_idx and
+ *                    sel_w [B, H, Tq, topk], 1 <= Tq <= 64. The Tq tokens are the LAST Tq tokens of the
+ *                    cache (their K, V and any completed landmark already in it): token i sits at
+ *                    position cache_len[b] - Tq + i and sees the chunks that have ended at or before it,
+ *                    the prefill's causal rule (so the result equals the forward's last Tq rows).
+ *                    Tq > 1 requires topk <= 32. Every query row is scored on the tensor cores together
+ *                    with the other rows that share its key head (up to 16 per pass over the landmarks).
  *
  * Unknown flag bits give HSA_ERR_INVALID_ARG. hsa_backward_ex writes dQ (the attention query's
  * gradient, taken back through the normalisation when it is on) and, when Qs is given, dQs (the
@@ -195,11 +203,12 @@ hsa_status hsa_forward_ex(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 
                           unsigned flags, hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace,
                           size_t workspace_bytes, void *stream);
 
-size_t hsa_decode_ex_workspace_size(int B, int H, int Hkv, int64_t Tmax, int D, int chunk, int topk, unsigned flags);
+size_t hsa_decode_ex_workspace_size(int B, int H, int Hkv, int Tq, int64_t Tmax, int D, int chunk, int topk,
+                                    unsigned flags);
 
 hsa_status hsa_decode_ex(const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
-                         const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B, int H, int Hkv, int D,
-                         int chunk, int topk, float scale, unsigned flags, hsa_bf16 *out, int32_t *sel_idx,
+                         const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B, int H, int Hkv, int Tq,
+                         int D, int chunk, int topk, float scale, unsigned flags, hsa_bf16 *out, int32_t *sel_idx,
                          float *sel_w, void *workspace, size_t workspace_bytes, void *stream);
 
 size_t hsa_backward_ex_workspace_size(int B, int H, int Hkv, int T, int D, int chunk, int topk, unsigned flags);

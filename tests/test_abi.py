@@ -134,12 +134,14 @@ def test_backward_ex_rejects_invalid_calls_on_host(kw, status):
 
 
 def test_decode_ex_rejects_invalid_calls_on_host():
-    args = dict(qs=None, q=FAKE, Kc=FAKE, Vc=FAKE, Lc=FAKE, cache_len=FAKE, Tmax=1 << 20, B=2, H=2, Hkv=2, D=128,
-                chunk=64, topk=16, scale=0.0, flags=8, out=FAKE, sel_idx=None, sel_w=None, ws=FAKE, ws_bytes=1 << 40,
-                stream=None)
+    args = dict(qs=None, q=FAKE, Kc=FAKE, Vc=FAKE, Lc=FAKE, cache_len=FAKE, Tmax=1 << 20, B=2, H=2, Hkv=2, Tq=1,
+                D=128, chunk=64, topk=16, scale=0.0, flags=8, out=FAKE, sel_idx=None, sel_w=None, ws=FAKE,
+                ws_bytes=1 << 40, stream=None)
     assert hsa.lib().hsa_decode_ex(*args.values()) == -1
-    args.update(flags=1, Hkv=3)
-    assert hsa.lib().hsa_decode_ex(*args.values()) == -1
+    for kw, status in ((dict(flags=1, Hkv=3), -1), (dict(flags=0, Tq=0), -1), (dict(flags=0, Tq=65), -1),
+                       (dict(flags=0, Tq=2, topk=40), -2), (dict(flags=0, Tq=4, ws_bytes=16), -3)):
+        a = dict(args, **kw)
+        assert hsa.lib().hsa_decode_ex(*a.values()) == status, kw
 
 
 def test_ex_workspace_sizes_cover_the_options():

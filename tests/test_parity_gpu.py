@@ -440,3 +440,74 @@ def test_backward_grouped_heads_match_oracle(oracle_mod, B, H, Hkv, T, D, topk, 
     assert grads[1].shape == (B, Hkv, T, D) and grads[3].shape == (B, Hkv, T // 64, D)
     for g, r, n in zip(grads, ref, ("dQ", "dK", "dV", "dL", "dQs")):
         grad_close(host(g), r, n)
+
+
+# ---------------------------------------------------------------------------------------------
+# several query tokens per decode step: token i of Tq sits at cache_len - Tq + i (the prefill's causal
+# rule), so each token is a one-token decode against the cache cut at its own position
+
+
+def check_decode_multi(oracle_mod, q, Kc, Vc, Lc, lens, topk, qs=None, qk_norm=False):
+    B, H, Tq, D = q.shape
+    out, idx, w = hsa.hsa_decode(q, Kc, Vc, Lc, lens, topk, qs=qs, qk_norm=qk_norm)
+    torch.cuda.synchronize()
+    assert out.shape == (B, H, Tq, D) and idx.shape == (B, H, Tq, topk)
+    for i in range(Tq):
+        lens_i = (lens - Tq + i + 1).clamp(min=0)
+        orc = oracle_decode(oracle_mod, q[:, :, i].contiguous(), Kc, Vc, Lc, lens_i, topk,
+                            qs=None if qs is None else qs[:, :, i].contiguous(), qk_norm=qk_norm)
+        g_idx = idx[:, :, i].reshape(B * H, topk).cpu().numpy()
+        g_w = w[:, :, i].reshape(B * H, topk).cpu().numpy()
+        g_out = host(out[:, :, i]).reshape(B * H, D)
+        for r in range(B * H):
+            gs = set(g_idx[r][g_idx[r] >= 0].tolist())
+            os_ = set(orc["sel_idx"][r][orc["sel_idx"][r] >= 0].tolist())
+            if gs != os_:
+                assert orc["sel_s"][r, len(os_) - 1] - orc["next_s"][r] < 1e-3, f"token {i} row {r}: selection differs"
+                continue
+            assert np.abs(g_out[r] - orc["out"][r]).max() <= 2e-2
+            og = dict(zip(orc["sel_idx"][r].tolist(), orc["sel_w"][r].tolist()))
+            for c, ww in zip(g_idx[r].tolist(), g_w[r].tolist()):
+                if c >= 0:
+                    assert abs(ww - og[c]) <= 1e-3
+    return out, idx, w
+
+
+@pytest.mark.parametrize("B,H,Hkv,D,lens,Tq,topk", [
+    (2, 4, 4, 128, [9000, 4100], 5, 16),           # one query head per key head, 5 tokens: 5 rows per pass
+    (1, 8, 2, 64, [64 * 300 + 7], 4, 32),           # 4 heads x 4 tokens = 16 rows per key head
+    (2, 2, 1, 128, [64 * 200, 64 * 200 - 3], 16, 8),  # 2 heads x 16 tokens: two row groups of 16
+    (3, 2, 2, 64, [130, 64 * 50 + 63, 64], 7, 8),    # tokens with no complete chunk, crossing chunk ends
+])
+def test_decode_multi_token_matches_oracle(oracle_mod, B, H, Hkv, D, lens, Tq, topk):
+    Tmax = max(lens) + 64
+    q = inputs.forward_inputs(B, H, Tq, D, 2000 + Tq + D, device=DEV)[0]
+    _, Kc, Vc, Lc, lens_t, _ = inputs.decode_inputs(B, Hkv, lens, D, seed=71 + Tq, Tmax=Tmax, device=DEV)
+    out, idx, w = check_decode_multi(oracle_mod, q, Kc, Vc, Lc, lens_t, topk)
+    for b in range(B):
+        for i in range(Tq):
+            if (lens[b] - Tq + i + 1) // 64 == 0:
+                assert torch.all(out[b, :, i] == 0) and torch.all(idx[b, :, i] == -1)
+
+
+def test_decode_multi_token_equals_forward_last_rows(oracle_mod):
+    """The last Tq rows of a prefill, decoded in one step against the same tensors as the cache."""
+    B, H, Hkv, T, D, topk, Tq = 1, 4, 2, 64 * 40 + 9, 128, 16, 12
+    Q, K, V, L = gqa_inputs(B, H, Hkv, T, D, 2100)
+    q = Q[:, :, T - Tq:].contiguous()
+    lens = torch.tensor([T], dtype=torch.int64, device=DEV)
+    out_d, idx_d, w_d = hsa.hsa_decode(q, K, V, L, lens, topk)
+    Qh, Kh, Vh, Lh = (host(x) for x in (Q, K, V, L))
+    rows = np.asarray([(bh * T + t) for bh in range(B * H) for t in range(T - Tq, T)])
+    orc = oracle_mod.forward(Qh, Kh, Vh, Lh, chunk=64, topk=topk, scale=1 / math.sqrt(D), rows=rows)
+    compare_forward_rows(oracle_mod, host(out_d).reshape(-1, D), host(idx_d).reshape(-1, topk),
+                         host(w_d).reshape(-1, topk), orc, Qh, Kh, Vh, Lh, rows, 64, 1 / math.sqrt(D))
+
+
+def test_decode_multi_token_with_options(oracle_mod):
+    B, H, Hkv, D, lens, Tq, topk = 2, 4, 2, 128, [64 * 90 + 1, 64 * 33], 3, 8
+    Tmax = max(lens) + 64
+    q = inputs.forward_inputs(B, H, Tq, D, 2200, device=DEV)[0]
+    qs = inputs.forward_inputs(B, H, Tq, D, 2201, device=DEV)[0]
+    _, Kc, Vc, Lc, lens_t, _ = inputs.decode_inputs(B, Hkv, lens, D, seed=81, Tmax=Tmax, device=DEV)
+    check_decode_multi(oracle_mod, q, Kc, Vc, Lc, lens_t, topk, qs=qs, qk_norm=True)

@@ -121,12 +121,12 @@ struct DecLayout {
     size_t bytes;
 };
 
-DecLayout dec_layout(void *ws, int B, int H, int Hkv, int64_t Tmax, int D, int topk) {
+DecLayout dec_layout(void *ws, int B, int H, int Hkv, int Tq, int64_t Tmax, int D, int topk) {
     DecLayout l{};
     Carver c{static_cast<char *>(ws)};
-    const hsa::DecodePlan pl = hsa::decode_plan(Tmax / 64, topk, B, H, Hkv);
+    const hsa::DecodePlan pl = hsa::decode_plan(Tmax / 64, topk, B, H, Hkv, Tq);
     const int64_t nsplit = pl.nsplit;
-    const size_t BH = (size_t)B * H;
+    const size_t BH = (size_t)B * H * Tq;  // query rows
     l.err = c.take<int32_t>(1);  // first: hsa_workspace_status reads it at offset 0
     l.cand = c.take<uint64_t>(BH * nsplit * topk);
     l.counters = c.take<unsigned>(2 * BH);
@@ -243,19 +243,21 @@ hsa_status hsa_forward_ex(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 
 size_t hsa_decode_workspace_size(int B, int H, int64_t Tmax, int D, int chunk, int topk) {
     (void)chunk;
     if (B < 1 || H < 1 || Tmax < 0 || D < 1 || topk < 1) return 0;
-    return dec_layout(nullptr, B, H, H, Tmax, D, topk).bytes;
+    return dec_layout(nullptr, B, H, H, 1, Tmax, D, topk).bytes;
 }
 
-size_t hsa_decode_ex_workspace_size(int B, int H, int Hkv, int64_t Tmax, int D, int chunk, int topk, unsigned flags) {
+size_t hsa_decode_ex_workspace_size(int B, int H, int Hkv, int Tq, int64_t Tmax, int D, int chunk, int topk,
+                                    unsigned flags) {
     (void)chunk;
     (void)flags;
-    if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || Tmax < 0 || D < 1 || topk < 1) return 0;
-    return dec_layout(nullptr, B, H, Hkv, Tmax, D, topk).bytes;
+    if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || Tq < 1 || Tmax < 0 || D < 1 || topk < 1) return 0;
+    return dec_layout(nullptr, B, H, Hkv, Tq, Tmax, D, topk).bytes;
 }
 
 static hsa_status decode_impl(const char *name, const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *Kc,
                               const hsa_bf16 *Vc, const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B,
-                              int H, int Hkv, int D, int chunk, int topk, float scale, bool qk_norm, hsa_bf16 *out,
+                              int H, int Hkv, int Tq, int D, int chunk, int topk, float scale, bool qk_norm,
+                              hsa_bf16 *out,
                               int32_t *sel_idx, float *sel_w, void *workspace, size_t workspace_bytes,
                               void *stream) {
     g_last_error.clear();
@@ -270,16 +272,22 @@ static hsa_status decode_impl(const char *name, const hsa_bf16 *qs, const hsa_bf
         return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned (cache_len 8-byte)");
     if ((sel_idx && !aligned16(sel_idx)) || (sel_w && !aligned16(sel_w)))
         return fail(HSA_ERR_INVALID_ARG, "sel_idx / sel_w must be 16-byte aligned");
-    if (hsa::decode_plan_smem(hsa::decode_plan(Tmax / 64, topk, B, H, Hkv), topk) > 227 * 1024)
+    if (Tq < 1 || Tq > 64) return fail(HSA_ERR_INVALID_ARG, "Tq must be in [1, 64] (got %d)", Tq);
+    if ((double)B * H * Tq >= 2147483647.0) return fail(HSA_ERR_UNSUPPORTED, "B*H*Tq must stay below 2^31");
+    const hsa::DecodePlan plan = hsa::decode_plan(Tmax / 64, topk, B, H, Hkv, Tq);
+    if (Tq > 1 && !plan.grouped)
+        return fail(HSA_ERR_UNSUPPORTED, "several query tokens per step need topk <= 32 (got %d) and a cache whose "
+                    "landmark ranges fit the grouped scan", topk);
+    if (hsa::decode_plan_smem(plan, topk) > 227 * 1024)
         return fail(HSA_ERR_UNSUPPORTED, "Tmax=%lld too large for topk=%d (scan merge exceeds shared memory)",
                     (long long)Tmax, topk);
-    DecLayout need = dec_layout(nullptr, B, H, Hkv, Tmax, D, topk);
+    DecLayout need = dec_layout(nullptr, B, H, Hkv, Tq, Tmax, D, topk);
     if ((st = check_ws(workspace, workspace_bytes, need.bytes)) != HSA_OK) return st;
-    DecLayout l = dec_layout(workspace, B, H, Hkv, Tmax, D, topk);
+    DecLayout l = dec_layout(workspace, B, H, Hkv, Tq, Tmax, D, topk);
     hsa::DecodeArgs a{};
     a.qs = qs; a.q = q; a.Kc = Kc; a.Vc = Vc; a.Lc = Lc; a.cache_len = cache_len;
     a.Tmax = Tmax; a.Nmax = Tmax / 64;
-    a.B = B; a.H = H; a.Hkv = Hkv; a.D = D; a.K = topk;
+    a.B = B; a.H = H; a.Hkv = Hkv; a.Tq = Tq; a.D = D; a.K = topk;
     a.scale = resolve_scale(scale, D);
     a.out = out;
     a.sel_idx = sel_idx ? sel_idx : l.sel_idx;
@@ -297,19 +305,19 @@ hsa_status hsa_decode(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
                       const int64_t *cache_len, int64_t Tmax, int B, int H, int D, int chunk, int topk,
                       float scale, hsa_bf16 *out, int32_t *sel_idx, float *sel_w, void *workspace,
                       size_t workspace_bytes, void *stream) {
-    return decode_impl("hsa_decode", q, q, Kc, Vc, Lc, cache_len, Tmax, B, H, H, D, chunk, topk, scale, false, out,
+    return decode_impl("hsa_decode", q, q, Kc, Vc, Lc, cache_len, Tmax, B, H, H, 1, D, chunk, topk, scale, false, out,
                        sel_idx, sel_w, workspace, workspace_bytes, stream);
 }
 
 hsa_status hsa_decode_ex(const hsa_bf16 *qs, const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_bf16 *Vc,
-                         const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B, int H, int Hkv, int D,
-                         int chunk, int topk, float scale, unsigned flags, hsa_bf16 *out, int32_t *sel_idx,
+                         const hsa_bf16 *Lc, const int64_t *cache_len, int64_t Tmax, int B, int H, int Hkv, int Tq,
+                         int D, int chunk, int topk, float scale, unsigned flags, hsa_bf16 *out, int32_t *sel_idx,
                          float *sel_w, void *workspace, size_t workspace_bytes, void *stream) {
     g_last_error.clear();
     hsa_status st = check_ex(H, Hkv, flags);
     if (st != HSA_OK) return st;
-    return decode_impl("hsa_decode_ex", qs ? qs : q, q, Kc, Vc, Lc, cache_len, Tmax, B, H, Hkv, D, chunk, topk, scale,
-                       (flags & HSA_QK_NORM) != 0, out, sel_idx, sel_w, workspace, workspace_bytes, stream);
+    return decode_impl("hsa_decode_ex", qs ? qs : q, q, Kc, Vc, Lc, cache_len, Tmax, B, H, Hkv, Tq, D, chunk, topk,
+                       scale, (flags & HSA_QK_NORM) != 0, out, sel_idx, sel_w, workspace, workspace_bytes, stream);
 }
 
 size_t hsa_backward_workspace_size(int B, int H, int T, int D, int chunk, int topk) {

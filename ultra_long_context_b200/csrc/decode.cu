@@ -326,9 +326,12 @@ __device__ inline uint64_t warp_topk_scores(const float *sc, int n, int64_t c0, 
     return lane < K ? best : 0ull;
 }
 
-// grid (nsplit, B*Hkv): the landmark range sp of key head kvh, for its Gh <= 16 query heads. The
-// scores of a tile of 8 landmarks for all heads are one m16n8k16 tensor-core product per 16 columns of
-// D (rows: the heads; M = 16 is below the tcgen05 tile, so the warp-level MMA). The reduction index is
+// grid (nsplit, B*Hkv, ceil(R / 16)): the landmark range sp of key head kvh, for 16 of its R = Gh * Tq
+// query rows (Gh query heads, Tq query tokens each; row r = g * Tq + i is token i of head g, and the
+// rows of a key head are consecutive in q). Token i sits at position cache_len - Tq + i and sees the
+// chunks that have ended at or before it. The scores of a tile of 8 landmarks for the 16 rows are one
+// m16n8k16 tensor-core product per 16 columns of D (M = 16 is below the tcgen05 tile, so the
+// warp-level MMA). The reduction index is
 // permuted the same way in both operands, so that each lane loads whole 16-byte chunks: lane (g, t4)
 // holds columns 32 s + 8 t4 .. + 7 of head rows g, g + 8 and of landmark g of the tile, and k-steps
 // 2 s, 2 s + 1 take the first and the second half of that chunk.
@@ -337,7 +340,7 @@ constexpr int kDecodeGroupThreads = 512;  // one CTA per SM: 16 warps stream, th
 template <int D>
 __global__ void __launch_bounds__(kDecodeGroupThreads, 1) decode_scan_group_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ Lc, const int64_t *__restrict__ cache_len, int Hkv,
-    int Gh, int64_t Nmax, int split, int nsplit, int K, float scale, uint64_t *__restrict__ cand) {
+    int R, int Tq, int64_t Nmax, int split, int nsplit, int K, float scale, uint64_t *__restrict__ cand) {
     constexpr int S = D / 32;      // 16-byte chunks per lane per row
     constexpr int NWARP = kDecodeGroupThreads / 32;
     constexpr int U = 4;           // landmark tiles in flight per warp
@@ -348,21 +351,26 @@ __global__ void __launch_bounds__(kDecodeGroupThreads, 1) decode_scan_group_kern
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t4 = lane & 3;
-    const int sp = blockIdx.x, kvh = blockIdx.y, b = kvh / Hkv;
-    int64_t nb = cache_len[b] / kChunk;
-    nb = nb < 0 ? 0 : (nb > Nmax ? Nmax : nb);
+    const int sp = blockIdx.x, kvh = blockIdx.y, b = kvh / Hkv, r0 = blockIdx.z * 16;
+    const int rows = min(16, R - r0);
+    const int64_t len = cache_len[b];
+    auto n_of = [&](int r) {  // chunks seen by row r: its token sits at len - Tq + r % Tq
+        int64_t n = (len - Tq + r % Tq + 1) / kChunk;
+        return n < 0 ? (int64_t)0 : (n > Nmax ? Nmax : n);
+    };
+    const int64_t nb = n_of(Tq - 1);  // the last token sees the most
     const int64_t c0 = (int64_t)sp * split;
     const int64_t c1 = min(c0 + (int64_t)split, nb);
     const int nloc = c1 > c0 ? (int)(c1 - c0) : 0;
-    const size_t bh0 = (size_t)kvh * Gh;  // first query head of the group
+    const size_t q0 = (size_t)kvh * R + r0;  // q row of this CTA's first row
 
     uint32_t a[S][2][4];
 #pragma unroll
     for (int s = 0; s < S; ++s) {
-        const uint4 qa = g < Gh ? *reinterpret_cast<const uint4 *>(q + (bh0 + g) * D + 32 * s + 8 * t4)
-                                : make_uint4(0u, 0u, 0u, 0u);
-        const uint4 qb = g + 8 < Gh ? *reinterpret_cast<const uint4 *>(q + (bh0 + g + 8) * D + 32 * s + 8 * t4)
-                                    : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 qa = g < rows ? *reinterpret_cast<const uint4 *>(q + (q0 + g) * D + 32 * s + 8 * t4)
+                                  : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 qb = g + 8 < rows ? *reinterpret_cast<const uint4 *>(q + (q0 + g + 8) * D + 32 * s + 8 * t4)
+                                      : make_uint4(0u, 0u, 0u, 0u);
         a[s][0][0] = qa.x; a[s][0][1] = qb.x; a[s][0][2] = qa.y; a[s][0][3] = qb.y;
         a[s][1][0] = qa.z; a[s][1][1] = qb.z; a[s][1][2] = qa.w; a[s][1][3] = qb.w;
     }
@@ -390,20 +398,22 @@ __global__ void __launch_bounds__(kDecodeGroupThreads, 1) decode_scan_group_kern
                 mma_bf16_16816(acc, a[s][1], v[u][s].z, v[u][s].w);
             }
             const int i0 = tile * 8 + 2 * t4;  // acc: heads g (0, 1) and g + 8 (2, 3), landmarks i0, i0 + 1
-            if (g < Gh) {
+            if (g < rows) {
                 if (i0 < nloc) sc[g * ld + i0] = acc[0] * scale;
                 if (i0 + 1 < nloc) sc[g * ld + i0 + 1] = acc[1] * scale;
             }
-            if (g + 8 < Gh) {
+            if (g + 8 < rows) {
                 if (i0 < nloc) sc[(g + 8) * ld + i0] = acc[2] * scale;
                 if (i0 + 1 < nloc) sc[(g + 8) * ld + i0 + 1] = acc[3] * scale;
             }
         }
     }
     __syncthreads();
-    for (int h = warp; h < Gh; h += NWARP) {
-        const uint64_t best = warp_topk_scores(sc + h * ld, nloc, c0, K, stage + warp * 64);
-        if (lane < K) cand[((bh0 + h) * nsplit + sp) * K + lane] = best;
+    for (int h = warp; h < rows; h += NWARP) {  // one row per warp; the row's own causal limit
+        const int64_t cr = min(c1, n_of(r0 + h));
+        const int nr = cr > c0 ? (int)(cr - c0) : 0;
+        const uint64_t best = warp_topk_scores(sc + h * ld, nr, c0, K, stage + warp * 64);
+        if (lane < K) cand[((q0 + h) * nsplit + sp) * K + lane] = best;
     }
 }
 
@@ -429,7 +439,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_merge_kernel(const uint
 template <int D, bool QKN>
 __global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ Kc, const uint16_t *__restrict__ Vc, int64_t Tmax,
-    int Gh, int K, float scale, const int32_t *__restrict__ sel_idx, const float *__restrict__ sel_w,
+    int Gh, int Tq, int K, float scale, const int32_t *__restrict__ sel_idx, const float *__restrict__ sel_w,
     float *__restrict__ partial, unsigned *counters, uint16_t *__restrict__ out) {
     constexpr int LPL = D / 8, LPW = 32 / LPL, NWARP = kDecodeThreads / 32;
     constexpr int GROUPS = kDecodeThreads / LPL;  // key groups for the P.V pass
@@ -462,7 +472,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
 #pragma unroll
             for (int e = 0; e < 8; ++e) qr[e] *= rq;
         }
-        const size_t row0 = ((size_t)(bh / Gh) * Tmax + (size_t)c * kChunk);  // the key head's cache
+        const size_t row0 = ((size_t)(bh / Tq / Gh) * Tmax + (size_t)c * kChunk);  // the key head's cache
         constexpr int ROUNDS = kChunk / (NWARP * LPW);
         const int sl = tid % LPL, grp = tid / LPL;
         // issue every K and V load of this thread up front so both overlap the logit math
@@ -575,18 +585,29 @@ static size_t decode_group_smem(int split) {
 }
 constexpr int kDecodeGroupMaxSplit = 3072;
 
-DecodePlan decode_plan(int64_t Nmax, int K, int B, int H, int Hkv) {
+DecodePlan decode_plan(int64_t Nmax, int K, int B, int H, int Hkv, int Tq) {
     DecodePlan p{};
     const int Gh = Hkv > 0 ? H / Hkv : 1;
-    if (Gh >= 2 && Gh <= 16 && K <= 32 && Nmax > 0) {
+    const int R = Gh * (Tq > 0 ? Tq : 1);  // query rows per key head
+    p.row_groups = (R + 15) / 16;
+    if (R >= 2 && K <= 32 && Nmax <= 0) {  // no chunk at all: one empty range
+        p.grouped = true;
+        p.split = 64;
+        p.nsplit = 1;
+        return p;
+    }
+    if (R >= 2 && K <= 32) {
         // one CTA per SM in a single wave, >= 256 landmarks per range; the merge keeps every candidate in
         // shared memory (ranges * K <= 8192, ranges <= 512)
-        int64_t ns = (int64_t)kDecodeSms / ((int64_t)B * Hkv);
+        int64_t ns = (int64_t)kDecodeSms / ((int64_t)B * Hkv * p.row_groups);
         ns = ns < 1 ? 1 : ns;
         const int64_t by_min = (Nmax + 255) / 256;
         ns = ns < by_min ? ns : by_min;
         const int64_t cap = (8192 / K < 512) ? 8192 / K : 512;
         ns = ns < cap ? ns : cap;
+        // ranges longer than the shared-memory score rows hold: more ranges (several waves), up to the cap
+        const int64_t by_smem = (Nmax + kDecodeGroupMaxSplit - 1) / kDecodeGroupMaxSplit;
+        if (ns < by_smem) ns = by_smem < cap ? by_smem : cap;
         int64_t split = (Nmax + ns - 1) / ns;
         split = (split + 63) / 64 * 64;
         if (split <= kDecodeGroupMaxSplit) {
@@ -624,21 +645,22 @@ static cudaError_t launch_attend(const DecodeArgs &a, dim3 grid, cudaStream_t s)
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     auto kern = a.qk_norm ? decode_attend_kernel<D, true> : decode_attend_kernel<D, false>;
-    return cudaLaunchKernelEx(&cfg, kern, a.q, a.Kc, a.Vc, a.Tmax, a.H / a.Hkv, a.K, a.scale, (const int32_t *)a.sel_idx,
-                              (const float *)a.sel_w, a.partial, a.counters + a.B * a.H, a.out);
+    return cudaLaunchKernelEx(&cfg, kern, a.q, a.Kc, a.Vc, a.Tmax, a.H / a.Hkv, a.Tq, a.K, a.scale,
+                              (const int32_t *)a.sel_idx,
+                              (const float *)a.sel_w, a.partial, a.counters + (size_t)a.B * a.H * a.Tq, a.out);
 }
 
 template <int D>
 static cudaError_t launch_decode_grouped(const DecodeArgs &a, const DecodePlan &pl, cudaStream_t s) {
-    const int Gh = a.H / a.Hkv;
+    const int R = a.H / a.Hkv * a.Tq, rows_q = a.B * a.H * a.Tq;
     const size_t gsmem = decode_group_smem(pl.split);
     cudaError_t e = cudaFuncSetAttribute(decode_scan_group_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)gsmem);
     if (e != cudaSuccess) return e;
     {
         HSA_PROF("decode_scan", s);
-        decode_scan_group_kernel<D><<<dim3(pl.nsplit, a.B * a.Hkv), kDecodeGroupThreads, gsmem, s>>>(
-            a.qs, a.Lc, a.cache_len, a.Hkv, Gh, a.Nmax, pl.split, pl.nsplit, a.K, a.scale, a.cand);
+        decode_scan_group_kernel<D><<<dim3(pl.nsplit, a.B * a.Hkv, pl.row_groups), kDecodeGroupThreads, gsmem, s>>>(
+            a.qs, a.Lc, a.cache_len, a.Hkv, R, a.Tq, a.Nmax, pl.split, pl.nsplit, a.K, a.scale, a.cand);
         e = cudaGetLastError();
     }
     if (e != cudaSuccess) return e;
@@ -646,7 +668,7 @@ static cudaError_t launch_decode_grouped(const DecodeArgs &a, const DecodePlan &
     e = cudaFuncSetAttribute(decode_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(a.B * a.H);
+    cfg.gridDim = dim3(rows_q);
     cfg.blockDim = dim3(kDecodeThreads);
     cfg.dynamicSmemBytes = msmem;
     cfg.stream = s;
@@ -661,24 +683,26 @@ static cudaError_t launch_decode_grouped(const DecodeArgs &a, const DecodePlan &
     }
     if (e != cudaSuccess) return e;
     HSA_PROF("decode_attend", s);
-    return launch_attend<D>(a, dim3(a.K, a.B * a.H), s);
+    return launch_attend<D>(a, dim3(a.K, rows_q), s);
 }
 
 cudaError_t launch_decode(const DecodeArgs &a0, cudaStream_t s) {
     DecodeArgs a = a0;
     if (a.Hkv <= 0) a.Hkv = a.H;
+    if (a.Tq <= 0) a.Tq = 1;
     if (a.H % a.Hkv != 0) return cudaErrorInvalidValue;
-    const DecodePlan pl = decode_plan(a.Nmax, a.K, a.B, a.H, a.Hkv);
+    const DecodePlan pl = decode_plan(a.Nmax, a.K, a.B, a.H, a.Hkv, a.Tq);
     if (pl.grouped) {
         cudaError_t e;
         {
             HSA_PROF("memset", s);
-            e = cudaMemsetAsync(a.counters, 0, 2 * (size_t)a.B * a.H * sizeof(unsigned), s);
+            e = cudaMemsetAsync(a.counters, 0, 2 * (size_t)a.B * a.H * a.Tq * sizeof(unsigned), s);
         }
         if (e != cudaSuccess) return e;
         e = a.D == 128 ? launch_decode_grouped<128>(a, pl, s) : launch_decode_grouped<64>(a, pl, s);
         return e != cudaSuccess ? e : cudaGetLastError();
     }
+    if (a.Tq != 1) return cudaErrorInvalidValue;  // several query tokens need the grouped scan (K <= 32)
     const int split = decode_split_size(a.Nmax, a.K, a.B * a.H);
     const int nsplit = (int)((a.Nmax + split - 1) / split) > 0 ? (int)((a.Nmax + split - 1) / split) : 1;
     const size_t smem = decode_scan_smem(split, nsplit, a.K);

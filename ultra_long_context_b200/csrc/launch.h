@@ -16,13 +16,14 @@ struct DecodeArgs {
     int64_t Tmax, Nmax;
     int B, H, D, K;
     int Hkv;           // key/value/landmark heads (H a multiple; query head h reads h / (H / Hkv))
+    int Tq;            // query tokens per sequence and head (q, out: [B, H, Tq, D]); 0 means 1
     float scale;
     uint16_t *out;
-    int32_t *sel_idx;  // [B*H, K] (caller's or workspace)
-    float *sel_w;      // [B*H, K]
-    uint64_t *cand;    // [B*H, nsplit, K]
-    unsigned *counters;  // [2, B*H]
-    float *partial;    // [B*H, K, D]
+    int32_t *sel_idx;  // [B*H*Tq, K] (caller's or workspace)
+    float *sel_w;      // [B*H*Tq, K]
+    uint64_t *cand;    // [B*H*Tq, nsplit, K]
+    unsigned *counters;  // [2, B*H*Tq]
+    float *partial;    // [B*H*Tq, K, D]
     bool qk_norm;      // Step 3 attends with q / max(|q|, eps) and k / max(|k|, eps)
 };
 int decode_split_size(int64_t Nmax, int K, int BH);
@@ -31,9 +32,10 @@ size_t decode_scan_smem(int split, int nsplit, int K);
 // one CTA per (range, key head) scores all query heads of the group and a merge kernel follows.
 struct DecodePlan {
     int split, nsplit;
+    int row_groups;  // grouped: CTAs per (range, key head), 16 query rows each
     bool grouped;
 };
-DecodePlan decode_plan(int64_t Nmax, int K, int B, int H, int Hkv);
+DecodePlan decode_plan(int64_t Nmax, int K, int B, int H, int Hkv, int Tq);
 size_t decode_plan_smem(const DecodePlan &p, int K);  // the largest dynamic shared memory of its kernels
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 

@@ -35,8 +35,9 @@ SIGNATURES = {
                      _I),
     "hsa_forward_ex_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _U], _SZ),
     "hsa_forward_ex": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _U, _P, _P, _P, _P, _SZ, _P], _I),
-    "hsa_decode_ex_workspace_size": ([_I, _I, _I, _I64, _I, _I, _I, _U], _SZ),
-    "hsa_decode_ex": ([_P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _F, _U, _P, _P, _P, _P, _SZ, _P], _I),
+    "hsa_decode_ex_workspace_size": ([_I, _I, _I, _I, _I64, _I, _I, _I, _U], _SZ),
+    "hsa_decode_ex": ([_P, _P, _P, _P, _P, _P, _I64, _I, _I, _I, _I, _I, _I, _I, _F, _U, _P, _P, _P, _P, _SZ, _P],
+                      _I),
     "hsa_backward_ex_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _U], _SZ),
     "hsa_backward_ex": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _U, _P, _P, _P, _P, _P,
                          _P, _SZ, _P], _I),
@@ -186,25 +187,29 @@ def hsa_decode_workspace_size(B, H, Tmax, D, chunk=64, topk=16):
     return int(lib().hsa_decode_workspace_size(B, H, Tmax, D, chunk, topk))
 
 
-def hsa_decode_ex_workspace_size(B, H, Hkv, Tmax, D, chunk=64, topk=16, flags=0):
-    return int(lib().hsa_decode_ex_workspace_size(B, H, Hkv, Tmax, D, chunk, topk, flags))
+def hsa_decode_ex_workspace_size(B, H, Hkv, Tmax, D, chunk=64, topk=16, flags=0, Tq=1):
+    return int(lib().hsa_decode_ex_workspace_size(B, H, Hkv, Tq, Tmax, D, chunk, topk, flags))
 
 
 def hsa_decode(q, Kc, Vc, Lc, cache_len, topk, scale=0.0, chunk=64, out=None, sel_idx=None, sel_w=None,
                workspace=None, stream=None, qs=None, qk_norm=False):
-    """HSA decode. q [B, H, D], Kc / Vc [B, Hkv, Tmax, D], Lc [B, Hkv, Tmax // 64, D] bf16; cache_len [B]
-    int64 (Hkv = H unless key/value heads are grouped).
+    """HSA decode. q [B, H, D] (or [B, H, Tq, D]: the last Tq tokens of each cache in one step),
+    Kc / Vc [B, Hkv, Tmax, D], Lc [B, Hkv, Tmax // 64, D] bf16; cache_len [B] int64 (Hkv = H unless key/value
+    heads are grouped).
 
-    qs: a separate retrieval query [B, H, D] bf16, or None when q does both. qk_norm: Step 3 attends with
-    the L2-normalised query and keys. Any of the three calls hsa_decode_ex, else hsa_decode.
-    Returns (out [B, H, D] bf16, sel_idx [B, H, topk] int32, sel_w [B, H, topk] fp32).
+    qs: a separate retrieval query shaped like q, or None when q does both. qk_norm: Step 3 attends with
+    the L2-normalised query and keys. Any option (or Tq > 1) calls hsa_decode_ex, else hsa_decode.
+    Returns (out shaped like q, sel_idx [..., topk] int32, sel_w [..., topk] fp32).
     """
-    B, H, D = q.shape
+    multi = q.dim() == 4
+    B, H, D = q.shape[0], q.shape[1], q.shape[-1]
+    Tq = q.shape[2] if multi else 1
+    qshape = tuple(q.shape)
     Hkv, Tmax = Kc.shape[1], Kc.shape[2]
     dev = q.device
-    _need(q, "q", torch.bfloat16, (B, H, D), dev)
+    _need(q, "q", torch.bfloat16, qshape, dev)
     if qs is not None:
-        _need(qs, "qs", torch.bfloat16, (B, H, D), dev)
+        _need(qs, "qs", torch.bfloat16, qshape, dev)
     _need(Kc, "Kc", torch.bfloat16, (B, Hkv, Tmax, D), dev)
     _need(Vc, "Vc", torch.bfloat16, (B, Hkv, Tmax, D), dev)
     _need(Lc, "Lc", torch.bfloat16, (B, Hkv, Tmax // chunk, D), dev)
@@ -212,10 +217,10 @@ def hsa_decode(q, Kc, Vc, Lc, cache_len, topk, scale=0.0, chunk=64, out=None, se
     if out is None:
         out = torch.empty_like(q)
     if sel_idx is None:
-        sel_idx = torch.empty((B, H, topk), dtype=torch.int32, device=dev)
+        sel_idx = torch.empty(qshape[:-1] + (topk,), dtype=torch.int32, device=dev)
     if sel_w is None:
-        sel_w = torch.empty((B, H, topk), dtype=torch.float32, device=dev)
-    if qs is None and not qk_norm and Hkv == H:
+        sel_w = torch.empty(qshape[:-1] + (topk,), dtype=torch.float32, device=dev)
+    if qs is None and not qk_norm and Hkv == H and not multi:
         nbytes = hsa_decode_workspace_size(B, H, Tmax, D, chunk, topk)
         ws = _workspace(nbytes, dev, workspace)
         wp, wn = _aligned(ws)
@@ -224,10 +229,10 @@ def hsa_decode(q, Kc, Vc, Lc, cache_len, topk, scale=0.0, chunk=64, out=None, se
         _check("hsa_decode", st)
     else:
         fl = _flags(qk_norm)
-        ws = _workspace(hsa_decode_ex_workspace_size(B, H, Hkv, Tmax, D, chunk, topk, fl), dev, workspace)
+        ws = _workspace(hsa_decode_ex_workspace_size(B, H, Hkv, Tmax, D, chunk, topk, fl, Tq), dev, workspace)
         wp, wn = _aligned(ws)
         st = lib().hsa_decode_ex(_ptr(qs), _ptr(q), _ptr(Kc), _ptr(Vc), _ptr(Lc), _ptr(cache_len), Tmax, B, H, Hkv,
-                                 D, chunk, topk, float(scale), fl, _ptr(out), _ptr(sel_idx), _ptr(sel_w), wp, wn,
+                                 Tq, D, chunk, topk, float(scale), fl, _ptr(out), _ptr(sel_idx), _ptr(sel_w), wp, wn,
                                  _stream(dev, stream))
         _check("hsa_decode_ex", st)
     return out, sel_idx, sel_w

@@ -430,9 +430,38 @@ def main():
             "tokens_per_s": round(whole_job_rate(Bg * w.T, world, g_ms), 1),
             "token_heads_per_s": round(whole_job_rate(Bg * w.T * Hg, world, g_ms), 1),
             "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_g.items()}}
-        extra["fwd_options"] = dict(workload=w.name, steps=osteps, **opts)
         del gQ, gK, gV, gL, gout, gidx, gw, gws
         torch.cuda.empty_cache()
+        # variable-length batches in the packed token-major layout: the headline batch itself (2 x 32768,
+        # the cost of the layout moves), and 65536 tokens in 7 sequences of 1K to 32K
+        tm = lambda x: x.transpose(1, 2).reshape(-1, x.shape[1], x.shape[3]).contiguous()
+        for name, lens in (("varlen_equal_2x32k", [w.T, w.T]),
+                           ("varlen_mixed_7seq", [32768, 16384, 8192, 4096, 2048, 1024, 1024])):
+            vQ = torch.cat([tm(inputs.forward_inputs(1, w.H, T, w.D, w.seed + 20 + i, landmarks=w.landmarks,
+                                                     device=dev)[0]) for i, T in enumerate(lens)])
+            vK, vV = torch.empty_like(vQ).normal_(), torch.empty_like(vQ).normal_()
+            vL = torch.randn((sum(T // 64 for T in lens), w.H, w.D), device=dev).to(torch.bfloat16)
+            cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32, device=dev)
+            vout = torch.empty_like(vQ)
+            vidx = torch.empty((vQ.shape[0], w.H, w.topk), dtype=torch.int32, device=dev)
+            vw = torch.empty((vQ.shape[0], w.H, w.topk), dtype=torch.float32, device=dev)
+            vws = torch.empty(hsa.lib().hsa_forward_varlen_workspace_size(len(lens), w.H, w.H, max(lens), w.D, 64,
+                                                                          w.topk, 0) + 256, dtype=torch.uint8,
+                              device=dev)
+
+            def fwd_var():
+                hsa.hsa_forward_varlen(vQ, vK, vV, vL, cu, max(lens), w.topk, out=vout, sel_idx=vidx, sel_w=vw,
+                                       workspace=vws)
+
+            v_ms = timed(fwd_var, osteps, args.warmup, world) / osteps
+            prof_v = kernel_profile(fwd_var, osteps)
+            opts[name] = {"lengths": lens, "ms_per_step": round(v_ms, 4),
+                          "tokens_per_s": round(whole_job_rate(sum(lens), world, v_ms), 1),
+                          "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)}
+                                      for k, (c, t) in prof_v.items()}}
+            del vQ, vK, vV, vL, vout, vidx, vw, vws
+            torch.cuda.empty_cache()
+        extra["fwd_options"] = dict(workload=w.name, steps=osteps, **opts)
 
     # ---------------- decode, 16M-token cache ----------------
     if not args.skip_decode:

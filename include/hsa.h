@@ -220,6 +220,40 @@ hsa_status hsa_backward_ex(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16
                            size_t workspace_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * Variable-length batches in the packed, token-major layout (no counterpart on the pages: the
+ * layout model code holds between layers). Same operation, options, rules and errors as the *_ex
+ * calls, per sequence:
+ *   cu_seqlens  [B + 1] int32, DEVICE: sequence b holds tokens cu_seqlens[b] .. cu_seqlens[b+1] - 1
+ *               (cu_seqlens[0] = 0, non-decreasing, every length <= max_seqlen; not checked)
+ *   Q, Qs, out, dout [total, H, D] bf16;  K, V [total, Hkv, D] bf16  (total = cu_seqlens[B])
+ *   L           [total_chunks, Hkv, D] bf16: sequence b's floor(len_b / 64) landmarks one after another,
+ *               in sequence order (total_chunks = the sum of those counts)
+ *   sel_idx, sel_w [total, H, topk]: chunk ids within the token's own sequence (0 .. len_b/64 - 1)
+ *   dQ, dQs [total, H, D], dK, dV [total, Hkv, D], dL [total_chunks, Hkv, D] fp32 (overwritten)
+ * A fixed-length batch in [B, T, H, D] layout is the case cu_seqlens[b] = b * T.
+ * The library moves the rows to a head-major batch padded to max_seqlen in the workspace (streaming
+ * copies), runs the batched kernels with each sequence's length (padded rows select nothing and cost no
+ * attention work) and moves the results back. The *_varlen_workspace_size functions size the
+ * workspace for max_seqlen, with room for a separate retrieval query.
+ * ------------------------------------------------------------------------------------------- */
+size_t hsa_forward_varlen_workspace_size(int B, int H, int Hkv, int max_seqlen, int D, int chunk, int topk,
+                                         unsigned flags);
+
+hsa_status hsa_forward_varlen(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
+                              const hsa_bf16 *L, const int32_t *cu_seqlens, int B, int max_seqlen, int H, int Hkv,
+                              int D, int chunk, int topk, float scale, unsigned flags, hsa_bf16 *out,
+                              int32_t *sel_idx, float *sel_w, void *workspace, size_t workspace_bytes, void *stream);
+
+size_t hsa_backward_varlen_workspace_size(int B, int H, int Hkv, int max_seqlen, int D, int chunk, int topk,
+                                          unsigned flags);
+
+hsa_status hsa_backward_varlen(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
+                               const hsa_bf16 *L, const hsa_bf16 *out, const hsa_bf16 *dout, const int32_t *sel_idx,
+                               const float *sel_w, const int32_t *cu_seqlens, int B, int max_seqlen, int H, int Hkv,
+                               int D, int chunk, int topk, float scale, unsigned flags, float *dQ, float *dK, float *dV,
+                               float *dL, float *dQs, void *workspace, size_t workspace_bytes, void *stream);
+
+/* ---------------------------------------------------------------------------------------------
  * Measurement hooks (no counterpart on the pages; used to time each kernel live).
  *
  * hsa_profile_enable(1) starts recording a pair of CUDA events around every kernel launch and

@@ -511,3 +511,92 @@ def test_decode_multi_token_with_options(oracle_mod):
     qs = inputs.forward_inputs(B, H, Tq, D, 2201, device=DEV)[0]
     _, Kc, Vc, Lc, lens_t, _ = inputs.decode_inputs(B, Hkv, lens, D, seed=81, Tmax=Tmax, device=DEV)
     check_decode_multi(oracle_mod, q, Kc, Vc, Lc, lens_t, topk, qs=qs, qk_norm=True)
+
+
+# ---------------------------------------------------------------------------------------------
+# variable-length batches, packed token-major: each sequence is its own HSA problem
+
+
+def varlen_batch(lens, H, Hkv, D, seed, separate=False):
+    """Per-sequence [1, H, T, D] inputs and their packed token-major concatenation."""
+    seqs = []
+    for b, T in enumerate(lens):
+        Q = inputs.forward_inputs(1, H, T, D, seed + 2 * b, device=DEV)[0]
+        _, K, V, L = inputs.forward_inputs(1, Hkv, T, D, seed + 2 * b + 1, device=DEV)
+        Qs = inputs.forward_inputs(1, H, T, D, seed + 100 + b, device=DEV)[0] if separate else None
+        seqs.append((Q, K, V, L, Qs))
+    pack = lambda xs: torch.cat([x[0].transpose(0, 1) for x in xs]).contiguous()  # [1,h,t,d] -> [t,h,d]
+    packed = [pack([s_[i] for s_ in seqs]) for i in range(4)]
+    packed.append(pack([s_[4] for s_ in seqs]) if separate else None)
+    cu = torch.tensor([0] + list(np.cumsum(lens)), dtype=torch.int32, device=DEV)
+    return seqs, packed, cu
+
+
+@pytest.mark.parametrize("lens,H,Hkv,D,topk,opts", [
+    ([1000, 64, 30, 2500, 700], 4, 2, 128, 8, {}),
+    ([600, 129, 1700], 2, 2, 64, 16, {"qk_norm": True, "separate": True}),
+    ([40, 20], 2, 1, 128, 4, {}),                    # no sequence has a complete chunk
+])
+def test_forward_varlen_matches_per_sequence_oracle(oracle_mod, lens, H, Hkv, D, topk, opts):
+    sep, qk = opts.get("separate", False), opts.get("qk_norm", False)
+    seqs, (Q, K, V, L, Qs), cu = varlen_batch(lens, H, Hkv, D, 3000 + D, separate=sep)
+    out, idx, w = hsa.hsa_forward_varlen(Q, K, V, L, cu, max(lens), topk, Qs=Qs, qk_norm=qk)
+    sc = 1 / math.sqrt(D)
+    for b, (Qb, Kb, Vb, Lb, Qsb) in enumerate(seqs):
+        T = lens[b]
+        rows = slice(int(cu[b]), int(cu[b + 1]))
+        g = lambda x, n: host(x[rows].transpose(0, 1)).reshape(-1, n)  # [t,h,n] -> (h, t) rows
+        Qh, Kh, Vh, Lh = (host(x) for x in (Qb, Kb, Vb, Lb))
+        Qsh = None if Qsb is None else host(Qsb)
+        orc = oracle_mod.forward(Qh, Kh, Vh, Lh, chunk=64, topk=topk, scale=sc, Qs=Qsh, qk_norm=qk)
+        compare_forward_rows(oracle_mod, g(out, D), g(idx, topk), g(w, topk), orc, Qh, Kh, Vh, Lh,
+                             np.arange(H * T), 64, sc, Qs=Qsh, qk_norm=qk)
+
+
+def test_forward_varlen_equal_lengths_equals_batched_call():
+    """[B, T, H, D] is the equal-length case: the same kernels, so the same selection as the batched call
+    and the same output up to the order of the fp32 reductions (which is not fixed between runs)."""
+    B, H, T, D, topk = 2, 4, 1100, 128, 16
+    Q, K, V, L = inputs.forward_inputs(B, H, T, D, 3100, device=DEV)
+    out_b, idx_b, w_b = hsa.hsa_forward(Q, K, V, L, topk)
+    tm = lambda x: x.transpose(1, 2).reshape(-1, x.shape[1], x.shape[3]).contiguous()  # [B,H,T,D] -> [B*T,H,D]
+    cu = torch.arange(0, (B + 1) * T, T, dtype=torch.int32, device=DEV)
+    out_v, idx_v, w_v = hsa.hsa_forward_varlen(tm(Q), tm(K), tm(V), tm(L), cu, T, topk)
+    assert torch.equal(idx_v, tm(idx_b))
+    assert torch.equal(w_v, tm(w_b))
+    assert (out_v.float() - tm(out_b).float()).abs().max() <= 2e-2
+
+
+@pytest.mark.parametrize("lens,H,Hkv,D,topk,opts", [
+    ([700, 1300, 65], 4, 2, 128, 8, {}),
+    ([900, 300], 2, 2, 64, 8, {"separate": True, "qk_norm": True}),
+])
+def test_backward_varlen_matches_per_sequence_oracle(oracle_mod, lens, H, Hkv, D, topk, opts):
+    sep, qk = opts.get("separate", False), opts.get("qk_norm", False)
+    seqs, (Q, K, V, L, Qs), cu = varlen_batch(lens, H, Hkv, D, 3200 + D, separate=sep)
+    dO = torch.cat([inputs.upstream_grad(1, H, T, D, 3300 + T, device=DEV)[0].transpose(0, 1) for T in lens])
+    dO = dO.contiguous()
+    sc = 1 / math.sqrt(D)
+    outs, sels, ws_, refs = [], [], [], []
+    for b, (Qb, Kb, Vb, Lb, Qsb) in enumerate(seqs):
+        T = lens[b]
+        Qh, Kh, Vh, Lh = (host(x) for x in (Qb, Kb, Vb, Lb))
+        Qsh = None if Qsb is None else host(Qsb)
+        orc = oracle_mod.forward(Qh, Kh, Vh, Lh, chunk=64, topk=topk, scale=sc, Qs=Qsh, qk_norm=qk)
+        dOb = host(dO[int(cu[b]):int(cu[b + 1])].transpose(0, 1))[None]
+        refs.append(oracle_mod.backward(Qh, Kh, Vh, Lh, dOb, orc["sel_idx"].reshape(1, H, T, topk), chunk=64,
+                                        scale=sc, Qs=Qsh, qk_norm=qk))
+        outs.append(torch.as_tensor(orc["out"].reshape(H, T, D)).transpose(0, 1))
+        sels.append(torch.as_tensor(orc["sel_idx"].reshape(H, T, topk)).transpose(0, 1))
+        ws_.append(torch.as_tensor(orc["sel_w"].reshape(H, T, topk)).transpose(0, 1))
+    out = torch.cat(outs).to(DEV, torch.float32).to(torch.bfloat16).contiguous()
+    sel_idx = torch.cat(sels).to(DEV, torch.int32).contiguous()
+    sel_w = torch.cat(ws_).to(DEV, torch.float32).contiguous()
+    grads = hsa.hsa_backward_varlen(Q, K, V, L, out, dO, sel_idx, sel_w, cu, max(lens), Qs=Qs, qk_norm=qk)
+    cuN = np.concatenate([[0], np.cumsum([T // 64 for T in lens])])
+    for b, T in enumerate(lens):
+        r, rl = slice(int(cu[b]), int(cu[b + 1])), slice(int(cuN[b]), int(cuN[b + 1]))
+        names = ("dQ", "dK", "dV", "dL", "dQs")
+        for g, ref, n in zip(grads, refs[b], names):
+            gb = g[rl] if n == "dL" else g[r]
+            grad_close(host(gb.transpose(0, 1))[None], ref, f"{n} (sequence {b})")

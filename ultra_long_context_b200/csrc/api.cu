@@ -189,7 +189,8 @@ static hsa_status forward_impl(const char *name, const hsa_bf16 *Qs, const hsa_b
                                const hsa_bf16 *V, const hsa_bf16 *L, int B, int H, int Hkv, int T, int D, int chunk,
                                int topk,
                                float scale, bool qk_norm, hsa_bf16 *out, int32_t *sel_idx, float *sel_w,
-                               void *workspace, size_t workspace_bytes, void *stream) {
+                               void *workspace, size_t workspace_bytes, void *stream,
+                               const int32_t *cu_seqlens = nullptr) {
     g_last_error.clear();
     hsa_status st = check_common(B, H, D, chunk, topk, 32);
     if (st != HSA_OK) return st;
@@ -207,6 +208,7 @@ static hsa_status forward_impl(const char *name, const hsa_bf16 *Qs, const hsa_b
     FwdLayout l = fwd_layout(workspace, B, H, T, D, topk, false, false, qk_norm);
     hsa::ForwardArgs a{};
     a.qk_norm = qk_norm; a.Qn = l.Qn; a.Kn = l.Kn;
+    a.cu_seqlens = cu_seqlens;
     a.Qs = Qs; a.Q = Q; a.K = K; a.V = V; a.L = L;
     a.B = B; a.H = H; a.Hkv = Hkv; a.T = T; a.D = D; a.N = T / 64; a.topk = topk;
     a.scale = resolve_scale(scale, D);
@@ -395,6 +397,167 @@ hsa_status hsa_backward_ex(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16
     return backward_impl("hsa_backward_ex", Qs, Q, K, V, L, out, dout, sel_idx, sel_w, B, H, Hkv, T, D, chunk, topk,
                          scale, dQ, dK, dV, dL, dQs, Qs != nullptr, (flags & HSA_QK_NORM) != 0, workspace,
                          workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+// ---- variable-length batches: packed token-major tensors <-> a padded head-major batch ----
+
+struct VarlenLayout {
+    size_t inner;  // the padded call's own workspace, first, so that its status flag sits at offset 0
+    int32_t *cuN;
+    uint16_t *Q, *Qs, *K, *V, *L, *out, *dout;
+    int32_t *sel_idx;
+    float *sel_w;
+    float *dQ, *dK, *dV, *dL, *dQs;
+    size_t bytes;
+};
+
+static VarlenLayout varlen_layout(void *ws, int B, int H, int Hkv, int Tp, int D, int topk, bool qk_norm,
+                                  bool backward) {
+    VarlenLayout l{};
+    l.inner = round_up(backward ? fwd_layout(nullptr, B, H, Tp, D, topk, true, true, qk_norm).bytes
+                                : fwd_layout(nullptr, B, H, Tp, D, topk, false, false, qk_norm).bytes);
+    Carver c{ws ? static_cast<char *>(ws) + l.inner : nullptr};
+    const size_t rq = (size_t)B * H * Tp, rk = (size_t)B * Hkv * Tp, rl = (size_t)B * Hkv * (Tp / 64);
+    l.cuN = c.take<int32_t>((size_t)B + 1);
+    l.Q = c.take<uint16_t>(rq * D);
+    l.Qs = c.take<uint16_t>(rq * D);  // room for a separate retrieval query (used only when one is given)
+    l.K = c.take<uint16_t>(rk * D);
+    l.V = c.take<uint16_t>(rk * D);
+    l.L = c.take<uint16_t>(rl * D);
+    l.out = c.take<uint16_t>(rq * D);
+    l.sel_idx = c.take<int32_t>(rq * topk);
+    l.sel_w = c.take<float>(rq * topk);
+    if (backward) {
+        l.dout = c.take<uint16_t>(rq * D);
+        l.dQ = c.take<float>(rq * D);
+        l.dK = c.take<float>(rk * D);
+        l.dV = c.take<float>(rk * D);
+        l.dL = c.take<float>(rl * D);
+        l.dQs = c.take<float>(rq * D);
+    }
+    l.bytes = l.inner + c.used;
+    return l;
+}
+
+// Shared checks of the two varlen calls; fills the padded length Tp.
+static hsa_status varlen_check(const int32_t *cu_seqlens, int B, int max_seqlen, int H, int Hkv, int D, int chunk,
+                               int topk, unsigned flags) {
+    hsa_status st = check_ex(H, Hkv, flags);
+    if (st != HSA_OK) return st;
+    if ((st = check_common(B, H, D, chunk, topk, 32)) != HSA_OK) return st;
+    if (max_seqlen < 1) return fail(HSA_ERR_INVALID_ARG, "max_seqlen must be >= 1 (got %d)", max_seqlen);
+    if (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+        return fail(HSA_ERR_INVALID_ARG, "cu_seqlens must be a 4-byte aligned device array of B + 1 entries");
+    if ((double)B * H * max_seqlen * topk >= 2147483647.0)
+        return fail(HSA_ERR_UNSUPPORTED, "B*H*max_seqlen*topk must stay below 2^31");
+    return HSA_OK;
+}
+
+extern "C" {
+
+size_t hsa_forward_varlen_workspace_size(int B, int H, int Hkv, int max_seqlen, int D, int chunk, int topk,
+                                         unsigned flags) {
+    (void)chunk;
+    if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || max_seqlen < 1 || D < 1 || topk < 1) return 0;
+    return varlen_layout(nullptr, B, H, Hkv, max_seqlen, D, topk, (flags & HSA_QK_NORM) != 0, false).bytes;
+}
+
+hsa_status hsa_forward_varlen(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
+                              const hsa_bf16 *L, const int32_t *cu_seqlens, int B, int max_seqlen, int H, int Hkv,
+                              int D, int chunk, int topk, float scale, unsigned flags, hsa_bf16 *out,
+                              int32_t *sel_idx, float *sel_w, void *workspace, size_t workspace_bytes,
+                              void *stream) {
+    g_last_error.clear();
+    hsa_status st = varlen_check(cu_seqlens, B, max_seqlen, H, Hkv, D, chunk, topk, flags);
+    if (st != HSA_OK) return st;
+    if (!Q || !K || !V || !L || !out || !sel_idx || !sel_w)
+        return fail(HSA_ERR_INVALID_ARG, "Q, K, V, L, out, sel_idx and sel_w must not be NULL");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(L) || !aligned16(out) || (Qs && !aligned16(Qs)) ||
+        (reinterpret_cast<uintptr_t>(sel_idx) & 3u) || (reinterpret_cast<uintptr_t>(sel_w) & 3u))
+        return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned (sel_idx, sel_w 4-byte)");
+    const bool qk = (flags & HSA_QK_NORM) != 0;
+    const int Tp = max_seqlen;
+    if ((st = check_ws(workspace, workspace_bytes, varlen_layout(nullptr, B, H, Hkv, Tp, D, topk, qk, false).bytes)) !=
+        HSA_OK)
+        return st;
+    const VarlenLayout l = varlen_layout(workspace, B, H, Hkv, Tp, D, topk, qk, false);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = hsa::launch_chunk_offsets(cu_seqlens, B, l.cuN, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(Q, l.Q, cu_seqlens, B, H, Tp, D * 2, true, false, 0u, s);
+    if (e == cudaSuccess && Qs) e = hsa::launch_varlen_rows(Qs, l.Qs, cu_seqlens, B, H, Tp, D * 2, true, false, 0u, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(K, l.K, cu_seqlens, B, Hkv, Tp, D * 2, true, false, 0u, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(V, l.V, cu_seqlens, B, Hkv, Tp, D * 2, true, false, 0u, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(L, l.L, l.cuN, B, Hkv, Tp / 64, D * 2, true, false, 0u, s);
+    if (e != cudaSuccess) return cuda_status(e, "hsa_forward_varlen");
+    st = forward_impl("hsa_forward_varlen", Qs ? l.Qs : l.Q, l.Q, l.K, l.V, l.L, B, H, Hkv, Tp, D, chunk, topk, scale,
+                      qk, l.out, l.sel_idx, l.sel_w, workspace, l.inner, stream, cu_seqlens);
+    if (st != HSA_OK) return st;
+    e = hsa::launch_varlen_rows(l.out, out, cu_seqlens, B, H, Tp, D * 2, false, false, 0u, s);
+    if (e == cudaSuccess)
+        e = hsa::launch_varlen_rows(l.sel_idx, sel_idx, cu_seqlens, B, H, Tp, topk * 4, false, false, 0u, s);
+    if (e == cudaSuccess)
+        e = hsa::launch_varlen_rows(l.sel_w, sel_w, cu_seqlens, B, H, Tp, topk * 4, false, false, 0u, s);
+    return cuda_status(e, "hsa_forward_varlen");
+}
+
+size_t hsa_backward_varlen_workspace_size(int B, int H, int Hkv, int max_seqlen, int D, int chunk, int topk,
+                                          unsigned flags) {
+    (void)chunk;
+    if (B < 1 || H < 1 || Hkv < 1 || H % Hkv != 0 || max_seqlen < 1 || D < 1 || topk < 1) return 0;
+    return varlen_layout(nullptr, B, H, Hkv, max_seqlen, D, topk, (flags & HSA_QK_NORM) != 0, true).bytes;
+}
+
+hsa_status hsa_backward_varlen(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_bf16 *K, const hsa_bf16 *V,
+                               const hsa_bf16 *L, const hsa_bf16 *out, const hsa_bf16 *dout, const int32_t *sel_idx,
+                               const float *sel_w, const int32_t *cu_seqlens, int B, int max_seqlen, int H, int Hkv,
+                               int D, int chunk, int topk, float scale, unsigned flags, float *dQ, float *dK, float *dV,
+                               float *dL, float *dQs, void *workspace, size_t workspace_bytes, void *stream) {
+    g_last_error.clear();
+    hsa_status st = varlen_check(cu_seqlens, B, max_seqlen, H, Hkv, D, chunk, topk, flags);
+    if (st != HSA_OK) return st;
+    if (!Q || !K || !V || !L || !out || !dout || !sel_idx || !sel_w || !dQ || !dK || !dV || !dL)
+        return fail(HSA_ERR_INVALID_ARG, "tensor pointers must not be NULL (dQs: exactly when Qs is given)");
+    if ((Qs == nullptr) != (dQs == nullptr))
+        return fail(HSA_ERR_INVALID_ARG, "dQs must be given exactly when Qs is");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(L) || !aligned16(out) || !aligned16(dout) ||
+        !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) || !aligned16(dL) || (Qs && !aligned16(Qs)) ||
+        (dQs && !aligned16(dQs)) || (reinterpret_cast<uintptr_t>(sel_idx) & 3u) ||
+        (reinterpret_cast<uintptr_t>(sel_w) & 3u))
+        return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned (sel_idx, sel_w 4-byte)");
+    const bool qk = (flags & HSA_QK_NORM) != 0;
+    const int Tp = max_seqlen;
+    if ((st = check_ws(workspace, workspace_bytes, varlen_layout(nullptr, B, H, Hkv, Tp, D, topk, qk, true).bytes)) !=
+        HSA_OK)
+        return st;
+    const VarlenLayout l = varlen_layout(workspace, B, H, Hkv, Tp, D, topk, qk, true);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int row = D * 2;
+    cudaError_t e = hsa::launch_chunk_offsets(cu_seqlens, B, l.cuN, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(Q, l.Q, cu_seqlens, B, H, Tp, row, true, false, 0u, s);
+    if (e == cudaSuccess && Qs) e = hsa::launch_varlen_rows(Qs, l.Qs, cu_seqlens, B, H, Tp, row, true, false, 0u, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(K, l.K, cu_seqlens, B, Hkv, Tp, row, true, false, 0u, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(V, l.V, cu_seqlens, B, Hkv, Tp, row, true, false, 0u, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(L, l.L, l.cuN, B, Hkv, Tp / 64, row, true, false, 0u, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(out, l.out, cu_seqlens, B, H, Tp, row, true, false, 0u, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(dout, l.dout, cu_seqlens, B, H, Tp, row, true, false, 0u, s);
+    // padded rows select nothing: chunk -1, weight 0
+    if (e == cudaSuccess)
+        e = hsa::launch_varlen_rows(sel_idx, l.sel_idx, cu_seqlens, B, H, Tp, topk * 4, true, true, 0xffffffffu, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(sel_w, l.sel_w, cu_seqlens, B, H, Tp, topk * 4, true, true, 0u, s);
+    if (e != cudaSuccess) return cuda_status(e, "hsa_backward_varlen");
+    st = backward_impl("hsa_backward_varlen", Qs ? l.Qs : nullptr, l.Q, l.K, l.V, l.L, l.out, l.dout, l.sel_idx,
+                       l.sel_w, B, H, Hkv, Tp, D, chunk, topk, scale, l.dQ, l.dK, l.dV, l.dL, Qs ? l.dQs : nullptr,
+                       Qs != nullptr, qk, workspace, l.inner, stream);
+    if (st != HSA_OK) return st;
+    const int frow = D * 4;
+    e = hsa::launch_varlen_rows(l.dQ, dQ, cu_seqlens, B, H, Tp, frow, false, false, 0u, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(l.dK, dK, cu_seqlens, B, Hkv, Tp, frow, false, false, 0u, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(l.dV, dV, cu_seqlens, B, Hkv, Tp, frow, false, false, 0u, s);
+    if (e == cudaSuccess) e = hsa::launch_varlen_rows(l.dL, dL, l.cuN, B, Hkv, Tp / 64, frow, false, false, 0u, s);
+    if (e == cudaSuccess && Qs) e = hsa::launch_varlen_rows(l.dQs, dQs, cu_seqlens, B, H, Tp, frow, false, false, 0u, s);
+    return cuda_status(e, "hsa_backward_varlen");
 }
 
 }  // extern "C"

@@ -53,6 +53,9 @@ struct ForwardArgs {
     const uint16_t *Q, *K, *V, *L;
     int B, H, T, D, N, topk;
     int Hkv;  // key/value/landmark heads: K, V [B, Hkv, T, D], L [B, Hkv, N, D]
+    // optional: sequences padded to T; sequence b has cu_seqlens[b+1] - cu_seqlens[b] valid tokens, and
+    // the rows past them select nothing (output 0, selection -1 / 0)
+    const int32_t *cu_seqlens;
     float scale;
     uint16_t *out;
     int32_t *sel_idx;  // [B*H*T, topk] (caller's or workspace)
@@ -89,7 +92,7 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
                             int32_t *chunk_count, int32_t *chunk_off, int32_t *tile_off, int32_t *chunk_cursor,
                             int32_t *pair_row,
                             float *pair_w, int32_t *pair_slot, PairTile *tiles, int32_t *num_tiles, int max_tiles,
-                            int tile_pairs, bool counts_ready, cudaStream_t s);
+                            int tile_pairs, bool counts_ready, cudaStream_t s, const int32_t *cu_seqlens = nullptr);
 
 struct BackwardArgs {
     const uint16_t *Qs;  // separate retrieval queries, or NULL when Q retrieves too
@@ -133,6 +136,14 @@ cudaError_t launch_l2norm_rows(const uint16_t *X0, uint16_t *Y0, size_t R0, cons
 // In place, per row: dX <- dX taken back through that normalisation of X (fp32 gradients).
 cudaError_t launch_l2norm_grad_rows(const uint16_t *X, float *dX, size_t rows, int D, cudaStream_t s);
 constexpr float kQkNormEps = 1e-6f;
+
+// Variable-length batches (varlen.cu). cuN[b] = the packed landmark row of sequence b's first chunk.
+cudaError_t launch_chunk_offsets(const int32_t *cu, int B, int32_t *cuN, cudaStream_t s);
+// Rows between the packed token-major layout [total, Hs, row] (sequence b at rows cu[b] ..) and the
+// head-major batch [B, Hs, Tp, row]; with fill_pad, pack fills the batch rows past a sequence's end
+// with `fill` (the rows no kernel reads are left alone otherwise).
+cudaError_t launch_varlen_rows(const void *src, void *dst, const int32_t *cu, int B, int Hs, int Tp, int row_bytes,
+                               bool pack, bool fill_pad, uint32_t fill, cudaStream_t s);
 
 // Message returned by hsa_last_error() on the calling thread.
 void set_last_error(const char *msg);

@@ -137,9 +137,12 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_kernel(const int32_t *_
                                                                 int32_t *__restrict__ chunk_cursor,
                                                                 int32_t *__restrict__ pair_row,
                                                                 float *__restrict__ pair_w,
-                                                                int32_t *__restrict__ pair_slot) {
+                                                                int32_t *__restrict__ pair_slot,
+                                                                const int32_t *__restrict__ cu_seqlens, int H) {
     extern __shared__ int s_mem[];
     const int bh = blockIdx.y;
+    const int Tv = cu_seqlens ? min(T, cu_seqlens[bh / H + 1] - cu_seqlens[bh / H]) : T;
+    if ((int)(blockIdx.x * kDispatchRows) >= Tv) return;
     const bool use_smem = N <= kSmemHistMax / 2;
     int *s_cnt = s_mem, *s_base = s_mem + (use_smem ? N : 0);
     const int t = blockIdx.x * kDispatchRows + threadIdx.x;
@@ -147,7 +150,7 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_kernel(const int32_t *_
     if (use_smem) {
         for (int i = threadIdx.x; i < N; i += blockDim.x) s_cnt[i] = 0;
         __syncthreads();
-        if (t < T)
+        if (t < Tv)
             for (int j = 0; j < K; ++j)
                 if (si[j] >= 0 && si[j] < N) atomicAdd(&s_cnt[si[j]], 1);
         __syncthreads();
@@ -158,7 +161,7 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_kernel(const int32_t *_
         }
         __syncthreads();
     }
-    if (t >= T) return;
+    if (t >= Tv) return;
     const size_t row = (size_t)bh * T + t;
     for (int j = 0; j < K; ++j) {
         const int c = si[j];
@@ -181,7 +184,7 @@ constexpr int kSortedScatterMaxN = 2048;
 __global__ void __launch_bounds__(kDispatchRows) scatter_sorted_kernel(
     const int32_t *__restrict__ sel_idx, const float *__restrict__ sel_w, int T, int N, int K,
     const int32_t *__restrict__ chunk_off, int32_t *__restrict__ chunk_cursor, int32_t *__restrict__ pair_row,
-    float *__restrict__ pair_w, int32_t *__restrict__ pair_slot) {
+    float *__restrict__ pair_w, int32_t *__restrict__ pair_slot, const int32_t *__restrict__ cu_seqlens, int H) {
     extern __shared__ int s_mem[];
     int *s_cnt = s_mem;                  // [N] entries per chunk in this block
     int *s_scan = s_cnt + N;             // [N] exclusive scan of s_cnt
@@ -192,11 +195,13 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_sorted_kernel(
     __shared__ int s_warp[33];
     const int bh = blockIdx.y, tid = threadIdx.x;
     const int t0 = blockIdx.x * kDispatchRows;
+    const int Tv = cu_seqlens ? min(T, cu_seqlens[bh / H + 1] - cu_seqlens[bh / H]) : T;  // rows past it: none
+    if (t0 >= Tv) return;
     const int t = t0 + tid;
     for (int i = tid; i < N; i += blockDim.x) { s_cnt[i] = 0; s_cur[i] = 0; }
     __syncthreads();
     const int32_t *si = sel_idx + ((size_t)bh * T + (t < T ? t : 0)) * K;
-    if (t < T)
+    if (t < Tv)
         for (int j = 0; j < K; ++j) {
             const int c = si[j];
             if (c >= 0 && c < N) atomicAdd(&s_cnt[c], 1);
@@ -216,7 +221,7 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_sorted_kernel(
         off += cnt;
     }
     __syncthreads();
-    if (t < T)
+    if (t < Tv)
         for (int j = 0; j < K; ++j) {
             const int c = si[j];
             if (c < 0 || c >= N) continue;
@@ -235,9 +240,16 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_sorted_kernel(
     }
 }
 
-__global__ void finalize_kernel(const float *__restrict__ o_acc, uint16_t *__restrict__ out, size_t n8) {
-    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= n8) return;
+// o_acc -> out (bf16, round to nearest even), 8 elements per thread; grid (ceil(T*D/8/256), B*H). With
+// cu_seqlens (sequences padded to T), the rows past a sequence's end are skipped: the caller never reads
+// them.
+__global__ void finalize_kernel(const float *__restrict__ o_acc, uint16_t *__restrict__ out,
+                                const int32_t *__restrict__ cu_seqlens, int T, int H, int D) {
+    const int bh = blockIdx.y;
+    const int Tv = cu_seqlens ? min(T, cu_seqlens[bh / H + 1] - cu_seqlens[bh / H]) : T;
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;  // 8-element unit within this (b, h)
+    if (j >= Tv * (D / 8)) return;
+    const size_t i = (size_t)bh * T * (D / 8) + j;
     const float4 a = reinterpret_cast<const float4 *>(o_acc)[2 * i];
     const float4 b = reinterpret_cast<const float4 *>(o_acc)[2 * i + 1];
     uint4 r;
@@ -259,7 +271,7 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
                             int32_t *chunk_count, int32_t *chunk_off, int32_t *tile_off, int32_t *chunk_cursor,
                             int32_t *pair_row,
                             float *pair_w, int32_t *pair_slot, PairTile *tiles, int32_t *num_tiles, int max_tiles,
-                            int tile_pairs, bool counts_ready, cudaStream_t s) {
+                            int tile_pairs, bool counts_ready, cudaStream_t s, const int32_t *cu_seqlens) {
     const int BH = B * H, M = BH * N;
     dim3 dgrid((T + kDispatchRows - 1) / kDispatchRows, BH);
     const size_t hsmem = N <= kSmemHistMax ? (size_t)N * sizeof(int) : 0;
@@ -287,7 +299,8 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
         if (e != cudaSuccess) return e;
         HSA_PROF("dispatch_scatter", s);
         scatter_sorted_kernel<<<dgrid, kDispatchRows, ssmem, s>>>(sel_idx, sel_w, T, N, topk, chunk_off,
-                                                                  chunk_cursor, pair_row, pair_w, pair_slot);
+                                                                  chunk_cursor, pair_row, pair_w, pair_slot,
+                                                                  cu_seqlens, H);
     } else {
         const size_t ssmem = N <= kSmemHistMax / 2 ? 2 * (size_t)N * sizeof(int) : 0;
         if (ssmem > 48 * 1024) {
@@ -296,7 +309,7 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
         }
         HSA_PROF("dispatch_scatter", s);
         scatter_kernel<<<dgrid, kDispatchRows, ssmem, s>>>(sel_idx, sel_w, T, N, topk, chunk_off, chunk_cursor,
-                                                           pair_row, pair_w, pair_slot);
+                                                           pair_row, pair_w, pair_slot, cu_seqlens, H);
     }
     return cudaGetLastError();
 }
@@ -314,7 +327,7 @@ cudaError_t launch_forward(const ForwardArgs &a0, cudaStream_t s) {
         a.K = a0.Kn;
     }
     const int BH = a.B * a.H;
-    const size_t rows = (size_t)BH * a.T, chunks = (size_t)BH * a.N;
+    const size_t chunks = (size_t)BH * a.N;
     cudaError_t e;
     {
         HSA_PROF("memset", s);
@@ -327,20 +340,21 @@ cudaError_t launch_forward(const ForwardArgs &a0, cudaStream_t s) {
     e = launch_score_tc(a, s);
     if (e != cudaSuccess) return e;
     if (a.N == 0) {
-        const size_t n8 = rows * a.D / 8;
         HSA_PROF("finalize", s);
-        finalize_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a.o_acc, a.out, n8);
+        finalize_kernel<<<dim3((unsigned)(((size_t)a.T * a.D / 8 + 255) / 256), BH), 256, 0, s>>>(
+            a.o_acc, a.out, a.cu_seqlens, a.T, a.H, a.D);
         return cudaGetLastError();
     }
     e = launch_dispatch(a.sel_idx, a.sel_w, a.B, a.H, a.T, a.N, a.topk, a.chunk_count, a.chunk_off, a.tile_off,
-                        a.chunk_cursor, a.pair_row, a.pair_w, nullptr, a.tiles, a.num_tiles, a.max_tiles, 128, true, s);
+                        a.chunk_cursor, a.pair_row, a.pair_w, nullptr, a.tiles, a.num_tiles, a.max_tiles, 128, true, s,
+                        a.cu_seqlens);
     if (e != cudaSuccess) return e;
     e = launch_attn_tc(a, s);
     if (e != cudaSuccess) return e;
-    const size_t n8 = rows * a.D / 8;
     {
         HSA_PROF("finalize", s);
-        finalize_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, s>>>(a.o_acc, a.out, n8);
+        finalize_kernel<<<dim3((unsigned)(((size_t)a.T * a.D / 8 + 255) / 256), BH), 256, 0, s>>>(
+            a.o_acc, a.out, a.cu_seqlens, a.T, a.H, a.D);
     }
     return cudaGetLastError();
 }

@@ -79,7 +79,8 @@ struct StSmem {
 
 template <int D, int K>
 __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_t *__restrict__ Q, int T, int N,
-                                                                   int Gh, float scale, int kout,
+                                                                   int Gh, int H, const int32_t *__restrict__ cu_seqlens,
+                                                                   float scale, int kout,
                                                                    int32_t *__restrict__ sel_idx,
                                                                    float *__restrict__ sel_w, float *__restrict__ o_acc,
                                                                    int32_t *__restrict__ chunk_count,
@@ -103,17 +104,21 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
     const int bh = blockIdx.y, kvh = bh / Gh;  // Gh query heads share a landmark head
     const int t0 = tile * kStRows;
     const int nrows = min(kStRows, T - t0);
-    const int t_last = t0 + nrows - 1;
-    const int n_max = min(N, (t_last + 1) / kChunk);
+    // valid tokens of this sequence: all T, or its length when the batch holds sequences padded to T
+    const int Tv = cu_seqlens ? min(T, cu_seqlens[bh / H + 1] - cu_seqlens[bh / H]) : T;
+    const int t_last = min(t0 + nrows - 1, Tv - 1);
+    const int n_max = t_last >= 0 ? min(N, (t_last + 1) / kChunk) : 0;
     const int nblk = (n_max + kStCols - 1) / kStCols;
     const size_t out0 = ((size_t)bh * T + t0) * kout;  // the tile's rows are contiguous
 
+    // rows past the sequence's end (padded batches) are never read: no accumulator, no selection written
+    const int nv = max(0, min(nrows, Tv - t0));
     {  // this tile's rows of the fp32 output accumulator start at zero (the chunk attention adds into them)
         float4 *acc = reinterpret_cast<float4 *>(o_acc + ((size_t)bh * T + t0) * D);
-        for (int i = tid; i < nrows * (D / 4); i += kStThreads) acc[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        for (int i = tid; i < nv * (D / 4); i += kStThreads) acc[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
     if (nblk == 0) {  // no token of this tile has a complete chunk
-        for (int i = tid; i < nrows * kout; i += kStThreads) {
+        for (int i = tid; i < nv * kout; i += kStThreads) {
             sel_idx[out0 + i] = -1;
             sel_w[out0 + i] = 0.0f;
         }
@@ -193,7 +198,7 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
     } else {
         // ---------------- selecting warps: one token row per thread ----------------
         const int my_t = t0 + tid;
-        const int my_n = my_t < T ? min(N, (my_t + 1) / kChunk) : 0;
+        const int my_n = my_t < Tv ? min(N, (my_t + 1) / kChunk) : 0;
         const int k_keep = min(kout, my_n);
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
 
@@ -329,7 +334,7 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
             }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kStConsumers) : "memory");
-        for (int i = tid; i < nrows * kout; i += kStConsumers) {
+        for (int i = tid; i < nv * kout; i += kStConsumers) {
             sel_idx[out0 + i] = st_idx[i];
             sel_w[out0 + i] = st_w[i];
         }
@@ -354,7 +359,8 @@ static cudaError_t launch_st(const ForwardArgs &a, const CUtensorMap &tl, cudaSt
     if (e != cudaSuccess) return e;
     dim3 grid((a.T + kStRows - 1) / kStRows, a.B * a.H);
     HSA_PROF("score_topk", s);
-    score_topk_tc_kernel<D, K><<<grid, kStThreads, smem, s>>>(a.Qs, a.T, a.N, a.H / a.Hkv, a.scale, a.topk,
+    score_topk_tc_kernel<D, K><<<grid, kStThreads, smem, s>>>(a.Qs, a.T, a.N, a.H / a.Hkv, a.H, a.cu_seqlens,
+                                                              a.scale, a.topk,
                                                               a.sel_idx, a.sel_w, a.o_acc, a.chunk_count, a.err, tl);
     return cudaGetLastError();
 }

@@ -41,6 +41,12 @@ SIGNATURES = {
     "hsa_backward_ex_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _U], _SZ),
     "hsa_backward_ex": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _U, _P, _P, _P, _P, _P,
                          _P, _SZ, _P], _I),
+    "hsa_forward_varlen_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _U], _SZ),
+    "hsa_forward_varlen": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _U, _P, _P, _P, _P, _SZ, _P],
+                           _I),
+    "hsa_backward_varlen_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _U], _SZ),
+    "hsa_backward_varlen": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _U, _P, _P,
+                             _P, _P, _P, _P, _SZ, _P], _I),
     "hsa_profile_enable": ([_I], _I),
     "hsa_profile_summary": ([ctypes.c_char_p, _SZ], _I),
 }
@@ -315,6 +321,75 @@ def hsa_backward(Q, K, V, L, out, dout, sel_idx, sel_w, scale=0.0, chunk=64, gra
                                _ptr(sel_w), B, H, Hkv, T, D, chunk, topk, float(scale), fl, _ptr(dQ), _ptr(dK),
                                _ptr(dV), _ptr(dL) if dL.numel() else None, _ptr(dQs), wp, wn, _stream(dev, stream))
     _check("hsa_backward_ex", st)
+    return (dQ, dK, dV, dL) if Qs is None else (dQ, dK, dV, dL, dQs)
+
+
+def _varlen_shapes(Q, K, L, cu_seqlens, chunk):
+    total, H, D = Q.shape
+    Hkv = K.shape[1]
+    B = cu_seqlens.numel() - 1
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or B < 1:
+        raise ValueError("cu_seqlens must be an int32 CUDA tensor of B + 1 offsets")
+    return total, H, Hkv, D, B
+
+
+def hsa_forward_varlen(Q, K, V, L, cu_seqlens, max_seqlen, topk, scale=0.0, chunk=64, out=None, sel_idx=None,
+                       sel_w=None, workspace=None, stream=None, Qs=None, qk_norm=False):
+    """HSA forward of a variable-length batch in the packed token-major layout: Q [total, H, D], K, V
+    [total, Hkv, D], L [total_chunks, Hkv, D] bf16 (each sequence's floor(len / 64) landmarks in order),
+    cu_seqlens [B + 1] int32 on the device, every length <= max_seqlen. Returns (out [total, H, D],
+    sel_idx / sel_w [total, H, topk]; chunk ids within each sequence)."""
+    total, H, Hkv, D, B = _varlen_shapes(Q, K, L, cu_seqlens, chunk)
+    dev = Q.device
+    _need(Q, "Q", torch.bfloat16, (total, H, D), dev)
+    if Qs is not None:
+        _need(Qs, "Qs", torch.bfloat16, (total, H, D), dev)
+    for n, t in (("K", K), ("V", V)):
+        _need(t, n, torch.bfloat16, (total, Hkv, D), dev)
+    _need(L, "L", torch.bfloat16, (L.shape[0], Hkv, D), dev)
+    out = torch.empty_like(Q) if out is None else out
+    sel_idx = torch.empty((total, H, topk), dtype=torch.int32, device=dev) if sel_idx is None else sel_idx
+    sel_w = torch.empty((total, H, topk), dtype=torch.float32, device=dev) if sel_w is None else sel_w
+    fl = _flags(qk_norm)
+    ws = _workspace(int(lib().hsa_forward_varlen_workspace_size(B, H, Hkv, max_seqlen, D, chunk, topk, fl)), dev,
+                    workspace)
+    wp, wn = _aligned(ws)
+    st = lib().hsa_forward_varlen(_ptr(Qs), _ptr(Q), _ptr(K), _ptr(V), _ptr(L) if L.numel() else _ptr(Q),
+                                  _ptr(cu_seqlens), B, max_seqlen, H, Hkv, D, chunk, topk, float(scale), fl, _ptr(out),
+                                  _ptr(sel_idx), _ptr(sel_w), wp, wn, _stream(dev, stream))
+    _check("hsa_forward_varlen", st)
+    return out, sel_idx, sel_w
+
+
+def hsa_backward_varlen(Q, K, V, L, out, dout, sel_idx, sel_w, cu_seqlens, max_seqlen, scale=0.0, chunk=64,
+                        workspace=None, stream=None, Qs=None, qk_norm=False):
+    """Backward of hsa_forward_varlen for its selection. Returns (dQ, dK, dV, dL) fp32 in the packed
+    layout (and dQs with a separate retrieval query)."""
+    total, H, Hkv, D, B = _varlen_shapes(Q, K, L, cu_seqlens, chunk)
+    topk = sel_idx.shape[-1]
+    dev = Q.device
+    for n, t in (("Q", Q), ("out", out), ("dout", dout)):
+        _need(t, n, torch.bfloat16, (total, H, D), dev)
+    for n, t in (("K", K), ("V", V)):
+        _need(t, n, torch.bfloat16, (total, Hkv, D), dev)
+    _need(sel_idx, "sel_idx", torch.int32, (total, H, topk), dev)
+    _need(sel_w, "sel_w", torch.float32, (total, H, topk), dev)
+    dQ = torch.empty((total, H, D), dtype=torch.float32, device=dev)
+    dK = torch.empty((total, Hkv, D), dtype=torch.float32, device=dev)
+    dV = torch.empty((total, Hkv, D), dtype=torch.float32, device=dev)
+    dL = torch.empty(tuple(L.shape), dtype=torch.float32, device=dev)
+    dQs = torch.empty_like(dQ) if Qs is not None else None
+    fl = _flags(qk_norm)
+    ws = _workspace(int(lib().hsa_backward_varlen_workspace_size(B, H, Hkv, max_seqlen, D, chunk, topk, fl)), dev,
+                    workspace)
+    wp, wn = _aligned(ws)
+    # a zero-row L / dL still needs a valid (never read) 16-byte aligned pointer
+    lp = _ptr(L) if L.numel() else _ptr(Q)
+    dlp = _ptr(dL) if dL.numel() else _ptr(dQ)
+    st = lib().hsa_backward_varlen(_ptr(Qs), _ptr(Q), _ptr(K), _ptr(V), lp, _ptr(out), _ptr(dout), _ptr(sel_idx),
+                                   _ptr(sel_w), _ptr(cu_seqlens), B, max_seqlen, H, Hkv, D, chunk, topk, float(scale),
+                                   fl, _ptr(dQ), _ptr(dK), _ptr(dV), dlp, _ptr(dQs), wp, wn, _stream(dev, stream))
+    _check("hsa_backward_varlen", st)
     return (dQ, dK, dV, dL) if Qs is None else (dQ, dK, dV, dL, dQs)
 
 

@@ -177,7 +177,7 @@ def kernel_profile(fn, steps):
 # current kernels on these workloads; set back to None whenever the kernel changes.
 TRAFFIC_BYTES = {
     ("fwd_t32k_h8_d128_k16", "chunk_attn"): 737_362_176 + 241_751_808,
-    ("fwd_t32k_h8_d128_k16", "score_topk"): None,  # kernel changed since the last capture
+    ("fwd_t32k_h8_d128_k16", "score_topk"): 136_421_120 + 276_684_544,
     # captured on a 4M-token cache (134.3 MB of landmarks read per scan); the scan's traffic grows in
     # proportion to the landmarks, so the 16M-token figure is four times that capture
     ("decode_16m_b1_h8_d128_k32", "decode_scan"): 4 * (134_291_456 + 143_872),
@@ -299,6 +299,8 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-options", action="store_true",
                     help="skip the timings of the optional paths (query-key norm, separate retrieval query)")
+    ap.add_argument("--grouped-decode-only", action="store_true",
+                    help="of the decode, time only the 16:1 grouped-head case (small footprint, for profiling)")
     ap.add_argument("--decode-cache-len", type=int, default=None,
                     help="override the decode cache length (small cases for profiling)")
     args = ap.parse_args()
@@ -471,55 +473,56 @@ def main():
 
             wd = dataclasses.replace(wd, name=f"decode_{args.decode_cache_len}_b1_h8_d128_k32",
                                      cache_len=args.decode_cache_len)
-        q, Kc, Vc, Lc, lens, _ = inputs.workload_inputs(wd, device=dev)
-        dout_ = torch.empty_like(q)
-        didx = torch.empty((wd.B, wd.H, wd.topk), dtype=torch.int32, device=dev)
-        dw = torch.empty((wd.B, wd.H, wd.topk), dtype=torch.float32, device=dev)
-        dws = torch.empty(hsa.hsa_decode_workspace_size(wd.B, wd.H, wd.cache_len, wd.D, 64, wd.topk) + 256,
-                          dtype=torch.uint8, device=dev)
-
-        def dec():
-            hsa.hsa_decode(q, Kc, Vc, Lc, lens, wd.topk, out=dout_, sel_idx=didx, sel_w=dw, workspace=dws)
-
         dsteps = max(args.steps, 50)
-        dms = timed(dec, dsteps, args.warmup, world) / dsteps
-        prof_dec = kernel_profile(dec, dsteps)
         n = wd.cache_len // 64
-        scan_bytes = wd.B * wd.H * (n * wd.D * 2 + wd.D * 2)
-        gather_bytes = wd.B * wd.H * wd.topk * 2 * 64 * wd.D * 2
-        hbm_peak = peaks["hbm_gbs"]
-        extra["decode_16m"] = {
-            "workload": wd.name, "us_per_token": round(dms * 1e3 / wd.B, 3), "ms_per_step": round(dms, 5),
-            "steps": dsteps,
-            "roofline": roofline_entry("decode_scan", prof_dec, scan_bytes, "GB/s", hbm_peak, "hbm",
-                                       f"{peak_kind} hbm_gbs", TRAFFIC_BYTES.get((wd.name, "decode_scan"))),
-            "step_vs_hbm": {"algorithmic_bytes": scan_bytes + gather_bytes,
-                            "achieved_GBs": round((scan_bytes + gather_bytes) / (dms / 1e3) / 1e9, 1),
-                            "frac": round((scan_bytes + gather_bytes) / (dms / 1e3) / 1e9 / hbm_peak, 4)},
-            "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_dec.items()},
-        }
-        if not args.skip_options:  # 4 query tokens per sequence in one step (e.g. verifying 4 drafted tokens)
-            Tq = 4
-            mq = inputs.forward_inputs(wd.B, wd.H, Tq, wd.D, wd.seed + 5, device=dev)[0]
-            mout = torch.empty_like(mq)
-            midx = torch.empty((wd.B, wd.H, Tq, wd.topk), dtype=torch.int32, device=dev)
-            mw = torch.empty((wd.B, wd.H, Tq, wd.topk), dtype=torch.float32, device=dev)
-            mws = torch.empty(hsa.hsa_decode_ex_workspace_size(wd.B, wd.H, wd.H, wd.cache_len, wd.D, 64, wd.topk, 0, Tq)
-                              + 256, dtype=torch.uint8, device=dev)
+        if not args.grouped_decode_only:
+            q, Kc, Vc, Lc, lens, _ = inputs.workload_inputs(wd, device=dev)
+            dout_ = torch.empty_like(q)
+            didx = torch.empty((wd.B, wd.H, wd.topk), dtype=torch.int32, device=dev)
+            dw = torch.empty((wd.B, wd.H, wd.topk), dtype=torch.float32, device=dev)
+            dws = torch.empty(hsa.hsa_decode_workspace_size(wd.B, wd.H, wd.cache_len, wd.D, 64, wd.topk) + 256,
+                              dtype=torch.uint8, device=dev)
 
-            def dec_multi():
-                hsa.hsa_decode(mq, Kc, Vc, Lc, lens, wd.topk, out=mout, sel_idx=midx, sel_w=mw, workspace=mws)
+            def dec():
+                hsa.hsa_decode(q, Kc, Vc, Lc, lens, wd.topk, out=dout_, sel_idx=didx, sel_w=dw, workspace=dws)
 
-            mms = timed(dec_multi, dsteps, args.warmup, world) / dsteps
-            prof_m = kernel_profile(dec_multi, dsteps)
-            extra["decode_16m"]["multi_token_4"] = {
-                "shape": f"B{wd.B} H{wd.H} Tq{Tq} cache {wd.cache_len} D{wd.D} topk{wd.topk}",
-                "us_per_step": round(mms * 1e3, 3), "us_per_token": round(mms * 1e3 / (wd.B * Tq), 3),
-                "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_m.items()}}
-            del mq, mout, mws
-        del q, Kc, Vc, Lc, dws
-        torch.cuda.empty_cache()
-        if not args.skip_options:  # 16 query heads on one key/value head, same cache length
+            dms = timed(dec, dsteps, args.warmup, world) / dsteps
+            prof_dec = kernel_profile(dec, dsteps)
+            scan_bytes = wd.B * wd.H * (n * wd.D * 2 + wd.D * 2)
+            gather_bytes = wd.B * wd.H * wd.topk * 2 * 64 * wd.D * 2
+            hbm_peak = peaks["hbm_gbs"]
+            extra["decode_16m"] = {
+                "workload": wd.name, "us_per_token": round(dms * 1e3 / wd.B, 3), "ms_per_step": round(dms, 5),
+                "steps": dsteps,
+                "roofline": roofline_entry("decode_scan", prof_dec, scan_bytes, "GB/s", hbm_peak, "hbm",
+                                           f"{peak_kind} hbm_gbs", TRAFFIC_BYTES.get((wd.name, "decode_scan"))),
+                "step_vs_hbm": {"algorithmic_bytes": scan_bytes + gather_bytes,
+                                "achieved_GBs": round((scan_bytes + gather_bytes) / (dms / 1e3) / 1e9, 1),
+                                "frac": round((scan_bytes + gather_bytes) / (dms / 1e3) / 1e9 / hbm_peak, 4)},
+                "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_dec.items()},
+            }
+            if not args.skip_options:  # 4 query tokens per sequence in one step (e.g. verifying 4 drafted tokens)
+                Tq = 4
+                mq = inputs.forward_inputs(wd.B, wd.H, Tq, wd.D, wd.seed + 5, device=dev)[0]
+                mout = torch.empty_like(mq)
+                midx = torch.empty((wd.B, wd.H, Tq, wd.topk), dtype=torch.int32, device=dev)
+                mw = torch.empty((wd.B, wd.H, Tq, wd.topk), dtype=torch.float32, device=dev)
+                mbytes = hsa.hsa_decode_ex_workspace_size(wd.B, wd.H, wd.H, wd.cache_len, wd.D, 64, wd.topk, 0, Tq)
+                mws = torch.empty(mbytes + 256, dtype=torch.uint8, device=dev)
+
+                def dec_multi():
+                    hsa.hsa_decode(mq, Kc, Vc, Lc, lens, wd.topk, out=mout, sel_idx=midx, sel_w=mw, workspace=mws)
+
+                mms = timed(dec_multi, dsteps, args.warmup, world) / dsteps
+                prof_m = kernel_profile(dec_multi, dsteps)
+                extra["decode_16m"]["multi_token_4"] = {
+                    "shape": f"B{wd.B} H{wd.H} Tq{Tq} cache {wd.cache_len} D{wd.D} topk{wd.topk}",
+                    "us_per_step": round(mms * 1e3, 3), "us_per_token": round(mms * 1e3 / (wd.B * Tq), 3),
+                    "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_m.items()}}
+                del mq, mout, mws
+            del q, Kc, Vc, Lc, dws
+            torch.cuda.empty_cache()
+        if not args.skip_options or args.grouped_decode_only:  # 16 query heads on one key/value head
             Hg = 16
             gq = inputs.decode_inputs(wd.B, Hg, 0, wd.D, seed=wd.seed + 3, Tmax=64, device=dev)[0]
             _, gKc, gVc, gLc, glens, _ = inputs.decode_inputs(wd.B, 1, wd.cache_len, wd.D, seed=wd.seed + 4,
@@ -536,7 +539,7 @@ def main():
             gms = timed(dec_gqa, dsteps, args.warmup, world) / dsteps
             prof_gd = kernel_profile(dec_gqa, dsteps)
             lm_bytes = wd.B * (n * wd.D * 2)  # one landmark head, read once from HBM at best
-            extra["decode_16m"]["grouped_heads_16to1"] = {
+            extra.setdefault("decode_16m", {})["grouped_heads_16to1"] = {
                 "shape": f"B{wd.B} H{Hg} Hkv1 cache {wd.cache_len} D{wd.D} topk{wd.topk}",
                 "us_per_token": round(gms * 1e3 / wd.B, 3),
                 "landmark_bytes": lm_bytes,

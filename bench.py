@@ -361,24 +361,61 @@ def main():
                      for k, (c, t) in prof_fwd.items()}
 
         # ---------------- e2e: host buffers through the public API ----------------
+        # Every step copies its inputs from pinned host memory and reads its output back, as an input
+        # pipeline does: step i + 1's inputs go up on one stream while step i computes on the current
+        # stream, and step i's output comes back on a third (inputs and outputs double-buffered on the
+        # device). All the copies of the timed steps are inside the timed region.
         hQ, hK, hV, hL = (x.cpu().pin_memory() for x in (Q, K, V, L))
-        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        dQ_, dK_, dV_, dL_ = (torch.empty_like(x) for x in (Q, K, V, L))
+        hout = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
+        dev_in = [tuple(torch.empty_like(x) for x in (Q, K, V, L)) for _ in range(2)]
+        dev_out = [torch.empty_like(out) for _ in range(2)]
+        s_up, s_down = torch.cuda.Stream(), torch.cuda.Stream()
+        comp = torch.cuda.current_stream()
+        ev_in, ev_used, ev_out, ev_read = ([torch.cuda.Event() for _ in range(2)] for _ in range(4))
 
-        def e2e_step():
-            dQ_.copy_(hQ, non_blocking=True)
-            dK_.copy_(hK, non_blocking=True)
-            dV_.copy_(hV, non_blocking=True)
-            dL_.copy_(hL, non_blocking=True)
-            hsa.hsa_forward(dQ_, dK_, dV_, dL_, w.topk, out=out, sel_idx=sel_idx, sel_w=sel_w, workspace=ws)
-            hout.copy_(out, non_blocking=True)
+        def upload(i):
+            b = i % 2
+            with torch.cuda.stream(s_up):
+                if i >= 2:
+                    s_up.wait_event(ev_used[b])  # step i - 2 is done reading this buffer
+                for d, h in zip(dev_in[b], (hQ, hK, hV, hL)):
+                    d.copy_(h, non_blocking=True)
+                ev_in[b].record(s_up)
 
-        e2e_ms = timed(e2e_step, args.steps, args.warmup, world) / args.steps
+        def e2e_run(n):
+            upload(0)
+            for i in range(n):
+                b = i % 2
+                if i + 1 < n:
+                    upload(i + 1)
+                comp.wait_event(ev_in[b])
+                if i >= 2:
+                    comp.wait_event(ev_read[b])  # step i - 2's output has been read back
+                dq, dk, dv, dl = dev_in[b]
+                hsa.hsa_forward(dq, dk, dv, dl, w.topk, out=dev_out[b], sel_idx=sel_idx, sel_w=sel_w, workspace=ws)
+                ev_used[b].record(comp)
+                ev_out[b].record(comp)
+                with torch.cuda.stream(s_down):
+                    s_down.wait_event(ev_out[b])
+                    hout[b].copy_(dev_out[b], non_blocking=True)
+                    ev_read[b].record(s_down)
+            comp.wait_stream(s_up)
+            comp.wait_stream(s_down)
+
+        e2e_run(args.warmup)
+        barrier(world)
+        t0_ev, t1_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0_ev.record(comp)
+        e2e_run(args.steps)
+        t1_ev.record(comp)
+        barrier(world)
+        e2e_ms = max_over_ranks(t0_ev.elapsed_time(t1_ev), world) / args.steps
         h2d = sum(x.numel() * x.element_size() for x in (hQ, hK, hV, hL))
-        d2h = hout.numel() * hout.element_size()
+        d2h = hout[0].numel() * hout[0].element_size()
         e2e = {"value": whole_job_rate(tokens, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)}
-        del hQ, hK, hV, hL, hout, dQ_, dK_, dV_, dL_
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
+               "pipeline": "inputs of step i+1 uploaded and step i's output read back while step i computes"}
+        del hQ, hK, hV, hL, hout, dev_in, dev_out
 
     extra = {}
     # ---------------- optional paths on the same 32K workload ----------------

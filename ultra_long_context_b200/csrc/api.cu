@@ -296,8 +296,9 @@ static hsa_status decode_impl(const char *name, const hsa_bf16 *qs, const hsa_bf
     a.sel_w = sel_w ? sel_w : l.sel_w;
     a.cand = l.cand; a.counters = l.counters; a.partial = l.partial;
     a.qk_norm = qk_norm;
-    // the decode kernels never wait on one another; the flag is cleared so that a status query
-    // after this call reports this call
+    a.err = l.err;
+    // the flag is cleared so that a status query after this call reports this call (only the grouped
+    // scan has bounded waits, on its own bulk copies)
     cudaError_t ce = cudaMemsetAsync(l.err, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
     if (ce != cudaSuccess) return cuda_status(ce, name);
     return cuda_status(hsa::launch_decode(a, static_cast<cudaStream_t>(stream)), name);

@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "launch.h"
 #include "profile.h"
+#include "tc.cuh"
 
 namespace hsa {
 
@@ -271,83 +272,94 @@ __device__ inline uint64_t warp_merge_desc(uint64_t a, uint64_t b) {
     return m;
 }
 
-// The exact top K (K <= 32) of one head's n scores sc[0..n) (chunks c0 + i), by one warp; lane l < K
-// returns the l-th largest key (0 = empty). Filter: the elements are cut into 64 disjoint groups (lane
-// l, even or odd rounds); if K group maxima are at or above a value, so are K different scores, so the
-// K-th largest group maximum tau is a lower bound of the K-th largest score and nothing below it can be
-// selected. The survivors (and, once K keys are kept, only keys above the K-th kept) are staged in
-// groups of 32, sorted, and merged into the running top 32.
-__device__ inline uint64_t warp_topk_scores(const float *sc, int n, int64_t c0, int K, uint64_t *stage) {
-    const int lane = threadIdx.x & 31;
-    float m0 = -INFINITY, m1 = -INFINITY;
-    for (int r = 0; 32 * r < n; ++r) {
-        const int i = 32 * r + lane;
-        if (i < n) {
-            if (r & 1) m1 = fmaxf(m1, sc[i]);
-            else m0 = fmaxf(m0, sc[i]);
-        }
-    }
-    // tau = the largest group maximum v with at least K group maxima >= v (-inf if none: keep all)
-    int ge0 = 0, ge1 = 0;
-#pragma unroll 8
-    for (int j = 0; j < 32; ++j) {
-        const float x0 = __shfl_sync(0xffffffffu, m0, j), x1 = __shfl_sync(0xffffffffu, m1, j);
-        ge0 += (x0 >= m0 ? 1 : 0) + (x1 >= m0 ? 1 : 0);
-        ge1 += (x0 >= m1 ? 1 : 0) + (x1 >= m1 ? 1 : 0);
-    }
-    float tau = fmaxf(ge0 >= K ? m0 : -INFINITY, ge1 >= K ? m1 : -INFINITY);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) tau = fmaxf(tau, __shfl_xor_sync(0xffffffffu, tau, o));
-    // thr: tau, raised to the K-th kept score once K keys are kept; a score equal to it can still win on
-    // the lower chunk index, so the float test keeps ties and the merge decides on the full key
+// Running exact top K (K <= 32) of one row's scores, kept by one warp across the sub-blocks of a range:
+// lane l < K holds the l-th largest key so far (0 = empty). A score at or above the current K-th kept
+// score (ties included: the lower chunk may still win on the key) is staged; every 32 staged keys are
+// sorted and merged in, and the threshold rises with the K-th kept key.
+struct WarpTopK {
     uint64_t best = 0ull;
-    float thr = tau;
+    float thr = -INFINITY;
     int ns = 0;  // staged keys (warp-uniform)
-    for (int r = 0; r < n; r += 32) {
-        const int i = r + lane;
-        const bool cand = i < n && sc[i] >= thr;
-        const unsigned bal = __ballot_sync(0xffffffffu, cand);
-        if (bal == 0u) continue;
-        if (cand) stage[ns + __popc(bal & ((1u << lane) - 1u))] = make_key(sc[i], (uint32_t)(c0 + i));
-        ns += __popc(bal);
-        __syncwarp();
-        if (ns >= 32) {
-            best = warp_merge_desc(best, warp_sort_desc(stage[lane]));
-            const uint64_t rest = lane + 32 < ns ? stage[lane + 32] : 0ull;
+
+    __device__ void feed(const float *sc, int n, int64_t c0, int K, uint64_t *stage) {
+        const int lane = threadIdx.x & 31;
+        for (int r = 0; r < n; r += 32) {
+            const int i = r + lane;
+            const bool cand = i < n && sc[i] >= thr;
+            const unsigned bal = __ballot_sync(0xffffffffu, cand);
+            if (bal == 0u) continue;
+            if (cand) stage[ns + __popc(bal & ((1u << lane) - 1u))] = make_key(sc[i], (uint32_t)(c0 + i));
+            ns += __popc(bal);
             __syncwarp();
-            if (lane + 32 < ns) stage[lane] = rest;
-            __syncwarp();
-            ns -= 32;
-            const uint64_t kth = __shfl_sync(0xffffffffu, best, K - 1);  // 0 until K keys are kept
-            if (kth != 0ull) thr = fmaxf(thr, key_score(kth));
+            if (ns >= 32) {
+                best = warp_merge_desc(best, warp_sort_desc(stage[lane]));
+                const uint64_t rest = lane + 32 < ns ? stage[lane + 32] : 0ull;
+                __syncwarp();
+                if (lane + 32 < ns) stage[lane] = rest;
+                __syncwarp();
+                ns -= 32;
+                const uint64_t kth = __shfl_sync(0xffffffffu, best, K - 1);  // 0 until K keys are kept
+                if (kth != 0ull) thr = fmaxf(thr, key_score(kth));
+            }
         }
     }
-    if (ns > 0) best = warp_merge_desc(best, warp_sort_desc(lane < ns ? stage[lane] : 0ull));
-    return lane < K ? best : 0ull;
-}
+    __device__ uint64_t finish(int K, const uint64_t *stage) {
+        const int lane = threadIdx.x & 31;
+        if (ns > 0) best = warp_merge_desc(best, warp_sort_desc(lane < ns ? stage[lane] : 0ull));
+        ns = 0;
+        return lane < K ? best : 0ull;
+    }
+};
+
+constexpr int kDecodeGroupThreads = 768;  // warps 0-7 score the sub-blocks, warps 8-23 select (one row each)
+constexpr int kGsScorers = 8;
+constexpr int kGsSelectors = 16;
+constexpr int kGsSub = 128;                // landmarks per sub-block (one bulk copy)
+constexpr int kGsStages = 4;               // sub-blocks in flight
+constexpr int kGsBufs = 4;                 // score buffers: the scorers may run this many sub-blocks ahead
+
+template <int D>
+struct GsSmem {
+    static constexpr uint32_t STAGE = kGsSub * D * 2;                 // bf16 rows, 64-column boxes, 128 B swizzle
+    static constexpr uint32_t SC = kGsStages * STAGE;                       // [kGsBufs][16][kGsSub + 8] fp32
+    static constexpr uint32_t STG = SC + kGsBufs * 16 * (kGsSub + 8) * 4;   // [16 rows][64] staged keys
+    // full[kGsStages] (copies landed), empty[kGsStages] (scorers read them), ready / free[kGsBufs] (scores)
+    static constexpr uint32_t BAR = STG + 16 * 64 * 8;
+    static constexpr uint32_t BYTES = BAR + (2 * kGsStages + 2 * kGsBufs) * 8;
+    static constexpr size_t DYN = BYTES + 1024;                       // + alignment of the stages
+};
 
 // grid (nsplit, B*Hkv, ceil(R / 16)): the landmark range sp of key head kvh, for 16 of its R = Gh * Tq
 // query rows (Gh query heads, Tq query tokens each; row r = g * Tq + i is token i of head g, and the
 // rows of a key head are consecutive in q). Token i sits at position cache_len - Tq + i and sees the
-// chunks that have ended at or before it. The scores of a tile of 8 landmarks for the 16 rows are one
-// m16n8k16 tensor-core product per 16 columns of D (M = 16 is below the tcgen05 tile, so the
-// warp-level MMA). The reduction index is
-// permuted the same way in both operands, so that each lane loads whole 16-byte chunks: lane (g, t4)
-// holds columns 32 s + 8 t4 .. + 7 of head rows g, g + 8 and of landmark g of the tile, and k-steps
-// 2 s, 2 s + 1 take the first and the second half of that chunk.
-constexpr int kDecodeGroupThreads = 512;  // one CTA per SM: 16 warps stream, then one head per warp selects
-
+// chunks that have ended at or before it.
+// The range streams through shared memory in sub-blocks of 128 landmarks by bulk tensor copies (four in
+// flight, so no register holds a load). Scorer warps turn each sub-block into scores: the scores of a
+// tile of 8 landmarks for the 16 rows are one m16n8k16 tensor-core product per 16 columns of D (M = 16
+// is below the tcgen05 tile, so the warp-level MMA). The reduction index is permuted alike in both
+// operands so that each lane reads whole 16-byte chunks: lane (g, t4) takes columns 32 s + 8 t4 .. + 7
+// of head rows g, g + 8 and of landmark g of the tile, and k-steps 2 s, 2 s + 1 take the two halves of
+// that chunk. Selector warps (one per row) fold each sub-block's scores into the rows' running top K
+// while the scorers work on the next ones (kGsBufs score buffers; mbarriers hand them over, every
+// wait bounded).
 template <int D>
 __global__ void __launch_bounds__(kDecodeGroupThreads, 1) decode_scan_group_kernel(
-    const uint16_t *__restrict__ q, const uint16_t *__restrict__ Lc, const int64_t *__restrict__ cache_len, int Hkv,
-    int R, int Tq, int64_t Nmax, int split, int nsplit, int K, float scale, uint64_t *__restrict__ cand) {
-    constexpr int S = D / 32;      // 16-byte chunks per lane per row
-    constexpr int NWARP = kDecodeGroupThreads / 32;
-    constexpr int U = 4;           // landmark tiles in flight per warp
+    const uint16_t *__restrict__ q, const __grid_constant__ CUtensorMap tmL, const int64_t *__restrict__ cache_len,
+    int Hkv, int R, int Tq, int64_t Nmax, int split, int nsplit, int K, float scale, uint64_t *__restrict__ cand,
+    int32_t *__restrict__ err) {
+    using SM = GsSmem<D>;
+    constexpr int S = D / 32;  // 16-byte chunks per lane per row
+    constexpr int LD = kGsSub + 8;  // score row stride (fewer bank conflicts on the fragment stores)
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    const int ld = split + 8;      // score row stride (fewer bank conflicts on the fragment stores)
-    float *sc = reinterpret_cast<float *>(smem_raw);                             // [16][ld]
-    uint64_t *stage = reinterpret_cast<uint64_t *>(smem_raw + (size_t)16 * ld * sizeof(float));  // [NWARP][64]
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sb = (raw + 1023u) & ~1023u;
+    unsigned char *smem = smem_raw + (sb - raw);
+    float *sc = reinterpret_cast<float *>(smem + SM::SC);
+    uint64_t *stage = reinterpret_cast<uint64_t *>(smem + SM::STG);
+    auto full = [&](int st) { return sb + SM::BAR + 8u * st; };
+    auto empty = [&](int st) { return sb + SM::BAR + 8u * (kGsStages + st); };
+    auto ready = [&](int bf) { return sb + SM::BAR + 8u * (2 * kGsStages + bf); };
+    auto freeb = [&](int bf) { return sb + SM::BAR + 8u * (2 * kGsStages + kGsBufs + bf); };
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t4 = lane & 3;
@@ -362,58 +374,121 @@ __global__ void __launch_bounds__(kDecodeGroupThreads, 1) decode_scan_group_kern
     const int64_t c0 = (int64_t)sp * split;
     const int64_t c1 = min(c0 + (int64_t)split, nb);
     const int nloc = c1 > c0 ? (int)(c1 - c0) : 0;
+    const int nsub = (nloc + kGsSub - 1) / kGsSub;
     const size_t q0 = (size_t)kvh * R + r0;  // q row of this CTA's first row
 
-    uint32_t a[S][2][4];
-#pragma unroll
-    for (int s = 0; s < S; ++s) {
-        const uint4 qa = g < rows ? *reinterpret_cast<const uint4 *>(q + (q0 + g) * D + 32 * s + 8 * t4)
-                                  : make_uint4(0u, 0u, 0u, 0u);
-        const uint4 qb = g + 8 < rows ? *reinterpret_cast<const uint4 *>(q + (q0 + g + 8) * D + 32 * s + 8 * t4)
-                                      : make_uint4(0u, 0u, 0u, 0u);
-        a[s][0][0] = qa.x; a[s][0][1] = qb.x; a[s][0][2] = qa.y; a[s][0][3] = qb.y;
-        a[s][1][0] = qa.z; a[s][1][1] = qb.z; a[s][1][2] = qa.w; a[s][1][3] = qb.w;
-    }
-    const uint16_t *Lh = Lc + (size_t)kvh * Nmax * D;
-    const int ntile = (nloc + 7) / 8;
-    for (int t0 = warp; t0 < ntile; t0 += NWARP * U) {
-        uint4 v[U][S];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int tile = t0 + u * NWARP;
-            const int i = tile * 8 + g;
-#pragma unroll
-            for (int s = 0; s < S; ++s)
-                v[u][s] = (tile < ntile && i < nloc) ? ld_stream16(Lh + (c0 + i) * D + 32 * s + 8 * t4)
-                                                     : make_uint4(0u, 0u, 0u, 0u);
+    if (tid == 0) {
+        for (int st = 0; st < kGsStages; ++st) {
+            tc::mbar_init(full(st), 1);
+            tc::mbar_init(empty(st), kGsScorers);
         }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int tile = t0 + u * NWARP;  // warp-uniform
-            if (tile >= ntile) break;
-            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-            for (int s = 0; s < S; ++s) {
-                mma_bf16_16816(acc, a[s][0], v[u][s].x, v[u][s].y);
-                mma_bf16_16816(acc, a[s][1], v[u][s].z, v[u][s].w);
-            }
-            const int i0 = tile * 8 + 2 * t4;  // acc: heads g (0, 1) and g + 8 (2, 3), landmarks i0, i0 + 1
-            if (g < rows) {
-                if (i0 < nloc) sc[g * ld + i0] = acc[0] * scale;
-                if (i0 + 1 < nloc) sc[g * ld + i0 + 1] = acc[1] * scale;
-            }
-            if (g + 8 < rows) {
-                if (i0 < nloc) sc[(g + 8) * ld + i0] = acc[2] * scale;
-                if (i0 + 1 < nloc) sc[(g + 8) * ld + i0 + 1] = acc[3] * scale;
-            }
+        for (int bf = 0; bf < kGsBufs; ++bf) {
+            tc::mbar_init(ready(bf), kGsScorers);
+            tc::mbar_init(freeb(bf), kGsSelectors);
         }
+        tc::fence_mbar_init();
     }
     __syncthreads();
-    for (int h = warp; h < rows; h += NWARP) {  // one row per warp; the row's own causal limit
-        const int64_t cr = min(c1, n_of(r0 + h));
-        const int nr = cr > c0 ? (int)(cr - c0) : 0;
-        const uint64_t best = warp_topk_scores(sc + h * ld, nr, c0, K, stage + warp * 64);
-        if (lane < K) cand[((q0 + h) * nsplit + sp) * K + lane] = best;
+    auto load = [&](int i) {  // sub-block i into stage i % kGsStages
+        const int st = i % kGsStages;
+        tc::mbar_arrive_expect_tx(full(st), SM::STAGE);
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+            tc::tma_load_2d(sb + st * SM::STAGE + h * kGsSub * 128, &tmL, h * 64,
+                            (int)(kvh * Nmax + c0 + (int64_t)i * kGsSub), full(st));
+    };
+    int issued = 0;
+    if (tid == 0)
+        for (; issued < kGsStages && issued < nsub; ++issued) load(issued);
+    bool ok = true;
+
+    if (warp < kGsScorers) {
+        // ---------------- scorers ----------------
+        uint32_t a[S][2][4];
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            const uint4 qa = g < rows ? *reinterpret_cast<const uint4 *>(q + (q0 + g) * D + 32 * s + 8 * t4)
+                                      : make_uint4(0u, 0u, 0u, 0u);
+            const uint4 qb = g + 8 < rows ? *reinterpret_cast<const uint4 *>(q + (q0 + g + 8) * D + 32 * s + 8 * t4)
+                                          : make_uint4(0u, 0u, 0u, 0u);
+            a[s][0][0] = qa.x; a[s][0][1] = qb.x; a[s][0][2] = qa.y; a[s][0][3] = qb.y;
+            a[s][1][0] = qa.z; a[s][1][1] = qb.z; a[s][1][2] = qa.w; a[s][1][3] = qb.w;
+        }
+        for (int i = 0; i < nsub && ok; ++i) {
+            const int st = i % kGsStages, bf = i % kGsBufs;
+            ok = __all_sync(0xffffffffu,
+                            tc::mbar_wait(full(st), (uint32_t)(i / kGsStages) & 1u) &&
+                                (i < kGsBufs || tc::mbar_wait(freeb(bf), (uint32_t)((i / kGsBufs) - 1) & 1u)));
+            if (!ok) break;  // (the scores of sub-block i - kGsBufs have been consumed)
+            const int nt = min(kGsSub, nloc - i * kGsSub);
+            const uint32_t stg = sb + st * SM::STAGE;
+            float *scb = sc + bf * 16 * LD;  // buffer bf
+            for (int tile = warp; tile * 8 < nt; tile += kGsScorers) {
+                float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                for (int s = 0; s < S; ++s) {
+                    const int jj = (4 * s + t4) & 7;  // 16-byte chunk within the 64-column box
+                    uint4 v;
+                    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                 : "r"(stg + ((4 * s + t4) >> 3) * kGsSub * 128 + tc::sw128(tile * 8 + g, jj)));
+                    mma_bf16_16816(acc, a[s][0], v.x, v.y);
+                    mma_bf16_16816(acc, a[s][1], v.z, v.w);
+                }
+                const int i0 = tile * 8 + 2 * t4;  // acc: rows g (0, 1) and g + 8 (2, 3), landmarks i0, i0 + 1
+                if (g < rows) {
+                    if (i0 < nt) scb[g * LD + i0] = acc[0] * scale;
+                    if (i0 + 1 < nt) scb[g * LD + i0 + 1] = acc[1] * scale;
+                }
+                if (g + 8 < rows) {
+                    if (i0 < nt) scb[(g + 8) * LD + i0] = acc[2] * scale;
+                    if (i0 + 1 < nt) scb[(g + 8) * LD + i0 + 1] = acc[3] * scale;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(ready(bf));  // this warp's scores of sub-block i are written
+                tc::mbar_arrive(empty(st));  // and its reads of the stage are done
+            }
+            if (warp == 0) {  // refill the stage once every scorer has read it (lane 0; the warp waits)
+                bool w_ok = true;
+                if (lane == 0 && issued < nsub) {
+                    w_ok = tc::mbar_wait(empty(st), (uint32_t)(i / kGsStages) & 1u);
+                    if (w_ok) {
+                        tc::fence_proxy_async_smem();
+                        load(issued++);
+                    }
+                }
+                ok = __all_sync(0xffffffffu, w_ok);
+                if (!ok) break;
+            }
+        }
+    } else {
+        // ---------------- selectors: one row each ----------------
+        const int r = warp - kGsScorers;
+        WarpTopK sel;
+        const int64_t lim = r < rows ? min(c1, n_of(r0 + r)) : c0;
+        for (int i = 0; i < nsub && ok; ++i) {
+            const int bf = i % kGsBufs;
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(ready(bf), (uint32_t)(i / kGsBufs) & 1u));
+            if (!ok) break;
+            const int nt = min(kGsSub, nloc - i * kGsSub);
+            const int64_t base = c0 + (int64_t)i * kGsSub;
+            const int64_t nr = min((int64_t)nt, lim - base);
+            if (nr > 0) sel.feed(sc + (bf * 16 + r) * LD, (int)nr, base, K, stage + r * 64);  // buffer bf
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(freeb(bf));
+        }
+        if (r < rows) {
+            const uint64_t best = sel.finish(K, stage + r * 64);
+            if (lane < K) cand[((q0 + r) * nsplit + sp) * K + lane] = best;
+        }
+    }
+    if (!ok) {  // a wait ran out: report it, and wait (bounded) for the copies this CTA issued
+        if (err && lane == 0) atomicOr(err, 1);
+        if (tid == 0)
+            for (int i = issued > kGsStages ? issued - kGsStages : 0; i < issued; ++i)
+                tc::mbar_wait(full(i % kGsStages), (uint32_t)(i / kGsStages) & 1u);
     }
 }
 
@@ -578,12 +653,6 @@ size_t decode_scan_smem(int split, int nsplit, int K) {
     return (cap + 128) * sizeof(uint64_t) + 256 * sizeof(uint32_t) + 8 * sizeof(int);
 }
 
-// Grouped scan: scores of 16 head rows per landmark (fp32, row stride split + 8) plus the warps'
-// staging and merge buffers.
-static size_t decode_group_smem(int split) {
-    return (size_t)16 * (split + 8) * sizeof(float) + (size_t)(kDecodeGroupThreads / 32) * 64 * sizeof(uint64_t);
-}
-constexpr int kDecodeGroupMaxSplit = 3072;
 
 DecodePlan decode_plan(int64_t Nmax, int K, int B, int H, int Hkv, int Tq) {
     DecodePlan p{};
@@ -605,17 +674,12 @@ DecodePlan decode_plan(int64_t Nmax, int K, int B, int H, int Hkv, int Tq) {
         ns = ns < by_min ? ns : by_min;
         const int64_t cap = (8192 / K < 512) ? 8192 / K : 512;
         ns = ns < cap ? ns : cap;
-        // ranges longer than the shared-memory score rows hold: more ranges (several waves), up to the cap
-        const int64_t by_smem = (Nmax + kDecodeGroupMaxSplit - 1) / kDecodeGroupMaxSplit;
-        if (ns < by_smem) ns = by_smem < cap ? by_smem : cap;
         int64_t split = (Nmax + ns - 1) / ns;
-        split = (split + 63) / 64 * 64;
-        if (split <= kDecodeGroupMaxSplit) {
-            p.grouped = true;
-            p.split = (int)split;
-            p.nsplit = (int)((Nmax + split - 1) / split);
-            return p;
-        }
+        split = (split + kGsSub - 1) / kGsSub * kGsSub;  // whole sub-blocks
+        p.grouped = true;
+        p.split = (int)split;
+        p.nsplit = (int)((Nmax + split - 1) / split);
+        return p;
     }
     p.split = decode_split_size(Nmax, K, B * H);
     const int64_t ns = (Nmax + p.split - 1) / p.split;
@@ -626,7 +690,7 @@ DecodePlan decode_plan(int64_t Nmax, int K, int B, int H, int Hkv, int Tq) {
 size_t decode_plan_smem(const DecodePlan &p, int K) {
     if (!p.grouped) return decode_scan_smem(p.split, p.nsplit, K);
     const size_t merge = ((size_t)p.nsplit * K + 128) * sizeof(uint64_t) + 256 * sizeof(uint32_t) + 8 * sizeof(int);
-    const size_t scan = decode_group_smem(p.split);
+    const size_t scan = GsSmem<128>::DYN;
     return merge > scan ? merge : scan;
 }
 
@@ -653,14 +717,18 @@ static cudaError_t launch_attend(const DecodeArgs &a, dim3 grid, cudaStream_t s)
 template <int D>
 static cudaError_t launch_decode_grouped(const DecodeArgs &a, const DecodePlan &pl, cudaStream_t s) {
     const int R = a.H / a.Hkv * a.Tq, rows_q = a.B * a.H * a.Tq;
-    const size_t gsmem = decode_group_smem(pl.split);
+    const size_t gsmem = GsSmem<D>::DYN;
     cudaError_t e = cudaFuncSetAttribute(decode_scan_group_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)gsmem);
     if (e != cudaSuccess) return e;
+    CUtensorMap tm;  // landmark rows [B*Hkv*Nmax, D]; boxes of kGsSub rows (with no chunk: never read)
+    const uint64_t lrows = (uint64_t)a.B * a.Hkv * a.Nmax;
+    if (!make_tmap_bf16(&tm, lrows > 0 ? (const void *)a.Lc : (const void *)a.q, lrows > 0 ? lrows : 1, D, kGsSub))
+        return cudaErrorInvalidValue;
     {
         HSA_PROF("decode_scan", s);
         decode_scan_group_kernel<D><<<dim3(pl.nsplit, a.B * a.Hkv, pl.row_groups), kDecodeGroupThreads, gsmem, s>>>(
-            a.qs, a.Lc, a.cache_len, a.Hkv, R, a.Tq, a.Nmax, pl.split, pl.nsplit, a.K, a.scale, a.cand);
+            a.qs, tm, a.cache_len, a.Hkv, R, a.Tq, a.Nmax, pl.split, pl.nsplit, a.K, a.scale, a.cand, a.err);
         e = cudaGetLastError();
     }
     if (e != cudaSuccess) return e;

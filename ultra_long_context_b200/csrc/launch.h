@@ -25,6 +25,7 @@ struct DecodeArgs {
     unsigned *counters;  // [2, B*H*Tq]
     float *partial;    // [B*H*Tq, K, D]
     bool qk_norm;      // Step 3 attends with q / max(|q|, eps) and k / max(|k|, eps)
+    int32_t *err;      // [1] or NULL: set when a bounded device wait ran out (grouped scan)
 };
 int decode_split_size(int64_t Nmax, int K, int BH);
 size_t decode_scan_smem(int split, int nsplit, int K);

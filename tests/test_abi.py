@@ -153,3 +153,40 @@ def test_ex_workspace_sizes_cover_the_options():
         hsa.hsa_backward_workspace_size(1, 4, 4096, 128, 64, 16) + 4 * 4096 * 16 * 4  # ds per pair
     assert hsa.hsa_decode_ex_workspace_size(1, 8, 8, 1 << 20, 128, 64, 32, 1) == \
         hsa.hsa_decode_workspace_size(1, 8, 1 << 20, 128, 64, 32)
+
+
+def _fwd_varlen(**kw):
+    args = dict(Qs=None, Q=FAKE, K=FAKE, V=FAKE, L=FAKE, cu=FAKE, B=3, max_seqlen=1000, H=4, Hkv=2, D=128, chunk=64,
+                topk=8, scale=0.0, flags=0, out=FAKE, sel_idx=FAKE, sel_w=FAKE, ws=FAKE, ws_bytes=1 << 40, stream=None)
+    args.update(kw)
+    return hsa.lib().hsa_forward_varlen(*args.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(cu=None), -1), (dict(cu=ctypes.c_void_p((1 << 20) + 2)), -1), (dict(max_seqlen=0), -1), (dict(B=0), -1),
+    (dict(Hkv=3), -1), (dict(flags=2), -1), (dict(out=None), -1), (dict(sel_w=None), -1), (dict(Q=ODD), -1),
+    (dict(D=96), -2), (dict(topk=33), -2), (dict(ws_bytes=64), -3), (dict(ws=None), -3),
+])
+def test_forward_varlen_rejects_invalid_calls_on_host(kw, status):
+    assert _fwd_varlen(**kw) == status
+    assert hsa.hsa_last_error() != ""
+
+
+def test_backward_varlen_rejects_invalid_calls_on_host():
+    args = dict(Qs=None, Q=FAKE, K=FAKE, V=FAKE, L=FAKE, out=FAKE, dout=FAKE, sel_idx=FAKE, sel_w=FAKE, cu=FAKE, B=2,
+                max_seqlen=500, H=2, Hkv=2, D=64, chunk=64, topk=8, scale=0.0, flags=0, dQ=FAKE, dK=FAKE, dV=FAKE,
+                dL=FAKE, dQs=None, ws=FAKE, ws_bytes=1 << 40, stream=None)
+    for kw, status in ((dict(dQs=FAKE), -1), (dict(Qs=FAKE), -1), (dict(dL=None), -1), (dict(cu=None), -1),
+                       (dict(ws_bytes=16), -3)):
+        a = dict(args, **kw)
+        assert hsa.lib().hsa_backward_varlen(*a.values()) == status, kw
+
+
+def test_varlen_workspace_covers_the_padded_batch():
+    B, H, Hkv, T, D, K = 3, 4, 2, 1000, 128, 8
+    padded = B * H * T * D * 2  # one padded bf16 query batch
+    assert hsa.lib().hsa_forward_varlen_workspace_size(B, H, Hkv, T, D, 64, K, 0) >= \
+        hsa.hsa_forward_workspace_size(B, H, T, D, 64, K) + 3 * padded
+    assert hsa.lib().hsa_backward_varlen_workspace_size(B, H, Hkv, T, D, 64, K, 0) > \
+        hsa.lib().hsa_forward_varlen_workspace_size(B, H, Hkv, T, D, 64, K, 0)
+    assert hsa.lib().hsa_forward_varlen_workspace_size(B, H, 3, T, D, 64, K, 0) == 0  # H not a multiple of Hkv

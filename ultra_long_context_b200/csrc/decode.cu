@@ -138,7 +138,7 @@ __device__ void merge_ranges(const uint64_t *all, int nsplit, int K, uint64_t *k
 }
 
 template <int D>
-__global__ void __launch_bounds__(kDecodeThreads) decode_scan_kernel(
+__global__ void __launch_bounds__(kDecodeThreads, 4) decode_scan_kernel(
     const uint16_t *__restrict__ q, const uint16_t *__restrict__ Lc, const int64_t *__restrict__ cache_len, int H,
     int Gh, int64_t Nmax, int split, int nsplit, int K, float scale, uint64_t *__restrict__ cand, unsigned *counters,
     int32_t *__restrict__ sel_idx, float *__restrict__ sel_w) {
@@ -630,7 +630,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_attend_kernel(
 
 // Landmarks per scan range. The scan is HBM-bound and every range costs the same, so the ranges are
 // sized for a single wave of CTAs: B*H*ranges <= kDecodeWaveCtas (148 SMs x 4 resident CTAs of
-// 256 threads at the kernel's register count). A range keeps at least 256 landmarks and at most
+// 256 threads: the scan's launch bound holds it to 64 registers, without spills). A range keeps at least 256 landmarks and at most
 // 6144 (its keys live in shared memory), and ranges*K <= 8192 (the merge holds all candidates).
 constexpr int64_t kDecodeSms = 148;
 constexpr int64_t kDecodeWaveCtas = kDecodeSms * 4;

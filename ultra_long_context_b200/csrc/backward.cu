@@ -13,7 +13,9 @@
 // The pairs are processed chunk-major with the same dispatch as the forward (tiles of <= 64 pairs
 // of one chunk): the chunk's K, V and the tile's gathered Q, dO rows sit in shared memory, the five
 // contractions run on the tensor cores, and every gradient is accumulated with fp32 vector
-// reductions (a chunk may span several tiles, a token several chunks).
+// reductions (a chunk may span several tiles, a token several chunks). This file holds the delta
+// kernel, the head-dim-64 chunk kernel (mma.sync; head dim 128 runs bwd_tc.cu), the query-gradient
+// finish for a separate retrieval query or query-key normalisation, and the launch sequence.
 #include "common.cuh"
 #include "launch.h"
 #include "profile.h"

@@ -10,8 +10,15 @@
 //                          range (block radix select on unique 64-bit keys), writes K candidates.
 //                          The last CTA of each (b, h) to finish (atomic ticket, no waiting) merges
 //                          the candidates of all ranges exactly and writes sel_idx / sel_w.
-//   decode_attend_kernel   grid (K, B*H). One CTA per selected chunk: 64 logits, softmax, P.V_c;
-//                          the last CTA of each (b, h) blends the K chunk outputs and writes out.
+//   decode_attend_kernel   grid (K, B*H*Tq). One CTA per selected chunk: 64 logits, softmax, P.V_c;
+//                          the last CTA of each query row blends the K chunk outputs and writes out.
+//
+// When several query rows read the same landmarks (grouped key/value heads, several query tokens per
+// step) and K <= 32, the scan is the grouped one instead:
+//   decode_scan_group_kernel  grid (ranges, B*Hkv, row groups of 16). Bulk-copied landmark sub-blocks,
+//                          tensor-core scores for 16 rows at a time, one selector warp per row keeping
+//                          a running exact top K; writes K candidates per row and range.
+//   decode_merge_kernel    grid (B*H*Tq). The exact merge of one row's range candidates.
 #include "common.cuh"
 #include "launch.h"
 #include "profile.h"

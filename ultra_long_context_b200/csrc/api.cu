@@ -93,13 +93,14 @@ FwdLayout fwd_layout(void *ws, int B, int H, int T, int D, int topk, bool backwa
     l.err = c.take<int32_t>(1);  // first: hsa_workspace_status reads it at offset 0
     const size_t rows = (size_t)B * H * T, chunks = (size_t)B * H * (T / 64), pairs = rows * topk;
     l.max_tiles = (int)hsa::forward_max_tiles(B, H, T, topk);
+    // right after the error flag: the three are zeroed by one memset
+    l.chunk_count = c.take<int32_t>(chunks);
+    l.chunk_cursor = c.take<int32_t>(chunks);
     l.o_acc = backward ? nullptr : c.take<float>(rows * D);
     l.sel_idx = backward ? nullptr : c.take<int32_t>(pairs);
     l.sel_w = backward ? nullptr : c.take<float>(pairs);
-    l.chunk_count = c.take<int32_t>(chunks);
     l.chunk_off = c.take<int32_t>(chunks + 1);
     l.tile_off = c.take<int32_t>(chunks + 1);
-    l.chunk_cursor = c.take<int32_t>(chunks);
     l.pair_row = c.take<int32_t>(pairs);
     l.pair_w = c.take<float>(pairs);
     l.tiles = c.take<hsa::PairTile>((size_t)l.max_tiles);

@@ -411,9 +411,7 @@ cudaError_t launch_backward(const BackwardArgs &a0, cudaStream_t s) {
         if (e == cudaSuccess) e = cudaMemsetAsync(a.dV, 0, kv_rows * a.D * sizeof(float), s);
         if (e == cudaSuccess && a.N > 0)
             e = cudaMemsetAsync(a.dL, 0, (size_t)a.B * a.Hkv * a.N * a.D * sizeof(float), s);
-        if (e == cudaSuccess && a.N > 0) e = cudaMemsetAsync(a.chunk_count, 0, chunks * sizeof(int32_t), s);
-        if (e == cudaSuccess && a.N > 0) e = cudaMemsetAsync(a.chunk_cursor, 0, chunks * sizeof(int32_t), s);
-        if (e == cudaSuccess && a.err) e = cudaMemsetAsync(a.err, 0, sizeof(int32_t), s);
+        if (e == cudaSuccess) e = zero_dispatch_state(a.err, a.chunk_count, a.chunk_cursor, a.N > 0 ? chunks : 0, s);
         // with chunks, dq_finish_kernel writes every row of dQs
         if (e == cudaSuccess && a.dQs && a.N == 0) e = cudaMemsetAsync(a.dQs, 0, rows * a.D * sizeof(float), s);
     }

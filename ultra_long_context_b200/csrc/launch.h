@@ -89,6 +89,11 @@ cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s);
 // tile work list, and the (token row, weight[, slot]) pair arrays. The lists are per query head even
 // when query heads share key heads: a tile's pairs then all write accumulator rows of one query head,
 // which keeps the rows that the concurrent tiles reduce into within L2.
+// Zeroes the error flag and the dispatch's chunk counts and cursors: one memset when the workspace
+// holds them in that order with at most alignment padding between them, else three.
+cudaError_t zero_dispatch_state(int32_t *err, int32_t *chunk_count, int32_t *chunk_cursor, size_t chunks,
+                                cudaStream_t s);
+
 cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, int H, int T, int N, int topk,
                             int32_t *chunk_count, int32_t *chunk_off, int32_t *tile_off, int32_t *chunk_cursor,
                             int32_t *pair_row,

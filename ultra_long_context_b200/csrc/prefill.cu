@@ -35,12 +35,21 @@ __global__ void __launch_bounds__(kDispatchRows) count_kernel(const int32_t *__r
         for (int i = threadIdx.x; i < N; i += blockDim.x) s_hist[i] = 0;
         __syncthreads();
     }
-    const int t = blockIdx.x * kDispatchRows + threadIdx.x;
-    if (t < T) {
-        const int32_t *si = sel_idx + ((size_t)bh * T + t) * K;
-        for (int j = 0; j < K; ++j) {
-            const int c = si[j];
-            if (c < 0 || c >= N) continue;  // -1 = empty slot; ids past N are ignored
+    // the block's rows are contiguous in [B, H, T, K]: one flat, coalesced range of entries
+    const int t0 = blockIdx.x * kDispatchRows;
+    const int nent = max(0, min(kDispatchRows, T - t0)) * K;
+    const int32_t *si = sel_idx + ((size_t)bh * T + t0) * K;
+    for (int eb = 0; eb < nent; eb += 8 * kDispatchRows) {  // 8 loads in flight per thread
+        int cb[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int e = eb + k * kDispatchRows + threadIdx.x;
+            cb[k] = e < nent ? si[e] : -1;
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int c = cb[k];
+            if (c < 0 || c >= N) continue;  // -1 = empty slot (or past the block's rows); ids past N are ignored
             if (use_smem) atomicAdd(&s_hist[c], 1);
             else atomicAdd(&chunk_count[(size_t)bh * N + c], 1);
         }
@@ -81,33 +90,65 @@ __device__ inline int block_exclusive_scan(int v, int *s_warp, int &total) {
     return res;
 }
 
-// One CTA: exclusive offsets of every chunk's pair list and of its tiles (<= kPairTile pairs each).
+// One CTA: exclusive offsets of every chunk's pair list and of its tiles (<= tp pairs each). Rounds
+// of 8192 counts, 8 contiguous ones per thread loaded and stored as vectors where they are whole (the
+// tables are 256-byte aligned), each round's block scan carried into the next.
+constexpr int kScanPer = 8;
+
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t *__restrict__ chunk_count, int M,
                                                     int32_t *__restrict__ chunk_off, int32_t *__restrict__ tile_off,
                                                     int32_t *__restrict__ num_tiles, int max_tiles, int tp) {
     __shared__ int s_warp[33];
-    const int per = (M + blockDim.x - 1) / blockDim.x;
-    const int lo = min(M, (int)threadIdx.x * per), hi = min(M, lo + per);
-    int sum = 0, tsum = 0;
-    for (int i = lo; i < hi; ++i) {
-        const int c = chunk_count[i];
-        sum += c;
-        tsum += (c + tp - 1) / tp;
-    }
-    int total, ttotal;
-    int off = block_exclusive_scan(sum, s_warp, total);
-    int toff = block_exclusive_scan(tsum, s_warp, ttotal);
-    for (int i = lo; i < hi; ++i) {
-        const int c = chunk_count[i];
-        chunk_off[i] = off;
-        tile_off[i] = toff;
-        off += c;
-        toff += (c + tp - 1) / tp;
+    int carry = 0, tcarry = 0;
+    for (int base = 0; base < M; base += (int)blockDim.x * kScanPer) {
+        const int lo = base + (int)threadIdx.x * kScanPer;
+        int c[kScanPer];
+        if (lo + kScanPer <= M) {  // lo is a multiple of 8 ints: 32-byte aligned in the 256-aligned table
+            const int4 a = reinterpret_cast<const int4 *>(chunk_count + lo)[0];
+            const int4 b = reinterpret_cast<const int4 *>(chunk_count + lo)[1];
+            c[0] = a.x; c[1] = a.y; c[2] = a.z; c[3] = a.w;
+            c[4] = b.x; c[5] = b.y; c[6] = b.z; c[7] = b.w;
+        } else {
+#pragma unroll
+            for (int k = 0; k < kScanPer; ++k) c[k] = lo + k < M ? chunk_count[lo + k] : 0;
+        }
+        int sum = 0, tsum = 0;
+#pragma unroll
+        for (int k = 0; k < kScanPer; ++k) {
+            sum += c[k];
+            tsum += (c[k] + tp - 1) / tp;
+        }
+        int total, ttotal;
+        int off = block_exclusive_scan(sum, s_warp, total) + carry;
+        int toff = block_exclusive_scan(tsum, s_warp, ttotal) + tcarry;
+        int o[kScanPer], to[kScanPer];
+#pragma unroll
+        for (int k = 0; k < kScanPer; ++k) {
+            o[k] = off;
+            to[k] = toff;
+            off += c[k];
+            toff += (c[k] + tp - 1) / tp;
+        }
+        if (lo + kScanPer <= M) {
+            reinterpret_cast<int4 *>(chunk_off + lo)[0] = make_int4(o[0], o[1], o[2], o[3]);
+            reinterpret_cast<int4 *>(chunk_off + lo)[1] = make_int4(o[4], o[5], o[6], o[7]);
+            reinterpret_cast<int4 *>(tile_off + lo)[0] = make_int4(to[0], to[1], to[2], to[3]);
+            reinterpret_cast<int4 *>(tile_off + lo)[1] = make_int4(to[4], to[5], to[6], to[7]);
+        } else {
+#pragma unroll
+            for (int k = 0; k < kScanPer; ++k)
+                if (lo + k < M) {
+                    chunk_off[lo + k] = o[k];
+                    tile_off[lo + k] = to[k];
+                }
+        }
+        carry += total;
+        tcarry += ttotal;
     }
     if (threadIdx.x == 0) {
-        chunk_off[M] = total;
-        tile_off[M] = ttotal;
-        num_tiles[0] = min(ttotal, max_tiles);
+        chunk_off[M] = carry;
+        tile_off[M] = tcarry;
+        num_tiles[0] = min(tcarry, max_tiles);
     }
 }
 
@@ -177,36 +218,61 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_kernel(const int32_t *_
 
 // Scatter as a block-level counting sort: the block's (token, slot) entries are ranked by chunk in
 // shared memory first, so each chunk's run of entries from this block is written to consecutive
-// pair-list positions (coalesced stores instead of one scattered store per entry). Used when the
-// chunk count per (b, h) fits the shared-memory tables (N <= kSortedScatterMaxN).
+// pair-list positions (coalesced stores instead of one scattered store per entry). The block's entries
+// are contiguous in [B, H, T, K]: they are read as one flat, coalesced range, with a batch of loads
+// in flight per thread (a load per iteration would leave every thread waiting on memory latency),
+// and the shared-memory atomic that counts an entry also returns its rank within its chunk, so one
+// pass both counts and ranks. Used when the chunk count per (b, h) fits the shared-memory tables
+// (N <= kSortedScatterMaxN).
 constexpr int kSortedScatterMaxN = 2048;
+constexpr int kRankBits = 14;  // rank of an entry within its chunk (< kDispatchRows * 64 entries per block)
+constexpr int kScatterBatch = 8;  // entries per thread whose loads are in flight together
 
 __global__ void __launch_bounds__(kDispatchRows) scatter_sorted_kernel(
     const int32_t *__restrict__ sel_idx, const float *__restrict__ sel_w, int T, int N, int K,
     const int32_t *__restrict__ chunk_off, int32_t *__restrict__ chunk_cursor, int32_t *__restrict__ pair_row,
     float *__restrict__ pair_w, int32_t *__restrict__ pair_slot, const int32_t *__restrict__ cu_seqlens, int H) {
     extern __shared__ int s_mem[];
+    const int nent_max = kDispatchRows * K;
     int *s_cnt = s_mem;                  // [N] entries per chunk in this block
     int *s_scan = s_cnt + N;             // [N] exclusive scan of s_cnt
     int *s_gbase = s_scan + N;           // [N] global position of this block's run for the chunk
-    int *s_cur = s_gbase + N;            // [N] ranks handed out so far
-    int *s_key = s_cur + N;              // [rows * K] (c << 14) | (t_local << 6) | slot, sorted by chunk
-    float *s_wt = reinterpret_cast<float *>(s_key + kDispatchRows * K);
+    int *s_tmp = s_gbase + N;            // [rows * K] (c << kRankBits) | rank, in entry order; -1: empty slot
+    int *s_key = s_tmp + nent_max;       // [rows * K] (c << kRankBits) | entry, sorted by chunk
+    float *s_wt = reinterpret_cast<float *>(s_key + nent_max);
     __shared__ int s_warp[33];
     const int bh = blockIdx.y, tid = threadIdx.x;
     const int t0 = blockIdx.x * kDispatchRows;
     const int Tv = cu_seqlens ? min(T, cu_seqlens[bh / H + 1] - cu_seqlens[bh / H]) : T;  // rows past it: none
     if (t0 >= Tv) return;
-    const int t = t0 + tid;
-    for (int i = tid; i < N; i += blockDim.x) { s_cnt[i] = 0; s_cur[i] = 0; }
+    const int nent = min(kDispatchRows, Tv - t0) * K;
+    const size_t e0 = ((size_t)bh * T + t0) * K;  // the block's first entry in [B, H, T, K]
+    for (int i = tid; i < N; i += blockDim.x) s_cnt[i] = 0;
     __syncthreads();
-    const int32_t *si = sel_idx + ((size_t)bh * T + (t < T ? t : 0)) * K;
-    if (t < Tv)
-        for (int j = 0; j < K; ++j) {
-            const int c = si[j];
-            if (c >= 0 && c < N) atomicAdd(&s_cnt[c], 1);
+    // count and rank; kScatterBatch loads in flight per thread before their atomics
+    for (int eb = 0; eb < nent; eb += kScatterBatch * kDispatchRows) {
+        int cb[kScatterBatch];
+#pragma unroll
+        for (int k = 0; k < kScatterBatch; ++k) {
+            const int e = eb + k * kDispatchRows + tid;
+            cb[k] = e < nent ? sel_idx[e0 + e] : -1;
         }
+#pragma unroll
+        for (int k = 0; k < kScatterBatch; ++k) {
+            const int e = eb + k * kDispatchRows + tid, c = cb[k];
+            if (e < nent) s_tmp[e] = (c >= 0 && c < N) ? (c << kRankBits) | atomicAdd(&s_cnt[c], 1) : -1;
+        }
+    }
     __syncthreads();
+    // this block's run of each chunk in the global lists: the atomics (chunks tid + 256 k) go out
+    // before the block scan and are used after it
+    int gpos[kSortedScatterMaxN / kDispatchRows];
+#pragma unroll
+    for (int k = 0; k < kSortedScatterMaxN / kDispatchRows; ++k) {
+        const int i = tid + k * kDispatchRows;
+        const int cnt = i < N ? s_cnt[i] : 0;
+        gpos[k] = cnt ? atomicAdd(&chunk_cursor[(size_t)bh * N + i], cnt) + chunk_off[(size_t)bh * N + i] : 0;
+    }
     // block exclusive scan of the N counts (contiguous segment per thread)
     const int per = (N + blockDim.x - 1) / blockDim.x;
     const int lo = min(N, tid * per), hi = min(N, lo + per);
@@ -215,28 +281,42 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_sorted_kernel(
     int total;
     int off = block_exclusive_scan(sum, s_warp, total);
     for (int i = lo; i < hi; ++i) {
-        const int cnt = s_cnt[i];
         s_scan[i] = off;
-        s_gbase[i] = cnt ? chunk_off[(size_t)bh * N + i] + atomicAdd(&chunk_cursor[(size_t)bh * N + i], cnt) : 0;
-        off += cnt;
+        off += s_cnt[i];
+    }
+#pragma unroll
+    for (int k = 0; k < kSortedScatterMaxN / kDispatchRows; ++k) {
+        const int i = tid + k * kDispatchRows;
+        if (i < N) s_gbase[i] = gpos[k];
     }
     __syncthreads();
-    if (t < Tv)
-        for (int j = 0; j < K; ++j) {
-            const int c = si[j];
-            if (c < 0 || c >= N) continue;
-            const int p = s_scan[c] + atomicAdd(&s_cur[c], 1);
-            s_key[p] = (c << 14) | (tid << 6) | j;
-            s_wt[p] = sel_w[((size_t)bh * T + t) * K + j];
+    for (int eb = 0; eb < nent; eb += kScatterBatch * kDispatchRows) {
+        int vb[kScatterBatch];
+        float wb[kScatterBatch];
+#pragma unroll
+        for (int k = 0; k < kScatterBatch; ++k) {
+            const int e = eb + k * kDispatchRows + tid;
+            vb[k] = e < nent ? s_tmp[e] : -1;
+            wb[k] = e < nent ? sel_w[e0 + e] : 0.0f;
         }
+#pragma unroll
+        for (int k = 0; k < kScatterBatch; ++k) {
+            const int v = vb[k];
+            if (v < 0) continue;
+            const int c = v >> kRankBits;
+            const int p = s_scan[c] + (v & ((1 << kRankBits) - 1));
+            s_key[p] = (c << kRankBits) | (eb + k * kDispatchRows + tid);
+            s_wt[p] = wb[k];
+        }
+    }
     __syncthreads();
     for (int i = tid; i < total; i += blockDim.x) {
         const int key = s_key[i];
-        const int c = key >> 14, tl = (key >> 6) & 0xff, j = key & 63;
+        const int c = key >> kRankBits, e = key & ((1 << kRankBits) - 1);
         const int pos = s_gbase[c] + (i - s_scan[c]);
-        pair_row[pos] = (int32_t)((size_t)bh * T + t0 + tl);
+        pair_row[pos] = (int32_t)((size_t)bh * T + t0 + e / K);
         pair_w[pos] = s_wt[i];
-        if (pair_slot) pair_slot[pos] = j;
+        if (pair_slot) pair_slot[pos] = e % K;
     }
 }
 
@@ -261,6 +341,19 @@ __global__ void finalize_kernel(const float *__restrict__ o_acc, uint16_t *__res
 }
 
 // ------------------------------------------------------------------------------------------------
+cudaError_t zero_dispatch_state(int32_t *err, int32_t *chunk_count, int32_t *chunk_cursor, size_t chunks,
+                                cudaStream_t s) {
+    const char *e0 = reinterpret_cast<const char *>(err);
+    const char *c0 = reinterpret_cast<const char *>(chunk_count), *c1 = c0 + chunks * sizeof(int32_t);
+    const char *u0 = reinterpret_cast<const char *>(chunk_cursor), *u1 = u0 + chunks * sizeof(int32_t);
+    if (err && c0 >= e0 + sizeof(int32_t) && c0 - e0 <= 256 && u0 >= c1 && u0 - c1 <= 256)
+        return cudaMemsetAsync(err, 0, (size_t)(u1 - e0), s);
+    cudaError_t e = chunks ? cudaMemsetAsync(chunk_count, 0, chunks * sizeof(int32_t), s) : cudaSuccess;
+    if (e == cudaSuccess && chunks) e = cudaMemsetAsync(chunk_cursor, 0, chunks * sizeof(int32_t), s);
+    if (e == cudaSuccess && err) e = cudaMemsetAsync(err, 0, sizeof(int32_t), s);
+    return e;
+}
+
 size_t forward_max_tiles(int B, int H, int T, int topk) {
     const size_t pairs = (size_t)B * H * T * topk;
     const size_t chunks = (size_t)B * H * (T / kChunk);
@@ -292,8 +385,8 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
         tile_list_kernel<<<(M + 7) / 8, 256, 0, s>>>(chunk_count, chunk_off, tile_off, M, tiles, max_tiles,
                                                      tile_pairs);
     }
-    if (N <= kSortedScatterMaxN) {
-        const size_t ssmem = 4 * (size_t)N * sizeof(int) + (size_t)kDispatchRows * topk * (sizeof(int) + sizeof(float));
+    if (N <= kSortedScatterMaxN && topk <= 64) {  // ranks and entries fit kRankBits
+        const size_t ssmem = 3 * (size_t)N * sizeof(int) + (size_t)kDispatchRows * topk * 3 * sizeof(int);
         cudaError_t e = cudaFuncSetAttribute(scatter_sorted_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)ssmem);
         if (e != cudaSuccess) return e;
@@ -332,9 +425,7 @@ cudaError_t launch_forward(const ForwardArgs &a0, cudaStream_t s) {
     {
         HSA_PROF("memset", s);
         // o_acc is zeroed by the score kernel, tile by tile
-        e = cudaMemsetAsync(a.chunk_count, 0, chunks * sizeof(int32_t), s);
-        if (e == cudaSuccess) e = cudaMemsetAsync(a.chunk_cursor, 0, chunks * sizeof(int32_t), s);
-        if (e == cudaSuccess) e = cudaMemsetAsync(a.err, 0, sizeof(int32_t), s);
+        e = zero_dispatch_state(a.err, a.chunk_count, a.chunk_cursor, chunks, s);
     }
     if (e != cudaSuccess) return e;
     e = launch_score_tc(a, s);

@@ -12,8 +12,9 @@
 // and TMEM buffers / warpgroups b = j % 2:
 //   warps 16-19 loaders: the tile's Q rows gathered with cp.async (a warp-wide copy covers whole
 //               256-byte rows) into the 128-byte-swizzled layout tcgen05 reads, two tiles of copies in
-//               flight per thread; K_c and V_c as 64-row TMA tiles. The next tile's token ids are
-//               prefetched while the copies run;
+//               flight per thread; K_c and V_c as 64-row TMA tiles. A tile's Q copies are published
+//               right after the next tile's are issued; tile descriptors are fetched two tiles ahead
+//               and token ids one tile ahead, so the loop never waits on a dependent load;
 //   warp 20     MMA issuer: allocates TMEM; one thread issues S(j) = Q K^T and O(j) = P V as soon as
 //               each is ready (neither order is forced); O takes P straight from TMEM (A operand in
 //               TMEM); completion via tcgen05.commit. S buffer b is free again as soon as O(j) has
@@ -168,7 +169,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
         const int lw = warp - kTcLoaderWarp0, lt = tid - 32 * kTcLoaderWarp0;
         const int rsub = lane / CPR, ch = lane % CPR;
         const int myr = 32 * lw + lane;  // the tile row whose token id this thread fetches
+        // descriptors run two tiles ahead and token ids one tile ahead, so no load the loop waits on
+        // is issued less than a tile before it is needed
         PairTile t = mine > 0 ? tiles[blockIdx.x] : PairTile{0, 0, 0, 0};
+        PairTile t_next = mine > 1 ? tiles[blockIdx.x + G] : PairTile{0, 0, 0, 0};
         int myrow = (mine > 0 && myr < t.count) ? pair_row[t.start + myr] : -1;
         float myw = (mine > 0 && myr < t.count) ? pair_w[t.start + myr] : 0.0f;
         int pending = -1;  // tile whose Q copies are in flight and not yet published
@@ -201,19 +205,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
                                src >= 0 ? 16 : 0);
             }
             cp_async_commit();
-            // the next tile's descriptor and token ids, fetched while the copies run
-            if (j + 1 < mine) {
-                t = tiles[blockIdx.x + (size_t)(j + 1) * G];
-                const bool valid = myr < t.count;
-                myrow = valid ? pair_row[t.start + myr] : -1;
-                myw = valid ? pair_w[t.start + myr] : 0.0f;
-            }
-            if (pending >= 0) {  // publish the previous tile once its copies have landed
+            // publish the previous tile once its copies have landed, before anything that could wait
+            if (pending >= 0) {
                 cp_async_wait<1>();
                 tc::fence_proxy_async_smem();
                 tc::mbar_arrive(bar(kQkFull + pending % kTcQkSlots));
             }
             pending = j;
+            // the next tile's token ids (its descriptor is already here) and the descriptor after it,
+            // fetched while the copies run
+            if (j + 1 < mine) {
+                t = t_next;
+                const bool valid = myr < t.count;
+                myrow = valid ? pair_row[t.start + myr] : -1;
+                myw = valid ? pair_w[t.start + myr] : 0.0f;
+                if (j + 2 < mine) t_next = tiles[blockIdx.x + (size_t)(j + 2) * G];
+            }
         }
         cp_async_wait<0>();
         if (ok && pending >= 0) {

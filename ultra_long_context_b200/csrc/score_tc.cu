@@ -297,9 +297,14 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
                     if (eq && need_eq <= 0) continue;
                     need_eq -= eq ? 1 : 0;
                     // output slot: after the kept values above x, ties in chunk order
-                    int lo = 0;
+                    // ls[jj] - x is positive exactly when ls[jj] > x (no flush to zero here); times +inf it
+                    // saturates to 1, and to 0 when it is zero (the NaN saturates to 0) or negative.
+                    // Entries past k_keep are <= tau <= x and add nothing. This runs on the FMA pipe,
+                    // which the kernel leaves idle, instead of the ALU pipe that bounds it.
+                    float lq[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-                    for (int jj = 0; jj < K; ++jj) lo += (jj < k_keep && ls[jj] > x) ? 1 : 0;
+                    for (int jj = 0; jj < K; ++jj) lq[jj & 3] += __saturatef((ls[jj] - x) * INFINITY);
+                    const int lo = (int)((lq[0] + lq[1]) + (lq[2] + lq[3]));
                     const uint64_t freeb = ~used & (~0ull << lo);
                     const int slot = __ffsll((long long)freeb) - 1;
                     if (slot < 0 || slot >= k_keep) continue;  // only if pass 2 disagreed with pass 1

@@ -22,24 +22,37 @@
 
 namespace hsa {
 
-// delta_t = dO_t . O_t (bf16 inputs, fp32), one warp per token row.
+// delta_t = dO_t . O_t (bf16 inputs, fp32). D/8 lanes per token row (one 16-byte vector each), and
+// kDeltaGroups groups of rows per warp whose loads are all in flight before the first product: the
+// kernel streams out and dout once and is bound by HBM.
+constexpr int kDeltaGroups = 4;
+
 template <int D>
-__global__ void delta_kernel(const uint16_t *__restrict__ out, const uint16_t *__restrict__ dout, size_t rows,
-                             float *__restrict__ delta) {
-    const size_t row = (size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    float acc = 0.0f;
-    for (int d = lane * 8; d < D; d += 32 * 8) {
-        const uint4 o = *reinterpret_cast<const uint4 *>(out + row * D + d);
-        const uint4 g = *reinterpret_cast<const uint4 *>(dout + row * D + d);
-        acc = fmaf(bf16_lo(o.x), bf16_lo(g.x), acc); acc = fmaf(bf16_hi(o.x), bf16_hi(g.x), acc);
-        acc = fmaf(bf16_lo(o.y), bf16_lo(g.y), acc); acc = fmaf(bf16_hi(o.y), bf16_hi(g.y), acc);
-        acc = fmaf(bf16_lo(o.z), bf16_lo(g.z), acc); acc = fmaf(bf16_hi(o.z), bf16_hi(g.z), acc);
-        acc = fmaf(bf16_lo(o.w), bf16_lo(g.w), acc); acc = fmaf(bf16_hi(o.w), bf16_hi(g.w), acc);
+__global__ void __launch_bounds__(256) delta_kernel(const uint16_t *__restrict__ out, const uint16_t *__restrict__ dout,
+                                                    size_t rows, float *__restrict__ delta) {
+    constexpr int LPR = D / 8, RPW = 32 / LPR;  // lanes per row, rows per warp-wide load
+    const int lane = threadIdx.x & 31, sub = lane % LPR, rw = lane / LPR;
+    const size_t warp_g = (size_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+    const size_t row0 = warp_g * (RPW * kDeltaGroups) + rw;
+    uint4 o[kDeltaGroups], g[kDeltaGroups];
+#pragma unroll
+    for (int u = 0; u < kDeltaGroups; ++u) {
+        const size_t r = row0 + (size_t)u * RPW;
+        o[u] = r < rows ? *reinterpret_cast<const uint4 *>(out + r * D + sub * 8) : make_uint4(0u, 0u, 0u, 0u);
+        g[u] = r < rows ? *reinterpret_cast<const uint4 *>(dout + r * D + sub * 8) : make_uint4(0u, 0u, 0u, 0u);
     }
-    acc = warp_sum(acc);
-    if (lane == 0) delta[row] = acc;
+#pragma unroll
+    for (int u = 0; u < kDeltaGroups; ++u) {
+        float acc = 0.0f;
+        acc = fmaf(bf16_lo(o[u].x), bf16_lo(g[u].x), acc); acc = fmaf(bf16_hi(o[u].x), bf16_hi(g[u].x), acc);
+        acc = fmaf(bf16_lo(o[u].y), bf16_lo(g[u].y), acc); acc = fmaf(bf16_hi(o[u].y), bf16_hi(g[u].y), acc);
+        acc = fmaf(bf16_lo(o[u].z), bf16_lo(g[u].z), acc); acc = fmaf(bf16_hi(o[u].z), bf16_hi(g[u].z), acc);
+        acc = fmaf(bf16_lo(o[u].w), bf16_lo(g[u].w), acc); acc = fmaf(bf16_hi(o[u].w), bf16_hi(g[u].w), acc);
+#pragma unroll
+        for (int x = LPR / 2; x > 0; x >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, x);
+        const size_t r = row0 + (size_t)u * RPW;
+        if (sub == 0 && r < rows) delta[r] = acc;
+    }
 }
 
 constexpr int kBwdThreads = 128;  // 4 warps x 16 pairs
@@ -416,7 +429,8 @@ cudaError_t launch_backward(const BackwardArgs &a0, cudaStream_t s) {
         if (e == cudaSuccess && a.dQs && a.N == 0) e = cudaMemsetAsync(a.dQs, 0, rows * a.D * sizeof(float), s);
     }
     if (e != cudaSuccess || a.N == 0) return e;
-    const unsigned dblocks = (unsigned)((rows + 7) / 8);
+    const size_t rows_per_block = 8 * (32 / (a.D / 8)) * kDeltaGroups;  // 8 warps
+    const unsigned dblocks = (unsigned)((rows + rows_per_block - 1) / rows_per_block);
     {
         HSA_PROF("bwd_delta", s);
         if (a.D == 128) delta_kernel<128><<<dblocks, 256, 0, s>>>(a.out, a.dout, rows, a.delta);

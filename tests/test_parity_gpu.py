@@ -85,6 +85,18 @@ def test_forward_full_size_32k_sampled_rows(oracle_mod):
     assert stats["rows"] == len(rows)
 
 
+def test_forward_more_chunks_than_the_shared_tables(oracle_mod):
+    """131,173 tokens = 2049 complete chunks, past the score kernel's shared-memory pair count (1024
+    chunks) and the sorted scatter's tables (2048 chunks): the global-atomic count and the plain scatter
+    run. Sampled rows, with the chunk boundaries around both limits."""
+    B, H, T, D, topk = 1, 1, 64 * 2049 + 37, 64, 8
+    rng = np.random.default_rng(11)
+    edges = [0, 63, 64, 64 * 1024 - 1, 64 * 1024, 64 * 1025 - 1, 64 * 2048 - 1, 64 * 2048, 64 * 2049 - 1, T - 1]
+    rows = np.unique(np.concatenate([rng.integers(0, T, 384), edges]))
+    stats, _ = run_forward_case(oracle_mod, B, H, T, D, topk, seed=77, landmarks="chunk_mean", rows=rows)
+    assert stats["rows"] == len(rows)
+
+
 def test_forward_is_deterministic_in_selection_and_close_in_output():
     Q, K, V, L = inputs.forward_inputs(1, 2, 4096, 128, 3, device=DEV)
     o1, i1, w1 = hsa.hsa_forward(Q, K, V, L, 16)

@@ -11,10 +11,11 @@
 // uses Q/K slot j % 2 (free again once S(j) is computed), V slot j % 3 (free once O(j) is computed)
 // and TMEM buffers / warpgroups b = j % 2:
 //   warps 16-19 loaders: the tile's Q rows gathered with cp.async (a warp-wide copy covers whole
-//               256-byte rows) into the 128-byte-swizzled layout tcgen05 reads, two tiles of copies in
-//               flight per thread; K_c and V_c as 64-row TMA tiles. A tile's Q copies are published
-//               right after the next tile's are issued; tile descriptors are fetched two tiles ahead
-//               and token ids one tile ahead, so the loop never waits on a dependent load;
+//               256-byte rows) into the 128-byte-swizzled layout tcgen05 reads, up to two tiles of
+//               copies in flight per thread; K_c and V_c as 64-row TMA tiles. Each loader thread's
+//               arrival on the tile's barrier is tied to its copies (cp.async.mbarrier.arrive), so a
+//               tile is published the moment its rows land; tile descriptors are fetched two tiles
+//               ahead and token ids one tile ahead, so the loop never waits on a dependent load;
 //   warp 20     MMA issuer: allocates TMEM; one thread issues S(j) = Q K^T and O(j) = P V as soon as
 //               each is ready (neither order is forced); O takes P straight from TMEM (A operand in
 //               TMEM); completion via tcgen05.commit. S buffer b is free again as soon as O(j) has
@@ -83,6 +84,12 @@ enum { kQkFull = 0, kQkEmpty = kTcQkSlots, kVFull = 2 * kTcQkSlots, kVEmpty = kV
        kSFull = kVEmpty + kTcVSlots, kPFull = kSFull + kTcGroups,
        kOFull = kPFull + kTcGroups, kSEmpty = kOFull + kTcGroups, kOEmpty = kSEmpty + kTcGroups,
        kEReady = kOEmpty + kTcGroups /* [group][2 slots] */ };
+
+// Arrive on an mbarrier once every cp.async this thread has issued so far has completed (the arrival
+// counts against the barrier's expected count: no increment first).
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t mbar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(mbar) : "memory");
+}
 
 // Slabs [cb0, cb1) of 32 O columns of one tile, scaled by f and added into the tokens' fp32 rows:
 // TMEM (thread = row) -> this warp's padded smem tile -> read back so that each warp-wide reduction
@@ -175,7 +182,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
         PairTile t_next = mine > 1 ? tiles[blockIdx.x + G] : PairTile{0, 0, 0, 0};
         int myrow = (mine > 0 && myr < t.count) ? pair_row[t.start + myr] : -1;
         float myw = (mine > 0 && myr < t.count) ? pair_w[t.start + myr] : 0.0f;
-        int pending = -1;  // tile whose Q copies are in flight and not yet published
         for (int j = 0; j < mine && ok; ++j) {
             const int sq = j % kTcQkSlots, sv = j % kTcVSlots;
             ok = tc::mbar_wait(bar(kQkEmpty + sq), ((uint32_t)(j / kTcQkSlots) & 1u) ^ 1u) &&
@@ -205,13 +211,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
                                src >= 0 ? 16 : 0);
             }
             cp_async_commit();
-            // publish the previous tile once its copies have landed, before anything that could wait
-            if (pending >= 0) {
-                cp_async_wait<1>();
-                tc::fence_proxy_async_smem();
-                tc::mbar_arrive(bar(kQkFull + pending % kTcQkSlots));
-            }
-            pending = j;
+            // this thread's arrival on qk_full fires by itself once its copies so far (this tile's among
+            // them) have landed, so a tile is published when its rows are in shared memory, whatever
+            // the loader waits for next; the MMA thread fences the proxies after its wait
+            cp_async_mbar_arrive_noinc(bar(kQkFull + sq));
             // the next tile's token ids (its descriptor is already here) and the descriptor after it,
             // fetched while the copies run
             if (j + 1 < mine) {
@@ -222,11 +225,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
                 if (j + 2 < mine) t_next = tiles[blockIdx.x + (size_t)(j + 2) * G];
             }
         }
-        cp_async_wait<0>();
-        if (ok && pending >= 0) {
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(bar(kQkFull + pending % kTcQkSlots));
-        }
+        cp_async_wait<0>();  // nothing in flight when the CTA exits
     } else if (warp == kTcMmaWarp) {
         // ================= MMA issuer =================
         if (lane == 0 && mine > 0) {
@@ -274,6 +273,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
                     tc::mbar_test(bar(kQkFull + next_s % kTcQkSlots), (uint32_t)(next_s / kTcQkSlots) & 1u) &&
                     tc::mbar_test(bar(kSEmpty + (next_s & 1)), ((uint32_t)(next_s >> 1) & 1u) ^ 1u)) {
                     tc::fence_after();
+                    tc::fence_proxy_async_smem();  // the Q rows came by cp.async (generic proxy)
                     issue_s(next_s++);
                     progress = true;
                 }

@@ -260,6 +260,35 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
             const int b = g % nblk;
             const int ncol = min(kStCols, my_n - b * kStCols);
             const uint32_t valid = ncol >= 32 ? 0xffffffffu : (ncol > 0 ? (1u << ncol) - 1u : 0u);
+            if (g == 0) {
+                // the first block seeds the list: its K largest of 32 values by a bitonic sorting
+                // network in registers (240 compare-exchanges, each a min and a max), where inserting
+                // all 32 one by one costs 32 passes over the list and a loop step each
+                float a[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) a[i] = v[i];
+                if (ncol < 32) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) a[i] = i < ncol ? a[i] : -INFINITY;
+                }
+#pragma unroll
+                for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+                    for (int jj = k >> 1; jj > 0; jj >>= 1)
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int l = i ^ jj;
+                            if (l > i) {  // descending where bit k of i is clear (k = 32: the whole list)
+                                const float hi = fmaxf(a[i], a[l]), lo = fminf(a[i], a[l]);
+                                const bool desc = (i & k) == 0;
+                                a[i] = desc ? hi : lo;
+                                a[l] = desc ? lo : hi;
+                            }
+                        }
+#pragma unroll
+                for (int i = 0; i < K; ++i) ls[i] = a[i];
+                continue;  // nothing else of the loop body applies to pass 1's first block
+            }
             // every score of the block to this thread's column; one bit per candidate
             uint32_t m = 0;
             if (g < nblk) {  // warp-uniform

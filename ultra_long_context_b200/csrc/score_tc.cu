@@ -21,7 +21,8 @@
 //   * Pass 1 keeps, per row, the K largest score VALUES in a sorted register list: the candidates
 //     are the scores above the current K-th value, each inserted with
 //     new[i] = max(old[i], min(old[i-1], x)), which touches every slot independently (no dependent
-//     chain). The K-th value tau results.
+//     chain). The first block seeds the list through a bitonic sorting network on its 32 values
+//     instead. The K-th value tau results.
 //   * Pass 2 recomputes the same blocks (bit-identical: same operands, same instruction sequence);
 //     the candidates are the scores >= tau, visited in chunk order, and it keeps every one above tau
 //     plus the lowest-index ones equal to tau until K are kept -- exactly the stable-sort rule. A

@@ -176,8 +176,8 @@ def kernel_profile(fn, steps):
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of the
 # current kernels on these workloads; set back to None whenever the kernel changes.
 TRAFFIC_BYTES = {
-    ("fwd_t32k_h8_d128_k16", "chunk_attn"): 737_530_112 + 234_890_752,
-    ("fwd_t32k_h8_d128_k16", "score_topk"): 136_410_368 + 277_807_872,
+    ("fwd_t32k_h8_d128_k16", "chunk_attn"): 737_464_576 + 234_949_888,
+    ("fwd_t32k_h8_d128_k16", "score_topk"): 136_419_072 + 277_083_392,
     # captured on a 4M-token cache (134.3 MB of landmarks read per scan); the scan's traffic grows in
     # proportion to the landmarks, so the 16M-token figure is four times that capture
     ("decode_16m_b1_h8_d128_k32", "decode_scan"): 4 * (134_291_456 + 143_872),

@@ -183,6 +183,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_scan_kernel(
         qr[6] = bf16_lo(v.w) * scale; qr[7] = bf16_hi(v.w) * scale;
     }
     const uint16_t *Lbh = Lc + (size_t)kvh * Nmax * D;
+    float gm[UNROLL];  // running maximum score of each of this lane group's UNROLL landmark streams
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) gm[u] = -INFINITY;
     for (int64_t base = c0 + (int64_t)warp * WARP_SPAN; base < c1; base += (int64_t)NWARP * WARP_SPAN) {
         uint4 v[UNROLL];
 #pragma unroll
@@ -196,29 +199,39 @@ __global__ void __launch_bounds__(kDecodeThreads, 4) decode_scan_kernel(
 #pragma unroll
             for (int o = LPL / 2; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
             const int64_t c = base + u * LPW + g;
+            if (c < c1) gm[u] = fmaxf(gm[u], p);
             if (sub == 0 && c < c1) keys[c - c0] = make_key(p, (uint32_t)c);
         }
     }
     __syncthreads();
-    // Exact pre-filter before the selection: the first S0 = K * G keys form K groups of G; the smallest
-    // of the K group maxima, tau, has at least K keys of the range at or above it, so no key below tau
-    // can be in the range's top K. The keys >= tau are compacted in place (in rounds that are read
-    // whole before any of their slots is written), and the radix selection runs over those only.
-    constexpr int G = 32;
-    const int S0 = K * G;
+    // Exact pre-filter before the selection. Each lane group kept, during the stream, the maximum score
+    // of each of its UNROLL landmark streams: NG disjoint groups of the range. The K largest group maxima
+    // are K different landmarks, so the range's K-th largest score is at least the K-th largest group
+    // maximum, tau, and no key below tau can be in the range's top K. The keys >= tau are compacted in
+    // place (in rounds that are read whole before any of their slots is written), and the selection
+    // runs over those only.
+    constexpr int NG = NWARP * LPW * UNROLL;  // 128 (D = 128) or 256 (D = 64) groups
     int nkeys = nloc;
-    if (nloc >= 2 * S0) {
-        unsigned long long *tau_s = reinterpret_cast<unsigned long long *>(topk);  // scratch until selection
-        if (tid == 0) *tau_s = ~0ull;
-        __syncthreads();
-        if (tid < K) {
-            uint64_t m = 0;
-            for (int i = 0; i < G; ++i) m = max(m, keys[tid * G + i]);
-            atomicMin(tau_s, (unsigned long long)m);
+    if (nloc >= 4 * K && K <= NG) {
+        float *gmax = reinterpret_cast<float *>(topk);  // scratch until the selection (topk, sorted: 1 KB)
+        if (sub == 0) {
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) gmax[(warp * LPW + g) * UNROLL + u] = gm[u];
         }
         __syncthreads();
-        const uint64_t tau = *tau_s;
-        nkeys = compact_at_least(keys, nloc, tau, misc);
+        for (int i = tid; i < NG; i += kDecodeThreads) {  // rank of each group maximum; ties by position
+            const float x = gmax[i];
+            int rank = 0;
+            for (int jj = 0; jj < NG; ++jj) {
+                const float y = gmax[jj];
+                rank += (y > x || (y == x && jj < i)) ? 1 : 0;
+            }
+            if (rank == K - 1) misc[6] = __float_as_int(x);
+        }
+        __syncthreads();
+        const float tau = __int_as_float(misc[6]);
+        __syncthreads();  // gmax (topk) is free again
+        nkeys = compact_at_least(keys, nloc, make_key(tau, 0xffffffffu), misc);
     }
     // the range's top K, in descending order (the merge reads each range's maximum at its head)
     int cnt;

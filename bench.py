@@ -180,7 +180,7 @@ TRAFFIC_BYTES = {
     ("fwd_t32k_h8_d128_k16", "score_topk"): 136_419_072 + 277_083_392,
     # captured on a 4M-token cache (134.3 MB of landmarks read per scan); the scan's traffic grows in
     # proportion to the landmarks, so the 16M-token figure is four times that capture
-    ("decode_16m_b1_h8_d128_k32", "decode_scan"): 4 * (134_291_456 + 143_872),
+    ("decode_16m_b1_h8_d128_k32", "decode_scan"): 4 * (134_294_016 + 454_656),
     ("fwdbwd_t64k_h8_d128_k16", "chunk_bwd"): 2_291_017_000 + 1_258_746_000,
 }
 # fp32 reductions into L2-resident rows, 4 rows x 128 B per red.global.add.v4.f32, 16-24 warps per SM:

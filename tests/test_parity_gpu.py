@@ -200,7 +200,9 @@ def test_decode_full_size(oracle_mod, name):
 
 @pytest.mark.parametrize("B,H,T,D,topk", [(1, 2, 1100, 64, 8), (1, 1, 2048 + 64, 128, 16), (2, 1, 700, 128, 5),
                                            # chunks with thousands of pairs: several work units each
-                                           (1, 2, 8192 + 81, 128, 16)])
+                                           (1, 2, 8192 + 81, 128, 16),
+                                           # 2049 chunks: the dispatch's plain scatter writes the slots
+                                           (1, 1, 64 * 2049 + 5, 64, 2)])
 def test_backward_matches_oracle(oracle_mod, B, H, T, D, topk):
     Q, K, V, L = inputs.forward_inputs(B, H, T, D, 500 + T, device=DEV)
     dO = inputs.upstream_grad(B, H, T, D, 500 + T, device=DEV)

@@ -41,8 +41,8 @@
  *     never expected, but possible on a faulty device) sets a status flag that lives in the first
  *     bytes of the call's workspace and lets the kernel unwind; the call itself has already
  *     returned (calls are asynchronous). hsa_workspace_status() reads that flag.
- *   - Supported now: D in {64, 128}, chunk == 64. Forward/backward: 1 <= topk <= 32;
- *     decode: 1 <= topk <= 64. Anything else returns HSA_ERR_UNSUPPORTED.
+ *   - Supported now: D in {64, 128}, chunk == 64, 1 <= topk <= 64 (the per-token procedure's default is
+ *     64; the "Build Your Own" recipe gives 16-64). Anything else returns HSA_ERR_UNSUPPORTED.
  *   - Every output element is written (including padding and all-zero rows).
  *   - Inputs must be finite; NaN/Inf inputs give unspecified results.
  *   - On any non-OK status, hsa_last_error() returns a message for the calling thread.

@@ -37,7 +37,7 @@ def _load():
         lib.hsa_oracle_scores_rows.argtypes = [_f32p, _f32p, _i64, _i64, _i64, _i64, _i64, _i64, ctypes.c_double,
                                                _i64, _i64p, _f64p]
         lib.hsa_oracle_decode_select.argtypes = [_f32p, _f32p, _i64p, _i64, _i64, _i64, _i64, _i64, _i64, _i64,
-                                                 ctypes.c_double, _i32p, _f64p, _f64p, _f64p]
+                                                 ctypes.c_double, _i32p, _f64p, _f64p, _f64p, _f64p]
         lib.hsa_oracle_attend_gathered.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _i32p, _i64, _i64, _i64, _i64,
                                                    ctypes.c_double, _int, _f64p, _f64p]
         lib.hsa_oracle_backward.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _i32p, _i64, _i64, _i64, _i64,
@@ -136,9 +136,10 @@ def scores(Q, L, rows, chunk=64, scale=None):
     return out
 
 
-def decode_select(q, Lc, cache_len, chunk=64, topk=16, scale=None):
+def decode_select(q, Lc, cache_len, chunk=64, topk=16, scale=None, all_scores=False):
     """Decode retrieval: q [B, H, D] (retrieval queries), Lc [B, Hkv, Nmax, D], cache_len [B] -> selection
-    dict [B, H, topk]."""
+    dict [B, H, topk]. With all_scores, the dict also holds all_s [B, H, Nmax]: every retrieval score
+    (NaN for chunks the token does not see)."""
     q, qp = _f32(q)
     Lc, lp = _f32(Lc)
     B, H, D = q.shape
@@ -150,11 +151,15 @@ def decode_select(q, Lc, cache_len, chunk=64, topk=16, scale=None):
     sel_s = np.zeros((B, H, topk), np.float64)
     sel_w = np.zeros((B, H, topk), np.float64)
     next_s = np.zeros((B, H), np.float64)
+    all_s = np.zeros((B, H, Nmax), np.float64) if all_scores else None
     rc = _load().hsa_oracle_decode_select(qp, lp, _ptr(cl, _i64p), B, H, Lc.shape[1], D, Nmax, chunk, topk, scale,
                                           _ptr(sel_idx, _i32p), _ptr(sel_s, _f64p), _ptr(sel_w, _f64p),
-                                          _ptr(next_s, _f64p))
+                                          _ptr(next_s, _f64p), _ptr(all_s, _f64p))
     _check(rc, "hsa_oracle_decode_select")
-    return dict(sel_idx=sel_idx, sel_s=sel_s, sel_w=sel_w, next_s=next_s)
+    res = dict(sel_idx=sel_idx, sel_s=sel_s, sel_w=sel_w, next_s=next_s)
+    if all_scores:
+        res["all_s"] = all_s
+    return res
 
 
 def attend_gathered(q, Lg, Kg, Vg, nsel, scale=None, qs=None, qk_norm=False):

@@ -59,6 +59,19 @@ def forward(Q, K, V, L, chunk, topk, scale, Qs=None, qk_norm=False, eps=1e-6):
     return out, sel_idx, sel_w
 
 
+def scores(Qs, L, chunk, scale):
+    """Dense masked score matrix of Step 2: Qs [B, H, T, D], L [B, Hkv, N, D] -> [B, H, T, N] float64 with
+    NaN where chunk c has not ended at or before token t (the same einsum as ``forward``)."""
+    Qs, L = (np.asarray(x, np.float64) for x in (Qs, L))
+    B, H, T, D = Qs.shape
+    L = np.repeat(L, H // L.shape[1], axis=1)
+    N = L.shape[2]
+    t = np.arange(T)
+    admissible = (np.arange(N)[None, :] + 1) * chunk - 1 <= t[:, None]
+    S = scale * np.einsum("bhtd,bhnd->bhtn", Qs, L)
+    return np.where(admissible, S, np.nan)
+
+
 def best_subset(scores, k):
     """Top-k by exhaustive search: the k-subset with the largest score sum (distinct scores only)."""
     best, best_sum = None, -np.inf

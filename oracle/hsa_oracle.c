@@ -294,11 +294,13 @@ int hsa_oracle_scores_rows(const float *Q, const float *L, int64_t B, int64_t H,
  *   sequence b's cache
  * The new token sees every chunk that is complete in its cache: n = cache_len / chunk (R1 with
  * the query placed at the last cached position). Outputs per (b, h): sel_idx, sel_s, sel_w
- * [B, H, topk] as in hsa_oracle_forward_rows, and next_s [B, H].
+ * [B, H, topk] as in hsa_oracle_forward_rows, and next_s [B, H]. all_s (optional, [B, H, Nmax]) receives
+ * every retrieval score of Step 2, NaN for the chunks the token does not see: what a near-tie judgement
+ * of another selection needs.
  */
 int hsa_oracle_decode_select(const float *q, const float *Lc, const int64_t *cache_len, int64_t B, int64_t H,
                              int64_t Hkv, int64_t D, int64_t Nmax, int64_t chunk, int64_t topk, double scale,
-                             int32_t *sel_idx, double *sel_s, double *sel_w, double *next_s) {
+                             int32_t *sel_idx, double *sel_s, double *sel_w, double *next_s, double *all_s) {
     if (!q || !Lc || !cache_len || !sel_idx || D < 1 || chunk < 1 || topk < 1 || Hkv < 1 || H % Hkv != 0)
         return ORACLE_EINVAL;
     const int64_t G = H / Hkv;
@@ -318,6 +320,8 @@ int hsa_oracle_decode_select(const float *q, const float *Lc, const int64_t *cac
             status = ORACLE_ENOMEM;
         } else {
             for (int64_t c = 0; c < n; ++c) score[c] = retrieval_score(q + bh * D, Lc + (kvh * Nmax + c) * D, D, scale);
+            if (all_s)
+                for (int64_t c = 0; c < Nmax; ++c) all_s[bh * Nmax + c] = c < n ? score[c] : NAN;
             double nxt;
             int64_t k = select_topk(score, n, topk, sel, ss, &nxt);
             if (k < 0) {

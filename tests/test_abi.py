@@ -50,7 +50,7 @@ def _fwd(**kw):
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(D=96), -2), (dict(D=256), -2), (dict(chunk=32), -2), (dict(topk=33), -2),
+    (dict(D=96), -2), (dict(D=256), -2), (dict(chunk=32), -2), (dict(topk=65), -2),
     (dict(topk=0), -1), (dict(B=0), -1), (dict(T=0), -1), (dict(Q=None), -1), (dict(out=None), -1),
     (dict(L=None), -1), (dict(K=ODD), -1), (dict(sel_w=ODD), -1),
     (dict(ws=None), -3), (dict(ws_bytes=100), -3), (dict(ws=ctypes.c_void_p((1 << 20) + 16)), -3),
@@ -84,7 +84,7 @@ def _bwd(**kw):
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(D=32), -2), (dict(topk=40), -2), (dict(sel_idx=None), -1), (dict(dL=None), -1), (dict(dout=ODD), -1),
+    (dict(D=32), -2), (dict(topk=65), -2), (dict(sel_idx=None), -1), (dict(dL=None), -1), (dict(dout=ODD), -1),
     (dict(ws=None), -3),
 ])
 def test_backward_rejects_invalid_calls_on_host(kw, status):
@@ -165,7 +165,7 @@ def _fwd_varlen(**kw):
 @pytest.mark.parametrize("kw,status", [
     (dict(cu=None), -1), (dict(cu=ctypes.c_void_p((1 << 20) + 2)), -1), (dict(max_seqlen=0), -1), (dict(B=0), -1),
     (dict(Hkv=3), -1), (dict(flags=2), -1), (dict(out=None), -1), (dict(sel_w=None), -1), (dict(Q=ODD), -1),
-    (dict(D=96), -2), (dict(topk=33), -2), (dict(ws_bytes=64), -3), (dict(ws=None), -3),
+    (dict(D=96), -2), (dict(topk=65), -2), (dict(ws_bytes=64), -3), (dict(ws=None), -3),
 ])
 def test_forward_varlen_rejects_invalid_calls_on_host(kw, status):
     assert _fwd_varlen(**kw) == status

@@ -283,6 +283,29 @@ def test_decode_equals_last_prefill_row(oracle_mod, T):
     np.testing.assert_allclose(sel["sel_w"].reshape(B * H, topk), r["sel_w"], rtol=0, atol=1e-15)
 
 
+@pytest.mark.parametrize("lens,Hkv", [([128, 130], 2), ([127, 96], 1)])
+def test_decode_all_scores_match_dense_scores(oracle_mod, lens, Hkv):
+    """The decode's full score list (used to judge another selection on near-tie rows) is the dense
+    score matrix's row of the token at cache_len - 1, NaN for chunks it does not see; its stable
+    descending order starts with the selection."""
+    B, H, D, chunk, topk, Tmax = 2, 2, 8, 8, 3, 136
+    Q, K, V, L = bf16_arrays(B, H, Tmax, D, chunk, seed=33)
+    L = L[:, :Hkv]
+    q = np.stack([Q[b, :, lens[b] - 1] for b in range(B)])
+    scale = 1 / math.sqrt(D)
+    sel = oracle_mod.decode_select(q, L, lens, chunk=chunk, topk=topk, scale=scale, all_scores=True)
+    S = brute.scores(Q, L, chunk, scale)
+    for b in range(B):
+        ref = S[b, :, lens[b] - 1]                                   # [H, N]
+        np.testing.assert_allclose(sel["all_s"][b], ref, rtol=0, atol=1e-13)
+        assert np.array_equal(np.isnan(sel["all_s"][b]), np.isnan(ref))
+        for h in range(H):
+            s = np.where(np.isnan(ref[h]), -np.inf, ref[h])
+            n = int((~np.isnan(ref[h])).sum())
+            order = np.argsort(-s, kind="stable")[:min(topk, n)]
+            assert sel["sel_idx"][b, h, :len(order)].tolist() == order.tolist()
+
+
 def test_decode_short_and_ragged_caches(oracle_mod):
     B, H, D, chunk, topk = 3, 1, 4, 8, 2
     q = np.random.default_rng(3).standard_normal((B, H, D)).astype(np.float32)

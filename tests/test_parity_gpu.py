@@ -5,7 +5,7 @@ import numpy as np
 import pytest
 import torch
 
-from tests.parity import compare_forward_rows, grad_close
+from tests.parity import OUT_MAX_ABS, TIE, W_MAX_ABS, compare_forward_rows, grad_close
 from ultra_long_context_b200 import hsa, inputs
 
 pytestmark = pytest.mark.gpu
@@ -53,14 +53,20 @@ def run_forward_case(oracle_mod, B, H, T, D, topk, seed, landmarks="iid", rows=N
     (1, 1, 64 * 40 + 63, 128, 3, "chunk_mean"),
     (1, 2, 2048 + 64, 128, 32, "chunk_mean"),  # the 32-wide selection list at head dim 128
     (1, 1, 3000, 128, 24, "iid"),              # kout below the list length, ragged tail
+    # topk up to 64 (the per-token procedure's default): rows with n_t below and above topk, ragged tails
+    (1, 2, 4096 + 640 + 37, 64, 64, "iid"),
+    (1, 2, 4096 + 1000, 128, 48, "chunk_mean"),
+    (2, 1, 64 * 70 + 11, 128, 64, "chunk_mean"),
+    (1, 1, 3000, 64, 64, "iid"),               # n_t < topk on every row
 ])
 def test_forward_matches_oracle(oracle_mod, B, H, T, D, topk, landmarks):
     stats, _ = run_forward_case(oracle_mod, B, H, T, D, topk, seed=100 + T + topk, landmarks=landmarks)
     assert stats["rows"] == B * H * T
 
 
-def test_forward_equal_scores_keep_lowest_chunks(oracle_mod):
-    B, H, T, D, topk = 1, 2, 640, 64, 4
+@pytest.mark.parametrize("T,D,topk", [(640, 64, 4), (64 * 90 + 5, 128, 64), (64 * 70, 64, 48)])
+def test_forward_equal_scores_keep_lowest_chunks(oracle_mod, T, D, topk):
+    B, H = 1, 2
     Q, K, V, L = inputs.forward_inputs(B, H, T, D, 7, device=DEV)
     L[:] = L[:, :, :1, :]
     out, idx, w = hsa.hsa_forward(Q, K, V, L, topk)
@@ -114,7 +120,7 @@ def oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, chunk=64, qs=None, qk_n
     B, H, D = q.shape
     scale = scale or 1 / math.sqrt(D)
     sel = oracle_mod.decode_select(host(q if qs is None else qs), host(Lc), lens.cpu().numpy(), chunk=chunk, topk=topk,
-                                   scale=scale)
+                                   scale=scale, all_scores=True)
     if Kc.shape[1] != H:  # grouped key heads: each query head gathers from its key head's cache
         Kc, Vc, Lc = (x.repeat_interleave(H // Kc.shape[1], dim=1) for x in (Kc, Vc, Lc))
     idx = torch.as_tensor(sel["sel_idx"], device=Kc.device, dtype=torch.int64).clamp(min=0)   # [B,H,k]
@@ -127,7 +133,58 @@ def oracle_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, chunk=64, qs=None, qk_n
                                         scale=scale, qk_norm=qk_norm,
                                         qs=None if qs is None else host(qs).reshape(B * H, D))
     return dict(out=out, sel_idx=sel["sel_idx"].reshape(B * H, topk), sel_w=w, sel_s=sel["sel_s"].reshape(B * H, topk),
-                next_s=sel["next_s"].reshape(-1))
+                next_s=sel["next_s"].reshape(-1), all_s=sel["all_s"].reshape(B * H, -1))
+
+
+def compare_decode_rows(oracle_mod, orc, g_idx, g_w, g_out, q, Kc, Vc, Lc, qs=None, qk_norm=False, scale=None,
+                        chunk=64, label=""):
+    """Decode rows (flat (b, h)) against the oracle, by the rule of the forward (tests/parity.py): equal
+    selection sets, or a near-tie row (oracle K-th and (K+1)-th scores within 1e-3) whose GPU-kept chunks
+    all score within 1e-3 of the oracle's K-th score and whose output matches the oracle evaluated on the
+    GPU's set. Returns the number of near-tie rows."""
+    BH, D = g_out.shape
+    H = q.shape[1]
+    G = H // Kc.shape[1]
+    scale = scale or 1 / math.sqrt(D)
+    topk = g_idx.shape[1]
+    tie_rows = []
+    for i in range(BH):
+        gs, os_ = set(g_idx[i][g_idx[i] >= 0].tolist()), set(orc["sel_idx"][i][orc["sel_idx"][i] >= 0].tolist())
+        if gs != os_:
+            assert len(gs) == len(os_), f"{label}(b,h)={i}: {len(gs)} chunks kept, oracle keeps {len(os_)}"
+            k = len(os_)
+            s_k = orc["sel_s"][i, k - 1]
+            assert s_k - orc["next_s"][i] < TIE, f"{label}(b,h)={i}: selection differs, gap {s_k - orc['next_s'][i]:.3g}"
+            for c in gs:
+                assert orc["all_s"][i, c] >= s_k - TIE, f"{label}(b,h)={i}: chunk {c} is not a near-tie choice"
+            tie_rows.append(i)
+            continue
+        d = np.abs(g_out[i] - orc["out"][i])
+        assert d.max() <= OUT_MAX_ABS, f"{label}(b,h)={i}: max-abs {d.max():.4g}"
+        og = dict(zip(orc["sel_idx"][i].tolist(), orc["sel_w"][i].tolist()))
+        for c, ww in zip(g_idx[i].tolist(), g_w[i].tolist()):
+            if c >= 0:
+                assert abs(ww - og[c]) <= W_MAX_ABS
+    if tie_rows:  # the oracle's Steps 3-4 on the GPU's (valid) selection of those rows
+        n = len(tie_rows)
+        Lg = np.zeros((n, topk, D), np.float32)
+        Kg = np.zeros((n, topk, chunk, D), np.float32)
+        Vg = np.zeros_like(Kg)
+        nsel = np.zeros(n, np.int32)
+        for r, i in enumerate(tie_rows):
+            b, hk = i // H, (i % H) // G
+            kept = [int(c) for c in g_idx[i] if c >= 0]
+            for j, c in enumerate(kept):
+                Lg[r, j] = host(Lc[b, hk, c])
+                Kg[r, j] = host(Kc[b, hk, c * chunk:(c + 1) * chunk])
+                Vg[r, j] = host(Vc[b, hk, c * chunk:(c + 1) * chunk])
+            nsel[r] = len(kept)
+        qr = host(q).reshape(BH, D)[tie_rows]
+        qsr = None if qs is None else host(qs).reshape(BH, D)[tie_rows]
+        o, _ = oracle_mod.attend_gathered(qr, Lg, Kg, Vg, nsel, scale=scale, qs=qsr, qk_norm=qk_norm)
+        dt = np.abs(g_out[tie_rows] - o)
+        assert dt.max() <= OUT_MAX_ABS, f"{label}near-tie rows: max-abs {dt.max():.4g}"
+    return len(tie_rows)
 
 
 def check_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, qs=None, qk_norm=False, scale=None):
@@ -138,20 +195,11 @@ def check_decode(oracle_mod, q, Kc, Vc, Lc, lens, topk, qs=None, qk_norm=False, 
     g_idx = idx.reshape(B * H, topk).cpu().numpy()
     g_w = w.reshape(B * H, topk).cpu().numpy()
     g_out = host(out).reshape(B * H, D)
-    for i in range(B * H):
-        gs, os_ = set(g_idx[i][g_idx[i] >= 0].tolist()), set(orc["sel_idx"][i][orc["sel_idx"][i] >= 0].tolist())
-        if gs != os_:
-            k = len(os_)
-            assert orc["sel_s"][i, k - 1] - orc["next_s"][i] < 1e-3, f"(b,h)={i}: selection differs"
-            continue
-        d = np.abs(g_out[i] - orc["out"][i])
-        assert d.max() <= 2e-2
-        og = dict(zip(orc["sel_idx"][i].tolist(), orc["sel_w"][i].tolist()))
-        for c, ww in zip(g_idx[i].tolist(), g_w[i].tolist()):
-            if c >= 0:
-                assert abs(ww - og[c]) <= 1e-3
+    ties = compare_decode_rows(oracle_mod, orc, g_idx, g_w, g_out, q, Kc, Vc, Lc, qs=qs, qk_norm=qk_norm,
+                               scale=scale)
     # ordering: by score descending (ties to the lower index) -> sel_w non-increasing
     assert np.all(np.diff(g_w, axis=1) <= 1e-6)
+    check_decode.near_tie_rows = ties
     return out, idx, w
 
 
@@ -188,6 +236,7 @@ def test_decode_full_size(oracle_mod, name):
     w = inputs.WORKLOADS[name]
     q, Kc, Vc, Lc, lens, needle = inputs.workload_inputs(w, device=DEV)
     out, idx, ww = check_decode(oracle_mod, q, Kc, Vc, Lc, lens, w.topk)
+    print(f"{name}: {check_decode.near_tie_rows} of {w.B * w.H} (b, h) rows took the near-tie branch")
     for b in range(w.B):
         assert torch.all(idx[b, :, 0] == int(needle[b]))
     del q, Kc, Vc, Lc
@@ -202,7 +251,9 @@ def test_decode_full_size(oracle_mod, name):
                                            # chunks with thousands of pairs: several work units each
                                            (1, 2, 8192 + 81, 128, 16),
                                            # 2049 chunks: the dispatch's plain scatter writes the slots
-                                           (1, 1, 64 * 2049 + 5, 64, 2)])
+                                           (1, 1, 64 * 2049 + 5, 64, 2),
+                                           # topk up to 64
+                                           (1, 1, 4096 + 128 + 9, 128, 64), (1, 2, 64 * 60 + 3, 64, 48)])
 def test_backward_matches_oracle(oracle_mod, B, H, T, D, topk):
     Q, K, V, L = inputs.forward_inputs(B, H, T, D, 500 + T, device=DEV)
     dO = inputs.upstream_grad(B, H, T, D, 500 + T, device=DEV)
@@ -246,6 +297,36 @@ def test_backward_full_size_properties():
             assert torch.all(dL[b, h][~hit] == 0)
             assert torch.all(dK[b, h].reshape(N, 64 * D)[~hit] == 0)
             assert torch.all(dV[b, h].reshape(N, 64 * D)[~hit] == 0)
+
+
+def test_backward_full_size_two_heads_match_oracle(oracle_mod):
+    """B1 T65536 H8 D128 topk16, in the launch configuration the benchmark times: the forward runs on
+    the GPU for the whole batch, then heads 0 and 7 (each an independent B1 H1 problem) are given the
+    oracle's own forward (selection, weights, bf16 output) and the backward of the whole batch runs on
+    the GPU. Their dQ, dK, dV and dL are compared element by element with the oracle's backward; the
+    GPU forward of those two heads is compared with the oracle too."""
+    w = inputs.WORKLOADS["fwdbwd_t64k_h8_d128_k16"]
+    Q, K, V, L, dO = inputs.workload_inputs(w, device=DEV)
+    out, idx, sw = hsa.hsa_forward(Q, K, V, L, w.topk)
+    torch.cuda.synchronize()
+    T, D, topk = w.T, w.D, w.topk
+    scale = 1 / math.sqrt(D)
+    refs = {}
+    for h in (0, w.H - 1):
+        Qh, Kh, Vh, Lh, dOh = (host(x[:, h:h + 1]) for x in (Q, K, V, L, dO))
+        orc = oracle_mod.forward(Qh, Kh, Vh, Lh, chunk=64, topk=topk, scale=scale)
+        compare_forward_rows(oracle_mod, host(out[:, h]).reshape(-1, D), idx[:, h].reshape(-1, topk).cpu().numpy(),
+                             sw[:, h].reshape(-1, topk).cpu().numpy(), orc, Qh, Kh, Vh, Lh, np.arange(T), 64, scale)
+        idx[:, h] = torch.as_tensor(orc["sel_idx"].reshape(1, T, topk), device=DEV)
+        sw[:, h] = torch.as_tensor(orc["sel_w"].reshape(1, T, topk), dtype=torch.float32, device=DEV)
+        out[:, h] = torch.as_tensor(orc["out"].reshape(1, T, D), dtype=torch.float32, device=DEV).to(torch.bfloat16)
+        refs[h] = oracle_mod.backward(Qh, Kh, Vh, Lh, dOh, orc["sel_idx"].reshape(1, 1, T, topk), chunk=64,
+                                      scale=scale)
+    grads = hsa.hsa_backward(Q, K, V, L, out, dO, idx, sw)
+    torch.cuda.synchronize()
+    for h, ref in refs.items():
+        for g, r, n in zip(grads, ref, ("dQ", "dK", "dV", "dL")):
+            grad_close(host(g[:, h:h + 1]), r, f"{n} head {h}")
 
 
 def test_workspace_status_clear_after_calls():
@@ -296,7 +377,8 @@ def test_decode_separate_retrieval_query_matches_oracle(oracle_mod, D, lens, top
     assert not torch.equal(idx, idx_q)
 
 
-@pytest.mark.parametrize("B,H,T,D,topk", [(1, 2, 2048 + 64, 128, 16), (1, 2, 1100, 64, 8)])
+@pytest.mark.parametrize("B,H,T,D,topk", [(1, 2, 2048 + 64, 128, 16), (1, 2, 1100, 64, 8),
+                                           (1, 1, 4096 + 256, 128, 64)])  # two slot groups per token
 def test_backward_separate_retrieval_query_matches_oracle(oracle_mod, B, H, T, D, topk):
     Q, K, V, L = inputs.forward_inputs(B, H, T, D, 800 + T, device=DEV)
     Qs = inputs.forward_inputs(B, H, T, D, 900 + T, device=DEV)[0]
@@ -473,17 +555,9 @@ def check_decode_multi(oracle_mod, q, Kc, Vc, Lc, lens, topk, qs=None, qk_norm=F
         g_idx = idx[:, :, i].reshape(B * H, topk).cpu().numpy()
         g_w = w[:, :, i].reshape(B * H, topk).cpu().numpy()
         g_out = host(out[:, :, i]).reshape(B * H, D)
-        for r in range(B * H):
-            gs = set(g_idx[r][g_idx[r] >= 0].tolist())
-            os_ = set(orc["sel_idx"][r][orc["sel_idx"][r] >= 0].tolist())
-            if gs != os_:
-                assert orc["sel_s"][r, len(os_) - 1] - orc["next_s"][r] < 1e-3, f"token {i} row {r}: selection differs"
-                continue
-            assert np.abs(g_out[r] - orc["out"][r]).max() <= 2e-2
-            og = dict(zip(orc["sel_idx"][r].tolist(), orc["sel_w"][r].tolist()))
-            for c, ww in zip(g_idx[r].tolist(), g_w[r].tolist()):
-                if c >= 0:
-                    assert abs(ww - og[c]) <= 1e-3
+        compare_decode_rows(oracle_mod, orc, g_idx, g_w, g_out, q[:, :, i].contiguous(), Kc, Vc, Lc,
+                            qs=None if qs is None else qs[:, :, i].contiguous(), qk_norm=qk_norm,
+                            label=f"token {i} ")
     return out, idx, w
 
 

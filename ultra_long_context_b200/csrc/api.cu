@@ -194,7 +194,7 @@ static hsa_status forward_impl(const char *name, const hsa_bf16 *Qs, const hsa_b
                                void *workspace, size_t workspace_bytes, void *stream,
                                const int32_t *cu_seqlens = nullptr) {
     g_last_error.clear();
-    hsa_status st = check_common(B, H, D, chunk, topk, 32);
+    hsa_status st = check_common(B, H, D, chunk, topk, 64);
     if (st != HSA_OK) return st;
     if (T < 1) return fail(HSA_ERR_INVALID_ARG, "T must be >= 1 (got %d)", T);
     if ((double)B * H * T * topk >= 2147483647.0 || (double)B * H * T * D >= 9.0e15)
@@ -344,7 +344,7 @@ static hsa_status backward_impl(const char *name, const hsa_bf16 *Qs, const hsa_
                                 int chunk, int topk, float scale, float *dQ, float *dK, float *dV, float *dL, float *dQs,
                                 bool qslc, bool qk_norm, void *workspace, size_t workspace_bytes, void *stream) {
     g_last_error.clear();
-    hsa_status st = check_common(B, H, D, chunk, topk, 32);
+    hsa_status st = check_common(B, H, D, chunk, topk, 64);
     if (st != HSA_OK) return st;
     if (T < 1) return fail(HSA_ERR_INVALID_ARG, "T must be >= 1 (got %d)", T);
     if ((double)B * H * T * topk >= 2147483647.0)
@@ -449,7 +449,7 @@ static hsa_status varlen_check(const int32_t *cu_seqlens, int B, int max_seqlen,
                                int topk, unsigned flags) {
     hsa_status st = check_ex(H, Hkv, flags);
     if (st != HSA_OK) return st;
-    if ((st = check_common(B, H, D, chunk, topk, 32)) != HSA_OK) return st;
+    if ((st = check_common(B, H, D, chunk, topk, 64)) != HSA_OK) return st;
     if (max_seqlen < 1) return fail(HSA_ERR_INVALID_ARG, "max_seqlen must be >= 1 (got %d)", max_seqlen);
     if (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
         return fail(HSA_ERR_INVALID_ARG, "cu_seqlens must be a 4-byte aligned device array of B + 1 entries");

@@ -330,26 +330,29 @@ __global__ void __launch_bounds__(256) dq_finish_kernel(const int32_t *__restric
     float acc[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) acc[i] = 0.0f;
-    // lane j holds slot j's chunk and ds (K <= 32); the landmark loads of the slots are independent, so
-    // several are in flight at once
-    const int c_l = lane < K ? sel_idx[row * K + lane] : -1;
-    const float ds_l = lane < K ? ds_pair[row * K + lane] : 0.0f;
+    // slots in groups of 32: lane j holds slot j0 + j's chunk and ds; the landmark loads of the slots are
+    // independent, so several are in flight at once
+    for (int j0 = 0; j0 < K; j0 += 32) {
+        const int kj = min(32, K - j0);
+        const int c_l = lane < kj ? sel_idx[row * K + j0 + lane] : -1;
+        const float ds_l = lane < kj ? ds_pair[row * K + j0 + lane] : 0.0f;
 #pragma unroll 8
-    for (int j = 0; j < K; ++j) {
-        const int c = __shfl_sync(0xffffffffu, c_l, j);
-        const float ds = __shfl_sync(0xffffffffu, ds_l, j);
-        if (c < 0 || c >= N) continue;  // empty slot (the dispatch skips the same ids); warp-uniform
-        const uint16_t *lr = L + (kvh * N + c) * D + lane * PER;
-        if constexpr (PER == 4) {
-            const uint2 v = *reinterpret_cast<const uint2 *>(lr);
-            acc[0] = fmaf(ds, bf16_lo(v.x), acc[0]);
-            acc[1] = fmaf(ds, bf16_hi(v.x), acc[1]);
-            acc[2] = fmaf(ds, bf16_lo(v.y), acc[2]);
-            acc[3] = fmaf(ds, bf16_hi(v.y), acc[3]);
-        } else {
-            const uint32_t v = *reinterpret_cast<const uint32_t *>(lr);
-            acc[0] = fmaf(ds, bf16_lo(v), acc[0]);
-            acc[1] = fmaf(ds, bf16_hi(v), acc[1]);
+        for (int j = 0; j < kj; ++j) {
+            const int c = __shfl_sync(0xffffffffu, c_l, j);
+            const float ds = __shfl_sync(0xffffffffu, ds_l, j);
+            if (c < 0 || c >= N) continue;  // empty slot (the dispatch skips the same ids); warp-uniform
+            const uint16_t *lr = L + (kvh * N + c) * D + lane * PER;
+            if constexpr (PER == 4) {
+                const uint2 v = *reinterpret_cast<const uint2 *>(lr);
+                acc[0] = fmaf(ds, bf16_lo(v.x), acc[0]);
+                acc[1] = fmaf(ds, bf16_hi(v.x), acc[1]);
+                acc[2] = fmaf(ds, bf16_lo(v.y), acc[2]);
+                acc[3] = fmaf(ds, bf16_hi(v.y), acc[3]);
+            } else {
+                const uint32_t v = *reinterpret_cast<const uint32_t *>(lr);
+                acc[0] = fmaf(ds, bf16_lo(v), acc[0]);
+                acc[1] = fmaf(ds, bf16_hi(v), acc[1]);
+            }
         }
     }
     float *dq = dQ + row * D + lane * PER;

@@ -37,19 +37,20 @@ hsa_status fail(hsa_status st, const std::string &msg) {
 
 size_t round_up(size_t x) { return (x + 255) / 256 * 256; }
 
-// Layout inside the fixed array: candidates, ticket counters, selection (when the caller passes
-// none), per-chunk partial outputs -- the scratch the decode kernels need.
+// Layout inside the fixed array: error flag, candidates, ticket counters, selection (when the caller
+// passes none), per-chunk partial outputs -- the scratch the decode kernels need. The number of scan
+// ranges comes from the same plan that hsa_decode's workspace and launches use (one query row per key
+// head here), so the two cannot disagree.
 struct NoAllocLayout {
-    size_t cand, counters, sel_idx, sel_w, partial, total;
+    size_t err, cand, counters, sel_idx, sel_w, partial, total;
 };
 
-NoAllocLayout layout(int B, int H, int64_t Tmax, int D, int topk) {
-    const int64_t Nmax = Tmax / hsa::kChunk;
-    const int split = hsa::decode_split_size(Nmax, topk, B * H);
-    const int64_t nsplit = Nmax > 0 ? (Nmax + split - 1) / split : 1;
+NoAllocLayout layout(const hsa::DecodePlan &plan, int B, int H, int D, int topk) {
+    const int64_t nsplit = plan.nsplit;
     const size_t BH = (size_t)B * H;
     NoAllocLayout l{};
     size_t off = 0;
+    l.err = off;      off += round_up(sizeof(int32_t));
     l.cand = off;     off += round_up(BH * nsplit * topk * sizeof(uint64_t));
     l.counters = off; off += round_up(2 * BH * sizeof(unsigned));
     l.sel_idx = off;  off += round_up(BH * topk * sizeof(int32_t));
@@ -100,11 +101,10 @@ hsa_status hsa_decode_noalloc(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_b
         return fail(HSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned (cache_len 8-byte)");
     const int64_t Nmax = Tmax / hsa::kChunk;
     if (Nmax >= 2147483647LL) return fail(HSA_ERR_UNSUPPORTED, "Tmax / 64 must stay below 2^31");
-    const int split = hsa::decode_split_size(Nmax, topk, B * H);
-    const int64_t nsplit = Nmax > 0 ? (Nmax + split - 1) / split : 1;
-    if (hsa::decode_scan_smem(split, (int)nsplit, topk) > 227 * 1024)
+    const hsa::DecodePlan plan = hsa::decode_plan(Nmax, topk, B, H, H, 1);
+    if (hsa::decode_plan_smem(plan, topk) > 227 * 1024)
         return fail(HSA_ERR_UNSUPPORTED, "Tmax too large for this topk (scan merge exceeds shared memory)");
-    const NoAllocLayout l = layout(B, H, Tmax, D, topk);
+    const NoAllocLayout l = layout(plan, B, H, D, topk);
     if (l.total > kNoAllocScratchBytes) {
         char buf[256];
         snprintf(buf, sizeof(buf),
@@ -128,6 +128,7 @@ hsa_status hsa_decode_noalloc(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_b
     a.cand = reinterpret_cast<uint64_t *>(b + l.cand);
     a.counters = reinterpret_cast<unsigned *>(b + l.counters);  // zeroed by launch_decode every call
     a.partial = reinterpret_cast<float *>(b + l.partial);
+    a.err = reinterpret_cast<int32_t *>(b + l.err);
     const cudaError_t e = hsa::launch_decode(a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(HSA_ERR_CUDA, std::string("hsa_decode_noalloc: ") + cudaGetErrorString(e));
     return HSA_OK;

@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
                             }
                         }
 #pragma unroll
-                for (int i = 0; i < K; ++i) ls[i] = a[i];
+                for (int i = 0; i < K; ++i) ls[i] = i < 32 ? a[i] : -INFINITY;
                 continue;  // nothing else of the loop body applies to pass 1's first block
             }
             // every score of the block to this thread's column; one bit per candidate
@@ -409,7 +409,8 @@ static cudaError_t launch_st_d(const ForwardArgs &a, cudaStream_t s) {
         return cudaErrorInvalidValue;
     if (a.topk <= 8) return launch_st<D, 8>(a, tl, s);
     if (a.topk <= 16) return launch_st<D, 16>(a, tl, s);
-    return launch_st<D, 32>(a, tl, s);
+    if (a.topk <= 32) return launch_st<D, 32>(a, tl, s);
+    return launch_st<D, 64>(a, tl, s);
 }
 
 cudaError_t launch_score_tc(const ForwardArgs &a, cudaStream_t s) {

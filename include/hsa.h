@@ -254,6 +254,22 @@ hsa_status hsa_backward_varlen(const hsa_bf16 *Qs, const hsa_bf16 *Q, const hsa_
                                float *dL, float *dQs, void *workspace, size_t workspace_bytes, void *stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * Self-test of the bounded device waits (no counterpart on the pages; failure detection).
+ *
+ * Every kernel waits on mbarriers with a bounded number of probes; a wait that runs out records the
+ * failure in the status flag of the call's workspace, lets the kernel unwind (its copies finish, its
+ * TMEM is freed) and returns, so hsa_workspace_status() reports HSA_ERR_TIMEOUT instead of the device
+ * hanging. In a healthy run no wait runs out, so this call makes one run out on purpose: it clears the
+ * flag at the start of `workspace` (>= 256 bytes, 256-byte aligned, device memory), then launches one
+ * warp on `stream` that allocates TMEM, waits with the kernels' own helper -- but at most `probes`
+ * probes, 1 <= probes <= 2^20 -- on an mbarrier whose only expected arrival is never made, records the
+ * timeout as the kernels do, frees its TMEM and exits. Nothing faults; the context stays usable; the next
+ * operator call on the same workspace clears the flag again. Returns HSA_ERR_WORKSPACE or
+ * HSA_ERR_INVALID_ARG (host checks, nothing launched) or HSA_ERR_CUDA.
+ * ------------------------------------------------------------------------------------------- */
+hsa_status hsa_selftest_bounded_wait(void *workspace, size_t workspace_bytes, unsigned probes, void *stream);
+
+/* ---------------------------------------------------------------------------------------------
  * Measurement hooks (no counterpart on the pages; used to time each kernel live).
  *
  * hsa_profile_enable(1) starts recording a pair of CUDA events around every kernel launch and

@@ -190,3 +190,13 @@ def test_varlen_workspace_covers_the_padded_batch():
     assert hsa.lib().hsa_backward_varlen_workspace_size(B, H, Hkv, T, D, 64, K, 0) > \
         hsa.lib().hsa_forward_varlen_workspace_size(B, H, Hkv, T, D, 64, K, 0)
     assert hsa.lib().hsa_forward_varlen_workspace_size(B, H, 3, T, D, 64, K, 0) == 0  # H not a multiple of Hkv
+
+
+def test_selftest_bounded_wait_checks_its_workspace_on_host():
+    """The bounded-wait self-test validates its arguments before launching anything."""
+    f = hsa.lib().hsa_selftest_bounded_wait
+    assert f(None, 1 << 20, 100, None) == -3
+    assert f(ctypes.c_void_p((1 << 20) + 16), 1 << 20, 100, None) == -3   # not 256-byte aligned
+    assert f(FAKE, 64, 100, None) == -3                                    # too small
+    assert f(FAKE, 1 << 20, 0, None) == -1
+    assert f(FAKE, 1 << 20, (1 << 20) + 1, None) == -1

@@ -1,4 +1,5 @@
 """Parity of the CUDA path (through the C ABI) with the CPU oracle, on seeded synthetic inputs."""
+import ctypes
 import math
 
 import numpy as np
@@ -345,6 +346,27 @@ def test_workspace_status_clear_after_calls():
     wsd = torch.empty(hsa.hsa_decode_workspace_size(2, 2, 5056, D, 64, topk), dtype=torch.uint8, device=DEV)
     hsa.hsa_decode(q, Kc, Vc, Lc, lens_t, topk, workspace=wsd)
     hsa.hsa_workspace_status(wsd)
+
+
+def test_bounded_wait_that_runs_out_reports_timeout():
+    """A bounded device wait that runs out (the self-test's mbarrier never gets its arrival) is reported
+    as HSA_ERR_TIMEOUT by hsa_workspace_status, nothing faults, and the next operator call -- on the same
+    workspace, which it clears, and on a fresh one -- runs clean with the same results."""
+    B, H, T, D, topk = 1, 2, 1100, 128, 8
+    Q, K, V, L = inputs.forward_inputs(B, H, T, D, 23, device=DEV)
+    ws = torch.empty(hsa.hsa_forward_workspace_size(B, H, T, D, 64, topk), dtype=torch.uint8, device=DEV)
+    stream = torch.cuda.current_stream()
+    st = hsa.lib().hsa_selftest_bounded_wait(hsa._ptr(ws), ws.numel(), 2000, ctypes.c_void_p(stream.cuda_stream))
+    assert st == 0, hsa.hsa_last_error()
+    with pytest.raises(hsa.HSAError, match="HSA_ERR_TIMEOUT"):
+        hsa.hsa_workspace_status(ws)
+    out, idx, w = hsa.hsa_forward(Q, K, V, L, topk, workspace=ws)
+    hsa.hsa_workspace_status(ws)
+    ws2 = torch.empty_like(ws)
+    out2, idx2, w2 = hsa.hsa_forward(Q, K, V, L, topk, workspace=ws2)
+    hsa.hsa_workspace_status(ws2)
+    assert torch.equal(idx, idx2) and torch.equal(w, w2)
+    assert (out.float() - out2.float()).abs().max().item() <= 2e-2
 
 
 # ---------------------------------------------------------------------------------------------

@@ -60,7 +60,7 @@ struct StSmem {
     static constexpr int NB = (int)(kStTmemCols - QCOLS) / kStCols;   // TMEM score buffers
     static constexpr uint32_t LH = kStCols * 128;                     // one 64-column half of a block
     static constexpr uint32_t LB = KH * LH;                           // one landmark stage
-    static constexpr uint32_t STAGE = 128 * K * 8;                    // output staging: idx + w per row
+    static constexpr uint32_t STAGE = 128 * (K + 1) * 8;              // output staging: idx + w, padded rows
     // region U holds the landmark stages during the loop and the output staging at the end
     static constexpr uint32_t U = kStLStages * LB > STAGE ? kStLStages * LB : STAGE;
     // [33][128] fp32: a block's scores, one column per thread; [K+1][128] int32: the chunk of each
@@ -291,22 +291,23 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
                 continue;  // nothing else of the loop body applies to pass 1's first block
             }
             // every score of the block to this thread's column; one bit per candidate
-            uint32_t m = 0;
+            // the mask is built in four independent parts (no 32-long dependency chain through one register)
+            uint32_t mp[4] = {0u, 0u, 0u, 0u};
             if (g < nblk) {  // warp-uniform
                 const float thr = ls[K - 1];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     cv[128 * i] = v[i];
-                    m |= v[i] > thr ? 1u << i : 0u;
+                    mp[i & 3] |= v[i] > thr ? 1u << i : 0u;
                 }
             } else {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     cv[128 * i] = v[i];
-                    m |= v[i] >= tau ? 1u << i : 0u;
+                    mp[i & 3] |= v[i] >= tau ? 1u << i : 0u;
                 }
             }
-            m &= valid;
+            uint32_t m = ((mp[0] | mp[1]) | (mp[2] | mp[3])) & valid;
             if (g < nblk) {  // pass 1: insert the candidates that still beat the K-th value
                 while (m) {
                     const int i = __ffs(m) - 1;
@@ -347,8 +348,9 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
         // weights from the sorted values, and the tile's rows staged in shared memory (the landmark
         // stages are free: every MMA has completed)
         asm volatile("bar.sync 1, %0;" ::"n"(kStConsumers) : "memory");
+        // rows of kout + 1 entries: a row per thread without shared-memory bank conflicts
         int32_t *st_idx = reinterpret_cast<int32_t *>(s);
-        float *st_w = reinterpret_cast<float *>(s) + kStRows * kout;
+        float *st_w = reinterpret_cast<float *>(s) + kStRows * (kout + 1);
         if (tid < nrows) {
             const float top = ls[0];
             float z = 0.0f;
@@ -360,8 +362,8 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
                 if (i >= kout) break;
                 const bool u = (used >> i) & 1ull;
                 const int c = u ? cc[128 * i] : -1;
-                st_idx[tid * kout + i] = c;
-                st_w[tid * kout + i] = u ? expf((ls[i] - top) * scale) * rz : 0.0f;
+                st_idx[tid * (kout + 1) + i] = c;
+                st_w[tid * (kout + 1) + i] = u ? expf((ls[i] - top) * scale) * rz : 0.0f;
                 if (u) {
                     if (hist_smem) atomicAdd(&s_hist[c], 1);
                     else atomicAdd(&chunk_count[(size_t)bh * N + c], 1);
@@ -370,8 +372,9 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kStConsumers) : "memory");
         for (int i = tid; i < nv * kout; i += kStConsumers) {
-            sel_idx[out0 + i] = st_idx[i];
-            sel_w[out0 + i] = st_w[i];
+            const int rr = i / kout, j = i - rr * kout;
+            sel_idx[out0 + i] = st_idx[rr * (kout + 1) + j];
+            sel_w[out0 + i] = st_w[rr * (kout + 1) + j];
         }
         if (hist_smem)  // the tile's per-chunk counts into the dispatch's histogram
             for (int i = tid; i < n_max; i += kStConsumers)

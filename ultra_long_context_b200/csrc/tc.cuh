@@ -194,10 +194,10 @@ __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
 }
 __device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 
-// Waits for the phase with parity `parity` to complete; false if it did not within the bound
-// (about 2^22 probes, seconds of wall time).
-__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
-    for (uint32_t i = 0; i < (1u << 22); ++i) {
+// Waits for the phase with parity `parity` to complete; false if it did not within max_probes probes
+// (each probe may suspend the thread for a short, system-dependent time).
+__device__ __forceinline__ bool mbar_wait_n(uint32_t mbar, uint32_t parity, uint32_t max_probes) {
+    for (uint32_t i = 0; i < max_probes; ++i) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
@@ -210,6 +210,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
     }
     return false;
 }
+// The kernels' bound: about 2^22 probes, seconds of wall time.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) { return mbar_wait_n(mbar, parity, 1u << 22); }
 
 // Non-blocking probe: has the phase with parity `parity` completed?
 __device__ __forceinline__ bool mbar_test(uint32_t mbar, uint32_t parity) {

@@ -47,6 +47,7 @@ SIGNATURES = {
     "hsa_backward_varlen_workspace_size": ([_I, _I, _I, _I, _I, _I, _I, _U], _SZ),
     "hsa_backward_varlen": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _U, _P, _P,
                              _P, _P, _P, _P, _SZ, _P], _I),
+    "hsa_selftest_bounded_wait": ([_P, _SZ, _U, _P], _I),
     "hsa_profile_enable": ([_I], _I),
     "hsa_profile_summary": ([ctypes.c_char_p, _SZ], _I),
 }

@@ -1,4 +1,4 @@
-// bwd_tc.cu -- gradients of the HSA forward on the 5th-generation tensor cores (head dim 128).
+// bwd_tc.cu -- gradients of the HSA forward on the 5th-generation tensor cores (head dims 64 and 128).
 //
 // Explainer page of "Every Token Counts", "How It Works (Technically)", Step 4: the fusion weight
 // w = softmax(s over the selected chunks) multiplies the chunk output, so the loss gradient reaches
@@ -23,6 +23,8 @@
 // warpgroups: one half of the dQ columns each, and the unit's dV or dK), 12-15 loaders (cp.async
 // gathers of Q and dO rows, TMA tiles of K and V; dL from a tile's Q rows before its stage is
 // reloaded), 16 MMA issuer.
+// Head dim 64 uses the same layout: a Q or dO tile keeps two 64-column halves, the second zero (set
+// once), so dK^T and dV^T stay M = 128 products whose rows 64-127 come out zero and are not read.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -39,8 +41,7 @@ constexpr int kBtLoaderWarp0 = 12;                // warps 12-15
 constexpr int kBtMmaWarp = 16;
 constexpr int kBtThreads = 32 * (kBtMmaWarp + 1);  // 544
 
-struct BtSmem {  // head dim 128
-    static constexpr int D = 128;
+struct BtSmem {  // head dims 64 and 128 (64: the second half of a Q / dO tile holds zeros)
     static constexpr uint32_t HALF = 16384;            // [128 rows][128 B]: 64 columns of a Q / dO tile
     static constexpr uint32_t QD = 4 * HALF;           // Q tile (two halves) + dO tile (two halves)
     static constexpr uint32_t KH = 8192;               // [64 rows][128 B]: 64 columns of K or V
@@ -117,7 +118,7 @@ struct BtCursor {
     }
 };
 
-template <bool QSLC>
+template <int D, bool QSLC>
 __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
     const uint16_t *__restrict__ Q, const uint16_t *__restrict__ L, const uint16_t *__restrict__ dout,
     const float *__restrict__ delta, int T, int N, float scale, const PairTile *__restrict__ units,
@@ -129,7 +130,8 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
     // QSLC: separate retrieval queries Qs. dL takes ds times the retrieval query (read from global
     // memory), dQ leaves out the ds L_c term, and ds goes to ds_pair[token row, slot].
     using SM = BtSmem;
-    constexpr int D = SM::D;
+    static_assert(D == 64 || D == 128, "head dims 64 and 128");
+    constexpr int KHALVES = D / 64;  // 64-column halves of a K / V tile
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sb = (raw + 1023u) & ~1023u;  // 1 KB aligned (swizzle atoms)
@@ -146,6 +148,14 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid < 4 * D) s_dl[tid] = 0.0f;  // ordered before use by the __syncthreads below
+    if constexpr (D == 64) {  // the zero halves of both stages' Q and dO tiles (never written again)
+        for (int i = tid; i < 4 * (int)SM::HALF / 16; i += kBtThreads) {
+            const int h = i / (SM::HALF / 16), o = i % (SM::HALF / 16);  // h: stage 0/1, tile Q/dO
+            *reinterpret_cast<uint4 *>(s + SM::STG + (h >> 1) * SM::QD + (2 * (h & 1) + 1) * SM::HALF + 16 * o) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+        tc::fence_proxy_async_smem();  // generic-proxy stores -> tensor core reads
+    }
     const int nunits = num_units[0];
     const int G = gridDim.x;
     const int mine = (int)blockIdx.x < nunits ? (nunits - 1 - (int)blockIdx.x) / G + 1 : 0;
@@ -210,12 +220,13 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             ok = ok && tc::mbar_wait(bar(kBQdFull + stl), (uint32_t)(jl >> 1) & 1u) &&
                  tc::mbar_wait(bar(kBEReady + slot), (uint32_t)(jl >> 2) & 1u);
             if (!ok) return;
-            const int cc = lt & 15, gq = lt >> 4;
+            // CPR column chunks x (128 / CPR) groups of CPR pairs
+            const int cc = lt % CPR, gq = lt / CPR;
             const unsigned char *qt = s + SM::STG + stl * SM::QD + (cc >> 3) * SM::HALF;
             float a8[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll 4
-            for (int i = 0; i < 16; ++i) {
-                const int p = 16 * gq + i;
+            for (int i = 0; i < CPR; ++i) {
+                const int p = CPR * gq + i;
                 uint4 qv;
                 if constexpr (QSLC) {  // the retrieval query's row (the stage's metadata is still this tile's)
                     const int rp = s_row[stl * 128 + p];
@@ -231,9 +242,11 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                 a8[6] = fmaf(dsp, bf16_lo(qv.w), a8[6]); a8[7] = fmaf(dsp, bf16_hi(qv.w), a8[7]);
             }
 #pragma unroll
-            for (int k = 0; k < 8; ++k) a8[k] += __shfl_xor_sync(0xffffffffu, a8[k], 16);  // same cc
+            for (int o = CPR; o < 32; o <<= 1)  // the lanes of this warp with the same cc
+#pragma unroll
+                for (int k = 0; k < 8; ++k) a8[k] += __shfl_xor_sync(0xffffffffu, a8[k], o);
             float4 *own = reinterpret_cast<float4 *>(s_dl + lw * D + 8 * cc);  // only this lane writes these
-            if (lane < 16) {
+            if (lane < CPR) {
                 const float4 x0 = own[0], x1 = own[1];
                 own[0] = make_float4(x0.x + a8[0], x0.y + a8[1], x0.z + a8[2], x0.w + a8[3]);
                 own[1] = make_float4(x1.x + a8[4], x1.y + a8[5], x1.z + a8[6], x1.w + a8[7]);
@@ -241,10 +254,11 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             if (lag.last_tile()) {  // the unit's dL: thread lt = column d
                 const int bhl = lag.u.chunk / N / Gh, cl = lag.u.chunk % N;  // key head
                 asm volatile("bar.sync 2, 128;" ::: "memory");  // every loader warp's partials are in s_dl
-                atomicAdd(dL + ((size_t)bhl * N + cl) * D + lt,
-                          scale * ((s_dl[lt] + s_dl[D + lt]) + (s_dl[2 * D + lt] + s_dl[3 * D + lt])));
+                if (lt < D)
+                    atomicAdd(dL + ((size_t)bhl * N + cl) * D + lt,
+                              scale * ((s_dl[lt] + s_dl[D + lt]) + (s_dl[2 * D + lt] + s_dl[3 * D + lt])));
                 asm volatile("bar.sync 2, 128;" ::: "memory");  // all reads done before the owners reset
-                if (lane < 16) own[0] = own[1] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (lane < CPR) own[0] = own[1] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             }
             lag.next();
         };
@@ -276,10 +290,10 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                 // copies of this tile are already in flight); the next unit's tiles are prefetched to L2
                 ok = tc::mbar_wait(bar(kBKvEmpty), ((uint32_t)cur.k & 1u) ^ 1u);
                 if (ok) {
-                    tc::mbar_arrive_expect_tx(bar(kBKvFull), 4 * SM::KH);
+                    tc::mbar_arrive_expect_tx(bar(kBKvFull), 2 * KHALVES * SM::KH);
                     const int y = bh * T + c * kChunk;
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
+                    for (int h = 0; h < KHALVES; ++h) {
                         tc::tma_load_2d(sb + SM::KO + h * SM::KH, &tmK, h * 64, y, bar(kBKvFull));
                         tc::tma_load_2d(sb + SM::VO + h * SM::KH, &tmV, h * 64, y, bar(kBKvFull));
                     }
@@ -287,7 +301,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                         const PairTile nu = units[blockIdx.x + (size_t)(cur.k + 1) * G];
                         const int yn = (nu.chunk / N / Gh) * T + (nu.chunk % N) * kChunk;
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
+                        for (int h = 0; h < KHALVES; ++h) {
                             tc::tma_prefetch_2d(&tmK, h * 64, yn);
                             tc::tma_prefetch_2d(&tmV, h * 64, yn);
                         }
@@ -312,7 +326,8 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
         if (lane == 0 && mine > 0) {
             constexpr uint32_t id_s = tc::idesc_bf16(128, 64, 0, 0);   // S, dP': A, B K-major
             constexpr uint32_t id_q = tc::idesc_bf16(128, D, 0, 1);    // dQ: A K-major, B (K) MN-major
-            constexpr uint32_t id_t = tc::idesc_bf16(D, 64, 1, 1);     // dK^T, dV^T: A, B MN-major
+            constexpr uint32_t id_t = tc::idesc_bf16(128, 64, 1, 1);   // dK^T, dV^T: A, B MN-major (M = D, or
+                                                                       // 128 with zero rows past D = 64)
             BtCursor cs = cur, cg = cur;  // S / dP' and gradient cursors
             uint32_t idle = 0;
             while (!cg.done()) {
@@ -396,7 +411,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                 // of unit k - 4 is done with that slot, since this tile's S needed unit k - 1's last
                 // MMA, which needed the epilogue of a tile after unit k - 4's last
                 const int bhu = cur.u.chunk / N / Gh, cu = cur.u.chunk % N;  // key head
-                s_L[(cur.k & 3) * 128 + r] = __uint_as_float((uint32_t)L[((size_t)bhu * N + cu) * D + r] << 16);
+                if (r < D) s_L[(cur.k & 3) * 128 + r] = __uint_as_float((uint32_t)L[((size_t)bhu * N + cu) * D + r] << 16);
             }
             const uint32_t tS = tmem + lane_off + SM::S_COL;
             const uint32_t tDP = tmem + lane_off + SM::DP_COL;
@@ -468,7 +483,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             tc::mbar_arrive(bar(kBEReady + slot));
         }
     } else {
-        // ================= dQ epilogue: warpgroup e takes columns [64 e, 64 e + 64) =================
+        // ================= dQ epilogue: warpgroup e takes columns [D/2 e, D/2 e + D/2) =================
         const int e = (warp - kBtEpiWarp0) >> 2;
         const int r = (warp & 3) * 32 + lane;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
@@ -487,8 +502,8 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
             const float ds = QSLC ? 0.0f : e_ds[slot * 128 + r];  // the ds L_c term belongs to dQ only without Qs
             const float *Lr = s_L + (cur.k & 3) * 128;  // published with e_ready
 #pragma unroll 1
-            for (int cb = 0; cb < 64 / (int)SM::SLAB; ++cb) {
-                const int col0 = 64 * e + cb * (int)SM::SLAB;
+            for (int cb = 0; cb < D / 2 / (int)SM::SLAB; ++cb) {
+                const int col0 = D / 2 * e + cb * (int)SM::SLAB;
                 float o[16];
                 tc::tmem_ld16(tmem + lane_off + SM::DQ_COL + b * 128 + col0, o);
                 __syncwarp();  // the previous slab has been read back
@@ -521,12 +536,14 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                 float *dst = e == 0 ? dV : dK;
                 const float f = e == 0 ? 1.0f : scale;
                 const uint32_t tacc = tmem + lane_off + (e == 0 ? SM::DV_COL : SM::DK_COL);
+                if ((warp & 3) * 32 < D) {  // lanes past D hold the zero rows of a head-dim-64 product
 #pragma unroll 1
-                for (int h = 0; h < 2; ++h) {
-                    float v[32];
-                    tc::tmem_ld32(tacc + 32 * h, v);
+                    for (int h = 0; h < 2; ++h) {
+                        float v[32];
+                        tc::tmem_ld32(tacc + 32 * h, v);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) atomicAdd(dst + (krow0 + 32 * h + i) * D + r, f * v[i]);
+                        for (int i = 0; i < 32; ++i) atomicAdd(dst + (krow0 + 32 * h + i) * D + r, f * v[i]);
+                    }
                 }
                 tc::fence_before();
                 tc::mbar_arrive(bar(kBAccEmpty));
@@ -543,9 +560,10 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
 }
 
 cudaError_t launch_backward_tc(const BackwardArgs &a, cudaStream_t s) {
-    if (a.D != BtSmem::D) return cudaErrorInvalidValue;
+    if (a.D != 64 && a.D != 128) return cudaErrorInvalidValue;
     const size_t smem = BtSmem::DYN;
-    auto kern = a.Qs ? chunk_bwd_tc_kernel<true> : chunk_bwd_tc_kernel<false>;
+    auto kern = a.D == 128 ? (a.Qs ? chunk_bwd_tc_kernel<128, true> : chunk_bwd_tc_kernel<128, false>)
+                           : (a.Qs ? chunk_bwd_tc_kernel<64, true> : chunk_bwd_tc_kernel<64, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const uint64_t rows = (uint64_t)a.B * a.Hkv * a.T;  // units address K, V by key head

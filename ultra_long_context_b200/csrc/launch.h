@@ -40,14 +40,17 @@ DecodePlan decode_plan(int64_t Nmax, int K, int B, int H, int Hkv, int Tq);
 size_t decode_plan_smem(const DecodePlan &p, int K);  // the largest dynamic shared memory of its kernels
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 
-// Chunk-major work list entry: one tile of up to kPairTile (token, slot) pairs of one chunk.
+// Chunk-major work list entry: one tile (forward: <= 128 pairs) or work unit (backward: <= kBwdUnitPairs)
+// of (token, slot) pairs of one chunk.
 struct PairTile {
     int32_t chunk;  // flat (b*H + h) * N + c
     int32_t start;  // first pair (offset into the pair arrays)
-    int32_t count;  // pairs in this tile (1 .. kPairTile)
+    int32_t count;  // pairs in this tile
     int32_t pad;
 };
-constexpr int kPairTile = 64;  // pairs per tile of the mma.sync kernels (backward)
+// The work list is sized for tiles of at least kPairTile pairs (every chunk adds one partial tile), which
+// covers both the forward's tiles and the backward's units.
+constexpr int kPairTile = 64;
 
 struct ForwardArgs {
     const uint16_t *Qs;  // retrieval queries (scores, fusion weights); Q attends
@@ -127,7 +130,7 @@ struct BackwardArgs {
     uint16_t *Qn, *Kn;     // [B*H*T, D] and [B*Hkv*T, D]
 };
 cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t s);
-// Gradients on the tcgen05 tensor cores (bwd_tc.cu), head dim 128; work units of up to 1024 pairs.
+// Gradients on the tcgen05 tensor cores (bwd_tc.cu), head dims 64 and 128; work units of up to 1024 pairs.
 constexpr int kBwdUnitPairs = 1024;
 cudaError_t launch_backward_tc(const BackwardArgs &a, cudaStream_t s);
 

@@ -180,12 +180,12 @@ def kernel_profile(fn, steps):
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of the
 # current kernels on these workloads; set back to None whenever the kernel changes.
 TRAFFIC_BYTES = {
-    ("fwd_t32k_h8_d128_k16", "chunk_attn"): 737_464_576 + 234_949_888,
-    ("fwd_t32k_h8_d128_k16", "score_topk"): 136_419_072 + 277_083_392,
+    ("fwd_t32k_h8_d128_k16", "chunk_attn"): 737_926_144 + 235_332_096,
+    ("fwd_t32k_h8_d128_k16", "score_topk"): 136_418_560 + 276_941_568,
     # captured on a 4M-token cache (134.3 MB of landmarks read per scan); the scan's traffic grows in
     # proportion to the landmarks, so the 16M-token figure is four times that capture
     ("decode_16m_b1_h8_d128_k32", "decode_scan"): 4 * (134_294_016 + 454_656),
-    ("fwdbwd_t64k_h8_d128_k16", "chunk_bwd"): 2_291_017_000 + 1_258_746_000,
+    ("fwdbwd_t64k_h8_d128_k16", "chunk_bwd"): 2_288_028_416 + 1_252_866_048,
 }
 SCORE_LIMITER = "ALU pipe (per-row top-K selection); the tensor pipe idles between blocks"
 # fp32 reductions into L2-resident rows, 4 rows x 128 B per red.global.add.v4.f32, 16-24 warps per SM:
@@ -412,6 +412,7 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--skip-prefill", action="store_true", help="time only the decode / backward parts")
     ap.add_argument("--skip-decode", action="store_true")
+    ap.add_argument("--skip-decode-1m", action="store_true", help="of the decode, time only the 16M-token cache")
     ap.add_argument("--skip-backward", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-options", action="store_true",
@@ -690,12 +691,30 @@ def main():
                                       "kind": "oracle",
                                       "sample": f"{rows1} token-head rows drawn uniformly from the 4K workload, "
                                                 f"fp64 oracle with OpenMP, {spent1:.1f} s wall"}
+        # forward + backward at head dim 64 on the same shape (the tcgen05 backward's head-dim-64 form)
+        dO1 = inputs.upstream_grad(w1.B, w1.H, w1.T, w1.D, w1.seed + rank, device=dev)
+        bws1 = torch.empty(hsa.hsa_backward_workspace_size(w1.B, w1.H, w1.T, w1.D, 64, w1.topk) + 256,
+                           dtype=torch.uint8, device=dev)
+        g1 = tuple(torch.empty(x.shape, dtype=torch.float32, device=dev) for x in (Q1, K1, V1, L1))
+
+        def fwdbwd1():
+            flush.zero_()
+            fwd1()
+            hsa.hsa_backward(Q1, K1, V1, L1, out1, dO1, idx1, sw1, grads=g1, workspace=bws1)
+
+        fb_ms = max(1e-6, timed(fwdbwd1, steps1, args.warmup, world) / steps1 - fl_ms)
+        prof_fb1 = kernel_profile(fwdbwd1, steps1)
+        entry1["fwdbwd_d64"] = {
+            "ms_per_step": round(fb_ms, 5), "tokens_per_s": round(whole_job_rate(w1.B * w1.T, world, fb_ms), 1),
+            "roofline": roofline_entry("chunk_bwd", prof_fb1, 10.0 * 64 * w1.D * pairs1, "TFLOP/s", tensor_peak,
+                                       "tensor", tensor_kind),
+            "kernels": {k: {"launches": c, "avg_us": round(t / c * 1e3, 2)} for k, (c, t) in prof_fb1.items()}}
         extra["fwd_4k"] = entry1
-        del Q1, K1, V1, L1, out1, idx1, sw1, ws1, flush
+        del Q1, K1, V1, L1, out1, idx1, sw1, ws1, flush, dO1, bws1, g1
         torch.cuda.empty_cache()
 
     # ---------------- decode, 1M-token caches, batch 16 ----------------
-    if not args.skip_decode and not args.grouped_decode_only:
+    if not args.skip_decode and not args.grouped_decode_only and not args.skip_decode_1m:
         wm = inputs.WORKLOADS["decode_1m_b16_h8_d128_k16"]
         extra["decode_1m"] = decode_entry(hsa, inputs, wm, dev, max(args.steps, 50), args.warmup, world, peaks,
                                           peak_kind, cpu=rank == 0 and world == 1 and not args.skip_cpu)

@@ -182,9 +182,7 @@ def kernel_profile(fn, steps):
 TRAFFIC_BYTES = {
     ("fwd_t32k_h8_d128_k16", "chunk_attn"): 737_926_144 + 235_332_096,
     ("fwd_t32k_h8_d128_k16", "score_topk"): 136_418_560 + 276_941_568,
-    # captured on a 4M-token cache (134.3 MB of landmarks read per scan); the scan's traffic grows in
-    # proportion to the landmarks, so the 16M-token figure is four times that capture
-    ("decode_16m_b1_h8_d128_k32", "decode_scan"): 4 * (134_294_016 + 454_656),
+    ("decode_16m_b1_h8_d128_k32", "decode_scan"): 536_948_992 + 3_297_792,
     ("fwdbwd_t64k_h8_d128_k16", "chunk_bwd"): 2_288_028_416 + 1_252_866_048,
 }
 SCORE_LIMITER = "ALU pipe (per-row top-K selection); the tensor pipe idles between blocks"

@@ -16,8 +16,8 @@
 //               arrival on the tile's barrier is tied to its copies (cp.async.mbarrier.arrive), so a
 //               tile is published the moment its rows land; tile descriptors are fetched two tiles
 //               ahead and token ids one tile ahead, so the loop never waits on a dependent load;
-//   warp 20     MMA issuer: allocates TMEM; one thread issues S(j) = Q K^T and O(j) = P V as soon as
-//               each is ready (neither order is forced); O takes P straight from TMEM (A operand in
+//   warp 20     MMA issuer: allocates TMEM; the warp runs the issue loop and one elected lane issues
+//               S(j) = Q K^T and O(j) = P V as soon as each is ready (neither order is forced); O takes P straight from TMEM (A operand in
 //               TMEM); completion via tcgen05.commit. S buffer b is free again as soon as O(j) has
 //               read P, so the next softmax of a warpgroup overlaps the epilogue of the previous tile;
 //   warps 0-7   two softmax warpgroups (b = 0, 1), one thread per pair row: S row from TMEM, exact
@@ -227,8 +227,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
         }
         cp_async_wait<0>();  // nothing in flight when the CTA exits
     } else if (warp == kTcMmaWarp) {
-        // ================= MMA issuer =================
-        if (lane == 0 && mine > 0) {
+        // ================= MMA issuer: the whole warp runs the loop, one elected lane issues =================
+        if (mine > 0) {
             constexpr uint32_t idesc_s = tc::idesc_bf16(kTcTile, kChunk, 0, 0);
             constexpr uint32_t idesc_o = tc::idesc_bf16(kTcTile, D, 0, 1);
             auto issue_s = [&](int jj) {  // S(jj) = Q(jj) K_c(jj)^T into TMEM buffer jj % 2
@@ -238,22 +238,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t koff = (uint32_t)((ks & 3) * 32);  // K step inside a 128-byte row
-                    tc::mma_bf16_ss(tmem + SM::S_COL + b * kChunk, tc::desc_kmajor(sq + (ks >> 2) * 16384 + koff),
+                    tc::mma_bf16_ss_w(tmem + SM::S_COL + b * kChunk, tc::desc_kmajor(sq + (ks >> 2) * 16384 + koff),
                                     tc::desc_kmajor(sk + (ks >> 2) * 8192 + koff), idesc_s, ks > 0 ? 1u : 0u);
                 }
-                tc::commit(bar(kSFull + b));
-                tc::commit(bar(kQkEmpty + jj % kTcQkSlots));  // Q and K are free once S is computed
+                tc::commit_w(bar(kSFull + b));
+                tc::commit_w(bar(kQkEmpty + jj % kTcQkSlots));  // Q and K are free once S is computed
             };
             auto issue_o = [&](int jj) {  // O(jj) = P(jj) V_c(jj), P read from TMEM
                 const int b = jj & 1;
                 const uint32_t sv = sb + SM::VS + (jj % kTcVSlots) * SM::KB;
 #pragma unroll
                 for (int ks = 0; ks < kChunk / 16; ++ks)
-                    tc::mma_bf16_ts(tmem + SM::O_COL + b * D, tmem + SM::S_COL + b * kChunk + ks * 8,
+                    tc::mma_bf16_ts_w(tmem + SM::O_COL + b * D, tmem + SM::S_COL + b * kChunk + ks * 8,
                                     tc::desc_mnmajor(sv + ks * 2048, 8192), idesc_o, ks > 0 ? 1u : 0u);
-                tc::commit(bar(kOFull + b));
-                tc::commit(bar(kSEmpty + b));                // P has been read: S buffer b is free
-                tc::commit(bar(kVEmpty + jj % kTcVSlots));   // and V slot jj % 3
+                tc::commit_w(bar(kOFull + b));
+                tc::commit_w(bar(kSEmpty + b));                // P has been read: S buffer b is free
+                tc::commit_w(bar(kVEmpty + jj % kTcVSlots));   // and V slot jj % 3
             };
             // Issue whichever is ready first: O(next_o) once its P is in TMEM and the epilogue of tile
             // next_o - 2 has read O buffer b, or S(next_s) once its operands have landed and O(next_s - 2)

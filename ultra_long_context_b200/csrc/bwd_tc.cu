@@ -323,7 +323,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
         cp_async_wait<0>();
     } else if (warp == kBtMmaWarp) {
         // ================= MMA issuer =================
-        if (lane == 0 && mine > 0) {
+        if (mine > 0) {  // the whole warp runs the issue loop; one elected lane issues (tc::*_w)
             constexpr uint32_t id_s = tc::idesc_bf16(128, 64, 0, 0);   // S, dP': A, B K-major
             constexpr uint32_t id_q = tc::idesc_bf16(128, D, 0, 1);    // dQ: A K-major, B (K) MN-major
             constexpr uint32_t id_t = tc::idesc_bf16(128, 64, 1, 1);   // dK^T, dV^T: A, B MN-major (M = D, or
@@ -340,22 +340,22 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                     const uint32_t sq = sb + SM::STG + st * SM::QD, sdo = sq + 2 * SM::HALF;
 #pragma unroll 1
                     for (int ks = 0; ks < kChunk / 16; ++ks)  // dQ = dS K: K = 64 keys
-                        tc::mma_bf16_ss(tmem + SM::DQ_COL + st * 128, tc::desc_kmajor(sb + SM::DS + ks * 32),
+                        tc::mma_bf16_ss_w(tmem + SM::DQ_COL + st * 128, tc::desc_kmajor(sb + SM::DS + ks * 32),
                                         tc::desc_mnmajor(sb + SM::KO + ks * 2048, SM::KH), id_q, ks > 0 ? 1u : 0u);
                     const uint32_t acc0 = cg.first_tile() ? 0u : 1u;
 #pragma unroll 1
                     for (int ks = 0; ks < kBtTile / 16; ++ks) {  // K = the tile's 128 pairs
-                        tc::mma_bf16_ss(tmem + SM::DV_COL, tc::desc_mnmajor(sdo + ks * 2048, SM::HALF),
+                        tc::mma_bf16_ss_w(tmem + SM::DV_COL, tc::desc_mnmajor(sdo + ks * 2048, SM::HALF),
                                         tc::desc_mnmajor(sb + SM::WP + ks * 2048, 8192), id_t, ks > 0 ? 1u : acc0);
-                        tc::mma_bf16_ss(tmem + SM::DK_COL, tc::desc_mnmajor(sq + ks * 2048, SM::HALF),
+                        tc::mma_bf16_ss_w(tmem + SM::DK_COL, tc::desc_mnmajor(sq + ks * 2048, SM::HALF),
                                         tc::desc_mnmajor(sb + SM::DS + ks * 2048, 8192), id_t, ks > 0 ? 1u : acc0);
                     }
-                    tc::commit(bar(kBDqFull + st));
-                    tc::commit(bar(kBDsEmpty));
-                    tc::commit(bar(kBQdEmpty + st));
+                    tc::commit_w(bar(kBDqFull + st));
+                    tc::commit_w(bar(kBDsEmpty));
+                    tc::commit_w(bar(kBQdEmpty + st));
                     if (cg.last_tile()) {
-                        tc::commit(bar(kBAccFull));
-                        tc::commit(bar(kBKvEmpty));
+                        tc::commit_w(bar(kBAccFull));
+                        tc::commit_w(bar(kBKvEmpty));
                     }
                     cg.next();
                     progress = true;
@@ -371,12 +371,12 @@ __global__ void __launch_bounds__(kBtThreads, 1) chunk_bwd_tc_kernel(
                     for (int ks = 0; ks < D / 16; ++ks) {
                         const uint32_t koff = (uint32_t)((ks >> 2) * SM::HALF + (ks & 3) * 32);
                         const uint32_t kk = (uint32_t)((ks >> 2) * SM::KH + (ks & 3) * 32);
-                        tc::mma_bf16_ss(tmem + SM::S_COL, tc::desc_kmajor(sq + koff),
+                        tc::mma_bf16_ss_w(tmem + SM::S_COL, tc::desc_kmajor(sq + koff),
                                         tc::desc_kmajor(sb + SM::KO + kk), id_s, ks > 0 ? 1u : 0u);
-                        tc::mma_bf16_ss(tmem + SM::DP_COL, tc::desc_kmajor(sdo + koff),
+                        tc::mma_bf16_ss_w(tmem + SM::DP_COL, tc::desc_kmajor(sdo + koff),
                                         tc::desc_kmajor(sb + SM::VO + kk), id_s, ks > 0 ? 1u : 0u);
                     }
-                    tc::commit(bar(kBSFull));
+                    tc::commit_w(bar(kBSFull));
                     cs.next();
                     progress = true;
                 }

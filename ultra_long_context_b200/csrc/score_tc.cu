@@ -11,7 +11,8 @@
 // 50 KB of shared memory, so four CTAs (16 selecting warps) share an SM.
 //   * The Q tile lives in TMEM: each selecting thread loads its own row and writes it to its lane
 //     (tcgen05.st, two bf16 per column), and the MMA reads it as the A operand.
-//   * Warp 4 (one lane) is the producer: 32-landmark blocks arrive by TMA in the 128-byte-swizzled
+//   * Warp 4 is the producer (the warp runs it, one elected lane issues): 32-landmark blocks arrive by
+//     TMA in the 128-byte-swizzled
 //     layout (three stages), and it issues S_blk = Q L_blk^T (M = 128, N = 32, fp32) into one of the
 //     TMEM score buffers. Full/empty mbarriers link it to warps 0-3, which run decoupled.
 //   * Scores are compared unscaled (the scale is positive, so the order is the same); it enters the
@@ -151,15 +152,15 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
     bool ok = true;
 
     if (warp == kStConsumers / 32) {
-        // ---------------- producer ----------------
-        if (lane == 0) {
+        // ---------------- producer: the whole warp runs it, one elected lane issues (tc::*_w) ----------------
+        {
             auto load_l = [&](int h) {  // landmark block h % nblk into stage h % 3
                 const int st = h % kStLStages;
                 const uint32_t dst = sb + st * SM::LB;
-                tc::mbar_arrive_expect_tx(full_l(st), SM::LB);
+                tc::mbar_arrive_expect_tx_w(full_l(st), SM::LB);
 #pragma unroll
                 for (int k = 0; k < SM::KH; ++k)
-                    tc::tma_load_2d(dst + k * SM::LH, &tmL, k * 64, kvh * N + (h % nblk) * kStCols, full_l(st));
+                    tc::tma_load_2d_w(dst + k * SM::LH, &tmL, k * 64, kvh * N + (h % nblk) * kStCols, full_l(st));
             };
             int nload = 0, nmma = 0;
             for (; nload < kStLStages && nload < G; ++nload) load_l(nload);
@@ -176,10 +177,10 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
                 const uint32_t lb = sb + st * SM::LB;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)  // K step of 16: 8 TMEM columns of Q, 32 B of a swizzled row
-                    tc::mma_bf16_ts(tmem + SM::QCOLS + buf * kStCols, tmem + ks * 8,
+                    tc::mma_bf16_ts_w(tmem + SM::QCOLS + buf * kStCols, tmem + ks * 8,
                                     tc::desc_kmajor(lb + (ks >> 2) * SM::LH + (ks & 3) * 32), idesc, ks > 0 ? 1u : 0u);
-                tc::commit(full_s(buf));
-                tc::commit(empty_l(st));
+                tc::commit_w(full_s(buf));
+                tc::commit_w(empty_l(st));
                 nmma = g + 1;
                 if (g + kStLStages < G) {  // refill this stage once MMA(g) has read it
                     if (!tc::mbar_wait(empty_l(st), (uint32_t)(g / kStLStages) & 1u)) {

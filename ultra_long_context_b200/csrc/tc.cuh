@@ -61,6 +61,35 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
+// Whole-warp forms: every lane of the warp runs the issuing code, so descriptors and addresses stay
+// warp-uniform values (no per-instruction moves into uniform registers, which made a single issuing
+// lane slow), and one lane chosen by elect.sync issues. All 32 lanes must execute them, converged, and
+// a warp must keep issuing and committing through these forms (the elected lane is then always the
+// same one, which commit's tracking of "this thread's" operations relies on).
+__device__ __forceinline__ void mma_bf16_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void mma_bf16_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void commit_w(uint32_t mbar) {
+    asm volatile("{\n\t.reg .pred e;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(mbar)
+                 : "memory");
+}
 __device__ __forceinline__ void commit(uint32_t mbar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
                  : "memory");
@@ -250,6 +279,23 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int 
             dst),
         "l"(tmap), "r"(x), "r"(y), "r"(mbar)
         : "memory");
+}
+// Whole-warp forms (see mma_bf16_ss_w): every lane executes, one elected lane acts.
+__device__ __forceinline__ void tma_load_2d_w(uint32_t dst, const void *tmap, int x, int y, uint32_t mbar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];\n\t}\n" ::"r"(dst),
+        "l"(tmap), "r"(x), "r"(y), "r"(mbar)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_w(uint32_t mbar, uint32_t bytes) {
+    asm volatile("{\n\t.reg .pred e;\n\t.reg .b64 st;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "@e mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}\n" ::"r"(mbar),
+                 "r"(bytes)
+                 : "memory");
 }
 // Prefetch a 2D tile of a tensor map into L2 (no shared memory, no completion to wait for).
 __device__ __forceinline__ void tma_prefetch_2d(const void *tmap, int x, int y) {

@@ -64,10 +64,10 @@ struct StSmem {
     static constexpr uint32_t STAGE = 128 * (K + 1) * 8;              // output staging: idx + w, padded rows
     // region U holds the landmark stages during the loop and the output staging at the end
     static constexpr uint32_t U = kStLStages * LB > STAGE ? kStLStages * LB : STAGE;
-    // [33][128] fp32: a block's scores, one column per thread; [K+1][128] int32: the chunk of each
-    // output slot.
+    // [128][36] fp32: a block's scores, one padded row per thread (16-byte stores without bank
+    // conflicts); [K+1][128] int32: the chunk of each output slot.
     static constexpr uint32_t CV = U;
-    static constexpr uint32_t CC = CV + 33 * 128 * 4;
+    static constexpr uint32_t CC = CV + 128 * 36 * 4;
     static constexpr uint32_t HIST = CC + (K + 1) * 128 * 4;  // int[kStHistMax]: selected pairs per chunk
     static constexpr uint32_t BAR = HIST + kStHistMax * 4;  // q_ready, full_l[3], empty_l[3], full_s[NB], empty_s[NB]
     static constexpr int NBAR = 1 + 2 * kStLStages + 2 * NB;
@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
         }
 
         // Scores are compared unscaled (scale > 0 keeps their order); the scale enters the weights only.
-        float *cv = reinterpret_cast<float *>(s + SM::CV) + tid;  // this thread's column: a block's scores
+        float *cv = reinterpret_cast<float *>(s + SM::CV) + tid * 36;  // this thread's row: a block's scores
         int *cc = reinterpret_cast<int *>(s + SM::CC) + tid;      // chunk of each output slot
         float ls[K];  // pass 1: the K largest score values of this row, descending
 #pragma unroll
@@ -294,26 +294,23 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
             // every score of the block to this thread's column; one bit per candidate
             // the mask is built in four independent parts (no 32-long dependency chain through one register)
             uint32_t mp[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                reinterpret_cast<float4 *>(cv)[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
             if (g < nblk) {  // warp-uniform
                 const float thr = ls[K - 1];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    cv[128 * i] = v[i];
-                    mp[i & 3] |= v[i] > thr ? 1u << i : 0u;
-                }
+                for (int i = 0; i < 32; ++i) mp[i & 3] |= v[i] > thr ? 1u << i : 0u;
             } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    cv[128 * i] = v[i];
-                    mp[i & 3] |= v[i] >= tau ? 1u << i : 0u;
-                }
+                for (int i = 0; i < 32; ++i) mp[i & 3] |= v[i] >= tau ? 1u << i : 0u;
             }
             uint32_t m = ((mp[0] | mp[1]) | (mp[2] | mp[3])) & valid;
             if (g < nblk) {  // pass 1: insert the candidates that still beat the K-th value
                 while (m) {
                     const int i = __ffs(m) - 1;
                     m &= m - 1;
-                    const float x = cv[128 * i];
+                    const float x = cv[i];
                     if (x > ls[K - 1]) {
 #pragma unroll
                         for (int j = K - 1; j > 0; --j) ls[j] = fmaxf(ls[j], fminf(ls[j - 1], x));
@@ -324,7 +321,7 @@ __global__ void __launch_bounds__(kStThreads) score_topk_tc_kernel(const uint16_
                 while (m) {
                     const int i = __ffs(m) - 1;
                     m &= m - 1;
-                    const float x = cv[128 * i];
+                    const float x = cv[i];
                     const bool eq = !(x > tau);
                     if (eq && need_eq <= 0) continue;
                     need_eq -= eq ? 1 : 0;

@@ -221,8 +221,9 @@ def test_decode_matches_oracle(oracle_mod, B, H, D, Tmax, lens, topk):
             assert torch.all(idx[b, :, 0] == int(needle[b]))
 
 
-def test_decode_equals_forward_last_row():
-    B, H, T, D, topk = 2, 2, 4096 + 64, 128, 16
+@pytest.mark.parametrize("T,D,topk", [(4096 + 64, 128, 16), (64 * 150 + 64, 64, 64)])
+def test_decode_equals_forward_last_row(T, D, topk):
+    B, H = 2, 2
     Q, K, V, L = inputs.forward_inputs(B, H, T, D, 11, device=DEV)
     out, idx, w = hsa.hsa_forward(Q, K, V, L, topk)
     lens = torch.full((B,), T, dtype=torch.int64, device=DEV)

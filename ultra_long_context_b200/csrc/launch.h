@@ -85,6 +85,8 @@ struct ForwardArgs {
 size_t forward_max_tiles(int B, int H, int T, int topk);
 // Step 2 scores + top-K + fusion weights on the tcgen05 tensor cores (score_tc.cu).
 cudaError_t launch_score_tc(const ForwardArgs &a, cudaStream_t s);
+// K <= 16: the persistent scoring kernel (score_wide.cu); cudaErrorInvalidValue for larger K.
+cudaError_t launch_score_wide(const ForwardArgs &a, cudaStream_t s);
 // Step 3 + blend on the tcgen05 tensor cores (attn_tc.cu); tiles of up to 128 pairs.
 cudaError_t launch_attn_tc(const ForwardArgs &a, cudaStream_t s);
 cudaError_t launch_forward(const ForwardArgs &a, cudaStream_t s);

@@ -428,7 +428,7 @@ cudaError_t launch_forward(const ForwardArgs &a0, cudaStream_t s) {
         e = zero_dispatch_state(a.err, a.chunk_count, a.chunk_cursor, chunks, s);
     }
     if (e != cudaSuccess) return e;
-    e = launch_score_tc(a, s);
+    e = a.topk <= 16 ? launch_score_wide(a, s) : launch_score_tc(a, s);
     if (e != cudaSuccess) return e;
     if (a.N == 0) {
         HSA_PROF("finalize", s);

@@ -48,7 +48,8 @@ constexpr int kSwLoaderWarp = 16;  // warps 0-15 select
 constexpr int kSwMmaWarp = 17;
 constexpr int kSwZeroWarp = 18;
 constexpr int kSwThreads = 32 * (kSwZeroWarp + 1);  // 608
-constexpr int kSwHist = 2048;   // chunks per (b, h) counted in shared memory
+constexpr int kSwSlot = 32;     // key slot stride: slot j of a lane at [j * 32] of its half's slots
+constexpr int kSwHist = 1024;   // chunks per (b, h) counted in shared memory (per tile, two buffers)
 
 template <int D, int K>
 struct SwSmem {
@@ -60,18 +61,24 @@ struct SwSmem {
     static constexpr uint32_t QT = KH * QH;             // one Q tile
     static constexpr uint32_t LST = 0;                  // landmark stages
     static constexpr uint32_t QST = LST + kSwStages * LB;  // Q staging: two tiles
-    static constexpr uint32_t CAND = QST + 2 * QT;      // u64 keys [tile][half][K][128 rows]
-    static constexpr uint32_t HIST = CAND + NG * kSwItem * 8;  // int[kSwHist]
-    // l_full[4], l_empty[4], q_sfull[2], q_sempty[2], q_tfull[2], s_full[2][2], s_empty[2][2]
+    // u64 keys [pair][half][K][32 lanes]; a pair is the two warps (one per column half) that share 32
+    // rows, and its region also holds the swapped group maxima before pass 2
+    static constexpr uint32_t PAIR = 2 * K * kSwSlot * 8;
+    static constexpr uint32_t CAND = QST + 2 * QT;
+    static constexpr uint32_t HIST = CAND + 8 * PAIR;   // int[tile][2 buffers][kSwHist]
+    static constexpr uint32_t HIST_BYTES = 4 * kSwHist * 4;
+    // l_full[4], l_empty[4], q_sfull[2], q_sempty[2], q_tfull[2], s_full[2][2], s_empty[2][2],
+    // h_full[2][2], h_free[2][2]
     // pass 2's score scratch of each tile, float [32][256 threads]: a tile's Q staging (32 KB at
     // D = 128) is free between the copy of the next item's Q and the end of that tile's pass 2; at
     // D = 64 it is too small and the scratch has its own region
     static constexpr uint32_t SCR_TILE = 32 * 256 * 4;
     static constexpr bool SCR_IN_Q = QT >= SCR_TILE;
-    static constexpr uint32_t SCR = SCR_IN_Q ? QST : HIST + kSwHist * 4;
+    static constexpr uint32_t SCR = SCR_IN_Q ? QST : HIST + HIST_BYTES;
     static constexpr uint32_t SCR_STRIDE = SCR_IN_Q ? QT : SCR_TILE;  // tile u at SCR + u * SCR_STRIDE
-    static constexpr uint32_t BAR = SCR_IN_Q ? HIST + kSwHist * 4 : SCR + 2 * SCR_TILE;
-    static constexpr int NBAR = 2 * kSwStages + 6 + 8;
+    static constexpr uint32_t BAR = SCR_IN_Q ? HIST + HIST_BYTES : SCR + 2 * SCR_TILE;
+    // + h_full[tile][buffer], h_free[tile][buffer]
+    static constexpr int NBAR = 2 * kSwStages + 6 + 8 + 8;
     static constexpr uint32_t TMEM = BAR + NBAR * 8;
     static constexpr uint32_t BYTES = TMEM + 16;
     static constexpr size_t DYN = BYTES + 1024;
@@ -108,7 +115,7 @@ __device__ __forceinline__ int sw_nmax(int r0, int n, int Tv, int N) {
 }
 
 // This half's key slots once more than K keys have reached tau0: the K largest so far are kept (slot j
-// at buf[j * 128]); kmin is the smallest of them and kslot its slot (kmin 0: not yet computed -- valid
+// at buf[j * kSwSlot]); kmin is the smallest of them and kslot its slot (kmin 0: not yet computed -- valid
 // keys are never 0). Rare: only rows whose half has more than K scores at or above tau0.
 struct SwHalf {
     int cnt;
@@ -122,7 +129,7 @@ __device__ __noinline__ SwHalf sw_keep_slow(const float *v, int sw, uint32_t m, 
         h.kmin = buf[0];
         h.kslot = 0;
         for (int j = 1; j < K; ++j) {
-            const uint64_t x = buf[j * 128];
+            const uint64_t x = buf[j * kSwSlot];
             if (x < h.kmin) {
                 h.kmin = x;
                 h.kslot = j;
@@ -134,16 +141,16 @@ __device__ __noinline__ SwHalf sw_keep_slow(const float *v, int sw, uint32_t m, 
         m &= m - 1;
         const uint64_t key = make_key(v[(((i >> 2) ^ sw) << 2) + (i & 3)], (uint32_t)(c0 + i));
         if (h.cnt < K) {
-            buf[h.cnt * 128] = key;
+            buf[h.cnt * kSwSlot] = key;
             if (++h.cnt < K) continue;
         } else {
             if (key <= h.kmin) continue;
-            buf[h.kslot * 128] = key;
+            buf[h.kslot * kSwSlot] = key;
         }
         h.kmin = buf[0];  // the full slots' minimum
         h.kslot = 0;
         for (int j = 1; j < K; ++j) {
-            const uint64_t x = buf[j * 128];
+            const uint64_t x = buf[j * kSwSlot];
             if (x < h.kmin) {
                 h.kmin = x;
                 h.kslot = j;
@@ -187,14 +194,18 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
     auto q_tfull = [&](int u) { return bar(2 * kSwStages + 4 + u); };
     auto s_full = [&](int u, int b) { return bar(2 * kSwStages + 6 + 2 * u + b); };
     auto s_empty = [&](int u, int b) { return bar(2 * kSwStages + 10 + 2 * u + b); };
-    int *s_hist = reinterpret_cast<int *>(s + SM::HIST);
+    auto h_full = [&](int u, int b) { return bar(2 * kSwStages + 14 + 2 * u + b); };
+    auto h_free = [&](int u, int b) { return bar(2 * kSwStages + 18 + 2 * u + b); };
+    // pair counts per chunk of an item, per tile, double-buffered by item: the selectors add, the zero
+    // warp adds the buffer into the dispatch's counts and clears it
+    auto hist = [&](int u, int b) { return reinterpret_cast<int *>(s + SM::HIST) + (2 * u + b) * kSwHist; };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = gridDim.x, cta = blockIdx.x;
     const int P = (T + kSwItem - 1) / kSwItem;
     auto seq_len = [&](int bh) { return cu_seqlens ? min(T, cu_seqlens[bh / H + 1] - cu_seqlens[bh / H]) : T; };
 
-    for (int i = tid; i < kSwHist; i += kSwThreads) s_hist[i] = 0;
+    for (int i = tid; i < 4 * kSwHist; i += kSwThreads) hist(0, 0)[i] = 0;
     if (warp == kSwMmaWarp) tc::tmem_alloc(sb + SM::TMEM, SM::NCOLS);
     if (tid == 0) {
         for (int i = 0; i < kSwStages; ++i) {
@@ -208,6 +219,8 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
             for (int b = 0; b < 2; ++b) {
                 tc::mbar_init(s_full(u, b), 1);
                 tc::mbar_init(s_empty(u, b), 8);
+                tc::mbar_init(h_full(u, b), 8);
+                tc::mbar_init(h_free(u, b), 1);
             }
         }
         tc::fence_mbar_init();
@@ -315,26 +328,50 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
         __syncwarp();
     } else if (warp == kSwZeroWarp) {
         // ---------------- the items' rows of the fp32 output accumulator start at zero ----------------
-        SwItem it = sw_item(0, G, cta, P, BH);
-        for (int k = 0; it.valid; ++k) {
+        // it also adds each finished item's per-chunk pair counts into the dispatch's counts, one item
+        // behind the zeroing
+        auto flush = [&](int kk, const SwItem &f) {
+            const int nmax = min(kSwHist, sw_nmax(f.t0, kSwItem, seq_len(f.bh), N));
+            for (int u = 0; u < 2 && ok; ++u) {
+                ok = tc::mbar_wait(h_full(u, kk & 1), (uint32_t)(kk >> 1) & 1u);
+                if (!ok) break;
+                int *hb = hist(u, kk & 1);
+                for (int i = lane; i < nmax; i += 32) {
+                    const int x = hb[i];
+                    if (x) {
+                        atomicAdd(&chunk_count[(size_t)f.bh * N + i], x);
+                        hb[i] = 0;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(h_free(u, kk & 1));
+            }
+        };
+        SwItem it = sw_item(0, G, cta, P, BH), prev{0, 0, false};
+        int k = 0;
+        for (; it.valid && ok; ++k) {
             const int nv = max(0, min(kSwItem, min(T, seq_len(it.bh)) - it.t0));
             float4 *acc = reinterpret_cast<float4 *>(o_acc + ((size_t)it.bh * T + it.t0) * D);
             for (int i = lane; i < nv * (D / 4); i += 32) acc[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (k > 0) flush(k - 1, prev);
+            prev = it;
             it = sw_item(k + 1, G, cta, P, BH);
         }
+        if (ok && k > 0) flush(k - 1, prev);
     } else {
         // ---------------- selectors: tile u, column half hf of each block, one token row per thread pair ----------------
         const int u = warp >> 3, hf = (warp >> 2) & 1, r = (warp & 3) * 32 + lane;
-        const int bar_tile = 2 + u;  // named barrier of this tile's 256 selectors
+        const int pair = u * 4 + (warp & 3);
+        const int bar_pair = 1 + pair;  // named barrier of the two warps of this row range (64 threads)
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        // this half's K key slots (slot j at [j * 128]); the partner's; and, aliasing them before pass 2,
-        // the sorted group maxima (float, j at [j * 128])
-        uint64_t *kb = reinterpret_cast<uint64_t *>(s + SM::CAND) + (size_t)((u * 2 + hf) * K) * kSwRows + r;
-        const uint64_t *kb_o = reinterpret_cast<const uint64_t *>(s + SM::CAND) + (size_t)((u * 2 + (hf ^ 1)) * K) * kSwRows + r;
-        // (inside this tile's own key slots: the other tile is not synchronised with this one)
-        float *gx = reinterpret_cast<float *>(s + SM::CAND) + (size_t)u * 4 * K * kSwRows + (size_t)(hf * K) * kSwRows + r;
-        const float *gx_o =
-            reinterpret_cast<const float *>(s + SM::CAND) + (size_t)u * 4 * K * kSwRows + (size_t)((hf ^ 1) * K) * kSwRows + r;
+        // the pair's region: this half's K key slots (slot j at [j * 32]) and the partner's; before pass
+        // 2 the same bytes hold the swapped, sorted group maxima (float, j at [j * 32]). Only the pair
+        // touches its region, so two named-barrier steps of the pair order every access.
+        unsigned char *preg = s + SM::CAND + pair * SM::PAIR;
+        uint64_t *kb = reinterpret_cast<uint64_t *>(preg) + hf * K * kSwSlot + lane;
+        const uint64_t *kb_o = reinterpret_cast<const uint64_t *>(preg) + (hf ^ 1) * K * kSwSlot + lane;
+        float *gx = reinterpret_cast<float *>(preg) + hf * K * kSwSlot + lane;
+        const float *gx_o = reinterpret_cast<const float *>(preg) + (hf ^ 1) * K * kSwSlot + lane;
         uint32_t gs = 0;  // score blocks taken so far
         // this thread's half of the row of Q of item kk from the staging into TMEM (item parity kk & 1)
         auto copy_q = [&](int kk, bool release) -> bool {
@@ -442,18 +479,18 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
                         }
                     }
 #pragma unroll
-            for (int j = 0; j < K; ++j) gx[j * kSwRows] = gm[j];
-            asm volatile("bar.sync %0, 256;" ::"r"(bar_tile) : "memory");
+            for (int j = 0; j < K; ++j) gx[j * kSwSlot] = gm[j];
+            asm volatile("bar.sync %0, 64;" ::"r"(bar_pair) : "memory");
             float tmin = INFINITY;
 #pragma unroll
-            for (int j = 0; j < K; ++j) tmin = fminf(tmin, fmaxf(gm[j], gx_o[(K - 1 - j) * kSwRows]));
+            for (int j = 0; j < K; ++j) tmin = fminf(tmin, fmaxf(gm[j], gx_o[(K - 1 - j) * kSwSlot]));
             const float tau0 = my_n > K ? tmin : -INFINITY;
             // the next item's Q into TMEM, while this one's second pass runs
             const SwItem nx = sw_item(k + 1, G, cta, P, BH);
             if (ok && nx.valid && !copy_q(k + 1, false)) ok = false;
-            // every thread of the tile has read its partner's maxima (the key slots reuse them) and its
-            // next row of Q (pass 2's scratch reuses the staging)
-            asm volatile("bar.sync %0, 256;" ::"r"(bar_tile) : "memory");
+            // the partner has read these maxima before the key slots reuse them (pass 2's scratch is this
+            // thread's own part of the staging: the 16-byte chunks of its own row of Q, just copied)
+            asm volatile("bar.sync %0, 64;" ::"r"(bar_pair) : "memory");
 
             // pass 2: this half's K largest keys among the scores >= tau0
             SwHalf hs{0, 0ull, 0};
@@ -484,7 +521,7 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
                     while (m) {
                         const int i = __ffs(m) - 1;
                         m &= m - 1;
-                        kb[(pos++) * kSwRows] = make_key(*scr_at(i), (uint32_t)(c0 + i));
+                        kb[(pos++) * kSwSlot] = make_key(*scr_at(i), (uint32_t)(c0 + i));
                     }
                     hs.cnt = pos;
                 } else {
@@ -501,7 +538,7 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
             // the union come out of one bitonic merge (both threads of the row hold all K)
             uint64_t a[K];
 #pragma unroll
-            for (int j = 0; j < K; ++j) a[j] = j < hs.cnt ? kb[j * kSwRows] : 0ull;
+            for (int j = 0; j < K; ++j) a[j] = j < hs.cnt ? kb[j * kSwSlot] : 0ull;
 #pragma unroll
             for (int kk = 2; kk <= K; kk <<= 1)
 #pragma unroll
@@ -517,11 +554,11 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
                         }
                     }
 #pragma unroll
-            for (int j = 0; j < K; ++j) kb[j * kSwRows] = a[j];
-            asm volatile("bar.sync %0, 256;" ::"r"(bar_tile) : "memory");
+            for (int j = 0; j < K; ++j) kb[j * kSwSlot] = a[j];
+            asm volatile("bar.sync %0, 64;" ::"r"(bar_pair) : "memory");
 #pragma unroll
             for (int j = 0; j < K; ++j) {
-                const uint64_t o = kb_o[(K - 1 - j) * kSwRows];
+                const uint64_t o = kb_o[(K - 1 - j) * kSwSlot];
                 a[j] = a[j] > o ? a[j] : o;
             }
 #pragma unroll
@@ -535,6 +572,10 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
                         a[l] = lo;
                     }
                 }
+            // the item's histogram buffer was added in by the zero warp two items ago
+            int *hb = hist(u, k & 1);
+            if (ok && k >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(h_free(u, k & 1), (uint32_t)((k >> 1) - 1) & 1u)))
+                ok = false;
             if (ok && t < min(T, Tv)) {
                 // fusion weights (Step 4): softmax of the kept scores, fp32, max-subtracted; this thread
                 // writes slots K/2 hf .. K/2 hf + K/2 - 1
@@ -561,7 +602,7 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
                     ci[i] = kept ? key_index(ak) : -1;
                     wi[i] = kept ? ek * rz : 0.0f;
                     if (kept) {
-                        if (ci[i] < kSwHist) atomicAdd(&s_hist[ci[i]], 1);
+                        if (ci[i] < kSwHist) atomicAdd(&hb[ci[i]], 1);
                         else atomicAdd(&chunk_count[(size_t)it.bh * N + ci[i]], 1);
                     }
                 }
@@ -584,17 +625,11 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
                     }
                 }
             }
-            // the item's pair counts into the dispatch's histogram
-            asm volatile("bar.sync 1, 512;" ::: "memory");
-            const int nmax = min(kSwHist, sw_nmax(it.t0, kSwItem, Tv, N));
-            for (int i = tid; i < nmax; i += 512) {
-                const int x = s_hist[i];
-                if (x) {
-                    atomicAdd(&chunk_count[(size_t)it.bh * N + i], x);
-                    s_hist[i] = 0;
-                }
-            }
-            ok = bar_and(1, 512, ok);
+            // this warp's counts are in: the zero warp may add the buffer once all 8 warps of the tile are
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(h_full(u, k & 1));
+            // the pair agrees on the outcome and stops together (its named barriers stay matched)
+            ok = bar_and(bar_pair, 64, ok);
             if (!ok) break;
             it = nx;
         }

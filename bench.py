@@ -181,7 +181,7 @@ def kernel_profile(fn, steps):
 # current kernels on these workloads; set back to None whenever the kernel changes.
 TRAFFIC_BYTES = {
     ("fwd_t32k_h8_d128_k16", "chunk_attn"): 737_926_144 + 235_332_096,
-    ("fwd_t32k_h8_d128_k16", "score_topk"): None,  # the persistent kernel: not yet captured
+    ("fwd_t32k_h8_d128_k16", "score_topk"): 136_467_456 + 279_436_032,
     ("decode_16m_b1_h8_d128_k32", "decode_scan"): 536_948_992 + 3_297_792,
     ("fwdbwd_t64k_h8_d128_k16", "chunk_bwd"): 2_288_028_416 + 1_252_866_048,
 }

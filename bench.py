@@ -160,6 +160,15 @@ def timed(fn, steps, warmup, world):
     return max_over_ranks(e0.elapsed_time(e1), world)
 
 
+def clean(*workspaces):
+    """Raise if a bounded device wait of the last call on any of these workspaces ran out (a timed number
+    from such a run would be meaningless)."""
+    from ultra_long_context_b200 import hsa
+
+    for ws in workspaces:
+        hsa.hsa_workspace_status(ws)
+
+
 def kernel_profile(fn, steps):
     """Per-launch-site device time over `steps` calls, from the library's event hooks."""
     import torch
@@ -308,6 +317,7 @@ def decode_entry(hsa, inputs, wd, dev, steps, warmup, world, peaks, peak_kind, c
         hsa.hsa_decode(q, Kc, Vc, Lc, lens, wd.topk, out=dout_, sel_idx=didx, sel_w=dw, workspace=dws)
 
     dms = timed(dec, steps, warmup, world) / steps
+    clean(dws)
     prof = kernel_profile(dec, steps)
     n = wd.cache_len // 64
     scan_bytes = wd.B * wd.H * (n * wd.D * 2 + wd.D * 2)
@@ -460,6 +470,7 @@ def main():
             hsa.hsa_forward(Q, K, V, L, w.topk, out=out, sel_idx=sel_idx, sel_w=sel_w, workspace=ws)
 
         ms = timed(fwd, args.steps, args.warmup, world)
+        clean(ws)
         ms_per_step = ms / args.steps
         tokens = w.B * w.T
         value = whole_job_rate(tokens, world, ms_per_step)
@@ -553,6 +564,7 @@ def main():
             hsa.hsa_forward(Q, K, V, L, w.topk, out=out, sel_idx=sel_idx, sel_w=sel_w, workspace=ws_n, qk_norm=True)
 
         n_ms = timed(fwd_norm, osteps, args.warmup, world) / osteps
+        clean(ws_n)
         prof_n = kernel_profile(fwd_norm, osteps)
         norm_bytes = 2 * (2 * w.B * w.H * w.T * w.D * 2)  # read Q and K, write their normalised copies
         opts["qk_norm"] = {
@@ -567,6 +579,7 @@ def main():
             hsa.hsa_forward(Q, K, V, L, w.topk, out=out, sel_idx=sel_idx, sel_w=sel_w, workspace=ws, Qs=Qs_)
 
         s_ms = timed(fwd_qs, osteps, args.warmup, world) / osteps
+        clean(ws)
         opts["separate_retrieval_query"] = {
             "ms_per_step": round(s_ms, 4), "tokens_per_s": round(whole_job_rate(w.B * w.T, world, s_ms), 1),
             "vs_plain": round(s_ms / ms_per_step, 4)}
@@ -582,6 +595,7 @@ def main():
             hsa.hsa_forward(Q, K, V, L, k64, out=out, sel_idx=idx_64, sel_w=w_64, workspace=ws_64)
 
         k_ms = timed(fwd_k64, osteps, args.warmup, world) / osteps
+        clean(ws_64)
         prof_k = kernel_profile(fwd_k64, osteps)
         pairs_64 = pairs_closed_form(w, k64)
         opts["topk_64"] = {
@@ -608,6 +622,7 @@ def main():
             hsa.hsa_forward(gQ, gK, gV, gL, w.topk, out=gout, sel_idx=gidx, sel_w=gw, workspace=gws)
 
         g_ms = timed(fwd_gqa, osteps, args.warmup, world) / osteps
+        clean(gws)
         prof_g = kernel_profile(fwd_gqa, osteps)
         opts["grouped_heads_16to1"] = {
             "shape": f"B{Bg} H{Hg} Hkv{Hkv_g} T{w.T} D{w.D} topk{w.topk}", "ms_per_step": round(g_ms, 4),
@@ -638,6 +653,7 @@ def main():
                                        workspace=vws)
 
             v_ms = timed(fwd_var, osteps, args.warmup, world) / osteps
+            clean(vws)
             prof_v = kernel_profile(fwd_var, osteps)
             opts[name] = {"lengths": lens, "ms_per_step": round(v_ms, 4),
                           "tokens_per_s": round(whole_job_rate(sum(lens), world, v_ms), 1),
@@ -668,6 +684,7 @@ def main():
 
         steps1 = max(args.steps, 50)
         ms1 = timed(fwd1_cold, steps1, args.warmup, world) / steps1
+        clean(ws1)
         fl_ms = timed(lambda: flush.zero_(), steps1, args.warmup, world) / steps1
         ms1_fwd = max(1e-6, ms1 - fl_ms)
         prof1 = kernel_profile(fwd1_cold, steps1)
@@ -741,6 +758,7 @@ def main():
                 hsa.hsa_decode(q, Kc, Vc, Lc, lens, wd.topk, out=dout_, sel_idx=didx, sel_w=dw, workspace=dws)
 
             dms = timed(dec, dsteps, args.warmup, world) / dsteps
+            clean(dws)
             prof_dec = kernel_profile(dec, dsteps)
             scan_bytes = wd.B * wd.H * (n * wd.D * 2 + wd.D * 2)
             gather_bytes = wd.B * wd.H * wd.topk * 2 * 64 * wd.D * 2
@@ -776,6 +794,7 @@ def main():
                     hsa.hsa_decode(mq, Kc, Vc, Lc, lens, wd.topk, out=mout, sel_idx=midx, sel_w=mw, workspace=mws)
 
                 mms = timed(dec_multi, dsteps, args.warmup, world) / dsteps
+                clean(mws)
                 prof_m = kernel_profile(dec_multi, dsteps)
                 extra["decode_16m"]["multi_token_4"] = {
                     "shape": f"B{wd.B} H{wd.H} Tq{Tq} cache {wd.cache_len} D{wd.D} topk{wd.topk}",
@@ -799,6 +818,7 @@ def main():
                 hsa.hsa_decode(gq, gKc, gVc, gLc, glens, wd.topk, out=gout_, sel_idx=gidx_, sel_w=gw_, workspace=gdws)
 
             gms = timed(dec_gqa, dsteps, args.warmup, world) / dsteps
+            clean(gdws)
             prof_gd = kernel_profile(dec_gqa, dsteps)
             lm_bytes = wd.B * (n * wd.D * 2)  # one landmark head, read once from HBM at best
             extra.setdefault("decode_16m", {})["grouped_heads_16to1"] = {
@@ -831,6 +851,7 @@ def main():
 
         bsteps = max(3, args.steps // 2)
         bms = timed(fwdbwd, bsteps, args.warmup, world) / bsteps
+        clean(fws, bws)
         prof_b = kernel_profile(fwdbwd, bsteps)
         sf, af, bpairs = forward_work(wb, bidx)
         bwd_flops = 10.0 * 64 * wb.D * bpairs
@@ -855,6 +876,7 @@ def main():
                 hsa.hsa_backward(bQ, bK, bV, bL, bout, bdO, bidx, bw, grads=grads, workspace=bws_n, qk_norm=True)
 
             nms = timed(fwdbwd_norm, bsteps, args.warmup, world) / bsteps
+            clean(fws_n, bws_n)
             prof_bn = kernel_profile(fwdbwd_norm, bsteps)
             extra["fwdbwd_64k"]["qk_norm"] = {
                 "ms_per_step": round(nms, 4), "vs_plain": round(nms / bms, 4),

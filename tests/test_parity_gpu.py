@@ -647,6 +647,9 @@ def varlen_batch(lens, H, Hkv, D, seed, separate=False):
     ([1000, 64, 30, 2500, 700], 4, 2, 128, 8, {}),
     ([600, 129, 1700], 2, 2, 64, 16, {"qk_norm": True, "separate": True}),
     ([40, 20], 2, 1, 128, 4, {}),                    # no sequence has a complete chunk
+    # one long sequence among short ones, padded to its length: most of the scoring kernel's work items
+    # (256 rows of one head) lie past their sequence's end, in long runs per CTA
+    ([16384] + [100] * 7, 2, 2, 128, 16, {}),
 ])
 def test_forward_varlen_matches_per_sequence_oracle(oracle_mod, lens, H, Hkv, D, topk, opts):
     sep, qk = opts.get("separate", False), opts.get("qk_norm", False)

@@ -1,7 +1,7 @@
 // api.cu -- the C ABI declared in include/hsa.h: host-side validation, workspace carving and
 // launches on the caller's stream. Nothing here allocates device memory or computes any part of the
 // operator (hsa_workspace_status alone synchronises, by its definition); every step of HSA runs in the
-// kernels of decode.cu / prefill.cu / score_tc.cu / attn_tc.cu / backward.cu / bwd_tc.cu / qknorm.cu /
+// kernels of decode.cu / prefill.cu / score_wide.cu / score_tc.cu / attn_tc.cu / backward.cu / bwd_tc.cu / qknorm.cu /
 // varlen.cu.
 #include <cmath>
 #include <cstdarg>

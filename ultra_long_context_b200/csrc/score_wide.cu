@@ -67,7 +67,7 @@ struct SwSmem {
     static constexpr uint32_t CAND = QST + 2 * QT;
     static constexpr uint32_t HIST = CAND + 8 * PAIR;   // int[tile][2 buffers][kSwHist]
     static constexpr uint32_t HIST_BYTES = 4 * kSwHist * 4;
-    // l_full[4], l_empty[4], q_sfull[2], q_sempty[2], q_tfull[2], s_full[2][2], s_empty[2][2],
+    // l_full[4], l_empty[4], q_sfull[2], q_sempty[2], two unused slots, s_full[2][2], s_empty[2][2],
     // h_full[2][2], h_free[2][2]
     // pass 2's score scratch of each tile, float [32][256 threads]: a tile's Q staging (32 KB at
     // D = 128) is free between the copy of the next item's Q and the end of that tile's pass 2; at
@@ -79,7 +79,8 @@ struct SwSmem {
     static constexpr uint32_t BAR = SCR_IN_Q ? HIST + HIST_BYTES : SCR + 2 * SCR_TILE;
     // + h_full[tile][buffer], h_free[tile][buffer]
     static constexpr int NBAR = 2 * kSwStages + 6 + 8 + 8;
-    static constexpr uint32_t TMEM = BAR + NBAR * 8;
+    static constexpr uint32_t QCNT = BAR + NBAR * 8;     // unsigned[2]: warps' Q copies into TMEM, per tile
+    static constexpr uint32_t TMEM = QCNT + 8;
     static constexpr uint32_t BYTES = TMEM + 16;
     static constexpr size_t DYN = BYTES + 1024;
     static_assert(DYN <= 227 * 1024, "shared memory budget");
@@ -191,7 +192,10 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
     auto l_empty = [&](int st) { return bar(kSwStages + st); };
     auto q_sfull = [&](int u) { return bar(2 * kSwStages + u); };
     auto q_sempty = [&](int u) { return bar(2 * kSwStages + 2 + u); };
-    auto q_tfull = [&](int u) { return bar(2 * kSwStages + 4 + u); };
+    // the selectors' copies of an item's Q into TMEM are counted in q_cnt[tile] (8 per item), not on an
+    // mbarrier: the MMA warp waits only for items whose tile has products, and a phase-parity wait that
+    // skips items can pass two phases early; a count cannot
+    unsigned *q_cnt = reinterpret_cast<unsigned *>(s + SM::QCNT);
     auto s_full = [&](int u, int b) { return bar(2 * kSwStages + 6 + 2 * u + b); };
     auto s_empty = [&](int u, int b) { return bar(2 * kSwStages + 10 + 2 * u + b); };
     auto h_full = [&](int u, int b) { return bar(2 * kSwStages + 14 + 2 * u + b); };
@@ -215,7 +219,7 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
         for (int u = 0; u < 2; ++u) {
             tc::mbar_init(q_sfull(u), 1);
             tc::mbar_init(q_sempty(u), 8);
-            tc::mbar_init(q_tfull(u), 8);
+            q_cnt[u] = 0u;
             for (int b = 0; b < 2; ++b) {
                 tc::mbar_init(s_full(u, b), 1);
                 tc::mbar_init(s_empty(u, b), 8);
@@ -286,7 +290,23 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
             const int nb0 = (sw_nmax(it.t0, kSwRows, Tv, N) + kSwCols - 1) / kSwCols;
             const int nb1 = (sw_nmax(it.t0 + kSwRows, kSwRows, Tv, N) + kSwCols - 1) / kSwCols;
             const int nblk = max(nb0, nb1);
-            ok = tc::mbar_wait(q_tfull(0), (uint32_t)k & 1u) && tc::mbar_wait(q_tfull(1), (uint32_t)k & 1u);
+            // the item's Q in TMEM, for the tiles that have products: all 8 warps of the tile have copied
+            // items 0 .. k (bounded wait on the count, acquire)
+            for (int u = 0; u < 2 && ok; ++u) {
+                if ((u ? nb1 : nb0) == 0) continue;
+                const unsigned target = 8u * (unsigned)(k + 1);
+                uint32_t probe = 0;
+                for (;;) {
+                    unsigned c;
+                    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(c) : "r"(smem_u32(&q_cnt[u])) : "memory");
+                    if (c >= target) break;
+                    if (++probe > (1u << 24)) {
+                        ok = false;
+                        break;
+                    }
+                    __nanosleep(32);
+                }
+            }
             tc::fence_after();
             for (int pass = 0; pass < 2 && ok; ++pass) {
                 for (int b = 0; b < nblk && ok; ++b) {
@@ -404,7 +424,7 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
             tc::fence_before();
             __syncwarp();
             if (lane == 0) {
-                tc::mbar_arrive(q_tfull(u));
+                asm volatile("red.release.cta.shared::cta.add.u32 [%0], 1;" ::"r"(smem_u32(&q_cnt[u])) : "memory");
                 if (release) tc::mbar_arrive(q_sempty(u));
             }
             return true;

@@ -130,8 +130,8 @@ DecLayout dec_layout(void *ws, int B, int H, int Hkv, int Tq, int64_t Tmax, int 
     const int64_t nsplit = pl.nsplit;
     const size_t BH = (size_t)B * H * Tq;  // query rows
     l.err = c.take<int32_t>(1);  // first: hsa_workspace_status reads it at offset 0
+    l.counters = c.take<unsigned>(2 * BH);  // right after the flag: launch_decode zeroes both with one memset
     l.cand = c.take<uint64_t>(BH * nsplit * topk);
-    l.counters = c.take<unsigned>(2 * BH);
     l.sel_idx = c.take<int32_t>(BH * topk);
     l.sel_w = c.take<float>(BH * topk);
     l.partial = c.take<float>(BH * topk * D);
@@ -298,11 +298,7 @@ static hsa_status decode_impl(const char *name, const hsa_bf16 *qs, const hsa_bf
     a.sel_w = sel_w ? sel_w : l.sel_w;
     a.cand = l.cand; a.counters = l.counters; a.partial = l.partial;
     a.qk_norm = qk_norm;
-    a.err = l.err;
-    // the flag is cleared so that a status query after this call reports this call (only the grouped
-    // scan has bounded waits, on its own bulk copies)
-    cudaError_t ce = cudaMemsetAsync(l.err, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
-    if (ce != cudaSuccess) return cuda_status(ce, name);
+    a.err = l.err;  // cleared by launch_decode with the counters, so a status query reports this call
     return cuda_status(hsa::launch_decode(a, static_cast<cudaStream_t>(stream)), name);
 }
 

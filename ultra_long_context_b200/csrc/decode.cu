@@ -774,6 +774,17 @@ static cudaError_t launch_decode_grouped(const DecodeArgs &a, const DecodePlan &
     return launch_attend<D>(a, dim3(a.K, rows_q), s);
 }
 
+// The per-call reset: the ticket counters and the error flag. Both workspace layouts put the counters
+// right after the flag, so one memset covers both (one graph node less per decode step).
+static cudaError_t zero_decode_state(const DecodeArgs &a, size_t rows, cudaStream_t s) {
+    char *f = reinterpret_cast<char *>(a.err), *c = reinterpret_cast<char *>(a.counters);
+    const size_t cb = 2 * rows * sizeof(unsigned);
+    if (f && c > f && (size_t)(c - f) <= 4096) return cudaMemsetAsync(f, 0, (size_t)(c - f) + cb, s);
+    cudaError_t e = cudaMemsetAsync(c, 0, cb, s);
+    if (e == cudaSuccess && f) e = cudaMemsetAsync(f, 0, sizeof(int32_t), s);
+    return e;
+}
+
 cudaError_t launch_decode(const DecodeArgs &a0, cudaStream_t s) {
     DecodeArgs a = a0;
     if (a.Hkv <= 0) a.Hkv = a.H;
@@ -784,7 +795,7 @@ cudaError_t launch_decode(const DecodeArgs &a0, cudaStream_t s) {
         cudaError_t e;
         {
             HSA_PROF("memset", s);
-            e = cudaMemsetAsync(a.counters, 0, 2 * (size_t)a.B * a.H * a.Tq * sizeof(unsigned), s);
+            e = zero_decode_state(a, (size_t)a.B * a.H * a.Tq, s);
         }
         if (e != cudaSuccess) return e;
         e = a.D == 128 ? launch_decode_grouped<128>(a, pl, s) : launch_decode_grouped<64>(a, pl, s);
@@ -798,7 +809,7 @@ cudaError_t launch_decode(const DecodeArgs &a0, cudaStream_t s) {
     cudaError_t e;
     {
         HSA_PROF("memset", s);
-        e = cudaMemsetAsync(a.counters, 0, 2 * (size_t)BH * sizeof(unsigned), s);
+        e = zero_decode_state(a, (size_t)BH, s);
     }
     if (e != cudaSuccess) return e;
     dim3 g1(nsplit, BH), g2(a.K, BH);

@@ -37,7 +37,7 @@ hsa_status fail(hsa_status st, const std::string &msg) {
 
 size_t round_up(size_t x) { return (x + 255) / 256 * 256; }
 
-// Layout inside the fixed array: error flag, candidates, ticket counters, selection (when the caller
+// Layout inside the fixed array: error flag, ticket counters, candidates, selection (when the caller
 // passes none), per-chunk partial outputs -- the scratch the decode kernels need. The number of scan
 // ranges comes from the same plan that hsa_decode's workspace and launches use (one query row per key
 // head here), so the two cannot disagree.
@@ -51,8 +51,8 @@ NoAllocLayout layout(const hsa::DecodePlan &plan, int B, int H, int D, int topk)
     NoAllocLayout l{};
     size_t off = 0;
     l.err = off;      off += round_up(sizeof(int32_t));
+    l.counters = off; off += round_up(2 * BH * sizeof(unsigned));  // after the flag: one memset clears both
     l.cand = off;     off += round_up(BH * nsplit * topk * sizeof(uint64_t));
-    l.counters = off; off += round_up(2 * BH * sizeof(unsigned));
     l.sel_idx = off;  off += round_up(BH * topk * sizeof(int32_t));
     l.sel_w = off;    off += round_up(BH * topk * sizeof(float));
     l.partial = off;  off += round_up(BH * topk * D * sizeof(float));
@@ -126,7 +126,7 @@ hsa_status hsa_decode_noalloc(const hsa_bf16 *q, const hsa_bf16 *Kc, const hsa_b
     a.sel_idx = sel_idx ? sel_idx : reinterpret_cast<int32_t *>(b + l.sel_idx);
     a.sel_w = sel_w ? sel_w : reinterpret_cast<float *>(b + l.sel_w);
     a.cand = reinterpret_cast<uint64_t *>(b + l.cand);
-    a.counters = reinterpret_cast<unsigned *>(b + l.counters);  // zeroed by launch_decode every call
+    a.counters = reinterpret_cast<unsigned *>(b + l.counters);  // zeroed (with the flag) by launch_decode
     a.partial = reinterpret_cast<float *>(b + l.partial);
     a.err = reinterpret_cast<int32_t *>(b + l.err);
     const cudaError_t e = hsa::launch_decode(a, static_cast<cudaStream_t>(stream));

@@ -456,6 +456,9 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
             const int my_n = t < Tv ? min(N, (t + 1) / kChunk) : 0;
             const int k_keep = min(kout, my_n);
             const int nbu = (sw_nmax(it.t0 + u * kSwRows, kSwRows, Tv, N) + kSwCols - 1) / kSwCols;
+            // a tile with no row inside its sequence (padded batches) skips the sorting networks; it still
+            // takes part in every hand-off and barrier of the item (the condition is the same for the pair)
+            const bool live = it.t0 + u * kSwRows < min(T, Tv);
             float v[32];
 
             // pass 1: this half's K group maxima; group j takes columns j, j + K, .. of the half
@@ -484,20 +487,22 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
             // bitonic network), swap them through shared memory, and the K largest of the union are
             // max(A[j], B[K-1-j]) (a bitonic merge step), whose minimum is tau0. With n <= K every score
             // is kept.
+            if (live) {
 #pragma unroll
-            for (int kk = 2; kk <= K; kk <<= 1)
+                for (int kk = 2; kk <= K; kk <<= 1)
 #pragma unroll
-                for (int jj = kk >> 1; jj > 0; jj >>= 1)
+                    for (int jj = kk >> 1; jj > 0; jj >>= 1)
 #pragma unroll
-                    for (int i = 0; i < K; ++i) {
-                        const int l = i ^ jj;
-                        if (l > i) {
-                            const float hi = fmaxf(gm[i], gm[l]), lo = fminf(gm[i], gm[l]);
-                            const bool desc = (i & kk) == 0;
-                            gm[i] = desc ? hi : lo;
-                            gm[l] = desc ? lo : hi;
+                        for (int i = 0; i < K; ++i) {
+                            const int l = i ^ jj;
+                            if (l > i) {
+                                const float hi = fmaxf(gm[i], gm[l]), lo = fminf(gm[i], gm[l]);
+                                const bool desc = (i & kk) == 0;
+                                gm[i] = desc ? hi : lo;
+                                gm[l] = desc ? lo : hi;
+                            }
                         }
-                    }
+            }
 #pragma unroll
             for (int j = 0; j < K; ++j) gx[j * kSwSlot] = gm[j];
             asm volatile("bar.sync %0, 64;" ::"r"(bar_pair) : "memory");
@@ -559,39 +564,43 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
             uint64_t a[K];
 #pragma unroll
             for (int j = 0; j < K; ++j) a[j] = j < hs.cnt ? kb[j * kSwSlot] : 0ull;
+            if (live) {
 #pragma unroll
-            for (int kk = 2; kk <= K; kk <<= 1)
+                for (int kk = 2; kk <= K; kk <<= 1)
 #pragma unroll
-                for (int jj = kk >> 1; jj > 0; jj >>= 1)
+                    for (int jj = kk >> 1; jj > 0; jj >>= 1)
+#pragma unroll
+                        for (int i = 0; i < K; ++i) {
+                            const int l = i ^ jj;
+                            if (l > i) {
+                                const uint64_t hi = a[i] > a[l] ? a[i] : a[l], lo = a[i] > a[l] ? a[l] : a[i];
+                                const bool desc = (i & kk) == 0;
+                                a[i] = desc ? hi : lo;
+                                a[l] = desc ? lo : hi;
+                            }
+                        }
+#pragma unroll
+                for (int j = 0; j < K; ++j) kb[j * kSwSlot] = a[j];
+            }
+            asm volatile("bar.sync %0, 64;" ::"r"(bar_pair) : "memory");
+            if (live) {
+#pragma unroll
+                for (int j = 0; j < K; ++j) {
+                    const uint64_t o = kb_o[(K - 1 - j) * kSwSlot];
+                    a[j] = a[j] > o ? a[j] : o;
+                }
+#pragma unroll
+                for (int jj = K >> 1; jj > 0; jj >>= 1)
 #pragma unroll
                     for (int i = 0; i < K; ++i) {
                         const int l = i ^ jj;
                         if (l > i) {
                             const uint64_t hi = a[i] > a[l] ? a[i] : a[l], lo = a[i] > a[l] ? a[l] : a[i];
-                            const bool desc = (i & kk) == 0;
-                            a[i] = desc ? hi : lo;
-                            a[l] = desc ? lo : hi;
+                            a[i] = hi;
+                            a[l] = lo;
                         }
                     }
-#pragma unroll
-            for (int j = 0; j < K; ++j) kb[j * kSwSlot] = a[j];
-            asm volatile("bar.sync %0, 64;" ::"r"(bar_pair) : "memory");
-#pragma unroll
-            for (int j = 0; j < K; ++j) {
-                const uint64_t o = kb_o[(K - 1 - j) * kSwSlot];
-                a[j] = a[j] > o ? a[j] : o;
             }
-#pragma unroll
-            for (int jj = K >> 1; jj > 0; jj >>= 1)
-#pragma unroll
-                for (int i = 0; i < K; ++i) {
-                    const int l = i ^ jj;
-                    if (l > i) {
-                        const uint64_t hi = a[i] > a[l] ? a[i] : a[l], lo = a[i] > a[l] ? a[l] : a[i];
-                        a[i] = hi;
-                        a[l] = lo;
-                    }
-                }
             // the item's histogram buffer was added in by the zero warp two items ago
             int *hb = hist(u, k & 1);
             if (ok && k >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(h_free(u, k & 1), (uint32_t)((k >> 1) - 1) & 1u)))

@@ -160,6 +160,26 @@ def timed(fn, steps, warmup, world):
     return max_over_ranks(e0.elapsed_time(e1), world)
 
 
+def timed_after(prep, fn, steps, warmup, world):
+    """Device time of fn alone, per step, with prep (an L2 flush) run before each step outside the timed
+    interval: a pair of CUDA events brackets each fn call on the current stream (max over ranks, ms)."""
+    import torch
+
+    for _ in range(warmup):
+        prep()
+        fn()
+    barrier(world)
+    s = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in ev:
+        prep()
+        e0.record(s)
+        fn()
+        e1.record(s)
+    barrier(world)
+    return max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps, world)
+
+
 def clean(*workspaces):
     """Raise if a bounded device wait of the last call on any of these workspaces ran out (a timed number
     from such a run would be meaningless)."""
@@ -683,17 +703,15 @@ def main():
             fwd1()
 
         steps1 = max(args.steps, 50)
-        ms1 = timed(fwd1_cold, steps1, args.warmup, world) / steps1
+        ms1_fwd = timed_after(flush.zero_, fwd1, steps1, args.warmup, world)
         clean(ws1)
-        fl_ms = timed(lambda: flush.zero_(), steps1, args.warmup, world) / steps1
-        ms1_fwd = max(1e-6, ms1 - fl_ms)
         prof1 = kernel_profile(fwd1_cold, steps1)
         sf1, af1, pairs1 = forward_work(w1, idx1)
         entry1 = {
-            "workload": w1.name, "config": forward_config(w1, world) | {"l2": "L2 flushed between steps (256 MB "
-                                                                               "write, timed apart and subtracted)"},
+            "workload": w1.name, "config": forward_config(w1, world) | {"l2": "L2 flushed before each step (256 MB "
+                                                                               "write, outside the per-step events)"},
             "tokens_per_s": round(whole_job_rate(w1.B * w1.T, world, ms1_fwd), 1), "ms_per_step": round(ms1_fwd, 5),
-            "steps": steps1, "flush_ms": round(fl_ms, 5),
+            "steps": steps1,
             "roofline": roofline_entry("chunk_attn", prof1, af1, "TFLOP/s", tensor_peak, "tensor", tensor_kind),
             "roofline_score_topk": roofline_entry("score_topk", prof1, sf1, "TFLOP/s", tensor_peak, "tensor",
                                                   tensor_kind),
@@ -714,12 +732,12 @@ def main():
         g1 = tuple(torch.empty(x.shape, dtype=torch.float32, device=dev) for x in (Q1, K1, V1, L1))
 
         def fwdbwd1():
-            flush.zero_()
             fwd1()
             hsa.hsa_backward(Q1, K1, V1, L1, out1, dO1, idx1, sw1, grads=g1, workspace=bws1)
 
-        fb_ms = max(1e-6, timed(fwdbwd1, steps1, args.warmup, world) / steps1 - fl_ms)
-        prof_fb1 = kernel_profile(fwdbwd1, steps1)
+        fb_ms = timed_after(flush.zero_, fwdbwd1, steps1, args.warmup, world)
+        clean(ws1, bws1)
+        prof_fb1 = kernel_profile(lambda: (flush.zero_(), fwdbwd1()), steps1)
         entry1["fwdbwd_d64"] = {
             "ms_per_step": round(fb_ms, 5), "tokens_per_s": round(whole_job_rate(w1.B * w1.T, world, fb_ms), 1),
             "roofline": roofline_entry("chunk_bwd", prof_fb1, 10.0 * 64 * w1.D * pairs1, "TFLOP/s", tensor_peak,

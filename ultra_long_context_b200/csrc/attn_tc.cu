@@ -125,6 +125,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) chunk_attn_tc_kernel(
     const int32_t *__restrict__ num_tiles, const int32_t *__restrict__ pair_row, const float *__restrict__ pair_w,
     float *__restrict__ o_acc, int32_t *__restrict__ err, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV) {
+    // launched as a programmatic dependent of the dispatch: its tile list first. No early release of the
+    // finalize: its blocks would sit beside this persistent kernel's for its whole run.
+    pdl_wait();
     using SM = TcAttnSmem<D>;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -408,8 +411,10 @@ static cudaError_t launch_attn_tc_d(const ForwardArgs &a, cudaStream_t s) {
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = sms < a.max_tiles ? sms : a.max_tiles;
     HSA_PROF("chunk_attn", s);
-    chunk_attn_tc_kernel<D><<<grid, kTcThreads, smem, s>>>(a.Q, a.T, a.N, a.H / a.Hkv, a.scale, a.tiles,
-                                                            a.num_tiles, a.pair_row, a.pair_w, a.o_acc, a.err, tk, tv);
+    e = launch_pdl(chunk_attn_tc_kernel<D>, dim3(grid), dim3(kTcThreads), smem, s, a.Q, a.T, a.N, a.H / a.Hkv,
+                   a.scale, (const PairTile *)a.tiles, (const int32_t *)a.num_tiles, (const int32_t *)a.pair_row,
+                   (const float *)a.pair_w, a.o_acc, a.err, tk, tv);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -37,6 +37,14 @@ __device__ __forceinline__ uint64_t make_key(float s, uint32_t idx) {
 __device__ __forceinline__ float key_score(uint64_t k) { return ordered_to_float((uint32_t)(k >> 32)); }
 __device__ __forceinline__ int key_index(uint64_t k) { return (int)(0xffffffffu - (uint32_t)k); }
 
+// Programmatic dependent launch. A kernel that may be launched as a programmatic dependent calls
+// pdl_wait() before anything else: it returns once the previous kernel in the stream has completed and
+// its memory is visible (a no-op under an ordinary launch). pdl_launch_dependents() lets the next
+// kernel's blocks be scheduled once every block of this grid has issued it, so they are resident and
+// waiting when this grid ends; the launch latency is hidden, the ordering is that of the stream.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -28,6 +28,8 @@ constexpr int kSmemHistMax = 8192;  // chunks per (b, h) histogrammed in shared 
 
 __global__ void __launch_bounds__(kDispatchRows) count_kernel(const int32_t *__restrict__ sel_idx, int T, int N,
                                                               int K, int32_t *__restrict__ chunk_count) {
+    pdl_launch_dependents();
+    pdl_wait();
     extern __shared__ int s_hist[];
     const int bh = blockIdx.y;
     const bool use_smem = N <= kSmemHistMax;
@@ -98,6 +100,8 @@ constexpr int kScanPer = 8;
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t *__restrict__ chunk_count, int M,
                                                     int32_t *__restrict__ chunk_off, int32_t *__restrict__ tile_off,
                                                     int32_t *__restrict__ num_tiles, int max_tiles, int tp) {
+    pdl_launch_dependents();
+    pdl_wait();
     __shared__ int s_warp[33];
     int carry = 0, tcarry = 0;
     for (int base = 0; base < M; base += (int)blockDim.x * kScanPer) {
@@ -157,6 +161,8 @@ __global__ void __launch_bounds__(256) tile_list_kernel(const int32_t *__restric
                                                         const int32_t *__restrict__ chunk_off,
                                                         const int32_t *__restrict__ tile_off, int M,
                                                         PairTile *__restrict__ tiles, int max_tiles, int tp) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int i = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (i >= M) return;
@@ -180,6 +186,8 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_kernel(const int32_t *_
                                                                 float *__restrict__ pair_w,
                                                                 int32_t *__restrict__ pair_slot,
                                                                 const int32_t *__restrict__ cu_seqlens, int H) {
+    // no early release of the dependent: the persistent attention kernel would take SMs from this one
+    pdl_wait();
     extern __shared__ int s_mem[];
     const int bh = blockIdx.y;
     const int Tv = cu_seqlens ? min(T, cu_seqlens[bh / H + 1] - cu_seqlens[bh / H]) : T;
@@ -232,6 +240,8 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_sorted_kernel(
     const int32_t *__restrict__ sel_idx, const float *__restrict__ sel_w, int T, int N, int K,
     const int32_t *__restrict__ chunk_off, int32_t *__restrict__ chunk_cursor, int32_t *__restrict__ pair_row,
     float *__restrict__ pair_w, int32_t *__restrict__ pair_slot, const int32_t *__restrict__ cu_seqlens, int H) {
+    // no early release of the dependent: the persistent attention kernel would take SMs from this one
+    pdl_wait();
     extern __shared__ int s_mem[];
     const int nent_max = kDispatchRows * K;
     int *s_cnt = s_mem;                  // [N] entries per chunk in this block
@@ -325,6 +335,8 @@ __global__ void __launch_bounds__(kDispatchRows) scatter_sorted_kernel(
 // them.
 __global__ void finalize_kernel(const float *__restrict__ o_acc, uint16_t *__restrict__ out,
                                 const int32_t *__restrict__ cu_seqlens, int T, int H, int D) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int bh = blockIdx.y;
     const int Tv = cu_seqlens ? min(T, cu_seqlens[bh / H + 1] - cu_seqlens[bh / H]) : T;
     const int j = blockIdx.x * blockDim.x + threadIdx.x;  // 8-element unit within this (b, h)
@@ -374,16 +386,20 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
     }
     if (!counts_ready) {  // the forward's score kernel has counted them already
         HSA_PROF("dispatch_count", s);
-        count_kernel<<<dgrid, kDispatchRows, hsmem, s>>>(sel_idx, T, N, topk, chunk_count);
+        cudaError_t e = launch_pdl(count_kernel, dgrid, dim3(kDispatchRows), hsmem, s, sel_idx, T, N, topk, chunk_count);
+        if (e != cudaSuccess) return e;
     }
     {
         HSA_PROF("dispatch_scan", s);
-        scan_kernel<<<1, 1024, 0, s>>>(chunk_count, M, chunk_off, tile_off, num_tiles, max_tiles, tile_pairs);
+        cudaError_t e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, s, chunk_count, M, chunk_off, tile_off,
+                                   num_tiles, max_tiles, tile_pairs);
+        if (e != cudaSuccess) return e;
     }
     {
         HSA_PROF("dispatch_tiles", s);
-        tile_list_kernel<<<(M + 7) / 8, 256, 0, s>>>(chunk_count, chunk_off, tile_off, M, tiles, max_tiles,
-                                                     tile_pairs);
+        cudaError_t e = launch_pdl(tile_list_kernel, dim3((M + 7) / 8), dim3(256), 0, s, chunk_count, chunk_off,
+                                   tile_off, M, tiles, max_tiles, tile_pairs);
+        if (e != cudaSuccess) return e;
     }
     if (N <= kSortedScatterMaxN && topk <= 64) {  // ranks and entries fit kRankBits
         const size_t ssmem = 3 * (size_t)N * sizeof(int) + (size_t)kDispatchRows * topk * 3 * sizeof(int);
@@ -391,9 +407,9 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
                                              (int)ssmem);
         if (e != cudaSuccess) return e;
         HSA_PROF("dispatch_scatter", s);
-        scatter_sorted_kernel<<<dgrid, kDispatchRows, ssmem, s>>>(sel_idx, sel_w, T, N, topk, chunk_off,
-                                                                  chunk_cursor, pair_row, pair_w, pair_slot,
-                                                                  cu_seqlens, H);
+        e = launch_pdl(scatter_sorted_kernel, dgrid, dim3(kDispatchRows), ssmem, s, sel_idx, sel_w, T, N, topk,
+                       chunk_off, chunk_cursor, pair_row, pair_w, pair_slot, cu_seqlens, H);
+        if (e != cudaSuccess) return e;
     } else {
         const size_t ssmem = N <= kSmemHistMax / 2 ? 2 * (size_t)N * sizeof(int) : 0;
         if (ssmem > 48 * 1024) {
@@ -401,8 +417,9 @@ cudaError_t launch_dispatch(const int32_t *sel_idx, const float *sel_w, int B, i
             if (e != cudaSuccess) return e;
         }
         HSA_PROF("dispatch_scatter", s);
-        scatter_kernel<<<dgrid, kDispatchRows, ssmem, s>>>(sel_idx, sel_w, T, N, topk, chunk_off, chunk_cursor,
-                                                           pair_row, pair_w, pair_slot, cu_seqlens, H);
+        cudaError_t e = launch_pdl(scatter_kernel, dgrid, dim3(kDispatchRows), ssmem, s, sel_idx, sel_w, T, N, topk,
+                                   chunk_off, chunk_cursor, pair_row, pair_w, pair_slot, cu_seqlens, H);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }
@@ -444,8 +461,9 @@ cudaError_t launch_forward(const ForwardArgs &a0, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     {
         HSA_PROF("finalize", s);
-        finalize_kernel<<<dim3((unsigned)(((size_t)a.T * a.D / 8 + 255) / 256), BH), 256, 0, s>>>(
-            a.o_acc, a.out, a.cu_seqlens, a.T, a.H, a.D);
+        e = launch_pdl(finalize_kernel, dim3((unsigned)(((size_t)a.T * a.D / 8 + 255) / 256), BH), dim3(256), 0, s,
+                       a.o_acc, a.out, a.cu_seqlens, a.T, a.H, a.D);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }

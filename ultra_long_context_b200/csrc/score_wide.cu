@@ -181,6 +181,7 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
     int32_t *__restrict__ sel_idx, float *__restrict__ sel_w, float *__restrict__ o_acc,
     int32_t *__restrict__ chunk_count, int32_t *__restrict__ err, const __grid_constant__ CUtensorMap tmQ,
     const __grid_constant__ CUtensorMap tmL) {
+    pdl_launch_dependents();  // the dispatch's scan may be scheduled (it waits for this grid)
     using SM = SwSmem<D, K>;
     constexpr int KH = SM::KH;
     extern __shared__ unsigned char smem_raw[];

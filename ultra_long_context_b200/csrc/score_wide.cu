@@ -9,28 +9,35 @@
 // Work item: 256 consecutive token rows of one (batch, head), as two 128-row tiles that share every
 // landmark block. One CTA per SM walks its items: items are ordered longest rows first and dealt to
 // the CTAs in snake order (CTA c takes items c, 2G - 1 - c, 2G + c, ...), which evens out their cost.
-//   * Warp 8 (loader): TMA copies of each item's two Q tiles into a staging area and of 64-landmark
+//   * Warp 16 (loader): TMA copies of each item's two Q tiles into a staging area and of 64-landmark
 //     blocks (128-byte swizzle) through a four-stage ring. An item's blocks go through the ring twice
 //     (two passes over the row); the next item's Q tiles are copied between the two.
-//   * Warp 9 (MMA): S_blk = Q L_blk^T (M = 128, N = 64, fp32) for each tile into one of the tile's two
-//     TMEM score buffers. Q is the A operand from TMEM (two bf16 per column), double-buffered by item.
-//   * Warps 0-3 / 4-7 (selectors of tile 0 / 1): one token row per thread (= TMEM lane).
-//       - The row of Q goes from the staging into TMEM: the next item's while this one runs.
-//       - Pass 1 keeps 2K group maxima per row: group j holds the chunks j, j + 2K, j + 4K, ... of
-//         every block (one max per score). They are maxima of disjoint sets of scores, so the K-th
-//         largest of them, tau0, has K different chunks at or above it: the row's K-th largest score is
-//         at least tau0, and no score below tau0 can be kept.
-//       - Pass 2 (the same products, recomputed: bit-identical) appends the exact 64-bit keys of the
-//         scores >= tau0 -- ordered score, then lower chunk first -- to a per-row buffer of 2K keys. On
-//         i.i.d. scores about 1.3 K of them reach tau0; a buffer that would overflow is first cut to
-//         its K largest keys, after which a key must beat the K-th kept one (ties stay exact: the keys
-//         are unique).
-//       - The buffer's keys are sorted by a bitonic network in registers; the K largest, in order, are
-//         the row's selection. Scores are compared unscaled (the scale is positive, so the order is the
-//         same); the scale enters the fusion weights only.
-//   * Warp 10 zeroes the item's rows of the fp32 output accumulator (the chunk attention adds into
-//     them). The selectors also count the selected pairs per chunk for the dispatch (a shared-memory
-//     histogram per item).
+//   * Warp 17 (MMA): S_blk = Q L_blk^T (M = 128, N = 64, fp32) for each tile into one of the tile's two
+//     TMEM score buffers. Q is the A operand from TMEM (two bf16 per column), double-buffered by item;
+//     the selectors' copies of it are counted in shared memory and the MMA warp waits on the count.
+//   * Warps 0-15 (selectors): warp w serves tile w / 8, column half (w / 4) % 2 of every block and the
+//     32 rows (w % 4) * 32 .. + 31 (= its TMEM lanes): two threads per token row, one per half.
+//       - Each thread copies its half of the row of Q from the staging into TMEM: the next item's while
+//         this one runs.
+//       - Pass 1 keeps 2K group maxima per row, K per half: group j of a half holds its columns j,
+//         j + K, ... of every block (one max per score). They are maxima of disjoint sets of scores, so
+//         the K-th largest of all 2K, tau0, has K different chunks at or above it: the row's K-th largest
+//         score is at least tau0, and no score below tau0 can be kept. Each half sorts its maxima, the
+//         pair swaps them, and tau0 = min_j max(A[j], B[K-1-j]).
+//       - Pass 2 (the same products, recomputed: bit-identical) stages each block's scores in shared
+//         memory, marks the scores >= tau0 on the FMA pipe, and makes exact 64-bit keys -- ordered
+//         score, then lower chunk first -- for those only. Each half keeps its K largest keys (on
+//         i.i.d. scores about 1.3 K reach tau0 per row; a half with more keeps its K largest, one by
+//         one; ties stay exact: the keys are unique).
+//       - Each half sorts its keys (bitonic network in registers), the pair swaps them, and a bitonic
+//         merge step gives the row's K largest in order; each thread writes half of the output slots.
+//         Scores are compared unscaled (the scale is positive, so the order is the same); the scale
+//         enters the fusion weights only.
+//   * Warp 18 zeroes the item's rows of the fp32 output accumulator (the chunk attention adds into
+//     them) and adds each finished item's pair counts per chunk, which the selectors gather in a
+//     per-tile shared-memory histogram, into the dispatch's counts.
+// The two warps of a row range meet on their own named barrier; the other hand-offs are mbarriers, each
+// waited at every one of its phases in turn, and every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 

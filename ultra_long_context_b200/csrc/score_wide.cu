@@ -55,6 +55,8 @@ constexpr int kSwLoaderWarp = 16;  // warps 0-15 select
 constexpr int kSwMmaWarp = 17;
 constexpr int kSwZeroWarp = 18;
 constexpr int kSwThreads = 32 * (kSwZeroWarp + 1);  // 608
+constexpr int kSwMaxSeqs = 256;    // padded batches: sequences ordered in shared memory (else every item is dealt)
+constexpr int kSwMaxLevels = 1024; // 256-row levels counted in shared memory (T <= 262144)
 constexpr int kSwSlot = 32;     // key slot stride: slot j of a lane at [j * 32] of its half's slots
 constexpr int kSwHist = 1024;   // chunks per (b, h) counted in shared memory (per tile, two buffers)
 
@@ -88,7 +90,9 @@ struct SwSmem {
     static constexpr int NBAR = 2 * kSwStages + 6 + 8 + 8;
     static constexpr uint32_t QCNT = BAR + NBAR * 8;     // unsigned[2]: warps' Q copies into TMEM, per tile
     static constexpr uint32_t TMEM = QCNT + 8;
-    static constexpr uint32_t BYTES = TMEM + 16;
+    static constexpr uint32_t SEQ = TMEM + 16;                       // int[kSwMaxSeqs]: sequences by length
+    static constexpr uint32_t CUM = SEQ + kSwMaxSeqs * 4;             // int[kSwMaxLevels + 1]: items before a level
+    static constexpr uint32_t BYTES = CUM + (kSwMaxLevels + 1) * 4;
     static constexpr size_t DYN = BYTES + 1024;
     static_assert(DYN <= 227 * 1024, "shared memory budget");
     // TMEM columns: Q [item parity][tile] (D/2 each), then S [tile][buffer] (64 each)
@@ -113,6 +117,29 @@ __device__ __forceinline__ SwItem sw_item(int k, int G, int c, int P, int BH) {
         it.t0 = (P - 1 - level) * kSwItem;  // longest rows first
         it.valid = true;
     }
+    return it;
+}
+
+// The k-th work item of this CTA in a padded batch: only the (sequence, head, 256-row block) items with a
+// row inside their sequence exist. s_cum[L] counts the items of the levels before level L (level 0 =
+// the longest rows) and s_seq lists the sequences by length, longest first, so the sequences that reach
+// a level are a prefix of it; within a level the items go by that order, then by head.
+__device__ __forceinline__ SwItem sw_item_seq(int k, int G, int c, int P, int H, const int *s_cum,
+                                              const int *s_seq) {
+    const int pos = (k & 1) ? G - 1 - c : c;
+    const long long i = (long long)k * G + pos;
+    SwItem it{0, 0, false};
+    if (i >= s_cum[P]) return it;
+    int lo = 0, hi = P;  // s_cum[lo] <= i < s_cum[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (s_cum[mid] <= i) lo = mid;
+        else hi = mid;
+    }
+    const int o = (int)(i - s_cum[lo]);
+    it.bh = s_seq[o / H] * H + o % H;
+    it.t0 = (P - 1 - lo) * kSwItem;
+    it.valid = true;
     return it;
 }
 
@@ -216,8 +243,52 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
     const int G = gridDim.x, cta = blockIdx.x;
     const int P = (T + kSwItem - 1) / kSwItem;
     auto seq_len = [&](int bh) { return cu_seqlens ? min(T, cu_seqlens[bh / H + 1] - cu_seqlens[bh / H]) : T; };
+    // padded batches: deal only the items with a row inside their sequence (tables built below)
+    const int nseq = BH / H;
+    const bool by_seq = cu_seqlens != nullptr && nseq <= kSwMaxSeqs && P <= kSwMaxLevels;
+    int *s_seq = reinterpret_cast<int *>(s + SM::SEQ);
+    int *s_cum = reinterpret_cast<int *>(s + SM::CUM);
+    auto item_of = [&](int k) {
+        return by_seq ? sw_item_seq(k, G, cta, P, H, s_cum, s_seq) : sw_item(k, G, cta, P, BH);
+    };
 
     for (int i = tid; i < 4 * kSwHist; i += kSwThreads) hist(0, 0)[i] = 0;
+    if (by_seq) {
+        auto len = [&](int b) { return max(0, min(T, cu_seqlens[b + 1] - cu_seqlens[b])); };
+        for (int b = tid; b < nseq; b += kSwThreads) {  // rank by length, longest first (ties: lower index)
+            const int lb = len(b);
+            int rank = 0;
+            for (int b2 = 0; b2 < nseq; ++b2) {
+                const int l2 = len(b2);
+                rank += (l2 > lb || (l2 == lb && b2 < b)) ? 1 : 0;
+            }
+            s_seq[rank] = b;
+        }
+        for (int L = tid; L < P; L += kSwThreads) {  // sequences with a row at or past the level's first row
+            const int t0 = (P - 1 - L) * kSwItem;
+            int n = 0;
+            for (int b2 = 0; b2 < nseq; ++b2) n += len(b2) > t0 ? 1 : 0;
+            s_cum[L + 1] = n * H;
+        }
+        __syncthreads();
+        if (warp == 0) {  // prefix sum over the levels: lane l sums its consecutive run, then a warp scan
+            const int per = (P + 31) / 32, l0 = lane * per;
+            int run = 0;
+            for (int L = l0; L < min(P, l0 + per); ++L) run += s_cum[L + 1];
+            int incl = run;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int x = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += x;
+            }
+            int acc = incl - run;  // items of the levels before this lane's run
+            if (lane == 0) s_cum[0] = 0;
+            for (int L = l0; L < min(P, l0 + per); ++L) {
+                acc += s_cum[L + 1];
+                s_cum[L + 1] = acc;
+            }
+        }
+    }
     if (warp == kSwMmaWarp) tc::tmem_alloc(sb + SM::TMEM, SM::NCOLS);
     if (tid == 0) {
         for (int i = 0; i < kSwStages; ++i) {
@@ -270,13 +341,13 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
                                   l_full(st));
             ++h;
         };
-        SwItem it = sw_item(0, G, cta, P, BH);
+        SwItem it = item_of(0);
         if (it.valid) load_q(it);
         for (int k = 0; it.valid && ok; ++k) {
             const int nblk = (sw_nmax(it.t0, kSwItem, seq_len(it.bh), N) + kSwCols - 1) / kSwCols;
             const int kvh = it.bh / Gh;
             for (int b = 0; b < nblk && ok; ++b) load_l(kvh, b);  // pass 1
-            const SwItem nx = sw_item(k + 1, G, cta, P, BH);
+            const SwItem nx = item_of(k + 1);
             if (nx.valid && ok) load_q(nx);
             for (int b = 0; b < nblk && ok; ++b) load_l(kvh, b);  // pass 2
             it = nx;
@@ -292,7 +363,7 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
         // ---------------- MMA issuer: the whole warp runs it, one elected lane issues ----------------
         constexpr uint32_t idesc = tc::idesc_bf16(kSwRows, kSwCols, 0, 0);
         uint32_t h = 0, g[2] = {0, 0};
-        SwItem it = sw_item(0, G, cta, P, BH);
+        SwItem it = item_of(0);
         for (int k = 0; it.valid && ok; ++k) {
             const int Tv = seq_len(it.bh);
             const int nb0 = (sw_nmax(it.t0, kSwRows, Tv, N) + kSwCols - 1) / kSwCols;
@@ -345,7 +416,7 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
                     ++h;
                 }
             }
-            it = sw_item(k + 1, G, cta, P, BH);
+            it = item_of(k + 1);
         }
         if (!ok) {  // the products in flight complete before TMEM is released
             for (int u = 0; u < 2; ++u)
@@ -375,7 +446,7 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
                 if (lane == 0) tc::mbar_arrive(h_free(u, kk & 1));
             }
         };
-        SwItem it = sw_item(0, G, cta, P, BH), prev{0, 0, false};
+        SwItem it = item_of(0), prev{0, 0, false};
         int k = 0;
         for (; it.valid && ok; ++k) {
             const int nv = max(0, min(kSwItem, min(T, seq_len(it.bh)) - it.t0));
@@ -383,7 +454,7 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
             for (int i = lane; i < nv * (D / 4); i += 32) acc[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             if (k > 0) flush(k - 1, prev);
             prev = it;
-            it = sw_item(k + 1, G, cta, P, BH);
+            it = item_of(k + 1);
         }
         if (ok && k > 0) flush(k - 1, prev);
     } else {
@@ -449,7 +520,7 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
             return true;
         };
 
-        SwItem it = sw_item(0, G, cta, P, BH);
+        SwItem it = item_of(0);
         if (it.valid) ok = copy_q(0, true);
         // this thread's scores in its tile's scratch: one 128-byte row, its 16-byte chunks XOR-swizzled by
         // (row % 8) so that a warp's 16-byte stores do not conflict; column i at scr_at(i)
@@ -519,7 +590,7 @@ __global__ void __launch_bounds__(kSwThreads, 1) score_topk_wide_kernel(
             for (int j = 0; j < K; ++j) tmin = fminf(tmin, fmaxf(gm[j], gx_o[(K - 1 - j) * kSwSlot]));
             const float tau0 = my_n > K ? tmin : -INFINITY;
             // the next item's Q into TMEM, while this one's second pass runs
-            const SwItem nx = sw_item(k + 1, G, cta, P, BH);
+            const SwItem nx = item_of(k + 1);
             if (ok && nx.valid && !copy_q(k + 1, false)) ok = false;
             // the partner has read these maxima before the key slots reuse them (pass 2's scratch is this
             // thread's own part of the staging: the 16-byte chunks of its own row of Q, just copied)

@@ -9,6 +9,7 @@
 // Work item: 256 consecutive token rows of one (batch, head), as two 128-row tiles that share every
 // landmark block. One CTA per SM walks its items: items are ordered longest rows first and dealt to
 // the CTAs in snake order (CTA c takes items c, 2G - 1 - c, 2G + c, ...), which evens out their cost.
+// In a padded batch (per-sequence lengths) only the items with a row inside their sequence exist.
 //   * Warp 16 (loader): TMA copies of each item's two Q tiles into a staging area and of 64-landmark
 //     blocks (128-byte swizzle) through a four-stage ring. An item's blocks go through the ring twice
 //     (two passes over the row); the next item's Q tiles are copied between the two.
